@@ -1,0 +1,202 @@
+// fp64 CPU oracle of the sparse-attention layer: IndexPool -> lightning
+// indexer -> top-k blocks -> softmax attention over the selected MLA latent
+// rows.
+//
+// TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, obviously correct
+// definition that the CUDA path is checked against.  Only the test suite,
+// the smoke check and the benchmark's CPU-baseline leg may load it; the
+// product path never does.  It shares no code, header, table or helper with
+// the CUDA library.
+//
+// Sources (web pages, cited by title and section):
+//  [W1] "GLM-5.3-Flash: 하이브리드 희소·선형 어텐션과 IndexPool·EPD로 1M 컨텍스트를
+//       오픈 소스로 서빙하는 방법" -- sections "희소 어텐션: 인덱서로 필요한
+//       토큰만" and "IndexPool: 인덱서 KV 캐시를 4배 압축" (the pooling formula).
+//  [W3] "GLM-5.3 Sparse Attention은 연산량을 줄이지만 HBM 수요는 지속된다" --
+//       section "GLM-5.3 Sparse Attention이 실제로 바꾸는 것" (indexer -> top-k ->
+//       MLA on the selected positions; dense below the 2048-position budget).
+//  [W4] "GLM-5.3-Flash vs Qwen3.8-Flash-Next: 두 중국 AI 연구소가 독립적으로 같은
+//       모델 설계로 수렴한 이유" -- section "수렴점 2 — 4배 압축 후 2,048 토큰만
+//       유지" (32-head indexer, top-2048, 4-token blocks x 512) and section
+//       "의견이 갈리는 지점 — 위치 인코딩" (NoPE: no rotary term).
+//  The indexer formula I(t,b) = sum_h w_{t,h} ReLU(q_{t,h} . k_b) is not on
+//  the pages; it is the DeepSeek sparse-attention indexer form that [W3]
+//  names, fixed by the workload specification.
+//
+// Every floating-point step is done in fp64.  The only roundings are the
+// ones the method's storage formats impose: the pooled key is stored as
+// bf16 (one round-to-nearest-even of the exact fp64 sum), and the top-k
+// decision is taken on the score rounded to fp32, the precision in which
+// scores are stored and ranked on the device.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+double bf16_to_f64(uint16_t h) {
+  uint32_t u = static_cast<uint32_t>(h) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return static_cast<double>(f);
+}
+
+// Round a finite double to the nearest bf16 (8 significant bits), ties to
+// even, by scaling to an integer significand and rounding once.
+uint16_t f64_to_bf16_rne(double v) {
+  if (v == 0.0) return std::signbit(v) ? 0x8000 : 0x0000;
+  int e = 0;
+  std::frexp(std::fabs(v), &e);         // |v| = m * 2^e, m in [0.5, 1)
+  int qe = e - 8;                       // weight of the last kept bit
+  if (qe < -133) qe = -133;             // bf16 subnormal spacing
+  double r = std::nearbyint(std::ldexp(std::fabs(v), -qe));  // exact scale
+  double a = std::ldexp(r, qe);
+  float f = static_cast<float>(a);      // exact: a has <= 8 significant bits
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  uint16_t h = static_cast<uint16_t>(u >> 16);
+  if (std::signbit(v)) h |= 0x8000;
+  return h;
+}
+
+int pick_threads(int nthreads) {
+  if (nthreads > 0) return nthreads;
+  unsigned hc = std::thread::hardware_concurrency();
+  return hc ? static_cast<int>(hc) : 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+int orc_threads(int requested) { return pick_threads(requested); }
+
+uint16_t orc_bf16_rne(double v) { return f64_to_bf16_rne(v); }
+
+// IndexPool cache write [W1 "IndexPool"]: block b holds tokens 4b..4b+3 in
+// time order and k_pool[b] = sum_{i=0..3} w_i k[4b+i], with sum_i w_i = 1.
+// Only complete blocks are pooled: n_tok / pool of them.
+void orc_pool(const uint16_t* raw, int64_t n_tok, int dim, int pool,
+              const double* w, uint16_t* pooled) {
+  const int64_t nblk = n_tok / pool;
+  for (int64_t b = 0; b < nblk; ++b) {
+    for (int d = 0; d < dim; ++d) {
+      double acc = 0.0;
+      for (int i = 0; i < pool; ++i)
+        acc += w[i] * bf16_to_f64(raw[(b * pool + i) * dim + d]);
+      pooled[b * dim + d] = f64_to_bf16_rne(acc);
+    }
+  }
+}
+
+// Lightning-indexer score of every pooled block against one query
+// [W3 "실제로 바꾸는 것"; formula as fixed by the workload specification]:
+//   s[b] = sum_h w_h * max(0, sum_d q[h][d] * k_pool[b][d]).
+void orc_score(const uint16_t* q, const double* w_head, int heads, int dim,
+               const uint16_t* keys, int64_t nblk, double* out, int nthreads) {
+  std::vector<double> qd(static_cast<size_t>(heads) * dim);
+  for (size_t i = 0; i < qd.size(); ++i) qd[i] = bf16_to_f64(q[i]);
+  auto work = [&](int64_t b0, int64_t b1) {
+    std::vector<double> kd(dim);
+    for (int64_t b = b0; b < b1; ++b) {
+      for (int d = 0; d < dim; ++d) kd[d] = bf16_to_f64(keys[b * dim + d]);
+      double s = 0.0;
+      for (int h = 0; h < heads; ++h) {
+        double dot = 0.0;
+        for (int d = 0; d < dim; ++d) dot += qd[h * dim + d] * kd[d];
+        s += w_head[h] * (dot > 0.0 ? dot : 0.0);
+      }
+      out[b] = s;
+    }
+  };
+  const int nt = pick_threads(nthreads);
+  if (nt <= 1 || nblk < 4096) {
+    work(0, nblk);
+    return;
+  }
+  std::vector<std::thread> pool;
+  for (int t = 0; t < nt; ++t) {
+    int64_t b0 = nblk * t / nt, b1 = nblk * (t + 1) / nt;
+    pool.emplace_back(work, b0, b1);
+  }
+  for (auto& th : pool) th.join();
+}
+
+// Top-k block selection [W4 "수렴점 2": keep the 512 highest-scoring 4-token
+// blocks]: full sort on (score descending, block ascending) -- equal scores
+// go to the lower block index -- keep the first min(K, nblk), return them
+// in ascending block order.  Scores are compared after rounding to fp32;
+// -0 and +0 compare equal.
+int64_t orc_topk(const double* s, int64_t nblk, int64_t K, int32_t* idx_out) {
+  std::vector<std::pair<float, int64_t>> v(static_cast<size_t>(nblk));
+  for (int64_t b = 0; b < nblk; ++b) v[b] = {static_cast<float>(s[b]), b};
+  std::sort(v.begin(), v.end(), [](const auto& a, const auto& c) {
+    if (a.first != c.first) return a.first > c.first;
+    return a.second < c.second;
+  });
+  const int64_t k = std::min(K, nblk);
+  std::vector<int64_t> sel(static_cast<size_t>(k));
+  for (int64_t i = 0; i < k; ++i) sel[i] = v[i].second;
+  std::sort(sel.begin(), sel.end());
+  for (int64_t i = 0; i < k; ++i) idx_out[i] = static_cast<int32_t>(sel[i]);
+  return k;
+}
+
+// Positions attended by a query that sees n_vis tokens: the 4 tokens of
+// every selected block, then the partial tail n_vis - n_vis % pool .. n_vis-1
+// (those tokens have no pooled key yet, so they are always kept).
+int64_t orc_token_set(const int32_t* idx, int64_t count, int64_t n_vis,
+                      int pool, int64_t* pos_out) {
+  int64_t m = 0;
+  for (int64_t j = 0; j < count; ++j)
+    for (int i = 0; i < pool; ++i) pos_out[m++] = static_cast<int64_t>(idx[j]) * pool + i;
+  for (int64_t t = (n_vis / pool) * pool; t < n_vis; ++t) pos_out[m++] = t;
+  return m;
+}
+
+// Softmax attention of every head over the gathered latent rows
+// [W3 "실제로 바꾸는 것": MLA runs on the selected positions only].
+// Absorbed MLA with NoPE [W4 "위치 인코딩"]: the latent row c_t is both key and
+// value, shared by all heads:
+//   z_t = sm_scale * q_h . c_t,  o_h = sum_t softmax(z)_t c_t,
+//   lse_h = log sum_t exp(z_t).
+void orc_attention(const uint16_t* q, int heads, int dim, const uint16_t* rows,
+                   int64_t S, double sm_scale, double* out, double* lse) {
+  if (S <= 0) {  // a query that sees no token: zero output, lse = -inf
+    for (int64_t i = 0; i < static_cast<int64_t>(heads) * dim; ++i) out[i] = 0.0;
+    if (lse)
+      for (int h = 0; h < heads; ++h) lse[h] = -INFINITY;
+    return;
+  }
+  std::vector<double> c(static_cast<size_t>(S) * dim);
+  for (size_t i = 0; i < c.size(); ++i) c[i] = bf16_to_f64(rows[i]);
+  std::vector<double> z(static_cast<size_t>(S));
+  for (int h = 0; h < heads; ++h) {
+    std::vector<double> qh(dim);
+    for (int d = 0; d < dim; ++d) qh[d] = bf16_to_f64(q[h * dim + d]);
+    double m = -INFINITY;
+    for (int64_t t = 0; t < S; ++t) {
+      double dot = 0.0;
+      for (int d = 0; d < dim; ++d) dot += qh[d] * c[t * dim + d];
+      z[t] = sm_scale * dot;
+      m = std::max(m, z[t]);
+    }
+    double l = 0.0;
+    for (int64_t t = 0; t < S; ++t) {
+      z[t] = std::exp(z[t] - m);
+      l += z[t];
+    }
+    for (int d = 0; d < dim; ++d) {
+      double acc = 0.0;
+      for (int64_t t = 0; t < S; ++t) acc += z[t] * c[t * dim + d];
+      out[h * dim + d] = acc / l;
+    }
+    if (lse) lse[h] = m + std::log(l);
+  }
+}
+
+}  // extern "C"
