@@ -1,0 +1,282 @@
+/*
+ * libspx -- the sparse-attention layer of a hybrid long-context decoder on
+ * NVIDIA B200 (sm_100a).
+ *
+ * One sparse-attention layer takes four steps per query token:
+ *   1. IndexPool cache write: every 4 consecutive raw indexer keys are folded
+ *      into one pooled key k_pool = sum_i w_i k_i with learned weights that
+ *      sum to 1.  Source: [W1] section "IndexPool: 인덱서 KV 캐시를 4배 압축".
+ *   2. Lightning indexer: every complete pooled block b is scored against the
+ *      query, s[b] = sum_h w_h ReLU(q_h . k_pool[b]), 32 heads x 128 dims.
+ *      Source: [W4] section "수렴점 2 — 4배 압축 후 2,048 토큰만 유지" (32-head
+ *      indexer, top-2048) and [W3] section "GLM-5.3 Sparse Attention이 실제로
+ *      바꾸는 것" (the DeepSeek sparse-attention indexer; its ReLU-weighted form
+ *      is the one fixed by the workload specification, the pages give none).
+ *   3. Top-k: the 512 highest-scoring blocks (= 2048 tokens) are kept; equal
+ *      scores go to the lower block index.  Source: [W4] "수렴점 2".
+ *   4. Sparse MLA attention: softmax attention of every head over the latent
+ *      rows of the tokens of the selected blocks plus the query's partial
+ *      tail block (tokens that have no pooled key yet).  With 2051 visible
+ *      tokens or fewer every token is kept, i.e. the layer is exactly dense
+ *      attention.  Sources: [W3] "실제로 바꾸는 것" (MLA on the selected
+ *      positions only; dense below the 2048-position budget) and [W4] section
+ *      "의견이 갈리는 지점 — 위치 인코딩" (NoPE: no rotary component).
+ *
+ * Pages cited:
+ *   [W1] "GLM-5.3-Flash: 하이브리드 희소·선형 어텐션과 IndexPool·EPD로 1M 컨텍스트를
+ *        오픈 소스로 서빙하는 방법"
+ *   [W3] "GLM-5.3 Sparse Attention은 연산량을 줄이지만 HBM 수요는 지속된다"
+ *   [W4] "GLM-5.3-Flash vs Qwen3.8-Flash-Next: 두 중국 AI 연구소가 독립적으로 같은
+ *        모델 설계로 수렴한 이유"
+ *
+ * Conventions shared by every call
+ *   - All tensor arguments are DEVICE pointers to caller-owned memory, dense
+ *     row-major, with the shapes given per call.  bf16 tensors are passed as
+ *     void* (IEEE bfloat16 bit patterns).  The library never allocates, frees
+ *     or synchronises; scratch memory is a caller buffer sized by the
+ *     matching *_workspace_size call (256-byte aligned).
+ *   - Calls are asynchronous on the given stream (a cudaStream_t; NULL is the
+ *     legacy default stream).  A call that returns SPX_OK has enqueued its
+ *     kernels; device-side faults surface at the caller's next
+ *     synchronisation.  The library holds no per-call state and is safe to
+ *     call from several host threads.
+ *   - Arguments are validated on the host before anything is launched: a call
+ *     that returns an error has enqueued nothing.
+ *   - Per-sequence lengths live on the device (int64).  `max_len` is a host
+ *     upper bound on every visible length of the call; kernels clamp the
+ *     device lengths to it, so a length above the bound is read as the bound
+ *     and never causes an out-of-range access.
+ *   - v1 supports idx_heads = 32, idx_dim = 128, pool = 4, topk_blocks = 512,
+ *     latent = 512 and heads a multiple of 16 in [16, 128]; other values
+ *     return SPX_ERR_UNSUPPORTED.
+ */
+#ifndef SPX_H_
+#define SPX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPX_API __attribute__((visibility("default")))
+#else
+#define SPX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the same handle type, declared here without CUDA headers). */
+typedef struct CUstream_st* spx_stream;
+
+typedef enum spx_status {
+  SPX_OK = 0,
+  SPX_ERR_INVALID_ARG = 1, /* null pointer, non-finite or negative scalar   */
+  SPX_ERR_SHAPE = 2,       /* sizes, strides or capacities inconsistent     */
+  SPX_ERR_UNSUPPORTED = 3, /* dims outside what v1 implements                */
+  SPX_ERR_WORKSPACE = 4,   /* workspace null, misaligned or too small        */
+  SPX_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed    */
+  SPX_ERR_DEVICE = 6       /* a kernel reported a device-side error          */
+} spx_status;
+
+/* Layer dimensions. */
+typedef struct spx_dims {
+  int32_t idx_heads;   /* indexer heads (32)                         */
+  int32_t idx_dim;     /* indexer key/query width (128)              */
+  int32_t pool;        /* tokens per pooled block (4)                */
+  int32_t topk_blocks; /* blocks kept per query (512)                */
+  int32_t heads;       /* MLA query heads (multiple of 16, <= 128)   */
+  int32_t latent;      /* MLA latent width (512)                     */
+  float sm_scale;      /* softmax scale applied to q . c (finite, > 0) */
+} spx_dims;
+
+/* Optional CUDA events (cudaEvent_t handles, or NULL) that the fused calls
+ * record on their stream immediately before and after the indexer-scoring
+ * launch, so a caller can time that kernel inside a larger step. */
+typedef struct spx_timing {
+  void* score_begin;
+  void* score_end;
+} spx_timing;
+
+/* Name of a status code ("SPX_OK", ...).  Never NULL. */
+SPX_API const char* spx_status_string(spx_status s);
+
+/* Library version string. */
+SPX_API const char* spx_version(void);
+
+/* Fills *d with the dimensions of the layer described by the pages
+ * (32 x 128 indexer, pool 4, top-512 blocks, latent 512) and the given MLA
+ * head count and softmax scale. */
+SPX_API spx_status spx_dims_init(spx_dims* d, int32_t heads, float sm_scale);
+
+/* Number of kernels this process has launched through the library so far
+ * (all devices, all threads).  Lets a caller count launches in a region. */
+SPX_API uint64_t spx_launch_count(void);
+
+/* Reads and clears the device-side error word that kernels set when one of
+ * their bounded waits gives up (a pipeline that did not make progress within
+ * about two seconds).  Synchronises the given stream.  *code is 0 when no
+ * kernel reported an error since the last call. */
+SPX_API spx_status spx_device_error(int32_t* code, spx_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 1 -- IndexPool cache write.  [W1] "IndexPool": k_pool = sum_i w_i k_i,
+ * i = 1..4, sum_i w_i = 1, learned w.
+ *
+ * Appends n_new raw indexer keys per sequence.  Token p of sequence b (0-based
+ * position in the sequence) belongs to block p / 4 at slot p % 4.  For every
+ * block that the append completes, the pooled key
+ *     pooled_k[b][blk][d] = bf16_rne( sum_{i=0..3} pool_w[i] * key(4 blk + i)[d] )
+ * is written (the sum is formed in fp32 and rounded once to bf16), taking
+ * the older keys of the block from `tail`.  Keys of the still-incomplete last
+ * block are stored in tail[b][p % 4].  The caller advances its lengths by
+ * n_new afterwards.
+ *
+ *   raw_k     bf16 [B, n_new, idx_dim]        keys of the appended tokens
+ *   pool_w    HOST float [pool]               sum must be 1 within 1e-6
+ *   tail      bf16 [B, pool-1, idx_dim]       raw keys of incomplete blocks (in/out)
+ *   pooled_k  bf16 [B, cap_blk, idx_dim]      pooled-key cache (out)
+ *   len_dev   DEVICE int64 [B]                tokens already appended per sequence
+ *   max_len   host bound: len_dev[b] + n_new <= max_len <= pool * cap_blk
+ * Errors: SPX_ERR_INVALID_ARG for null pointers or weights that do not sum
+ * to 1; SPX_ERR_SHAPE for B < 1, n_new < 0 or max_len out of range.
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_pool_append(const spx_dims* d, int32_t B, const void* raw_k,
+                           int32_t n_new, const float* pool_w, void* tail,
+                           void* pooled_k, int64_t cap_blk,
+                           const int64_t* len_dev, int64_t max_len,
+                           spx_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 2 -- lightning-indexer scores of every complete block (decode: one
+ * query per sequence).  [W4] "수렴점 2" (32-head lightning indexer);
+ * formula as fixed by the workload specification:
+ *     scores[b][blk] = sum_h w_head[b][h] * max(0, sum_d q_idx[b][h][d] * pooled_k[b][blk][d])
+ * for blk < n_vis[b] / pool.  Products are exact, sums are fp32.
+ *
+ *   q_idx     bf16 [B, idx_heads, idx_dim]
+ *   w_head    float [B, idx_heads]
+ *   pooled_k  bf16 [B, cap_blk, idx_dim]
+ *   n_vis     DEVICE int64 [B]   visible tokens per sequence (clamped to max_len)
+ *   scores    float [B, score_stride]; entries blk >= n_vis[b]/pool untouched
+ *   Requires max_len <= pool * cap_blk and score_stride >= max_len / pool.
+ * Runs on the tensor cores (tcgen05) with TMA-staged key tiles.
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_index_score(const spx_dims* d, int32_t B, const void* q_idx,
+                           const float* w_head, const void* pooled_k,
+                           int64_t cap_blk, const int64_t* n_vis,
+                           int64_t max_len, float* scores, int64_t score_stride,
+                           spx_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 3 -- top-k blocks per row.  [W4] "수렴점 2": keep the 512
+ * highest-scoring blocks (2048 tokens).  Ties go to the lower block index;
+ * -0 and +0 are equal; scores must be finite.  Rows with nblk <= topk_blocks
+ * keep every block ([W3]: no larger pool to reduce -> dense).
+ *
+ *   scores    float [rows, score_stride]   only blk < n_vis[r]/pool are read
+ *   n_vis     DEVICE int64 [rows]
+ *   idx       int32 [rows, topk_blocks]    selected block ids, ascending,
+ *                                          padded with -1 after count[r]
+ *   count     int32 [rows]                 min(topk_blocks, n_vis[r]/pool)
+ *   ws        workspace of spx_topk_workspace_size(d, rows, max_len) bytes
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_topk_workspace_size(const spx_dims* d, int32_t rows,
+                                   int64_t max_len, size_t* bytes);
+SPX_API spx_status spx_topk_blocks(const spx_dims* d, int32_t rows,
+                           const float* scores, int64_t score_stride,
+                           const int64_t* n_vis, int64_t max_len, int32_t* idx,
+                           int32_t* count, void* ws, size_t ws_bytes,
+                           spx_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 4 -- sparse MLA attention over the selected latent rows.
+ * [W3] "실제로 바꾸는 것": attention runs on the selected positions only;
+ * absorbed MLA with NoPE ([W4] "위치 인코딩"): the latent row c_t is both key
+ * and value, shared by all heads.  For row r the attended set is
+ *     S_r = { 4 idx[r][j] + i : j < count[r], i < 4 }  U  { 4 floor(n/4) .. n-1 }
+ * with n = n_vis[r], and for every head h
+ *     out[r][h] = sum_{t in S_r} softmax_t(sm_scale * q[r][h] . c_t) c_t,
+ *     lse[r][h] = log sum_t exp(sm_scale * q[r][h] . c_t)   (natural log).
+ * Block ids outside [0, n/4) are skipped.  An empty set gives out = 0 and
+ * lse = -inf.
+ *
+ *   q         bf16 [rows, heads, latent]
+ *   latent    bf16; row r reads tokens latent + r*seq_stride + t*latent,
+ *             t < cap_tok (seq_stride 0: all rows share one cache)
+ *   idx,count as produced by spx_topk_blocks
+ *   n_vis     DEVICE int64 [rows]   (clamped to min(max_len, cap_tok))
+ *   out       bf16 [rows, heads, latent]
+ *   lse       float [rows, heads] or NULL
+ *   ws        workspace of spx_attn_workspace_size(d, rows, max_len) bytes
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_attn_workspace_size(const spx_dims* d, int32_t rows,
+                                   int64_t max_len, size_t* bytes);
+SPX_API spx_status spx_sparse_mla_attn(const spx_dims* d, int32_t rows, const void* q,
+                               const void* latent, int64_t seq_stride,
+                               int64_t cap_tok, const int32_t* idx,
+                               const int32_t* count, const int64_t* n_vis,
+                               int64_t max_len, void* out, float* lse, void* ws,
+                               size_t ws_bytes, spx_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Fused decode step: steps 1-4 for one new token per sequence, in one call.
+ * If raw_k is non-NULL the step first appends raw_k[b] (bf16 [B, 1, idx_dim])
+ * at position len_dev[b], and the query sees n = len_dev[b] + 1 tokens;
+ * with raw_k NULL nothing is appended and n = len_dev[b].  The result is
+ * identical, bit for bit, to calling spx_pool_append, spx_index_score,
+ * spx_topk_blocks and spx_sparse_mla_attn in turn.
+ *
+ *   latent    bf16 [B, cap_tok, latent]  (the new token's latent row must
+ *             already be stored at position len_dev[b])
+ *   idx_out, count_out   optional (NULL) copies of the selection, e.g. to
+ *             reuse it in the next layers
+ *   max_len   host bound on n for every sequence; <= pool*cap_blk, <= cap_tok
+ *   ws        workspace of spx_decode_workspace_size(d, B, max_len) bytes
+ *   timing    optional events around the scoring launch (may be NULL)
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_decode_workspace_size(const spx_dims* d, int32_t B,
+                                     int64_t max_len, size_t* bytes);
+SPX_API spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k,
+                            const float* pool_w, void* tail, void* pooled_k,
+                            int64_t cap_blk, const int64_t* len_dev,
+                            const void* q_idx, const float* w_head,
+                            const void* q, const void* latent, int64_t cap_tok,
+                            int64_t max_len, void* out, float* lse,
+                            int32_t* idx_out, int32_t* count_out, void* ws,
+                            size_t ws_bytes, const spx_timing* timing,
+                            spx_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Chunked causal prefill of one sequence: T new tokens appended after pos0
+ * cached tokens.  Query t (0-based in the chunk, absolute position pos0 + t)
+ * sees n_t = pos0 + t + 1 tokens: it scores the floor(n_t/4) complete blocks
+ * (including blocks completed inside this chunk), keeps the top 512, and
+ * always keeps its own partial block.  Steps: IndexPool append of the T raw
+ * keys, causal indexer scoring as one tensor-core GEMM (keys x (queries x
+ * heads)), per-query top-k, sparse attention.
+ *
+ *   raw_k     bf16 [T, idx_dim];  q_idx bf16 [T, idx_heads, idx_dim]
+ *   w_head    float [T, idx_heads];  q bf16 [T, heads, latent]
+ *   tail, pooled_k   the sequence's caches, as for spx_pool_append (B = 1)
+ *   pos0      HOST int64: tokens already cached; pos0 + T <= pool*cap_blk
+ *   latent    bf16 [cap_tok, latent], rows 0 .. pos0+T-1 filled
+ *   out       bf16 [T, heads, latent];  lse float [T, heads] or NULL
+ *   ws        workspace of spx_prefill_workspace_size(d, T, pos0) bytes
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_prefill_workspace_size(const spx_dims* d, int32_t T,
+                                      int64_t pos0, size_t* bytes);
+SPX_API spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k,
+                             const float* pool_w, void* tail, void* pooled_k,
+                             int64_t cap_blk, int64_t pos0, const void* q_idx,
+                             const float* w_head, const void* q,
+                             const void* latent, int64_t cap_tok, void* out,
+                             float* lse, int32_t* idx_out, int32_t* count_out,
+                             void* ws, size_t ws_bytes,
+                             const spx_timing* timing, spx_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPX_H_ */

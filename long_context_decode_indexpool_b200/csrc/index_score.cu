@@ -1,0 +1,404 @@
+// Lightning-indexer scoring on the 5th-generation tensor cores.
+//
+// [W4] "GLM-5.3-Flash vs Qwen3.8-Flash-Next: 두 중국 AI 연구소가 독립적으로 같은
+// 모델 설계로 수렴한 이유", section "수렴점 2 — 4배 압축 후 2,048 토큰만 유지":
+// a 32-head lightning indexer scores the pooled keys.  The score of block b
+// for query t is s = sum_h w_{t,h} ReLU(q_{t,h} . k_pool[b]) (the DeepSeek
+// indexer form named by [W3] "GLM-5.3 Sparse Attention은 연산량을 줄이지만 HBM
+// 수요는 지속된다", section "GLM-5.3 Sparse Attention이 실제로 바꾸는 것").
+//
+// The dot products form a GEMM with the keys as the M side:
+//   D[128 keys x N] = K_tile[128 x 128] * Qg[N x 128]^T,  N = 32 * NQ,
+// where Qg stacks the 32 heads of NQ queries that share the key tiles (decode:
+// NQ = 1, one query per sequence, its own keys; prefill: NQ = 8 consecutive
+// queries of one sequence).  With the keys on M, TMEM lane i holds key i and
+// its N head dot products sit in that lane's columns, so the ReLU-weighted
+// sum over heads is a per-thread loop in the epilogue: no cross-thread
+// reduction at all.
+//
+// Roles (192 threads, one CTA per SM, persistent over a contiguous range of
+// (query group, key tile) work items):
+//   warp 0      TMA producer: key tiles into a kStages ring (two 16 KiB
+//               boxes of 64 dims, 128-byte swizzle), query groups into
+//               kQSlots slots.
+//   warp 1      allocates TMEM; one lane issues 8 tcgen05.mma (K = 16 each)
+//               per tile into one of two TMEM accumulators.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator row, ReLU, weighted
+//               head sum in fp32, causal/length mask, store of fp32 scores.
+// Every wait is bounded; on a timeout the CTA drains and exits with the
+// device error word set.
+#include "spx_device.cuh"
+#include "spx_internal.h"
+
+namespace spx {
+
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr int kTileM = 128;
+constexpr int kHalfBytes = kTileM * 64 * 2;  // 128 rows x 128 bytes
+constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KiB: one tile of 128 keys
+constexpr int kThreads = 192;
+
+template <int NQ>
+struct Cfg {
+  static constexpr int kN = 32 * NQ;
+  static constexpr int kStages = NQ == 1 ? 6 : 4;
+  static constexpr int kQSlots = NQ == 1 ? 2 : 1;
+  static constexpr int kQHalf = kN * 128;
+  static constexpr int kQBytes = 2 * kQHalf;
+  static constexpr int kTmemCols = 2 * kN;
+  static constexpr int kBarOff = kStages * kTileBytes + kQSlots * kQBytes + kN * 4 + NQ * 8;
+  static constexpr int kNumBars = 2 * kStages + 2 * kQSlots + 4 + 1;
+  static constexpr int kSmem = 1024 + kBarOff + kNumBars * 8 + 16;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, kN);
+};
+
+struct KParams {
+  const float* w_head;
+  const int64_t* n_vis;
+  float* scores;
+  int64_t score_stride;
+  int64_t max_len;
+  int rows;
+  int groups;
+  int shared_keys;
+};
+
+template <int NQ>
+__device__ __forceinline__ int64_t row_blocks(const KParams& p, int row) {
+  int64_t n = p.n_vis[row];
+  n = n < 0 ? 0 : (n > p.max_len ? p.max_len : n);
+  return n / kPool;
+}
+
+template <int NQ>
+__device__ __forceinline__ int group_tiles(const KParams& p, int g) {
+  int64_t nb = 0;
+#pragma unroll
+  for (int j = 0; j < NQ; ++j) {
+    const int r = g * NQ + j;
+    if (r < p.rows) {
+      const int64_t v = row_blocks<NQ>(p, r);
+      nb = v > nb ? v : nb;
+    }
+  }
+  return static_cast<int>((nb + kTileM - 1) / kTileM);
+}
+
+template <int NQ>
+struct Walker {
+  int g, t, nt;
+  __device__ void init(const KParams& p, int g0, int t0) {
+    g = g0;
+    t = t0;
+    nt = group_tiles<NQ>(p, g0);
+  }
+  __device__ void advance(const KParams& p) {
+    if (++t >= nt) {
+      t = 0;
+      do {
+        ++g;
+        nt = (g < p.groups) ? group_tiles<NQ>(p, g) : 1;
+      } while (nt == 0);
+    }
+  }
+};
+
+__device__ __forceinline__ void named_sync_epilogue() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+template <int NQ>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_index_score(const __grid_constant__ CUtensorMap map_k,
+                  const __grid_constant__ CUtensorMap map_q, const KParams p) {
+  using C = Cfg<NQ>;
+  extern __shared__ uint8_t dyn_smem[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* a_smem = smem;
+  uint8_t* q_smem = smem + C::kStages * kTileBytes;
+  float* w_smem = reinterpret_cast<float*>(q_smem + C::kQSlots * C::kQBytes);
+  int64_t* nb_smem = reinterpret_cast<int64_t*>(w_smem + C::kN);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = full + C::kStages;
+  uint64_t* qfull = empty + C::kStages;
+  uint64_t* qempty = qfull + C::kQSlots;
+  uint64_t* accfull = qempty + C::kQSlots;
+  uint64_t* accempty = accfull + 2;
+  uint64_t* drain = accempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  __shared__ int s_scan[33];
+  __shared__ int s_g0, s_t0;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- locate this CTA's contiguous range of work items -------------------
+  int64_t total = 0;
+  for (int base = 0; base < p.groups; base += kThreads) {
+    const int g = base + tid;
+    int sum;
+    block_excl_scan(g < p.groups ? group_tiles<NQ>(p, g) : 0, s_scan, &sum);
+    total += sum;
+  }
+  const int64_t lo = total * blockIdx.x / gridDim.x;
+  const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
+  if (lo >= hi) return;  // uniform
+  {
+    int64_t run = 0;
+    for (int base = 0; base < p.groups; base += kThreads) {
+      const int g = base + tid;
+      const int c = g < p.groups ? group_tiles<NQ>(p, g) : 0;
+      int sum;
+      const int ex = block_excl_scan(c, s_scan, &sum);
+      if (c > 0 && run + ex <= lo && lo < run + ex + c) {
+        s_g0 = g;
+        s_t0 = static_cast<int>(lo - run - ex);
+      }
+      run += sum;
+      if (run > lo) break;  // uniform
+    }
+  }
+  const int n_items = static_cast<int>(hi - lo);
+
+  // ---- barriers and TMEM ---------------------------------------------------
+  if (tid == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < C::kQSlots; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qempty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&accfull[s], 1);
+      mbar_init(&accempty[s], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ======================= TMA producer =================================
+    if (lane == 0) {
+      prefetch_tensormap(&map_k);
+      prefetch_tensormap(&map_q);
+      Walker<NQ> w;
+      w.init(p, s_g0, s_t0);
+      int stage = 0, cur_g = -1, qs = C::kQSlots - 1;
+      uint32_t ph = 0, qe_ph[2] = {0, 0};
+      int issued = 0, q_issued_slot = -1;
+      uint32_t q_issued_ph = 0;
+      for (int i = 0; i < n_items; ++i) {
+        if (w.g != cur_g) {
+          qs = (qs + 1) % C::kQSlots;
+          if (!mbar_wait(&qempty[qs], qe_ph[qs] ^ 1, abort_flag)) break;
+          qe_ph[qs] ^= 1;
+          uint8_t* dst = q_smem + qs * C::kQBytes;
+          mbar_arrive_expect_tx(&qfull[qs], C::kQBytes);
+          tma_load_2d(dst, &map_q, &qfull[qs], 0, w.g * C::kN);
+          tma_load_2d(dst + C::kQHalf, &map_q, &qfull[qs], 64, w.g * C::kN);
+          q_issued_slot = qs;
+          q_issued_ph = qe_ph[qs] ^ 1;
+          cur_g = w.g;
+        }
+        if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) break;
+        uint8_t* dst = a_smem + stage * kTileBytes;
+        const int kb = p.shared_keys ? 0 : w.g;
+        mbar_arrive_expect_tx(&full[stage], kTileBytes);
+        tma_load_3d(dst, &map_k, &full[stage], 0, w.t * kTileM, kb);
+        tma_load_3d(dst + kHalfBytes, &map_k, &full[stage], 64, w.t * kTileM, kb);
+        ++issued;
+        if (++stage == C::kStages) {
+          stage = 0;
+          ph ^= 1;
+        }
+        w.advance(p);
+      }
+      if (*abort_flag) {
+        // Let the copies already issued land before the CTA exits.
+        int first = issued > C::kStages ? issued - C::kStages : 0;
+        for (int i = first; i < issued; ++i) {
+          volatile int no_abort = 0;
+          mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1, &no_abort);
+        }
+        if (q_issued_slot >= 0) {
+          volatile int no_abort = 0;
+          mbar_wait(&qfull[q_issued_slot], q_issued_ph, &no_abort);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer ====================================
+    if (lane == 0) {
+      Walker<NQ> w;
+      w.init(p, s_g0, s_t0);
+      int stage = 0, acc = 0, cur_g = -1, qs = C::kQSlots - 1;
+      uint32_t ph = 0, acc_ph = 0, qf_ph[2] = {0, 0};
+      const uint32_t a_base = smem_u32(a_smem);
+      const uint32_t q_base = smem_u32(q_smem);
+      for (int i = 0; i < n_items; ++i) {
+        if (w.g != cur_g) {
+          if (cur_g >= 0) umma_commit(&qempty[qs]);
+          qs = (qs + 1) % C::kQSlots;
+          if (!mbar_wait(&qfull[qs], qf_ph[qs], abort_flag)) break;
+          qf_ph[qs] ^= 1;
+          cur_g = w.g;
+        }
+        if (!mbar_wait(&accempty[acc], acc_ph ^ 1, abort_flag)) break;
+        if (!mbar_wait(&full[stage], ph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::kN);
+        const uint32_t a0 = a_base + stage * kTileBytes;
+        const uint32_t b0 = q_base + qs * C::kQBytes;
+#pragma unroll
+        for (int k = 0; k < kIdxDim / 16; ++k) {
+          const uint32_t koff = (k & 3) * 32;
+          const uint64_t ad = sdesc_kmajor_sw128(a0 + (k >> 2) * kHalfBytes + koff);
+          const uint64_t bd = sdesc_kmajor_sw128(b0 + (k >> 2) * C::kQHalf + koff);
+          umma_bf16(d, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&empty[stage]);
+        umma_commit(&accfull[acc]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          ph ^= 1;
+        }
+        acc ^= 1;
+        if (acc == 0) acc_ph ^= 1;
+        w.advance(p);
+      }
+      // Wait for every MMA issued by this thread before TMEM is released.
+      umma_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+  } else {
+    // ======================= epilogue =====================================
+    const int quarter = warp & 3;  // TMEM lanes quarter*32 .. +31
+    const int et = tid - 64;       // 0..127
+    const int row_in_tile = quarter * 32 + lane;
+    Walker<NQ> w;
+    w.init(p, s_g0, s_t0);
+    int acc = 0, cur_g = -1;
+    uint32_t acc_ph = 0;
+    for (int i = 0; i < n_items; ++i) {
+      if (w.g != cur_g) {
+        named_sync_epilogue();
+        for (int j = et; j < C::kN; j += 128) {
+          const int r = w.g * NQ + j / kIdxHeads;
+          w_smem[j] = r < p.rows ? p.w_head[static_cast<int64_t>(r) * kIdxHeads + (j % kIdxHeads)] : 0.f;
+        }
+        if (et < NQ) {
+          const int r = w.g * NQ + et;
+          nb_smem[et] = r < p.rows ? row_blocks<NQ>(p, r) : 0;
+        }
+        named_sync_epilogue();
+        cur_g = w.g;
+      }
+      if (!mbar_wait(&accfull[acc], acc_ph, abort_flag)) break;
+      tc_fence_after();
+      const int64_t blk = static_cast<int64_t>(w.t) * kTileM + row_in_tile;
+#pragma unroll 1
+      for (int j = 0; j < NQ; ++j) {
+        const int r = w.g * NQ + j;
+        if (r >= p.rows) break;  // uniform
+        float v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(acc * C::kN + j * 32),
+                           v);
+        const float* wj = w_smem + j * kIdxHeads;
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < kIdxHeads; ++h) s = __fmaf_rn(wj[h], v[h] > 0.f ? v[h] : 0.f, s);
+        if (blk < nb_smem[j]) p.scores[static_cast<int64_t>(r) * p.score_stride + blk] = s;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_ph ^= 1;
+      w.advance(p);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+template <int NQ>
+cudaError_t launch_nq(const ScoreArgs& a, cudaStream_t stream) {
+  using C = Cfg<NQ>;
+  CUtensorMap map_k, map_q;
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(kIdxDim), static_cast<uint64_t>(a.cap_blk),
+                              static_cast<uint64_t>(a.key_batches)};
+    const uint64_t strides[2] = {kIdxDim * 2ull, static_cast<uint64_t>(a.cap_blk) * kIdxDim * 2ull};
+    const uint32_t box[3] = {64, kTileM, 1};
+    if (!encode_tensor_map(&map_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.pooled_k, dims,
+                           strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(kIdxDim),
+                              static_cast<uint64_t>(a.rows) * kIdxHeads};
+    const uint64_t strides[1] = {kIdxDim * 2ull};
+    const uint32_t box[2] = {64, static_cast<uint32_t>(C::kN)};
+    if (!encode_tensor_map(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q_idx, dims, strides,
+                           box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_index_score<NQ>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  KParams p;
+  p.w_head = a.w_head;
+  p.n_vis = a.n_vis;
+  p.scores = a.scores;
+  p.score_stride = a.score_stride;
+  p.max_len = a.max_len;
+  p.rows = a.rows;
+  p.groups = (a.rows + NQ - 1) / NQ;
+  p.shared_keys = a.key_batches == 1 && a.rows > 1 ? 1 : 0;
+  if (NQ > 1) p.shared_keys = 1;
+  const int64_t max_blk = a.max_len / kPool;
+  const int64_t tiles_ub = static_cast<int64_t>(p.groups) * ((max_blk + kTileM - 1) / kTileM);
+  if (tiles_ub == 0) return cudaSuccess;
+  const int grid = static_cast<int>(tiles_ub < a.num_sms ? tiles_ub : a.num_sms);
+  k_index_score<NQ><<<grid, kThreads, C::kSmem, stream>>>(map_k, map_q, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_index_score(const ScoreArgs& a, cudaStream_t stream) {
+  if (a.nq == 1) return launch_nq<1>(a, stream);
+  if (a.nq == 8) return launch_nq<8>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace spx

@@ -1,0 +1,527 @@
+// C ABI of libspx: host-side validation, workspace layout and launch
+// sequencing.  Every check runs before the first launch of a call, so a call
+// that returns an error has enqueued nothing.  No allocation, no
+// synchronisation (except spx_device_error, which says so).
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "spx.h"
+#include "spx_device.cuh"
+#include "spx_internal.h"
+
+namespace spx {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
+  return fn(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gd, gs, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+int device_sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+}  // namespace spx
+
+using namespace spx;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool al4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+spx_status check_dims(const spx_dims* d) {
+  if (!d) return SPX_ERR_INVALID_ARG;
+  if (d->idx_heads != kIdxHeads || d->idx_dim != kIdxDim || d->pool != kPool ||
+      d->topk_blocks != kTopK || d->latent != kLatent)
+    return SPX_ERR_UNSUPPORTED;
+  if (d->heads < kHeadGroup || d->heads > kMaxHeads || d->heads % kHeadGroup != 0)
+    return SPX_ERR_UNSUPPORTED;
+  if (!std::isfinite(d->sm_scale) || !(d->sm_scale > 0.f)) return SPX_ERR_INVALID_ARG;
+  return SPX_OK;
+}
+
+spx_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SPX_OK : SPX_ERR_CUDA; }
+
+// Score row stride used inside the fused calls: max_blk rounded up to 64.
+inline int64_t score_stride_for(int64_t max_len) {
+  const int64_t mb = max_len / kPool;
+  return (mb + 63) / 64 * 64;
+}
+
+// Workspace of the fused calls:
+//   n_vis [rows] int64 | scores [rows, stride] f32 | idx [rows, 512] | count [rows]
+//   | top-k scratch | attention scratch
+struct FusedLayout {
+  size_t nvis, scores, idx, count, topk, attn, total;
+  int64_t stride;
+  TopkPlan tp;
+  AttnPlan ap;
+};
+
+FusedLayout fused_layout(int rows, int heads, int64_t max_len) {
+  FusedLayout L{};
+  L.stride = score_stride_for(max_len);
+  L.tp = plan_topk(rows, max_len);
+  L.ap = plan_attn(rows, heads, max_len, device_sm_count());
+  size_t o = 0;
+  L.nvis = o;
+  o += up(static_cast<size_t>(rows) * 8);
+  L.scores = o;
+  o += up(static_cast<size_t>(rows) * L.stride * 4);
+  L.idx = o;
+  o += up(static_cast<size_t>(rows) * kTopK * 4);
+  L.count = o;
+  o += up(static_cast<size_t>(rows) * 4);
+  L.topk = o;
+  o += up(L.tp.ws_bytes);
+  L.attn = o;
+  o += up(L.ap.ws_bytes);
+  L.total = o;
+  return L;
+}
+
+spx_status check_pool_w(const float* w, float out[4]) {
+  if (!w) return SPX_ERR_INVALID_ARG;
+  double s = 0.0;
+  for (int i = 0; i < kPool; ++i) {
+    if (!std::isfinite(w[i])) return SPX_ERR_INVALID_ARG;
+    out[i] = w[i];
+    s += w[i];
+  }
+  if (std::fabs(s - 1.0) > 1e-6) return SPX_ERR_INVALID_ARG;
+  return SPX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spx_status_string(spx_status s) {
+  switch (s) {
+    case SPX_OK: return "SPX_OK";
+    case SPX_ERR_INVALID_ARG: return "SPX_ERR_INVALID_ARG";
+    case SPX_ERR_SHAPE: return "SPX_ERR_SHAPE";
+    case SPX_ERR_UNSUPPORTED: return "SPX_ERR_UNSUPPORTED";
+    case SPX_ERR_WORKSPACE: return "SPX_ERR_WORKSPACE";
+    case SPX_ERR_CUDA: return "SPX_ERR_CUDA";
+    case SPX_ERR_DEVICE: return "SPX_ERR_DEVICE";
+  }
+  return "SPX_ERR_UNKNOWN";
+}
+
+const char* spx_version(void) { return "libspx 0.1.0 (sm_100a)"; }
+
+uint64_t spx_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+spx_status spx_dims_init(spx_dims* d, int32_t heads, float sm_scale) {
+  if (!d) return SPX_ERR_INVALID_ARG;
+  d->idx_heads = kIdxHeads;
+  d->idx_dim = kIdxDim;
+  d->pool = kPool;
+  d->topk_blocks = kTopK;
+  d->heads = heads;
+  d->latent = kLatent;
+  d->sm_scale = sm_scale;
+  return check_dims(d);
+}
+
+spx_status spx_device_error(int32_t* code, spx_stream stream) {
+  if (!code) return SPX_ERR_INVALID_ARG;
+  int v = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return SPX_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SPX_ERR_CUDA;
+  const int zero = 0;
+  if (v != 0) {
+    if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) !=
+        cudaSuccess)
+      return SPX_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SPX_ERR_CUDA;
+  }
+  *code = v;
+  return SPX_OK;
+}
+
+// ---------------------------------------------------------------------------
+spx_status spx_pool_append(const spx_dims* d, int32_t B, const void* raw_k, int32_t n_new,
+                           const float* pool_w, void* tail, void* pooled_k, int64_t cap_blk,
+                           const int64_t* len_dev, int64_t max_len, spx_stream stream) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  float w[4];
+  if ((st = check_pool_w(pool_w, w)) != SPX_OK) return st;
+  if (B < 1 || B > 65535 || n_new < 0 || cap_blk < 1) return SPX_ERR_SHAPE;
+  if (max_len < n_new || max_len > kPool * cap_blk) return SPX_ERR_SHAPE;
+  if (!tail || !pooled_k || !len_dev || (n_new > 0 && !raw_k)) return SPX_ERR_INVALID_ARG;
+  if (!al16(tail) || !al16(pooled_k) || (raw_k && !al16(raw_k)) || (len_dev && !al4(len_dev)))
+    return SPX_ERR_INVALID_ARG;
+  if (n_new == 0) return SPX_OK;
+  PoolAppendArgs a{};
+  a.B = B;
+  a.raw_k = raw_k;
+  a.n_new = n_new;
+  for (int i = 0; i < 4; ++i) a.w[i] = w[i];
+  a.tail = tail;
+  a.pooled_k = pooled_k;
+  a.cap_blk = cap_blk;
+  a.len_dev = len_dev;
+  a.len_host = 0;
+  a.max_len = max_len;
+  a.nvis_out = nullptr;
+  return cuda_status(launch_pool_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+spx_status spx_index_score(const spx_dims* d, int32_t B, const void* q_idx, const float* w_head,
+                           const void* pooled_k, int64_t cap_blk, const int64_t* n_vis,
+                           int64_t max_len, float* scores, int64_t score_stride,
+                           spx_stream stream) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (B < 1 || cap_blk < 1 || max_len < 0 || max_len > kPool * cap_blk) return SPX_ERR_SHAPE;
+  if (cap_blk > (int64_t(1) << 31) - 1 || static_cast<int64_t>(B) * kIdxHeads > (1ll << 31) - 1)
+    return SPX_ERR_SHAPE;
+  if (score_stride < max_len / kPool) return SPX_ERR_SHAPE;
+  if (!q_idx || !w_head || !pooled_k || !n_vis || !scores) return SPX_ERR_INVALID_ARG;
+  if (!al16(q_idx) || !al16(pooled_k) || !al4(w_head) || !al4(scores)) return SPX_ERR_INVALID_ARG;
+  ScoreArgs a{};
+  a.nq = 1;
+  a.rows = B;
+  a.key_batches = B;
+  a.q_idx = q_idx;
+  a.w_head = w_head;
+  a.pooled_k = pooled_k;
+  a.cap_blk = cap_blk;
+  a.n_vis = n_vis;
+  a.max_len = max_len;
+  a.scores = scores;
+  a.score_stride = score_stride;
+  a.num_sms = device_sm_count();
+  return cuda_status(launch_index_score(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+spx_status spx_topk_workspace_size(const spx_dims* d, int32_t rows, int64_t max_len,
+                                   size_t* bytes) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (!bytes) return SPX_ERR_INVALID_ARG;
+  if (rows < 1 || rows > 65535 || max_len < 0) return SPX_ERR_SHAPE;
+  *bytes = plan_topk(rows, max_len).ws_bytes;
+  return SPX_OK;
+}
+
+spx_status spx_topk_blocks(const spx_dims* d, int32_t rows, const float* scores,
+                           int64_t score_stride, const int64_t* n_vis, int64_t max_len,
+                           int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                           spx_stream stream) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (rows < 1 || rows > 65535 || max_len < 0) return SPX_ERR_SHAPE;
+  if (max_len / kPool > (int64_t(1) << 31) - 1) return SPX_ERR_SHAPE;
+  if (score_stride < max_len / kPool) return SPX_ERR_SHAPE;
+  if (!scores || !n_vis || !idx || !count) return SPX_ERR_INVALID_ARG;
+  if (!al4(scores) || !al4(idx) || !al4(count)) return SPX_ERR_INVALID_ARG;
+  const TopkPlan p = plan_topk(rows, max_len);
+  if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes || !al16(ws))) return SPX_ERR_WORKSPACE;
+  return cuda_status(launch_topk(p, scores, score_stride, n_vis, max_len, idx, count, ws,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+spx_status spx_attn_workspace_size(const spx_dims* d, int32_t rows, int64_t max_len,
+                                   size_t* bytes) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (!bytes) return SPX_ERR_INVALID_ARG;
+  if (rows < 1 || rows > 65535 || max_len < 0) return SPX_ERR_SHAPE;
+  *bytes = plan_attn(rows, d->heads, max_len, device_sm_count()).ws_bytes;
+  return SPX_OK;
+}
+
+spx_status spx_sparse_mla_attn(const spx_dims* d, int32_t rows, const void* q, const void* latent,
+                               int64_t seq_stride, int64_t cap_tok, const int32_t* idx,
+                               const int32_t* count, const int64_t* n_vis, int64_t max_len,
+                               void* out, float* lse, void* ws, size_t ws_bytes,
+                               spx_stream stream) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (rows < 1 || rows > 65535 || max_len < 0 || cap_tok < 1 || seq_stride < 0)
+    return SPX_ERR_SHAPE;
+  if (seq_stride != 0 && seq_stride < cap_tok * kLatent) return SPX_ERR_SHAPE;
+  if (!q || !latent || !idx || !count || !n_vis || !out) return SPX_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(latent) || !al16(out) || !al4(idx) || !al4(count) || (lse && !al4(lse)))
+    return SPX_ERR_INVALID_ARG;
+  const AttnPlan p = plan_attn(rows, d->heads, max_len, device_sm_count());
+  if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes || !al16(ws))) return SPX_ERR_WORKSPACE;
+  AttnArgs a{};
+  a.q = q;
+  a.latent = latent;
+  a.seq_stride = seq_stride;
+  a.cap_tok = cap_tok;
+  a.idx = idx;
+  a.count = count;
+  a.n_vis = n_vis;
+  a.max_len = max_len;
+  a.sm_scale = d->sm_scale;
+  a.out = out;
+  a.lse = lse;
+  a.ws = ws;
+  return cuda_status(launch_attn(p, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------------------
+spx_status spx_decode_workspace_size(const spx_dims* d, int32_t B, int64_t max_len,
+                                     size_t* bytes) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (!bytes) return SPX_ERR_INVALID_ARG;
+  if (B < 1 || B > 65535 || max_len < 0) return SPX_ERR_SHAPE;
+  *bytes = fused_layout(B, d->heads, max_len).total;
+  return SPX_OK;
+}
+
+spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, const float* pool_w,
+                            void* tail, void* pooled_k, int64_t cap_blk, const int64_t* len_dev,
+                            const void* q_idx, const float* w_head, const void* q,
+                            const void* latent, int64_t cap_tok, int64_t max_len, void* out,
+                            float* lse, int32_t* idx_out, int32_t* count_out, void* ws,
+                            size_t ws_bytes, const spx_timing* timing, spx_stream stream) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  float w[4] = {0.f, 0.f, 0.f, 0.f};
+  if (raw_k && (st = check_pool_w(pool_w, w)) != SPX_OK) return st;
+  if (B < 1 || B > 65535 || cap_blk < 1 || cap_tok < 1 || max_len < 1) return SPX_ERR_SHAPE;
+  if (max_len > kPool * cap_blk || max_len > cap_tok) return SPX_ERR_SHAPE;
+  if (cap_blk > (int64_t(1) << 31) - 1 || static_cast<int64_t>(B) * kIdxHeads > (1ll << 31) - 1)
+    return SPX_ERR_SHAPE;
+  if (!pooled_k || !len_dev || !q_idx || !w_head || !q || !latent || !out)
+    return SPX_ERR_INVALID_ARG;
+  if (raw_k && !tail) return SPX_ERR_INVALID_ARG;
+  if (!al16(pooled_k) || !al16(q_idx) || !al16(q) || !al16(latent) || !al16(out) ||
+      !al4(w_head) || !al4(len_dev) || (raw_k && (!al16(raw_k) || !al16(tail))) ||
+      (lse && !al4(lse)) || (idx_out && !al4(idx_out)) || (count_out && !al4(count_out)))
+    return SPX_ERR_INVALID_ARG;
+  const FusedLayout L = fused_layout(B, d->heads, max_len);
+  if (!ws || ws_bytes < L.total || !al16(ws)) return SPX_ERR_WORKSPACE;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int64_t* n_vis = reinterpret_cast<int64_t*>(base + L.nvis);
+  float* scores = reinterpret_cast<float*>(base + L.scores);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + L.idx);
+  int32_t* count = count_out ? count_out : reinterpret_cast<int32_t*>(base + L.count);
+
+  // 1. append (or just copy the lengths) -> n_vis
+  PoolAppendArgs pa{};
+  pa.B = B;
+  pa.raw_k = raw_k;
+  pa.n_new = raw_k ? 1 : 0;
+  for (int i = 0; i < 4; ++i) pa.w[i] = w[i];
+  pa.tail = tail;
+  pa.pooled_k = pooled_k;
+  pa.cap_blk = cap_blk;
+  pa.len_dev = len_dev;
+  pa.len_host = 0;
+  pa.max_len = max_len;
+  pa.nvis_out = n_vis;
+  cudaError_t e = launch_pool_append(pa, s);
+  if (e != cudaSuccess) return SPX_ERR_CUDA;
+
+  // 2. indexer scores
+  if (timing && timing->score_begin &&
+      cudaEventRecord(static_cast<cudaEvent_t>(timing->score_begin), s) != cudaSuccess)
+    return SPX_ERR_CUDA;
+  ScoreArgs sa{};
+  sa.nq = 1;
+  sa.rows = B;
+  sa.key_batches = B;
+  sa.q_idx = q_idx;
+  sa.w_head = w_head;
+  sa.pooled_k = pooled_k;
+  sa.cap_blk = cap_blk;
+  sa.n_vis = n_vis;
+  sa.max_len = max_len;
+  sa.scores = scores;
+  sa.score_stride = L.stride;
+  sa.num_sms = device_sm_count();
+  if ((e = launch_index_score(sa, s)) != cudaSuccess) return SPX_ERR_CUDA;
+  if (timing && timing->score_end &&
+      cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
+    return SPX_ERR_CUDA;
+
+  // 3. top-k
+  if ((e = launch_topk(L.tp, scores, L.stride, n_vis, max_len, idx, count, base + L.topk, s)) !=
+      cudaSuccess)
+    return SPX_ERR_CUDA;
+
+  // 4. attention
+  AttnArgs aa{};
+  aa.q = q;
+  aa.latent = latent;
+  aa.seq_stride = cap_tok * kLatent;
+  aa.cap_tok = cap_tok;
+  aa.idx = idx;
+  aa.count = count;
+  aa.n_vis = n_vis;
+  aa.max_len = max_len;
+  aa.sm_scale = d->sm_scale;
+  aa.out = out;
+  aa.lse = lse;
+  aa.ws = base + L.attn;
+  return cuda_status(launch_attn(L.ap, aa, s));
+}
+
+// ---------------------------------------------------------------------------
+spx_status spx_prefill_workspace_size(const spx_dims* d, int32_t T, int64_t pos0,
+                                      size_t* bytes) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (!bytes) return SPX_ERR_INVALID_ARG;
+  if (T < 1 || T > 65535 || pos0 < 0) return SPX_ERR_SHAPE;
+  *bytes = fused_layout(T, d->heads, pos0 + T).total;
+  return SPX_OK;
+}
+
+spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, const float* pool_w,
+                             void* tail, void* pooled_k, int64_t cap_blk, int64_t pos0,
+                             const void* q_idx, const float* w_head, const void* q,
+                             const void* latent, int64_t cap_tok, void* out, float* lse,
+                             int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
+                             const spx_timing* timing, spx_stream stream) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  float w[4];
+  if ((st = check_pool_w(pool_w, w)) != SPX_OK) return st;
+  if (T < 1 || T > 65535 || pos0 < 0 || cap_blk < 1 || cap_tok < 1) return SPX_ERR_SHAPE;
+  const int64_t max_len = pos0 + T;
+  if (max_len > kPool * cap_blk || max_len > cap_tok) return SPX_ERR_SHAPE;
+  if (cap_blk > (int64_t(1) << 31) - 1) return SPX_ERR_SHAPE;
+  if (!raw_k || !tail || !pooled_k || !q_idx || !w_head || !q || !latent || !out)
+    return SPX_ERR_INVALID_ARG;
+  if (!al16(raw_k) || !al16(tail) || !al16(pooled_k) || !al16(q_idx) || !al16(q) ||
+      !al16(latent) || !al16(out) || !al4(w_head) || (lse && !al4(lse)) ||
+      (idx_out && !al4(idx_out)) || (count_out && !al4(count_out)))
+    return SPX_ERR_INVALID_ARG;
+  const FusedLayout L = fused_layout(T, d->heads, max_len);
+  if (!ws || ws_bytes < L.total || !al16(ws)) return SPX_ERR_WORKSPACE;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int64_t* n_vis = reinterpret_cast<int64_t*>(base + L.nvis);
+  float* scores = reinterpret_cast<float*>(base + L.scores);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + L.idx);
+  int32_t* count = count_out ? count_out : reinterpret_cast<int32_t*>(base + L.count);
+
+  PoolAppendArgs pa{};
+  pa.B = 1;
+  pa.raw_k = raw_k;
+  pa.n_new = T;
+  for (int i = 0; i < 4; ++i) pa.w[i] = w[i];
+  pa.tail = tail;
+  pa.pooled_k = pooled_k;
+  pa.cap_blk = cap_blk;
+  pa.len_dev = nullptr;
+  pa.len_host = pos0;
+  pa.max_len = max_len;
+  pa.nvis_out = nullptr;
+  cudaError_t e = launch_pool_append(pa, s);
+  if (e != cudaSuccess) return SPX_ERR_CUDA;
+  if ((e = launch_prefill_nvis(n_vis, T, pos0, s)) != cudaSuccess) return SPX_ERR_CUDA;
+
+  if (timing && timing->score_begin &&
+      cudaEventRecord(static_cast<cudaEvent_t>(timing->score_begin), s) != cudaSuccess)
+    return SPX_ERR_CUDA;
+  ScoreArgs sa{};
+  sa.nq = 8;
+  sa.rows = T;
+  sa.key_batches = 1;
+  sa.q_idx = q_idx;
+  sa.w_head = w_head;
+  sa.pooled_k = pooled_k;
+  sa.cap_blk = cap_blk;
+  sa.n_vis = n_vis;
+  sa.max_len = max_len;
+  sa.scores = scores;
+  sa.score_stride = L.stride;
+  sa.num_sms = device_sm_count();
+  if ((e = launch_index_score(sa, s)) != cudaSuccess) return SPX_ERR_CUDA;
+  if (timing && timing->score_end &&
+      cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
+    return SPX_ERR_CUDA;
+
+  if ((e = launch_topk(L.tp, scores, L.stride, n_vis, max_len, idx, count, base + L.topk, s)) !=
+      cudaSuccess)
+    return SPX_ERR_CUDA;
+
+  AttnArgs aa{};
+  aa.q = q;
+  aa.latent = latent;
+  aa.seq_stride = 0;
+  aa.cap_tok = cap_tok;
+  aa.idx = idx;
+  aa.count = count;
+  aa.n_vis = n_vis;
+  aa.max_len = max_len;
+  aa.sm_scale = d->sm_scale;
+  aa.out = out;
+  aa.lse = lse;
+  aa.ws = base + L.attn;
+  return cuda_status(launch_attn(L.ap, aa, s));
+}
+
+}  // extern "C"

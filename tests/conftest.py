@@ -8,6 +8,16 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def build_lib():
+    """Builds libspx.so in-tree (without importing the package, which needs it)."""
+    import importlib.util
+    path = os.path.join(ROOT, "long_context_decode_indexpool_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_spx_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size workload")

@@ -1,0 +1,185 @@
+"""Whole-layer parity: the fused decode and prefill entry points on the
+workloads of the specification, in the configuration bench.py times,
+against the fp64 oracle (block ids bit-exact, outputs within tolerance),
+plus fused == composed bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from _gpu_helpers import (LSE_ATOL, assert_attention_close, bits_of, f64_of, need_gpu,
+                          oracle_attention_rows, to_dev_bf16)
+
+pytestmark = pytest.mark.gpu
+
+
+def _decode_state(name, **kw):
+    need_gpu()
+    import bench
+    return bench.DecodeState(synth.workload(name), torch.device("cuda", 0), **kw)
+
+
+def _oracle_decode(st, rows):
+    """Oracle steps 2-4 of the given local rows; pooled keys from the oracle's own pooling."""
+    res = []
+    for b in rows:
+        raw = st.raw_keys_host(b)
+        pooled = oracle.pool(raw, st.w.pool_weights())
+        r = oracle.decode_query(st.w.q_idx_np([st.b_offset + b])[0],
+                                st.w.w_head_np([st.b_offset + b])[0].astype(np.float64), pooled,
+                                st.L, st.w.q_np([st.b_offset + b])[0],
+                                lambda pos, b=b: st.latent_rows_host(b, pos), st.w.sm_scale)
+        r["pooled_last"] = pooled[-1]
+        res.append(r)
+    return res
+
+
+def _check_decode(st, rows):
+    st.step()
+    torch.cuda.synchronize()
+    spx = need_gpu()
+    assert spx.spx_device_error() == 0
+    idx = st.idx.cpu().numpy()
+    cnt = st.count.cpu().numpy()
+    out = f64_of(st.out)
+    lse = st.lse.cpu().numpy()
+    pooled_last = bits_of(st.pooled[:, -1])
+    ref = _oracle_decode(st, rows)
+    for i, b in enumerate(rows):
+        r = ref[i]
+        assert np.array_equal(pooled_last[b], r["pooled_last"]), f"pooled block of seq {b}"
+        assert cnt[b] == r["idx"].size
+        assert np.array_equal(idx[b, :cnt[b]], r["idx"]), f"seq {b}"
+        assert (idx[b, cnt[b]:] == -1).all()
+        assert np.allclose(lse[b], r["lse"], atol=LSE_ATOL, rtol=0)
+    assert_attention_close(out[rows], np.stack([r["out"] for r in ref]), st.w.name)
+    return ref
+
+
+def test_tiny_decode():
+    st = _decode_state("tiny")
+    ref = _check_decode(st, [0])
+    assert ref[0]["positions"].size == 2048  # 512 blocks x 4, no tail (L % 4 == 0)
+
+
+def test_dense_fallback_equals_dense_attention():
+    st = _decode_state("dense")
+    ref = _check_decode(st, list(range(st.B)))
+    for r in ref:
+        assert r["idx"].tolist() == list(range(384))
+        assert r["positions"].tolist() == list(range(1536))
+
+
+def test_mid_decode_all_rows():
+    st = _decode_state("mid")
+    _check_decode(st, list(range(st.B)))
+
+
+@pytest.mark.slow
+def test_1m_decode_bench_configuration():
+    """The benchmark's workload, all four sequences, in the bench's launch configuration."""
+    st = _decode_state("1m")
+    ref = _check_decode(st, list(range(st.B)))
+    # the needles dominate the selection: most selected blocks are needles
+    for b, r in enumerate(ref):
+        nb = set(st.w.needle_blocks(b).tolist())
+        assert len(nb & set(r["idx"].tolist())) >= 256
+
+
+def test_fused_equals_composed_and_no_append_path():
+    spx = need_gpu()
+    st = _decode_state("mid", B=3)
+    st.step()
+    torch.cuda.synchronize()
+    out_f, idx_f, cnt_f, lse_f = st.out.clone(), st.idx.clone(), st.count.clone(), st.lse.clone()
+    d, B, L = st.d, st.B, st.L
+    # composed: append, score, top-k, attention
+    len_after = torch.full((B,), L, dtype=torch.int64, device="cuda")
+    spx.spx_pool_append(d, B, st.raw_new, 1, st.pool_w, st.tail, st.pooled, st.cap_blk,
+                        st.len_dev, L)
+    stride = L // 4
+    scores = torch.empty(B, stride, device="cuda")
+    spx.spx_index_score(d, B, st.q_idx, st.w_head, st.pooled, st.cap_blk, len_after, L, scores,
+                        stride)
+    idx = torch.empty_like(st.idx)
+    cnt = torch.empty_like(st.count)
+    ws = spx.workspace(spx.spx_topk_workspace_size(d, B, L), "cuda")
+    spx.spx_topk_blocks(d, B, scores, stride, len_after, L, idx, cnt, ws)
+    out = torch.empty_like(st.out)
+    lse = torch.empty_like(st.lse)
+    ws2 = spx.workspace(spx.spx_attn_workspace_size(d, B, L), "cuda")
+    spx.spx_sparse_mla_attn(d, B, st.q, st.latent, L * 512, L, idx, cnt, len_after, L, out, lse,
+                            ws2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_f) and torch.equal(cnt, cnt_f)
+    assert torch.equal(out.view(torch.int16), out_f.view(torch.int16))
+    assert torch.equal(lse, lse_f)
+    # raw_k = NULL: no append, the query sees len_dev tokens (here L after the append)
+    spx.spx_decode_fused(d, B, None, None, st.tail, st.pooled, st.cap_blk, len_after, st.q_idx,
+                         st.w_head, st.q, st.latent, st.cap_tok, L, out, lse, idx, cnt, st.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_f)
+    assert torch.equal(out.view(torch.int16), out_f.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------
+# Chunked prefill
+# ----------------------------------------------------------------------------
+def _prefill_state(pos0, T):
+    need_gpu()
+    import bench
+    return bench.PrefillState(synth.workload("prefill"), torch.device("cuda", 0), pos0=pos0, T=T)
+
+
+def _check_prefill(st, queries):
+    spx = need_gpu()
+    st.step()
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    raw = st.raw_keys_host()
+    pw = st.w.pool_weights()
+    pooled = oracle.pool(raw, pw)
+    total = st.pos0 + st.T
+    got_pooled = bits_of(st.pooled[0, : total // 4])
+    lo = st.pos0 // 4
+    assert np.array_equal(got_pooled[lo:], pooled[lo:]), "pooled blocks of the chunk"
+    idx = st.idx.cpu().numpy()
+    cnt = st.count.cpu().numpy()
+    out = f64_of(st.out)
+    lse = st.lse.cpu().numpy()
+    rows = st.pos0 + np.asarray(queries)
+    q_idx = st.w.q_idx_np(rows)
+    w_head = st.w.w_head_np(rows).astype(np.float64)
+    q = st.w.q_np(rows)
+    outs = []
+    for i, t in enumerate(queries):
+        n = st.pos0 + t + 1
+        s, sel, pos = oracle.select_query(q_idx[i], w_head[i], pooled, n)
+        assert cnt[t] == sel.size, f"query {t}"
+        assert np.array_equal(idx[t, :cnt[t]], sel), f"query {t}"
+        o, l = oracle.attention(q[i], st.w.latent_np(0, pos), st.w.sm_scale)
+        assert np.allclose(lse[t], l, atol=LSE_ATOL, rtol=0), f"query {t}"
+        outs.append(o)
+    assert_attention_close(out[list(queries)], np.stack(outs), "prefill")
+
+
+def test_prefill_small_all_queries():
+    # cache of 8190 tokens (a 2-token tail), 100 new tokens: crosses the
+    # 2048-block budget boundary and several tiles of 128 blocks
+    st = _prefill_state(8190, 100)
+    _check_prefill(st, list(range(100)))
+
+
+def test_prefill_short_context_dense():
+    # every query sees fewer than 2052 tokens: all blocks selected
+    st = _prefill_state(1000, 64)
+    _check_prefill(st, list(range(64)))
+
+
+@pytest.mark.slow
+def test_prefill_full_chunk_sampled():
+    st = _prefill_state(None, None)
+    qs = [0, 1, 2, 3, 4, 5, 6, 7, 8, 1023, 1024, 1025, 1026, 1027, 2047, 2048, 3071, 4091,
+          4092, 4093, 4094, 4095]
+    _check_prefill(st, qs)
