@@ -478,6 +478,9 @@ def run_decode(args, world, rank, local):
     ev_score = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(K)]
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for a, b in ev_score:  # torch creates its events on first record
+        a.record(stream)
+        b.record(stream)
     barrier(world)
     torch.cuda.synchronize(device)
     clocks = ClockSampler(device.index)
@@ -588,6 +591,10 @@ def run_prefill(args, world, rank, local):
                 for _ in range(K)]
     ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(K)]
+    for a, b in ev_score:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize(device)
     barrier(world)
     clocks = ClockSampler(device.index)
     clocks.start()
@@ -621,6 +628,45 @@ def run_prefill(args, world, rank, local):
     }
 
 
+def run_score_only(args, world, rank, local):
+    """The decode scoring kernel alone on the 1M workload's pooled cache
+    (no latent cache is built): for kernel profiling."""
+    spx = spx_module()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = synth.workload(args.workload)
+    st = DecodeState(w, device, b_offset=shard_offset(rank, w.B), build_latent=False)
+    B, L = st.B, st.L
+    stride = L // synth.POOL
+    n_vis = torch.full((B,), L, dtype=torch.int64, device=device)
+    spx.spx_pool_append(st.d, B, st.raw_new, 1, st.pool_w, st.tail, st.pooled, st.cap_blk,
+                        st.len_dev, L)
+    scores = torch.empty(B, stride, device=device)
+
+    def launch():
+        spx.spx_index_score(st.d, B, st.q_idx, st.w_head, st.pooled, st.cap_blk, n_vis, L, scores,
+                            stride)
+
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    stream = torch.cuda.current_stream(device)
+    for a, b in evs:
+        a.record(stream)
+        launch()
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    us = [a.elapsed_time(b) * 1e3 for a, b in evs]
+    hbm = measured_peaks()[0]
+    alg = score_algorithmic_bytes([L // synth.POOL] * B, B)
+    avg = sum(us) / len(us)
+    return {"mode": "score-only", "workload": w.name, "avg_us": avg, "min_us": min(us),
+            "achieved_gbs": alg / (avg * 1e-6) / 1e9, "frac_of_measured_hbm": alg / (avg * 1e-6) / 1e9 / hbm,
+            "algorithmic_bytes": alg}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -629,6 +675,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("spx", "reference"), default="spx")
     ap.add_argument("--workload", default="1m", choices=synth.WORKLOADS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--score-only", action="store_true",
+                    help="time the decode scoring kernel alone (profiling aid)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
@@ -637,12 +685,15 @@ def main(argv=None):
         return 1
     world, rank, local = dist_setup()
     try:
-        if args.workload == "prefill":
+        if args.score_only:
+            line = run_score_only(args, world, rank, local)
+        elif args.workload == "prefill":
             line = run_prefill(args, world, rank, local)
         else:
             line = run_decode(args, world, rank, local)
         if rank == 0 and line is not None:
-            if world == 1 and not args.no_cpu_baseline and args.workload != "prefill":
+            if (world == 1 and not args.no_cpu_baseline and args.workload != "prefill"
+                    and not args.score_only):
                 line["cpu_baseline"] = cpu_baseline(synth.workload(args.workload),
                                                     torch.device("cuda", local))
             print(json.dumps(line))

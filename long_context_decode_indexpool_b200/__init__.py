@@ -130,12 +130,21 @@ def _host_f32(arr):
     return a
 
 
+def _event_handle(ev):
+    """cudaEvent_t of a torch.cuda.Event (torch creates it on first record)."""
+    if ev is None:
+        return None
+    if not ev.cuda_event:
+        ev.record()
+    return ev.cuda_event
+
+
 def _timing(events):
     if events is None:
         return None
     t = spx_timing()
-    t.score_begin = events[0].cuda_event if events[0] is not None else None
-    t.score_end = events[1].cuda_event if events[1] is not None else None
+    t.score_begin = _event_handle(events[0])
+    t.score_end = _event_handle(events[1])
     return ctypes.byref(t)
 
 
