@@ -190,6 +190,31 @@ SPX_API spx_status spx_topk_blocks(const spx_dims* d, int32_t rows,
                            spx_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * spx_topk_blocks_noalloc -- the same selection as spx_topk_blocks, for
+ * callers that cannot allocate or pass scratch memory (for example code that
+ * runs inside a framework whose allocator owns all device memory, or a
+ * serving path where cudaMalloc's device-wide synchronisation is not
+ * allowed).  The pages describe no such entry point; it is an addition of
+ * this library.
+ *
+ * The candidate lists live in one array built into the library, of
+ * SPX_TOPK_NOALLOC_SCRATCH_BYTES bytes, held on every GPU that loads the
+ * library until the process exits.  The call allocates nothing.  Calls whose
+ * scratch need (spx_topk_workspace_size) exceeds that size return
+ * SPX_ERR_WORKSPACE before launching anything.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress), so make that
+ * first call before any stream capture.  All calls share the array: calls
+ * whose kernels overlap on the GPU race and must be serialised by the caller.
+ * Arguments and results are those of spx_topk_blocks.
+ * ------------------------------------------------------------------------- */
+#define SPX_TOPK_NOALLOC_SCRATCH_BYTES (4u << 20)
+SPX_API spx_status spx_topk_blocks_noalloc(const spx_dims* d, int32_t rows,
+                                           const float* scores, int64_t score_stride,
+                                           const int64_t* n_vis, int64_t max_len,
+                                           int32_t* idx, int32_t* count,
+                                           spx_stream stream);
+
+/* ---------------------------------------------------------------------------
  * Step 4 -- sparse MLA attention over the selected latent rows.
  * [W3] "실제로 바꾸는 것": attention runs on the selected positions only;
  * absorbed MLA with NoPE ([W4] "위치 인코딩"): the latent row c_t is both key

@@ -68,6 +68,7 @@ _SIGS = {
     "spx_index_score": ([_DIMS, _I32, _P, _P, _P, _I64, _P, _I64, _P, _I64, _P], ctypes.c_int),
     "spx_topk_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_topk_blocks": ([_DIMS, _I32, _P, _I64, _P, _I64, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "spx_topk_blocks_noalloc": ([_DIMS, _I32, _P, _I64, _P, _I64, _P, _P, _P], ctypes.c_int),
     "spx_attn_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_sparse_mla_attn": ([_DIMS, _I32, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P],
                             ctypes.c_int),
@@ -189,6 +190,18 @@ def spx_topk_blocks(d, rows, scores, score_stride, n_vis, max_len, idx, count, w
     _check(_lib.spx_topk_blocks(ctypes.byref(d), rows, _ptr(scores), score_stride, _ptr(n_vis),
                                 max_len, _ptr(idx), _ptr(count), _ptr(ws), ws_bytes,
                                 _stream(stream)), "spx_topk_blocks")
+
+
+def spx_topk_blocks_noalloc(d, rows, scores, score_stride, n_vis, max_len, idx, count,
+                            stream=None):
+    """spx_topk_blocks without a caller workspace: the library's built-in
+    scratch array is used (see include/spx.h for its size and rules)."""
+    _check(_lib.spx_topk_blocks_noalloc(ctypes.byref(d), rows, _ptr(scores), score_stride,
+                                        _ptr(n_vis), max_len, _ptr(idx), _ptr(count),
+                                        _stream(stream)), "spx_topk_blocks_noalloc")
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 def spx_attn_workspace_size(d, rows, max_len) -> int:
