@@ -42,7 +42,9 @@ __global__ void __launch_bounds__(kPoolThreads)
                   float w2, float w3, __nv_bfloat16* __restrict__ tail,
                   __nv_bfloat16* __restrict__ pooled, int64_t cap_blk,
                   const int64_t* __restrict__ len_dev, int64_t len_host, int64_t max_len,
-                  int64_t* __restrict__ nvis_out) {
+                  int64_t* __restrict__ nvis_out, uint32_t* __restrict__ init_hist,
+                  int32_t* __restrict__ init_first, int32_t* __restrict__ init_last,
+                  int32_t* __restrict__ init_idx, int32_t* __restrict__ init_cnt) {
   const int b = blockIdx.y;
   int64_t len = len_dev ? len_dev[b] : len_host;
   // Clamp so that every access stays inside the caches whatever the device
@@ -50,7 +52,20 @@ __global__ void __launch_bounds__(kPoolThreads)
   if (len < 0) len = 0;
   if (len > max_len - n_new) len = max_len - n_new;
   const int64_t end = len + n_new;
-  if (nvis_out && blockIdx.x == 0 && threadIdx.x == 0) nvis_out[b] = end;
+  if (blockIdx.x == 0) {
+    if (nvis_out && threadIdx.x == 0) nvis_out[b] = end;
+    if (init_hist) {
+      for (int i = threadIdx.x; i < kSelHistBins; i += kPoolThreads)
+        init_hist[static_cast<int64_t>(b) * kSelHistBins + i] = 0u;
+      for (int i = threadIdx.x; i < kTopK; i += kPoolThreads)
+        init_idx[static_cast<int64_t>(b) * kTopK + i] = -1;
+      if (threadIdx.x == 0) {
+        init_first[b] = -1;
+        init_last[b] = -1;
+        init_cnt[b] = 0;
+      }
+    }
+  }
   if (n_new <= 0) return;
 
   const int64_t blk_lo = len / kPool;
@@ -105,7 +120,7 @@ __global__ void k_prefill_nvis(int64_t* __restrict__ n_vis, int T, int64_t pos0)
 }  // namespace
 
 cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream) {
-  if (a.n_new <= 0 && a.nvis_out == nullptr) return cudaSuccess;
+  if (a.n_new <= 0 && a.nvis_out == nullptr && a.init_hist == nullptr) return cudaSuccess;
   // Blocks an append can touch: at most ceil((n_new + 3) / 4) + 1.
   const int64_t blocks = (static_cast<int64_t>(a.n_new) + 2 * kPool) / kPool;
   dim3 grid(static_cast<unsigned>((blocks + kBlocksPerCta - 1) / kBlocksPerCta), a.B);
@@ -113,7 +128,8 @@ cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream) {
   k_pool_append<<<grid, kPoolThreads, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(a.raw_k), a.n_new, a.w[0], a.w[1], a.w[2], a.w[3],
       static_cast<__nv_bfloat16*>(a.tail), static_cast<__nv_bfloat16*>(a.pooled_k), a.cap_blk,
-      a.len_dev, a.len_host, a.max_len, a.nvis_out);
+      a.len_dev, a.len_host, a.max_len, a.nvis_out, a.init_hist, a.init_first, a.init_last,
+      a.init_idx, a.init_cnt);
   count_launches(1);
   return cudaGetLastError();
 }

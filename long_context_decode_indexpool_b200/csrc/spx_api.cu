@@ -135,6 +135,49 @@ FusedLayout fused_layout(int rows, int heads, int64_t max_len) {
   return L;
 }
 
+// Workspace of the fused decode call (selection fused into the scoring kernel):
+//   n_vis [B] | idx [B,512] | count [B] | hist [B,2048] | first, last [B]
+//   | total tiles | list keys, list ids [grid+B, 512] | list counts [grid+B]
+//   | attention scratch
+struct DecodeLayout {
+  size_t nvis, idx, count, hist, first, last, tiles, lkey, lidx, lcnt, attn, total;
+  int grid;
+  AttnPlan ap;
+};
+
+DecodeLayout decode_layout(int B, int heads, int64_t max_len) {
+  DecodeLayout L{};
+  const int sms = device_sm_count();
+  L.grid = score_grid(1, B, max_len, sms);
+  L.ap = plan_attn(B, heads, max_len, sms);
+  const size_t slots = static_cast<size_t>(L.grid) + B;
+  size_t o = 0;
+  L.nvis = o;
+  o += up(static_cast<size_t>(B) * 8);
+  L.idx = o;
+  o += up(static_cast<size_t>(B) * kTopK * 4);
+  L.count = o;
+  o += up(static_cast<size_t>(B) * 4);
+  L.hist = o;
+  o += up(static_cast<size_t>(B) * kSelHistBins * 4);
+  L.first = o;
+  o += up(static_cast<size_t>(B) * 4);
+  L.last = o;
+  o += up(static_cast<size_t>(B) * 4);
+  L.tiles = o;
+  o += up(8);
+  L.lkey = o;
+  o += up(slots * kTopK * 4);
+  L.lidx = o;
+  o += up(slots * kTopK * 4);
+  L.lcnt = o;
+  o += up(slots * 4);
+  L.attn = o;
+  o += up(L.ap.ws_bytes);
+  L.total = o;
+  return L;
+}
+
 spx_status check_pool_w(const float* w, float out[4]) {
   if (!w) return SPX_ERR_INVALID_ARG;
   double s = 0.0;
@@ -331,7 +374,7 @@ spx_status spx_decode_workspace_size(const spx_dims* d, int32_t B, int64_t max_l
   if (st != SPX_OK) return st;
   if (!bytes) return SPX_ERR_INVALID_ARG;
   if (B < 1 || B > 65535 || max_len < 0) return SPX_ERR_SHAPE;
-  *bytes = fused_layout(B, d->heads, max_len).total;
+  *bytes = decode_layout(B, d->heads, max_len).total;
   return SPX_OK;
 }
 
@@ -356,17 +399,20 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
       !al4(w_head) || !al4(len_dev) || (raw_k && (!al16(raw_k) || !al16(tail))) ||
       (lse && !al4(lse)) || (idx_out && !al4(idx_out)) || (count_out && !al4(count_out)))
     return SPX_ERR_INVALID_ARG;
-  const FusedLayout L = fused_layout(B, d->heads, max_len);
+  const DecodeLayout L = decode_layout(B, d->heads, max_len);
   if (!ws || ws_bytes < L.total || !al16(ws)) return SPX_ERR_WORKSPACE;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   int64_t* n_vis = reinterpret_cast<int64_t*>(base + L.nvis);
-  float* scores = reinterpret_cast<float*>(base + L.scores);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + L.idx);
   int32_t* count = count_out ? count_out : reinterpret_cast<int32_t*>(base + L.count);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.hist);
+  int32_t* row_first = reinterpret_cast<int32_t*>(base + L.first);
+  int32_t* row_last = reinterpret_cast<int32_t*>(base + L.last);
+  int64_t* tiles = reinterpret_cast<int64_t*>(base + L.tiles);
 
-  // 1. append (or just copy the lengths) -> n_vis
+  // 1. append (or just copy the lengths) -> n_vis; reset the selection state
   PoolAppendArgs pa{};
   pa.B = B;
   pa.raw_k = raw_k;
@@ -379,10 +425,15 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   pa.len_host = 0;
   pa.max_len = max_len;
   pa.nvis_out = n_vis;
+  pa.init_hist = hist;
+  pa.init_first = row_first;
+  pa.init_last = row_last;
+  pa.init_idx = idx;
+  pa.init_cnt = count;
   cudaError_t e = launch_pool_append(pa, s);
   if (e != cudaSuccess) return SPX_ERR_CUDA;
 
-  // 2. indexer scores
+  // 2+3. indexer scores with the top-k selection fused in
   if (timing && timing->score_begin &&
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_begin), s) != cudaSuccess)
     return SPX_ERR_CUDA;
@@ -396,18 +447,33 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   sa.cap_blk = cap_blk;
   sa.n_vis = n_vis;
   sa.max_len = max_len;
-  sa.scores = scores;
-  sa.score_stride = L.stride;
+  sa.scores = nullptr;
+  sa.score_stride = 0;
   sa.num_sms = device_sm_count();
+  sa.sel_ghist = hist;
+  sa.sel_list_key = reinterpret_cast<uint32_t*>(base + L.lkey);
+  sa.sel_list_idx = reinterpret_cast<int32_t*>(base + L.lidx);
+  sa.sel_list_cnt = reinterpret_cast<int32_t*>(base + L.lcnt);
+  sa.sel_row_first = row_first;
+  sa.sel_row_last = row_last;
+  sa.sel_total = tiles;
   if ((e = launch_index_score(sa, s)) != cudaSuccess) return SPX_ERR_CUDA;
   if (timing && timing->score_end &&
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
     return SPX_ERR_CUDA;
-
-  // 3. top-k
-  if ((e = launch_topk(L.tp, scores, L.stride, n_vis, max_len, idx, count, base + L.topk, s)) !=
-      cudaSuccess)
-    return SPX_ERR_CUDA;
+  SelectMergeArgs ma{};
+  ma.rows = B;
+  ma.grid = L.grid;
+  ma.ghist = hist;
+  ma.list_key = sa.sel_list_key;
+  ma.list_idx = sa.sel_list_idx;
+  ma.list_cnt = sa.sel_list_cnt;
+  ma.row_first = row_first;
+  ma.row_last = row_last;
+  ma.total = tiles;
+  ma.out_idx = idx;
+  ma.out_cnt = count;
+  if ((e = launch_select_merge(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
 
   // 4. attention
   AttnArgs aa{};

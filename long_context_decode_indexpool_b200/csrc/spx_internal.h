@@ -30,6 +30,13 @@ struct PoolAppendArgs {
   int64_t len_host;
   int64_t max_len;
   int64_t* nvis_out;  // optional: receives len + n_new per sequence
+  // optional per-sequence initialisation of the fused selection state:
+  // hist[b][..] = 0, first[b] = last[b] = -1, idx[b][0..512) = -1, cnt[b] = 0
+  uint32_t* init_hist;
+  int32_t* init_first;
+  int32_t* init_last;
+  int32_t* init_idx;
+  int32_t* init_cnt;
 };
 cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_nvis(int64_t* n_vis, int T, int64_t pos0, cudaStream_t stream);
@@ -46,11 +53,42 @@ struct ScoreArgs {
   int64_t cap_blk;
   const int64_t* n_vis;  // [rows]
   int64_t max_len;
-  float* scores;
+  float* scores;        // written unless the selection is fused
   int64_t score_stride;
   int num_sms;
+  // fused top-k, first stage (decode, nq == 1): set sel_ghist to enable;
+  // see index_score.cu.  ghist must be zero and row_first/row_last -1 on
+  // entry.  The second stage is launch_select_merge.
+  uint32_t* sel_ghist;     // [rows, kSelHistBins]
+  uint32_t* sel_list_key;  // [score_grid + rows, 512]
+  int32_t* sel_list_idx;   // [score_grid + rows, 512]
+  int32_t* sel_list_cnt;   // [score_grid + rows]
+  int32_t* sel_row_first;  // [rows]
+  int32_t* sel_row_last;   // [rows]
+  int64_t* sel_total;      // [1]
 };
+constexpr int kSelHistBins = 2048;
+// Grid size of the scoring kernel for the given call shape.
+int score_grid(int nq, int rows, int64_t max_len, int num_sms);
 cudaError_t launch_index_score(const ScoreArgs& a, cudaStream_t stream);
+
+// Second stage of the fused decode selection: per row, the complete
+// histogram gives an exact lower bound; the CTA lists are filtered and merged
+// into the row's 512 block ids (ascending, -1 padded) and count.
+struct SelectMergeArgs {
+  int rows;
+  int grid;  // grid of the scoring launch
+  const uint32_t* ghist;
+  const uint32_t* list_key;
+  const int32_t* list_idx;
+  const int32_t* list_cnt;
+  const int32_t* row_first;
+  const int32_t* row_last;
+  const int64_t* total;
+  int32_t* out_idx;
+  int32_t* out_cnt;
+};
+cudaError_t launch_select_merge(const SelectMergeArgs& a, cudaStream_t stream);
 
 // Top-k blocks.
 struct TopkPlan {

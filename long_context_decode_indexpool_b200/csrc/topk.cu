@@ -12,7 +12,7 @@
 //
 // Level 1: a CTA takes a contiguous chunk of one row's scores (8192 by
 // default), finds the K-th largest key by four 8-bit radix passes over
-// shared-memory histograms (warp-aggregated atomics), then keeps every key
+// shared-memory histograms, then keeps every key
 // above it and the lowest-index keys equal to it.  A block-wide exclusive
 // scan places the survivors in index order, so every list is ascending.
 // Level 2+: a CTA merges up to 32 lists of one row (concatenated in chunk
@@ -20,7 +20,7 @@
 // writes the row's block ids, ascending, padded with -1.
 // The K best of a union are among the K best of each part, under the same
 // strict order, so the result equals a full sort of the row.
-#include "spx_device.cuh"
+#include "select.cuh"
 #include "spx_internal.h"
 
 namespace spx {
@@ -29,112 +29,6 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kMergeFanIn = 32;  // lists merged per CTA
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if ((u & 0x7FFFFFFFu) == 0) u = 0;  // -0 == +0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-struct SelectSmem {
-  int hist[256];
-  int scan[33];
-  int digit;
-  int above;
-};
-
-// Selects the best min(K, n_valid) of the candidates held by the block:
-// thread i holds E candidates at positions i*E .. i*E+E-1 (valid if bit set).
-// Calls emit(slot, out_pos) for each survivor, in position order per thread
-// with out_pos increasing with position across the block.  Returns the
-// number of survivors (same in every thread).
-template <int E, typename Emit>
-__device__ __forceinline__ int block_select(const uint32_t (&key)[E], uint32_t valid, int K,
-                                            SelectSmem& sm, Emit emit) {
-  const int tid = threadIdx.x, lane = tid & 31;
-  int total;
-  {
-    int n_all;
-    int pos = block_excl_scan(__popc(valid), sm.scan, &n_all);
-    if (n_all <= K) {  // uniform: keep every candidate
-#pragma unroll
-      for (int i = 0; i < E; ++i)
-        if ((valid >> i) & 1u) emit(i, pos++);
-      return n_all;
-    }
-  }
-
-  uint32_t prefix = 0, pmask = 0;
-  int remaining = K;
-#pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = tid; b < 256; b += blockDim.x) sm.hist[b] = 0;
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-      const bool ok = ((valid >> i) & 1u) && ((key[i] & pmask) == prefix);
-      const uint32_t dig = ok ? ((key[i] >> shift) & 255u) : 256u;
-      const unsigned peers = __match_any_sync(0xffffffffu, dig);
-      if (ok && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[dig], __popc(peers));
-    }
-    __syncthreads();
-    if (tid < 32) {
-      // lane L owns bins 255-8L .. 248-8L (descending)
-      int local[8], lsum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        local[j] = sm.hist[255 - (lane * 8 + j)];
-        lsum += local[j];
-      }
-      int incl = lsum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-      }
-      int cum = incl - lsum;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (cum < remaining && remaining <= cum + local[j]) {
-          sm.digit = 255 - (lane * 8 + j);
-          sm.above = cum;
-        }
-        cum += local[j];
-      }
-    }
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(sm.digit) << shift;
-    pmask |= 255u << shift;
-    remaining -= sm.above;
-    __syncthreads();
-  }
-  // prefix is the K-th largest key; `remaining` ties at it are kept.
-  int ngt = 0, neq = 0;
-#pragma unroll
-  for (int i = 0; i < E; ++i) {
-    if ((valid >> i) & 1u) {
-      ngt += key[i] > prefix;
-      neq += key[i] == prefix;
-    }
-  }
-  int eq_tot;
-  const int eq_before = block_excl_scan(neq, sm.scan, &eq_tot);
-  int take = remaining - eq_before;
-  take = take < 0 ? 0 : (take > neq ? neq : take);
-  int pos = block_excl_scan(ngt + take, sm.scan, &total);
-#pragma unroll
-  for (int i = 0; i < E; ++i) {
-    if ((valid >> i) & 1u) {
-      if (key[i] > prefix) {
-        emit(i, pos++);
-      } else if (key[i] == prefix && take > 0) {
-        --take;
-        emit(i, pos++);
-      }
-    }
-  }
-  return total;
-}
 
 __device__ __forceinline__ int64_t clamp_blocks(const int64_t* n_vis, int r, int64_t max_len) {
   int64_t n = n_vis[r];
@@ -151,6 +45,7 @@ __global__ void __launch_bounds__(kThreads)
                  int32_t* __restrict__ out_cnt, int32_t* __restrict__ final_idx,
                  int32_t* __restrict__ final_cnt) {
   __shared__ SelectSmem sm;
+  uint32_t thr;
   const int r = blockIdx.y, c = blockIdx.x;
   const int64_t nblk = clamp_blocks(n_vis, r, max_len);
   const int64_t start = static_cast<int64_t>(c) * (kThreads * E);
@@ -170,7 +65,7 @@ __global__ void __launch_bounds__(kThreads)
   const int list = r * nchunks + c;
   if (final_idx) {
     int32_t* dst = final_idx + static_cast<int64_t>(r) * kTopK;
-    const int n = block_select<E>(key, valid, kTopK, sm, [&](int i, int pos) {
+    const int n = group_select<E, kThreads, 0>(key, valid, kTopK, threadIdx.x, sm, &thr, [&](int i, int pos) {
       dst[pos] = static_cast<int32_t>(my0 + i);
     });
     for (int j = n + threadIdx.x; j < kTopK; j += kThreads) dst[j] = -1;
@@ -178,7 +73,7 @@ __global__ void __launch_bounds__(kThreads)
   } else {
     uint32_t* kd = out_key + static_cast<int64_t>(list) * kTopK;
     int32_t* id = out_idx + static_cast<int64_t>(list) * kTopK;
-    const int n = block_select<E>(key, valid, kTopK, sm, [&](int i, int pos) {
+    const int n = group_select<E, kThreads, 0>(key, valid, kTopK, threadIdx.x, sm, &thr, [&](int i, int pos) {
       kd[pos] = key[i];
       id[pos] = static_cast<int32_t>(my0 + i);
     });
@@ -195,6 +90,7 @@ __global__ void __launch_bounds__(kThreads)
                  int32_t* __restrict__ out_cnt, int32_t* __restrict__ final_idx,
                  int32_t* __restrict__ final_cnt) {
   __shared__ SelectSmem sm;
+  uint32_t thr;
   const int r = blockIdx.y, c = blockIdx.x;
   const int first_list = c * kMergeFanIn;
   const int nl = min(kMergeFanIn, in_lists - first_list);
@@ -220,19 +116,177 @@ __global__ void __launch_bounds__(kThreads)
   }
   if (final_idx) {
     int32_t* dst = final_idx + static_cast<int64_t>(r) * kTopK;
-    const int n = block_select<E>(key, valid, kTopK, sm, [&](int i, int pos) { dst[pos] = idx[i]; });
+    const int n = group_select<E, kThreads, 0>(key, valid, kTopK, threadIdx.x, sm, &thr, [&](int i, int pos) { dst[pos] = idx[i]; });
     for (int j = n + threadIdx.x; j < kTopK; j += kThreads) dst[j] = -1;
     if (threadIdx.x == 0) final_cnt[r] = n;
   } else {
     const int64_t list = static_cast<int64_t>(r) * out_lists + c;
     uint32_t* kd = out_key + list * kTopK;
     int32_t* id = out_idx + list * kTopK;
-    const int n = block_select<E>(key, valid, kTopK, sm, [&](int i, int pos) {
+    const int n = group_select<E, kThreads, 0>(key, valid, kTopK, threadIdx.x, sm, &thr, [&](int i, int pos) {
       kd[pos] = key[i];
       id[pos] = idx[i];
     });
     if (threadIdx.x == 0) out_cnt[list] = n;
   }
+}
+
+// Second stage of the decode selection fused into the scoring kernel: one
+// CTA per row.  The row's histogram is complete here (the scoring launch has
+// finished), so the bin holding the 512th-largest key gives an exact lower
+// bound; only list entries at or above it are gathered (index order = CTA
+// order), then an exact top-512 picks the result.
+constexpr int kSelBins = kSelHistBins;
+constexpr int kSelShift = 32 - 11;
+constexpr int kMergeCap = kThreads * 16;  // buffered candidates (E = 16)
+constexpr int kMergePer = 4;              // list entries per thread per round
+
+__global__ void __launch_bounds__(kThreads)
+    k_select_merge(const uint32_t* __restrict__ ghist, const uint32_t* __restrict__ list_key,
+                   const int32_t* __restrict__ list_idx, const int32_t* __restrict__ list_cnt,
+                   const int32_t* __restrict__ row_first, const int32_t* __restrict__ row_last,
+                   const int64_t* __restrict__ total_p, int G, int32_t* __restrict__ out_idx,
+                   int32_t* __restrict__ out_cnt) {
+  extern __shared__ uint8_t dyn[];
+  uint32_t* buf_key = reinterpret_cast<uint32_t*>(dyn);
+  int32_t* buf_idx = reinterpret_cast<int32_t*>(buf_key + kMergeCap);
+  __shared__ SelectSmem sm;
+  __shared__ int seg_off[kThreads + 1];
+  __shared__ uint32_t s_theta;
+  const int r = blockIdx.x, tid = threadIdx.x;
+  const int c_first = row_first[r], c_last = row_last[r];
+  if (c_first < 0 || c_last < c_first) return;  // no tile: outputs stay as initialised
+  const int64_t total = *total_p;
+
+  // 1. exact lower bound: thread t owns bins kSelBins-1-4t .. kSelBins-4-4t
+  {
+    const uint32_t* h = ghist + static_cast<int64_t>(r) * kSelBins;
+    int c[4], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      c[j] = static_cast<int>(h[kSelBins - 1 - (tid * 4 + j)]);
+      sum += c[j];
+    }
+    if (tid == 0) s_theta = 0;
+    int tot;
+    int cum = group_excl_scan<kThreads, 0>(sum, tid, sm.scan, &tot);
+    if (tot >= kTopK) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (cum < kTopK && kTopK <= cum + c[j])
+          s_theta = static_cast<uint32_t>(kSelBins - 1 - (tid * 4 + j)) << kSelShift;
+        cum += c[j];
+      }
+    }
+    __syncthreads();
+  }
+  uint32_t theta = s_theta, tkeep = s_theta;
+
+  // 2. list offsets of the row's CTAs, in CTA order
+  const int nseg = c_last - c_first + 1;
+  int nbuf = 0;
+  for (int sb = 0; sb < nseg; sb += kThreads) {
+    const int c = c_first + sb + tid;
+    int m = 0;
+    if (sb + tid < nseg && (total * (c + 1) / G) > (total * c / G))
+      m = list_cnt[static_cast<int64_t>(c) + r];
+    int mtot;
+    const int moff = group_excl_scan<kThreads, 0>(m, tid, sm.scan, &mtot);
+    seg_off[tid] = moff;
+    __syncthreads();
+    const int nsg = min(kThreads, nseg - sb);
+    // 3. gather in rounds; thread t takes entries base + 4t .. base + 4t + 3
+    for (int base = 0; base < mtot; base += kThreads * kMergePer) {
+      uint32_t k[kMergePer];
+      int32_t ix[kMergePer];
+      int npass = 0;
+      uint32_t pass = 0;
+#pragma unroll
+      for (int u = 0; u < kMergePer; ++u) {
+        const int f = base + tid * kMergePer + u;
+        k[u] = 0;
+        ix[u] = 0;
+        if (f < mtot) {
+          int lo_s = 0, hi_s = nsg - 1;  // last segment with seg_off <= f
+          while (lo_s < hi_s) {
+            const int mid = (lo_s + hi_s + 1) >> 1;
+            if (seg_off[mid] <= f) lo_s = mid; else hi_s = mid - 1;
+          }
+          const int64_t sl = static_cast<int64_t>(c_first + sb + lo_s) + r;
+          const int j = f - seg_off[lo_s];
+          k[u] = list_key[sl * kTopK + j];
+          ix[u] = list_idx[sl * kTopK + j];
+          if (k[u] >= theta) {
+            pass |= 1u << u;
+            ++npass;
+          }
+        }
+      }
+      int ptot;
+      int pos = nbuf + group_excl_scan<kThreads, 0>(npass, tid, sm.scan, &ptot);
+#pragma unroll
+      for (int u = 0; u < kMergePer; ++u) {
+        if ((pass >> u) & 1u) {
+          buf_key[pos] = k[u];
+          buf_idx[pos] = ix[u];
+          ++pos;
+        }
+      }
+      nbuf += ptot;
+      if (nbuf > kMergeCap - kThreads * kMergePer) {  // compact in place
+        __syncthreads();
+        uint32_t kk[16];
+        int32_t ii[16];
+        uint32_t valid = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int q = tid * 16 + i;
+          kk[i] = 0;
+          ii[i] = 0;
+          if (q < nbuf) {
+            kk[i] = buf_key[q];
+            ii[i] = buf_idx[q];
+            if (kk[i] >= tkeep) valid |= 1u << i;
+          }
+        }
+        __syncthreads();
+        uint32_t thr;
+        nbuf = group_select<16, kThreads, 0>(kk, valid, kTopK, tid, sm, &thr, [&](int i, int p) {
+          buf_key[p] = kk[i];
+          buf_idx[p] = ii[i];
+        });
+        if (thr != 0) {
+          const uint32_t t1 = thr == 0xFFFFFFFFu ? thr : thr + 1;
+          theta = t1 > theta ? t1 : theta;
+          tkeep = thr > tkeep ? thr : tkeep;
+        }
+      }
+      __syncthreads();
+    }
+    __syncthreads();
+  }
+
+  // 4. the row's result
+  uint32_t kk[16];
+  int32_t ii[16];
+  uint32_t valid = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int q = tid * 16 + i;
+    kk[i] = 0;
+    ii[i] = 0;
+    if (q < nbuf) {
+      kk[i] = buf_key[q];
+      ii[i] = buf_idx[q];
+      if (kk[i] >= tkeep) valid |= 1u << i;
+    }
+  }
+  uint32_t thr;
+  int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
+  const int n = group_select<16, kThreads, 0>(kk, valid, kTopK, tid, sm, &thr,
+                                               [&](int i, int p) { dst[p] = ii[i]; });
+  for (int j = n + tid; j < kTopK; j += kThreads) dst[j] = -1;
+  if (tid == 0) out_cnt[r] = n;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -247,6 +301,25 @@ cudaError_t launch_merge_e(dim3 grid, cudaStream_t s, const uint32_t* ik, const 
 }
 
 }  // namespace
+
+cudaError_t launch_select_merge(const SelectMergeArgs& a, cudaStream_t stream) {
+  if (a.rows == 0) return cudaSuccess;
+  constexpr int kSmem = kMergeCap * 8;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k_select_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  k_select_merge<<<a.rows, kThreads, kSmem, stream>>>(a.ghist, a.list_key, a.list_idx, a.list_cnt,
+                                                      a.row_first, a.row_last, a.total, a.grid,
+                                                      a.out_idx, a.out_cnt);
+  count_launches(1);
+  return cudaGetLastError();
+}
 
 TopkPlan plan_topk(int rows, int64_t max_len) {
   TopkPlan p{};

@@ -123,6 +123,44 @@ def test_fused_equals_composed_and_no_append_path():
     assert torch.equal(out.view(torch.int16), out_f.view(torch.int16))
 
 
+@pytest.mark.parametrize("levels", [4, 256])
+def test_fused_selection_heavy_ties(levels):
+    """Rows whose scores take few distinct values: the 512th score is shared by
+    thousands of blocks spread over every CTA of the row, so the fused
+    selection must resolve ties at the cut inside CTAs and in the merge."""
+    spx = need_gpu()
+    rng = np.random.default_rng(levels)
+    B, nblk = 3, 100003
+    L = 4 * nblk + 1  # one tail token
+    # pooled key b = c_b * e_0; query heads all e_0 with weight 1: s_b = 32 c_b
+    c = rng.integers(0, levels, (B, nblk)).astype(np.float32)
+    c[1, :] = 7.0  # a row of equal scores
+    keys = np.zeros((B, nblk + 1, 128), np.float32)  # capacity for the tail token's block
+    keys[:, :nblk, 0] = c
+    pooled = torch.from_numpy(keys).to(torch.bfloat16).cuda()
+    q_idx = torch.zeros(B, 32, 128, dtype=torch.bfloat16, device="cuda")
+    q_idx[:, :, 0] = 1.0
+    w_head = torch.ones(B, 32, device="cuda")
+    d = spx.dims(16, 1.0)
+    latent = torch.zeros(B, L, 512, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(B, 16, 512, dtype=torch.bfloat16, device="cuda")
+    len_dev = torch.full((B,), L, dtype=torch.int64, device="cuda")
+    out = torch.empty(B, 16, 512, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(B, 512, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(B, dtype=torch.int32, device="cuda")
+    ws = spx.workspace(spx.spx_decode_workspace_size(d, B, L), "cuda")
+    spx.spx_decode_fused(d, B, None, None, None, pooled, nblk + 1, len_dev, q_idx, w_head, q,
+                         latent, L, L, out, None, idx, cnt, ws)
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    idx = idx.cpu().numpy()
+    cnt = cnt.cpu().numpy()
+    for r in range(B):
+        ref = oracle.topk(32.0 * c[r].astype(np.float64), 512)
+        assert cnt[r] == 512 and np.array_equal(idx[r], ref), f"row {r}"
+    assert idx[1].tolist() == list(range(512))
+
+
 # ----------------------------------------------------------------------------
 # Chunked prefill
 # ----------------------------------------------------------------------------
