@@ -70,7 +70,7 @@ constexpr int kEpi = 128;                    // epilogue threads
 constexpr int kHistBins = 2048;              // top 11 key bits
 constexpr int kHistShift = 21;
 constexpr int kBufCap = 2048;                // candidate buffer entries
-constexpr int kFirstFlush = 4;               // tiles before the first histogram flush
+constexpr int kEarlyFlush = 4;               // tiles between the first two flushes
 constexpr int kFlushTiles = 16;              // tiles between later flushes
 constexpr int kMergeUnroll = 4;              // list entries in flight per thread
 
@@ -179,7 +179,7 @@ struct SelState {
   int par;
   int since_flush;
   bool snap_pending;   // a snapshot copy is in flight (cp.async group)
-  bool first_flush_done;
+  int flushes;         // flushes done in the current row
   uint32_t theta;      // admission bound for new (higher-index) candidates
   uint32_t tkeep;      // bound for candidates already in the buffer (<= theta)
 };
@@ -553,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       S.par = 0;
       S.since_flush = 0;
       S.snap_pending = false;
-      S.first_flush_done = false;
+      S.flushes = 0;
       S.theta = 0;
       S.tkeep = 0;
       for (int b = et; b < kHistBins; b += kEpi) S.lhist[b] = 0;
@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       S.theta = 0;
       S.tkeep = 0;
       S.since_flush = 0;
-      S.first_flush_done = false;
+      S.flushes = 0;
     };
 
     for (int i = 0; i < n_items; ++i) {
@@ -643,9 +643,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t key = order_key(sc[0]);
         if (valid) atomicAdd(&S.lhist[key >> kHistShift], 1u);
         sel_append(S, valid && key >= S.theta, key, static_cast<int32_t>(blk), quarter, lane);
-        if (++S.since_flush >= (S.first_flush_done ? kFlushTiles : kFirstFlush)) {
+        if (++S.since_flush >= (S.flushes >= 2 ? kFlushTiles : kEarlyFlush)) {
           sel_flush(S, p.ghist + static_cast<int64_t>(w.g) * kHistBins, et, S.snap_pending);
-          S.first_flush_done = true;
+          ++S.flushes;
         }
         if (S.nbuf > kBufCap - kEpi) sel_compact(S, et);
       } else {

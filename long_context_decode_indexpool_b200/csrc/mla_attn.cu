@@ -1,4 +1,5 @@
-// Sparse MLA attention over the gathered latent rows of the selected tokens.
+// Sparse MLA attention over the gathered latent rows of the selected tokens,
+// on the 5th-generation tensor cores.
 //
 // [W3] "GLM-5.3 Sparse Attention은 연산량을 줄이지만 HBM 수요는 지속된다", section
 // "GLM-5.3 Sparse Attention이 실제로 바꾸는 것": the core multi-head latent
@@ -11,14 +12,25 @@
 //   out[h] = sum_t softmax_t(sm_scale * q_h . c_t) c_t   over the token set S
 //   S = tokens of the selected blocks  U  the query's partial tail block.
 //
-// Kernel (one CTA = one query row, 16 heads, one split of the token list):
-// 64-token sub-tiles of latent rows are gathered with 16-byte cp.async into
-// a double-buffered, XOR-swizzled shared-memory tile (each selected block is
-// 4 KiB contiguous in HBM).  QK^T and PV run on bf16 tensor-core MMAs with
-// fp32 accumulation; the softmax is online in base 2 (exp2 of
-// sm_scale*log2(e)-scaled logits).  Splits of one (row, head group) write
-// unnormalised partial outputs with their running max and sum; a merge
-// kernel combines them with the log-sum-exp rule.
+// One CTA = one query row, 64 heads, one split of the row's token list.
+// The list is walked in tiles of 64 tokens:
+//   * gather: 128 threads copy the tile's latent rows (each selected block is
+//     4 KiB contiguous in HBM) with 16-byte cp.async into shared memory in the
+//     128-byte-swizzle K-major layout (8 regions of 64 dims), double-buffered;
+//   * S = Q C^T: 32 tcgen05.mma (M = 64 heads, N = 64 tokens, K = 16) into
+//     TMEM lanes 16-31 of each 32-lane quarter (an M = 64 accumulator uses
+//     lanes 0-15 of each quarter, so the other half is free);
+//   * softmax: the thread that owns TMEM lane 16+i of warp w holds the logits
+//     of head 16w+i for the tile, masks skipped/absent tokens, keeps the
+//     running max m (base 2) and sum l, writes P (bf16) to shared memory.  The
+//     running max is raised lazily: only when a tile's max exceeds it by more
+//     than 8 (so p <= 2^8) is O rescaled, by the partner thread that owns
+//     lane i (the O row of the same head);
+//   * O += P C: 8 tcgen05.mma (M = 64, N = 256, K = 16; C is read in its
+//     MN-major form from the same shared-memory tile) into TMEM lanes 0-15,
+//     columns 0-511.
+// A split writes out/lse directly (one split) or an unnormalised partial with
+// its (m, l) for the merge kernel (log-sum-exp rule).
 #include "spx_device.cuh"
 #include "spx_internal.h"
 
@@ -26,16 +38,19 @@ namespace spx {
 
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kSub = 64;                       // tokens per sub-tile
-constexpr int kRowBytes = kLatent * 2;         // 1024
-constexpr int kQSmem = kHeadGroup * kRowBytes; // 16 KiB
-constexpr int kKVSmem = kSub * kRowBytes;      // 64 KiB
-constexpr int kPSmem = kHeadGroup * kSub * 2;  // 2 KiB
-constexpr int kSmemBytes = 128 + kQSmem + 2 * kKVSmem + kPSmem + 2 * kSub * 8 +
-                           2 * kWarps * kHeadGroup * 4;
+constexpr int kThreads = 128;
+constexpr int kTT = 64;                         // tokens per tile
+constexpr int kHG = 64;                         // heads per CTA (MMA M)
+constexpr int kRegion = 64 * 128;               // [64 rows x 128 B] = 8 KiB
+constexpr int kQBytes = 8 * kRegion;            // 64 KiB
+constexpr int kKVBytes = 8 * kRegion;           // 64 KiB per tile
+constexpr int kPBytes = kRegion;                // [64 heads x 64 tokens] bf16
+constexpr int kSmemBytes = 1024 + kQBytes + 2 * kKVBytes + kPBytes + 2 * kTT * 8 + 64;
 constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLazy = 8.f;                    // rescale threshold (log2 units)
+constexpr uint32_t kIdescQK = idesc_bf16_f32(64, kTT);
+// PV: B (the latent tile) is MN-major: set the "transpose B" bit.
+constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256) | (1u << 16);
 
 struct KParams {
   const __nv_bfloat16* q;
@@ -46,14 +61,13 @@ struct KParams {
   const int32_t* count;
   const int64_t* n_vis;
   int heads;
-  int groups;
   int nsplit;
   int split_tokens;
   float scale_log2;
   __nv_bfloat16* out;
   float* lse;
-  float* part_o;   // [rows, groups, nsplit, 16, 512]
-  float* part_ml;  // [rows, groups, nsplit, 16, 2]
+  float* part_o;   // [rows, nsplit, heads, 512]
+  float* part_ml;  // [rows, nsplit, heads, 2]
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -68,33 +82,47 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void mma_bf16(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+// Byte offset of 16-byte piece `c` (0..63) of row `r` in a tile stored as 8
+// regions of [64 rows x 128 B] with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+  return static_cast<uint32_t>((c >> 3) * kRegion + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Shared-memory descriptor of an MN-major operand in the 128-byte-swizzle
+// layout: 64-element groups along MN `lbo` bytes apart, 8-row groups along K
+// `sbo` bytes apart.
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const float* v) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// byte offset of 16-byte chunk `c` of row `r` in a swizzled tile with
-// `row_bytes` per row (chunk index XOR row mod 8)
-__device__ __forceinline__ uint32_t swz(int r, int c, int row_bytes) {
-  return static_cast<uint32_t>(r * row_bytes + ((c ^ (r & 7)) << 4));
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 struct RowInfo {
@@ -128,291 +156,328 @@ __device__ __forceinline__ int64_t token_pos(const KParams& p, int r, const RowI
 
 __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   extern __shared__ uint8_t dyn[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 127) &
-                                           ~static_cast<uintptr_t>(127));
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
   uint8_t* q_s = sm;
-  uint8_t* kv_s = q_s + kQSmem;
-  uint8_t* p_s = kv_s + 2 * kKVSmem;
-  int64_t* pos_s = reinterpret_cast<int64_t*>(p_s + kPSmem);  // [2][64]
-  float* red_max = reinterpret_cast<float*>(pos_s + 2 * kSub);  // [8][16]
-  float* red_sum = red_max + kWarps * kHeadGroup;             // [8][16]
+  uint8_t* kv_s = q_s + kQBytes;
+  uint8_t* p_s = kv_s + 2 * kKVBytes;
+  int64_t* pos_s = reinterpret_cast<int64_t*>(p_s + kPBytes);  // [2][64]
+  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(pos_s + 2 * kTT);
+  uint64_t* bar_pv = bar_qk + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_pv + 1);
 
-  const int split = blockIdx.x, r = blockIdx.y, g = blockIdx.z;
+  const int split = blockIdx.x, r = blockIdx.y, hg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h0 = hg * kHG;
   const RowInfo ri = row_info(p, r);
   const int j_begin = split * p.split_tokens;
   const int j_end = min(ri.S, j_begin + p.split_tokens);
-  const int nsub = j_end > j_begin ? (j_end - j_begin + kSub - 1) / kSub : 0;
-  const int h0 = lane >> 2;  // rows h0 and h0 + 8 of the accumulator fragments
-  const int64_t unit = (static_cast<int64_t>(r) * p.groups + g);
+  const int ntiles = j_end > j_begin ? (j_end - j_begin + kTT - 1) / kTT : 0;
+  // head owned by this thread: lanes 0-15 hold O rows, lanes 16-31 S rows
+  const int hloc = warp * 16 + (lane & 15);
+  const int head = h0 + hloc;
+  const bool head_ok = head < p.heads;
 
-  if (nsub == 0) {
-    if (p.nsplit == 1) {
-      for (int i = tid; i < kHeadGroup * kLatent; i += kThreads)
-        p.out[(static_cast<int64_t>(r) * p.heads + g * kHeadGroup) * kLatent + i] =
+  if (ntiles == 0) {
+    for (int i = tid; i < kHG * kLatent; i += kThreads) {
+      const int hh = h0 + i / kLatent;
+      if (hh >= p.heads) continue;
+      if (p.nsplit == 1)
+        p.out[(static_cast<int64_t>(r) * p.heads + hh) * kLatent + i % kLatent] =
             __float2bfloat16_rn(0.f);
-      if (p.lse && tid < kHeadGroup)
-        p.lse[static_cast<int64_t>(r) * p.heads + g * kHeadGroup + tid] = -INFINITY;
-    } else {
-      const int64_t base = (unit * p.nsplit + split) * kHeadGroup;
-      for (int i = tid; i < kHeadGroup * kLatent; i += kThreads) p.part_o[base * kLatent + i] = 0.f;
-      if (tid < kHeadGroup) {
-        p.part_ml[(base + tid) * 2] = -INFINITY;
-        p.part_ml[(base + tid) * 2 + 1] = 0.f;
+      else
+        p.part_o[((static_cast<int64_t>(r) * p.nsplit + split) * p.heads + hh) * kLatent +
+                 i % kLatent] = 0.f;
+    }
+    if (tid < kHG && h0 + tid < p.heads) {
+      const int hh = h0 + tid;
+      if (p.nsplit == 1) {
+        if (p.lse) p.lse[static_cast<int64_t>(r) * p.heads + hh] = -INFINITY;
+      } else {
+        const int64_t b = (static_cast<int64_t>(r) * p.nsplit + split) * p.heads + hh;
+        p.part_ml[b * 2] = -INFINITY;
+        p.part_ml[b * 2 + 1] = 0.f;
       }
     }
     return;
   }
 
+  if (tid == 0) {
+    mbar_init(bar_qk, 1);
+    mbar_init(bar_pv, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+
   const __nv_bfloat16* lat = p.latent + static_cast<int64_t>(r) * p.seq_stride;
   const uint32_t q_u = smem_u32(q_s), kv_u = smem_u32(kv_s), p_u = smem_u32(p_s);
 
-  // Q tile [16 heads x 512] -> shared (part of the first cp.async group)
+  // Q [64 heads x 512] (heads beyond H zero-filled): part of the first group
   {
-    const __nv_bfloat16* qg =
-        p.q + (static_cast<int64_t>(r) * p.heads + g * kHeadGroup) * kLatent;
-    for (int c = tid; c < kHeadGroup * (kLatent / 8); c += kThreads) {
-      const int h = c >> 6, ch = c & 63;
-      cp_async16(q_u + swz(h, ch, kRowBytes), qg + h * kLatent + ch * 8, true);
+    const __nv_bfloat16* qr = p.q + (static_cast<int64_t>(r) * p.heads) * kLatent;
+    for (int c = tid; c < kHG * 64; c += kThreads) {
+      const int h = c >> 6, piece = c & 63;
+      const bool ok = h0 + h < p.heads;
+      cp_async16(q_u + sw_off(h, piece),
+                 qr + static_cast<int64_t>(ok ? h0 + h : 0) * kLatent + piece * 8, ok);
     }
   }
-
-  auto fill_pos = [&](int sub, int buf) {
-    if (tid < kSub) {
-      const int j = j_begin + sub * kSub + tid;
-      pos_s[buf * kSub + tid] = j < j_end ? token_pos(p, r, ri, j) : -1;
+  auto fill_pos = [&](int tile, int buf) {
+    if (tid < kTT) {
+      const int j = j_begin + tile * kTT + tid;
+      pos_s[buf * kTT + tid] = j < j_end ? token_pos(p, r, ri, j) : -1;
     }
   };
-  auto issue_kv = [&](int buf) {
-    const uint32_t dst = kv_u + buf * kKVSmem;
-    const int64_t* ps = pos_s + buf * kSub;
+  auto gather = [&](int buf) {
+    const uint32_t dst = kv_u + buf * kKVBytes;
+    const int64_t* ps = pos_s + buf * kTT;
 #pragma unroll 4
-    for (int i = 0; i < (kSub * (kLatent / 8)) / kThreads; ++i) {
+    for (int i = 0; i < (kTT * 64) / kThreads; ++i) {
       const int c = i * kThreads + tid;
-      const int t = c >> 6, ch = c & 63;
+      const int t = c >> 6, piece = c & 63;
       const int64_t pos = ps[t];
-      const __nv_bfloat16* src = lat + (pos >= 0 ? pos : 0) * kLatent + ch * 8;
-      cp_async16(dst + swz(t, ch, kRowBytes), src, pos >= 0);
+      cp_async16(dst + sw_off(t, piece), lat + (pos >= 0 ? pos : 0) * kLatent + piece * 8,
+                 pos >= 0);
     }
+    cp_async_commit();
   };
 
   fill_pos(0, 0);
   __syncthreads();
-  issue_kv(0);
-  cp_async_commit();
-
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_run[2] = {0.f, 0.f};
-  float o[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-
-  for (int sub = 0; sub < nsub; ++sub) {
-    const int buf = sub & 1;
-    if (sub + 1 < nsub) {
-      fill_pos(sub + 1, buf ^ 1);
-      __syncthreads();
-      issue_kv(buf ^ 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-
-    const uint32_t kvb = kv_u + buf * kKVSmem;
-    const int64_t* ps = pos_s + buf * kSub;
-
-    // ---- S = Q K^T for this warp's 8 tokens ------------------------------
-    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int kk = 0; kk < kLatent / 16; kk += 2) {
-      uint32_t b0, b1, b2, b3;
-      {
-        const int t = warp * 8 + (lane & 7);
-        const int ch = kk * 2 + (lane >> 3);
-        ldsm_x4(kvb + swz(t, ch, kRowBytes), b0, b1, b2, b3);
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        uint32_t a0, a1, a2, a3;
-        const int row = lane & 15;
-        const int ch = (kk + u) * 2 + (lane >> 4);
-        ldsm_x4(q_u + swz(row, ch, kRowBytes), a0, a1, a2, a3);
-        if (u == 0)
-          mma_bf16(sacc, a0, a1, a2, a3, b0, b1);
-        else
-          mma_bf16(sacc, a0, a1, a2, a3, b2, b3);
-      }
-    }
-
-    // ---- online softmax ---------------------------------------------------
-    const int tcol = warp * 8 + 2 * (lane & 3);
-    const bool v0 = ps[tcol] >= 0, v1 = ps[tcol + 1] >= 0;
-    float x[4];
-    x[0] = v0 ? sacc[0] * p.scale_log2 : -INFINITY;
-    x[1] = v1 ? sacc[1] * p.scale_log2 : -INFINITY;
-    x[2] = v0 ? sacc[2] * p.scale_log2 : -INFINITY;
-    x[3] = v1 ? sacc[3] * p.scale_log2 : -INFINITY;
-    float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]);
-#pragma unroll
-    for (int o2 = 1; o2 < 4; o2 <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
-    }
-    if ((lane & 3) == 0) {
-      red_max[warp * kHeadGroup + h0] = mx0;
-      red_max[warp * kHeadGroup + h0 + 8] = mx1;
-    }
-    __syncthreads();
-    float tm0 = -INFINITY, tm1 = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      tm0 = fmaxf(tm0, red_max[w * kHeadGroup + h0]);
-      tm1 = fmaxf(tm1, red_max[w * kHeadGroup + h0 + 8]);
-    }
-    const float mn0 = fmaxf(m_run[0], tm0), mn1 = fmaxf(m_run[1], tm1);
-    const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m_run[0] - mn0);
-    const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m_run[1] - mn1);
-    float pv[4];
-    pv[0] = x[0] == -INFINITY ? 0.f : exp2f(x[0] - mn0);
-    pv[1] = x[1] == -INFINITY ? 0.f : exp2f(x[1] - mn0);
-    pv[2] = x[2] == -INFINITY ? 0.f : exp2f(x[2] - mn1);
-    pv[3] = x[3] == -INFINITY ? 0.f : exp2f(x[3] - mn1);
-    l_run[0] = l_run[0] * al0 + pv[0] + pv[1];
-    l_run[1] = l_run[1] * al1 + pv[2] + pv[3];
-    m_run[0] = mn0;
-    m_run[1] = mn1;
-    {
-      const uint32_t off = static_cast<uint32_t>((lane & 3) * 4);
-      __nv_bfloat162 w0 = __floats2bfloat162_rn(pv[0], pv[1]);
-      __nv_bfloat162 w1 = __floats2bfloat162_rn(pv[2], pv[3]);
-      *reinterpret_cast<__nv_bfloat162*>(p_s + swz(h0, warp, kSub * 2) + off) = w0;
-      *reinterpret_cast<__nv_bfloat162*>(p_s + swz(h0 + 8, warp, kSub * 2) + off) = w1;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      o[i][0] *= al0;
-      o[i][1] *= al0;
-      o[i][2] *= al1;
-      o[i][3] *= al1;
-    }
-    __syncthreads();
-
-    // ---- O += P V for this warp's 64 dims -------------------------------------
-#pragma unroll
-    for (int kk = 0; kk < kSub / 16; ++kk) {
-      uint32_t a0, a1, a2, a3;
-      {
-        const int row = lane & 15;
-        const int ch = kk * 2 + (lane >> 4);
-        ldsm_x4(p_u + swz(row, ch, kSub * 2), a0, a1, a2, a3);
-      }
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t b0, b1, b2, b3;
-        const int t = kk * 16 + (lane & 15);
-        const int ch = warp * 8 + np * 2 + (lane >> 4);
-        ldsm_x4_t(kvb + swz(t, ch, kRowBytes), b0, b1, b2, b3);
-        mma_bf16(o[2 * np], a0, a1, a2, a3, b0, b1);
-        mma_bf16(o[2 * np + 1], a0, a1, a2, a3, b2, b3);
-      }
-    }
-    __syncthreads();
-  }
-
-  // ---- row sums over the quad and the warps ----------------------------------
-  float l0 = l_run[0], l1 = l_run[1];
-#pragma unroll
-  for (int o2 = 1; o2 < 4; o2 <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, o2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
-  }
-  if ((lane & 3) == 0) {
-    red_sum[warp * kHeadGroup + h0] = l0;
-    red_sum[warp * kHeadGroup + h0 + 8] = l1;
-  }
+  gather(0);  // group: Q + tile 0
+  tc_fence_before();
   __syncthreads();
-  float L0 = 0.f, L1 = 0.f;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    L0 += red_sum[w * kHeadGroup + h0];
-    L1 += red_sum[w * kHeadGroup + h0 + 8];
-  }
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  // MMA destinations: O in the lower half of each 32-lane quarter (lanes
+  // 0-15, columns 0-511), S in the upper half (lanes 16-31, columns 0-63).
+  const uint32_t t_o = tmem;
+  const uint32_t t_s = tmem + (16u << 16);
+  const uint32_t my_lane_base = static_cast<uint32_t>(warp * 32) << 16;
 
-  const int dcol = warp * 64 + 2 * (lane & 3);
-  if (p.nsplit == 1) {
-    const float inv0 = L0 > 0.f ? 1.f / L0 : 0.f, inv1 = L1 > 0.f ? 1.f / L1 : 0.f;
-    __nv_bfloat16* o0 = p.out + (static_cast<int64_t>(r) * p.heads + g * kHeadGroup + h0) * kLatent;
-    __nv_bfloat16* o1 = o0 + 8 * kLatent;
+  float m_run = -INFINITY, l_run = 0.f;  // meaningful in the S-lane threads
+  bool ok_all = true;
+
+  for (int j = 0; j < ntiles; ++j) {
+    const int buf = j & 1;
+    cp_async_wait<0>();
+    fence_proxy_async();
+    __syncthreads();
+
+    // ---- S = Q C^T --------------------------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t kvb = kv_u + buf * kKVBytes;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      *reinterpret_cast<__nv_bfloat162*>(o0 + dcol + 8 * i) =
-          __floats2bfloat162_rn(o[i][0] * inv0, o[i][1] * inv0);
-      *reinterpret_cast<__nv_bfloat162*>(o1 + dcol + 8 * i) =
-          __floats2bfloat162_rn(o[i][2] * inv1, o[i][3] * inv1);
+      for (int k = 0; k < kLatent / 16; ++k) {
+        const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
+        umma_bf16(t_s, sdesc_kmajor_sw128(q_u + off), sdesc_kmajor_sw128(kvb + off), kIdescQK,
+                  k > 0 ? 1u : 0u);
+      }
+      umma_commit(bar_qk);
     }
-    if (p.lse && warp == 0 && (lane & 3) == 0) {
-      float* ls = p.lse + static_cast<int64_t>(r) * p.heads + g * kHeadGroup;
-      ls[h0] = L0 > 0.f ? (m_run[0] + __log2f(L0)) * kLn2 : -INFINITY;
-      ls[h0 + 8] = L1 > 0.f ? (m_run[1] + __log2f(L1)) * kLn2 : -INFINITY;
+    // the previous PV must be done before its buffer is refilled and before
+    // P or O are touched again
+    if (j > 0) {
+      volatile int no_abort = 0;
+      ok_all &= mbar_wait(bar_pv, (j - 1) & 1, &no_abort);
     }
-  } else {
-    const int64_t base = (unit * p.nsplit + split) * kHeadGroup;
-    float* po0 = p.part_o + (base + h0) * kLatent;
-    float* po1 = po0 + 8 * kLatent;
+    if (j + 1 < ntiles) {
+      fill_pos(j + 1, buf ^ 1);
+      __syncthreads();
+      gather(buf ^ 1);
+    }
+    {
+      volatile int no_abort = 0;
+      ok_all &= mbar_wait(bar_qk, j & 1, &no_abort);
+    }
+    tc_fence_after();
+
+    // ---- softmax -----------------------------------------------------------
+    // A warp reads its own 32-lane quarter: lanes 16-31 receive the S rows
+    // (lanes 0-15 receive O columns 0-63, unused here).
+    float s[kTT];
+    tmem_ld_32x32b_x32(tmem + my_lane_base, s);
+    tmem_ld_32x32b_x32(tmem + my_lane_base + 32, s + 32);
+    const int64_t* ps = pos_s + buf * kTT;
+    float mt = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      *reinterpret_cast<float2*>(po0 + dcol + 8 * i) = make_float2(o[i][0], o[i][1]);
-      *reinterpret_cast<float2*>(po1 + dcol + 8 * i) = make_float2(o[i][2], o[i][3]);
+    for (int t = 0; t < kTT; ++t) {
+      s[t] = ps[t] >= 0 ? s[t] * p.scale_log2 : -INFINITY;
+      mt = fmaxf(mt, s[t]);
     }
-    if (warp == 0 && (lane & 3) == 0) {
-      p.part_ml[(base + h0) * 2] = m_run[0];
-      p.part_ml[(base + h0) * 2 + 1] = L0;
-      p.part_ml[(base + h0 + 8) * 2] = m_run[1];
-      p.part_ml[(base + h0 + 8) * 2 + 1] = L1;
+    float alpha = 1.f;
+    if (lane >= 16) {
+      if (m_run == -INFINITY) {
+        m_run = mt;
+      } else if (mt > m_run + kLazy) {
+        alpha = exp2f(m_run - mt);
+        m_run = mt;
+      }
+    }
+    // O rows live in the partner lane (lane - 16): rescale there if needed
+    const float alpha_o = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
+    if (__any_sync(0xffffffffu, alpha_o != 1.f) && j > 0) {
+      // whole warp: lanes 0-15 scale their O rows, lanes 16-31 rewrite what they read
+      const float f = lane < 16 ? alpha_o : 1.f;
+#pragma unroll 1
+      for (int c = 0; c < kLatent; c += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(t_o + my_lane_base + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= f;
+        tmem_st_32x32b_x32(t_o + my_lane_base + c, v);
+      }
+    }
+    if (lane >= 16) {
+      float lsum = 0.f;
+      uint32_t packed[kTT / 2];
+#pragma unroll
+      for (int t = 0; t < kTT; t += 2) {
+        const float a = s[t] == -INFINITY ? 0.f : exp2f(s[t] - m_run);
+        const float b = s[t + 1] == -INFINITY ? 0.f : exp2f(s[t + 1] - m_run);
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
+        lsum += __low2float(h2) + __high2float(h2);
+        packed[t / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      l_run = l_run * alpha + lsum;
+      // row hloc of P: 8 pieces of 16 B
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t a = p_u + hloc * 128 + ((c ^ (hloc & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(packed[4 * c]),
+                     "r"(packed[4 * c + 1]), "r"(packed[4 * c + 2]), "r"(packed[4 * c + 3])
+                     : "memory");
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- O += P C ----------------------------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t kvb = kv_u + buf * kKVBytes;
+#pragma unroll
+      for (int k = 0; k < kTT / 16; ++k) {
+        const uint64_t ad = sdesc_kmajor_sw128(p_u + k * 32);
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+          const uint64_t bd =
+              sdesc_mn_sw128(kvb + nh * 4 * kRegion + k * 16 * 128, kRegion, 1024);
+          umma_bf16(t_o + nh * 256, ad, bd, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+        }
+      }
+      umma_commit(bar_pv);
     }
   }
+  {
+    volatile int no_abort = 0;
+    ok_all &= mbar_wait(bar_pv, (ntiles - 1) & 1, &no_abort);
+  }
+  tc_fence_after();
+
+  // ---- epilogue: lanes 0-15 own the O rows -----------------------------------
+  const float m_h = __shfl_sync(0xffffffffu, m_run, (lane & 15) + 16);
+  const float l_h = __shfl_sync(0xffffffffu, l_run, (lane & 15) + 16);
+  const bool writer = lane < 16 && head_ok && ok_all;
+#pragma unroll 1
+  for (int c = 0; c < kLatent; c += 32) {
+    float v[32];
+    tmem_ld_32x32b_x32(t_o + my_lane_base + c, v);
+    if (writer) {
+      if (p.nsplit == 1) {
+        const float inv = l_h > 0.f ? 1.f / l_h : 0.f;
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * i] * inv, v[2 * i + 1] * inv);
+          w[i] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(
+            p.out + (static_cast<int64_t>(r) * p.heads + head) * kLatent + c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      } else {
+        float4* dst = reinterpret_cast<float4*>(
+            p.part_o + ((static_cast<int64_t>(r) * p.nsplit + split) * p.heads + head) * kLatent +
+            c);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+    }
+  }
+  if (writer) {
+    if (p.nsplit == 1) {
+      if (p.lse)
+        p.lse[static_cast<int64_t>(r) * p.heads + head] =
+            l_h > 0.f ? (m_h + __log2f(l_h)) * kLn2 : -INFINITY;
+    } else {
+      const int64_t b = (static_cast<int64_t>(r) * p.nsplit + split) * p.heads + head;
+      p.part_ml[b * 2] = l_h > 0.f ? m_h : -INFINITY;
+      p.part_ml[b * 2 + 1] = l_h;
+    }
+  }
+  if (!ok_all && tid == 0) atomicExch(&g_device_error, kErrWaitTimeout);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// Combines the split partials of one (row, head group):
+// Combines the split partials of one (row, head):
 //   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  out = sum_s O_s 2^(m_s - M) / L.
-__global__ void __launch_bounds__(256) k_attn_merge(const float* __restrict__ part_o,
+__global__ void __launch_bounds__(128) k_attn_merge(const float* __restrict__ part_o,
                                                     const float* __restrict__ part_ml,
-                                                    int nsplit, int heads, int groups,
+                                                    int nsplit, int heads,
                                                     __nv_bfloat16* __restrict__ out,
                                                     float* __restrict__ lse) {
-  const int r = blockIdx.x, g = blockIdx.y;
-  const int64_t unit = static_cast<int64_t>(r) * groups + g;
-  for (int e = threadIdx.x; e < kHeadGroup * (kLatent / 4); e += blockDim.x) {
-    const int h = e / (kLatent / 4), d4 = e % (kLatent / 4);
+  __shared__ float s_w[64];
+  __shared__ float s_inv, s_lse;
+  const int r = blockIdx.x, hh = blockIdx.y;
+  auto base_of = [&](int s) { return (static_cast<int64_t>(r) * nsplit + s) * heads + hh; };
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s)
-      M = fmaxf(M, part_ml[((unit * nsplit + s) * kHeadGroup + h) * 2]);
+    for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, part_ml[base_of(s) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-      for (int s = 0; s < nsplit; ++s) {
-        const int64_t base = (unit * nsplit + s) * kHeadGroup + h;
-        const float m = part_ml[base * 2];
-        if (m == -INFINITY) continue;
-        const float wgt = exp2f(m - M);
-        L += part_ml[base * 2 + 1] * wgt;
-        const float4 v = *reinterpret_cast<const float4*>(part_o + base * kLatent + d4 * 4);
-        acc.x += v.x * wgt;
-        acc.y += v.y * wgt;
-        acc.z += v.z * wgt;
-        acc.w += v.w * wgt;
-      }
+    for (int s = lane; s < nsplit; s += 32) {
+      const float m = part_ml[base_of(s) * 2];
+      const float wgt = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
+      s_w[s] = wgt;
+      L += part_ml[base_of(s) * 2 + 1] * wgt;
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    __nv_bfloat16* o = out + (static_cast<int64_t>(r) * heads + g * kHeadGroup + h) * kLatent + d4 * 4;
-    reinterpret_cast<__nv_bfloat162*>(o)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    reinterpret_cast<__nv_bfloat162*>(o)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    if (lse && d4 == 0)
-      lse[static_cast<int64_t>(r) * heads + g * kHeadGroup + h] =
-          L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) {
+      s_inv = L > 0.f ? 1.f / L : 0.f;
+      s_lse = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+    }
   }
+  __syncthreads();
+  const int d4 = threadIdx.x;  // 128 threads x 4 dims
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < nsplit; ++s) {
+    const float wgt = s_w[s];
+    if (wgt == 0.f) continue;
+    const float4 v = *reinterpret_cast<const float4*>(part_o + base_of(s) * kLatent + d4 * 4);
+    acc.x += v.x * wgt;
+    acc.y += v.y * wgt;
+    acc.z += v.z * wgt;
+    acc.w += v.w * wgt;
+  }
+  const float inv = s_inv;
+  __nv_bfloat16* o = out + (static_cast<int64_t>(r) * heads + hh) * kLatent + d4 * 4;
+  reinterpret_cast<__nv_bfloat162*>(o)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  reinterpret_cast<__nv_bfloat162*>(o)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  if (lse && threadIdx.x == 0) lse[static_cast<int64_t>(r) * heads + hh] = s_lse;
 }
 
 }  // namespace
@@ -421,7 +486,7 @@ AttnPlan plan_attn(int rows, int heads, int64_t max_len, int num_sms) {
   AttnPlan p{};
   p.rows = rows;
   p.heads = heads;
-  p.groups = heads / kHeadGroup;
+  p.groups = (heads + kHG - 1) / kHG;
   const int64_t max_blk = max_len / kPool;
   int64_t s_max = (max_blk > kTopK ? kTopK : max_blk) * kPool + kPool - 1;
   if (s_max > max_len) s_max = max_len;
@@ -430,12 +495,18 @@ AttnPlan plan_attn(int rows, int heads, int64_t max_len, int num_sms) {
   int nsplit = 1;
   if (units < num_sms) nsplit = static_cast<int>((num_sms + units - 1) / units);
   int64_t ts = (s_max + nsplit - 1) / nsplit;
-  ts = (ts + kSub - 1) / kSub * kSub;
+  ts = (ts + kTT - 1) / kTT * kTT;
+  if (ts < 2 * kTT) ts = 2 * kTT;  // at least two tiles per split: fewer partials
   p.split_tokens = static_cast<int>(ts);
   p.nsplit = static_cast<int>((s_max + ts - 1) / ts);
+  if (p.nsplit > 64) {  // the merge keeps at most 64 split weights
+    ts = ((s_max + 63) / 64 + kTT - 1) / kTT * kTT;
+    p.split_tokens = static_cast<int>(ts);
+    p.nsplit = static_cast<int>((s_max + ts - 1) / ts);
+  }
   p.ws_bytes = 0;
   if (p.nsplit > 1) {
-    const size_t n = static_cast<size_t>(units) * p.nsplit * kHeadGroup;
+    const size_t n = static_cast<size_t>(rows) * p.nsplit * heads;
     p.ws_bytes = ((n * kLatent * 4 + 255) & ~static_cast<size_t>(255)) + n * 2 * 4;
   }
   return p;
@@ -461,13 +532,12 @@ cudaError_t launch_attn(const AttnPlan& pl, const AttnArgs& a, cudaStream_t stre
   p.count = a.count;
   p.n_vis = a.n_vis;
   p.heads = pl.heads;
-  p.groups = pl.groups;
   p.nsplit = pl.nsplit;
   p.split_tokens = pl.split_tokens;
   p.scale_log2 = a.sm_scale * 1.44269504088896340736f;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
-  const size_t n = static_cast<size_t>(pl.rows) * pl.groups * pl.nsplit * kHeadGroup;
+  const size_t n = static_cast<size_t>(pl.rows) * pl.nsplit * pl.heads;
   p.part_o = static_cast<float*>(a.ws);
   p.part_ml = pl.nsplit > 1
                   ? reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
@@ -478,8 +548,8 @@ cudaError_t launch_attn(const AttnPlan& pl, const AttnArgs& a, cudaStream_t stre
   count_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || pl.nsplit == 1) return e;
-  k_attn_merge<<<dim3(pl.rows, pl.groups), 256, 0, stream>>>(p.part_o, p.part_ml, pl.nsplit,
-                                                             pl.heads, pl.groups, p.out, p.lse);
+  k_attn_merge<<<dim3(pl.rows, pl.heads), 128, 0, stream>>>(p.part_o, p.part_ml, pl.nsplit,
+                                                            pl.heads, p.out, p.lse);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -78,10 +78,51 @@ __device__ __forceinline__ int group_select(const uint32_t (&key)[E], uint32_t v
       return n_all;
     }
   }
+  // Bits shared by every valid key need no histogram: find them from the
+  // group-wide min and max first (this also avoids the worst same-address
+  // atomic contention, on the leading digits).
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0;
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    if ((valid >> i) & 1u) {
+      kmin = key[i] < kmin ? key[i] : kmin;
+      kmax = key[i] > kmax ? key[i] : kmax;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint32_t a = __shfl_xor_sync(0xffffffffu, kmin, o);
+    const uint32_t b = __shfl_xor_sync(0xffffffffu, kmax, o);
+    kmin = a < kmin ? a : kmin;
+    kmax = b > kmax ? b : kmax;
+  }
+  if (lane == 0) {
+    sm.hist[(gtid >> 5) * 2] = static_cast<int>(kmin);
+    sm.hist[(gtid >> 5) * 2 + 1] = static_cast<int>(kmax);
+  }
+  group_sync<NT, BAR>();
+  kmin = 0xFFFFFFFFu;
+  kmax = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const uint32_t a = static_cast<uint32_t>(sm.hist[2 * w]);
+    const uint32_t b = static_cast<uint32_t>(sm.hist[2 * w + 1]);
+    kmin = a < kmin ? a : kmin;
+    kmax = b > kmax ? b : kmax;
+  }
+  group_sync<NT, BAR>();
+  // All valid keys lie in [kmin, kmax], so they share every bit above the
+  // highest bit where kmin and kmax differ.
+  const uint32_t diff = kmin ^ kmax;
   uint32_t prefix = 0, pmask = 0;
   int remaining = K;
 #pragma unroll 1
   for (int shift = 24; shift >= 0; shift -= 8) {
+    if ((diff >> shift) == 0) {  // uniform: this digit is common to all keys
+      prefix |= kmin & (255u << shift);
+      pmask |= 255u << shift;
+      continue;
+    }
     for (int b = gtid; b < 256; b += NT) sm.hist[b] = 0;
     group_sync<NT, BAR>();
 #pragma unroll
