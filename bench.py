@@ -317,8 +317,11 @@ def dist_setup():
 
 
 def max_over_ranks(value: float, world: int, device) -> float:
+    """Max of a per-rank value (the slowest rank's time) over the process group."""
     if world == 1:
         return value
+    if torch.distributed.get_backend() == "gloo":
+        device = torch.device("cpu")
     t = torch.tensor([value], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())

@@ -87,7 +87,7 @@ struct Cfg {
   static constexpr int kNbOff = kWOff + kN * 4;
   static constexpr int kSelOff = (kNbOff + NQ * 8 + 15) & ~15;
   static constexpr int kSelBytes =
-      SELECT ? (2 * kHistBins * 4 + kBufCap * 8 + static_cast<int>(sizeof(SelectSmem)) + 64 +
+      SELECT ? (2 * kHistBins * 4 + pad32(kBufCap) * 8 + static_cast<int>(sizeof(SelectSmem)) + 64 +
                 (kEpi + 1) * 4)
              : 0;
   static constexpr int kBarOff = (kSelOff + kSelBytes + 7) & ~7;
@@ -200,8 +200,8 @@ __device__ __forceinline__ void sel_append(SelState& S, bool pass, uint32_t key,
   }
   if (pass) {
     const int pos = S.nbuf + off + __popc(bal & ((1u << lane) - 1u));
-    S.buf_key[pos] = key;
-    S.buf_idx[pos] = idx;
+    S.buf_key[pad32(pos)] = key;
+    S.buf_idx[pad32(pos)] = idx;
   }
   S.nbuf += tot;
   S.par ^= 1;
@@ -219,16 +219,16 @@ __device__ __forceinline__ void sel_compact(SelState& S, int et) {
     key[i] = 0;
     idx[i] = 0;
     if (j < S.nbuf) {
-      key[i] = S.buf_key[j];
-      idx[i] = S.buf_idx[j];
+      key[i] = S.buf_key[pad32(j)];
+      idx[i] = S.buf_idx[pad32(j)];
       if (key[i] >= S.tkeep) valid |= 1u << i;
     }
   }
   epi_sync();
   uint32_t thr;
   const int n = group_select<16, kEpi, 1>(key, valid, kTopK, et, *S.ss, &thr, [&](int i, int pos) {
-    S.buf_key[pos] = key[i];
-    S.buf_idx[pos] = idx[i];
+    S.buf_key[pad32(pos)] = key[i];
+    S.buf_idx[pad32(pos)] = idx[i];
   });
   if (thr != 0) {
     // Later arrivals have higher block ids, so one equal to thr loses to the
@@ -544,8 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       S.lhist = reinterpret_cast<uint32_t*>(sel);
       S.snap = S.lhist + kHistBins;
       S.buf_key = S.snap + kHistBins;
-      S.buf_idx = reinterpret_cast<int32_t*>(S.buf_key + kBufCap);
-      S.ss = reinterpret_cast<SelectSmem*>(S.buf_idx + kBufCap);
+      S.buf_idx = reinterpret_cast<int32_t*>(S.buf_key + pad32(kBufCap));
+      S.ss = reinterpret_cast<SelectSmem*>(S.buf_idx + pad32(kBufCap));
       S.wcnt = reinterpret_cast<int*>(S.ss + 1);
       S.misc = S.wcnt + 8;
       S.seg_off = S.misc + 8;
@@ -575,8 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       sel_compact(S, et);
       const int64_t slot = static_cast<int64_t>(blockIdx.x) + r;
       for (int i = et; i < S.nbuf; i += kEpi) {
-        p.list_key[slot * kTopK + i] = S.buf_key[i];
-        p.list_idx[slot * kTopK + i] = S.buf_idx[i];
+        p.list_key[slot * kTopK + i] = S.buf_key[pad32(i)];
+        p.list_idx[slot * kTopK + i] = S.buf_idx[pad32(i)];
       }
       if (et == 0) {
         p.list_cnt[slot] = S.nbuf;

@@ -380,40 +380,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   }
   tc_fence_after();
 
-  // ---- epilogue: lanes 0-15 own the O rows -----------------------------------
+  // ---- epilogue: lanes 0-15 own the O rows ----------------------------------
+  // The rows go through shared memory (the latent tiles are free now) so that
+  // all 128 threads store them to global memory in coalesced 16-byte pieces.
   const float m_h = __shfl_sync(0xffffffffu, m_run, (lane & 15) + 16);
   const float l_h = __shfl_sync(0xffffffffu, l_run, (lane & 15) + 16);
-  const bool writer = lane < 16 && head_ok && ok_all;
+  const bool single = p.nsplit == 1;
+  const float scale_o = single ? (l_h > 0.f ? 1.f / l_h : 0.f) : 1.f;
+  // staging: single split -> bf16 rows of 1 KiB; partial -> fp32 rows of 2 KiB
+  // (64 rows x 2 KiB = 128 KiB = both latent buffers).  16-byte pieces are
+  // rotated by the row index to spread the banks.
+  uint8_t* stage = kv_s;
+  const int row_bytes = single ? kLatent * 2 : kLatent * 4;
+  const int pieces = row_bytes / 16;
 #pragma unroll 1
   for (int c = 0; c < kLatent; c += 32) {
     float v[32];
     tmem_ld_32x32b_x32(t_o + my_lane_base + c, v);
-    if (writer) {
-      if (p.nsplit == 1) {
-        const float inv = l_h > 0.f ? 1.f / l_h : 0.f;
+    if (lane < 16) {
+      if (single) {
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * i] * inv, v[2 * i + 1] * inv);
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * i] * scale_o, v[2 * i + 1] * scale_o);
           w[i] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        uint4* dst = reinterpret_cast<uint4*>(
-            p.out + (static_cast<int64_t>(r) * p.heads + head) * kLatent + c);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int i = 0; i < 4; ++i) {
+          const int piece = (c * 2 / 16 + i + hloc) % pieces;
+          *reinterpret_cast<uint4*>(stage + hloc * row_bytes + piece * 16) =
+              make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
       } else {
-        float4* dst = reinterpret_cast<float4*>(
-            p.part_o + ((static_cast<int64_t>(r) * p.nsplit + split) * p.heads + head) * kLatent +
-            c);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        for (int i = 0; i < 8; ++i) {
+          const int piece = (c * 4 / 16 + i + hloc) % pieces;
+          *reinterpret_cast<float4*>(stage + hloc * row_bytes + piece * 16) =
+              make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
       }
     }
   }
-  if (writer) {
-    if (p.nsplit == 1) {
+  if (lane < 16 && head_ok && ok_all) {
+    if (single) {
       if (p.lse)
         p.lse[static_cast<int64_t>(r) * p.heads + head] =
             l_h > 0.f ? (m_h + __log2f(l_h)) * kLn2 : -INFINITY;
@@ -421,6 +430,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       const int64_t b = (static_cast<int64_t>(r) * p.nsplit + split) * p.heads + head;
       p.part_ml[b * 2] = l_h > 0.f ? m_h : -INFINITY;
       p.part_ml[b * 2 + 1] = l_h;
+    }
+  }
+  __syncthreads();
+  if (ok_all) {
+    const int nrows = min(kHG, p.heads - h0);
+    uint8_t* gbase = single ? reinterpret_cast<uint8_t*>(p.out + (static_cast<int64_t>(r) * p.heads + h0) * kLatent)
+                            : reinterpret_cast<uint8_t*>(p.part_o + ((static_cast<int64_t>(r) * p.nsplit + split) * p.heads + h0) * kLatent);
+    for (int e = tid; e < nrows * pieces; e += kThreads) {
+      const int row = e / pieces, piece = e % pieces;
+      const int sp = (piece + row) % pieces;
+      *reinterpret_cast<uint4*>(gbase + static_cast<int64_t>(row) * row_bytes + piece * 16) =
+          *reinterpret_cast<const uint4*>(stage + row * row_bytes + sp * 16);
     }
   }
   if (!ok_all && tid == 0) atomicExch(&g_device_error, kErrWaitTimeout);
@@ -464,14 +485,23 @@ __global__ void __launch_bounds__(128) k_attn_merge(const float* __restrict__ pa
   __syncthreads();
   const int d4 = threadIdx.x;  // 128 threads x 4 dims
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < nsplit; ++s) {
-    const float wgt = s_w[s];
-    if (wgt == 0.f) continue;
-    const float4 v = *reinterpret_cast<const float4*>(part_o + base_of(s) * kLatent + d4 * 4);
-    acc.x += v.x * wgt;
-    acc.y += v.y * wgt;
-    acc.z += v.z * wgt;
-    acc.w += v.w * wgt;
+  for (int s0 = 0; s0 < nsplit; s0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {  // independent loads in flight
+      const int s = s0 + u;
+      v[u] = s < nsplit && s_w[s] != 0.f
+                 ? *reinterpret_cast<const float4*>(part_o + base_of(s) * kLatent + d4 * 4)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float wgt = s0 + u < nsplit ? s_w[s0 + u] : 0.f;
+      acc.x += v[u].x * wgt;
+      acc.y += v[u].y * wgt;
+      acc.z += v[u].z * wgt;
+      acc.w += v[u].w * wgt;
+    }
   }
   const float inv = s_inv;
   __nv_bfloat16* o = out + (static_cast<int64_t>(r) * heads + hh) * kLatent + d4 * 4;

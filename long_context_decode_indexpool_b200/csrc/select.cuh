@@ -20,6 +20,11 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Shared-memory candidate buffers are padded by one word per 32 entries: a
+// thread that owns 16 consecutive entries then reads them without bank
+// conflicts (entry p lives at word p + p/32).
+__host__ __device__ constexpr int pad32(int p) { return p + (p >> 5); }
+
 template <int NT, int BAR>
 __device__ __forceinline__ void group_sync() {
   if constexpr (BAR == 0) {

@@ -149,10 +149,11 @@ __global__ void __launch_bounds__(kThreads)
                    int32_t* __restrict__ out_cnt) {
   extern __shared__ uint8_t dyn[];
   uint32_t* buf_key = reinterpret_cast<uint32_t*>(dyn);
-  int32_t* buf_idx = reinterpret_cast<int32_t*>(buf_key + kMergeCap);
+  int32_t* buf_idx = reinterpret_cast<int32_t*>(buf_key + pad32(kMergeCap));
   __shared__ SelectSmem sm;
   __shared__ int seg_off[kThreads + 1];
   __shared__ uint32_t s_theta;
+  __shared__ int s_bin, s_above;
   const int r = blockIdx.x, tid = threadIdx.x;
   const int c_first = row_first[r], c_last = row_last[r];
   if (c_first < 0 || c_last < c_first) return;  // no tile: outputs stay as initialised
@@ -167,20 +168,29 @@ __global__ void __launch_bounds__(kThreads)
       c[j] = static_cast<int>(h[kSelBins - 1 - (tid * 4 + j)]);
       sum += c[j];
     }
-    if (tid == 0) s_theta = 0;
+    if (tid == 0) {
+      s_theta = 0;
+      s_bin = -1;
+      s_above = 0;
+    }
     int tot;
     int cum = group_excl_scan<kThreads, 0>(sum, tid, sm.scan, &tot);
-    if (tot >= kTopK) {
+    if (tot > kTopK) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (cum < kTopK && kTopK <= cum + c[j])
-          s_theta = static_cast<uint32_t>(kSelBins - 1 - (tid * 4 + j)) << kSelShift;
+        if (cum < kTopK && kTopK <= cum + c[j]) {
+          const int bin = kSelBins - 1 - (tid * 4 + j);
+          s_theta = static_cast<uint32_t>(bin) << kSelShift;
+          s_bin = bin;
+          s_above = cum;  // keys in higher bins: all of them are selected
+        }
         cum += c[j];
       }
     }
     __syncthreads();
   }
   uint32_t theta = s_theta, tkeep = s_theta;
+  const int cut_bin = s_bin, above = s_above;
 
   // 2. list offsets of the row's CTAs, in CTA order
   const int nseg = c_last - c_first + 1;
@@ -227,8 +237,8 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
       for (int u = 0; u < kMergePer; ++u) {
         if ((pass >> u) & 1u) {
-          buf_key[pos] = k[u];
-          buf_idx[pos] = ix[u];
+          buf_key[pad32(pos)] = k[u];
+          buf_idx[pad32(pos)] = ix[u];
           ++pos;
         }
       }
@@ -244,16 +254,16 @@ __global__ void __launch_bounds__(kThreads)
           kk[i] = 0;
           ii[i] = 0;
           if (q < nbuf) {
-            kk[i] = buf_key[q];
-            ii[i] = buf_idx[q];
+            kk[i] = buf_key[pad32(q)];
+            ii[i] = buf_idx[pad32(q)];
             if (kk[i] >= tkeep) valid |= 1u << i;
           }
         }
         __syncthreads();
         uint32_t thr;
         nbuf = group_select<16, kThreads, 0>(kk, valid, kTopK, tid, sm, &thr, [&](int i, int p) {
-          buf_key[p] = kk[i];
-          buf_idx[p] = ii[i];
+          buf_key[pad32(p)] = kk[i];
+          buf_idx[pad32(p)] = ii[i];
         });
         if (thr != 0) {
           const uint32_t t1 = thr == 0xFFFFFFFFu ? thr : thr + 1;
@@ -266,25 +276,42 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
   }
 
-  // 4. the row's result
+  // 4. the row's result.  Every candidate in a bin above the cut bin is
+  // selected (there are `above` of them, all present); the K - above best of
+  // the cut bin (ties: lower block) complete the set.  Those share their top
+  // 11 key bits, so the radix passes over them skip the leading digits.
   uint32_t kk[16];
   int32_t ii[16];
-  uint32_t valid = 0;
+  uint32_t in_cut = 0, sure = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int q = tid * 16 + i;
     kk[i] = 0;
     ii[i] = 0;
     if (q < nbuf) {
-      kk[i] = buf_key[q];
-      ii[i] = buf_idx[q];
-      if (kk[i] >= tkeep) valid |= 1u << i;
+      kk[i] = buf_key[pad32(q)];
+      ii[i] = buf_idx[pad32(q)];
+      if (kk[i] >= tkeep) {
+        const int bin = static_cast<int>(kk[i] >> kSelShift);
+        if (cut_bin < 0 || bin > cut_bin) sure |= 1u << i;
+        else if (bin == cut_bin) in_cut |= 1u << i;
+      }
     }
   }
-  uint32_t thr;
+  uint32_t chosen = 0;
+  if (cut_bin >= 0) {  // uniform
+    uint32_t thr;
+    group_select<16, kThreads, 0>(kk, in_cut, kTopK - above, tid, sm, &thr,
+                                  [&](int i, int) { chosen |= 1u << i; });
+  }
+  const uint32_t take = sure | chosen;
+  int n;
+  int pos = group_excl_scan<kThreads, 0>(__popc(take), tid, sm.scan, &n);
   int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
-  const int n = group_select<16, kThreads, 0>(kk, valid, kTopK, tid, sm, &thr,
-                                               [&](int i, int p) { dst[p] = ii[i]; });
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (((take >> i) & 1u) && pos < kTopK) dst[pos++] = ii[i];
+  if (n > kTopK) n = kTopK;  // cannot happen for consistent inputs
   for (int j = n + tid; j < kTopK; j += kThreads) dst[j] = -1;
   if (tid == 0) out_cnt[r] = n;
 }
@@ -304,7 +331,7 @@ cudaError_t launch_merge_e(dim3 grid, cudaStream_t s, const uint32_t* ik, const 
 
 cudaError_t launch_select_merge(const SelectMergeArgs& a, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
-  constexpr int kSmem = kMergeCap * 8;
+  constexpr int kSmem = pad32(kMergeCap) * 8;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
