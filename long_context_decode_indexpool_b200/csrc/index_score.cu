@@ -72,7 +72,6 @@ constexpr int kHistShift = 21;
 constexpr int kBufCap = 2048;                // candidate buffer entries
 constexpr int kEarlyFlush = 4;               // tiles between the first two flushes
 constexpr int kFlushTiles = 16;              // tiles between later flushes
-constexpr int kMergeUnroll = 4;              // list entries in flight per thread
 
 template <int NQ, bool SELECT>
 struct Cfg {
@@ -436,6 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tensormap(&map_k);
       prefetch_tensormap(&map_q);
+      // per-row keys are read once (decode); keys shared by every query
+      // group (prefill) are re-read from L2
+      const uint64_t stream_pol = p.shared_keys ? l2_evict_normal_policy() : l2_evict_first_policy();
       Walker<NQ> w;
       w.init(p, s_g0, s_t0, lo);
       int stage = 0, cur_g = -1, qs = C::kQSlots - 1;
@@ -459,8 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* dst = a_smem + stage * kTileBytes;
         const int kb = p.shared_keys ? 0 : w.g;
         mbar_arrive_expect_tx(&full[stage], kTileBytes);
-        tma_load_3d(dst, &map_k, &full[stage], 0, w.t * kTileM, kb);
-        tma_load_3d(dst + kHalfBytes, &map_k, &full[stage], 64, w.t * kTileM, kb);
+        tma_load_3d_hint(dst, &map_k, &full[stage], 0, w.t * kTileM, kb, stream_pol);
+        tma_load_3d_hint(dst + kHalfBytes, &map_k, &full[stage], 64, w.t * kTileM, kb, stream_pol);
         ++issued;
         if (++stage == C::kStages) {
           stage = 0;

@@ -300,8 +300,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     // A warp reads its own 32-lane quarter: lanes 16-31 receive the S rows
     // (lanes 0-15 receive O columns 0-63, unused here).
     float s[kTT];
-    tmem_ld_32x32b_x32(tmem + my_lane_base, s);
-    tmem_ld_32x32b_x32(tmem + my_lane_base + 32, s + 32);
+    {
+      uint32_t* sr = reinterpret_cast<uint32_t*>(s);
+      tmem_ld_x32_async(tmem + my_lane_base, sr);
+      tmem_ld_x32_async(tmem + my_lane_base + 32, sr + 32);
+      tmem_ld_wait_regs<kTT>(sr);
+    }
     const int64_t* ps = pos_s + buf * kTT;
     float mt = -INFINITY;
 #pragma unroll
@@ -394,9 +398,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   const int row_bytes = single ? kLatent * 2 : kLatent * 4;
   const int pieces = row_bytes / 16;
 #pragma unroll 1
-  for (int c = 0; c < kLatent; c += 32) {
-    float v[32];
-    tmem_ld_32x32b_x32(t_o + my_lane_base + c, v);
+  for (int c0 = 0; c0 < kLatent; c0 += 128) {
+    float vv[128];
+    uint32_t* vr = reinterpret_cast<uint32_t*>(vv);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tmem_ld_x32_async(t_o + my_lane_base + c0 + 32 * q, vr + 32 * q);
+    tmem_ld_wait_regs<128>(vr);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = c0 + 32 * q;
+    const float* v = vv + 32 * q;
     if (lane < 16) {
       if (single) {
         uint32_t w[16];
@@ -420,6 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         }
       }
     }
+  }
   }
   if (lane < 16 && head_ok && ok_all) {
     if (single) {

@@ -134,12 +134,146 @@ __global__ void __launch_bounds__(kThreads)
 // Second stage of the decode selection fused into the scoring kernel: one
 // CTA per row.  The row's histogram is complete here (the scoring launch has
 // finished), so the bin holding the 512th-largest key gives an exact lower
-// bound; only list entries at or above it are gathered (index order = CTA
-// order), then an exact top-512 picks the result.
+// bound; only list entries at or above it take part (index order = CTA
+// order).  Every entry in a bin above the cut bin is selected; the best of
+// the cut bin (ties: lower block) complete the 512.
 constexpr int kSelBins = kSelHistBins;
 constexpr int kSelShift = 32 - 11;
-constexpr int kMergeCap = kThreads * 16;  // buffered candidates (E = 16)
-constexpr int kMergePer = 4;              // list entries per thread per round
+constexpr int kMergeCap = kThreads * 16;  // candidates held at once (16 per thread)
+constexpr int kMergePer = 4;              // list entries per thread per round (long rows)
+
+// Shared state of the final choice.
+struct MergeSmem {
+  int rh[3][128];  // radix histograms of the three 7-bit digits below the cut bin
+  int dig[3], abv[3];
+  uint32_t kmin, kmax;
+};
+
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// The row's result from the n buffered (key, block) pairs, in block order;
+// entries below lo_key are not candidates.  Every candidate above the cut
+// bin is selected; the (K - above) best of the cut bin (ties: lower block)
+// complete the set.  Writes the ascending block ids, -1 padded, and the
+// count.  This code runs once per row: its loops stay rolled, so that it is
+// short (instruction fetch, not arithmetic, bounds a one-pass kernel).
+__device__ __noinline__ void merge_final(const uint32_t* bk, const int32_t* bi, int n_in,
+                                         uint32_t lo_key, int cut_bin, int above, SelectSmem& sm,
+                                         MergeSmem& ms, int32_t* dst, int32_t* cnt_out) {
+  const int tid = threadIdx.x;
+  const int per = (n_in + kThreads - 1) / kThreads;
+  const int q0 = min(tid * per, n_in), q1 = min(q0 + per, n_in);
+  const bool cut = cut_bin >= 0;  // uniform
+  const uint32_t cut_lo = cut ? static_cast<uint32_t>(cut_bin) << kSelShift : 0u;
+  const uint32_t cut_hi = cut ? cut_lo | ((1u << kSelShift) - 1u) : 0xFFFFFFFFu;
+  const uint32_t in_lo = lo_key > cut_lo ? lo_key : cut_lo;
+  // candidate classes: sure (above the cut bin, or every candidate when no
+  // cut is needed) and in-cut
+  uint32_t T = 0xFFFFFFFFu;
+  int need_eq = 0;
+  if (cut) {
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0;
+#pragma unroll 1
+    for (int q = q0; q < q1; ++q) {
+      const uint32_t k = bk[pad32(q)];
+      if (k >= in_lo && k <= cut_hi) {
+        kmin = k < kmin ? k : kmin;
+        kmax = k > kmax ? k : kmax;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint32_t x = __shfl_xor_sync(0xffffffffu, kmin, o);
+      const uint32_t y = __shfl_xor_sync(0xffffffffu, kmax, o);
+      kmin = x < kmin ? x : kmin;
+      kmax = y > kmax ? y : kmax;
+    }
+    if ((tid & 31) == 0 && kmin <= kmax) {
+      atomicMin(&ms.kmin, kmin);
+      atomicMax(&ms.kmax, kmax);
+    }
+    __syncthreads();
+    // the candidates of the cut bin share every bit above the highest one
+    // where their min and max differ; the rest comes from radix passes
+    kmin = ms.kmin;
+    const uint32_t diff = kmin ^ ms.kmax;
+    uint32_t prefix = 0, pmask = 0;
+    int rem = kTopK - above;
+#pragma unroll 1
+    for (int d = 0; d < 3; ++d) {
+      const int shift = 14 - 7 * d;
+      if ((diff >> shift) == 0) {  // uniform
+        prefix |= kmin & (127u << shift);
+        pmask |= 127u << shift;
+        continue;
+      }
+#pragma unroll 1
+      for (int q = q0; q < q1; ++q) {
+        const uint32_t k = bk[pad32(q)];
+        if (k >= in_lo && k <= cut_hi && (k & pmask) == prefix)
+          atomicAdd(&ms.rh[d][(k >> shift) & 127u], 1);
+      }
+      __syncthreads();
+      if (tid < 32) {
+        int c[4], lsum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          c[j] = ms.rh[d][127 - (tid * 4 + j)];
+          lsum += c[j];
+        }
+        int cum = warp_incl_scan(lsum) - lsum;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (cum < rem && rem <= cum + c[j]) {
+            ms.dig[d] = 127 - (tid * 4 + j);
+            ms.abv[d] = cum;
+          }
+          cum += c[j];
+        }
+      }
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(ms.dig[d]) << shift;
+      pmask |= 127u << shift;
+      rem -= ms.abv[d];
+    }
+    T = cut_lo | (prefix & ((1u << kSelShift) - 1u));
+    need_eq = rem;
+  }
+  // chosen: every sure candidate, the in-cut ones above T and the first
+  // need_eq equal to T.  One scan of (above, equal) counts packed in 16-bit
+  // halves (at most 8192 each) places them.
+  auto sure = [&](uint32_t k) { return cut ? k > cut_hi : k >= lo_key; };
+  int ca = 0, ce = 0;
+#pragma unroll 1
+  for (int q = q0; q < q1; ++q) {
+    const uint32_t k = bk[pad32(q)];
+    if (sure(k)) ++ca;
+    else if (cut && k >= in_lo && k <= cut_hi) {
+      ca += k > T;
+      ce += k == T;
+    }
+  }
+  int tot;
+  const int ex = group_excl_scan<kThreads, 0>((ca << 16) | ce, tid, sm.scan, &tot);
+  int eq_seen = ex & 0xFFFF;
+  int pos = (ex >> 16) + min(need_eq, eq_seen);
+#pragma unroll 1
+  for (int q = q0; q < q1; ++q) {
+    const uint32_t k = bk[pad32(q)];
+    bool take = sure(k);
+    if (!take && cut && k >= in_lo && k <= cut_hi) {
+      if (k > T) take = true;
+      else if (k == T) take = eq_seen++ < need_eq;
+    }
+    if (take && pos < kTopK) dst[pos++] = bi[pad32(q)];
+  }
+  int n = (tot >> 16) + min(need_eq, tot & 0xFFFF);
+  if (n > kTopK) n = kTopK;  // cannot happen for consistent inputs
+  for (int j = n + tid; j < kTopK; j += kThreads) dst[j] = -1;
+  if (tid == 0) *cnt_out = n;
+}
 
 __global__ void __launch_bounds__(kThreads)
     k_select_merge(const uint32_t* __restrict__ ghist, const uint32_t* __restrict__ list_key,
@@ -151,62 +285,97 @@ __global__ void __launch_bounds__(kThreads)
   uint32_t* buf_key = reinterpret_cast<uint32_t*>(dyn);
   int32_t* buf_idx = reinterpret_cast<int32_t*>(buf_key + pad32(kMergeCap));
   __shared__ SelectSmem sm;
+  __shared__ MergeSmem ms;
   __shared__ int seg_off[kThreads + 1];
-  __shared__ uint32_t s_theta;
   __shared__ int s_bin, s_above;
   const int r = blockIdx.x, tid = threadIdx.x;
-  const int c_first = row_first[r], c_last = row_last[r];
-  if (c_first < 0 || c_last < c_first) return;  // no tile: outputs stay as initialised
-  const int64_t total = *total_p;
-
-  // 1. exact lower bound: thread t owns bins kSelBins-1-4t .. kSelBins-4-4t
-  {
-    const uint32_t* h = ghist + static_cast<int64_t>(r) * kSelBins;
-    int c[4], sum = 0;
+  // Loads that do not depend on the row's CTA range go out together: the
+  // histogram (thread t owns bins kSelBins-1-4t .. kSelBins-4-4t), the range,
+  // the tile total and the list count of CTA t (slot t + r).
+  const uint32_t* h = ghist + static_cast<int64_t>(r) * kSelBins;
+  int hc[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      c[j] = static_cast<int>(h[kSelBins - 1 - (tid * 4 + j)]);
-      sum += c[j];
-    }
-    if (tid == 0) {
-      s_theta = 0;
-      s_bin = -1;
-      s_above = 0;
-    }
+  for (int j = 0; j < 4; ++j) hc[j] = static_cast<int>(h[kSelBins - 1 - (tid * 4 + j)]);
+  const int c_first = row_first[r], c_last = row_last[r];
+  const int64_t total = *total_p;
+  const int m_pre = tid < G ? list_cnt[static_cast<int64_t>(tid) + r] : 0;
+  for (int b = tid; b < 3 * 128; b += kThreads) (&ms.rh[0][0])[b] = 0;
+  if (tid < 3) {
+    ms.dig[tid] = 0;
+    ms.abv[tid] = 0;
+  }
+  if (tid == 0) {
+    s_bin = -1;
+    s_above = 0;
+    ms.kmin = 0xFFFFFFFFu;
+    ms.kmax = 0;
+  }
+  if (c_first < 0 || c_last < c_first) return;  // no tile: outputs stay as initialised
+  const int nseg = c_last - c_first + 1;
+  auto has_tiles = [&](int c) { return (total * (c + 1) / G) > (total * c / G); };
+
+  // 1. exact lower bound from the complete histogram
+  {
+    int sum = hc[0] + hc[1] + hc[2] + hc[3];
     int tot;
     int cum = group_excl_scan<kThreads, 0>(sum, tid, sm.scan, &tot);
     if (tot > kTopK) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (cum < kTopK && kTopK <= cum + c[j]) {
-          const int bin = kSelBins - 1 - (tid * 4 + j);
-          s_theta = static_cast<uint32_t>(bin) << kSelShift;
-          s_bin = bin;
+        if (cum < kTopK && kTopK <= cum + hc[j]) {
+          s_bin = kSelBins - 1 - (tid * 4 + j);
           s_above = cum;  // keys in higher bins: all of them are selected
         }
-        cum += c[j];
+        cum += hc[j];
       }
     }
     __syncthreads();
   }
-  uint32_t theta = s_theta, tkeep = s_theta;
   const int cut_bin = s_bin, above = s_above;
+  const uint32_t theta = cut_bin < 0 ? 0u : static_cast<uint32_t>(cut_bin) << kSelShift;
+  int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
 
-  // 2. list offsets of the row's CTAs, in CTA order
-  const int nseg = c_last - c_first + 1;
+  // 2. list offsets, in CTA order (the scoring grid fits one CTA of threads)
+  int mtot = 0;
+  if (G <= kThreads) {  // uniform
+    const bool mine = tid >= c_first && tid <= c_last && has_tiles(tid);
+    const int off = group_excl_scan<kThreads, 0>(mine ? m_pre : 0, tid, sm.scan, &mtot);
+    if (tid >= c_first && tid <= c_last) seg_off[tid - c_first] = off;
+    if (tid == 0) seg_off[nseg] = mtot;
+    __syncthreads();
+  }
+  if (G <= kThreads && mtot <= kMergeCap) {  // uniform
+    // 3. every list entry straight into the buffer (asynchronous copies)
+#pragma unroll 1
+    for (int f = tid; f < mtot; f += kThreads) {
+      int lo_s = 0, hi_s = nseg - 1;  // last segment with seg_off <= f
+      while (lo_s < hi_s) {
+        const int mid = (lo_s + hi_s + 1) >> 1;
+        if (seg_off[mid] <= f) lo_s = mid; else hi_s = mid - 1;
+      }
+      const int64_t e = (static_cast<int64_t>(c_first + lo_s) + r) * kTopK + (f - seg_off[lo_s]);
+      cp_async4(buf_key + pad32(f), list_key + e);
+      cp_async4(buf_idx + pad32(f), list_idx + e);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    merge_final(buf_key, buf_idx, mtot, theta, cut_bin, above, sm, ms, dst, out_cnt + r);
+    return;
+  }
+
+  // Long rows (more candidates than fit at once, or a wider scoring grid):
+  // gather in rounds, compacting to the best 512 when the buffer fills up.
+  uint32_t thr_keep = theta, thr_admit = theta;
   int nbuf = 0;
   for (int sb = 0; sb < nseg; sb += kThreads) {
     const int c = c_first + sb + tid;
-    int m = 0;
-    if (sb + tid < nseg && (total * (c + 1) / G) > (total * c / G))
-      m = list_cnt[static_cast<int64_t>(c) + r];
-    int mtot;
-    const int moff = group_excl_scan<kThreads, 0>(m, tid, sm.scan, &mtot);
+    const int m = (sb + tid < nseg && has_tiles(c)) ? list_cnt[static_cast<int64_t>(c) + r] : 0;
+    int stot;
+    const int moff = group_excl_scan<kThreads, 0>(m, tid, sm.scan, &stot);
     seg_off[tid] = moff;
     __syncthreads();
     const int nsg = min(kThreads, nseg - sb);
-    // 3. gather in rounds; thread t takes entries base + 4t .. base + 4t + 3
-    for (int base = 0; base < mtot; base += kThreads * kMergePer) {
+    for (int base = 0; base < stot; base += kThreads * kMergePer) {
       uint32_t k[kMergePer];
       int32_t ix[kMergePer];
       int npass = 0;
@@ -216,7 +385,7 @@ __global__ void __launch_bounds__(kThreads)
         const int f = base + tid * kMergePer + u;
         k[u] = 0;
         ix[u] = 0;
-        if (f < mtot) {
+        if (f < stot) {
           int lo_s = 0, hi_s = nsg - 1;  // last segment with seg_off <= f
           while (lo_s < hi_s) {
             const int mid = (lo_s + hi_s + 1) >> 1;
@@ -226,7 +395,7 @@ __global__ void __launch_bounds__(kThreads)
           const int j = f - seg_off[lo_s];
           k[u] = list_key[sl * kTopK + j];
           ix[u] = list_idx[sl * kTopK + j];
-          if (k[u] >= theta) {
+          if (k[u] >= thr_admit) {
             pass |= 1u << u;
             ++npass;
           }
@@ -256,7 +425,7 @@ __global__ void __launch_bounds__(kThreads)
           if (q < nbuf) {
             kk[i] = buf_key[pad32(q)];
             ii[i] = buf_idx[pad32(q)];
-            if (kk[i] >= tkeep) valid |= 1u << i;
+            if (kk[i] >= thr_keep) valid |= 1u << i;
           }
         }
         __syncthreads();
@@ -266,54 +435,17 @@ __global__ void __launch_bounds__(kThreads)
           buf_idx[pad32(p)] = ii[i];
         });
         if (thr != 0) {
+          // a later entry equal to thr has a higher block id: it loses
           const uint32_t t1 = thr == 0xFFFFFFFFu ? thr : thr + 1;
-          theta = t1 > theta ? t1 : theta;
-          tkeep = thr > tkeep ? thr : tkeep;
+          thr_admit = t1 > thr_admit ? t1 : thr_admit;
+          thr_keep = thr > thr_keep ? thr : thr_keep;
         }
       }
       __syncthreads();
     }
     __syncthreads();
   }
-
-  // 4. the row's result.  Every candidate in a bin above the cut bin is
-  // selected (there are `above` of them, all present); the K - above best of
-  // the cut bin (ties: lower block) complete the set.  Those share their top
-  // 11 key bits, so the radix passes over them skip the leading digits.
-  uint32_t kk[16];
-  int32_t ii[16];
-  uint32_t in_cut = 0, sure = 0;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int q = tid * 16 + i;
-    kk[i] = 0;
-    ii[i] = 0;
-    if (q < nbuf) {
-      kk[i] = buf_key[pad32(q)];
-      ii[i] = buf_idx[pad32(q)];
-      if (kk[i] >= tkeep) {
-        const int bin = static_cast<int>(kk[i] >> kSelShift);
-        if (cut_bin < 0 || bin > cut_bin) sure |= 1u << i;
-        else if (bin == cut_bin) in_cut |= 1u << i;
-      }
-    }
-  }
-  uint32_t chosen = 0;
-  if (cut_bin >= 0) {  // uniform
-    uint32_t thr;
-    group_select<16, kThreads, 0>(kk, in_cut, kTopK - above, tid, sm, &thr,
-                                  [&](int i, int) { chosen |= 1u << i; });
-  }
-  const uint32_t take = sure | chosen;
-  int n;
-  int pos = group_excl_scan<kThreads, 0>(__popc(take), tid, sm.scan, &n);
-  int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    if (((take >> i) & 1u) && pos < kTopK) dst[pos++] = ii[i];
-  if (n > kTopK) n = kTopK;  // cannot happen for consistent inputs
-  for (int j = n + tid; j < kTopK; j += kThreads) dst[j] = -1;
-  if (tid == 0) out_cnt[r] = n;
+  merge_final(buf_key, buf_idx, nbuf, thr_keep, cut_bin, above, sm, ms, dst, out_cnt + r);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
