@@ -12,25 +12,35 @@
 //   out[h] = sum_t softmax_t(sm_scale * q_h . c_t) c_t   over the token set S
 //   S = tokens of the selected blocks  U  the query's partial tail block.
 //
-// One CTA = one query row, 64 heads, one split of the row's token list.
-// The list is walked in tiles of 64 tokens:
-//   * gather: 128 threads copy the tile's latent rows (each selected block is
-//     4 KiB contiguous in HBM) with 16-byte cp.async into shared memory in the
-//     128-byte-swizzle K-major layout (8 regions of 64 dims), double-buffered;
-//   * S = Q C^T: 32 tcgen05.mma (M = 64 heads, N = 64 tokens, K = 16) into
-//     TMEM lanes 16-31 of each 32-lane quarter (an M = 64 accumulator uses
-//     lanes 0-15 of each quarter, so the other half is free);
-//   * softmax: the thread that owns TMEM lane 16+i of warp w holds the logits
-//     of head 16w+i for the tile, masks skipped/absent tokens, keeps the
-//     running max m (base 2) and sum l, writes P (bf16) to shared memory.  The
-//     running max is raised lazily: only when a tile's max exceeds it by more
-//     than 8 (so p <= 2^8) is O rescaled, by the partner thread that owns
-//     lane i (the O row of the same head);
-//   * O += P C: 8 tcgen05.mma (M = 64, N = 256, K = 16; C is read in its
-//     MN-major form from the same shared-memory tile) into TMEM lanes 0-15,
-//     columns 0-511.
-// A split writes out/lse directly (one split) or an unnormalised partial with
-// its (m, l) for the merge kernel (log-sum-exp rule).
+// One CTA = one query row, 64 heads, one split of the row's token list.  The
+// token positions of the split (and a validity bit per token) are computed
+// once into shared memory; the list is then walked in tiles of 64 tokens.
+//
+// TMEM (128 lanes x 512 columns; an M = 64 accumulator puts row 16w+i of
+// the tile in lane 32w+i, or 32w+16+i with the lane offset 16):
+//   O dims   0-255: lanes 32w+i,    columns 0-255
+//   O dims 256-511: lanes 32w+16+i, columns 0-255
+//   S (64 tokens):  lanes 32w+16+i, columns 256+64b .. (b = S buffer 0/1)
+// The two threads of warp w that own TMEM lanes i and 16+i share head 16w+i:
+// each holds half of its output row, and for the softmax the thread of lane
+// 16+i hands the logits of tokens 0-31 to its partner (one shuffle each), so
+// both threads work on 32 logits.
+//
+// Per tile: 16-byte cp.async gather of the latent rows into the
+// 128-byte-swizzle K-major layout (double-buffered); S = Q C^T as 32
+// tcgen05.mma (M = 64, N = 64, K = 16); softmax in registers (running max in
+// base 2, raised lazily: O is rescaled only when a tile's max exceeds it by
+// more than 8); P (bf16) to shared memory; O += P C as 8 tcgen05.mma
+// (M = 64, N = 256, K = 16, C read MN-major from the same tile).  While the
+// first tile's softmax runs, the tensor core already computes the second
+// tile's logits.
+//
+// A row with a single split writes its normalised output directly.  The n
+// splits of one (row, head group) otherwise form a thread-block cluster: each
+// CTA writes its unnormalised O rows (fp32) and per-head (m, l) to global
+// memory (L2), the cluster barrier makes them visible, and CTA k combines
+// heads [k*64/n, (k+1)*64/n) of all splits with the log-sum-exp rule into
+// the bf16 output and the log-sum-exp.  No second kernel runs.
 #include "spx_device.cuh"
 #include "spx_internal.h"
 
@@ -45,12 +55,17 @@ constexpr int kRegion = 64 * 128;               // [64 rows x 128 B] = 8 KiB
 constexpr int kQBytes = 8 * kRegion;            // 64 KiB
 constexpr int kKVBytes = 8 * kRegion;           // 64 KiB per tile
 constexpr int kPBytes = kRegion;                // [64 heads x 64 tokens] bf16
-constexpr int kSmemBytes = 1024 + kQBytes + 2 * kKVBytes + kPBytes + 2 * kTT * 8 + 64;
+constexpr int kMaxList = kTopK * kPool + kPool - 1;             // tokens in a list, at most
+constexpr int kPosCap = (kMaxList + kTT - 1) / kTT * kTT;       // position slots
+constexpr int kMaxCluster = 16;                 // splits per (row, head group)
+constexpr int kSmemBytes = 1024 + kQBytes + 2 * kKVBytes + kPBytes + kPosCap * 8 +
+                           (kPosCap / 32) * 4 + kHG * 2 * 4 + 64;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLazy = 8.f;                    // rescale threshold (log2 units)
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, kTT);
 // PV: B (the latent tile) is MN-major: set the "transpose B" bit.
 constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256) | (1u << 16);
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct KParams {
   const __nv_bfloat16* q;
@@ -61,13 +76,13 @@ struct KParams {
   const int32_t* count;
   const int64_t* n_vis;
   int heads;
-  int nsplit;
-  int split_tokens;
+  int nsplit;        // = cluster size
+  int split_tokens;  // list entries per split (the last split takes the rest)
   float scale_log2;
   __nv_bfloat16* out;
   float* lse;
-  float* part_o;   // [rows, nsplit, heads, 512]
-  float* part_ml;  // [rows, nsplit, heads, 2]
+  float* part_o;   // [rows, groups, nsplit, 64, 512] unnormalised O (nsplit > 1)
+  float* part_ml;  // [rows, groups, nsplit, 64, 2]   (m, l)
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -86,6 +101,17 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Thread-block cluster helpers.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
 // Byte offset of 16-byte piece `c` (0..63) of row `r` in a tile stored as 8
 // regions of [64 rows x 128 B] with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t sw_off(int r, int c) {
@@ -159,367 +185,418 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* q_s = sm;
-  uint8_t* kv_s = q_s + kQBytes;
+  uint8_t* kv_s = q_s + kQBytes;  // two latent tiles; afterwards the received O rows
   uint8_t* p_s = kv_s + 2 * kKVBytes;
-  int64_t* pos_s = reinterpret_cast<int64_t*>(p_s + kPBytes);  // [2][64]
-  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(pos_s + 2 * kTT);
+  int64_t* pos_s = reinterpret_cast<int64_t*>(p_s + kPBytes);     // [kPosCap]
+  uint32_t* vm_s = reinterpret_cast<uint32_t*>(pos_s + kPosCap);  // [kPosCap / 32] valid bits
+  float* ml_s = reinterpret_cast<float*>(vm_s + kPosCap / 32);    // [64][2]: (m, l) per head
+  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(ml_s + 2 * kHG);
   uint64_t* bar_pv = bar_qk + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_pv + 1);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 3);
 
   const int split = blockIdx.x, r = blockIdx.y, hg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h0 = hg * kHG;
+  const int n_cl = p.nsplit;
   const RowInfo ri = row_info(p, r);
   const int j_begin = split * p.split_tokens;
-  const int j_end = min(ri.S, j_begin + p.split_tokens);
-  const int ntiles = j_end > j_begin ? (j_end - j_begin + kTT - 1) / kTT : 0;
-  // head owned by this thread: lanes 0-15 hold O rows, lanes 16-31 S rows
+  const int j_end = split == n_cl - 1 ? ri.S : min(ri.S, j_begin + p.split_tokens);
+  const int nlist = j_end > j_begin ? j_end - j_begin : 0;
+  const int ntiles = (nlist + kTT - 1) / kTT;
+  // head of this thread; lanes i and 16+i of a warp share it
   const int hloc = warp * 16 + (lane & 15);
-  const int head = h0 + hloc;
-  const bool head_ok = head < p.heads;
-
-  if (ntiles == 0) {
-    for (int i = tid; i < kHG * kLatent; i += kThreads) {
-      const int hh = h0 + i / kLatent;
-      if (hh >= p.heads) continue;
-      if (p.nsplit == 1)
-        p.out[(static_cast<int64_t>(r) * p.heads + hh) * kLatent + i % kLatent] =
-            __float2bfloat16_rn(0.f);
-      else
-        p.part_o[((static_cast<int64_t>(r) * p.nsplit + split) * p.heads + hh) * kLatent +
-                 i % kLatent] = 0.f;
-    }
-    if (tid < kHG && h0 + tid < p.heads) {
-      const int hh = h0 + tid;
-      if (p.nsplit == 1) {
-        if (p.lse) p.lse[static_cast<int64_t>(r) * p.heads + hh] = -INFINITY;
-      } else {
-        const int64_t b = (static_cast<int64_t>(r) * p.nsplit + split) * p.heads + hh;
-        p.part_ml[b * 2] = -INFINITY;
-        p.part_ml[b * 2 + 1] = 0.f;
-      }
-    }
-    return;
-  }
+  const int half = lane >> 4;  // 0: tokens 0-31 / dims 0-255, 1: tokens 32-63 / dims 256-511
+  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
 
   if (tid == 0) {
     mbar_init(bar_qk, 1);
     mbar_init(bar_pv, 1);
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
-  }
-
-  const __nv_bfloat16* lat = p.latent + static_cast<int64_t>(r) * p.seq_stride;
-  const uint32_t q_u = smem_u32(q_s), kv_u = smem_u32(kv_s), p_u = smem_u32(p_s);
-
-  // Q [64 heads x 512] (heads beyond H zero-filled): part of the first group
-  {
-    const __nv_bfloat16* qr = p.q + (static_cast<int64_t>(r) * p.heads) * kLatent;
-    for (int c = tid; c < kHG * 64; c += kThreads) {
-      const int h = c >> 6, piece = c & 63;
-      const bool ok = h0 + h < p.heads;
-      cp_async16(q_u + sw_off(h, piece),
-                 qr + static_cast<int64_t>(ok ? h0 + h : 0) * kLatent + piece * 8, ok);
-    }
-  }
-  auto fill_pos = [&](int tile, int buf) {
-    if (tid < kTT) {
-      const int j = j_begin + tile * kTT + tid;
-      pos_s[buf * kTT + tid] = j < j_end ? token_pos(p, r, ri, j) : -1;
-    }
-  };
-  auto gather = [&](int buf) {
-    const uint32_t dst = kv_u + buf * kKVBytes;
-    const int64_t* ps = pos_s + buf * kTT;
-#pragma unroll 4
-    for (int i = 0; i < (kTT * 64) / kThreads; ++i) {
-      const int c = i * kThreads + tid;
-      const int t = c >> 6, piece = c & 63;
-      const int64_t pos = ps[t];
-      cp_async16(dst + sw_off(t, piece), lat + (pos >= 0 ? pos : 0) * kLatent + piece * 8,
-                 pos >= 0);
-    }
-    cp_async_commit();
-  };
-
-  fill_pos(0, 0);
-  __syncthreads();
-  gather(0);  // group: Q + tile 0
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  // MMA destinations: O in the lower half of each 32-lane quarter (lanes
-  // 0-15, columns 0-511), S in the upper half (lanes 16-31, columns 0-63).
-  const uint32_t t_o = tmem;
-  const uint32_t t_s = tmem + (16u << 16);
-  const uint32_t my_lane_base = static_cast<uint32_t>(warp * 32) << 16;
-
-  float m_run = -INFINITY, l_run = 0.f;  // meaningful in the S-lane threads
+  float m_run = -INFINITY, l_run = 0.f;  // of head hloc (both threads)
   bool ok_all = true;
+  uint32_t tmem = 0;
 
-  for (int j = 0; j < ntiles; ++j) {
-    const int buf = j & 1;
-    cp_async_wait<0>();
-    fence_proxy_async();
+  if (ntiles > 0) {  // uniform
+    if (warp == 0) {
+      tmem_alloc(tmem_holder, 512);
+      tmem_relinquish();
+    }
+    const __nv_bfloat16* lat = p.latent + static_cast<int64_t>(r) * p.seq_stride;
+    const uint32_t q_u = smem_u32(q_s), kv_u = smem_u32(kv_s), p_u = smem_u32(p_s);
+
+    // Q [64 heads x 512] (heads beyond H zero-filled): part of the first group
+    {
+      const __nv_bfloat16* qr = p.q + (static_cast<int64_t>(r) * p.heads) * kLatent;
+#pragma unroll 4
+      for (int c = tid; c < kHG * 64; c += kThreads) {
+        const int h = c >> 6, piece = c & 63;
+        const bool ok = h0 + h < p.heads;
+        cp_async16(q_u + sw_off(h, piece),
+                   qr + static_cast<int64_t>(ok ? h0 + h : 0) * kLatent + piece * 8, ok);
+      }
+    }
+    // every token position of the split, once, with a validity bit per token
+#pragma unroll 1
+    for (int i0 = 0; i0 < ntiles * kTT; i0 += kThreads) {
+      const int i = i0 + tid;
+      int64_t pos = -1;
+      if (i < nlist) pos = token_pos(p, r, ri, j_begin + i);
+      if (i < ntiles * kTT) pos_s[i] = pos;
+      const uint32_t bits = __ballot_sync(0xffffffffu, pos >= 0);
+      if (lane == 0 && i < ntiles * kTT) vm_s[i >> 5] = bits;
+    }
     __syncthreads();
+    auto gather = [&](int tile) {
+      const uint32_t dst = kv_u + (tile & 1) * kKVBytes;
+      const int64_t* ps = pos_s + tile * kTT;
+#pragma unroll 4
+      for (int i = 0; i < (kTT * 64) / kThreads; ++i) {
+        const int c = i * kThreads + tid;
+        const int t = c >> 6, piece = c & 63;
+        const int64_t pos = ps[t];
+        cp_async16(dst + sw_off(t, piece), lat + (pos >= 0 ? pos : 0) * kLatent + piece * 8,
+                   pos >= 0);
+      }
+      cp_async_commit();
+    };
+    gather(0);                   // group: Q + tile 0
+    if (ntiles > 1) gather(1);   // group: tile 1
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    tmem = *tmem_holder;
+    const uint32_t t_o = tmem + lane_base;  // this warp's O rows (lanes i / 16+i)
 
-    // ---- S = Q C^T --------------------------------------------------------
-    if (tid == 0) {
+    // S = Q C^T of tile t into S buffer t&1 (issued by thread 0)
+    auto issue_qk = [&](int t) {
       tc_fence_after();
-      const uint32_t kvb = kv_u + buf * kKVBytes;
-#pragma unroll
+      const uint32_t kvb = kv_u + (t & 1) * kKVBytes;
+      const uint32_t d = tmem + (16u << 16) + 256 + 64 * (t & 1);
+#pragma unroll 4
       for (int k = 0; k < kLatent / 16; ++k) {
         const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
-        umma_bf16(t_s, sdesc_kmajor_sw128(q_u + off), sdesc_kmajor_sw128(kvb + off), kIdescQK,
+        umma_bf16(d, sdesc_kmajor_sw128(q_u + off), sdesc_kmajor_sw128(kvb + off), kIdescQK,
                   k > 0 ? 1u : 0u);
       }
       umma_commit(bar_qk);
-    }
-    // the previous PV must be done before its buffer is refilled and before
-    // P or O are touched again
-    if (j > 0) {
-      volatile int no_abort = 0;
-      ok_all &= mbar_wait(bar_pv, (j - 1) & 1, &no_abort);
-    }
-    if (j + 1 < ntiles) {
-      fill_pos(j + 1, buf ^ 1);
-      __syncthreads();
-      gather(buf ^ 1);
-    }
-    {
-      volatile int no_abort = 0;
-      ok_all &= mbar_wait(bar_qk, j & 1, &no_abort);
-    }
-    tc_fence_after();
+    };
 
-    // ---- softmax -----------------------------------------------------------
-    // A warp reads its own 32-lane quarter: lanes 16-31 receive the S rows
-    // (lanes 0-15 receive O columns 0-63, unused here).
-    float s[kTT];
-    {
-      uint32_t* sr = reinterpret_cast<uint32_t*>(s);
-      tmem_ld_x32_async(tmem + my_lane_base, sr);
-      tmem_ld_x32_async(tmem + my_lane_base + 32, sr + 32);
-      tmem_ld_wait_regs<kTT>(sr);
-    }
-    const int64_t* ps = pos_s + buf * kTT;
-    float mt = -INFINITY;
+    int qk_next = 0;  // first tile whose logits are not yet requested
+#pragma unroll 1
+    for (int j = 0; j < ntiles; ++j) {
+      const int buf = j & 1;
+      if (qk_next == j) {  // uniform
+        // tile j's copies are done (tile 1 is still in flight during tile 0)
+        if (j == 0 && ntiles > 1) cp_async_wait<1>();
+        else cp_async_wait<0>();
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) issue_qk(j);
+        qk_next = j + 1;
+      }
+      {
+        volatile int no_abort = 0;
+        ok_all &= mbar_wait(bar_qk, j & 1, &no_abort);
+      }
+      tc_fence_after();
+      if (j == 0 && ntiles > 1) {
+        // tile 1 was requested with tile 0: its logits overlap this softmax
+        cp_async_wait<0>();
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) issue_qk(1);
+        qk_next = 2;
+      }
+      // the previous PV must be done before its buffer is refilled and before
+      // P or O are touched again
+      if (j > 0) {
+        volatile int no_abort = 0;
+        ok_all &= mbar_wait(bar_pv, (j - 1) & 1, &no_abort);
+        if (j + 1 < ntiles && qk_next == j + 1) gather(j + 1);
+      }
+
+      // ---- softmax: 32 logits of head hloc per thread ----------------------
+      float s[32];
+      {
+        // lanes 16-31 receive the 64 logits of their head; tokens 0-31 go
+        // to the partner lane (lanes 0-15 receive unused columns)
+        uint32_t a[32], b[32];
+        tmem_ld_x32_async(tmem + lane_base + 256 + 64 * buf, a);
+        tmem_ld_x32_async(tmem + lane_base + 256 + 64 * buf + 32, b);
+        tmem_ld_wait_regs<32>(a);
+        tmem_ld_wait_regs<32>(b);
 #pragma unroll
-    for (int t = 0; t < kTT; ++t) {
-      s[t] = ps[t] >= 0 ? s[t] * p.scale_log2 : -INFINITY;
-      mt = fmaxf(mt, s[t]);
-    }
-    float alpha = 1.f;
-    if (lane >= 16) {
+        for (int t = 0; t < 32; ++t) {
+          const uint32_t x = __shfl_xor_sync(0xffffffffu, a[t], 16);
+          s[t] = __uint_as_float(half ? b[t] : x);
+        }
+      }
+      const uint32_t vm = vm_s[j * 2 + half];
+      float mx[8];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) s[t] = ((vm >> t) & 1u) ? s[t] * p.scale_log2 : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx[u] = fmaxf(fmaxf(s[4 * u], s[4 * u + 1]), fmaxf(s[4 * u + 2], s[4 * u + 3]));
+      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+      float alpha = 1.f;
       if (m_run == -INFINITY) {
         m_run = mt;
       } else if (mt > m_run + kLazy) {
         alpha = exp2f(m_run - mt);
         m_run = mt;
       }
-    }
-    // O rows live in the partner lane (lane - 16): rescale there if needed
-    const float alpha_o = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
-    if (__any_sync(0xffffffffu, alpha_o != 1.f) && j > 0) {
-      // whole warp: lanes 0-15 scale their O rows, lanes 16-31 rewrite what they read
-      const float f = lane < 16 ? alpha_o : 1.f;
+      if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
+        // each thread scales its half of the O row of its head
 #pragma unroll 1
-      for (int c = 0; c < kLatent; c += 32) {
-        float v[32];
-        tmem_ld_32x32b_x32(t_o + my_lane_base + c, v);
+        for (int c = 0; c < 256; c += 32) {
+          float v[32];
+          tmem_ld_32x32b_x32(t_o + c, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= f;
-        tmem_st_32x32b_x32(t_o + my_lane_base + c, v);
+          for (int i = 0; i < 32; ++i) v[i] *= alpha;
+          tmem_st_32x32b_x32(t_o + c, v);
+        }
       }
-    }
-    if (lane >= 16) {
-      float lsum = 0.f;
-      uint32_t packed[kTT / 2];
+      uint32_t packed[16];
+      float ps[8];
 #pragma unroll
-      for (int t = 0; t < kTT; t += 2) {
-        const float a = s[t] == -INFINITY ? 0.f : exp2f(s[t] - m_run);
-        const float b = s[t + 1] == -INFINITY ? 0.f : exp2f(s[t + 1] - m_run);
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
-        lsum += __low2float(h2) + __high2float(h2);
-        packed[t / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+      for (int u = 0; u < 8; ++u) {
+        float e[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) e[i] = s[4 * u + i] == -INFINITY ? 0.f : exp2f(s[4 * u + i] - m_run);
+        const __nv_bfloat162 a = __floats2bfloat162_rn(e[0], e[1]);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(e[2], e[3]);
+        packed[2 * u] = *reinterpret_cast<const uint32_t*>(&a);
+        packed[2 * u + 1] = *reinterpret_cast<const uint32_t*>(&b);
+        ps[u] = (__low2float(a) + __high2float(a)) + (__low2float(b) + __high2float(b));
       }
+      float lsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
       l_run = l_run * alpha + lsum;
-      // row hloc of P: 8 pieces of 16 B
+      // row hloc of P, pieces 4*half .. 4*half+3 (16 B each)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t a = p_u + hloc * 128 + ((c ^ (hloc & 7)) << 4);
+      for (int c = 0; c < 4; ++c) {
+        const int piece = 4 * half + c;
+        const uint32_t a = p_u + hloc * 128 + ((piece ^ (hloc & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(packed[4 * c]),
                      "r"(packed[4 * c + 1]), "r"(packed[4 * c + 2]), "r"(packed[4 * c + 3])
                      : "memory");
       }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
 
-    // ---- O += P C ----------------------------------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t kvb = kv_u + buf * kKVBytes;
+      // ---- O += P C --------------------------------------------------------
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t kvb = kv_u + buf * kKVBytes;
 #pragma unroll
-      for (int k = 0; k < kTT / 16; ++k) {
-        const uint64_t ad = sdesc_kmajor_sw128(p_u + k * 32);
+        for (int k = 0; k < kTT / 16; ++k) {
+          const uint64_t ad = sdesc_kmajor_sw128(p_u + k * 32);
 #pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
-          const uint64_t bd =
-              sdesc_mn_sw128(kvb + nh * 4 * kRegion + k * 16 * 128, kRegion, 1024);
-          umma_bf16(t_o + nh * 256, ad, bd, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+          for (int nh = 0; nh < 2; ++nh) {
+            const uint64_t bd =
+                sdesc_mn_sw128(kvb + nh * 4 * kRegion + k * 16 * 128, kRegion, 1024);
+            umma_bf16(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
+                      (j > 0 || k > 0) ? 1u : 0u);
+          }
         }
+        umma_commit(bar_pv);
       }
-      umma_commit(bar_pv);
     }
+    {
+      volatile int no_abort = 0;
+      ok_all &= mbar_wait(bar_pv, (ntiles - 1) & 1, &no_abort);
+    }
+    tc_fence_after();
   }
-  {
-    volatile int no_abort = 0;
-    ok_all &= mbar_wait(bar_pv, (ntiles - 1) & 1, &no_abort);
-  }
-  tc_fence_after();
 
-  // ---- epilogue: lanes 0-15 own the O rows ----------------------------------
-  // The rows go through shared memory (the latent tiles are free now) so that
-  // all 128 threads store them to global memory in coalesced 16-byte pieces.
-  const float m_h = __shfl_sync(0xffffffffu, m_run, (lane & 15) + 16);
-  const float l_h = __shfl_sync(0xffffffffu, l_run, (lane & 15) + 16);
-  const bool single = p.nsplit == 1;
-  const float scale_o = single ? (l_h > 0.f ? 1.f / l_h : 0.f) : 1.f;
-  // staging: single split -> bf16 rows of 1 KiB; partial -> fp32 rows of 2 KiB
-  // (64 rows x 2 KiB = 128 KiB = both latent buffers).  16-byte pieces are
-  // rotated by the row index to spread the banks.
-  uint8_t* stage = kv_s;
-  const int row_bytes = single ? kLatent * 2 : kLatent * 4;
-  const int pieces = row_bytes / 16;
+  // ---- output ----------------------------------------------------------------
+  const bool have = ntiles > 0 && ok_all && l_run > 0.f;
+  const int64_t unit = static_cast<int64_t>(r) * gridDim.z + hg;  // (row, head group)
+  if (n_cl == 1) {
+    // normalised bf16 rows of 1 KiB staged in the latent buffers (16-byte
+    // pieces rotated by the row to spread the banks), then stored coalesced
+    uint8_t* stage = kv_s;
+    const float inv = have ? 1.f / l_run : 0.f;
+    if (ntiles > 0) {
 #pragma unroll 1
-  for (int c0 = 0; c0 < kLatent; c0 += 128) {
-    float vv[128];
-    uint32_t* vr = reinterpret_cast<uint32_t*>(vv);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld_x32_async(t_o + my_lane_base + c0 + 32 * q, vr + 32 * q);
-    tmem_ld_wait_regs<128>(vr);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = c0 + 32 * q;
-    const float* v = vv + 32 * q;
-    if (lane < 16) {
-      if (single) {
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * i] * scale_o, v[2 * i + 1] * scale_o);
-          w[i] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem + lane_base + c0, v);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int piece = (c * 2 / 16 + i + hloc) % pieces;
-          *reinterpret_cast<uint4*>(stage + hloc * row_bytes + piece * 16) =
-              make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          uint32_t w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const __nv_bfloat162 h2 =
+                __floats2bfloat162_rn(v[8 * i + 2 * u] * inv, v[8 * i + 2 * u + 1] * inv);
+            w[u] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          const int piece = ((256 * half + c0) / 8 + i + hloc) & 63;
+          *reinterpret_cast<uint4*>(stage + hloc * 1024 + piece * 16) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
-      } else {
+      }
+    }
+    if (half == 0 && h0 + hloc < p.heads && p.lse)
+      p.lse[static_cast<int64_t>(r) * p.heads + h0 + hloc] =
+          have ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+    __syncthreads();
+    const int nrows = min(kHG, p.heads - h0);
+    uint8_t* gbase =
+        reinterpret_cast<uint8_t*>(p.out + (static_cast<int64_t>(r) * p.heads + h0) * kLatent);
+#pragma unroll 1
+    for (int e = tid; e < nrows * 64; e += kThreads) {
+      const int row = e >> 6, piece = e & 63;
+      const uint4 val =
+          ntiles > 0 ? *reinterpret_cast<const uint4*>(stage + row * 1024 + ((piece + row) & 63) * 16)
+                     : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(gbase + static_cast<int64_t>(row) * 1024 + piece * 16) = val;
+    }
+  } else {
+    // this split's unnormalised O rows and (m, l), fp32, to L2
+    float* po = p.part_o + ((unit * n_cl + split) * kHG) * kLatent;
+    if (ntiles > 0) {
+      // staged as [64 rows x 2 KiB] in the latent buffers (pieces rotated by
+      // the row), then stored coalesced
+      uint8_t* stage = kv_s;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem + lane_base + c0, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int piece = (c * 4 / 16 + i + hloc) % pieces;
-          *reinterpret_cast<float4*>(stage + hloc * row_bytes + piece * 16) =
+          const int piece = ((256 * half + c0) / 4 + i + hloc) & 127;
+          *reinterpret_cast<float4*>(stage + hloc * 2048 + piece * 16) =
               make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
       }
+      __syncthreads();
+#pragma unroll 4
+      for (int e = tid; e < kHG * 128; e += kThreads) {
+        const int row = e >> 7, piece = e & 127;
+        *reinterpret_cast<float4*>(po + row * kLatent + piece * 4) =
+            *reinterpret_cast<const float4*>(stage + row * 2048 + ((piece + row) & 127) * 16);
+      }
     }
-  }
-  }
-  if (lane < 16 && head_ok && ok_all) {
-    if (single) {
-      if (p.lse)
-        p.lse[static_cast<int64_t>(r) * p.heads + head] =
-            l_h > 0.f ? (m_h + __log2f(l_h)) * kLn2 : -INFINITY;
-    } else {
-      const int64_t b = (static_cast<int64_t>(r) * p.nsplit + split) * p.heads + head;
-      p.part_ml[b * 2] = l_h > 0.f ? m_h : -INFINITY;
-      p.part_ml[b * 2 + 1] = l_h;
+    if (half == 0) {
+      float* pm = p.part_ml + ((unit * n_cl + split) * kHG + hloc) * 2;
+      pm[0] = have ? m_run : -INFINITY;
+      pm[1] = have ? l_run : 0.f;
     }
-  }
-  __syncthreads();
-  if (ok_all) {
-    const int nrows = min(kHG, p.heads - h0);
-    uint8_t* gbase = single ? reinterpret_cast<uint8_t*>(p.out + (static_cast<int64_t>(r) * p.heads + h0) * kLatent)
-                            : reinterpret_cast<uint8_t*>(p.part_o + ((static_cast<int64_t>(r) * p.nsplit + split) * p.heads + h0) * kLatent);
-    for (int e = tid; e < nrows * pieces; e += kThreads) {
-      const int row = e / pieces, piece = e % pieces;
-      const int sp = (piece + row) % pieces;
-      *reinterpret_cast<uint4*>(gbase + static_cast<int64_t>(row) * row_bytes + piece * 16) =
-          *reinterpret_cast<const uint4*>(stage + row * row_bytes + sp * 16);
+    cluster_sync_all();  // every split's rows are in L2 and visible to the cluster
+    // CTA k combines heads [k*rows_per, (k+1)*rows_per) of the group:
+    // thread t takes dims 4t..4t+3 of each
+    const int k = static_cast<int>(cluster_rank());
+    const int rows_per = kHG / n_cl;
+    const float* pm_all = p.part_ml + (unit * n_cl) * kHG * 2;
+    const float* po_all = p.part_o + (unit * n_cl) * kHG * kLatent;
+#pragma unroll 1
+    for (int hh = 0; hh < rows_per; ++hh) {
+      const int h = k * rows_per + hh;
+      if (h0 + h >= p.heads) break;  // uniform
+      float2 ml[kMaxCluster];
+      float4 v[kMaxCluster];
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c) {
+        ml[c] = make_float2(-INFINITY, 0.f);
+        v[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c < n_cl) {
+          ml[c] = __ldcg(reinterpret_cast<const float2*>(pm_all + (c * kHG + h) * 2));
+          v[c] = __ldcg(reinterpret_cast<const float4*>(po_all + (c * kHG + h) * kLatent + tid * 4));
+        }
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c) M = fmaxf(M, ml[c].x);
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c) {
+        const float w = ml[c].x == -INFINITY ? 0.f : exp2f(ml[c].x - M);
+        L += ml[c].y * w;
+        if (w != 0.f) {
+          acc.x += v[c].x * w;
+          acc.y += v[c].y * w;
+          acc.z += v[c].z * w;
+          acc.w += v[c].w * w;
+        }
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      __nv_bfloat16* o = p.out + (static_cast<int64_t>(r) * p.heads + h0 + h) * kLatent + tid * 4;
+      const __nv_bfloat162 a2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(o) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&a2), *reinterpret_cast<const uint32_t*>(&b2));
+      if (tid == 0 && p.lse)
+        p.lse[static_cast<int64_t>(r) * p.heads + h0 + h] =
+            L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
     }
   }
   if (!ok_all && tid == 0) atomicExch(&g_device_error, kErrWaitTimeout);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, 512);
+  if (ntiles > 0) {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+  }
 }
 
-// Combines the split partials of one (row, head):
-//   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  out = sum_s O_s 2^(m_s - M) / L.
-__global__ void __launch_bounds__(128) k_attn_merge(const float* __restrict__ part_o,
-                                                    const float* __restrict__ part_ml,
-                                                    int nsplit, int heads,
-                                                    __nv_bfloat16* __restrict__ out,
-                                                    float* __restrict__ lse) {
-  __shared__ float s_w[64];
-  __shared__ float s_inv, s_lse;
-  const int r = blockIdx.x, hh = blockIdx.y;
-  auto base_of = [&](int s) { return (static_cast<int64_t>(r) * nsplit + s) * heads + hh; };
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    float M = -INFINITY;
-    for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, part_ml[base_of(s) * 2]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    for (int s = lane; s < nsplit; s += 32) {
-      const float m = part_ml[base_of(s) * 2];
-      const float wgt = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
-      s_w[s] = wgt;
-      L += part_ml[base_of(s) * 2 + 1] * wgt;
+// Largest cluster size n <= want (a power of two) for which the device can
+// run at least one cluster of the attention kernel.
+int max_cluster(int want) {
+  static int cache[64][5];
+  static bool done[64][5];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  for (int n = want; n > 1; n >>= 1) {
+    int lg = 0;
+    while ((1 << lg) < n) ++lg;
+    if (dev < 64 && done[dev][lg]) {
+      if (cache[dev][lg] > 0) return n;
+      continue;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) {
-      s_inv = L > 0.f ? 1.f / L : 0.f;
-      s_lse = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = n;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int num = 0;
+    if (cudaOccupancyMaxActiveClusters(&num, k_sparse_attn, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      num = 0;
     }
+    if (dev < 64) {
+      done[dev][lg] = true;
+      cache[dev][lg] = num;
+    }
+    if (num > 0) return n;
   }
-  __syncthreads();
-  const int d4 = threadIdx.x;  // 128 threads x 4 dims
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < nsplit; s0 += 8) {
-    float4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {  // independent loads in flight
-      const int s = s0 + u;
-      v[u] = s < nsplit && s_w[s] != 0.f
-                 ? *reinterpret_cast<const float4*>(part_o + base_of(s) * kLatent + d4 * 4)
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float wgt = s0 + u < nsplit ? s_w[s0 + u] : 0.f;
-      acc.x += v[u].x * wgt;
-      acc.y += v[u].y * wgt;
-      acc.z += v[u].z * wgt;
-      acc.w += v[u].w * wgt;
-    }
-  }
-  const float inv = s_inv;
-  __nv_bfloat16* o = out + (static_cast<int64_t>(r) * heads + hh) * kLatent + d4 * 4;
-  reinterpret_cast<__nv_bfloat162*>(o)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  reinterpret_cast<__nv_bfloat162*>(o)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-  if (lse && threadIdx.x == 0) lse[static_cast<int64_t>(r) * heads + hh] = s_lse;
+  return 1;
+}
+
+bool set_attrs() {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && attr_set[dev]) return true;
+  if (cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBytes) != cudaSuccess)
+    return false;
+  if (cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+      cudaSuccess)
+    return false;
+  if (dev < 64) attr_set[dev] = true;
+  return true;
 }
 
 }  // namespace
@@ -530,40 +607,37 @@ AttnPlan plan_attn(int rows, int heads, int64_t max_len, int num_sms) {
   p.heads = heads;
   p.groups = (heads + kHG - 1) / kHG;
   const int64_t max_blk = max_len / kPool;
-  int64_t s_max = (max_blk > kTopK ? kTopK : max_blk) * kPool + kPool - 1;
-  if (s_max > max_len) s_max = max_len;
-  if (s_max < 1) s_max = 1;
+  const int64_t bt = (max_blk > kTopK ? kTopK : max_blk) * kPool;  // block tokens in a list
   const int64_t units = static_cast<int64_t>(rows) * p.groups;
-  int nsplit = 1;
-  if (units < num_sms) nsplit = static_cast<int>((num_sms + units - 1) / units);
-  int64_t ts = (s_max + nsplit - 1) / nsplit;
+  // splits per (row, group): a power of two up to 16 that keeps every SM
+  // busy at most once and every split at least one tile long
+  int n = 1;
+  while (n < kMaxCluster && units * (2 * n) <= num_sms && bt / (2 * n) >= kTT) n *= 2;
+  p.nsplit = n;
+  int64_t ts = (bt + n - 1) / n;
   ts = (ts + kTT - 1) / kTT * kTT;
-  if (ts < 2 * kTT) ts = 2 * kTT;  // at least two tiles per split: fewer partials
+  if (ts < kTT) ts = kTT;
   p.split_tokens = static_cast<int>(ts);
-  p.nsplit = static_cast<int>((s_max + ts - 1) / ts);
-  if (p.nsplit > 64) {  // the merge keeps at most 64 split weights
-    ts = ((s_max + 63) / 64 + kTT - 1) / kTT * kTT;
-    p.split_tokens = static_cast<int>(ts);
-    p.nsplit = static_cast<int>((s_max + ts - 1) / ts);
-  }
   p.ws_bytes = 0;
-  if (p.nsplit > 1) {
-    const size_t n = static_cast<size_t>(rows) * p.nsplit * heads;
-    p.ws_bytes = ((n * kLatent * 4 + 255) & ~static_cast<size_t>(255)) + n * 2 * 4;
+  if (n > 1) {
+    const size_t units_n = static_cast<size_t>(units) * n * kHG;
+    p.ws_bytes = ((units_n * kLatent * 4 + 255) & ~static_cast<size_t>(255)) + units_n * 2 * 4;
   }
   return p;
 }
 
-cudaError_t launch_attn(const AttnPlan& pl, const AttnArgs& a, cudaStream_t stream) {
-  if (pl.rows == 0) return cudaSuccess;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+cudaError_t launch_attn(const AttnPlan& pl0, const AttnArgs& a, cudaStream_t stream) {
+  if (pl0.rows == 0) return cudaSuccess;
+  if (!set_attrs()) return cudaGetLastError();
+  AttnPlan pl = pl0;
+  if (pl.nsplit > 1) {
+    const int n = max_cluster(pl.nsplit);
+    if (n != pl.nsplit) {  // fewer, longer splits
+      const int64_t total = static_cast<int64_t>(pl.split_tokens) * pl.nsplit;
+      int64_t ts = (total + n - 1) / n;
+      pl.split_tokens = static_cast<int>((ts + kTT - 1) / kTT * kTT);
+      pl.nsplit = n;
+    }
   }
   KParams p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
@@ -579,20 +653,29 @@ cudaError_t launch_attn(const AttnPlan& pl, const AttnArgs& a, cudaStream_t stre
   p.scale_log2 = a.sm_scale * 1.44269504088896340736f;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
-  const size_t n = static_cast<size_t>(pl.rows) * pl.nsplit * pl.heads;
-  p.part_o = static_cast<float*>(a.ws);
-  p.part_ml = pl.nsplit > 1
-                  ? reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
-                                             ((n * kLatent * 4 + 255) & ~static_cast<size_t>(255)))
-                  : nullptr;
-  dim3 grid(pl.nsplit, pl.rows, pl.groups);
-  k_sparse_attn<<<grid, kThreads, kSmemBytes, stream>>>(p);
+  p.part_o = nullptr;
+  p.part_ml = nullptr;
+  if (pl.nsplit > 1) {
+    const size_t units_n = static_cast<size_t>(pl.rows) * pl.groups * pl.nsplit * kHG;
+    p.part_o = static_cast<float*>(a.ws);
+    p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
+                                         ((units_n * kLatent * 4 + 255) & ~static_cast<size_t>(255)));
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.nsplit, pl.rows, pl.groups);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = pl.nsplit;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_sparse_attn, p);
   count_launches(1);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || pl.nsplit == 1) return e;
-  k_attn_merge<<<dim3(pl.rows, pl.heads), 128, 0, stream>>>(p.part_o, p.part_ml, pl.nsplit,
-                                                            pl.heads, p.out, p.lse);
-  count_launches(1);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
