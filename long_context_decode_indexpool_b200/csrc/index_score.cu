@@ -27,28 +27,14 @@
 //               per tile into one of two TMEM accumulators.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator row, ReLU, weighted
 //               head sum in fp32, length mask; then either a store of the
-//               fp32 scores, or (SELECT) the fused top-k below.
+//               fp32 scores (and, with SELECT, a histogram of their keys).
 //
-// Fused top-k, first stage (SELECT, decode): the epilogue keeps, per row, an
-// index-ordered buffer of candidate blocks in shared memory.  A candidate
-// enters only if its key is >= theta, a lower bound of the row's final
-// 512th-largest key:
-//   * from time to time the CTA adds its 2048-bin histogram of the row's keys
-//     (top 11 key bits) into a global per-row histogram and takes an
-//     asynchronous snapshot of it (cp.async); at the next flush the highest
-//     bin b with at least 512 keys at or above it in the snapshot gives
-//     theta >= b's lower edge (any snapshot of monotone counts is a valid
-//     lower bound);
-//   * when the buffer fills, an exact in-place top-512 of the buffer raises
-//     the admission bound to its 512th key + 1 (a later, higher-index
-//     candidate equal to it loses the tie), while the buffered ties at that
-//     key stay eligible (they are filtered with the key itself).
-// When the CTA leaves a row it publishes its list (<= 512 entries, index
-// order) and, if it holds the row's first or last tile, its own index.  The
-// second stage (k_select_merge in topk.cu, the next launch) reads the
-// complete histogram, filters the lists of the row's CTAs (CTA order = index
-// order) and selects the 512 block ids.  The union of per-chunk exact top-512
-// lists contains the row's top-512, so the result is exact.
+// SELECT (decode): besides the scores, the epilogue counts the row's keys
+// (scores mapped to order-preserving 32-bit keys) in a 2048-bin shared-memory
+// histogram of their top 11 bits and adds it into a global per-row histogram
+// when it leaves the row.  Once the launch is complete that histogram locates
+// the bin of the row's 512th-largest key exactly; the selection kernel
+// (topk.cu) then only keeps blocks at or above that bin.
 //
 // Every wait is bounded; on a timeout the CTA drains and exits with the
 // device error word set.
@@ -69,14 +55,11 @@ constexpr int kThreads = 192;
 constexpr int kEpi = 128;                    // epilogue threads
 constexpr int kHistBins = 2048;              // top 11 key bits
 constexpr int kHistShift = 21;
-constexpr int kBufCap = 2048;                // candidate buffer entries
-constexpr int kEarlyFlush = 4;               // tiles between the first two flushes
-constexpr int kFlushTiles = 16;              // tiles between later flushes
 
 template <int NQ, bool SELECT>
 struct Cfg {
   static constexpr int kN = 32 * NQ;
-  static constexpr int kStages = SELECT ? 5 : (NQ == 1 ? 6 : 4);
+  static constexpr int kStages = NQ == 1 ? 6 : 4;
   static constexpr int kQSlots = NQ == 1 ? 2 : 1;
   static constexpr int kQHalf = kN * 128;
   static constexpr int kQBytes = 2 * kQHalf;
@@ -86,9 +69,7 @@ struct Cfg {
   static constexpr int kNbOff = kWOff + kN * 4;
   static constexpr int kSelOff = (kNbOff + NQ * 8 + 15) & ~15;
   static constexpr int kSelBytes =
-      SELECT ? (2 * kHistBins * 4 + pad32(kBufCap) * 8 + static_cast<int>(sizeof(SelectSmem)) + 64 +
-                (kEpi + 1) * 4)
-             : 0;
+      SELECT ? kHistBins * 4 : 0;
   static constexpr int kBarOff = (kSelOff + kSelBytes + 7) & ~7;
   static constexpr int kNumBars = 2 * kStages + 2 * kQSlots + 4 + 1;
   static constexpr int kSmem = 1024 + kBarOff + kNumBars * 8 + 16;
@@ -105,14 +86,7 @@ struct KParams {
   int rows;
   int groups;
   int shared_keys;
-  // fused selection, first stage (decode)
-  uint32_t* ghist;     // [rows, kHistBins]  zero on entry
-  uint32_t* list_key;  // [grid + rows, 512]
-  int32_t* list_idx;   // [grid + rows, 512]
-  int32_t* list_cnt;   // [grid + rows]
-  int32_t* row_first;  // [rows] CTA holding the row's first tile (-1 on entry)
-  int32_t* row_last;   // [rows] CTA holding the row's last tile (-1 on entry)
-  int64_t* total_out;  // [1] total tiles of the launch
+  uint32_t* ghist;     // SELECT: [rows, kHistBins] key histogram, zero on entry
 };
 
 template <int NQ>
@@ -161,188 +135,6 @@ struct Walker {
 };
 
 __device__ __forceinline__ void epi_sync() { group_sync<kEpi, 1>(); }
-
-// ---------------------------------------------------------------------------
-// Fused selection state of the epilogue warps (SELECT only).
-// ---------------------------------------------------------------------------
-struct SelState {
-  uint32_t* lhist;     // smem [kHistBins]: this CTA's counts since the last flush
-  uint32_t* snap;      // smem [kHistBins]: snapshot of the global histogram
-  uint32_t* buf_key;   // smem [kBufCap]
-  int32_t* buf_idx;    // smem [kBufCap]
-  SelectSmem* ss;      // smem
-  int* wcnt;           // smem [2][4]
-  int* misc;           // smem [8]: threshold broadcast
-  int* seg_off;        // smem [kEpi + 1]: list offsets during a merge
-  int nbuf;
-  int par;
-  int since_flush;
-  bool snap_pending;   // a snapshot copy is in flight (cp.async group)
-  int flushes;         // flushes done in the current row
-  uint32_t theta;      // admission bound for new (higher-index) candidates
-  uint32_t tkeep;      // bound for candidates already in the buffer (<= theta)
-};
-
-// Appends the passing elements of the 128 epilogue threads to the buffer in
-// the order (slot, lane), slot in [0, 4).
-__device__ __forceinline__ void sel_append(SelState& S, bool pass, uint32_t key, int32_t idx,
-                                           int slot, int lane) {
-  const unsigned bal = __ballot_sync(0xffffffffu, pass);
-  if (lane == 0) S.wcnt[S.par * 4 + slot] = __popc(bal);
-  epi_sync();
-  int off = 0, tot = 0;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = S.wcnt[S.par * 4 + q];
-    off += q < slot ? c : 0;
-    tot += c;
-  }
-  if (pass) {
-    const int pos = S.nbuf + off + __popc(bal & ((1u << lane) - 1u));
-    S.buf_key[pad32(pos)] = key;
-    S.buf_idx[pad32(pos)] = idx;
-  }
-  S.nbuf += tot;
-  S.par ^= 1;
-}
-
-// Exact in-place top-K of the buffer among keys >= tkeep; raises the bounds.
-__device__ __forceinline__ void sel_compact(SelState& S, int et) {
-  epi_sync();
-  uint32_t key[16];
-  int32_t idx[16];
-  uint32_t valid = 0;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int j = et * 16 + i;
-    key[i] = 0;
-    idx[i] = 0;
-    if (j < S.nbuf) {
-      key[i] = S.buf_key[pad32(j)];
-      idx[i] = S.buf_idx[pad32(j)];
-      if (key[i] >= S.tkeep) valid |= 1u << i;
-    }
-  }
-  epi_sync();
-  uint32_t thr;
-  const int n = group_select<16, kEpi, 1>(key, valid, kTopK, et, *S.ss, &thr, [&](int i, int pos) {
-    S.buf_key[pad32(pos)] = key[i];
-    S.buf_idx[pad32(pos)] = idx[i];
-  });
-  if (thr != 0) {
-    // Later arrivals have higher block ids, so one equal to thr loses to the
-    // kept ties: admit only keys above thr.  Kept entries equal to thr stay.
-    const uint32_t t1 = thr == 0xFFFFFFFFu ? thr : thr + 1;
-    S.theta = t1 > S.theta ? t1 : S.theta;
-    S.tkeep = thr > S.tkeep ? thr : S.tkeep;
-  }
-  S.nbuf = n;
-  epi_sync();
-}
-
-// Lower bound of the row's K-th largest key from a histogram `h` (shared
-// or global memory, kHistBins counts).  Thread et reads bins
-// kHistBins-1 - (j*128 + et): chunk j holds 128 consecutive bins in
-// descending order.  Chunk totals locate the chunk where the count from the
-// top reaches K, a scan inside it the bin.
-template <bool kGlobal>
-__device__ __forceinline__ uint32_t hist_threshold(const SelState& S, const uint32_t* h, int et) {
-  constexpr int kChunks = kHistBins / kEpi;
-  const int lane = et & 31, wid = et >> 5;
-  int c[kChunks];
-#pragma unroll
-  for (int j = 0; j < kChunks; ++j) {
-    const uint32_t* a = h + (kHistBins - 1 - (j * kEpi + et));
-    c[j] = static_cast<int>(kGlobal ? __ldcg(a) : *a);
-  }
-  int mine = 0;
-#pragma unroll
-  for (int j = 0; j < kChunks; ++j) {
-    int v = c[j];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == j) mine = v;
-  }
-  int* tmp = S.ss->hist;  // [4][32]; no selection runs concurrently
-  tmp[wid * 32 + lane] = lane < kChunks ? mine : 0;
-  epi_sync();
-  if (wid == 0) {
-    const int tj = tmp[lane] + tmp[32 + lane] + tmp[64 + lane] + tmp[96 + lane];
-    const int incl = warp_incl_scan(tj);
-    const int excl = incl - tj;
-    const unsigned m = __ballot_sync(0xffffffffu, excl < kTopK && kTopK <= incl);
-    const int J = m ? __ffs(m) - 1 : -1;
-    const int before = __shfl_sync(0xffffffffu, excl, J < 0 ? 0 : J);
-    if (lane == 0) {
-      S.misc[2] = J;
-      S.misc[3] = before;
-      S.misc[1] = 0;
-    }
-  }
-  epi_sync();
-  const int J = S.misc[2];
-  if (J >= 0) {  // uniform
-    const int before = S.misc[3];
-    int v = 0;
-#pragma unroll
-    for (int j = 0; j < kChunks; ++j) v = (j == J) ? c[j] : v;
-    int tot;
-    const int ex = group_excl_scan<kEpi, 1>(v, et, S.ss->scan, &tot);
-    if (before + ex < kTopK && kTopK <= before + ex + v)
-      S.misc[1] = static_cast<int>(static_cast<uint32_t>(kHistBins - 1 - (J * kEpi + et)) << kHistShift);
-    epi_sync();
-  }
-  const uint32_t t = static_cast<uint32_t>(S.misc[1]);
-  epi_sync();
-  return t;
-}
-
-// Snapshot of the row's global histogram into shared memory, in flight
-// until the next flush (16-byte cp.async through L2).
-__device__ __forceinline__ void snap_issue(SelState& S, const uint32_t* gh, int et) {
-  const uint32_t dst = smem_u32(S.snap);
-#pragma unroll
-  for (int i = 0; i < (kHistBins * 4) / (16 * kEpi); ++i) {
-    const int c = i * kEpi + et;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + c * 16),
-                 "l"(reinterpret_cast<const uint8_t*>(gh) + c * 16)
-                 : "memory");
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  S.snap_pending = true;
-}
-
-__device__ __forceinline__ void snap_wait(SelState& S) {
-  if (S.snap_pending) {
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    S.snap_pending = false;
-  }
-}
-
-// Adds the CTA's local counts into the row's global histogram (bins
-// j*128 + et: no shared-memory bank conflicts), tightens theta from the
-// snapshot taken at the previous flush, and starts the next snapshot.
-__device__ __forceinline__ void sel_flush(SelState& S, uint32_t* gh, int et, bool have_snap) {
-  snap_wait(S);
-  epi_sync();
-#pragma unroll 8
-  for (int j = 0; j < kHistBins / kEpi; ++j) {
-    const int b = j * kEpi + et;
-    const uint32_t c = S.lhist[b];
-    if (c) {
-      atomicAdd(gh + b, c);
-      S.lhist[b] = 0;
-    }
-  }
-  if (have_snap) {
-    const uint32_t t = hist_threshold<false>(S, S.snap, et);
-    S.theta = t > S.theta ? t : S.theta;
-    S.tkeep = t > S.tkeep ? t : S.tkeep;
-  }
-  epi_sync();  // every thread is done with the old snapshot
-  snap_issue(S, gh, et);
-  S.since_flush = 0;
-}
 
 }  // namespace
 
@@ -535,69 +327,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_in_tile = quarter * 32 + lane;
     Walker<NQ> w;
     w.init(p, s_g0, s_t0, lo);
-    int acc = 0, cur_g = -1, cur_nt = 0;
-    int64_t cur_gstart = 0;
+    int acc = 0, cur_g = -1;
     uint32_t acc_ph = 0;
     bool aborted = false;
 
-    SelState S;
+    uint32_t* lhist = reinterpret_cast<uint32_t*>(smem + C::kSelOff);  // SELECT
     if constexpr (SELECT) {
-      uint8_t* sel = smem + C::kSelOff;
-      S.lhist = reinterpret_cast<uint32_t*>(sel);
-      S.snap = S.lhist + kHistBins;
-      S.buf_key = S.snap + kHistBins;
-      S.buf_idx = reinterpret_cast<int32_t*>(S.buf_key + pad32(kBufCap));
-      S.ss = reinterpret_cast<SelectSmem*>(S.buf_idx + pad32(kBufCap));
-      S.wcnt = reinterpret_cast<int*>(S.ss + 1);
-      S.misc = S.wcnt + 8;
-      S.seg_off = S.misc + 8;
-      S.nbuf = 0;
-      S.par = 0;
-      S.since_flush = 0;
-      S.snap_pending = false;
-      S.flushes = 0;
-      S.theta = 0;
-      S.tkeep = 0;
-      for (int b = et; b < kHistBins; b += kEpi) S.lhist[b] = 0;
+      for (int b = et; b < kHistBins; b += kEpi) lhist[b] = 0;
       epi_sync();
     }
-
-    // Leaves row r: flush the counts, filter with the freshest snapshot,
-    // publish this CTA's list (and its index if it holds an end of the row).
-    auto finish_row = [&](int r, int64_t gstart, int nt) {
+    // Leaves row r (SELECT): adds the CTA's counts into the row's histogram.
+    auto flush_hist = [&](int r) {
       uint32_t* gh = p.ghist + static_cast<int64_t>(r) * kHistBins;
-      sel_flush(S, gh, et, S.snap_pending);
-      snap_wait(S);
       epi_sync();
-      {
-        const uint32_t t = hist_threshold<false>(S, S.snap, et);
-        S.theta = t > S.theta ? t : S.theta;
-        S.tkeep = t > S.tkeep ? t : S.tkeep;
-      }
-      sel_compact(S, et);
-      const int64_t slot = static_cast<int64_t>(blockIdx.x) + r;
-      for (int i = et; i < S.nbuf; i += kEpi) {
-        p.list_key[slot * kTopK + i] = S.buf_key[pad32(i)];
-        p.list_idx[slot * kTopK + i] = S.buf_idx[pad32(i)];
-      }
-      if (et == 0) {
-        p.list_cnt[slot] = S.nbuf;
-        if (gstart >= lo) p.row_first[r] = static_cast<int>(blockIdx.x);
-        if (gstart + nt <= hi) p.row_last[r] = static_cast<int>(blockIdx.x);
-        if (lo == 0) p.total_out[0] = total;
+#pragma unroll 4
+      for (int b = et; b < kHistBins; b += kEpi) {
+        const uint32_t c = lhist[b];
+        if (c) {
+          atomicAdd(gh + b, c);
+          lhist[b] = 0;
+        }
       }
       epi_sync();
-      S.nbuf = 0;
-      S.theta = 0;
-      S.tkeep = 0;
-      S.since_flush = 0;
-      S.flushes = 0;
     };
 
     for (int i = 0; i < n_items; ++i) {
       if (w.g != cur_g) {
         if constexpr (SELECT) {
-          if (cur_g >= 0) finish_row(cur_g, cur_gstart, cur_nt);
+          if (cur_g >= 0) flush_hist(cur_g);
         }
         epi_sync();
         for (int j = et; j < C::kN; j += kEpi) {
@@ -610,8 +367,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         epi_sync();
         cur_g = w.g;
-        cur_nt = w.nt;
-        cur_gstart = w.gstart;
       }
       if (!mbar_wait(&accfull[acc], acc_ph, abort_flag)) {
         aborted = true;
@@ -629,10 +384,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                static_cast<uint32_t>(acc * C::kN + j * 32),
                            v);
         const float* wj = w_smem + j * kIdxHeads;
-        float s = 0.f;
+        // four interleaved partial sums over the heads (short dependency chains)
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int h = 0; h < kIdxHeads; ++h) s = __fmaf_rn(wj[h], v[h] > 0.f ? v[h] : 0.f, s);
-        sc[j] = s;
+        for (int h = 0; h < kIdxHeads; ++h)
+          s4[h & 3] = __fmaf_rn(wj[h], v[h] > 0.f ? v[h] : 0.f, s4[h & 3]);
+        sc[j] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
       tc_fence_before();
       __syncwarp();
@@ -640,28 +397,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_ph ^= 1;
 
-      if constexpr (SELECT) {
-        const bool valid = blk < nb_smem[0];
-        const uint32_t key = order_key(sc[0]);
-        if (valid) atomicAdd(&S.lhist[key >> kHistShift], 1u);
-        sel_append(S, valid && key >= S.theta, key, static_cast<int32_t>(blk), quarter, lane);
-        if (++S.since_flush >= (S.flushes >= 2 ? kFlushTiles : kEarlyFlush)) {
-          sel_flush(S, p.ghist + static_cast<int64_t>(w.g) * kHistBins, et, S.snap_pending);
-          ++S.flushes;
-        }
-        if (S.nbuf > kBufCap - kEpi) sel_compact(S, et);
-      } else {
 #pragma unroll 1
-        for (int j = 0; j < NQ; ++j) {
-          const int r = w.g * NQ + j;
-          if (r >= p.rows) break;
-          if (blk < nb_smem[j]) p.scores[static_cast<int64_t>(r) * p.score_stride + blk] = sc[j];
+      for (int j = 0; j < NQ; ++j) {
+        const int r = w.g * NQ + j;
+        if (r >= p.rows) break;
+        if (blk < nb_smem[j]) {
+          p.scores[static_cast<int64_t>(r) * p.score_stride + blk] = sc[j];
+          if constexpr (SELECT) atomicAdd(&lhist[order_key(sc[j]) >> kHistShift], 1u);
         }
       }
       w.advance(p);
     }
     if constexpr (SELECT) {
-      if (!aborted && cur_g >= 0) finish_row(cur_g, cur_gstart, cur_nt);
+      if (!aborted && cur_g >= 0) flush_hist(cur_g);
     }
   }
 
@@ -714,12 +462,6 @@ cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
   p.groups = (a.rows + NQ - 1) / NQ;
   p.shared_keys = a.key_batches == 1 ? 1 : 0;
   p.ghist = a.sel_ghist;
-  p.list_key = a.sel_list_key;
-  p.list_idx = a.sel_list_idx;
-  p.list_cnt = a.sel_list_cnt;
-  p.row_first = a.sel_row_first;
-  p.row_last = a.sel_row_last;
-  p.total_out = a.sel_total;
   const int grid = score_grid(a.nq, a.rows, a.max_len, a.num_sms);
   if (grid == 0) return cudaSuccess;
   k_index_score<NQ, SELECT><<<grid, kThreads, C::kSmem, stream>>>(map_k, map_q, p);

@@ -43,8 +43,7 @@ __global__ void __launch_bounds__(kPoolThreads)
                   __nv_bfloat16* __restrict__ pooled, int64_t cap_blk,
                   const int64_t* __restrict__ len_dev, int64_t len_host, int64_t max_len,
                   int64_t* __restrict__ nvis_out, uint32_t* __restrict__ init_hist,
-                  int32_t* __restrict__ init_first, int32_t* __restrict__ init_last,
-                  int32_t* __restrict__ init_idx, int32_t* __restrict__ init_cnt) {
+                  int32_t* __restrict__ init_done) {
   const int b = blockIdx.y;
   int64_t len = len_dev ? len_dev[b] : len_host;
   // Clamp so that every access stays inside the caches whatever the device
@@ -57,13 +56,7 @@ __global__ void __launch_bounds__(kPoolThreads)
     if (init_hist) {
       for (int i = threadIdx.x; i < kSelHistBins; i += kPoolThreads)
         init_hist[static_cast<int64_t>(b) * kSelHistBins + i] = 0u;
-      for (int i = threadIdx.x; i < kTopK; i += kPoolThreads)
-        init_idx[static_cast<int64_t>(b) * kTopK + i] = -1;
-      if (threadIdx.x == 0) {
-        init_first[b] = -1;
-        init_last[b] = -1;
-        init_cnt[b] = 0;
-      }
+      if (threadIdx.x == 0) init_done[b] = 0;
     }
   }
   if (n_new <= 0) return;
@@ -128,8 +121,7 @@ cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream) {
   k_pool_append<<<grid, kPoolThreads, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(a.raw_k), a.n_new, a.w[0], a.w[1], a.w[2], a.w[3],
       static_cast<__nv_bfloat16*>(a.tail), static_cast<__nv_bfloat16*>(a.pooled_k), a.cap_blk,
-      a.len_dev, a.len_host, a.max_len, a.nvis_out, a.init_hist, a.init_first, a.init_last,
-      a.init_idx, a.init_cnt);
+      a.len_dev, a.len_host, a.max_len, a.nvis_out, a.init_hist, a.init_done);
   count_launches(1);
   return cudaGetLastError();
 }

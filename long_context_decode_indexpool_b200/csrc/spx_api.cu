@@ -135,22 +135,27 @@ FusedLayout fused_layout(int rows, int heads, int64_t max_len) {
   return L;
 }
 
-// Workspace of the fused decode call (selection fused into the scoring kernel):
-//   n_vis [B] | idx [B,512] | count [B] | hist [B,2048] | first, last [B]
-//   | total tiles | list keys, list ids [grid+B, 512] | list counts [grid+B]
-//   | attention scratch
+// Workspace of the fused decode call:
+//   n_vis [B] | idx [B,512] | count [B] | key histogram [B,2048] | done [B]
+//   | scores [B, stride] | list keys, list ids [B*nchunk, 512]
+//   | list counts [B*nchunk] | attention scratch
 struct DecodeLayout {
-  size_t nvis, idx, count, hist, first, last, tiles, lkey, lidx, lcnt, attn, total;
-  int grid;
+  size_t nvis, idx, count, hist, done, scores, lkey, lidx, lcnt, attn, total;
+  int64_t stride;  // scores per row, a multiple of 4
+  int nchunk;
   AttnPlan ap;
 };
 
 DecodeLayout decode_layout(int B, int heads, int64_t max_len) {
   DecodeLayout L{};
   const int sms = device_sm_count();
-  L.grid = score_grid(1, B, max_len, sms);
+  const int64_t max_blk = max_len / kPool;
+  L.stride = (max_blk + 3) / 4 * 4;
+  if (L.stride < 4) L.stride = 4;
+  L.nchunk = static_cast<int>((max_blk + kSelChunk - 1) / kSelChunk);
+  if (L.nchunk < 1) L.nchunk = 1;
   L.ap = plan_attn(B, heads, max_len, sms);
-  const size_t slots = static_cast<size_t>(L.grid) + B;
+  const size_t lists = static_cast<size_t>(B) * L.nchunk;
   size_t o = 0;
   L.nvis = o;
   o += up(static_cast<size_t>(B) * 8);
@@ -160,18 +165,16 @@ DecodeLayout decode_layout(int B, int heads, int64_t max_len) {
   o += up(static_cast<size_t>(B) * 4);
   L.hist = o;
   o += up(static_cast<size_t>(B) * kSelHistBins * 4);
-  L.first = o;
+  L.done = o;
   o += up(static_cast<size_t>(B) * 4);
-  L.last = o;
-  o += up(static_cast<size_t>(B) * 4);
-  L.tiles = o;
-  o += up(8);
+  L.scores = o;
+  o += up(static_cast<size_t>(B) * L.stride * 4);
   L.lkey = o;
-  o += up(slots * kTopK * 4);
+  o += up(lists * kTopK * 4);
   L.lidx = o;
-  o += up(slots * kTopK * 4);
+  o += up(lists * kTopK * 4);
   L.lcnt = o;
-  o += up(slots * 4);
+  o += up(lists * 4);
   L.attn = o;
   o += up(L.ap.ws_bytes);
   L.total = o;
@@ -400,6 +403,7 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
       (lse && !al4(lse)) || (idx_out && !al4(idx_out)) || (count_out && !al4(count_out)))
     return SPX_ERR_INVALID_ARG;
   const DecodeLayout L = decode_layout(B, d->heads, max_len);
+  if (L.nchunk > kMaxSelChunks) return SPX_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < L.total || !al16(ws)) return SPX_ERR_WORKSPACE;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -408,9 +412,8 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + L.idx);
   int32_t* count = count_out ? count_out : reinterpret_cast<int32_t*>(base + L.count);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.hist);
-  int32_t* row_first = reinterpret_cast<int32_t*>(base + L.first);
-  int32_t* row_last = reinterpret_cast<int32_t*>(base + L.last);
-  int64_t* tiles = reinterpret_cast<int64_t*>(base + L.tiles);
+  int32_t* done = reinterpret_cast<int32_t*>(base + L.done);
+  float* scores = reinterpret_cast<float*>(base + L.scores);
 
   // 1. append (or just copy the lengths) -> n_vis; reset the selection state
   PoolAppendArgs pa{};
@@ -426,14 +429,11 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   pa.max_len = max_len;
   pa.nvis_out = n_vis;
   pa.init_hist = hist;
-  pa.init_first = row_first;
-  pa.init_last = row_last;
-  pa.init_idx = idx;
-  pa.init_cnt = count;
+  pa.init_done = done;
   cudaError_t e = launch_pool_append(pa, s);
   if (e != cudaSuccess) return SPX_ERR_CUDA;
 
-  // 2+3. indexer scores with the top-k selection fused in
+  // 2. indexer scores and their key histogram
   if (timing && timing->score_begin &&
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_begin), s) != cudaSuccess)
     return SPX_ERR_CUDA;
@@ -447,33 +447,30 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   sa.cap_blk = cap_blk;
   sa.n_vis = n_vis;
   sa.max_len = max_len;
-  sa.scores = nullptr;
-  sa.score_stride = 0;
+  sa.scores = scores;
+  sa.score_stride = L.stride;
   sa.num_sms = device_sm_count();
   sa.sel_ghist = hist;
-  sa.sel_list_key = reinterpret_cast<uint32_t*>(base + L.lkey);
-  sa.sel_list_idx = reinterpret_cast<int32_t*>(base + L.lidx);
-  sa.sel_list_cnt = reinterpret_cast<int32_t*>(base + L.lcnt);
-  sa.sel_row_first = row_first;
-  sa.sel_row_last = row_last;
-  sa.sel_total = tiles;
   if ((e = launch_index_score(sa, s)) != cudaSuccess) return SPX_ERR_CUDA;
   if (timing && timing->score_end &&
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
     return SPX_ERR_CUDA;
-  SelectMergeArgs ma{};
+  // 3. top-512 blocks per row
+  SelectBlocksArgs ma{};
   ma.rows = B;
-  ma.grid = L.grid;
+  ma.scores = scores;
+  ma.score_stride = L.stride;
+  ma.n_vis = n_vis;
+  ma.max_len = max_len;
   ma.ghist = hist;
-  ma.list_key = sa.sel_list_key;
-  ma.list_idx = sa.sel_list_idx;
-  ma.list_cnt = sa.sel_list_cnt;
-  ma.row_first = row_first;
-  ma.row_last = row_last;
-  ma.total = tiles;
+  ma.nchunk = L.nchunk;
+  ma.list_key = reinterpret_cast<uint32_t*>(base + L.lkey);
+  ma.list_idx = reinterpret_cast<int32_t*>(base + L.lidx);
+  ma.list_cnt = reinterpret_cast<int32_t*>(base + L.lcnt);
+  ma.done = done;
   ma.out_idx = idx;
   ma.out_cnt = count;
-  if ((e = launch_select_merge(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
+  if ((e = launch_select_blocks(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
 
   // 4. attention
   AttnArgs aa{};

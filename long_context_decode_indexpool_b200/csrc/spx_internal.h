@@ -30,13 +30,10 @@ struct PoolAppendArgs {
   int64_t len_host;
   int64_t max_len;
   int64_t* nvis_out;  // optional: receives len + n_new per sequence
-  // optional per-sequence initialisation of the fused selection state:
-  // hist[b][..] = 0, first[b] = last[b] = -1, idx[b][0..512) = -1, cnt[b] = 0
+  // optional per-sequence initialisation of the decode selection state:
+  // hist[b][..] = 0, done[b] = 0
   uint32_t* init_hist;
-  int32_t* init_first;
-  int32_t* init_last;
-  int32_t* init_idx;
-  int32_t* init_cnt;
+  int32_t* init_done;
 };
 cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_nvis(int64_t* n_vis, int T, int64_t pos0, cudaStream_t stream);
@@ -53,42 +50,42 @@ struct ScoreArgs {
   int64_t cap_blk;
   const int64_t* n_vis;  // [rows]
   int64_t max_len;
-  float* scores;        // written unless the selection is fused
+  float* scores;        // [rows, score_stride]
   int64_t score_stride;
   int num_sms;
-  // fused top-k, first stage (decode, nq == 1): set sel_ghist to enable;
-  // see index_score.cu.  ghist must be zero and row_first/row_last -1 on
-  // entry.  The second stage is launch_select_merge.
-  uint32_t* sel_ghist;     // [rows, kSelHistBins]
-  uint32_t* sel_list_key;  // [score_grid + rows, 512]
-  int32_t* sel_list_idx;   // [score_grid + rows, 512]
-  int32_t* sel_list_cnt;   // [score_grid + rows]
-  int32_t* sel_row_first;  // [rows]
-  int32_t* sel_row_last;   // [rows]
-  int64_t* sel_total;      // [1]
+  // decode (nq == 1): when set, the keys of the scores are also counted in
+  // a per-row histogram of their top 11 bits (zero on entry), the input of
+  // launch_select_blocks.
+  uint32_t* sel_ghist;  // [rows, kSelHistBins]
 };
 constexpr int kSelHistBins = 2048;
 // Grid size of the scoring kernel for the given call shape.
 int score_grid(int nq, int rows, int64_t max_len, int num_sms);
 cudaError_t launch_index_score(const ScoreArgs& a, cudaStream_t stream);
 
-// Second stage of the fused decode selection: per row, the complete
-// histogram gives an exact lower bound; the CTA lists are filtered and merged
-// into the row's 512 block ids (ascending, -1 padded) and count.
-struct SelectMergeArgs {
+// Decode top-k from scores and their complete key histogram: per row, the
+// histogram locates the bin of the 512th-largest key; chunks of the row keep
+// their blocks at or above it (at most 512 each, index order) and the last
+// chunk to finish selects the row's 512 block ids (ascending, -1 padded) and
+// count.  done[] must be zero on entry and is zero again on exit.
+constexpr int kSelChunk = 8192;     // scores per selection CTA
+constexpr int kMaxSelChunks = 512;  // chunks per row (rows up to 16M tokens)
+struct SelectBlocksArgs {
   int rows;
-  int grid;  // grid of the scoring launch
-  const uint32_t* ghist;
-  const uint32_t* list_key;
-  const int32_t* list_idx;
-  const int32_t* list_cnt;
-  const int32_t* row_first;
-  const int32_t* row_last;
-  const int64_t* total;
+  const float* scores;
+  int64_t score_stride;
+  const int64_t* n_vis;
+  int64_t max_len;
+  const uint32_t* ghist;  // [rows, kSelHistBins]
+  int nchunk;             // ceil(max_len / kPool / kSelChunk) <= 512
+  uint32_t* list_key;     // [rows * nchunk, 512]
+  int32_t* list_idx;      // [rows * nchunk, 512]
+  int32_t* list_cnt;      // [rows * nchunk]
+  int32_t* done;          // [rows]
   int32_t* out_idx;
   int32_t* out_cnt;
 };
-cudaError_t launch_select_merge(const SelectMergeArgs& a, cudaStream_t stream);
+cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream);
 
 // Top-k blocks.
 struct TopkPlan {

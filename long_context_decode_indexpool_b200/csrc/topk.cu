@@ -131,12 +131,8 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// Second stage of the decode selection fused into the scoring kernel: one
-// CTA per row.  The row's histogram is complete here (the scoring launch has
-// finished), so the bin holding the 512th-largest key gives an exact lower
-// bound; only list entries at or above it take part (index order = CTA
-// order).  Every entry in a bin above the cut bin is selected; the best of
-// the cut bin (ties: lower block) complete the 512.
+// Decode selection (k_select_blocks below): keys are counted by their top 11
+// bits (sign, exponent, 2 mantissa bits) in 2048 bins.
 constexpr int kSelBins = kSelHistBins;
 constexpr int kSelShift = 32 - 11;
 constexpr int kMergeCap = kThreads * 16;  // candidates held at once (16 per thread)
@@ -148,10 +144,6 @@ struct MergeSmem {
   int dig[3], abv[3];
   uint32_t kmin, kmax;
 };
-
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
 
 // The row's result from the n buffered (key, block) pairs, in block order;
 // entries below lo_key are not candidates.  Every candidate above the cut
@@ -275,30 +267,46 @@ __device__ __noinline__ void merge_final(const uint32_t* bk, const int32_t* bi, 
   if (tid == 0) *cnt_out = n;
 }
 
+// Decode selection from the row's scores and its complete key histogram.
+// Grid (nchunk, rows), one CTA per chunk of kSelChunk scores (16 per thread):
+//   1. the histogram gives the bin of the row's 512th-largest key (every CTA
+//      of the row finds the same bin);
+//   2. the chunk's keys at or above that bin's lower edge are candidates; an
+//      exact top-512 of them (ties: lower block, the chunk's index order)
+//      becomes the chunk's list;
+//   3. the last CTA of the row to finish (a counter) gathers the lists (CTA
+//      order = index order) and makes the final choice.
+// The union of per-chunk exact top-512 lists holds the row's top-512, so the
+// result is exact.
 __global__ void __launch_bounds__(kThreads)
-    k_select_merge(const uint32_t* __restrict__ ghist, const uint32_t* __restrict__ list_key,
-                   const int32_t* __restrict__ list_idx, const int32_t* __restrict__ list_cnt,
-                   const int32_t* __restrict__ row_first, const int32_t* __restrict__ row_last,
-                   const int64_t* __restrict__ total_p, int G, int32_t* __restrict__ out_idx,
-                   int32_t* __restrict__ out_cnt) {
+    k_select_blocks(const float* __restrict__ scores, int64_t score_stride,
+                    const int64_t* __restrict__ n_vis, int64_t max_len,
+                    const uint32_t* __restrict__ ghist, int nchunk, uint32_t* __restrict__ list_key,
+                    int32_t* __restrict__ list_idx, int32_t* __restrict__ list_cnt,
+                    int32_t* __restrict__ done, int32_t* __restrict__ out_idx,
+                    int32_t* __restrict__ out_cnt) {
   extern __shared__ uint8_t dyn[];
   uint32_t* buf_key = reinterpret_cast<uint32_t*>(dyn);
   int32_t* buf_idx = reinterpret_cast<int32_t*>(buf_key + pad32(kMergeCap));
   __shared__ SelectSmem sm;
   __shared__ MergeSmem ms;
   __shared__ int seg_off[kThreads + 1];
-  __shared__ int s_bin, s_above;
-  const int r = blockIdx.x, tid = threadIdx.x;
-  // Loads that do not depend on the row's CTA range go out together: the
-  // histogram (thread t owns bins kSelBins-1-4t .. kSelBins-4-4t), the range,
-  // the tile total and the list count of CTA t (slot t + r).
+  __shared__ int s_bin, s_above, s_last;
+  const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x;
+  // Loads first: the histogram (thread t owns bins kSelBins-1-4t ..
+  // kSelBins-4-4t) and this thread's 16 scores.
   const uint32_t* h = ghist + static_cast<int64_t>(r) * kSelBins;
   int hc[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) hc[j] = static_cast<int>(h[kSelBins - 1 - (tid * 4 + j)]);
-  const int c_first = row_first[r], c_last = row_last[r];
-  const int64_t total = *total_p;
-  const int m_pre = tid < G ? list_cnt[static_cast<int64_t>(tid) + r] : 0;
+  for (int j = 0; j < 4; ++j) hc[j] = static_cast<int>(__ldcg(h + kSelBins - 1 - (tid * 4 + j)));
+  const int64_t nblk = clamp_blocks(n_vis, r, max_len);
+  const int64_t b0 = static_cast<int64_t>(c) * kSelChunk + tid * 16;
+  const float* row = scores + static_cast<int64_t>(r) * score_stride;
+  float4 sv[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)  // rows are padded to a multiple of 4 scores
+    sv[q] = b0 + 4 * q < nblk ? __ldcg(reinterpret_cast<const float4*>(row + b0 + 4 * q))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
   for (int b = tid; b < 3 * 128; b += kThreads) (&ms.rh[0][0])[b] = 0;
   if (tid < 3) {
     ms.dig[tid] = 0;
@@ -310,11 +318,8 @@ __global__ void __launch_bounds__(kThreads)
     ms.kmin = 0xFFFFFFFFu;
     ms.kmax = 0;
   }
-  if (c_first < 0 || c_last < c_first) return;  // no tile: outputs stay as initialised
-  const int nseg = c_last - c_first + 1;
-  auto has_tiles = [&](int c) { return (total * (c + 1) / G) > (total * c / G); };
 
-  // 1. exact lower bound from the complete histogram
+  // 1. the cut bin from the complete histogram
   {
     int sum = hc[0] + hc[1] + hc[2] + hc[3];
     int tot;
@@ -333,115 +338,130 @@ __global__ void __launch_bounds__(kThreads)
   }
   const int cut_bin = s_bin, above = s_above;
   const uint32_t theta = cut_bin < 0 ? 0u : static_cast<uint32_t>(cut_bin) << kSelShift;
-  int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
 
-  // 2. list offsets, in CTA order (the scoring grid fits one CTA of threads)
-  int mtot = 0;
-  if (G <= kThreads) {  // uniform
-    const bool mine = tid >= c_first && tid <= c_last && has_tiles(tid);
-    const int off = group_excl_scan<kThreads, 0>(mine ? m_pre : 0, tid, sm.scan, &mtot);
-    if (tid >= c_first && tid <= c_last) seg_off[tid - c_first] = off;
-    if (tid == 0) seg_off[nseg] = mtot;
-    __syncthreads();
+  // 2. this chunk's list
+  {
+    uint32_t key[16];
+    uint32_t valid = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float4 v = sv[i >> 2];
+      const float f = (i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w;
+      key[i] = order_key(f);
+      if (b0 + i < nblk && key[i] >= theta) valid |= 1u << i;
+    }
+    const int64_t slot = static_cast<int64_t>(r) * nchunk + c;
+    uint32_t* kd = list_key + slot * kTopK;
+    int32_t* id = list_idx + slot * kTopK;
+    uint32_t thr;
+    const int n = group_select<16, kThreads, 0>(key, valid, kTopK, tid, sm, &thr, [&](int i, int pos) {
+      kd[pos] = key[i];
+      id[pos] = static_cast<int32_t>(b0 + i);
+    });
+    if (tid == 0) list_cnt[slot] = n;
   }
-  if (G <= kThreads && mtot <= kMergeCap) {  // uniform
-    // 3. every list entry straight into the buffer (asynchronous copies)
+
+  // 3. the last CTA of the row continues
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(done + r, 1) == nchunk - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
+  const int64_t slot0 = static_cast<int64_t>(r) * nchunk;
+  const int m = tid < nchunk ? __ldcg(list_cnt + slot0 + tid) : 0;
+  int mtot;
+  const int off = group_excl_scan<kThreads, 0>(m, tid, sm.scan, &mtot);
+  if (tid < nchunk) seg_off[tid] = off;
+  if (tid == 0) seg_off[nchunk] = mtot;
+  __syncthreads();
+  if (tid == 0) done[r] = 0;  // ready for the next launch
+  if (mtot <= kMergeCap) {  // uniform: every list entry into the buffer
 #pragma unroll 1
     for (int f = tid; f < mtot; f += kThreads) {
-      int lo_s = 0, hi_s = nseg - 1;  // last segment with seg_off <= f
+      int lo_s = 0, hi_s = nchunk - 1;  // last segment with seg_off <= f
       while (lo_s < hi_s) {
         const int mid = (lo_s + hi_s + 1) >> 1;
         if (seg_off[mid] <= f) lo_s = mid; else hi_s = mid - 1;
       }
-      const int64_t e = (static_cast<int64_t>(c_first + lo_s) + r) * kTopK + (f - seg_off[lo_s]);
-      cp_async4(buf_key + pad32(f), list_key + e);
-      cp_async4(buf_idx + pad32(f), list_idx + e);
+      const int64_t e = (slot0 + lo_s) * kTopK + (f - seg_off[lo_s]);
+      buf_key[pad32(f)] = __ldcg(list_key + e);
+      buf_idx[pad32(f)] = __ldcg(list_idx + e);
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     merge_final(buf_key, buf_idx, mtot, theta, cut_bin, above, sm, ms, dst, out_cnt + r);
     return;
   }
 
-  // Long rows (more candidates than fit at once, or a wider scoring grid):
-  // gather in rounds, compacting to the best 512 when the buffer fills up.
+  // More candidates than fit at once (rows with a crowded cut bin): gather
+  // in rounds, compacting to the best 512 when the buffer fills up.
   uint32_t thr_keep = theta, thr_admit = theta;
   int nbuf = 0;
-  for (int sb = 0; sb < nseg; sb += kThreads) {
-    const int c = c_first + sb + tid;
-    const int m = (sb + tid < nseg && has_tiles(c)) ? list_cnt[static_cast<int64_t>(c) + r] : 0;
-    int stot;
-    const int moff = group_excl_scan<kThreads, 0>(m, tid, sm.scan, &stot);
-    seg_off[tid] = moff;
-    __syncthreads();
-    const int nsg = min(kThreads, nseg - sb);
-    for (int base = 0; base < stot; base += kThreads * kMergePer) {
-      uint32_t k[kMergePer];
-      int32_t ix[kMergePer];
-      int npass = 0;
-      uint32_t pass = 0;
+  for (int base = 0; base < mtot; base += kThreads * kMergePer) {
+    uint32_t k[kMergePer];
+    int32_t ix[kMergePer];
+    int npass = 0;
+    uint32_t pass = 0;
 #pragma unroll
-      for (int u = 0; u < kMergePer; ++u) {
-        const int f = base + tid * kMergePer + u;
-        k[u] = 0;
-        ix[u] = 0;
-        if (f < stot) {
-          int lo_s = 0, hi_s = nsg - 1;  // last segment with seg_off <= f
-          while (lo_s < hi_s) {
-            const int mid = (lo_s + hi_s + 1) >> 1;
-            if (seg_off[mid] <= f) lo_s = mid; else hi_s = mid - 1;
-          }
-          const int64_t sl = static_cast<int64_t>(c_first + sb + lo_s) + r;
-          const int j = f - seg_off[lo_s];
-          k[u] = list_key[sl * kTopK + j];
-          ix[u] = list_idx[sl * kTopK + j];
-          if (k[u] >= thr_admit) {
-            pass |= 1u << u;
-            ++npass;
-          }
+    for (int u = 0; u < kMergePer; ++u) {
+      const int f = base + tid * kMergePer + u;
+      k[u] = 0;
+      ix[u] = 0;
+      if (f < mtot) {
+        int lo_s = 0, hi_s = nchunk - 1;  // last segment with seg_off <= f
+        while (lo_s < hi_s) {
+          const int mid = (lo_s + hi_s + 1) >> 1;
+          if (seg_off[mid] <= f) lo_s = mid; else hi_s = mid - 1;
+        }
+        const int64_t e = (slot0 + lo_s) * kTopK + (f - seg_off[lo_s]);
+        k[u] = __ldcg(list_key + e);
+        ix[u] = __ldcg(list_idx + e);
+        if (k[u] >= thr_admit) {
+          pass |= 1u << u;
+          ++npass;
         }
       }
-      int ptot;
-      int pos = nbuf + group_excl_scan<kThreads, 0>(npass, tid, sm.scan, &ptot);
+    }
+    int ptot;
+    int pos = nbuf + group_excl_scan<kThreads, 0>(npass, tid, sm.scan, &ptot);
 #pragma unroll
-      for (int u = 0; u < kMergePer; ++u) {
-        if ((pass >> u) & 1u) {
-          buf_key[pad32(pos)] = k[u];
-          buf_idx[pad32(pos)] = ix[u];
-          ++pos;
-        }
+    for (int u = 0; u < kMergePer; ++u) {
+      if ((pass >> u) & 1u) {
+        buf_key[pad32(pos)] = k[u];
+        buf_idx[pad32(pos)] = ix[u];
+        ++pos;
       }
-      nbuf += ptot;
-      if (nbuf > kMergeCap - kThreads * kMergePer) {  // compact in place
-        __syncthreads();
-        uint32_t kk[16];
-        int32_t ii[16];
-        uint32_t valid = 0;
+    }
+    nbuf += ptot;
+    if (nbuf > kMergeCap - kThreads * kMergePer) {  // compact in place
+      __syncthreads();
+      uint32_t kk[16];
+      int32_t ii[16];
+      uint32_t valid = 0;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int q = tid * 16 + i;
-          kk[i] = 0;
-          ii[i] = 0;
-          if (q < nbuf) {
-            kk[i] = buf_key[pad32(q)];
-            ii[i] = buf_idx[pad32(q)];
-            if (kk[i] >= thr_keep) valid |= 1u << i;
-          }
-        }
-        __syncthreads();
-        uint32_t thr;
-        nbuf = group_select<16, kThreads, 0>(kk, valid, kTopK, tid, sm, &thr, [&](int i, int p) {
-          buf_key[pad32(p)] = kk[i];
-          buf_idx[pad32(p)] = ii[i];
-        });
-        if (thr != 0) {
-          // a later entry equal to thr has a higher block id: it loses
-          const uint32_t t1 = thr == 0xFFFFFFFFu ? thr : thr + 1;
-          thr_admit = t1 > thr_admit ? t1 : thr_admit;
-          thr_keep = thr > thr_keep ? thr : thr_keep;
+      for (int i = 0; i < 16; ++i) {
+        const int q = tid * 16 + i;
+        kk[i] = 0;
+        ii[i] = 0;
+        if (q < nbuf) {
+          kk[i] = buf_key[pad32(q)];
+          ii[i] = buf_idx[pad32(q)];
+          if (kk[i] >= thr_keep) valid |= 1u << i;
         }
       }
       __syncthreads();
+      uint32_t thr;
+      nbuf = group_select<16, kThreads, 0>(kk, valid, kTopK, tid, sm, &thr, [&](int i, int p) {
+        buf_key[pad32(p)] = kk[i];
+        buf_idx[pad32(p)] = ii[i];
+      });
+      if (thr != 0) {
+        // a later entry equal to thr has a higher block id: it loses
+        const uint32_t t1 = thr == 0xFFFFFFFFu ? thr : thr + 1;
+        thr_admit = t1 > thr_admit ? t1 : thr_admit;
+        thr_keep = thr > thr_keep ? thr : thr_keep;
+      }
     }
     __syncthreads();
   }
@@ -461,21 +481,22 @@ cudaError_t launch_merge_e(dim3 grid, cudaStream_t s, const uint32_t* ik, const 
 
 }  // namespace
 
-cudaError_t launch_select_merge(const SelectMergeArgs& a, cudaStream_t stream) {
-  if (a.rows == 0) return cudaSuccess;
+cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream) {
+  if (a.rows == 0 || a.nchunk == 0) return cudaSuccess;
+  if (a.nchunk > kThreads || (a.score_stride & 3) != 0) return cudaErrorInvalidValue;
   constexpr int kSmem = pad32(kMergeCap) * 8;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(k_select_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        cudaFuncSetAttribute(k_select_blocks, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  k_select_merge<<<a.rows, kThreads, kSmem, stream>>>(a.ghist, a.list_key, a.list_idx, a.list_cnt,
-                                                      a.row_first, a.row_last, a.total, a.grid,
-                                                      a.out_idx, a.out_cnt);
+  k_select_blocks<<<dim3(a.nchunk, a.rows), kThreads, kSmem, stream>>>(
+      a.scores, a.score_stride, a.n_vis, a.max_len, a.ghist, a.nchunk, a.list_key, a.list_idx,
+      a.list_cnt, a.done, a.out_idx, a.out_cnt);
   count_launches(1);
   return cudaGetLastError();
 }
