@@ -41,6 +41,7 @@
 #include "select.cuh"
 #include "spx_device.cuh"
 #include "spx_internal.h"
+#include "spx_launch.cuh"
 
 namespace spx {
 
@@ -165,6 +166,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int s_g0, s_t0;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    prefetch_tensormap(&map_k);
+    prefetch_tensormap(&map_q);
+  }
+  pdl_trigger();  // the next kernel's CTAs may be scheduled as SMs free up
+  pdl_wait();     // lengths, keys and the histogram come from the previous kernel
 
   // ---- locate this CTA's contiguous range of work items -------------------
   int64_t total = 0;
@@ -225,8 +232,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ======================= TMA producer =================================
     if (lane == 0) {
-      prefetch_tensormap(&map_k);
-      prefetch_tensormap(&map_q);
       // per-row keys are read once (decode); keys shared by every query
       // group (prefill) are re-read from L2
       const uint64_t stream_pol = p.shared_keys ? l2_evict_normal_policy() : l2_evict_first_policy();
@@ -464,8 +469,10 @@ cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
   p.ghist = a.sel_ghist;
   const int grid = score_grid(a.nq, a.rows, a.max_len, a.num_sms);
   if (grid == 0) return cudaSuccess;
-  k_index_score<NQ, SELECT><<<grid, kThreads, C::kSmem, stream>>>(map_k, map_q, p);
+  cudaError_t e = launch_ex(k_index_score<NQ, SELECT>, dim3(grid), dim3(kThreads), C::kSmem,
+                            stream, a.pdl, 1, map_k, map_q, p);
   count_launches(1);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

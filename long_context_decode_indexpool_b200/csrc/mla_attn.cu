@@ -43,6 +43,7 @@
 // the bf16 output and the log-sum-exp.  No second kernel runs.
 #include "spx_device.cuh"
 #include "spx_internal.h"
+#include "spx_launch.cuh"
 
 namespace spx {
 
@@ -198,44 +199,47 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h0 = hg * kHG;
   const int n_cl = p.nsplit;
-  const RowInfo ri = row_info(p, r);
-  const int j_begin = split * p.split_tokens;
-  const int j_end = split == n_cl - 1 ? ri.S : min(ri.S, j_begin + p.split_tokens);
-  const int nlist = j_end > j_begin ? j_end - j_begin : 0;
-  const int ntiles = (nlist + kTT - 1) / kTT;
   // head of this thread; lanes i and 16+i of a warp share it
   const int hloc = warp * 16 + (lane & 15);
   const int half = lane >> 4;  // 0: tokens 0-31 / dims 0-255, 1: tokens 32-63 / dims 256-511
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t q_u = smem_u32(q_s), kv_u = smem_u32(kv_s), p_u = smem_u32(p_s);
 
+  // ---- set-up that needs nothing from the previous kernel -------------------
   if (tid == 0) {
     mbar_init(bar_qk, 1);
     mbar_init(bar_pv, 1);
     fence_mbar_init();
   }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  // Q [64 heads x 512] (heads beyond H zero-filled): part of the first group
+  {
+    const __nv_bfloat16* qr = p.q + (static_cast<int64_t>(r) * p.heads) * kLatent;
+#pragma unroll 4
+    for (int c = tid; c < kHG * 64; c += kThreads) {
+      const int h = c >> 6, piece = c & 63;
+      const bool ok = h0 + h < p.heads;
+      cp_async16(q_u + sw_off(h, piece),
+                 qr + static_cast<int64_t>(ok ? h0 + h : 0) * kLatent + piece * 8, ok);
+    }
+  }
+  pdl_trigger();
+  pdl_wait();  // the selected blocks come from the previous kernel
+
+  const RowInfo ri = row_info(p, r);
+  const int j_begin = split * p.split_tokens;
+  const int j_end = split == n_cl - 1 ? ri.S : min(ri.S, j_begin + p.split_tokens);
+  const int nlist = j_end > j_begin ? j_end - j_begin : 0;
+  const int ntiles = (nlist + kTT - 1) / kTT;
   float m_run = -INFINITY, l_run = 0.f;  // of head hloc (both threads)
   bool ok_all = true;
   uint32_t tmem = 0;
 
   if (ntiles > 0) {  // uniform
-    if (warp == 0) {
-      tmem_alloc(tmem_holder, 512);
-      tmem_relinquish();
-    }
     const __nv_bfloat16* lat = p.latent + static_cast<int64_t>(r) * p.seq_stride;
-    const uint32_t q_u = smem_u32(q_s), kv_u = smem_u32(kv_s), p_u = smem_u32(p_s);
-
-    // Q [64 heads x 512] (heads beyond H zero-filled): part of the first group
-    {
-      const __nv_bfloat16* qr = p.q + (static_cast<int64_t>(r) * p.heads) * kLatent;
-#pragma unroll 4
-      for (int c = tid; c < kHG * 64; c += kThreads) {
-        const int h = c >> 6, piece = c & 63;
-        const bool ok = h0 + h < p.heads;
-        cp_async16(q_u + sw_off(h, piece),
-                   qr + static_cast<int64_t>(ok ? h0 + h : 0) * kLatent + piece * 8, ok);
-      }
-    }
     // every token position of the split, once, with a validity bit per token
 #pragma unroll 1
     for (int i0 = 0; i0 < ntiles * kTT; i0 += kThreads) {
@@ -414,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   }
 
   // ---- output ----------------------------------------------------------------
+  cp_async_wait<0>();  // (a split without tokens still has Q copies in flight)
   const bool have = ntiles > 0 && ok_all && l_run > 0.f;
   const int64_t unit = static_cast<int64_t>(r) * gridDim.z + hg;  // (row, head group)
   if (n_cl == 1) {
@@ -537,12 +542,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     }
   }
   if (!ok_all && tid == 0) atomicExch(&g_device_error, kErrWaitTimeout);
-  if (ntiles > 0) {
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 512);
-  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(*tmem_holder, 512);
 }
 
 // Largest cluster size n <= want (a power of two) for which the device can
@@ -661,19 +664,8 @@ cudaError_t launch_attn(const AttnPlan& pl0, const AttnArgs& a, cudaStream_t str
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
                                          ((units_n * kLatent * 4 + 255) & ~static_cast<size_t>(255)));
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.nsplit, pl.rows, pl.groups);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = pl.nsplit;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, k_sparse_attn, p);
+  cudaError_t e = launch_ex(k_sparse_attn, dim3(pl.nsplit, pl.rows, pl.groups), dim3(kThreads),
+                            kSmemBytes, stream, a.pdl, pl.nsplit, p);
   count_launches(1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -15,6 +15,7 @@
 // thread.  Only the first block of an append can read the tail, and only CTA
 // x = 0 handles it; that CTA also writes the new tail after a barrier, so no
 // tail slot is overwritten before it has been read.
+#include "spx_device.cuh"
 #include "spx_internal.h"
 
 namespace spx {
@@ -44,6 +45,7 @@ __global__ void __launch_bounds__(kPoolThreads)
                   const int64_t* __restrict__ len_dev, int64_t len_host, int64_t max_len,
                   int64_t* __restrict__ nvis_out, uint32_t* __restrict__ init_hist,
                   int32_t* __restrict__ init_done) {
+  pdl_trigger();
   const int b = blockIdx.y;
   int64_t len = len_dev ? len_dev[b] : len_host;
   // Clamp so that every access stays inside the caches whatever the device

@@ -451,6 +451,10 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   sa.score_stride = L.stride;
   sa.num_sms = device_sm_count();
   sa.sel_ghist = hist;
+  // Each kernel of the chain may start while its predecessor finishes (its
+  // set-up overlaps; it waits before reading the predecessor's output),
+  // except across a timing event.
+  sa.pdl = !(timing && timing->score_begin);
   if ((e = launch_index_score(sa, s)) != cudaSuccess) return SPX_ERR_CUDA;
   if (timing && timing->score_end &&
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
@@ -470,6 +474,7 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   ma.done = done;
   ma.out_idx = idx;
   ma.out_cnt = count;
+  ma.pdl = !(timing && timing->score_end);
   if ((e = launch_select_blocks(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
 
   // 4. attention
@@ -486,6 +491,7 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   aa.out = out;
   aa.lse = lse;
   aa.ws = base + L.attn;
+  aa.pdl = true;
   return cuda_status(launch_attn(L.ap, aa, s));
 }
 

@@ -98,6 +98,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Programmatic dependent launch: wait for the previous kernel of the stream
+// (a no-op when the launch did not allow an early start), and let the next
+// kernel of the stream start early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // L2 policy for data read once: its lines are the first to be replaced, so
 // a stream larger than L2 does not push out what other kernels reuse
 // (their code, lists, partial results).

@@ -57,6 +57,7 @@ struct ScoreArgs {
   // a per-row histogram of their top 11 bits (zero on entry), the input of
   // launch_select_blocks.
   uint32_t* sel_ghist;  // [rows, kSelHistBins]
+  bool pdl;             // may start while the previous kernel finishes
 };
 constexpr int kSelHistBins = 2048;
 // Grid size of the scoring kernel for the given call shape.
@@ -84,6 +85,7 @@ struct SelectBlocksArgs {
   int32_t* done;          // [rows]
   int32_t* out_idx;
   int32_t* out_cnt;
+  bool pdl;
 };
 cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream);
 
@@ -123,6 +125,7 @@ struct AttnArgs {
   void* out;
   float* lse;
   void* ws;
+  bool pdl;
 };
 cudaError_t launch_attn(const AttnPlan& p, const AttnArgs& a, cudaStream_t stream);
 

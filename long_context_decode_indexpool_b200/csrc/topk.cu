@@ -22,6 +22,7 @@
 // strict order, so the result equals a full sort of the row.
 #include "select.cuh"
 #include "spx_internal.h"
+#include "spx_launch.cuh"
 
 namespace spx {
 
@@ -293,6 +294,8 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ int seg_off[kThreads + 1];
   __shared__ int s_bin, s_above, s_last;
   const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();  // scores and histogram come from the scoring kernel
   // Loads first: the histogram (thread t owns bins kSelBins-1-4t ..
   // kSelBins-4-4t) and this thread's 16 scores.
   const uint32_t* h = ghist + static_cast<int64_t>(r) * kSelBins;
@@ -494,10 +497,12 @@ cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream)
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  k_select_blocks<<<dim3(a.nchunk, a.rows), kThreads, kSmem, stream>>>(
-      a.scores, a.score_stride, a.n_vis, a.max_len, a.ghist, a.nchunk, a.list_key, a.list_idx,
-      a.list_cnt, a.done, a.out_idx, a.out_cnt);
+  cudaError_t e = launch_ex(k_select_blocks, dim3(a.nchunk, a.rows), dim3(kThreads), kSmem,
+                            stream, a.pdl, 1, a.scores, a.score_stride, a.n_vis, a.max_len,
+                            a.ghist, a.nchunk, a.list_key, a.list_idx, a.list_cnt, a.done,
+                            a.out_idx, a.out_cnt);
   count_launches(1);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
