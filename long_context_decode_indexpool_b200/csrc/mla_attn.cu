@@ -49,7 +49,13 @@ namespace spx {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 160;                   // 4 worker warps + 1 MMA warp
+constexpr int kWork = 128;                      // worker threads
+// named barriers (0 is __syncthreads)
+constexpr int kBarWork = 1;                     // workers only
+constexpr int kBarData0 = 2;                    // tile data ready (S buffer 0 / 1)
+constexpr int kBarData1 = 3;
+constexpr int kBarP = 4;                        // P of a tile written
 constexpr int kTT = 64;                         // tokens per tile
 constexpr int kHG = 64;                         // heads per CTA (MMA M)
 constexpr int kRegion = 64 * 128;               // [64 rows x 128 B] = 8 KiB
@@ -102,6 +108,13 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // Thread-block cluster helpers.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile(
@@ -113,6 +126,23 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
+// Bulk copies (TMA engine, no tensor map): shared -> global and
+// global -> shared (completing on an mbarrier); 16-byte aligned, sizes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t sdst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          sdst),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Byte offset of 16-byte piece `c` (0..63) of row `r` in a tile stored as 8
 // regions of [64 rows x 128 B] with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t sw_off(int r, int c) {
@@ -186,29 +216,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* q_s = sm;
-  uint8_t* kv_s = q_s + kQBytes;  // two latent tiles; afterwards the received O rows
+  uint8_t* kv_s = q_s + kQBytes;  // two latent tiles; afterwards the combine rows
   uint8_t* p_s = kv_s + 2 * kKVBytes;
   int64_t* pos_s = reinterpret_cast<int64_t*>(p_s + kPBytes);     // [kPosCap]
   uint32_t* vm_s = reinterpret_cast<uint32_t*>(pos_s + kPosCap);  // [kPosCap / 32] valid bits
-  float* ml_s = reinterpret_cast<float*>(vm_s + kPosCap / 32);    // [64][2]: (m, l) per head
-  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(ml_s + 2 * kHG);
-  uint64_t* bar_pv = bar_qk + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 3);
+  float* ml_s = reinterpret_cast<float*>(vm_s + kPosCap / 32);    // [64][2] (spare)
+  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(ml_s + 2 * kHG);  // [2]: S buffer b done
+  uint64_t* bar_pv = bar_qk + 2;
+  uint64_t* bar_red = bar_qk + 3;  // combine: rows of the other splits
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 4);
 
   const int split = blockIdx.x, r = blockIdx.y, hg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool worker = tid < kWork;  // warps 0-3; warp 4 issues the MMAs
   const int h0 = hg * kHG;
   const int n_cl = p.nsplit;
-  // head of this thread; lanes i and 16+i of a warp share it
-  const int hloc = warp * 16 + (lane & 15);
+  // head of this thread; lanes i and 16+i of a worker warp share it
+  const int hloc = (warp & 3) * 16 + (lane & 15);
   const int half = lane >> 4;  // 0: tokens 0-31 / dims 0-255, 1: tokens 32-63 / dims 256-511
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const uint32_t q_u = smem_u32(q_s), kv_u = smem_u32(kv_s), p_u = smem_u32(p_s);
 
   // ---- set-up that needs nothing from the previous kernel -------------------
   if (tid == 0) {
-    mbar_init(bar_qk, 1);
+    mbar_init(&bar_qk[0], 1);
+    mbar_init(&bar_qk[1], 1);
     mbar_init(bar_pv, 1);
+    mbar_init(bar_red, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -216,10 +250,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     tmem_relinquish();
   }
   // Q [64 heads x 512] (heads beyond H zero-filled): part of the first group
-  {
+  if (worker) {
     const __nv_bfloat16* qr = p.q + (static_cast<int64_t>(r) * p.heads) * kLatent;
 #pragma unroll 4
-    for (int c = tid; c < kHG * 64; c += kThreads) {
+    for (int c = tid; c < kHG * 64; c += kWork) {
       const int h = c >> 6, piece = c & 63;
       const bool ok = h0 + h < p.heads;
       cp_async16(q_u + sw_off(h, piece),
@@ -240,23 +274,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
 
   if (ntiles > 0) {  // uniform
     const __nv_bfloat16* lat = p.latent + static_cast<int64_t>(r) * p.seq_stride;
-    // every token position of the split, once, with a validity bit per token
-#pragma unroll 1
-    for (int i0 = 0; i0 < ntiles * kTT; i0 += kThreads) {
-      const int i = i0 + tid;
-      int64_t pos = -1;
-      if (i < nlist) pos = token_pos(p, r, ri, j_begin + i);
-      if (i < ntiles * kTT) pos_s[i] = pos;
-      const uint32_t bits = __ballot_sync(0xffffffffu, pos >= 0);
-      if (lane == 0 && i < ntiles * kTT) vm_s[i >> 5] = bits;
-    }
-    __syncthreads();
     auto gather = [&](int tile) {
       const uint32_t dst = kv_u + (tile & 1) * kKVBytes;
       const int64_t* ps = pos_s + tile * kTT;
 #pragma unroll 4
-      for (int i = 0; i < (kTT * 64) / kThreads; ++i) {
-        const int c = i * kThreads + tid;
+      for (int i = 0; i < (kTT * 64) / kWork; ++i) {
+        const int c = i * kWork + tid;
         const int t = c >> 6, piece = c & 63;
         const int64_t pos = ps[t];
         cp_async16(dst + sw_off(t, piece), lat + (pos >= 0 ? pos : 0) * kLatent + piece * 8,
@@ -264,157 +287,188 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       }
       cp_async_commit();
     };
-    gather(0);                   // group: Q + tile 0
-    if (ntiles > 1) gather(1);   // group: tile 1
+    if (worker) {
+      // every token position of the split, once, with a validity bit per token
+#pragma unroll 1
+      for (int i0 = 0; i0 < ntiles * kTT; i0 += kWork) {
+        const int i = i0 + tid;
+        int64_t pos = -1;
+        if (i < nlist) pos = token_pos(p, r, ri, j_begin + i);
+        if (i < ntiles * kTT) pos_s[i] = pos;
+        const uint32_t bits = __ballot_sync(0xffffffffu, pos >= 0);
+        if (lane == 0 && i < ntiles * kTT) vm_s[i >> 5] = bits;
+      }
+      named_sync(kBarWork, kWork);
+      gather(0);                   // group: Q + tile 0
+      if (ntiles > 1) gather(1);   // group: tile 1
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     tmem = *tmem_holder;
-    const uint32_t t_o = tmem + lane_base;  // this warp's O rows (lanes i / 16+i)
 
-    // S = Q C^T of tile t into S buffer t&1 (issued by thread 0)
-    auto issue_qk = [&](int t) {
-      tc_fence_after();
-      const uint32_t kvb = kv_u + (t & 1) * kKVBytes;
-      const uint32_t d = tmem + (16u << 16) + 256 + 64 * (t & 1);
+    if (!worker) {
+      // ======================= MMA issuer (warp 4) ===========================
+      // S = Q C^T of tile t into S buffer t&1 (TMEM lanes 16-31 of each
+      // quarter, columns 256+64b ..), once the workers report its data.
+      auto qk = [&](int t) {
+        named_sync(kBarData0 + (t & 1), kThreads);
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t kvb = kv_u + (t & 1) * kKVBytes;
+          const uint32_t d = tmem + (16u << 16) + 256 + 64 * (t & 1);
 #pragma unroll 4
-      for (int k = 0; k < kLatent / 16; ++k) {
-        const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
-        umma_bf16(d, sdesc_kmajor_sw128(q_u + off), sdesc_kmajor_sw128(kvb + off), kIdescQK,
-                  k > 0 ? 1u : 0u);
-      }
-      umma_commit(bar_qk);
-    };
-
-    int qk_next = 0;  // first tile whose logits are not yet requested
-#pragma unroll 1
-    for (int j = 0; j < ntiles; ++j) {
-      const int buf = j & 1;
-      if (qk_next == j) {  // uniform
-        // tile j's copies are done (tile 1 is still in flight during tile 0)
-        if (j == 0 && ntiles > 1) cp_async_wait<1>();
-        else cp_async_wait<0>();
-        fence_proxy_async();
-        __syncthreads();
-        if (tid == 0) issue_qk(j);
-        qk_next = j + 1;
-      }
-      {
-        volatile int no_abort = 0;
-        ok_all &= mbar_wait(bar_qk, j & 1, &no_abort);
-      }
-      tc_fence_after();
-      if (j == 0 && ntiles > 1) {
-        // tile 1 was requested with tile 0: its logits overlap this softmax
-        cp_async_wait<0>();
-        fence_proxy_async();
-        __syncthreads();
-        if (tid == 0) issue_qk(1);
-        qk_next = 2;
-      }
-      // the previous PV must be done before its buffer is refilled and before
-      // P or O are touched again
-      if (j > 0) {
-        volatile int no_abort = 0;
-        ok_all &= mbar_wait(bar_pv, (j - 1) & 1, &no_abort);
-        if (j + 1 < ntiles && qk_next == j + 1) gather(j + 1);
-      }
-
-      // ---- softmax: 32 logits of head hloc per thread ----------------------
-      float s[32];
-      {
-        // lanes 16-31 receive the 64 logits of their head; tokens 0-31 go
-        // to the partner lane (lanes 0-15 receive unused columns)
-        uint32_t a[32], b[32];
-        tmem_ld_x32_async(tmem + lane_base + 256 + 64 * buf, a);
-        tmem_ld_x32_async(tmem + lane_base + 256 + 64 * buf + 32, b);
-        tmem_ld_wait_regs<32>(a);
-        tmem_ld_wait_regs<32>(b);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const uint32_t x = __shfl_xor_sync(0xffffffffu, a[t], 16);
-          s[t] = __uint_as_float(half ? b[t] : x);
+          for (int k = 0; k < kLatent / 16; ++k) {
+            const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
+            umma_bf16(d, sdesc_kmajor_sw128(q_u + off), sdesc_kmajor_sw128(kvb + off), kIdescQK,
+                      k > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_qk[t & 1]);
         }
-      }
-      const uint32_t vm = vm_s[j * 2 + half];
-      float mx[8];
-#pragma unroll
-      for (int t = 0; t < 32; ++t) s[t] = ((vm >> t) & 1u) ? s[t] * p.scale_log2 : -INFINITY;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mx[u] = fmaxf(fmaxf(s[4 * u], s[4 * u + 1]), fmaxf(s[4 * u + 2], s[4 * u + 3]));
-      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-      float alpha = 1.f;
-      if (m_run == -INFINITY) {
-        m_run = mt;
-      } else if (mt > m_run + kLazy) {
-        alpha = exp2f(m_run - mt);
-        m_run = mt;
-      }
-      if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
-        // each thread scales its half of the O row of its head
+        __syncwarp();
+      };
+      qk(0);
+      if (ntiles > 1) qk(1);
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
-          float v[32];
-          tmem_ld_32x32b_x32(t_o + c, v);
+      for (int j = 0; j < ntiles; ++j) {
+        // O += P C once the workers have written P of tile j
+        named_sync(kBarP, kThreads);
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t kvb = kv_u + (j & 1) * kKVBytes;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          tmem_st_32x32b_x32(t_o + c, v);
+          for (int k = 0; k < kTT / 16; ++k) {
+            const uint64_t ad = sdesc_kmajor_sw128(p_u + k * 32);
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+              const uint64_t bd =
+                  sdesc_mn_sw128(kvb + nh * 4 * kRegion + k * 16 * 128, kRegion, 1024);
+              umma_bf16(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
+                        (j > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(bar_pv);
         }
+        __syncwarp();
+        if (j + 2 < ntiles) qk(j + 2);
       }
-      uint32_t packed[16];
-      float ps[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        float e[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) e[i] = s[4 * u + i] == -INFINITY ? 0.f : exp2f(s[4 * u + i] - m_run);
-        const __nv_bfloat162 a = __floats2bfloat162_rn(e[0], e[1]);
-        const __nv_bfloat162 b = __floats2bfloat162_rn(e[2], e[3]);
-        packed[2 * u] = *reinterpret_cast<const uint32_t*>(&a);
-        packed[2 * u + 1] = *reinterpret_cast<const uint32_t*>(&b);
-        ps[u] = (__low2float(a) + __high2float(a)) + (__low2float(b) + __high2float(b));
-      }
-      float lsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
-      l_run = l_run * alpha + lsum;
-      // row hloc of P, pieces 4*half .. 4*half+3 (16 B each)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int piece = 4 * half + c;
-        const uint32_t a = p_u + hloc * 128 + ((piece ^ (hloc & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(packed[4 * c]),
-                     "r"(packed[4 * c + 1]), "r"(packed[4 * c + 2]), "r"(packed[4 * c + 3])
-                     : "memory");
-      }
-      fence_proxy_async();
-      tc_fence_before();
-      __syncthreads();
-
-      // ---- O += P C --------------------------------------------------------
-      if (tid == 0) {
+    } else {
+      // ======================= workers (warps 0-3) ==========================
+#pragma unroll 1
+      for (int j = 0; j < ntiles; ++j) {
+        const int buf = j & 1;
+        // report tile data to the MMA warp (tiles 0 and 1 were requested
+        // together; tile j >= 2 one iteration ago)
+        if (j == 0) {
+          if (ntiles > 1) cp_async_wait<1>();
+          else cp_async_wait<0>();
+          fence_proxy_async();
+          named_arrive(kBarData0, kThreads);
+          if (ntiles > 1) {
+            cp_async_wait<0>();
+            fence_proxy_async();
+            named_arrive(kBarData1, kThreads);
+          }
+        } else if (j >= 2) {
+          cp_async_wait<0>();
+          fence_proxy_async();
+          named_arrive(kBarData0 + buf, kThreads);
+        }
+        {
+          volatile int no_abort = 0;
+          ok_all &= mbar_wait(&bar_qk[buf], (j >> 1) & 1, &no_abort);
+        }
         tc_fence_after();
-        const uint32_t kvb = kv_u + buf * kKVBytes;
+        // the previous PV must be done before its buffer is refilled and before
+        // P or O are touched again
+        if (j > 0) {
+          volatile int no_abort = 0;
+          ok_all &= mbar_wait(bar_pv, (j - 1) & 1, &no_abort);
+          tc_fence_after();
+          if (j + 1 < ntiles) gather(j + 1);
+        }
+
+        // ---- softmax: 32 logits of head hloc per thread --------------------
+        float s[32];
+        {
+          // lanes 16-31 receive the 64 logits of their head; tokens 0-31 go
+          // to the partner lane (lanes 0-15 receive unused columns)
+          uint32_t a[32], b[32];
+          tmem_ld_x32_async(tmem + lane_base + 256 + 64 * buf, a);
+          tmem_ld_x32_async(tmem + lane_base + 256 + 64 * buf + 32, b);
+          tmem_ld_wait_regs<32>(a);
+          tmem_ld_wait_regs<32>(b);
 #pragma unroll
-        for (int k = 0; k < kTT / 16; ++k) {
-          const uint64_t ad = sdesc_kmajor_sw128(p_u + k * 32);
-#pragma unroll
-          for (int nh = 0; nh < 2; ++nh) {
-            const uint64_t bd =
-                sdesc_mn_sw128(kvb + nh * 4 * kRegion + k * 16 * 128, kRegion, 1024);
-            umma_bf16(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
-                      (j > 0 || k > 0) ? 1u : 0u);
+          for (int t = 0; t < 32; ++t) {
+            const uint32_t x = __shfl_xor_sync(0xffffffffu, a[t], 16);
+            s[t] = __uint_as_float(half ? b[t] : x);
           }
         }
-        umma_commit(bar_pv);
+        const uint32_t vm = vm_s[j * 2 + half];
+        float mx[8];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) s[t] = ((vm >> t) & 1u) ? s[t] * p.scale_log2 : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          mx[u] = fmaxf(fmaxf(s[4 * u], s[4 * u + 1]), fmaxf(s[4 * u + 2], s[4 * u + 3]));
+        float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+        float alpha = 1.f;
+        if (m_run == -INFINITY) {
+          m_run = mt;
+        } else if (mt > m_run + kLazy) {
+          alpha = exp2f(m_run - mt);
+          m_run = mt;
+        }
+        if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
+          // each thread scales its half of the O row of its head
+#pragma unroll 1
+          for (int c = 0; c < 256; c += 32) {
+            float v[32];
+            tmem_ld_32x32b_x32(tmem + lane_base + c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+            tmem_st_32x32b_x32(tmem + lane_base + c, v);
+          }
+        }
+        uint32_t packed[16];
+        float ps[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float e[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            e[i] = s[4 * u + i] == -INFINITY ? 0.f : exp2f(s[4 * u + i] - m_run);
+          const __nv_bfloat162 a = __floats2bfloat162_rn(e[0], e[1]);
+          const __nv_bfloat162 b = __floats2bfloat162_rn(e[2], e[3]);
+          packed[2 * u] = *reinterpret_cast<const uint32_t*>(&a);
+          packed[2 * u + 1] = *reinterpret_cast<const uint32_t*>(&b);
+          ps[u] = (__low2float(a) + __high2float(a)) + (__low2float(b) + __high2float(b));
+        }
+        float lsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+        l_run = l_run * alpha + lsum;
+        // row hloc of P, pieces 4*half .. 4*half+3 (16 B each)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int piece = 4 * half + c;
+          const uint32_t a = p_u + hloc * 128 + ((piece ^ (hloc & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(packed[4 * c]),
+                       "r"(packed[4 * c + 1]), "r"(packed[4 * c + 2]), "r"(packed[4 * c + 3])
+                       : "memory");
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        named_arrive(kBarP, kThreads);  // the MMA warp issues O += P C
       }
+      {
+        volatile int no_abort = 0;
+        ok_all &= mbar_wait(bar_pv, (ntiles - 1) & 1, &no_abort);
+      }
+      tc_fence_after();
     }
-    {
-      volatile int no_abort = 0;
-      ok_all &= mbar_wait(bar_pv, (ntiles - 1) & 1, &no_abort);
-    }
-    tc_fence_after();
+    __syncwarp();
   }
 
   // ---- output ----------------------------------------------------------------
@@ -426,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     // pieces rotated by the row to spread the banks), then stored coalesced
     uint8_t* stage = kv_s;
     const float inv = have ? 1.f / l_run : 0.f;
-    if (ntiles > 0) {
+    if (ntiles > 0 && worker) {
 #pragma unroll 1
       for (int c0 = 0; c0 < 256; c0 += 32) {
         float v[32];
@@ -446,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         }
       }
     }
-    if (half == 0 && h0 + hloc < p.heads && p.lse)
+    if (worker && half == 0 && h0 + hloc < p.heads && p.lse)
       p.lse[static_cast<int64_t>(r) * p.heads + h0 + hloc] =
           have ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
     __syncthreads();
@@ -454,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     uint8_t* gbase =
         reinterpret_cast<uint8_t*>(p.out + (static_cast<int64_t>(r) * p.heads + h0) * kLatent);
 #pragma unroll 1
-    for (int e = tid; e < nrows * 64; e += kThreads) {
+    for (int e = tid; worker && e < nrows * 64; e += kWork) {
       const int row = e >> 6, piece = e & 63;
       const uint4 val =
           ntiles > 0 ? *reinterpret_cast<const uint4*>(stage + row * 1024 + ((piece + row) & 63) * 16)
@@ -462,83 +516,101 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       *reinterpret_cast<uint4*>(gbase + static_cast<int64_t>(row) * 1024 + piece * 16) = val;
     }
   } else {
-    // this split's unnormalised O rows and (m, l), fp32, to L2
-    float* po = p.part_o + ((unit * n_cl + split) * kHG) * kLatent;
+    // This split's unnormalised O rows, fp32, staged in the latent buffers as
+    // [64 rows x 2 KiB] with 16-byte pieces rotated by the row (the same
+    // layout goes to L2 with one bulk copy), and its (m, l).
+    const int64_t first_row = (unit * n_cl + split) * kHG;
+    uint8_t* stage = kv_s;
+    const uint32_t stage_u = smem_u32(stage);
     if (ntiles > 0) {
-      // staged as [64 rows x 2 KiB] in the latent buffers (pieces rotated by
-      // the row), then stored coalesced
-      uint8_t* stage = kv_s;
+      if (worker) {
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 32) {
-        float v[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + c0, v);
+        for (int c0 = 0; c0 < 256; c0 += 32) {
+          float v[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + c0, v);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int piece = ((256 * half + c0) / 4 + i + hloc) & 127;
-          *reinterpret_cast<float4*>(stage + hloc * 2048 + piece * 16) =
-              make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 8; ++i) {
+            const int piece = ((256 * half + c0) / 4 + i + hloc) & 127;
+            *reinterpret_cast<float4*>(stage + hloc * 2048 + piece * 16) =
+                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
         }
       }
+      fence_proxy_async();
       __syncthreads();
-#pragma unroll 4
-      for (int e = tid; e < kHG * 128; e += kThreads) {
-        const int row = e >> 7, piece = e & 127;
-        *reinterpret_cast<float4*>(po + row * kLatent + piece * 4) =
-            *reinterpret_cast<const float4*>(stage + row * 2048 + ((piece + row) & 127) * 16);
+      if (tid == 0) {
+        bulk_store(p.part_o + first_row * kLatent, stage_u, kHG * kLatent * 4);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        asm volatile("fence.proxy.async.global;" ::: "memory");
       }
     }
-    if (half == 0) {
-      float* pm = p.part_ml + ((unit * n_cl + split) * kHG + hloc) * 2;
+    if (worker && half == 0) {
+      float* pm = p.part_ml + (first_row + hloc) * 2;
       pm[0] = have ? m_run : -INFINITY;
       pm[1] = have ? l_run : 0.f;
     }
     cluster_sync_all();  // every split's rows are in L2 and visible to the cluster
-    // CTA k combines heads [k*rows_per, (k+1)*rows_per) of the group:
-    // thread t takes dims 4t..4t+3 of each
+    // CTA k combines heads [k*rows_per, (k+1)*rows_per) of the group: the
+    // n_cl rows of each come back with bulk copies into the latent buffers
+    // (slot hh*n_cl + c), the weights 2^(m_c - M) / L from the (m, l).
     const int k = static_cast<int>(cluster_rank());
     const int rows_per = kHG / n_cl;
+    const int hk = k * rows_per;
+    int nh = p.heads - h0 - hk;
+    nh = nh < 0 ? 0 : (nh > rows_per ? rows_per : nh);
     const float* pm_all = p.part_ml + (unit * n_cl) * kHG * 2;
     const float* po_all = p.part_o + (unit * n_cl) * kHG * kLatent;
+    float* w_s = reinterpret_cast<float*>(p_s);  // [64] combine weights
+    if (nh > 0) {  // uniform
+      const int nrows = nh * n_cl;
+      if (tid == 0) mbar_arrive_expect_tx(bar_red, static_cast<uint32_t>(nrows) * 2048u);
+      if (tid < nrows) {
+        const int hh = tid / n_cl, c = tid % n_cl;
+        bulk_load(stage_u + tid * 2048, po_all + (static_cast<int64_t>(c) * kHG + hk + hh) * kLatent,
+                  2048u, bar_red);
+      }
+      if (tid < kHG) {  // warps 0-1: groups of n_cl lanes, one group per head
+        const int hh = tid / n_cl, c = tid % n_cl;
+        float2 ml = make_float2(-INFINITY, 0.f);
+        if (tid < nrows) ml = __ldcg(reinterpret_cast<const float2*>(pm_all + (c * kHG + hk + hh) * 2));
+        float M = ml.x;
+        for (int o = n_cl >> 1; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float e = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+        float L = ml.y * e;
+        for (int o = n_cl >> 1; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        w_s[tid] = L > 0.f ? e / L : 0.f;
+        if (c == 0 && tid < nrows && p.lse)
+          p.lse[static_cast<int64_t>(r) * p.heads + h0 + hk + hh] =
+              L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+      }
+      __syncthreads();
+      {
+        volatile int no_abort = 0;
+        ok_all &= mbar_wait(bar_red, 0, &no_abort);
+      }
 #pragma unroll 1
-    for (int hh = 0; hh < rows_per; ++hh) {
-      const int h = k * rows_per + hh;
-      if (h0 + h >= p.heads) break;  // uniform
-      float2 ml[kMaxCluster];
-      float4 v[kMaxCluster];
-#pragma unroll
-      for (int c = 0; c < kMaxCluster; ++c) {
-        ml[c] = make_float2(-INFINITY, 0.f);
-        v[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c < n_cl) {
-          ml[c] = __ldcg(reinterpret_cast<const float2*>(pm_all + (c * kHG + h) * 2));
-          v[c] = __ldcg(reinterpret_cast<const float4*>(po_all + (c * kHG + h) * kLatent + tid * 4));
+      for (int hh = 0; worker && hh < nh; ++hh) {
+        const int h = hk + hh;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int c = 0; c < n_cl; ++c) {
+          const float w = w_s[hh * n_cl + c];
+          if (w != 0.f) {  // uniform; rows of splits without tokens are not read
+            const float4 v = *reinterpret_cast<const float4*>(
+                stage + (hh * n_cl + c) * 2048 + ((tid + h) & 127) * 16);
+            acc.x += v.x * w;
+            acc.y += v.y * w;
+            acc.z += v.z * w;
+            acc.w += v.w * w;
+          }
         }
+        __nv_bfloat16* o = p.out + (static_cast<int64_t>(r) * p.heads + h0 + h) * kLatent + tid * 4;
+        const __nv_bfloat162 a2 = __floats2bfloat162_rn(acc.x, acc.y);
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(o) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&a2), *reinterpret_cast<const uint32_t*>(&b2));
       }
-      float M = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kMaxCluster; ++c) M = fmaxf(M, ml[c].x);
-      float L = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < kMaxCluster; ++c) {
-        const float w = ml[c].x == -INFINITY ? 0.f : exp2f(ml[c].x - M);
-        L += ml[c].y * w;
-        if (w != 0.f) {
-          acc.x += v[c].x * w;
-          acc.y += v[c].y * w;
-          acc.z += v[c].z * w;
-          acc.w += v[c].w * w;
-        }
-      }
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      __nv_bfloat16* o = p.out + (static_cast<int64_t>(r) * p.heads + h0 + h) * kLatent + tid * 4;
-      const __nv_bfloat162 a2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-      const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(o) =
-          make_uint2(*reinterpret_cast<const uint32_t*>(&a2), *reinterpret_cast<const uint32_t*>(&b2));
-      if (tid == 0 && p.lse)
-        p.lse[static_cast<int64_t>(r) * p.heads + h0 + h] =
-            L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
     }
   }
   if (!ok_all && tid == 0) atomicExch(&g_device_error, kErrWaitTimeout);
