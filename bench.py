@@ -269,6 +269,12 @@ class ClockSampler:
                 self.samples.append(line.strip())
         self.thread = threading.Thread(target=reader, daemon=True)
         self.thread.start()
+        # nvidia-smi takes a while to start: wait for its first line so that the
+        # sampling covers the timed region, then keep only later samples
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < 5.0 and self.proc.poll() is None:
+            time.sleep(0.01)
+        self.samples.clear()
 
     def stop(self):
         if self.proc is not None:

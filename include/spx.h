@@ -256,9 +256,13 @@ SPX_API spx_status spx_sparse_mla_attn(const spx_dims* d, int32_t rows, const vo
  *             already be stored at position len_dev[b])
  *   idx_out, count_out   optional (NULL) copies of the selection, e.g. to
  *             reuse it in the next layers
- *   max_len   host bound on n for every sequence; <= pool*cap_blk, <= cap_tok
+ *   max_len   host bound on n for every sequence; <= pool*cap_blk, <= cap_tok;
+ *             above 16,777,216 tokens the call returns SPX_ERR_UNSUPPORTED
  *   ws        workspace of spx_decode_workspace_size(d, B, max_len) bytes
- *   timing    optional events around the scoring launch (may be NULL)
+ *             (holds the scores, their key histogram and the selection lists)
+ *   timing    optional events around the scoring launch (may be NULL); the
+ *             kernels of the call may otherwise start before their
+ *             predecessor in the call has finished (they wait for its data)
  * ------------------------------------------------------------------------- */
 SPX_API spx_status spx_decode_workspace_size(const spx_dims* d, int32_t B,
                                      int64_t max_len, size_t* bytes);

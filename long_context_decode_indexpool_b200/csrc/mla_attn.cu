@@ -592,18 +592,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
 #pragma unroll 1
       for (int hh = 0; worker && hh < nh; ++hh) {
         const int h = hk + hh;
+        // all n_cl loads first (rows of splits without tokens are not read)
+        float w[kMaxCluster];
+        float4 v[kMaxCluster];
+#pragma unroll
+        for (int c = 0; c < kMaxCluster; ++c) {
+          w[c] = c < n_cl ? w_s[hh * n_cl + c] : 0.f;
+          v[c] = w[c] != 0.f ? *reinterpret_cast<const float4*>(
+                                   stage + (hh * n_cl + c) * 2048 + ((tid + h) & 127) * 16)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int c = 0; c < n_cl; ++c) {
-          const float w = w_s[hh * n_cl + c];
-          if (w != 0.f) {  // uniform; rows of splits without tokens are not read
-            const float4 v = *reinterpret_cast<const float4*>(
-                stage + (hh * n_cl + c) * 2048 + ((tid + h) & 127) * 16);
-            acc.x += v.x * w;
-            acc.y += v.y * w;
-            acc.z += v.z * w;
-            acc.w += v.w * w;
-          }
+#pragma unroll
+        for (int c = 0; c < kMaxCluster; ++c) {
+          acc.x += v[c].x * w[c];
+          acc.y += v[c].y * w[c];
+          acc.z += v[c].z * w[c];
+          acc.w += v[c].w * w[c];
         }
         __nv_bfloat16* o = p.out + (static_cast<int64_t>(r) * p.heads + h0 + h) * kLatent + tid * 4;
         const __nv_bfloat162 a2 = __floats2bfloat162_rn(acc.x, acc.y);
