@@ -61,6 +61,9 @@ constexpr int kHG = 64;                         // heads per CTA (MMA M)
 constexpr int kRegion = 64 * 128;               // [64 rows x 128 B] = 8 KiB
 constexpr int kQBytes = 8 * kRegion;            // 64 KiB
 constexpr int kKVBytes = 8 * kRegion;           // 64 KiB per tile
+// The two latent tiles share 8 regions of [128 rows x 128 B] (tile b in rows
+// 64b..64b+63), so that both together also form one N = 128 operand.
+constexpr int kKVRegion = 2 * kRegion;          // 16 KiB
 constexpr int kPBytes = kRegion;                // [64 heads x 64 tokens] bf16
 constexpr int kMaxList = kTopK * kPool + kPool - 1;             // tokens in a list, at most
 constexpr int kPosCap = (kMaxList + kTT - 1) / kTT * kTT;       // position slots
@@ -70,6 +73,7 @@ constexpr int kSmemBytes = 1024 + kQBytes + 2 * kKVBytes + kPBytes + kPosCap * 8
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLazy = 8.f;                    // rescale threshold (log2 units)
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, kTT);
+constexpr uint32_t kIdescQK2 = idesc_bf16_f32(64, 2 * kTT);  // both tiles at once
 // PV: B (the latent tile) is MN-major: set the "transpose B" bit.
 constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256) | (1u << 16);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -147,6 +151,10 @@ __device__ __forceinline__ void bulk_load(uint32_t sdst, const void* gsrc, uint3
 // regions of [64 rows x 128 B] with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t sw_off(int r, int c) {
   return static_cast<uint32_t>((c >> 3) * kRegion + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+// The same for row r (0..127) of the latent tile pair (regions of 16 KiB).
+__device__ __forceinline__ uint32_t kv_off(int r, int c) {
+  return static_cast<uint32_t>((c >> 3) * kKVRegion + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
 // Shared-memory descriptor of an MN-major operand in the 128-byte-swizzle
@@ -275,14 +283,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   if (ntiles > 0) {  // uniform
     const __nv_bfloat16* lat = p.latent + static_cast<int64_t>(r) * p.seq_stride;
     auto gather = [&](int tile) {
-      const uint32_t dst = kv_u + (tile & 1) * kKVBytes;
+      const int row0 = (tile & 1) * kTT;
       const int64_t* ps = pos_s + tile * kTT;
 #pragma unroll 4
       for (int i = 0; i < (kTT * 64) / kWork; ++i) {
         const int c = i * kWork + tid;
         const int t = c >> 6, piece = c & 63;
         const int64_t pos = ps[t];
-        cp_async16(dst + sw_off(t, piece), lat + (pos >= 0 ? pos : 0) * kLatent + piece * 8,
+        cp_async16(kv_u + kv_off(row0 + t, piece), lat + (pos >= 0 ? pos : 0) * kLatent + piece * 8,
                    pos >= 0);
       }
       cp_async_commit();
@@ -311,38 +319,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       // ======================= MMA issuer (warp 4) ===========================
       // S = Q C^T of tile t into S buffer t&1 (TMEM lanes 16-31 of each
       // quarter, columns 256+64b ..), once the workers report its data.
-      auto qk = [&](int t) {
+      // pair: tiles 0 and 1 as one N = 128 product (S buffers 0 and 1 are
+      // adjacent columns), committed to both buffers' barriers
+      auto qk = [&](int t, bool pair) {
         named_sync(kBarData0 + (t & 1), kThreads);
+        if (pair) named_sync(kBarData1, kThreads);
         if (lane == 0) {
           tc_fence_after();
-          const uint32_t kvb = kv_u + (t & 1) * kKVBytes;
+          const uint32_t kvb = kv_u + (t & 1) * kTT * 128;
           const uint32_t d = tmem + (16u << 16) + 256 + 64 * (t & 1);
 #pragma unroll 4
           for (int k = 0; k < kLatent / 16; ++k) {
-            const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
-            umma_bf16(d, sdesc_kmajor_sw128(q_u + off), sdesc_kmajor_sw128(kvb + off), kIdescQK,
-                      k > 0 ? 1u : 0u);
+            const uint32_t qoff = (k >> 2) * kRegion + (k & 3) * 32;
+            const uint32_t koff = (k >> 2) * kKVRegion + (k & 3) * 32;
+            umma_bf16(d, sdesc_kmajor_sw128(q_u + qoff), sdesc_kmajor_sw128(kvb + koff),
+                      pair ? kIdescQK2 : kIdescQK, k > 0 ? 1u : 0u);
           }
           umma_commit(&bar_qk[t & 1]);
+          if (pair) umma_commit(&bar_qk[1]);
         }
         __syncwarp();
       };
-      qk(0);
-      if (ntiles > 1) qk(1);
+      qk(0, ntiles > 1);
 #pragma unroll 1
       for (int j = 0; j < ntiles; ++j) {
         // O += P C once the workers have written P of tile j
         named_sync(kBarP, kThreads);
         if (lane == 0) {
           tc_fence_after();
-          const uint32_t kvb = kv_u + (j & 1) * kKVBytes;
+          const uint32_t kvb = kv_u + (j & 1) * kTT * 128;
 #pragma unroll
           for (int k = 0; k < kTT / 16; ++k) {
             const uint64_t ad = sdesc_kmajor_sw128(p_u + k * 32);
 #pragma unroll
             for (int nh = 0; nh < 2; ++nh) {
               const uint64_t bd =
-                  sdesc_mn_sw128(kvb + nh * 4 * kRegion + k * 16 * 128, kRegion, 1024);
+                  sdesc_mn_sw128(kvb + nh * 4 * kKVRegion + k * 16 * 128, kKVRegion, 1024);
               umma_bf16(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
                         (j > 0 || k > 0) ? 1u : 0u);
             }
@@ -350,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
           umma_commit(bar_pv);
         }
         __syncwarp();
-        if (j + 2 < ntiles) qk(j + 2);
+        if (j + 2 < ntiles) qk(j + 2, false);
       }
     } else {
       // ======================= workers (warps 0-3) ==========================
