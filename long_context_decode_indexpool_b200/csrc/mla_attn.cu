@@ -209,10 +209,10 @@ __device__ __forceinline__ RowInfo row_info(const KParams& p, int r) {
   return ri;
 }
 
-// token position of entry j of row r's list, or -1 (skipped block)
-__device__ __forceinline__ int64_t token_pos(const KParams& p, int r, const RowInfo& ri, int j) {
+// token position of entry j of row r's list, or -1 (skipped block); b is
+// the selected block id idx[r][j / 4] when j is in the selected part
+__device__ __forceinline__ int64_t token_pos_of(const RowInfo& ri, int j, int b) {
   if (j < ri.cnt * kPool) {
-    const int b = p.idx[static_cast<int64_t>(r) * kTopK + (j >> 2)];
     if (b < 0 || b >= ri.nblk) return -1;
     return static_cast<int64_t>(b) * kPool + (j & 3);
   }
@@ -271,6 +271,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   pdl_trigger();
   pdl_wait();  // the selected blocks come from the previous kernel
 
+  // the block id of this thread's first list entry goes out with the row's
+  // length and count (one round trip instead of two)
+  const int j_first = split * p.split_tokens + tid;
+  const int32_t* idx_row = p.idx + static_cast<int64_t>(r) * kTopK;
+  const int b_first = (worker && j_first < kTopK * kPool) ? idx_row[j_first >> 2] : -1;
   const RowInfo ri = row_info(p, r);
   const int j_begin = split * p.split_tokens;
   const int j_end = split == n_cl - 1 ? ri.S : min(ri.S, j_begin + p.split_tokens);
@@ -301,7 +306,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       for (int i0 = 0; i0 < ntiles * kTT; i0 += kWork) {
         const int i = i0 + tid;
         int64_t pos = -1;
-        if (i < nlist) pos = token_pos(p, r, ri, j_begin + i);
+        if (i < nlist) {
+          const int j = j_begin + i;
+          const int b = i0 == 0 ? b_first : (j < ri.cnt * kPool ? idx_row[j >> 2] : -1);
+          pos = token_pos_of(ri, j, b);
+        }
         if (i < ntiles * kTT) pos_s[i] = pos;
         const uint32_t bits = __ballot_sync(0xffffffffu, pos >= 0);
         if (lane == 0 && i < ntiles * kTT) vm_s[i >> 5] = bits;

@@ -221,3 +221,59 @@ def test_prefill_full_chunk_sampled():
     qs = [0, 1, 2, 3, 4, 5, 6, 7, 8, 1023, 1024, 1025, 1026, 1027, 2047, 2048, 3071, 4091,
           4092, 4093, 4094, 4095]
     _check_prefill(st, qs)
+
+
+def test_decode_ragged_lengths_one_call():
+    """Rows of very different lengths in one fused call: dense rows (<= 2051
+    tokens, one with a partial tail), a row whose 512th score is shared by
+    many blocks, and longer rows spread over several selection chunks."""
+    spx = need_gpu()
+    rng = np.random.default_rng(7)
+    lens = [9001, 2051, 1203, 20000, 36003, 4]  # tokens seen by each query
+    B, max_len = len(lens), 36004
+    cap_blk, cap_tok = max_len // 4 + 1, max_len
+    pw = np.array([0.5, 0.25, 0.125, 0.125])
+    keys = np.zeros((B, cap_blk, 128), np.uint16)
+    pooled_ref = []
+    for b, n in enumerate(lens):
+        raw = rng.integers(-8, 9, (n - n % 4, 128)).astype(np.float32)
+        if b == 3:
+            raw[:, :] = np.sign(raw)  # few distinct scores: a crowded cut bin
+        p = oracle.pool(synth.f32_to_bf16_bits_np(raw), pw)
+        keys[b, :p.shape[0]] = p
+        pooled_ref.append(p)
+    q_idx = synth.f32_to_bf16_bits_np(rng.integers(-4, 5, (B, 32, 128)).astype(np.float32))
+    w_head = np.array([0.25, 0.5, 1.0], np.float32)[rng.integers(0, 3, (B, 32))]
+    H = 64
+    q = synth.f32_to_bf16_bits_np((rng.standard_normal((B, H, 512)) / np.sqrt(512)).astype(np.float32))
+    # latent rows: multiples of 1/16 in [-1/2, 1/2] (exact in bf16), made on the device
+    g = torch.Generator(device="cuda").manual_seed(7)
+    lat_dev = (torch.randint(-8, 9, (B, cap_tok, 512), generator=g, device="cuda",
+                             dtype=torch.int16).to(torch.bfloat16) / 16)
+    dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    d = spx.dims(H, 1.0)
+    len_dev = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    out = torch.empty(B, H, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
+    idx = torch.empty(B, 512, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(B, dtype=torch.int32, device="cuda")
+    ws = spx.workspace(spx.spx_decode_workspace_size(d, B, max_len), "cuda")
+    spx.spx_decode_fused(d, B, None, None, None, dev(keys), cap_blk, len_dev, dev(q_idx),
+                         torch.from_numpy(w_head).cuda(), dev(q), lat_dev, cap_tok, max_len,
+                         out, lse, idx, cnt, ws)
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    got, lse = f64_of(out), lse.cpu().numpy()
+    refs = []
+    for b, n in enumerate(lens):
+        r = oracle.decode_query(q_idx[b], w_head[b].astype(np.float64), pooled_ref[b], n, q[b],
+                                lambda pos, b=b: bits_of(lat_dev[b, torch.from_numpy(pos).cuda()]),
+                                1.0)
+        assert cnt[b] == r["idx"].size, f"row {b}"
+        assert np.array_equal(idx[b, :cnt[b]], r["idx"]), f"row {b}"
+        assert (idx[b, cnt[b]:] == -1).all()
+        assert np.allclose(lse[b], r["lse"], atol=LSE_ATOL, rtol=0), f"row {b}"
+        refs.append(r["out"])
+    assert_attention_close(got, np.stack(refs), "ragged")
+    assert cnt[1] == 512 and cnt[2] == 300 and cnt[5] == 1
