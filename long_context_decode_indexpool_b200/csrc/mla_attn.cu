@@ -37,10 +37,12 @@
 //
 // A row with a single split writes its normalised output directly.  The n
 // splits of one (row, head group) otherwise form a thread-block cluster: each
-// CTA writes its unnormalised O rows (fp32) and per-head (m, l) to global
-// memory (L2), the cluster barrier makes them visible, and CTA k combines
-// heads [k*64/n, (k+1)*64/n) of all splits with the log-sum-exp rule into
-// the bf16 output and the log-sum-exp.  No second kernel runs.
+// CTA writes its output rows normalised by its own l (bf16, like P) and its
+// per-head (m, l) (fp32) to L2 with one bulk copy, the cluster barrier
+// publishes them, and CTA k reads back heads [k*64/n, (k+1)*64/n) of all
+// splits with bulk copies and combines them with the log-sum-exp rule
+// (weights 2^(m_s - M) l_s / L) into the bf16 output and the log-sum-exp.
+// No second kernel runs.
 #include "spx_device.cuh"
 #include "spx_internal.h"
 #include "spx_launch.cuh"
@@ -92,8 +94,8 @@ struct KParams {
   float scale_log2;
   __nv_bfloat16* out;
   float* lse;
-  float* part_o;   // [rows, groups, nsplit, 64, 512] unnormalised O (nsplit > 1)
-  float* part_ml;  // [rows, groups, nsplit, 64, 2]   (m, l)
+  __nv_bfloat16* part_o;  // [rows, groups, nsplit, 64, 512] O / l of each split (nsplit > 1)
+  float* part_ml;         // [rows, groups, nsplit, 64, 2]   (m, l)
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -496,31 +498,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   cp_async_wait<0>();  // (a split without tokens still has Q copies in flight)
   const bool have = ntiles > 0 && ok_all && l_run > 0.f;
   const int64_t unit = static_cast<int64_t>(r) * gridDim.z + hg;  // (row, head group)
-  if (n_cl == 1) {
-    // normalised bf16 rows of 1 KiB staged in the latent buffers (16-byte
-    // pieces rotated by the row to spread the banks), then stored coalesced
-    uint8_t* stage = kv_s;
+  // This split's output rows, normalised by its own l, as bf16 rows of 1 KiB
+  // staged in the latent buffers (16-byte pieces rotated by the row to spread
+  // the banks).
+  uint8_t* stage = kv_s;
+  const uint32_t stage_u = smem_u32(stage);
+  if (ntiles > 0 && worker) {
     const float inv = have ? 1.f / l_run : 0.f;
-    if (ntiles > 0 && worker) {
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 32) {
-        float v[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + c0, v);
+    for (int c0 = 0; c0 < 256; c0 += 32) {
+      float v[32];
+      tmem_ld_32x32b_x32(tmem + lane_base + c0, v);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t w[4];
+      for (int i = 0; i < 4; ++i) {
+        uint32_t w[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const __nv_bfloat162 h2 =
-                __floats2bfloat162_rn(v[8 * i + 2 * u] * inv, v[8 * i + 2 * u + 1] * inv);
-            w[u] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
-          const int piece = ((256 * half + c0) / 8 + i + hloc) & 63;
-          *reinterpret_cast<uint4*>(stage + hloc * 1024 + piece * 16) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+        for (int u = 0; u < 4; ++u) {
+          const __nv_bfloat162 h2 =
+              __floats2bfloat162_rn(v[8 * i + 2 * u] * inv, v[8 * i + 2 * u + 1] * inv);
+          w[u] = *reinterpret_cast<const uint32_t*>(&h2);
         }
+        const int piece = ((256 * half + c0) / 8 + i + hloc) & 63;
+        *reinterpret_cast<uint4*>(stage + hloc * 1024 + piece * 16) =
+            make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
+  }
+  if (n_cl == 1) {
     if (worker && half == 0 && h0 + hloc < p.heads && p.lse)
       p.lse[static_cast<int64_t>(r) * p.heads + h0 + hloc] =
           have ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
@@ -537,30 +541,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       *reinterpret_cast<uint4*>(gbase + static_cast<int64_t>(row) * 1024 + piece * 16) = val;
     }
   } else {
-    // This split's unnormalised O rows, fp32, staged in the latent buffers as
-    // [64 rows x 2 KiB] with 16-byte pieces rotated by the row (the same
-    // layout goes to L2 with one bulk copy), and its (m, l).
+    // The staged rows (same layout in L2, one bulk copy) and (m, l) of this
+    // split go to L2; the cluster barrier publishes them.
     const int64_t first_row = (unit * n_cl + split) * kHG;
-    uint8_t* stage = kv_s;
-    const uint32_t stage_u = smem_u32(stage);
     if (ntiles > 0) {
-      if (worker) {
-#pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 32) {
-          float v[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + c0, v);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int piece = ((256 * half + c0) / 4 + i + hloc) & 127;
-            *reinterpret_cast<float4*>(stage + hloc * 2048 + piece * 16) =
-                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          }
-        }
-      }
       fence_proxy_async();
       __syncthreads();
       if (tid == 0) {
-        bulk_store(p.part_o + first_row * kLatent, stage_u, kHG * kLatent * 4);
+        bulk_store(p.part_o + first_row * kLatent, stage_u, kHG * kLatent * 2);
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -571,25 +559,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       pm[0] = have ? m_run : -INFINITY;
       pm[1] = have ? l_run : 0.f;
     }
-    cluster_sync_all();  // every split's rows are in L2 and visible to the cluster
+    cluster_sync_all();
     // CTA k combines heads [k*rows_per, (k+1)*rows_per) of the group: the
     // n_cl rows of each come back with bulk copies into the latent buffers
-    // (slot hh*n_cl + c), the weights 2^(m_c - M) / L from the (m, l).
+    // (slot hh*n_cl + c); weights 2^(m_c - M) l_c / L from the (m, l).
     const int k = static_cast<int>(cluster_rank());
     const int rows_per = kHG / n_cl;
     const int hk = k * rows_per;
     int nh = p.heads - h0 - hk;
     nh = nh < 0 ? 0 : (nh > rows_per ? rows_per : nh);
     const float* pm_all = p.part_ml + (unit * n_cl) * kHG * 2;
-    const float* po_all = p.part_o + (unit * n_cl) * kHG * kLatent;
+    const __nv_bfloat16* po_all = p.part_o + (unit * n_cl) * kHG * kLatent;
     float* w_s = reinterpret_cast<float*>(p_s);  // [64] combine weights
     if (nh > 0) {  // uniform
       const int nrows = nh * n_cl;
-      if (tid == 0) mbar_arrive_expect_tx(bar_red, static_cast<uint32_t>(nrows) * 2048u);
+      if (tid == 0) mbar_arrive_expect_tx(bar_red, static_cast<uint32_t>(nrows) * 1024u);
       if (tid < nrows) {
         const int hh = tid / n_cl, c = tid % n_cl;
-        bulk_load(stage_u + tid * 2048, po_all + (static_cast<int64_t>(c) * kHG + hk + hh) * kLatent,
-                  2048u, bar_red);
+        bulk_load(stage_u + tid * 1024, po_all + (static_cast<int64_t>(c) * kHG + hk + hh) * kLatent,
+                  1024u, bar_red);
       }
       if (tid < kHG) {  // warps 0-1: groups of n_cl lanes, one group per head
         const int hh = tid / n_cl, c = tid % n_cl;
@@ -597,8 +585,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         if (tid < nrows) ml = __ldcg(reinterpret_cast<const float2*>(pm_all + (c * kHG + hk + hh) * 2));
         float M = ml.x;
         for (int o = n_cl >> 1; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        const float e = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-        float L = ml.y * e;
+        const float e = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M) * ml.y;
+        float L = e;
         for (int o = n_cl >> 1; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
         w_s[tid] = L > 0.f ? e / L : 0.f;
         if (c == 0 && tid < nrows && p.lse)
@@ -610,32 +598,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         volatile int no_abort = 0;
         ok_all &= mbar_wait(bar_red, 0, &no_abort);
       }
+      // thread t: 8 dims (one 16-byte piece) of one head, two heads per pass
 #pragma unroll 1
-      for (int hh = 0; worker && hh < nh; ++hh) {
+      for (int e = tid; worker && e < nh * 64; e += kWork) {
+        const int hh = e >> 6, piece = e & 63;
         const int h = hk + hh;
-        // all n_cl loads first (rows of splits without tokens are not read)
-        float w[kMaxCluster];
-        float4 v[kMaxCluster];
+        float wc[kMaxCluster];
+        uint4 v[kMaxCluster];
 #pragma unroll
         for (int c = 0; c < kMaxCluster; ++c) {
-          w[c] = c < n_cl ? w_s[hh * n_cl + c] : 0.f;
-          v[c] = w[c] != 0.f ? *reinterpret_cast<const float4*>(
-                                   stage + (hh * n_cl + c) * 2048 + ((tid + h) & 127) * 16)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+          wc[c] = c < n_cl ? w_s[hh * n_cl + c] : 0.f;
+          v[c] = wc[c] != 0.f ? *reinterpret_cast<const uint4*>(
+                                    stage + (hh * n_cl + c) * 1024 + ((piece + h) & 63) * 16)
+                              : make_uint4(0u, 0u, 0u, 0u);
         }
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < kMaxCluster; ++c) {
-          acc.x += v[c].x * w[c];
-          acc.y += v[c].y * w[c];
-          acc.z += v[c].z * w[c];
-          acc.w += v[c].w * w[c];
+          const uint32_t u[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&u[q]);
+            acc[2 * q] += __low2float(b2) * wc[c];
+            acc[2 * q + 1] += __high2float(b2) * wc[c];
+          }
         }
-        __nv_bfloat16* o = p.out + (static_cast<int64_t>(r) * p.heads + h0 + h) * kLatent + tid * 4;
-        const __nv_bfloat162 a2 = __floats2bfloat162_rn(acc.x, acc.y);
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc.z, acc.w);
-        *reinterpret_cast<uint2*>(o) =
-            make_uint2(*reinterpret_cast<const uint32_t*>(&a2), *reinterpret_cast<const uint32_t*>(&b2));
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+          o[q] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        *reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(r) * p.heads + h0 + h) * kLatent +
+                                  piece * 8) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
   }
@@ -722,7 +717,7 @@ AttnPlan plan_attn(int rows, int heads, int64_t max_len, int num_sms) {
   p.ws_bytes = 0;
   if (n > 1) {
     const size_t units_n = static_cast<size_t>(units) * n * kHG;
-    p.ws_bytes = ((units_n * kLatent * 4 + 255) & ~static_cast<size_t>(255)) + units_n * 2 * 4;
+    p.ws_bytes = ((units_n * kLatent * 2 + 255) & ~static_cast<size_t>(255)) + units_n * 2 * 4;
   }
   return p;
 }
@@ -758,9 +753,9 @@ cudaError_t launch_attn(const AttnPlan& pl0, const AttnArgs& a, cudaStream_t str
   p.part_ml = nullptr;
   if (pl.nsplit > 1) {
     const size_t units_n = static_cast<size_t>(pl.rows) * pl.groups * pl.nsplit * kHG;
-    p.part_o = static_cast<float*>(a.ws);
+    p.part_o = static_cast<__nv_bfloat16*>(a.ws);
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
-                                         ((units_n * kLatent * 4 + 255) & ~static_cast<size_t>(255)));
+                                         ((units_n * kLatent * 2 + 255) & ~static_cast<size_t>(255)));
   }
   cudaError_t e = launch_ex(k_sparse_attn, dim3(pl.nsplit, pl.rows, pl.groups), dim3(kThreads),
                             kSmemBytes, stream, a.pdl, pl.nsplit, p);
