@@ -118,16 +118,26 @@ class DecodeState:
         self.idx = torch.empty(B, synth.TOPK_BLOCKS, dtype=torch.int32, device=device)
         self.count = torch.empty(B, dtype=torch.int32, device=device)
         self.ws = spx.workspace(spx.spx_decode_workspace_size(self.d, B, L), device)
+        self._call = None
         torch.cuda.synchronize(device)
 
     def step(self, timing=None, raw_new=None, q_idx=None, w_head=None, q=None, out=None):
         spx = spx_module()
+        if self._call is None:  # device pointers and host arguments, resolved once
+            self._call = dict(
+                pool_w=spx.pool_weights(self.pool_w), tail=self.tail.data_ptr(),
+                pooled=self.pooled.data_ptr(), len_dev=self.len_dev.data_ptr(),
+                latent=self.latent.data_ptr(), lse=self.lse.data_ptr(), idx=self.idx.data_ptr(),
+                count=self.count.data_ptr(), ws=self.ws.data_ptr(),
+                ws_bytes=self.ws.numel() * self.ws.element_size(),
+                stream=torch.cuda.current_stream(self.device).cuda_stream)
+        c = self._call
         spx.spx_decode_fused(
-            self.d, self.B, self.raw_new if raw_new is None else raw_new, self.pool_w, self.tail,
-            self.pooled, self.cap_blk, self.len_dev, self.q_idx if q_idx is None else q_idx,
-            self.w_head if w_head is None else w_head, self.q if q is None else q, self.latent,
-            self.cap_tok, self.max_len, self.out if out is None else out, self.lse, self.idx,
-            self.count, self.ws, timing=timing)
+            self.d, self.B, self.raw_new if raw_new is None else raw_new, c["pool_w"], c["tail"],
+            c["pooled"], self.cap_blk, c["len_dev"], self.q_idx if q_idx is None else q_idx,
+            self.w_head if w_head is None else w_head, self.q if q is None else q, c["latent"],
+            self.cap_tok, self.max_len, self.out if out is None else out, c["lse"], c["idx"],
+            c["count"], c["ws"], ws_bytes=c["ws_bytes"], timing=timing, stream=c["stream"])
 
     # ---- host copies of what the oracle needs (generator output) ----
     def raw_keys_host(self, b: int) -> np.ndarray:
@@ -513,21 +523,27 @@ def run_decode(args, world, rank, local):
     score_avg = sum(score_ms) / len(score_ms)
 
     # ---- end to end: host buffers in, host result out, every step ----------
-    h_raw = st.raw_new.cpu().pin_memory()
-    h_qidx = st.q_idx.cpu().pin_memory()
-    h_w = st.w_head.cpu().pin_memory()
-    h_q = st.q.cpu().pin_memory()
+    # The step's inputs (new raw key, indexer query and weights, MLA query)
+    # travel in one pinned host buffer and one copy; the output comes back
+    # with one copy.
+    ins = (st.raw_new, st.q_idx, st.w_head, st.q)
+    sizes = [t.numel() * t.element_size() for t in ins]
+    offs = [0]
+    for n in sizes[:-1]:
+        offs.append(offs[-1] + (n + 255) // 256 * 256)
+    total = offs[-1] + sizes[-1]
+    h_in = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    for t, o, n in zip(ins, offs, sizes):
+        h_in[o:o + n].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
+    d_in = torch.empty(total, dtype=torch.uint8, device=device)
+    d_raw, d_qidx, d_w, d_q = (d_in[o:o + n].view(t.dtype).view(t.shape)
+                               for t, o, n in zip(ins, offs, sizes))
     h_out = torch.empty(st.out.shape, dtype=st.out.dtype, pin_memory=True)
-    d_raw, d_qidx, d_w, d_q = (torch.empty_like(st.raw_new), torch.empty_like(st.q_idx),
-                               torch.empty_like(st.w_head), torch.empty_like(st.q))
-    h2d = sum(t.numel() * t.element_size() for t in (h_raw, h_qidx, h_w, h_q))
+    h2d = total
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step():
-        d_raw.copy_(h_raw, non_blocking=True)
-        d_qidx.copy_(h_qidx, non_blocking=True)
-        d_w.copy_(h_w, non_blocking=True)
-        d_q.copy_(h_q, non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
         st.step(raw_new=d_raw, q_idx=d_qidx, w_head=d_w, q=d_q)
         h_out.copy_(st.out, non_blocking=True)
         stream.synchronize()

@@ -127,8 +127,14 @@ def version() -> str:
 
 
 def _host_f32(arr):
-    a = (ctypes.c_float * 4)(*[float(x) for x in arr])
-    return a
+    if isinstance(arr, ctypes.Array):
+        return arr
+    return (ctypes.c_float * 4)(*[float(x) for x in arr])
+
+
+def pool_weights(w):
+    """The 4 pooling weights as the host array the calls take (convert once, reuse)."""
+    return _host_f32(w)
 
 
 def _event_handle(ev):
