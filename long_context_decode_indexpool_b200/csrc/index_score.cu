@@ -24,7 +24,8 @@
 //               boxes of 64 dims, 128-byte swizzle), query groups into
 //               kQSlots slots.
 //   warp 1      allocates TMEM; one lane issues 8 tcgen05.mma (K = 16 each)
-//               per tile into one of two TMEM accumulators.
+//               per tile into a ring of TMEM accumulators (4 slots for one
+//               query per group, 2 for eight).
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator row, ReLU, weighted
 //               head sum in fp32, length mask; then either a store of the
 //               fp32 scores (and, with SELECT, a histogram of their keys).
@@ -64,7 +65,10 @@ struct Cfg {
   static constexpr int kQSlots = NQ == 1 ? 2 : 1;
   static constexpr int kQHalf = kN * 128;
   static constexpr int kQBytes = 2 * kQHalf;
-  static constexpr int kTmemCols = 2 * kN;
+  // TMEM accumulator ring: 4 slots of 32 columns for one query (the MMA of
+  // tile t+4 waits for the epilogue of tile t), 2 of 256 for eight
+  static constexpr int kAcc = NQ == 1 ? 4 : 2;
+  static constexpr int kTmemCols = kAcc * kN;
   static constexpr int kQOff = kStages * kTileBytes;
   static constexpr int kWOff = kQOff + kQSlots * kQBytes;
   static constexpr int kNbOff = kWOff + kN * 4;
@@ -72,7 +76,7 @@ struct Cfg {
   static constexpr int kSelBytes =
       SELECT ? kHistBins * 4 : 0;
   static constexpr int kBarOff = (kSelOff + kSelBytes + 7) & ~7;
-  static constexpr int kNumBars = 2 * kStages + 2 * kQSlots + 4 + 1;
+  static constexpr int kNumBars = 2 * kStages + 2 * kQSlots + 2 * kAcc + 1;
   static constexpr int kSmem = 1024 + kBarOff + kNumBars * 8 + 16;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, kN);
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -157,8 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qfull = empty + C::kStages;
   uint64_t* qempty = qfull + C::kQSlots;
   uint64_t* accfull = qempty + C::kQSlots;
-  uint64_t* accempty = accfull + 2;
-  uint64_t* drain = accempty + 2;
+  uint64_t* accempty = accfull + C::kAcc;
+  uint64_t* drain = accempty + C::kAcc;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&qfull[s], 1);
       mbar_init(&qempty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < C::kAcc; ++s) {
       mbar_init(&accfull[s], 1);
       mbar_init(&accempty[s], 4);
     }
@@ -316,8 +320,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           stage = 0;
           ph ^= 1;
         }
-        acc ^= 1;
-        if (acc == 0) acc_ph ^= 1;
+        if (++acc == C::kAcc) {
+          acc = 0;
+          acc_ph ^= 1;
+        }
         w.advance(p);
       }
       // Wait for every MMA issued by this thread before TMEM is released.
@@ -399,8 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accempty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_ph ^= 1;
+      if (++acc == C::kAcc) {
+        acc = 0;
+        acc_ph ^= 1;
+      }
 
 #pragma unroll 1
       for (int j = 0; j < NQ; ++j) {
