@@ -600,6 +600,62 @@ def run_decode(args, world, rank, local):
     return line
 
 
+def run_indexshare(args, world, rank, local):
+    """IndexShare decode ([W3] "IndexShare는 관련 토큰을 찾는 비용을 낮춘다": one
+    indexer per group of sparse layers): per step, layer 0 runs the whole path
+    (append, scores, top-512, attention) and the other N-1 layers run only the
+    attention on layer 0's selection, each with its own query and latent cache.
+    Reports amortised queries/s per layer."""
+    spx = spx_module()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = synth.workload(args.workload)
+    st = DecodeState(w, device, b_offset=shard_offset(rank, w.B))
+    B, L, H, N = st.B, st.L, st.H, args.indexshare
+    g = torch.Generator(device=device).manual_seed(1234 + rank)
+    lat = [torch.randn(B, st.cap_tok, synth.LATENT, generator=g, device=device).to(torch.bfloat16)
+           for _ in range(N - 1)]
+    qs = [(torch.randn(B, H, synth.LATENT, generator=g, device=device) * synth.MLA_Q_SCALE)
+          .to(torch.bfloat16) for _ in range(N - 1)]
+    outs = [torch.empty_like(st.out) for _ in range(N - 1)]
+    n_vis = torch.full((B,), L, dtype=torch.int64, device=device)  # after the append
+    ws_a = spx.workspace(spx.spx_attn_workspace_size(st.d, B, L), device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        st.step()
+        for l in range(N - 1):
+            spx.spx_sparse_mla_attn(st.d, B, qs[l], lat[l], st.cap_tok * synth.LATENT, st.cap_tok,
+                                    st.idx, st.count, n_vis, L, outs[l], None, ws_a)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    K = args.steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    ev0.record(stream)
+    for _ in range(K):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
+    if spx.spx_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    if rank != 0:
+        return None
+    per_layer_ms = ms / K / N
+    return {"metric": f"IndexShare decode: amortised per-layer queries/s, one indexer per {N} layers",
+            "value": B * world / (per_layer_ms * 1e-3), "unit": "queries/s per layer",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_layer": per_layer_ms,
+            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "dtype": "bf16",
+            "data": "synthetic (layer 0 as the decode workload; other layers N(0,1) latent, "
+                    "N(0,1)/sqrt(512) queries)",
+            "config": {"workload": w.name, "layers_per_indexer": N, "batch_per_gpu": B,
+                       "context": L, "heads": H}}
+
+
 def run_prefill(args, world, rank, local):
     spx = spx_module()
     device = torch.device("cuda", local)
@@ -704,6 +760,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("spx", "reference"), default="spx")
     ap.add_argument("--workload", default="1m", choices=synth.WORKLOADS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--indexshare", type=int, default=0, metavar="N",
+                    help="IndexShare decode: one indexer per N layers (reports per-layer rate)")
     ap.add_argument("--score-only", action="store_true",
                     help="time the decode scoring kernel alone (profiling aid)")
     args = ap.parse_args(argv)
@@ -716,13 +774,15 @@ def main(argv=None):
     try:
         if args.score_only:
             line = run_score_only(args, world, rank, local)
+        elif args.indexshare > 1:
+            line = run_indexshare(args, world, rank, local)
         elif args.workload == "prefill":
             line = run_prefill(args, world, rank, local)
         else:
             line = run_decode(args, world, rank, local)
         if rank == 0 and line is not None:
             if (world == 1 and not args.no_cpu_baseline and args.workload != "prefill"
-                    and not args.score_only):
+                    and not args.score_only and args.indexshare <= 1):
                 line["cpu_baseline"] = cpu_baseline(synth.workload(args.workload),
                                                     torch.device("cuda", local))
             print(json.dumps(line))

@@ -277,3 +277,33 @@ def test_decode_ragged_lengths_one_call():
         refs.append(r["out"])
     assert_attention_close(got, np.stack(refs), "ragged")
     assert cnt[1] == 512 and cnt[2] == 300 and cnt[5] == 1
+
+
+def test_indexshare_other_layer_on_shared_selection():
+    """IndexShare: a second layer attends over the first layer's selection
+    with its own query and latent cache (no indexer pass of its own)."""
+    spx = need_gpu()
+    st = _decode_state("tiny")
+    st.step()
+    torch.cuda.synchronize()
+    B, L, H = st.B, st.L, st.H
+    g = torch.Generator(device="cuda").manual_seed(11)
+    lat2 = (torch.randint(-8, 9, (B, st.cap_tok, 512), generator=g, device="cuda",
+                          dtype=torch.int16).to(torch.bfloat16) / 16)
+    q2 = (torch.randn(B, H, 512, generator=g, device="cuda") / 512 ** 0.5).to(torch.bfloat16)
+    n_vis = torch.full((B,), L, dtype=torch.int64, device="cuda")
+    out2 = torch.empty_like(st.out)
+    lse2 = torch.empty_like(st.lse)
+    ws = spx.workspace(spx.spx_attn_workspace_size(st.d, B, L), "cuda")
+    spx.spx_sparse_mla_attn(st.d, B, q2, lat2, st.cap_tok * 512, st.cap_tok, st.idx, st.count,
+                            n_vis, L, out2, lse2, ws)
+    torch.cuda.synchronize()
+    idx, cnt = st.idx.cpu().numpy(), st.count.cpu().numpy()
+    outs = []
+    for b in range(B):
+        pos = oracle.token_set(idx[b, :cnt[b]], L)
+        o, l = oracle.attention(bits_of(q2[b]), bits_of(lat2[b, torch.from_numpy(pos).cuda()]),
+                                st.w.sm_scale)
+        assert np.allclose(lse2[b].cpu().numpy(), l, atol=LSE_ATOL, rtol=0)
+        outs.append(o)
+    assert_attention_close(f64_of(out2), np.stack(outs), "indexshare")
