@@ -57,6 +57,12 @@ constexpr int kThreads = 192;
 constexpr int kEpi = 128;                    // epilogue threads
 constexpr int kHistBins = 2048;              // top 11 key bits
 constexpr int kHistShift = 21;
+// Decode work split: each CTA first takes an equal static range of 7/8 of the
+// tiles, then the rest in chunks of kDynChunk tiles from an atomic counter,
+// so that CTAs that stream faster take more and all finish together.
+constexpr int kDynChunk = 4;
+constexpr int kMaxDynGroups = 512;
+constexpr int kRing = 4;  // chunk indices handed from the TMA warp to the others
 
 template <int NQ, bool SELECT>
 struct Cfg {
@@ -92,6 +98,7 @@ struct KParams {
   int groups;
   int shared_keys;
   uint32_t* ghist;     // SELECT: [rows, kHistBins] key histogram, zero on entry
+  int* work_counter;   // zero on entry; NULL: static split only
 };
 
 template <int NQ>
@@ -139,6 +146,84 @@ struct Walker {
   }
 };
 
+// Shared description of the CTA's work: the static range, then (if enabled)
+// chunks of the dynamic pool taken by the TMA warp and posted in a ring.
+struct Sched {
+  int64_t lo;      // first static item
+  int n_static;    // static items
+  int g0, t0;      // (group, tile) of item lo
+  bool dyn;
+  int64_t dyn_begin, total;
+  int nchunk;
+  const int* pre;  // smem [groups + 1]: first flat tile of each group
+  int* ring;       // smem [kRing]
+  uint64_t* ring_full;
+  uint64_t* ring_empty;
+  int* counter;
+};
+
+enum Role { kProducer, kMmaRole, kEpiRole };
+
+// Yields the CTA's work items in order, the same sequence in every role.
+template <int NQ>
+struct WorkSrc {
+  Walker<NQ> w;
+  int left = 0;
+  bool started = false;
+  int slot = 0;
+  uint32_t ph = 0;
+
+  __device__ bool next(const KParams& p, const Sched& sc, Role role, int lane,
+                       volatile int* abort) {
+    if (!started) {
+      started = true;
+      if (sc.n_static > 0) {
+        w.init(p, sc.g0, sc.t0, sc.lo);
+        left = sc.n_static - 1;
+        return true;
+      }
+    } else if (left > 0) {
+      w.advance(p);
+      --left;
+      return true;
+    }
+    if (!sc.dyn) return false;
+    int k;
+    if (role == kProducer) {
+      if (!mbar_wait(&sc.ring_empty[slot], ph ^ 1, abort)) return false;
+      k = atomicAdd(sc.counter, 1);
+      if (k >= sc.nchunk) k = -1;
+      sc.ring[slot] = k;
+      mbar_arrive(&sc.ring_full[slot]);
+    } else {
+      if (!mbar_wait(&sc.ring_full[slot], ph, abort)) return false;
+      k = sc.ring[slot];
+      if (role == kMmaRole) {
+        mbar_arrive(&sc.ring_empty[slot]);
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sc.ring_empty[slot]);
+      }
+    }
+    if (++slot == kRing) {
+      slot = 0;
+      ph ^= 1;
+    }
+    if (k < 0) return false;
+    const int64_t f = sc.dyn_begin + static_cast<int64_t>(k) * kDynChunk;
+    const int64_t n = sc.total - f < kDynChunk ? sc.total - f : kDynChunk;
+    int lo_g = 0, hi_g = p.groups - 1;  // the group g with pre[g] <= f < pre[g+1]
+    while (lo_g < hi_g) {
+      const int mid = (lo_g + hi_g + 1) >> 1;
+      if (sc.pre[mid] <= f) lo_g = mid; else hi_g = mid - 1;
+    }
+    while (sc.pre[lo_g + 1] <= f) ++lo_g;  // skip groups without tiles
+    w.init(p, lo_g, static_cast<int>(f - sc.pre[lo_g]), f);
+    left = static_cast<int>(n) - 1;
+    return true;
+  }
+};
+
 __device__ __forceinline__ void epi_sync() { group_sync<kEpi, 1>(); }
 
 }  // namespace
@@ -168,6 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   __shared__ int s_scan[33];
   __shared__ int s_g0, s_t0;
+  __shared__ int s_pre[kMaxDynGroups + 1];
+  __shared__ int s_ring[kRing];
+  __shared__ __align__(8) uint64_t ring_bars[2 * kRing];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -177,34 +265,59 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();  // the next kernel's CTAs may be scheduled as SMs free up
   pdl_wait();     // lengths, keys and the histogram come from the previous kernel
 
-  // ---- locate this CTA's contiguous range of work items -------------------
+  // ---- this CTA's work: a contiguous static range, then dynamic chunks ----
+  const bool dyn = p.work_counter != nullptr && p.groups <= kMaxDynGroups;  // uniform
   int64_t total = 0;
   for (int base = 0; base < p.groups; base += kThreads) {
     const int g = base + tid;
     int sum;
-    block_excl_scan(g < p.groups ? group_tiles<NQ>(p, g) : 0, s_scan, &sum);
+    const int ex = block_excl_scan(g < p.groups ? group_tiles<NQ>(p, g) : 0, s_scan, &sum);
+    if (dyn && g < p.groups) s_pre[g] = static_cast<int>(total + ex);
     total += sum;
   }
+  if (dyn && tid == 0) s_pre[p.groups] = static_cast<int>(total);
   const int64_t G = gridDim.x;
-  const int64_t lo = total * blockIdx.x / G;
-  const int64_t hi = total * (blockIdx.x + 1) / G;
-  if (lo >= hi) return;  // uniform
-  {
+  Sched sc;
+  sc.dyn = dyn;
+  sc.total = total;
+  if (dyn) {
+    const int64_t per = total * 7 / (8 * G);
+    sc.lo = per * blockIdx.x;
+    sc.n_static = static_cast<int>(per);
+    sc.dyn_begin = per * G;
+    sc.nchunk = static_cast<int>((total - sc.dyn_begin + kDynChunk - 1) / kDynChunk);
+  } else {
+    sc.lo = total * blockIdx.x / G;
+    sc.n_static = static_cast<int>(total * (blockIdx.x + 1) / G - sc.lo);
+    sc.dyn_begin = total;
+    sc.nchunk = 0;
+    if (sc.n_static <= 0) return;  // uniform
+  }
+  sc.pre = s_pre;
+  sc.ring = s_ring;
+  sc.ring_full = ring_bars;
+  sc.ring_empty = ring_bars + kRing;
+  sc.counter = p.work_counter;
+  sc.g0 = 0;
+  sc.t0 = 0;
+  if (sc.n_static > 0) {
     int64_t run = 0;
     for (int base = 0; base < p.groups; base += kThreads) {
       const int g = base + tid;
       const int c = g < p.groups ? group_tiles<NQ>(p, g) : 0;
       int sum;
       const int ex = block_excl_scan(c, s_scan, &sum);
-      if (c > 0 && run + ex <= lo && lo < run + ex + c) {
+      if (c > 0 && run + ex <= sc.lo && sc.lo < run + ex + c) {
         s_g0 = g;
-        s_t0 = static_cast<int>(lo - run - ex);
+        s_t0 = static_cast<int>(sc.lo - run - ex);
       }
       run += sum;
-      if (run > lo) break;  // uniform
+      if (run > sc.lo) break;  // uniform
     }
+    __syncthreads();
+    sc.g0 = s_g0;
+    sc.t0 = s_t0;
   }
-  const int n_items = static_cast<int>(hi - lo);
 
   // ---- barriers and TMEM ---------------------------------------------------
   if (tid == 0) {
@@ -221,6 +334,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&accempty[s], 4);
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&ring_bars[s], 1);              // full: the TMA warp posted a chunk
+      mbar_init(&ring_bars[kRing + s], 1 + 4);  // empty: MMA thread + 4 epilogue warps read it
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -239,13 +356,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // per-row keys are read once (decode); keys shared by every query
       // group (prefill) are re-read from L2
       const uint64_t stream_pol = p.shared_keys ? l2_evict_normal_policy() : l2_evict_first_policy();
-      Walker<NQ> w;
-      w.init(p, s_g0, s_t0, lo);
+      WorkSrc<NQ> src;
+      const Walker<NQ>& w = src.w;
       int stage = 0, cur_g = -1, qs = C::kQSlots - 1;
       uint32_t ph = 0, qe_ph[2] = {0, 0};
       int issued = 0, q_issued_slot = -1;
       uint32_t q_issued_ph = 0;
-      for (int i = 0; i < n_items; ++i) {
+      while (src.next(p, sc, kProducer, lane, abort_flag)) {
         if (w.g != cur_g) {
           qs = (qs + 1) % C::kQSlots;
           if (!mbar_wait(&qempty[qs], qe_ph[qs] ^ 1, abort_flag)) break;
@@ -269,7 +386,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           stage = 0;
           ph ^= 1;
         }
-        w.advance(p);
       }
       if (*abort_flag) {
         // Let the copies already issued land before the CTA exits.
@@ -287,13 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ======================= MMA issuer ====================================
     if (lane == 0) {
-      Walker<NQ> w;
-      w.init(p, s_g0, s_t0, lo);
+      WorkSrc<NQ> src;
+      const Walker<NQ>& w = src.w;
       int stage = 0, acc = 0, cur_g = -1, qs = C::kQSlots - 1;
       uint32_t ph = 0, acc_ph = 0, qf_ph[2] = {0, 0};
       const uint32_t a_base = smem_u32(a_smem);
       const uint32_t q_base = smem_u32(q_smem);
-      for (int i = 0; i < n_items; ++i) {
+      while (src.next(p, sc, kMmaRole, lane, abort_flag)) {
         if (w.g != cur_g) {
           if (cur_g >= 0) umma_commit(&qempty[qs]);
           qs = (qs + 1) % C::kQSlots;
@@ -324,7 +440,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc = 0;
           acc_ph ^= 1;
         }
-        w.advance(p);
       }
       // Wait for every MMA issued by this thread before TMEM is released.
       umma_commit(drain);
@@ -336,8 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;  // TMEM lanes quarter*32 .. +31
     const int et = tid - 64;       // 0..127
     const int row_in_tile = quarter * 32 + lane;
-    Walker<NQ> w;
-    w.init(p, s_g0, s_t0, lo);
+    WorkSrc<NQ> src;
+    const Walker<NQ>& w = src.w;
     int acc = 0, cur_g = -1;
     uint32_t acc_ph = 0;
     bool aborted = false;
@@ -362,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       epi_sync();
     };
 
-    for (int i = 0; i < n_items; ++i) {
+    while (src.next(p, sc, kEpiRole, lane, abort_flag)) {
       if (w.g != cur_g) {
         if constexpr (SELECT) {
           if (cur_g >= 0) flush_hist(cur_g);
@@ -385,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int64_t blk = static_cast<int64_t>(w.t) * kTileM + row_in_tile;
-      float sc[NQ];
+      float scv[NQ];
 #pragma unroll 1
       for (int j = 0; j < NQ; ++j) {
         const int r = w.g * NQ + j;
@@ -400,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < kIdxHeads; ++h)
           s4[h & 3] = __fmaf_rn(wj[h], v[h] > 0.f ? v[h] : 0.f, s4[h & 3]);
-        sc[j] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        scv[j] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
       tc_fence_before();
       __syncwarp();
@@ -415,11 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = w.g * NQ + j;
         if (r >= p.rows) break;
         if (blk < nb_smem[j]) {
-          p.scores[static_cast<int64_t>(r) * p.score_stride + blk] = sc[j];
-          if constexpr (SELECT) atomicAdd(&lhist[order_key(sc[j]) >> kHistShift], 1u);
+          p.scores[static_cast<int64_t>(r) * p.score_stride + blk] = scv[j];
+          if constexpr (SELECT) atomicAdd(&lhist[order_key(scv[j]) >> kHistShift], 1u);
         }
       }
-      w.advance(p);
     }
     if constexpr (SELECT) {
       if (!aborted && cur_g >= 0) flush_hist(cur_g);
@@ -475,6 +589,7 @@ cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
   p.groups = (a.rows + NQ - 1) / NQ;
   p.shared_keys = a.key_batches == 1 ? 1 : 0;
   p.ghist = a.sel_ghist;
+  p.work_counter = a.work_counter;
   const int grid = score_grid(a.nq, a.rows, a.max_len, a.num_sms);
   if (grid == 0) return cudaSuccess;
   cudaError_t e = launch_ex(k_index_score<NQ, SELECT>, dim3(grid), dim3(kThreads), C::kSmem,

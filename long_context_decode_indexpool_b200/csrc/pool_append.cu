@@ -59,6 +59,7 @@ __global__ void __launch_bounds__(kPoolThreads)
       for (int i = threadIdx.x; i < kSelHistBins; i += kPoolThreads)
         init_hist[static_cast<int64_t>(b) * kSelHistBins + i] = 0u;
       if (threadIdx.x == 0) init_done[b] = 0;
+      if (threadIdx.x == 0 && b == 0) init_done[gridDim.y] = 0;  // the scoring work counter
     }
   }
   if (n_new <= 0) return;

@@ -136,7 +136,7 @@ FusedLayout fused_layout(int rows, int heads, int64_t max_len) {
 }
 
 // Workspace of the fused decode call:
-//   n_vis [B] | idx [B,512] | count [B] | key histogram [B,2048] | done [B]
+//   n_vis [B] | idx [B,512] | count [B] | key histogram [B,2048] | done [B+1]
 //   | scores [B, stride] | list keys, list ids [B*nchunk, 512]
 //   | list counts [B*nchunk] | attention scratch
 struct DecodeLayout {
@@ -165,8 +165,8 @@ DecodeLayout decode_layout(int B, int heads, int64_t max_len) {
   o += up(static_cast<size_t>(B) * 4);
   L.hist = o;
   o += up(static_cast<size_t>(B) * kSelHistBins * 4);
-  L.done = o;
-  o += up(static_cast<size_t>(B) * 4);
+  L.done = o;  // B chunk counters of the selection + the scoring work counter
+  o += up(static_cast<size_t>(B + 1) * 4);
   L.scores = o;
   o += up(static_cast<size_t>(B) * L.stride * 4);
   L.lkey = o;
@@ -451,6 +451,7 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   sa.score_stride = L.stride;
   sa.num_sms = device_sm_count();
   sa.sel_ghist = hist;
+  sa.work_counter = done + B;
   // Each kernel of the chain may start while its predecessor finishes (its
   // set-up overlaps; it waits before reading the predecessor's output),
   // except across a timing event.

@@ -31,7 +31,7 @@ struct PoolAppendArgs {
   int64_t max_len;
   int64_t* nvis_out;  // optional: receives len + n_new per sequence
   // optional per-sequence initialisation of the decode selection state:
-  // hist[b][..] = 0, done[b] = 0
+  // hist[b][..] = 0, done[b] = 0 for b < B, and done[B] = 0
   uint32_t* init_hist;
   int32_t* init_done;
 };
@@ -57,6 +57,7 @@ struct ScoreArgs {
   // a per-row histogram of their top 11 bits (zero on entry), the input of
   // launch_select_blocks.
   uint32_t* sel_ghist;  // [rows, kSelHistBins]
+  int* work_counter;    // optional, zero on entry: tiles are then shared out dynamically
   bool pdl;             // may start while the previous kernel finishes
 };
 constexpr int kSelHistBins = 2048;
