@@ -523,6 +523,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
             make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
+    if (n_cl > 1) {
+      // this warp's 16 rows (16 KiB, contiguous) go to L2 at once, while the
+      // other warps are still staging theirs
+      const int64_t first_row = (unit * n_cl + split) * kHG;
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        bulk_store(p.part_o + (first_row + warp * 16) * kLatent, stage_u + warp * 16 * 1024,
+                   16 * kLatent * 2);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+    }
   }
   if (n_cl == 1) {
     if (worker && half == 0 && h0 + hloc < p.heads && p.lse)
@@ -544,15 +556,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     // The staged rows (same layout in L2, one bulk copy) and (m, l) of this
     // split go to L2; the cluster barrier publishes them.
     const int64_t first_row = (unit * n_cl + split) * kHG;
-    if (ntiles > 0) {
-      fence_proxy_async();
-      __syncthreads();
-      if (tid == 0) {
-        bulk_store(p.part_o + first_row * kLatent, stage_u, kHG * kLatent * 2);
-        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-      }
+    if (ntiles > 0 && worker && lane == 0) {
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // this warp's rows are in L2
+      asm volatile("fence.proxy.async.global;" ::: "memory");
     }
     if (worker && half == 0) {
       float* pm = p.part_ml + (first_row + hloc) * 2;
