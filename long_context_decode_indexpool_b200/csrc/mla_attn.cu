@@ -71,7 +71,8 @@ constexpr int kMaxList = kTopK * kPool + kPool - 1;             // tokens in a l
 constexpr int kPosCap = (kMaxList + kTT - 1) / kTT * kTT;       // position slots
 constexpr int kMaxCluster = 16;                 // splits per (row, head group)
 constexpr int kSmemBytes = 1024 + kQBytes + 2 * kKVBytes + kPBytes + kPosCap * 8 +
-                           (kPosCap / 32) * 4 + kHG * 2 * 4 + 64;
+                           (kPosCap / 32) * 4 + 64;
+static_assert(((kPosCap * 8 + (kPosCap / 32) * 4) & 7) == 0, "barriers 8-byte aligned");
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLazy = 8.f;                    // rescale threshold (log2 units)
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, kTT);
@@ -230,8 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   uint8_t* p_s = kv_s + 2 * kKVBytes;
   int64_t* pos_s = reinterpret_cast<int64_t*>(p_s + kPBytes);     // [kPosCap]
   uint32_t* vm_s = reinterpret_cast<uint32_t*>(pos_s + kPosCap);  // [kPosCap / 32] valid bits
-  float* ml_s = reinterpret_cast<float*>(vm_s + kPosCap / 32);    // [64][2] (spare)
-  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(ml_s + 2 * kHG);  // [2]: S buffer b done
+  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(vm_s + kPosCap / 32);  // [2]: S buffer b done
   uint64_t* bar_pv = bar_qk + 2;
   uint64_t* bar_red = bar_qk + 3;  // combine: rows of the other splits
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 4);

@@ -112,6 +112,12 @@ def test_host_validation_rejects_before_launch(spx):
         spx.spx_decode_fused(d, 4, FAKE, [0.25] * 4, FAKE, FAKE, 2048, FAKE, FAKE, FAKE, FAKE,
                              FAKE, 8192, 8192, FAKE, ws=FAKE, ws_bytes=need - 256, stream=s)
     assert e.value.status == 4
+    # fused decode beyond 16M tokens per sequence: unsupported (512 selection chunks)
+    big = (1 << 24) + 4
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_decode_fused(d, 1, FAKE, [0.25] * 4, FAKE, FAKE, big // 4, FAKE, FAKE, FAKE, FAKE,
+                             FAKE, big, big, FAKE, ws=FAKE, ws_bytes=1 << 40, stream=s)
+    assert e.value.status == 3
     # prefill beyond the caches
     with pytest.raises(spx.SpxError) as e:
         spx.spx_prefill_chunk(d, 64, FAKE, [0.25] * 4, FAKE, FAKE, 16, 10, FAKE, FAKE, FAKE, FAKE,
