@@ -656,6 +656,49 @@ def run_indexshare(args, world, rank, local):
                        "context": L, "heads": H}}
 
 
+def run_host_latent(args, world, rank, local):
+    """Decode with the latent cache in pinned host memory ([W3] "HiSparse는 전체
+    이력을 GPU 밖으로 옮긴다": the full history lives off the GPU and only the
+    selected rows are fetched): the attention reads the 2048 selected rows per
+    query through the host link; pooled keys stay in HBM."""
+    spx = spx_module()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = synth.workload(args.workload)
+    st = DecodeState(w, device, b_offset=shard_offset(rank, w.B))
+    host_lat = st.latent.cpu().pin_memory()
+    st.latent = None  # the device copy is released; the call reads the host rows
+    torch.cuda.empty_cache()
+    st.latent = host_lat  # step() passes its data_ptr (mapped under unified addressing)
+    st._call = None
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        st.step()
+    torch.cuda.synchronize(device)
+    K = args.steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    ev0.record(stream)
+    for _ in range(K):
+        st.step()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
+    if spx.spx_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    if rank != 0:
+        return None
+    rows_bytes = st.B * (synth.TOPK_BLOCKS * synth.POOL) * synth.LATENT * 2
+    return {"metric": "decode queries/s with the latent cache in pinned host memory",
+            "value": st.B * world * K / (ms * 1e-3), "unit": "queries/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+            "scaling": "weak", "dtype": "bf16", "data": "synthetic",
+            "host_rows_gbs": rows_bytes / (ms / K * 1e-3) / 1e9,
+            "config": {"workload": w.name, "latent": "pinned host memory",
+                       "batch_per_gpu": st.B, "context": st.L}}
+
+
 def run_prefill(args, world, rank, local):
     spx = spx_module()
     device = torch.device("cuda", local)
@@ -760,6 +803,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("spx", "reference"), default="spx")
     ap.add_argument("--workload", default="1m", choices=synth.WORKLOADS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--host-latent", action="store_true",
+                    help="decode with the latent cache in pinned host memory")
     ap.add_argument("--indexshare", type=int, default=0, metavar="N",
                     help="IndexShare decode: one indexer per N layers (reports per-layer rate)")
     ap.add_argument("--score-only", action="store_true",
@@ -776,13 +821,16 @@ def main(argv=None):
             line = run_score_only(args, world, rank, local)
         elif args.indexshare > 1:
             line = run_indexshare(args, world, rank, local)
+        elif args.host_latent:
+            line = run_host_latent(args, world, rank, local)
         elif args.workload == "prefill":
             line = run_prefill(args, world, rank, local)
         else:
             line = run_decode(args, world, rank, local)
         if rank == 0 and line is not None:
             if (world == 1 and not args.no_cpu_baseline and args.workload != "prefill"
-                    and not args.score_only and args.indexshare <= 1):
+                    and not args.score_only and args.indexshare <= 1
+                    and not args.host_latent):
                 line["cpu_baseline"] = cpu_baseline(synth.workload(args.workload),
                                                     torch.device("cuda", local))
             print(json.dumps(line))

@@ -307,3 +307,26 @@ def test_indexshare_other_layer_on_shared_selection():
         assert np.allclose(lse2[b].cpu().numpy(), l, atol=LSE_ATOL, rtol=0)
         outs.append(o)
     assert_attention_close(f64_of(out2), np.stack(outs), "indexshare")
+
+
+def test_host_resident_latent_cache_is_bit_identical():
+    """HiSparse-style host-resident latent cache: the attention reads the
+    selected rows straight from pinned host memory; the result is the same,
+    bit for bit, as with the cache in HBM."""
+    spx = need_gpu()
+    st = _decode_state("tiny")
+    st.step()
+    torch.cuda.synchronize()
+    out_dev, lse_dev, idx_dev = st.out.clone(), st.lse.clone(), st.idx.clone()
+    host_lat = st.latent.cpu().pin_memory()  # mapped into the device's address space (UVA)
+    out = torch.empty_like(st.out)
+    lse = torch.empty_like(st.lse)
+    len_after = torch.full((st.B,), st.L, dtype=torch.int64, device="cuda")
+    spx.spx_decode_fused(st.d, st.B, None, None, st.tail, st.pooled, st.cap_blk, len_after,
+                         st.q_idx, st.w_head, st.q, host_lat.data_ptr(), st.cap_tok, st.L, out,
+                         lse, st.idx, st.count, st.ws)
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    assert torch.equal(st.idx, idx_dev)
+    assert torch.equal(out.view(torch.int16), out_dev.view(torch.int16))
+    assert torch.equal(lse, lse_dev)
