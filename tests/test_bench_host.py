@@ -1,0 +1,40 @@
+"""Host-side pieces of bench.py (no GPU): the algorithmic byte count the
+roofline uses, the clock-record summary and the recorded-traffic lookup."""
+import bench
+import synth
+
+
+def test_algorithmic_bytes_of_the_1m_scoring_launch():
+    w = synth.workload("1m")
+    nblk = [w.L // synth.POOL] * w.B
+    # 4 x 262,144 blocks x (256 B key + 4 B score) + 4 x (8 KiB query + 128 B weights)
+    assert bench.score_algorithmic_bytes(nblk, w.B) == 272_663_040
+
+
+def test_prefill_flops_count_the_causal_blocks():
+    # query t sees (pos0 + t + 1) // 4 complete blocks; 2 x 32 x 128 flop per block
+    assert bench.score_algorithmic_flops_prefill(8, 4) == 2 * 32 * 128 * (2 + 2 + 2 + 3)
+
+
+def _sampler(lines):
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples = list(lines)
+    return s
+
+
+def test_clock_summary_reports_median_and_active_reasons():
+    ok = "0, 1965, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Not Active"
+    capped = "0, 1800, 1965, 999.0, 0x4, Not Active, Not Active, Not Active, Active"
+    summ = _sampler([ok, capped, ok]).summary()
+    assert summ["sm_mhz"] == 1965.0 and summ["sm_max_mhz"] == 1965.0
+    assert summ["reasons"] == ["sw_power_cap"]
+    assert summ["samples"] == 3
+    hot = "0, 1500, 1965, 999.0, 0x40, Not Active, Active, Not Active, Not Active"
+    assert "hw_thermal_slowdown" in _sampler([hot]).summary()["reasons"]
+
+
+def test_recorded_traffic_matches_only_the_current_kernel_source():
+    t = bench.recorded_traffic("decode_1m")
+    alg = bench.score_algorithmic_bytes([262144] * 4, 4)
+    assert t is None or alg <= t < 1.05 * alg  # recorded for this source, no re-reads
+    assert bench.recorded_traffic("no such workload") is None
