@@ -647,43 +647,51 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   if (warp == 0) tmem_dealloc(*tmem_holder, 512);
 }
 
-// Largest cluster size n <= want (a power of two) for which the device can
-// run at least one cluster of the attention kernel.
-int max_cluster(int want) {
+// Number of clusters of n CTAs of the attention kernel the device can hold
+// at once (cached per device).
+int active_clusters(int n) {
   static int cache[64][5];
   static bool done[64][5];
   int dev = 0;
   cudaGetDevice(&dev);
-  for (int n = want; n > 1; n >>= 1) {
-    int lg = 0;
-    while ((1 << lg) < n) ++lg;
-    if (dev < 64 && done[dev][lg]) {
-      if (cache[dev][lg] > 0) return n;
-      continue;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(n, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = n;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    int num = 0;
-    if (cudaOccupancyMaxActiveClusters(&num, k_sparse_attn, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      num = 0;
-    }
-    if (dev < 64) {
-      done[dev][lg] = true;
-      cache[dev][lg] = num;
-    }
-    if (num > 0) return n;
+  int lg = 0;
+  while ((1 << lg) < n) ++lg;
+  if (dev < 64 && done[dev][lg]) return cache[dev][lg];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = n;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int num = 0;
+  if (cudaOccupancyMaxActiveClusters(&num, k_sparse_attn, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    num = 0;
   }
-  return 1;
+  if (dev < 64) {
+    done[dev][lg] = true;
+    cache[dev][lg] = num;
+  }
+  return num;
+}
+
+// Cluster size for `units` (row, head group) pairs, at most `want` (a power
+// of two): the largest size whose clusters all fit on the device at once (a
+// second wave of clusters would double the time), else the largest that fits
+// at all.
+int pick_cluster(int want, int64_t units) {
+  int fits_at_all = 1;
+  for (int n = want; n > 1; n >>= 1) {
+    const int num = active_clusters(n);
+    if (num >= units) return n;
+    if (num > 0 && fits_at_all == 1) fits_at_all = n;
+  }
+  return fits_at_all;
 }
 
 bool set_attrs() {
@@ -733,7 +741,7 @@ cudaError_t launch_attn(const AttnPlan& pl0, const AttnArgs& a, cudaStream_t str
   if (!set_attrs()) return cudaGetLastError();
   AttnPlan pl = pl0;
   if (pl.nsplit > 1) {
-    const int n = max_cluster(pl.nsplit);
+    const int n = pick_cluster(pl.nsplit, static_cast<int64_t>(pl.rows) * pl.groups);
     if (n != pl.nsplit) {  // fewer, longer splits
       const int64_t total = static_cast<int64_t>(pl.split_tokens) * pl.nsplit;
       int64_t ts = (total + n - 1) / n;
