@@ -228,12 +228,18 @@ SPX_API spx_status spx_topk_blocks_noalloc(const spx_dims* d, int32_t rows,
  *
  *   q         bf16 [rows, heads, latent]
  *   latent    bf16; row r reads tokens latent + r*seq_stride + t*latent,
- *             t < cap_tok (seq_stride 0: all rows share one cache)
- *   idx,count as produced by spx_topk_blocks
+ *             t < cap_tok (seq_stride 0: all rows share one cache).  Device
+ *             memory or pinned host memory mapped into the device's address
+ *             space (only the selected rows are read)
+ *   idx,count as produced by spx_topk_blocks (or by an earlier layer's
+ *             spx_decode_fused: one selection may serve several layers)
  *   n_vis     DEVICE int64 [rows]   (clamped to min(max_len, cap_tok))
  *   out       bf16 [rows, heads, latent]
  *   lse       float [rows, heads] or NULL
  *   ws        workspace of spx_attn_workspace_size(d, rows, max_len) bytes
+ *             (zero when each row runs in one CTA; otherwise the splits of a
+ *             row combine through it: their rows normalised by their own
+ *             softmax sum, in bf16, and their (max, sum) in fp32)
  * ------------------------------------------------------------------------- */
 SPX_API spx_status spx_attn_workspace_size(const spx_dims* d, int32_t rows,
                                    int64_t max_len, size_t* bytes);
