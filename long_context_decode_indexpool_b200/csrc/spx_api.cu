@@ -103,21 +103,25 @@ inline int64_t score_stride_for(int64_t max_len) {
   return (mb + 63) / 64 * 64;
 }
 
-// Workspace of the fused calls:
+// Workspace of the prefill call:
 //   n_vis [rows] int64 | scores [rows, stride] f32 | idx [rows, 512] | count [rows]
-//   | top-k scratch | attention scratch
+//   | key histograms [rows, 2048] | chunk counters [rows] | list keys, list
+//   ids [rows*nchunk, 512] | list counts [rows*nchunk] | attention scratch
 struct FusedLayout {
-  size_t nvis, scores, idx, count, topk, attn, total;
+  size_t nvis, scores, idx, count, hist, done, lkey, lidx, lcnt, attn, total;
   int64_t stride;
-  TopkPlan tp;
+  int nchunk;
   AttnPlan ap;
 };
 
 FusedLayout fused_layout(int rows, int heads, int64_t max_len) {
   FusedLayout L{};
   L.stride = score_stride_for(max_len);
-  L.tp = plan_topk(rows, max_len);
+  const int64_t max_blk = max_len / kPool;
+  L.nchunk = static_cast<int>((max_blk + kSelChunk - 1) / kSelChunk);
+  if (L.nchunk < 1) L.nchunk = 1;
   L.ap = plan_attn(rows, heads, max_len, device_sm_count());
+  const size_t lists = static_cast<size_t>(rows) * L.nchunk;
   size_t o = 0;
   L.nvis = o;
   o += up(static_cast<size_t>(rows) * 8);
@@ -127,8 +131,16 @@ FusedLayout fused_layout(int rows, int heads, int64_t max_len) {
   o += up(static_cast<size_t>(rows) * kTopK * 4);
   L.count = o;
   o += up(static_cast<size_t>(rows) * 4);
-  L.topk = o;
-  o += up(L.tp.ws_bytes);
+  L.hist = o;
+  o += up(static_cast<size_t>(rows) * kSelHistBins * 4);
+  L.done = o;
+  o += up(static_cast<size_t>(rows) * 4);
+  L.lkey = o;
+  o += up(lists * kTopK * 4);
+  L.lidx = o;
+  o += up(lists * kTopK * 4);
+  L.lcnt = o;
+  o += up(lists * 4);
   L.attn = o;
   o += up(L.ap.ws_bytes);
   L.total = o;
@@ -528,10 +540,13 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
       (idx_out && !al4(idx_out)) || (count_out && !al4(count_out)))
     return SPX_ERR_INVALID_ARG;
   const FusedLayout L = fused_layout(T, d->heads, max_len);
+  if (L.nchunk > kMaxSelChunks) return SPX_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < L.total || !al16(ws)) return SPX_ERR_WORKSPACE;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
+  // the selection's key histograms and chunk counters start at zero
+  if (cudaMemsetAsync(base + L.hist, 0, L.lkey - L.hist, s) != cudaSuccess) return SPX_ERR_CUDA;
   int64_t* n_vis = reinterpret_cast<int64_t*>(base + L.nvis);
   float* scores = reinterpret_cast<float*>(base + L.scores);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + L.idx);
@@ -574,9 +589,25 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
     return SPX_ERR_CUDA;
 
-  if ((e = launch_topk(L.tp, scores, L.stride, n_vis, max_len, idx, count, base + L.topk, s)) !=
-      cudaSuccess)
-    return SPX_ERR_CUDA;
+  // top-512 per query: key histograms of the scores, then the chunked
+  // selection with the exact cut bin (as in decode)
+  SelectBlocksArgs ma{};
+  ma.rows = T;
+  ma.scores = scores;
+  ma.score_stride = L.stride;
+  ma.n_vis = n_vis;
+  ma.max_len = max_len;
+  ma.ghist = reinterpret_cast<uint32_t*>(base + L.hist);
+  ma.nchunk = L.nchunk;
+  ma.list_key = reinterpret_cast<uint32_t*>(base + L.lkey);
+  ma.list_idx = reinterpret_cast<int32_t*>(base + L.lidx);
+  ma.list_cnt = reinterpret_cast<int32_t*>(base + L.lcnt);
+  ma.done = reinterpret_cast<int32_t*>(base + L.done);
+  ma.out_idx = idx;
+  ma.out_cnt = count;
+  ma.pdl = false;
+  if ((e = launch_key_hist(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
+  if ((e = launch_select_blocks(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
 
   AttnArgs aa{};
   aa.q = q;

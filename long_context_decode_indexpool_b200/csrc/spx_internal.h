@@ -89,6 +89,10 @@ struct SelectBlocksArgs {
   bool pdl;
 };
 cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream);
+// Fills the rows' key histograms (ghist, zero on entry) from scores written
+// without one (prefill); uses rows, scores, score_stride, n_vis, max_len,
+// ghist, nchunk and pdl of the same arguments.
+cudaError_t launch_key_hist(const SelectBlocksArgs& a, cudaStream_t stream);
 
 // Top-k blocks.
 struct TopkPlan {

@@ -268,6 +268,40 @@ __device__ __noinline__ void merge_final(const uint32_t* bk, const int32_t* bi, 
   if (tid == 0) *cnt_out = n;
 }
 
+// Key histogram of scores written by another kernel (prefill): grid
+// (chunks of kSelChunk, rows); each CTA counts its chunk's keys in shared
+// memory and adds the non-zero bins into the row's histogram (zero on entry).
+__global__ void __launch_bounds__(kThreads)
+    k_key_hist(const float* __restrict__ scores, int64_t score_stride,
+               const int64_t* __restrict__ n_vis, int64_t max_len, uint32_t* __restrict__ ghist) {
+  __shared__ uint32_t hist[kSelBins];
+  const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x;
+  pdl_trigger();
+  for (int b = tid; b < kSelBins; b += kThreads) hist[b] = 0;
+  pdl_wait();  // the scores come from the scoring kernel
+  const int64_t nblk = clamp_blocks(n_vis, r, max_len);
+  const int64_t b0 = static_cast<int64_t>(c) * kSelChunk + tid * 16;
+  const float* row = scores + static_cast<int64_t>(r) * score_stride;
+  float4 sv[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)  // rows are padded to a multiple of 4 scores
+    sv[q] = b0 + 4 * q < nblk ? __ldcg(reinterpret_cast<const float4*>(row + b0 + 4 * q))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float4 v = sv[i >> 2];
+    const float f = (i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w;
+    if (b0 + i < nblk) atomicAdd(&hist[order_key(f) >> kSelShift], 1u);
+  }
+  __syncthreads();
+  uint32_t* gh = ghist + static_cast<int64_t>(r) * kSelBins;
+  for (int b = tid; b < kSelBins; b += kThreads) {
+    const uint32_t n = hist[b];
+    if (n) atomicAdd(gh + b, n);
+  }
+}
+
 // Decode selection from the row's scores and its complete key histogram.
 // Grid (nchunk, rows), one CTA per chunk of kSelChunk scores (16 per thread):
 //   1. the histogram gives the bin of the row's 512th-largest key (every CTA
@@ -483,6 +517,17 @@ cudaError_t launch_merge_e(dim3 grid, cudaStream_t s, const uint32_t* ik, const 
 }
 
 }  // namespace
+
+cudaError_t launch_key_hist(const SelectBlocksArgs& a, cudaStream_t stream) {
+  if (a.rows == 0 || a.nchunk == 0) return cudaSuccess;
+  if ((a.score_stride & 3) != 0) return cudaErrorInvalidValue;
+  cudaError_t e = launch_ex(k_key_hist, dim3(a.nchunk, a.rows), dim3(kThreads), 0, stream, a.pdl,
+                            1, a.scores, a.score_stride, a.n_vis, a.max_len,
+                            const_cast<uint32_t*>(a.ghist));
+  count_launches(1);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream) {
   if (a.rows == 0 || a.nchunk == 0) return cudaSuccess;
