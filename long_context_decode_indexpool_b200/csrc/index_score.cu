@@ -40,6 +40,8 @@
 // Every wait is bounded; on a timeout the CTA drains and exits with the
 // device error word set.
 #include "select.cuh"
+#include <atomic>
+
 #include "spx_device.cuh"
 #include "spx_internal.h"
 #include "spx_launch.cuh"
@@ -570,7 +572,7 @@ cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
                            box, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {

@@ -43,6 +43,8 @@
 // splits with bulk copies and combines them with the log-sum-exp rule
 // (weights 2^(m_s - M) l_s / L) into the bf16 output and the log-sum-exp.
 // No second kernel runs.
+#include <atomic>
+
 #include "spx_device.cuh"
 #include "spx_internal.h"
 #include "spx_launch.cuh"
@@ -650,13 +652,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
 // Number of clusters of n CTAs of the attention kernel the device can hold
 // at once (cached per device).
 int active_clusters(int n) {
-  static int cache[64][5];
-  static bool done[64][5];
+  static std::atomic<int> cache[64][5];  // count + 1; 0: not queried yet
   int dev = 0;
   cudaGetDevice(&dev);
   int lg = 0;
   while ((1 << lg) < n) ++lg;
-  if (dev < 64 && done[dev][lg]) return cache[dev][lg];
+  if (dev < 64 && cache[dev][lg].load() > 0) return cache[dev][lg].load() - 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -673,10 +674,7 @@ int active_clusters(int n) {
     cudaGetLastError();
     num = 0;
   }
-  if (dev < 64) {
-    done[dev][lg] = true;
-    cache[dev][lg] = num;
-  }
+  if (dev < 64) cache[dev][lg].store(num + 1);
   return num;
 }
 
@@ -695,7 +693,7 @@ int pick_cluster(int want, int64_t units) {
 }
 
 bool set_attrs() {
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && attr_set[dev]) return true;

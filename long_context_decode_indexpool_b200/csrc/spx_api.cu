@@ -62,10 +62,10 @@ std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 int device_sm_count() {
-  static int cache[64] = {};
+  static std::atomic<int> cache[64];  // zero-initialised: not queried yet
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  if (dev >= 0 && dev < 64 && cache[dev].load()) return cache[dev].load();
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     n = 148;

@@ -20,6 +20,8 @@
 // writes the row's block ids, ascending, padded with -1.
 // The K best of a union are among the K best of each part, under the same
 // strict order, so the result equals a full sort of the row.
+#include <atomic>
+
 #include "select.cuh"
 #include "spx_internal.h"
 #include "spx_launch.cuh"
@@ -533,7 +535,7 @@ cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream)
   if (a.rows == 0 || a.nchunk == 0) return cudaSuccess;
   if (a.nchunk > kThreads || (a.score_stride & 3) != 0) return cudaErrorInvalidValue;
   constexpr int kSmem = pad32(kMergeCap) * 8;
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
