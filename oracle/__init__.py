@@ -53,6 +53,12 @@ def _load():
             lib.orc_pool.restype = None
             lib.orc_score.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P, i64, P, ctypes.c_int]
             lib.orc_score.restype = None
+            lib.orc_quant_i8.argtypes = [P, ctypes.c_int, P]
+            lib.orc_quant_i8.restype = ctypes.c_int
+            lib.orc_pool_i8.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P, P, P]
+            lib.orc_pool_i8.restype = None
+            lib.orc_score_i8.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P, P, i64, P, ctypes.c_int]
+            lib.orc_score_i8.restype = None
             lib.orc_topk.argtypes = [P, i64, i64, P]
             lib.orc_topk.restype = i64
             lib.orc_token_set.argtypes = [P, i64, i64, ctypes.c_int, P]
@@ -104,6 +110,44 @@ def score(q_bits: np.ndarray, w_head, keys_bits: np.ndarray, nthreads: int = 0) 
     out = np.zeros(nblk, dtype=np.float64)
     if nblk:
         _load().orc_score(_p(q), _p(w), heads, dim, _p(keys), nblk, _p(out), nthreads)
+    return out
+
+
+def quant_i8(x) -> tuple[np.ndarray, int]:
+    """INT8 code of one vector: (int8 codes, e) with x ~= 2^e * codes."""
+    v = np.ascontiguousarray(x, dtype=np.float64).reshape(-1)
+    codes = np.zeros(v.size, dtype=np.int8)
+    e = _load().orc_quant_i8(_p(v), v.size, _p(codes))
+    return codes, int(e)
+
+
+def pool_i8(raw_bits: np.ndarray, w, pool_size: int = POOL):
+    """IndexPool into the INT8 cache: [n_tok, dim] raw bf16 keys ->
+    (codes [n_tok // pool, dim] int8, scale [n_tok // pool] fp64)."""
+    raw = np.ascontiguousarray(raw_bits, dtype=np.uint16)
+    n_tok, dim = raw.shape
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    assert w.shape == (pool_size,)
+    nblk = n_tok // pool_size
+    codes = np.zeros((nblk, dim), dtype=np.int8)
+    scale = np.zeros(nblk, dtype=np.float64)
+    _load().orc_pool_i8(_p(raw), n_tok, dim, pool_size, _p(w), _p(codes), _p(scale))
+    return codes, scale
+
+
+def score_i8(q_bits: np.ndarray, w_head, codes: np.ndarray, scale, nthreads: int = 0) -> np.ndarray:
+    """Indexer scores [nblk] (fp64) of one query [heads, dim] against the INT8 cache."""
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    heads, dim = q.shape
+    w = np.ascontiguousarray(w_head, dtype=np.float64)
+    assert w.shape == (heads,)
+    c = np.ascontiguousarray(codes, dtype=np.int8)
+    sc = np.ascontiguousarray(scale, dtype=np.float64)
+    nblk = c.shape[0] if c.size else 0
+    assert nblk == 0 or (c.shape[1] == dim and sc.shape == (nblk,))
+    out = np.zeros(nblk, dtype=np.float64)
+    if nblk:
+        _load().orc_score_i8(_p(q), _p(w), heads, dim, _p(c), _p(sc), nblk, _p(out), nthreads)
     return out
 
 

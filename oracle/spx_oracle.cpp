@@ -25,7 +25,9 @@
 //
 // Every floating-point step is done in fp64.  The only roundings are the
 // ones the method's storage formats impose: the pooled key is stored as
-// bf16 (one round-to-nearest-even of the exact fp64 sum), and the top-k
+// bf16 (one round-to-nearest-even of the exact fp64 sum) or, in the INT8
+// cache, as int8 codes of that sum (one round-half-even after an exact
+// power-of-two scaling; the query heads likewise), and the top-k
 // decision is taken on the score rounded to fp32, the precision in which
 // scores are stored and ranked on the device.
 
@@ -111,6 +113,88 @@ void orc_score(const uint16_t* q, const double* w_head, int heads, int dim,
         s += w_head[h] * (dot > 0.0 ? dot : 0.0);
       }
       out[b] = s;
+    }
+  };
+  const int nt = pick_threads(nthreads);
+  if (nt <= 1 || nblk < 4096) {
+    work(0, nblk);
+    return;
+  }
+  std::vector<std::thread> pool;
+  for (int t = 0; t < nt; ++t) {
+    int64_t b0 = nblk * t / nt, b1 = nblk * (t + 1) / nt;
+    pool.emplace_back(work, b0, b1);
+  }
+  for (auto& th : pool) th.join();
+}
+
+// ---- INT8 pooled-key cache --------------------------------------------------
+// [W1] section "양자화: W8A8와 혼합 캐시": the indexer's far, compressed cache
+// entries are kept in INT8.  The page gives no scale convention; the reading
+// followed here: a vector x (one pooled block, or one query head) is stored
+// as symmetric codes c_i = round-half-even(x_i / 2^e) with one power-of-two
+// scale 2^e, e the smallest integer with max_i |x_i| <= 127 * 2^e (so every
+// |c_i| <= 127), e not below -149 (the smallest fp32 power of two); an
+// all-zero vector takes e = 0.
+
+// Returns e and writes the n codes.  The exponent is found by walking down
+// from one that satisfies the bound (amax < 2^(ilogb(amax) + 1)) until one
+// step further would break it.
+int orc_quant_i8(const double* x, int n, int8_t* codes) {
+  double amax = 0.0;
+  for (int i = 0; i < n; ++i) amax = std::max(amax, std::fabs(x[i]));
+  int e = 0;
+  if (amax > 0.0) {
+    e = std::ilogb(amax) + 1;
+    while (e > -149 && amax <= 127.0 * std::ldexp(1.0, e - 1)) --e;
+  }
+  for (int i = 0; i < n; ++i) {
+    const double c = std::nearbyint(std::ldexp(x[i], -e));  // exact scaling, then RNE
+    codes[i] = static_cast<int8_t>(c);
+  }
+  return e;
+}
+
+// IndexPool write into the INT8 cache: the exact pooled sum of each complete
+// block (as orc_pool, before any bf16 rounding) quantised per block; scale[b]
+// receives 2^e of block b.
+void orc_pool_i8(const uint16_t* raw, int64_t n_tok, int dim, int pool, const double* w,
+                 int8_t* codes, double* scale) {
+  const int64_t nblk = n_tok / pool;
+  std::vector<double> acc(dim);
+  for (int64_t b = 0; b < nblk; ++b) {
+    for (int d = 0; d < dim; ++d) {
+      double s = 0.0;
+      for (int i = 0; i < pool; ++i) s += w[i] * bf16_to_f64(raw[(b * pool + i) * dim + d]);
+      acc[d] = s;
+    }
+    scale[b] = std::ldexp(1.0, orc_quant_i8(acc.data(), dim, codes + b * dim));
+  }
+}
+
+// Indexer score against the INT8 cache: every query head h is quantised the
+// same way (codes qc_h, scale 2^{e_h}); then
+//   s[b] = scale[b] * sum_h w_h 2^{e_h} max(0, sum_d qc_h[d] * kc_b[d]),
+// i.e. the score of the dequantised query against the dequantised key.
+void orc_score_i8(const uint16_t* q, const double* w_head, int heads, int dim,
+                  const int8_t* codes, const double* scale, int64_t nblk, double* out,
+                  int nthreads) {
+  std::vector<int8_t> qc(static_cast<size_t>(heads) * dim);
+  std::vector<double> qs(heads), row(dim);
+  for (int h = 0; h < heads; ++h) {
+    for (int d = 0; d < dim; ++d) row[d] = bf16_to_f64(q[h * dim + d]);
+    qs[h] = std::ldexp(1.0, orc_quant_i8(row.data(), dim, qc.data() + h * dim));
+  }
+  auto work = [&](int64_t b0, int64_t b1) {
+    for (int64_t b = b0; b < b1; ++b) {
+      double s = 0.0;
+      for (int h = 0; h < heads; ++h) {
+        double dot = 0.0;
+        for (int d = 0; d < dim; ++d)
+          dot += static_cast<double>(qc[h * dim + d]) * static_cast<double>(codes[b * dim + d]);
+        s += w_head[h] * qs[h] * (dot > 0.0 ? dot : 0.0);
+      }
+      out[b] = scale[b] * s;
     }
   };
   const int nt = pick_threads(nthreads);

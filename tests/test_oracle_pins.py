@@ -382,3 +382,142 @@ def test_generator_scores_are_exact_in_fp32():
         partial = np.cumsum(np.maximum(dots, 0) * wh, axis=1)
         assert partial.max() < 2 ** 16
         assert np.array_equal(s * 256, np.round(s * 256))
+
+
+# ----------------------------------------------------------------------------
+# INT8 pooled-key cache
+# ----------------------------------------------------------------------------
+def test_quant_i8_closed_forms():
+    # values already on the grid with max |x| in [64, 127]: scale 1, codes = x
+    x = np.array([127, -64, 3, 0, -1, 100], np.float64)
+    c, e = oracle.quant_i8(x)
+    assert e == 0 and c.tolist() == x.astype(int).tolist()
+    # half-way cases go to the even code
+    c, e = oracle.quant_i8([127, 0.5, 1.5, 2.5, -2.5, -3.5])
+    assert e == 0 and c.tolist() == [127, 0, 2, 2, -2, -4]
+    # 127 * 2^e itself keeps that e; just above it needs e + 1
+    assert oracle.quant_i8([127 * 2.0 ** -5])[1] == -5
+    c, e = oracle.quant_i8([127.5, 1.0, 3.0])
+    assert e == 1 and c.tolist() == [64, 0, 2]
+    # the workload's query range: |q| <= 4 -> 2^-4, codes 16 q
+    c, e = oracle.quant_i8([4, -3, 1, 0.5])
+    assert e == -4 and c.tolist() == [64, -48, 16, 8]
+    # an all-zero vector: e = 0, zero codes
+    c, e = oracle.quant_i8(np.zeros(128))
+    assert e == 0 and not c.any()
+
+
+def test_quant_i8_invariants_random():
+    rng = np.random.default_rng(21)
+    for t in range(300):
+        mag = 2.0 ** rng.integers(-60, 60)
+        x = (rng.standard_normal(128) * mag).astype(np.float32).astype(np.float64)
+        if t % 7 == 0:
+            x[rng.integers(0, 128, 40)] = 0.0
+        c, e = oracle.quant_i8(x)
+        ci = c.astype(np.int64)
+        amax = np.abs(x).max()
+        # e is the smallest exponent that keeps every code within 127
+        assert amax <= 127 * 2.0 ** e and amax > 127 * 2.0 ** (e - 1)
+        assert 64 <= np.abs(ci).max() <= 127
+        # one rounding of an exact scaling: error at most half a step
+        assert (np.abs(x - ci * 2.0 ** e) <= 2.0 ** (e - 1)).all()
+        # a power-of-two change of the input only moves the exponent
+        c2, e2 = oracle.quant_i8(x * 2.0 ** 9)
+        assert e2 == e + 9 and np.array_equal(c2, c)
+
+
+def _grid_ints(rng, shape):
+    """Integers in [-127, 127] with every row's max |x| in [64, 127]."""
+    v = rng.integers(-127, 128, shape)
+    v[..., 0] = rng.choice([-1, 1], shape[:-1]) * rng.integers(64, 128, shape[:-1])
+    return v
+
+
+def test_pool_i8_on_grid_and_one_hot():
+    rng = np.random.default_rng(22)
+    key = _grid_ints(rng, (20, 128)).astype(np.float32)
+    raw = bits_of(np.repeat(key, POOL, axis=0))
+    # identical keys pool to the key itself, already on the grid: scale 1
+    codes, scale = oracle.pool_i8(raw, np.array([0.125, 0.5, 0.25, 0.125]))
+    assert np.array_equal(codes.astype(np.float32), key) and (scale == 1.0).all()
+    # one-hot weights subsample, then quantise: keys scaled by 2^-3 keep
+    # their codes and get scale 2^-3
+    raw2 = _grid_ints(rng, (80, 128)).astype(np.float32) / 8
+    for i in range(POOL):
+        w = np.zeros(POOL)
+        w[i] = 1.0
+        codes, scale = oracle.pool_i8(bits_of(raw2), w)
+        assert np.array_equal(codes.astype(np.float32), raw2[i::POOL] * 8)
+        assert (scale == 0.125).all()
+
+
+def test_pool_i8_dequantises_within_half_step_of_exact_pool():
+    rng = np.random.default_rng(23)
+    raw = bits_of(rng.integers(-8, 9, (400, 128)).astype(np.float32))
+    w = np.array([0.5, 0.25, 0.125, 0.125])
+    codes, scale = oracle.pool_i8(raw, w)
+    r = oracle.bf16_to_f64(raw).reshape(-1, POOL, 128)
+    exact = np.einsum("bid,i->bd", r, w)
+    deq = codes.astype(np.float64) * scale[:, None]
+    assert (np.abs(deq - exact) <= scale[:, None] / 2).all()
+    assert (np.abs(codes).max(axis=1) >= 64).all()
+
+
+def test_score_i8_integer_closed_form():
+    rng = np.random.default_rng(24)
+    heads, nblk = 32, 300
+    q = _grid_ints(rng, (heads, 128))
+    k = _grid_ints(rng, (nblk, 128))
+    w = np.array([0.25, 0.5, 1.0])[rng.integers(0, 3, heads)]
+    w[3] = -0.5  # a negative head weight keeps its sign
+    s = oracle.score_i8(bits_of(q.astype(np.float32)), w, k.astype(np.int8), np.ones(nblk))
+    # 4 s = sum_h (4 w_h) relu(k_b . q_h), in exact integers
+    exact = (np.maximum(k @ q.T, 0) * np.round(w * 4).astype(np.int64)).sum(axis=1)
+    assert np.array_equal(s * 4, exact.astype(np.float64))
+    # block scales multiply the block's score; a head quantised with scale
+    # 2^-3 (query / 8) contributes its dot times 2^-3
+    sc = 2.0 ** rng.integers(-6, 7, nblk)
+    s2 = oracle.score_i8(bits_of(q.astype(np.float32) / 8), w, k.astype(np.int8), sc)
+    assert np.array_equal(s2, s * sc / 8)
+
+
+def test_score_i8_is_bf16_score_of_dequantised_operands():
+    """Dequantised codes (<= 7 bits times a power of two) are exact in bf16,
+    so the INT8 score equals the bf16 score of the dequantised query and
+    keys, an independently pinned routine."""
+    w_ = synth.workload("mid")
+    raw = w_.raw_keys_np(0, 0, 8192)
+    codes, scale = oracle.pool_i8(raw, w_.pool_weights())
+    qb = w_.q_idx_np([1])[0]
+    wh = w_.w_head_np([1])[0].astype(np.float64)
+    q = oracle.bf16_to_f64(qb)
+    deq_q = np.stack([c * 2.0 ** e for c, e in (oracle.quant_i8(q[h]) for h in range(32))])
+    deq_k = codes.astype(np.float64) * scale[:, None]
+    s = oracle.score_i8(qb, wh, codes, scale)
+    ref = oracle.score(bits_of(deq_q), wh, bits_of(deq_k))
+    assert np.array_equal(s, ref)
+    # and the quantised scores rank close to the bf16 ones: the top 512 sets overlap
+    s_bf = oracle.score(qb, wh, oracle.pool(raw, w_.pool_weights()))
+    common = np.intersect1d(oracle.topk(s), oracle.topk(s_bf)).size
+    assert common >= 400
+
+
+def test_generator_i8_scores_are_exact_in_fp32():
+    """On the workloads, sum_h (w_h 2^e_h) relu(dot) is a sum of multiples of
+    its smallest head factor whose total stays below 2^24 of them, and every
+    dot is below 2^24: the device's fp32 head sum is exact in any order."""
+    for name in ("tiny", "mid", "1m"):
+        w_ = synth.workload(name)
+        raw = w_.raw_keys_np(0, 0, 32768)
+        codes, scale = oracle.pool_i8(raw, w_.pool_weights())
+        for row in (0, w_.B - 1):
+            q = oracle.bf16_to_f64(w_.q_idx_np([row])[0])
+            wh = w_.w_head_np([row])[0].astype(np.float64)
+            qc, qe = zip(*(oracle.quant_i8(q[h]) for h in range(32)))
+            f = wh * 2.0 ** np.array(qe)
+            dots = codes.astype(np.int64) @ np.stack(qc).astype(np.int64).T
+            assert np.abs(dots).max() < 2 ** 24
+            units = np.abs(f) / np.abs(f).min()
+            assert np.array_equal(units, np.round(units))
+            assert (np.maximum(dots, 0) * units).sum(axis=1).max() < 2 ** 24
