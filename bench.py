@@ -64,10 +64,12 @@ class DecodeState:
     Sequences b_offset .. b_offset+B-1 of the workload recipe.  The pooled
     cache holds the first L-1 tokens (built with spx_pool_append), the tail
     the last 3 of them; each step appends token L-1 and queries with n = L.
+    keys="int8" keeps the pooled keys in the INT8 cache (int8 codes plus one
+    scale per block, spx_pool_append_i8 / spx_decode_fused_i8).
     """
 
     def __init__(self, w: synth.Workload, device, b_offset: int = 0, B: int | None = None,
-                 build_latent: bool = True):
+                 build_latent: bool = True, keys: str = "bf16"):
         spx = spx_module()
         self.w = w
         self.device = device
@@ -80,7 +82,13 @@ class DecodeState:
         self.cap_blk = L // synth.POOL
         self.cap_tok = L
         bf16 = torch.bfloat16
-        self.pooled = torch.zeros(B, self.cap_blk, synth.IDX_DIM, dtype=bf16, device=device)
+        assert keys in ("bf16", "int8")
+        self.keys = keys
+        self.i8 = keys == "int8"
+        self.pooled = torch.zeros(B, self.cap_blk, synth.IDX_DIM,
+                                  dtype=torch.int8 if self.i8 else bf16, device=device)
+        self.k_scale = (torch.zeros(B, self.cap_blk, dtype=torch.float32, device=device)
+                        if self.i8 else None)
         self.tail = torch.zeros(B, synth.POOL - 1, synth.IDX_DIM, dtype=bf16, device=device)
         self.needles = {}
         for b in range(B):
@@ -92,9 +100,15 @@ class DecodeState:
                 t1 = min(L - 1, t + GEN_CHUNK_TOKENS)
                 raw = w.raw_keys_t(bg, t, t1, device, self.needles.get(b)).view(bf16)
                 ln = torch.tensor([t], dtype=torch.int64, device=device)
-                spx.spx_pool_append(self.d, 1, raw.reshape(1, t1 - t, synth.IDX_DIM), t1 - t,
-                                    self.pool_w, self.tail[b:b + 1], self.pooled[b:b + 1],
-                                    self.cap_blk, ln, t1)
+                if self.i8:
+                    spx.spx_pool_append_i8(self.d, 1, raw.reshape(1, t1 - t, synth.IDX_DIM),
+                                           t1 - t, self.pool_w, self.tail[b:b + 1],
+                                           self.pooled[b:b + 1], self.k_scale[b:b + 1],
+                                           self.cap_blk, ln, t1)
+                else:
+                    spx.spx_pool_append(self.d, 1, raw.reshape(1, t1 - t, synth.IDX_DIM), t1 - t,
+                                        self.pool_w, self.tail[b:b + 1], self.pooled[b:b + 1],
+                                        self.cap_blk, ln, t1)
                 t = t1
         self.latent = None
         if build_latent:
@@ -132,12 +146,23 @@ class DecodeState:
                 ws_bytes=self.ws.numel() * self.ws.element_size(),
                 stream=torch.cuda.current_stream(self.device).cuda_stream)
         c = self._call
-        spx.spx_decode_fused(
-            self.d, self.B, self.raw_new if raw_new is None else raw_new, c["pool_w"], c["tail"],
-            c["pooled"], self.cap_blk, c["len_dev"], self.q_idx if q_idx is None else q_idx,
-            self.w_head if w_head is None else w_head, self.q if q is None else q, c["latent"],
-            self.cap_tok, self.max_len, self.out if out is None else out, c["lse"], c["idx"],
-            c["count"], c["ws"], ws_bytes=c["ws_bytes"], timing=timing, stream=c["stream"])
+        raw_new = self.raw_new if raw_new is None else raw_new
+        q_idx = self.q_idx if q_idx is None else q_idx
+        w_head = self.w_head if w_head is None else w_head
+        q = self.q if q is None else q
+        out = self.out if out is None else out
+        if self.i8:
+            spx.spx_decode_fused_i8(
+                self.d, self.B, raw_new, c["pool_w"], c["tail"], c["pooled"], self.k_scale,
+                self.cap_blk, c["len_dev"], q_idx, w_head, q, c["latent"], self.cap_tok,
+                self.max_len, out, c["lse"], c["idx"], c["count"], c["ws"], ws_bytes=c["ws_bytes"],
+                timing=timing, stream=c["stream"])
+        else:
+            spx.spx_decode_fused(
+                self.d, self.B, raw_new, c["pool_w"], c["tail"], c["pooled"], self.cap_blk,
+                c["len_dev"], q_idx, w_head, q, c["latent"], self.cap_tok, self.max_len, out,
+                c["lse"], c["idx"], c["count"], c["ws"], ws_bytes=c["ws_bytes"], timing=timing,
+                stream=c["stream"])
 
     # ---- host copies of what the oracle needs (generator output) ----
     def raw_keys_host(self, b: int) -> np.ndarray:
@@ -354,11 +379,16 @@ def shard_offset(rank: int, per_rank: int) -> int:
     return rank * per_rank
 
 
-def score_algorithmic_bytes(nblk_per_row, rows: int) -> int:
-    """Bytes the scoring kernel must move: every pooled key read once (256 B),
-    every score written once (4 B), plus each query row (8 KiB) and its head
+def score_algorithmic_bytes(nblk_per_row, rows: int, keys: str = "bf16") -> int:
+    """Bytes the scoring kernel must move: every pooled key read once (256 B;
+    INT8 cache: 128 B of codes + a 4 B scale), every score written once
+    (4 B), plus each query row (8 KiB; INT8: 4 KiB of codes) and its head
     weights (128 B)."""
-    return int(sum(nblk_per_row)) * (synth.IDX_DIM * 2 + 4) + rows * (synth.IDX_HEADS * synth.IDX_DIM * 2 + synth.IDX_HEADS * 4)
+    if keys == "int8":
+        per_blk, per_row = synth.IDX_DIM + 4 + 4, synth.IDX_HEADS * synth.IDX_DIM + synth.IDX_HEADS * 4
+    else:
+        per_blk, per_row = synth.IDX_DIM * 2 + 4, synth.IDX_HEADS * synth.IDX_DIM * 2 + synth.IDX_HEADS * 4
+    return int(sum(nblk_per_row)) * per_blk + rows * per_row
 
 
 def score_algorithmic_flops_prefill(pos0: int, T: int) -> int:
@@ -484,7 +514,7 @@ def run_decode(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = synth.workload(args.workload)
-    st = DecodeState(w, device, b_offset=shard_offset(rank, w.B))
+    st = DecodeState(w, device, b_offset=shard_offset(rank, w.B), keys=args.keys)
     B, L = st.B, st.L
     stream = torch.cuda.current_stream(device)
 
@@ -566,9 +596,10 @@ def run_decode(args, world, rank, local):
         return None
     hbm, bf16, bf16s, src = measured_peaks()
     nblk = [L // synth.POOL] * B
-    alg = score_algorithmic_bytes(nblk, B)
+    alg = score_algorithmic_bytes(nblk, B, args.keys)
     achieved = alg / (score_avg * 1e-3) / 1e9
     queries = B * world * K
+    i8 = args.keys == "int8"
     line = {
         "metric": METRIC,
         "value": queries / (ms_max * 1e-3),
@@ -580,16 +611,19 @@ def run_decode(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "s8 indexer keys and queries (s32 dots), bf16 attention" if i8 else "bf16",
         "data": "synthetic (seeded generator; int-valued indexer keys, dyadic pool weights, "
                 "600 needles/seq, N(0,1) latent)",
         "config": {"workload": w.name, "batch_per_gpu": B, "context": L, "heads": st.H,
                    "indexer": "32 heads x 128, pool 4, top-512 blocks", "latent": 512,
+                   "pooled_keys": "int8 codes + fp32 scale per block" if i8 else "bf16",
                    "parallelism": f"dp{world} (independent sequences)",
-                   "l2": "inputs larger than L2 (256 MiB pooled keys + 4 GiB latent per GPU)"},
-        "roofline": {"bound": "hbm", "kernel": "k_index_score<1> (decode scoring)",
+                   "l2": "inputs larger than L2 (pooled keys + 4 GiB latent per GPU)"},
+        "roofline": {"bound": "hbm",
+                     "kernel": "k_index_score<1> (decode scoring" + (", INT8 cache)" if i8 else ")"),
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": f"{src} hbm_gbs", "traffic": recorded_traffic("decode_1m"),
+                     "peak_source": f"{src} hbm_gbs",
+                     "traffic": None if i8 else recorded_traffic("decode_1m"),
                      "algorithmic_bytes_per_launch": alg, "avg_launch_us": score_avg * 1e3,
                      "vs_8tbs": achieved / 8000.0},
         "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": "queries/s",
@@ -807,6 +841,8 @@ def main(argv=None):
                     help="decode with the latent cache in pinned host memory")
     ap.add_argument("--indexshare", type=int, default=0, metavar="N",
                     help="IndexShare decode: one indexer per N layers (reports per-layer rate)")
+    ap.add_argument("--keys", choices=("bf16", "int8"), default="bf16",
+                    help="pooled-key cache format of the decode workloads")
     ap.add_argument("--score-only", action="store_true",
                     help="time the decode scoring kernel alone (profiling aid)")
     args = ap.parse_args(argv)
@@ -830,7 +866,7 @@ def main(argv=None):
         if rank == 0 and line is not None:
             if (world == 1 and not args.no_cpu_baseline and args.workload != "prefill"
                     and not args.score_only and args.indexshare <= 1
-                    and not args.host_latent):
+                    and not args.host_latent and args.keys == "bf16"):
                 line["cpu_baseline"] = cpu_baseline(synth.workload(args.workload),
                                                     torch.device("cuda", local))
             print(json.dumps(line))

@@ -283,6 +283,60 @@ SPX_API spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* ra
                             spx_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * INT8 pooled-key cache.  [W1] section "양자화: W8A8와 혼합 캐시": the
+ * indexer's far, compressed cache entries are kept in INT8.  The page gives
+ * no scale convention; libspx stores each pooled block as 128 int8 codes
+ * plus one power-of-two scale:
+ *     e = the smallest integer with max_d |x_d| <= 127 * 2^e  (not below
+ *         -149; 0 for an all-zero block),
+ *     code_d = round-half-even(x_d / 2^e)  in [-127, 127],
+ *     k_scale = 2^e  (fp32),
+ * where x is the block's pooled value summed in fp32 (as spx_pool_append,
+ * before any bf16 rounding).  The scoring calls quantise every query head
+ * the same way (codes and 2^e_h) and compute
+ *     scores[b][blk] = k_scale[b][blk] * sum_h (w_head[b][h] * 2^e_h) *
+ *                      max(0, sum_d qcode[b][h][d] * code[b][blk][d])
+ * with the integer dot products exact (tcgen05 kind::i8, s32) and the head
+ * sum in fp32.  The key scan reads half the bytes of the bf16 cache.
+ *
+ *   pooled_k8  int8 [B, cap_blk, idx_dim]   codes (16-byte aligned base)
+ *   k_scale    float [B, cap_blk]           block scales (4-byte aligned)
+ * Other arguments, limits and errors as for the bf16 calls above; the
+ * raw-key tail stays bf16.
+ *
+ * spx_index_score_i8 needs a workspace of spx_index_score_i8_workspace_size
+ * bytes (the quantised queries); SPX_ERR_WORKSPACE if it is smaller, NULL
+ * or not 16-byte aligned.  spx_decode_fused_i8 takes the workspace of
+ * spx_decode_workspace_size and runs the same four launches as
+ * spx_decode_fused (the queries are quantised by its first kernel); its
+ * result equals spx_pool_append_i8, spx_index_score_i8, spx_topk_blocks and
+ * spx_sparse_mla_attn called in turn.
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_pool_append_i8(const spx_dims* d, int32_t B, const void* raw_k,
+                              int32_t n_new, const float* pool_w, void* tail,
+                              void* pooled_k8, float* k_scale, int64_t cap_blk,
+                              const int64_t* len_dev, int64_t max_len,
+                              spx_stream stream);
+SPX_API spx_status spx_index_score_i8_workspace_size(const spx_dims* d, int32_t B,
+                                             size_t* bytes);
+SPX_API spx_status spx_index_score_i8(const spx_dims* d, int32_t B, const void* q_idx,
+                              const float* w_head, const void* pooled_k8,
+                              const float* k_scale, int64_t cap_blk,
+                              const int64_t* n_vis, int64_t max_len, float* scores,
+                              int64_t score_stride, void* ws, size_t ws_bytes,
+                              spx_stream stream);
+SPX_API spx_status spx_decode_fused_i8(const spx_dims* d, int32_t B, const void* raw_k,
+                               const float* pool_w, void* tail, void* pooled_k8,
+                               float* k_scale, int64_t cap_blk,
+                               const int64_t* len_dev, const void* q_idx,
+                               const float* w_head, const void* q,
+                               const void* latent, int64_t cap_tok,
+                               int64_t max_len, void* out, float* lse,
+                               int32_t* idx_out, int32_t* count_out, void* ws,
+                               size_t ws_bytes, const spx_timing* timing,
+                               spx_stream stream);
+
+/* ---------------------------------------------------------------------------
  * Chunked causal prefill of one sequence: T new tokens appended after pos0
  * cached tokens.  Query t (0-based in the chunk, absolute position pos0 + t)
  * sees n_t = pos0 + t + 1 tokens: it scores the floor(n_t/4) complete blocks

@@ -75,6 +75,14 @@ _SIGS = {
     "spx_decode_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_decode_fused": ([_DIMS, _I32, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _I64, _I64, _P,
                           _P, _P, _P, _P, _SZ, ctypes.POINTER(spx_timing), _P], ctypes.c_int),
+    "spx_pool_append_i8": ([_DIMS, _I32, _P, _I32, _P, _P, _P, _P, _I64, _P, _I64, _P],
+                           ctypes.c_int),
+    "spx_index_score_i8_workspace_size": ([_DIMS, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "spx_index_score_i8": ([_DIMS, _I32, _P, _P, _P, _P, _I64, _P, _I64, _P, _I64, _P, _SZ, _P],
+                           ctypes.c_int),
+    "spx_decode_fused_i8": ([_DIMS, _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _I64, _I64,
+                             _P, _P, _P, _P, _P, _SZ, ctypes.POINTER(spx_timing), _P],
+                            ctypes.c_int),
     "spx_prefill_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_prefill_chunk": ([_DIMS, _I32, _P, _P, _P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P,
                            _P, _P, _P, _SZ, ctypes.POINTER(spx_timing), _P], ctypes.c_int),
@@ -245,6 +253,44 @@ def spx_decode_fused(d, B, raw_k, pool_w, tail, pooled_k, cap_blk, len_dev, q_id
                                  _ptr(latent), cap_tok, max_len, _ptr(out), _ptr(lse),
                                  _ptr(idx_out), _ptr(count_out), _ptr(ws), ws_bytes,
                                  _timing(timing), _stream(stream)), "spx_decode_fused")
+
+
+def spx_pool_append_i8(d, B, raw_k, n_new, pool_w, tail, pooled_k8, k_scale, cap_blk, len_dev,
+                       max_len, stream=None):
+    _check(_lib.spx_pool_append_i8(ctypes.byref(d), B, _ptr(raw_k), n_new, _host_f32(pool_w),
+                                   _ptr(tail), _ptr(pooled_k8), _ptr(k_scale), cap_blk,
+                                   _ptr(len_dev), max_len, _stream(stream)), "spx_pool_append_i8")
+
+
+def spx_index_score_i8_workspace_size(d, B) -> int:
+    n = _SZ(0)
+    _check(_lib.spx_index_score_i8_workspace_size(ctypes.byref(d), B, ctypes.byref(n)),
+           "spx_index_score_i8_workspace_size")
+    return n.value
+
+
+def spx_index_score_i8(d, B, q_idx, w_head, pooled_k8, k_scale, cap_blk, n_vis, max_len, scores,
+                       score_stride, ws, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.spx_index_score_i8(ctypes.byref(d), B, _ptr(q_idx), _ptr(w_head), _ptr(pooled_k8),
+                                   _ptr(k_scale), cap_blk, _ptr(n_vis), max_len, _ptr(scores),
+                                   score_stride, _ptr(ws), ws_bytes, _stream(stream)),
+           "spx_index_score_i8")
+
+
+def spx_decode_fused_i8(d, B, raw_k, pool_w, tail, pooled_k8, k_scale, cap_blk, len_dev, q_idx,
+                        w_head, q, latent, cap_tok, max_len, out, lse=None, idx_out=None,
+                        count_out=None, ws=None, ws_bytes=None, timing=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    pw = _host_f32(pool_w) if pool_w is not None else None
+    _check(_lib.spx_decode_fused_i8(ctypes.byref(d), B, _ptr(raw_k), pw, _ptr(tail),
+                                    _ptr(pooled_k8), _ptr(k_scale), cap_blk, _ptr(len_dev),
+                                    _ptr(q_idx), _ptr(w_head), _ptr(q), _ptr(latent), cap_tok,
+                                    max_len, _ptr(out), _ptr(lse), _ptr(idx_out),
+                                    _ptr(count_out), _ptr(ws), ws_bytes, _timing(timing),
+                                    _stream(stream)), "spx_decode_fused_i8")
 
 
 def spx_prefill_workspace_size(d, T, pos0) -> int:

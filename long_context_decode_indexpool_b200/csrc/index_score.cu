@@ -37,6 +37,14 @@
 // the bin of the row's 512th-largest key exactly; the selection kernel
 // (topk.cu) then only keeps blocks at or above that bin.
 //
+// INT8 cache (decode, [W1] section "양자화: W8A8와 혼합 캐시"): the keys are
+// int8 codes with one power-of-two scale per block and the query heads come
+// quantised the same way, their scales folded into w.  A tile is then one
+// 16 KiB box of 128-byte rows (half the bytes), the MMA is 4 tcgen05.mma
+// kind::i8 (K = 32 each) into exact s32 accumulators, and the epilogue takes
+// ReLU on the integer dot, sums w_h * dot over the heads in fp32 and
+// multiplies by the block's scale.
+//
 // Every wait is bounded; on a timeout the CTA drains and exits with the
 // device error word set.
 #include "select.cuh"
@@ -53,8 +61,7 @@ __device__ int g_device_error = 0;
 namespace {
 
 constexpr int kTileM = 128;
-constexpr int kHalfBytes = kTileM * 64 * 2;  // 128 rows x 128 bytes
-constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KiB: one tile of 128 keys
+constexpr int kHalfBytes = kTileM * 64 * 2;  // 128 rows x 128 bytes: one TMA box
 constexpr int kThreads = 192;
 constexpr int kEpi = 128;                    // epilogue threads
 constexpr int kHistBins = 2048;              // top 11 key bits
@@ -66,13 +73,17 @@ constexpr int kDynChunk = 4;
 constexpr int kMaxDynGroups = 512;
 constexpr int kRing = 4;  // chunk indices handed from the TMA warp to the others
 
-template <int NQ, bool SELECT>
+// I8: the INT8 cache (decode only): 128-byte key rows (one box per tile),
+// int8 query codes, kind::i8 MMAs into s32 accumulators.
+template <int NQ, bool SELECT, bool I8>
 struct Cfg {
+  static_assert(!I8 || NQ == 1, "the INT8 cache is scored one query per group");
   static constexpr int kN = 32 * NQ;
-  static constexpr int kStages = NQ == 1 ? 6 : 4;
+  static constexpr int kTileBytes = I8 ? kHalfBytes : 2 * kHalfBytes;  // 128 keys
+  static constexpr int kStages = I8 ? 10 : (NQ == 1 ? 6 : 4);
   static constexpr int kQSlots = NQ == 1 ? 2 : 1;
-  static constexpr int kQHalf = kN * 128;
-  static constexpr int kQBytes = 2 * kQHalf;
+  static constexpr int kQHalf = kN * 128;  // one 128-byte-wide box of Q
+  static constexpr int kQBytes = I8 ? kQHalf : 2 * kQHalf;
   // TMEM accumulator ring: 4 slots of 32 columns for one query (the MMA of
   // tile t+4 waits for the epilogue of tile t), 2 of 256 for eight
   static constexpr int kAcc = NQ == 1 ? 4 : 2;
@@ -86,12 +97,14 @@ struct Cfg {
   static constexpr int kBarOff = (kSelOff + kSelBytes + 7) & ~7;
   static constexpr int kNumBars = 2 * kStages + 2 * kQSlots + 2 * kAcc + 1;
   static constexpr int kSmem = 1024 + kBarOff + kNumBars * 8 + 16;
-  static constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, kN);
+  static constexpr uint32_t kIdesc = I8 ? idesc_s8_s32(kTileM, kN) : idesc_bf16_f32(kTileM, kN);
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 struct KParams {
   const float* w_head;
+  const float* k_scale;  // I8: [key batches, cap_blk] block scales
+  int64_t cap_blk;
   const int64_t* n_vis;
   float* scores;
   int64_t score_stride;
@@ -230,11 +243,11 @@ __device__ __forceinline__ void epi_sync() { group_sync<kEpi, 1>(); }
 
 }  // namespace
 
-template <int NQ, bool SELECT>
+template <int NQ, bool SELECT, bool I8>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_score(const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_q, const KParams p) {
-  using C = Cfg<NQ, SELECT>;
+  using C = Cfg<NQ, SELECT, I8>;
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -372,17 +385,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* dst = q_smem + qs * C::kQBytes;
           mbar_arrive_expect_tx(&qfull[qs], C::kQBytes);
           tma_load_2d(dst, &map_q, &qfull[qs], 0, w.g * C::kN);
-          tma_load_2d(dst + C::kQHalf, &map_q, &qfull[qs], 64, w.g * C::kN);
+          if constexpr (!I8) tma_load_2d(dst + C::kQHalf, &map_q, &qfull[qs], 64, w.g * C::kN);
           q_issued_slot = qs;
           q_issued_ph = qe_ph[qs] ^ 1;
           cur_g = w.g;
         }
         if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) break;
-        uint8_t* dst = a_smem + stage * kTileBytes;
+        uint8_t* dst = a_smem + stage * C::kTileBytes;
         const int kb = p.shared_keys ? 0 : w.g;
-        mbar_arrive_expect_tx(&full[stage], kTileBytes);
+        mbar_arrive_expect_tx(&full[stage], C::kTileBytes);
         tma_load_3d_hint(dst, &map_k, &full[stage], 0, w.t * kTileM, kb, stream_pol);
-        tma_load_3d_hint(dst + kHalfBytes, &map_k, &full[stage], 64, w.t * kTileM, kb, stream_pol);
+        if constexpr (!I8)
+          tma_load_3d_hint(dst + kHalfBytes, &map_k, &full[stage], 64, w.t * kTileM, kb, stream_pol);
         ++issued;
         if (++stage == C::kStages) {
           stage = 0;
@@ -423,14 +437,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&full[stage], ph, abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::kN);
-        const uint32_t a0 = a_base + stage * kTileBytes;
+        const uint32_t a0 = a_base + stage * C::kTileBytes;
         const uint32_t b0 = q_base + qs * C::kQBytes;
+        if constexpr (I8) {
+          // K = 32 int8 per MMA: four 32-byte steps along the 128-byte rows
 #pragma unroll
-        for (int k = 0; k < kIdxDim / 16; ++k) {
-          const uint32_t koff = (k & 3) * 32;
-          const uint64_t ad = sdesc_kmajor_sw128(a0 + (k >> 2) * kHalfBytes + koff);
-          const uint64_t bd = sdesc_kmajor_sw128(b0 + (k >> 2) * C::kQHalf + koff);
-          umma_bf16(d, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
+          for (int k = 0; k < kIdxDim / 32; ++k) {
+            const uint64_t ad = sdesc_kmajor_sw128(a0 + k * 32);
+            const uint64_t bd = sdesc_kmajor_sw128(b0 + k * 32);
+            umma_s8(d, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < kIdxDim / 16; ++k) {
+            const uint32_t koff = (k & 3) * 32;
+            const uint64_t ad = sdesc_kmajor_sw128(a0 + (k >> 2) * kHalfBytes + koff);
+            const uint64_t bd = sdesc_kmajor_sw128(b0 + (k >> 2) * C::kQHalf + koff);
+            umma_bf16(d, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
+          }
         }
         umma_commit(&empty[stage]);
         umma_commit(&accfull[acc]);
@@ -496,12 +520,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         epi_sync();
         cur_g = w.g;
       }
+      const int64_t blk = static_cast<int64_t>(w.t) * kTileM + row_in_tile;
+      float ksc = 1.f;  // I8: the block's scale, fetched before the wait
+      if constexpr (I8) {
+        if (blk < nb_smem[0])
+          ksc = __ldg(p.k_scale + (p.shared_keys ? 0 : static_cast<int64_t>(w.g)) * p.cap_blk + blk);
+      }
       if (!mbar_wait(&accfull[acc], acc_ph, abort_flag)) {
         aborted = true;
         break;
       }
       tc_fence_after();
-      const int64_t blk = static_cast<int64_t>(w.t) * kTileM + row_in_tile;
       float scv[NQ];
 #pragma unroll 1
       for (int j = 0; j < NQ; ++j) {
@@ -515,9 +544,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // four interleaved partial sums over the heads (short dependency chains)
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int h = 0; h < kIdxHeads; ++h)
-          s4[h & 3] = __fmaf_rn(wj[h], v[h] > 0.f ? v[h] : 0.f, s4[h & 3]);
+        for (int h = 0; h < kIdxHeads; ++h) {
+          float x;
+          if constexpr (I8) {
+            const int dot = __float_as_int(v[h]);  // exact s32 dot product
+            x = static_cast<float>(dot > 0 ? dot : 0);
+          } else {
+            x = v[h] > 0.f ? v[h] : 0.f;
+          }
+          s4[h & 3] = __fmaf_rn(wj[h], x, s4[h & 3]);
+        }
         scv[j] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        if constexpr (I8) scv[j] *= ksc;
       }
       tc_fence_before();
       __syncwarp();
@@ -550,11 +588,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 namespace {
 
-template <int NQ, bool SELECT>
+template <int NQ, bool SELECT, bool I8>
 cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
-  using C = Cfg<NQ, SELECT>;
+  using C = Cfg<NQ, SELECT, I8>;
   CUtensorMap map_k, map_q;
-  {
+  if constexpr (I8) {
+    // one 128-byte row per key and per query head
+    const uint64_t dims[3] = {static_cast<uint64_t>(kIdxDim), static_cast<uint64_t>(a.cap_blk),
+                              static_cast<uint64_t>(a.key_batches)};
+    const uint64_t strides[2] = {kIdxDim * 1ull, static_cast<uint64_t>(a.cap_blk) * kIdxDim};
+    const uint32_t box[3] = {kIdxDim, kTileM, 1};
+    if (!encode_tensor_map(&map_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.pooled_k, dims, strides,
+                           box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    const uint64_t qdims[2] = {static_cast<uint64_t>(kIdxDim),
+                               static_cast<uint64_t>(a.rows) * kIdxHeads};
+    const uint64_t qstrides[1] = {kIdxDim * 1ull};
+    const uint32_t qbox[2] = {kIdxDim, static_cast<uint32_t>(C::kN)};
+    if (!encode_tensor_map(&map_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q_idx, qdims, qstrides,
+                           qbox, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  } else {
     const uint64_t dims[3] = {static_cast<uint64_t>(kIdxDim), static_cast<uint64_t>(a.cap_blk),
                               static_cast<uint64_t>(a.key_batches)};
     const uint64_t strides[2] = {kIdxDim * 2ull, static_cast<uint64_t>(a.cap_blk) * kIdxDim * 2ull};
@@ -562,27 +616,27 @@ cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
     if (!encode_tensor_map(&map_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.pooled_k, dims,
                            strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
-  }
-  {
-    const uint64_t dims[2] = {static_cast<uint64_t>(kIdxDim),
-                              static_cast<uint64_t>(a.rows) * kIdxHeads};
-    const uint64_t strides[1] = {kIdxDim * 2ull};
-    const uint32_t box[2] = {64, static_cast<uint32_t>(C::kN)};
-    if (!encode_tensor_map(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q_idx, dims, strides,
-                           box, CU_TENSOR_MAP_SWIZZLE_128B))
+    const uint64_t qdims[2] = {static_cast<uint64_t>(kIdxDim),
+                               static_cast<uint64_t>(a.rows) * kIdxHeads};
+    const uint64_t qstrides[1] = {kIdxDim * 2ull};
+    const uint32_t qbox[2] = {64, static_cast<uint32_t>(C::kN)};
+    if (!encode_tensor_map(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q_idx, qdims, qstrides,
+                           qbox, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_index_score<NQ, SELECT>,
+    cudaError_t e = cudaFuncSetAttribute(k_index_score<NQ, SELECT, I8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   KParams p{};
   p.w_head = a.w_head;
+  p.k_scale = a.k_scale;
+  p.cap_blk = a.cap_blk;
   p.n_vis = a.n_vis;
   p.scores = a.scores;
   p.score_stride = a.score_stride;
@@ -594,7 +648,7 @@ cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
   p.work_counter = a.work_counter;
   const int grid = score_grid(a.nq, a.rows, a.max_len, a.num_sms);
   if (grid == 0) return cudaSuccess;
-  cudaError_t e = launch_ex(k_index_score<NQ, SELECT>, dim3(grid), dim3(kThreads), C::kSmem,
+  cudaError_t e = launch_ex(k_index_score<NQ, SELECT, I8>, dim3(grid), dim3(kThreads), C::kSmem,
                             stream, a.pdl, 1, map_k, map_q, p);
   count_launches(1);
   if (e != cudaSuccess) return e;
@@ -612,10 +666,14 @@ int score_grid(int nq, int rows, int64_t max_len, int num_sms) {
 
 cudaError_t launch_index_score(const ScoreArgs& a, cudaStream_t stream) {
   if (a.nq == 1) {
-    if (a.sel_ghist) return launch_cfg<1, true>(a, stream);
-    return launch_cfg<1, false>(a, stream);
+    if (a.i8) {
+      if (a.sel_ghist) return launch_cfg<1, true, true>(a, stream);
+      return launch_cfg<1, false, true>(a, stream);
+    }
+    if (a.sel_ghist) return launch_cfg<1, true, false>(a, stream);
+    return launch_cfg<1, false, false>(a, stream);
   }
-  if (a.nq == 8) return launch_cfg<8, false>(a, stream);
+  if (a.nq == 8 && !a.i8) return launch_cfg<8, false, false>(a, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -8,7 +8,11 @@
 // Block b holds tokens 4b..4b+3 in time order; w_i weighs the i-th of them.
 // A block is pooled when its last token is appended; until then its raw keys
 // wait in a 3-slot tail per sequence.  The pooled value is the fp32 sum
-// rounded once to bf16 (round-to-nearest-even).
+// rounded once to bf16 (round-to-nearest-even), or, in the INT8 cache
+// ([W1] section "양자화: W8A8와 혼합 캐시": far, compressed indexer entries in
+// INT8), that sum as int8 codes with one power-of-two scale per block
+// (i8_exponent / i8_code); the 16 threads of a block find its max |x| by
+// shuffles.
 //
 // Work split: grid (x, B).  CTA x of sequence b pools blocks
 // blk_lo + x*kBlocksPerCta ..; 16 threads per block, 8 dims (16 bytes) per
@@ -38,61 +42,133 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
   }
 }
 
-__global__ void __launch_bounds__(kPoolThreads)
-    k_pool_append(const __nv_bfloat16* __restrict__ raw_k, int n_new, float w0, float w1,
-                  float w2, float w3, __nv_bfloat16* __restrict__ tail,
-                  __nv_bfloat16* __restrict__ pooled, int64_t cap_blk,
-                  const int64_t* __restrict__ len_dev, int64_t len_host, int64_t max_len,
-                  int64_t* __restrict__ nvis_out, uint32_t* __restrict__ init_hist,
-                  int32_t* __restrict__ init_done) {
+// INT8 codes of the query heads of row b (the scoring kernel's B operand):
+// warp w quantises heads w, w+4, ..; lane l holds dims 4l..4l+3.  The
+// head's scale is folded into its weight: wq = w_head * 2^e.
+__device__ void quant_q_row(const __nv_bfloat16* __restrict__ q_idx,
+                            const float* __restrict__ w_head, int8_t* __restrict__ q8,
+                            float* __restrict__ wq, int b) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int h = warp; h < kIdxHeads; h += kPoolThreads / 32) {
+    const int64_t row = static_cast<int64_t>(b) * kIdxHeads + h;
+    const uint2 u = *reinterpret_cast<const uint2*>(q_idx + row * kIdxDim + 4 * lane);
+    const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    float amax = fmaxf(fmaxf(fabsf(x01.x), fabsf(x01.y)), fmaxf(fabsf(x23.x), fabsf(x23.y)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const int e = i8_exponent(amax);
+    const uint32_t packed = (static_cast<uint32_t>(i8_code(x01.x, e)) & 0xffu) |
+                            ((static_cast<uint32_t>(i8_code(x01.y, e)) & 0xffu) << 8) |
+                            ((static_cast<uint32_t>(i8_code(x23.x, e)) & 0xffu) << 16) |
+                            (static_cast<uint32_t>(i8_code(x23.y, e)) << 24);
+    *reinterpret_cast<uint32_t*>(q8 + row * kIdxDim + 4 * lane) = packed;
+    if (lane == 0) wq[row] = w_head[row] * ldexpf(1.f, e);
+  }
+}
+
+struct PoolKParams {
+  const __nv_bfloat16* raw_k;
+  int n_new;
+  float w[4];
+  __nv_bfloat16* tail;
+  void* pooled;        // bf16 rows, or int8 code rows
+  float* k_scale;      // int8 cache: per-block scale
+  int64_t cap_blk;
+  const int64_t* len_dev;
+  int64_t len_host;
+  int64_t max_len;
+  int64_t* nvis_out;
+  uint32_t* init_hist;
+  int32_t* init_done;
+  const __nv_bfloat16* q_idx;  // optional query quantisation (int8 cache)
+  const float* w_head;
+  int8_t* q8;
+  float* wq;
+};
+
+template <bool I8>
+__global__ void __launch_bounds__(kPoolThreads) k_pool_append(const PoolKParams p) {
   pdl_trigger();
   const int b = blockIdx.y;
-  int64_t len = len_dev ? len_dev[b] : len_host;
+  int64_t len = p.len_dev ? p.len_dev[b] : p.len_host;
   // Clamp so that every access stays inside the caches whatever the device
   // lengths hold.
   if (len < 0) len = 0;
-  if (len > max_len - n_new) len = max_len - n_new;
-  const int64_t end = len + n_new;
+  if (len > p.max_len - p.n_new) len = p.max_len - p.n_new;
+  const int64_t end = len + p.n_new;
   if (blockIdx.x == 0) {
-    if (nvis_out && threadIdx.x == 0) nvis_out[b] = end;
-    if (init_hist) {
+    if (p.nvis_out && threadIdx.x == 0) p.nvis_out[b] = end;
+    if (p.init_hist) {
       for (int i = threadIdx.x; i < kSelHistBins; i += kPoolThreads)
-        init_hist[static_cast<int64_t>(b) * kSelHistBins + i] = 0u;
-      if (threadIdx.x == 0) init_done[b] = 0;
-      if (threadIdx.x == 0 && b == 0) init_done[gridDim.y] = 0;  // the scoring work counter
+        p.init_hist[static_cast<int64_t>(b) * kSelHistBins + i] = 0u;
+      if (threadIdx.x == 0) p.init_done[b] = 0;
+      if (threadIdx.x == 0 && b == 0) p.init_done[gridDim.y] = 0;  // the scoring work counter
+    }
+    if constexpr (I8) {
+      if (p.q_idx) quant_q_row(p.q_idx, p.w_head, p.q8, p.wq, b);
     }
   }
-  if (n_new <= 0) return;
+  if (p.n_new <= 0) return;
 
   const int64_t blk_lo = len / kPool;
   const int64_t blk_done = end / kPool;  // blocks [blk_lo, blk_done) complete now
   const int chunk = threadIdx.x % kChunksPerRow;
   const int sub = threadIdx.x / kChunksPerRow;
-  const float w[4] = {w0, w1, w2, w3};
-  const __nv_bfloat16* raw_b = raw_k + static_cast<int64_t>(b) * n_new * kIdxDim;
-  __nv_bfloat16* tail_b = tail + static_cast<int64_t>(b) * (kPool - 1) * kIdxDim;
-  __nv_bfloat16* pooled_b = pooled + static_cast<int64_t>(b) * cap_blk * kIdxDim;
+  const __nv_bfloat16* raw_b = p.raw_k + static_cast<int64_t>(b) * p.n_new * kIdxDim;
+  __nv_bfloat16* tail_b = p.tail + static_cast<int64_t>(b) * (kPool - 1) * kIdxDim;
 
   const int64_t first = blk_lo + static_cast<int64_t>(blockIdx.x) * kBlocksPerCta;
   for (int pass = 0; pass < kBlocksPerCta / kBlocksPerPass; ++pass) {
-    const int64_t blk = first + pass * kBlocksPerPass + sub;
-    if (blk >= blk_done) break;
-    float acc[8];
+    const int64_t blk0 = first + pass * kBlocksPerPass;
+    if (blk0 >= blk_done) break;  // uniform
+    const int64_t blk = blk0 + sub;
+    const bool active = blk < blk_done;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (active) {
 #pragma unroll
-    for (int i = 0; i < kPool; ++i) {
-      const int64_t p = blk * kPool + i;
-      const __nv_bfloat16* src = (p < len) ? tail_b + (p % kPool) * kIdxDim
-                                           : raw_b + (p - len) * kIdxDim;
-      float f[8];
-      load8(src + chunk * 8, f);
+      for (int i = 0; i < kPool; ++i) {
+        const int64_t t = blk * kPool + i;
+        const __nv_bfloat16* src = (t < len) ? tail_b + (t % kPool) * kIdxDim
+                                             : raw_b + (t - len) * kIdxDim;
+        float f[8];
+        load8(src + chunk * 8, f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = (i == 0) ? f[e] * w[0] : __fmaf_rn(f[e], w[i], acc[e]);
+        for (int e = 0; e < 8; ++e) acc[e] = (i == 0) ? f[e] * p.w[0] : __fmaf_rn(f[e], p.w[i], acc[e]);
+      }
     }
-    uint4 o;
-    __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&o);
+    if constexpr (I8) {
+      // the block's 16 threads are lanes 0-15 or 16-31 of one warp
+      float amax = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) oh[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
-    *reinterpret_cast<uint4*>(pooled_b + blk * kIdxDim + chunk * 8) = o;
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(acc[e]));
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const int ex = i8_exponent(amax);
+      uint32_t w2[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        w2[h] = (static_cast<uint32_t>(i8_code(acc[4 * h], ex)) & 0xffu) |
+                ((static_cast<uint32_t>(i8_code(acc[4 * h + 1], ex)) & 0xffu) << 8) |
+                ((static_cast<uint32_t>(i8_code(acc[4 * h + 2], ex)) & 0xffu) << 16) |
+                (static_cast<uint32_t>(i8_code(acc[4 * h + 3], ex)) << 24);
+      if (active) {
+        int8_t* row = static_cast<int8_t*>(p.pooled) +
+                      (static_cast<int64_t>(b) * p.cap_blk + blk) * kIdxDim;
+        *reinterpret_cast<uint2*>(row + chunk * 8) = make_uint2(w2[0], w2[1]);
+        if (chunk == 0) p.k_scale[static_cast<int64_t>(b) * p.cap_blk + blk] = ldexpf(1.f, ex);
+      }
+    } else {
+      if (active) {
+        uint4 o;
+        __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oh[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+        __nv_bfloat16* row = static_cast<__nv_bfloat16*>(p.pooled) +
+                             (static_cast<int64_t>(b) * p.cap_blk + blk) * kIdxDim;
+        *reinterpret_cast<uint4*>(row + chunk * 8) = o;
+      }
+    }
   }
 
   // New keys of the still-incomplete last block go to the tail (CTA 0 only,
@@ -100,11 +176,18 @@ __global__ void __launch_bounds__(kPoolThreads)
   if (blockIdx.x == 0 && (end % kPool) != 0) {
     __syncthreads();
     const int64_t p0 = (end / kPool) * kPool;
-    for (int64_t p = (p0 > len ? p0 : len) + sub; p < end; p += kBlocksPerPass) {
-      const uint4 v = *reinterpret_cast<const uint4*>(raw_b + (p - len) * kIdxDim + chunk * 8);
-      *reinterpret_cast<uint4*>(tail_b + (p % kPool) * kIdxDim + chunk * 8) = v;
+    for (int64_t t = (p0 > len ? p0 : len) + sub; t < end; t += kBlocksPerPass) {
+      const uint4 v = *reinterpret_cast<const uint4*>(raw_b + (t - len) * kIdxDim + chunk * 8);
+      *reinterpret_cast<uint4*>(tail_b + (t % kPool) * kIdxDim + chunk * 8) = v;
     }
   }
+}
+
+// Query quantisation alone (standalone INT8 scoring call): one CTA per row.
+__global__ void __launch_bounds__(kPoolThreads)
+    k_quant_q(const __nv_bfloat16* __restrict__ q_idx, const float* __restrict__ w_head,
+              int8_t* __restrict__ q8, float* __restrict__ wq) {
+  quant_q_row(q_idx, w_head, q8, wq, blockIdx.x);
 }
 
 // n_vis of the prefill queries: query t sees pos0 + t + 1 tokens.
@@ -116,15 +199,42 @@ __global__ void k_prefill_nvis(int64_t* __restrict__ n_vis, int T, int64_t pos0)
 }  // namespace
 
 cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream) {
-  if (a.n_new <= 0 && a.nvis_out == nullptr && a.init_hist == nullptr) return cudaSuccess;
+  if (a.n_new <= 0 && a.nvis_out == nullptr && a.init_hist == nullptr && a.q_idx == nullptr)
+    return cudaSuccess;
   // Blocks an append can touch: at most ceil((n_new + 3) / 4) + 1.
   const int64_t blocks = (static_cast<int64_t>(a.n_new) + 2 * kPool) / kPool;
   dim3 grid(static_cast<unsigned>((blocks + kBlocksPerCta - 1) / kBlocksPerCta), a.B);
   if (grid.x == 0) grid.x = 1;
-  k_pool_append<<<grid, kPoolThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.raw_k), a.n_new, a.w[0], a.w[1], a.w[2], a.w[3],
-      static_cast<__nv_bfloat16*>(a.tail), static_cast<__nv_bfloat16*>(a.pooled_k), a.cap_blk,
-      a.len_dev, a.len_host, a.max_len, a.nvis_out, a.init_hist, a.init_done);
+  PoolKParams p{};
+  p.raw_k = static_cast<const __nv_bfloat16*>(a.raw_k);
+  p.n_new = a.n_new;
+  for (int i = 0; i < 4; ++i) p.w[i] = a.w[i];
+  p.tail = static_cast<__nv_bfloat16*>(a.tail);
+  p.pooled = a.pooled_k;
+  p.k_scale = a.k_scale;
+  p.cap_blk = a.cap_blk;
+  p.len_dev = a.len_dev;
+  p.len_host = a.len_host;
+  p.max_len = a.max_len;
+  p.nvis_out = a.nvis_out;
+  p.init_hist = a.init_hist;
+  p.init_done = a.init_done;
+  p.q_idx = static_cast<const __nv_bfloat16*>(a.q_idx);
+  p.w_head = a.w_head;
+  p.q8 = a.q8;
+  p.wq = a.wq;
+  if (a.i8)
+    k_pool_append<true><<<grid, kPoolThreads, 0, stream>>>(p);
+  else
+    k_pool_append<false><<<grid, kPoolThreads, 0, stream>>>(p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_q(int B, const void* q_idx, const float* w_head, int8_t* q8, float* wq,
+                           cudaStream_t stream) {
+  k_quant_q<<<B, kPoolThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(q_idx), w_head, q8,
+                                            wq);
   count_launches(1);
   return cudaGetLastError();
 }

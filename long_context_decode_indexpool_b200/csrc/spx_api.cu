@@ -150,9 +150,10 @@ FusedLayout fused_layout(int rows, int heads, int64_t max_len) {
 // Workspace of the fused decode call:
 //   n_vis [B] | idx [B,512] | count [B] | key histogram [B,2048] | done [B+1]
 //   | scores [B, stride] | list keys, list ids [B*nchunk, 512]
-//   | list counts [B*nchunk] | attention scratch
+//   | list counts [B*nchunk] | attention scratch | INT8 cache: query codes
+//   [B,32,128] int8 and head weights [B,32] with the query scales folded in
 struct DecodeLayout {
-  size_t nvis, idx, count, hist, done, scores, lkey, lidx, lcnt, attn, total;
+  size_t nvis, idx, count, hist, done, scores, lkey, lidx, lcnt, attn, q8, wq, total;
   int64_t stride;  // scores per row, a multiple of 4
   int nchunk;
   AttnPlan ap;
@@ -189,8 +190,17 @@ DecodeLayout decode_layout(int B, int heads, int64_t max_len) {
   o += up(lists * 4);
   L.attn = o;
   o += up(L.ap.ws_bytes);
+  L.q8 = o;
+  o += up(static_cast<size_t>(B) * kIdxHeads * kIdxDim);
+  L.wq = o;
+  o += up(static_cast<size_t>(B) * kIdxHeads * 4);
   L.total = o;
   return L;
+}
+
+// Workspace of the standalone INT8 scoring call: query codes | head weights.
+size_t score_i8_ws(int B) {
+  return up(static_cast<size_t>(B) * kIdxHeads * kIdxDim) + up(static_cast<size_t>(B) * kIdxHeads * 4);
 }
 
 spx_status check_pool_w(const float* w, float out[4]) {
@@ -258,9 +268,14 @@ spx_status spx_device_error(int32_t* code, spx_stream stream) {
 }
 
 // ---------------------------------------------------------------------------
-spx_status spx_pool_append(const spx_dims* d, int32_t B, const void* raw_k, int32_t n_new,
-                           const float* pool_w, void* tail, void* pooled_k, int64_t cap_blk,
-                           const int64_t* len_dev, int64_t max_len, spx_stream stream) {
+}  // extern "C"
+
+namespace {
+
+spx_status pool_append_impl(const spx_dims* d, int32_t B, const void* raw_k, int32_t n_new,
+                            const float* pool_w, void* tail, void* pooled_k, float* k_scale,
+                            bool i8, int64_t cap_blk, const int64_t* len_dev, int64_t max_len,
+                            spx_stream stream) {
   spx_status st = check_dims(d);
   if (st != SPX_OK) return st;
   float w[4];
@@ -270,8 +285,11 @@ spx_status spx_pool_append(const spx_dims* d, int32_t B, const void* raw_k, int3
   if (!tail || !pooled_k || !len_dev || (n_new > 0 && !raw_k)) return SPX_ERR_INVALID_ARG;
   if (!al16(tail) || !al16(pooled_k) || (raw_k && !al16(raw_k)) || (len_dev && !al4(len_dev)))
     return SPX_ERR_INVALID_ARG;
+  if (i8 && (!k_scale || !al4(k_scale))) return SPX_ERR_INVALID_ARG;
   if (n_new == 0) return SPX_OK;
   PoolAppendArgs a{};
+  a.i8 = i8;
+  a.k_scale = k_scale;
   a.B = B;
   a.raw_k = raw_k;
   a.n_new = n_new;
@@ -286,10 +304,10 @@ spx_status spx_pool_append(const spx_dims* d, int32_t B, const void* raw_k, int3
   return cuda_status(launch_pool_append(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-spx_status spx_index_score(const spx_dims* d, int32_t B, const void* q_idx, const float* w_head,
-                           const void* pooled_k, int64_t cap_blk, const int64_t* n_vis,
-                           int64_t max_len, float* scores, int64_t score_stride,
-                           spx_stream stream) {
+// Host checks shared by the bf16 and INT8 scoring calls.
+spx_status check_score_args(const spx_dims* d, int32_t B, const void* q_idx, const float* w_head,
+                            const void* pooled_k, int64_t cap_blk, const int64_t* n_vis,
+                            int64_t max_len, float* scores, int64_t score_stride) {
   spx_status st = check_dims(d);
   if (st != SPX_OK) return st;
   if (B < 1 || cap_blk < 1 || max_len < 0 || max_len > kPool * cap_blk) return SPX_ERR_SHAPE;
@@ -298,6 +316,35 @@ spx_status spx_index_score(const spx_dims* d, int32_t B, const void* q_idx, cons
   if (score_stride < max_len / kPool) return SPX_ERR_SHAPE;
   if (!q_idx || !w_head || !pooled_k || !n_vis || !scores) return SPX_ERR_INVALID_ARG;
   if (!al16(q_idx) || !al16(pooled_k) || !al4(w_head) || !al4(scores)) return SPX_ERR_INVALID_ARG;
+  return SPX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+spx_status spx_pool_append(const spx_dims* d, int32_t B, const void* raw_k, int32_t n_new,
+                           const float* pool_w, void* tail, void* pooled_k, int64_t cap_blk,
+                           const int64_t* len_dev, int64_t max_len, spx_stream stream) {
+  return pool_append_impl(d, B, raw_k, n_new, pool_w, tail, pooled_k, nullptr, false, cap_blk,
+                          len_dev, max_len, stream);
+}
+
+spx_status spx_pool_append_i8(const spx_dims* d, int32_t B, const void* raw_k, int32_t n_new,
+                              const float* pool_w, void* tail, void* pooled_k8, float* k_scale,
+                              int64_t cap_blk, const int64_t* len_dev, int64_t max_len,
+                              spx_stream stream) {
+  return pool_append_impl(d, B, raw_k, n_new, pool_w, tail, pooled_k8, k_scale, true, cap_blk,
+                          len_dev, max_len, stream);
+}
+
+spx_status spx_index_score(const spx_dims* d, int32_t B, const void* q_idx, const float* w_head,
+                           const void* pooled_k, int64_t cap_blk, const int64_t* n_vis,
+                           int64_t max_len, float* scores, int64_t score_stride,
+                           spx_stream stream) {
+  spx_status st =
+      check_score_args(d, B, q_idx, w_head, pooled_k, cap_blk, n_vis, max_len, scores, score_stride);
+  if (st != SPX_OK) return st;
   ScoreArgs a{};
   a.nq = 1;
   a.rows = B;
@@ -312,6 +359,51 @@ spx_status spx_index_score(const spx_dims* d, int32_t B, const void* q_idx, cons
   a.score_stride = score_stride;
   a.num_sms = device_sm_count();
   return cuda_status(launch_index_score(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+spx_status spx_index_score_i8_workspace_size(const spx_dims* d, int32_t B, size_t* bytes) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (!bytes) return SPX_ERR_INVALID_ARG;
+  if (B < 1 || B > 65535) return SPX_ERR_SHAPE;
+  *bytes = score_i8_ws(B);
+  return SPX_OK;
+}
+
+spx_status spx_index_score_i8(const spx_dims* d, int32_t B, const void* q_idx,
+                              const float* w_head, const void* pooled_k8, const float* k_scale,
+                              int64_t cap_blk, const int64_t* n_vis, int64_t max_len,
+                              float* scores, int64_t score_stride, void* ws, size_t ws_bytes,
+                              spx_stream stream) {
+  spx_status st = check_score_args(d, B, q_idx, w_head, pooled_k8, cap_blk, n_vis, max_len,
+                                   scores, score_stride);
+  if (st != SPX_OK) return st;
+  if (B > 65535) return SPX_ERR_SHAPE;
+  if (!k_scale) return SPX_ERR_INVALID_ARG;
+  if (!al4(k_scale)) return SPX_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < score_i8_ws(B) || !al16(ws)) return SPX_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int8_t* q8 = static_cast<int8_t*>(ws);
+  float* wq = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                       up(static_cast<size_t>(B) * kIdxHeads * kIdxDim));
+  cudaError_t e = launch_quant_q(B, q_idx, w_head, q8, wq, s);
+  if (e != cudaSuccess) return SPX_ERR_CUDA;
+  ScoreArgs a{};
+  a.nq = 1;
+  a.i8 = true;
+  a.k_scale = k_scale;
+  a.rows = B;
+  a.key_batches = B;
+  a.q_idx = q8;
+  a.w_head = wq;
+  a.pooled_k = pooled_k8;
+  a.cap_blk = cap_blk;
+  a.n_vis = n_vis;
+  a.max_len = max_len;
+  a.scores = scores;
+  a.score_stride = score_stride;
+  a.num_sms = device_sm_count();
+  return cuda_status(launch_index_score(a, s));
 }
 
 spx_status spx_topk_workspace_size(const spx_dims* d, int32_t rows, int64_t max_len,
@@ -393,12 +485,18 @@ spx_status spx_decode_workspace_size(const spx_dims* d, int32_t B, int64_t max_l
   return SPX_OK;
 }
 
-spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, const float* pool_w,
-                            void* tail, void* pooled_k, int64_t cap_blk, const int64_t* len_dev,
-                            const void* q_idx, const float* w_head, const void* q,
-                            const void* latent, int64_t cap_tok, int64_t max_len, void* out,
-                            float* lse, int32_t* idx_out, int32_t* count_out, void* ws,
-                            size_t ws_bytes, const spx_timing* timing, spx_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// The fused decode step for either pooled-key format (i8: int8 codes in
+// pooled_k plus block scales in k_scale).
+spx_status decode_impl(const spx_dims* d, int32_t B, const void* raw_k, const float* pool_w,
+                       void* tail, void* pooled_k, float* k_scale, bool i8, int64_t cap_blk,
+                       const int64_t* len_dev, const void* q_idx, const float* w_head,
+                       const void* q, const void* latent, int64_t cap_tok, int64_t max_len,
+                       void* out, float* lse, int32_t* idx_out, int32_t* count_out, void* ws,
+                       size_t ws_bytes, const spx_timing* timing, spx_stream stream) {
   spx_status st = check_dims(d);
   if (st != SPX_OK) return st;
   float w[4] = {0.f, 0.f, 0.f, 0.f};
@@ -410,6 +508,7 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   if (!pooled_k || !len_dev || !q_idx || !w_head || !q || !latent || !out)
     return SPX_ERR_INVALID_ARG;
   if (raw_k && !tail) return SPX_ERR_INVALID_ARG;
+  if (i8 && (!k_scale || !al4(k_scale))) return SPX_ERR_INVALID_ARG;
   if (!al16(pooled_k) || !al16(q_idx) || !al16(q) || !al16(latent) || !al16(out) ||
       !al4(w_head) || !al4(len_dev) || (raw_k && (!al16(raw_k) || !al16(tail))) ||
       (lse && !al4(lse)) || (idx_out && !al4(idx_out)) || (count_out && !al4(count_out)))
@@ -442,6 +541,16 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   pa.nvis_out = n_vis;
   pa.init_hist = hist;
   pa.init_done = done;
+  int8_t* q8 = reinterpret_cast<int8_t*>(base + L.q8);
+  float* wq = reinterpret_cast<float*>(base + L.wq);
+  if (i8) {
+    pa.i8 = true;
+    pa.k_scale = k_scale;
+    pa.q_idx = q_idx;  // quantised here for the scoring kernel
+    pa.w_head = w_head;
+    pa.q8 = q8;
+    pa.wq = wq;
+  }
   cudaError_t e = launch_pool_append(pa, s);
   if (e != cudaSuccess) return SPX_ERR_CUDA;
 
@@ -451,10 +560,12 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
     return SPX_ERR_CUDA;
   ScoreArgs sa{};
   sa.nq = 1;
+  sa.i8 = i8;
+  sa.k_scale = k_scale;
   sa.rows = B;
   sa.key_batches = B;
-  sa.q_idx = q_idx;
-  sa.w_head = w_head;
+  sa.q_idx = i8 ? static_cast<const void*>(q8) : q_idx;
+  sa.w_head = i8 ? wq : w_head;
   sa.pooled_k = pooled_k;
   sa.cap_blk = cap_blk;
   sa.n_vis = n_vis;
@@ -506,6 +617,33 @@ spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, con
   aa.ws = base + L.attn;
   aa.pdl = true;
   return cuda_status(launch_attn(L.ap, aa, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* raw_k, const float* pool_w,
+                            void* tail, void* pooled_k, int64_t cap_blk, const int64_t* len_dev,
+                            const void* q_idx, const float* w_head, const void* q,
+                            const void* latent, int64_t cap_tok, int64_t max_len, void* out,
+                            float* lse, int32_t* idx_out, int32_t* count_out, void* ws,
+                            size_t ws_bytes, const spx_timing* timing, spx_stream stream) {
+  return decode_impl(d, B, raw_k, pool_w, tail, pooled_k, nullptr, false, cap_blk, len_dev, q_idx,
+                     w_head, q, latent, cap_tok, max_len, out, lse, idx_out, count_out, ws,
+                     ws_bytes, timing, stream);
+}
+
+spx_status spx_decode_fused_i8(const spx_dims* d, int32_t B, const void* raw_k,
+                               const float* pool_w, void* tail, void* pooled_k8, float* k_scale,
+                               int64_t cap_blk, const int64_t* len_dev, const void* q_idx,
+                               const float* w_head, const void* q, const void* latent,
+                               int64_t cap_tok, int64_t max_len, void* out, float* lse,
+                               int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
+                               const spx_timing* timing, spx_stream stream) {
+  return decode_impl(d, B, raw_k, pool_w, tail, pooled_k8, k_scale, true, cap_blk, len_dev, q_idx,
+                     w_head, q, latent, cap_tok, max_len, out, lse, idx_out, count_out, ws,
+                     ws_bytes, timing, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -182,6 +182,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, signed 8-bit inputs, exact s32 accumulate.
+__device__ __forceinline__ void umma_s8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on `bar` when every tcgen05.mma issued so far by this thread
 // has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -200,6 +211,30 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
 }
+
+// Instruction descriptor of tcgen05.mma kind::i8: signed 8-bit A and B, s32
+// D (no saturation), both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+  return (2u << 4)                               // D format: s32
+         | (1u << 7)                             // A format: signed 8-bit
+         | (1u << 10)                            // B format: signed 8-bit
+         | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
+// INT8 cache codes: a vector with max |x| = amax is stored as
+// round-half-even(x / 2^e) with e the smallest integer such that
+// amax <= 127 * 2^e (not below -149; 0 for amax = 0).  With
+// amax = m 2^E, m in [0.5, 1): e = E - 7 when m <= 127/128, else E - 6.
+__device__ __forceinline__ int i8_exponent(float amax) {
+  if (!(amax > 0.f)) return 0;
+  int E = 0;
+  const float m = frexpf(amax, &E);
+  const int e = m <= 127.f / 128.f ? E - 7 : E - 6;
+  return e < -149 ? -149 : e;
+}
+
+__device__ __forceinline__ int i8_code(float x, int e) { return __float2int_rn(ldexpf(x, -e)); }
 
 // Shared-memory matrix descriptor for a K-major operand stored in the
 // 128-byte-swizzle canonical layout: rows of 128 bytes (64 bf16), 8-row

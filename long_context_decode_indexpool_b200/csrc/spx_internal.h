@@ -34,14 +34,32 @@ struct PoolAppendArgs {
   // hist[b][..] = 0, done[b] = 0 for b < B, and done[B] = 0
   uint32_t* init_hist;
   int32_t* init_done;
+  // INT8 cache: pooled_k holds int8 codes [B, cap_blk, 128] and k_scale the
+  // per-block scales [B, cap_blk]; with q_idx set, CTA 0 of each row also
+  // quantises that row's indexer query (q8 [B, 32, 128], wq [B, 32] =
+  // w_head times the head's scale) for the scoring kernel.
+  bool i8;
+  float* k_scale;
+  const void* q_idx;
+  const float* w_head;
+  int8_t* q8;
+  float* wq;
 };
 cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream);
+// Query quantisation alone (one CTA per row), as in launch_pool_append.
+cudaError_t launch_quant_q(int B, const void* q_idx, const float* w_head, int8_t* q8, float* wq,
+                           cudaStream_t stream);
 cudaError_t launch_prefill_nvis(int64_t* n_vis, int T, int64_t pos0, cudaStream_t stream);
 
 // Indexer scoring as a tcgen05 GEMM: tiles of 128 pooled keys (M) against
 // query groups of nq queries x 32 heads (N = 32 nq), K = 128.
 struct ScoreArgs {
   int nq;             // queries per group: 1 (decode) or 8 (prefill)
+  // INT8 cache (nq == 1): q_idx holds int8 query codes, w_head the weights
+  // with the head scales folded in, pooled_k int8 key codes and k_scale
+  // [key_batches, cap_blk] the block scales
+  bool i8;
+  const float* k_scale;
   int rows;           // query rows
   int key_batches;    // batches of the pooled-key cache (decode: rows; prefill: 1)
   const void* q_idx;  // [rows, 32, 128] bf16

@@ -134,3 +134,49 @@ def test_workspace_sizes_scale(spx):
     assert big < 64 << 20
     assert spx.spx_topk_workspace_size(d, 4, 2048) == 0  # one level, no scratch
     assert spx.spx_prefill_workspace_size(d, 4096, 131072) > 4096 * (135168 // 4) * 4
+
+
+def test_int8_cache_host_validation(spx):
+    d = spx.dims(64, 1.0)
+    s = 0
+    # the scale array is required and must be 4-byte aligned
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_pool_append_i8(d, 1, FAKE, 1, [0.25] * 4, FAKE, FAKE, None, 16, FAKE, 8, stream=s)
+    assert e.value.status == 1
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_pool_append_i8(d, 1, FAKE, 1, [0.25] * 4, FAKE, FAKE, FAKE + 2, 16, FAKE, 8, stream=s)
+    assert e.value.status == 1
+    # the bf16 checks apply too (weights summing to one, capacity)
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_pool_append_i8(d, 1, FAKE, 1, [0.5] * 4, FAKE, FAKE, FAKE, 16, FAKE, 8, stream=s)
+    assert e.value.status == 1
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_pool_append_i8(d, 1, FAKE, 1, [0.25] * 4, FAKE, FAKE, FAKE, 16, FAKE, 65, stream=s)
+    assert e.value.status == 2
+    # scoring: workspace holds the query codes and folded head weights
+    need = spx.spx_index_score_i8_workspace_size(d, 4)
+    assert need >= 4 * 32 * 128 + 4 * 32 * 4
+    assert spx.spx_index_score_i8_workspace_size(d, 8) > need
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_index_score_i8(d, 4, FAKE, FAKE, FAKE, FAKE, 1024, FAKE, 4096, FAKE, 1024, FAKE,
+                               ws_bytes=need - 1, stream=s)
+    assert e.value.status == 4
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_index_score_i8(d, 4, FAKE, FAKE, FAKE, None, 1024, FAKE, 4096, FAKE, 1024, FAKE,
+                               ws_bytes=need, stream=s)
+    assert e.value.status == 1
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_index_score_i8(d, 4, FAKE, FAKE, FAKE, FAKE, 1024, FAKE, 4096, FAKE, 1000, FAKE,
+                               ws_bytes=need, stream=s)
+    assert e.value.status == 2
+    # fused decode: same workspace as the bf16 call; scales required
+    need = spx.spx_decode_workspace_size(d, 4, 8192)
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_decode_fused_i8(d, 4, FAKE, [0.25] * 4, FAKE, FAKE, None, 2048, FAKE, FAKE, FAKE,
+                                FAKE, FAKE, 8192, 8192, FAKE, ws=FAKE, ws_bytes=need, stream=s)
+    assert e.value.status == 1
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_decode_fused_i8(d, 4, FAKE, [0.25] * 4, FAKE, FAKE, FAKE, 2048, FAKE, FAKE, FAKE,
+                                FAKE, FAKE, 8192, 8192, FAKE, ws=FAKE, ws_bytes=need - 256,
+                                stream=s)
+    assert e.value.status == 4

@@ -9,6 +9,9 @@ def test_algorithmic_bytes_of_the_1m_scoring_launch():
     nblk = [w.L // synth.POOL] * w.B
     # 4 x 262,144 blocks x (256 B key + 4 B score) + 4 x (8 KiB query + 128 B weights)
     assert bench.score_algorithmic_bytes(nblk, w.B) == 272_663_040
+    # INT8 cache: 128 B of codes + 4 B scale + 4 B score per block; 4 KiB of
+    # query codes + 128 B of weights per row
+    assert bench.score_algorithmic_bytes(nblk, w.B, "int8") == 4 * 262144 * 136 + 4 * (4096 + 128)
 
 
 def test_prefill_flops_count_the_causal_blocks():
