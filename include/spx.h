@@ -265,7 +265,8 @@ SPX_API spx_status spx_sparse_mla_attn(const spx_dims* d, int32_t rows, const vo
  *   max_len   host bound on n for every sequence; <= pool*cap_blk, <= cap_tok;
  *             above 16,777,216 tokens the call returns SPX_ERR_UNSUPPORTED
  *   ws        workspace of spx_decode_workspace_size(d, B, max_len) bytes
- *             (holds the scores, their key histogram and the selection lists)
+ *             (holds the scores, their key histogram, the selection lists
+ *             and, for spx_decode_fused_i8, the quantised indexer queries)
  *   timing    optional events around the scoring launch (may be NULL); the
  *             kernels of the call may otherwise start before their
  *             predecessor in the call has finished (they wait for its data)
