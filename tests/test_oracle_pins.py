@@ -453,15 +453,24 @@ def test_pool_i8_on_grid_and_one_hot():
 
 
 def test_pool_i8_dequantises_within_half_step_of_exact_pool():
+    """The codes quantise the exact pooled sum: within half a step of it.
+    With the workloads' 1/64-dyadic weights the sums need up to 11
+    significant bits, so a bf16 rounding before the quantisation would move
+    some codes by one step and break the bound."""
     rng = np.random.default_rng(23)
-    raw = bits_of(rng.integers(-8, 9, (400, 128)).astype(np.float32))
-    w = np.array([0.5, 0.25, 0.125, 0.125])
-    codes, scale = oracle.pool_i8(raw, w)
-    r = oracle.bf16_to_f64(raw).reshape(-1, POOL, 128)
-    exact = np.einsum("bid,i->bd", r, w)
-    deq = codes.astype(np.float64) * scale[:, None]
-    assert (np.abs(deq - exact) <= scale[:, None] / 2).all()
-    assert (np.abs(codes).max(axis=1) >= 64).all()
+    cases = [(bits_of(rng.integers(-8, 9, (400, 128)).astype(np.float32)),
+              np.array([0.5, 0.25, 0.125, 0.125]))]
+    mid = synth.workload("mid")
+    cases.append((mid.raw_keys_np(0, 0, 16384), mid.pool_weights()))
+    for raw, w in cases:
+        codes, scale = oracle.pool_i8(raw, w)
+        r = oracle.bf16_to_f64(raw).reshape(-1, POOL, 128)
+        exact = np.einsum("bid,i->bd", r, w)
+        deq = codes.astype(np.float64) * scale[:, None]
+        assert (np.abs(deq - exact) <= scale[:, None] / 2).all()
+        assert (np.abs(codes).max(axis=1) >= 64).all()
+    # the second case really needs more than bf16's 8 significant bits
+    assert not np.array_equal(exact, oracle.bf16_to_f64(oracle.pool(raw, w)))
 
 
 def test_score_i8_integer_closed_form():
