@@ -105,21 +105,28 @@ def _run_copy(tmp_root: str, name: str, source: str) -> int:
         f.write(source)
     code = RUNNER.format(pkg_parent=parent, root=ROOT, tests=os.path.join(ROOT, "tests"),
                          pins=os.path.join(ROOT, "tests", "test_oracle_pins.py"))
+    env = dict(os.environ, TMPDIR=parent)  # compiler temporaries stay in the scratch folder
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
-                       timeout=600)
+                       timeout=600, env=env)
     return r.returncode
 
 
-def test_pins_catch_planted_mistakes(tmp_path):
+def test_pins_catch_planted_mistakes():
     src = open(os.path.join(ORACLE_DIR, "spx_oracle.cpp")).read()
     jobs = {"unmodified": src}
     for name, (old, new) in MUTANTS.items():
         assert src.count(old) == 1, f"mutant {name!r} no longer matches the oracle source"
         jobs[name] = src.replace(old, new)
-    workers = max(1, min(8, os.cpu_count() or 1))
-    with cf.ThreadPoolExecutor(workers) as ex:
-        futs = {name: ex.submit(_run_copy, str(tmp_path), name, s) for name, s in jobs.items()}
-        rc = {name: f.result() for name, f in futs.items()}
+    # scratch inside the repository's (ignored) build folder, removed afterwards
+    scratch = os.path.join(ROOT, "_build", f"oracle_mutants_{os.getpid()}")
+    os.makedirs(scratch)
+    try:
+        workers = max(1, min(8, os.cpu_count() or 1))
+        with cf.ThreadPoolExecutor(workers) as ex:
+            futs = {name: ex.submit(_run_copy, scratch, name, s) for name, s in jobs.items()}
+            rc = {name: f.result() for name, f in futs.items()}
+    finally:
+        shutil.rmtree(scratch, ignore_errors=True)
     assert rc.pop("unmodified") == 0, "the unmodified oracle copy must pass its pins"
     survived = [name for name, code in rc.items() if code != 1]
     assert not survived, f"pins did not catch: {survived}"
