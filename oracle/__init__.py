@@ -59,6 +59,12 @@ def _load():
             lib.orc_pool_i8.restype = None
             lib.orc_score_i8.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P, P, i64, P, ctypes.c_int]
             lib.orc_score_i8.restype = None
+            lib.orc_e4m3_bits.argtypes = [ctypes.c_double]
+            lib.orc_e4m3_bits.restype = ctypes.c_uint8
+            lib.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+            lib.orc_e4m3_value.restype = ctypes.c_double
+            lib.orc_quant_e4m3.argtypes = [P, ctypes.c_int, P]
+            lib.orc_quant_e4m3.restype = ctypes.c_int
             lib.orc_topk.argtypes = [P, i64, i64, P]
             lib.orc_topk.restype = i64
             lib.orc_token_set.argtypes = [P, i64, i64, ctypes.c_int, P]
@@ -151,6 +157,42 @@ def score_i8(q_bits: np.ndarray, w_head, codes: np.ndarray, scale, nthreads: int
     return out
 
 
+def e4m3_bits(v: float) -> int:
+    """E4M3 bit pattern of the nearest-even E4M3 value of v (|v| <= 448)."""
+    return int(_load().orc_e4m3_bits(float(v)))
+
+
+def e4m3_value(bits) -> np.ndarray:
+    """Values (fp64) of E4M3 bit patterns."""
+    lib = _load()
+    table = np.array([lib.orc_e4m3_value(b) for b in range(256)], dtype=np.float64)
+    return table[np.asarray(bits, dtype=np.uint8)]
+
+
+def quant_e4m3(x) -> tuple[np.ndarray, int]:
+    """FP8 (E4M3) code of one vector: (uint8 codes, e) with x ~= 2^e * value(codes)."""
+    v = np.ascontiguousarray(x, dtype=np.float64).reshape(-1)
+    codes = np.zeros(v.size, dtype=np.uint8)
+    e = _load().orc_quant_e4m3(_p(v), v.size, _p(codes))
+    return codes, int(e)
+
+
+def latent_fp8(rows_bits: np.ndarray):
+    """FP8 latent cache of bf16 latent rows [S, D]: (codes [S, D] uint8, e [S])."""
+    rows = bf16_to_f64(np.asarray(rows_bits, dtype=np.uint16)).reshape(-1, np.shape(rows_bits)[-1])
+    out = [quant_e4m3(r) for r in rows]
+    codes = np.stack([c for c, _ in out]) if out else np.zeros((0, rows.shape[1]), np.uint8)
+    return codes, np.array([e for _, e in out], dtype=np.int64)
+
+
+def dequant_fp8_bits(codes: np.ndarray, e) -> np.ndarray:
+    """bf16 bits of the dequantised FP8 rows (exact: 4 significant bits times 2^k)."""
+    vals = e4m3_value(codes) * np.ldexp(1.0, np.asarray(e))[:, None]
+    bits = np.array([bf16_rne(v) for v in vals.reshape(-1)], dtype=np.uint16).reshape(vals.shape)
+    assert np.array_equal(bf16_to_f64(bits), vals)
+    return bits
+
+
 def topk(scores, K: int = TOPK_BLOCKS) -> np.ndarray:
     """Selected block ids (int32, ascending) of the top min(K, n) scores."""
     s = np.ascontiguousarray(scores, dtype=np.float64)
@@ -184,6 +226,13 @@ def select_query(q_idx_bits, w_head, pooled_bits, n_vis: int, K: int = TOPK_BLOC
     s = score(q_idx_bits, w_head, pooled_bits[:nblk], nthreads)
     idx = topk(s, K)
     return s, idx, token_set(idx, n_vis)
+
+
+def attention_fp8(q_bits: np.ndarray, rows_bits: np.ndarray, sm_scale: float):
+    """Attention over an FP8 latent cache: the rows are stored as E4M3 codes
+    with one power-of-two scale each, and attended in their dequantised form."""
+    codes, e = latent_fp8(rows_bits)
+    return attention(q_bits, dequant_fp8_bits(codes, e), sm_scale)
 
 
 def decode_query(q_idx_bits, w_head, pooled_bits, n_vis, q_bits, latent_rows_fn, sm_scale,

@@ -27,7 +27,9 @@
 // ones the method's storage formats impose: the pooled key is stored as
 // bf16 (one round-to-nearest-even of the exact fp64 sum) or, in the INT8
 // cache, as int8 codes of that sum (one round-half-even after an exact
-// power-of-two scaling; the query heads likewise), and the top-k
+// power-of-two scaling; the query heads likewise), a latent row of the
+// FP8 cache is stored as E4M3 codes of the row over a power-of-two scale
+// (one nearest-even rounding), and the top-k
 // decision is taken on the score rounded to fp32, the precision in which
 // scores are stored and ranked on the device.
 
@@ -208,6 +210,61 @@ void orc_score_i8(const uint16_t* q, const double* w_head, int heads, int dim,
     pool.emplace_back(work, b0, b1);
   }
   for (auto& th : pool) th.join();
+}
+
+// ---- FP8 (E4M3) latent cache -------------------------------------------------
+// [W1] section "양자화: W8A8와 혼합 캐시": recent, important cache entries are
+// kept in FP8.  Reading followed here for the MLA latent rows: a row x is
+// stored as E4M3 codes (4 exponent bits with bias 7, 3 mantissa bits,
+// largest finite value 448, subnormal step 2^-9) of x / 2^e, one
+// power-of-two scale 2^e per row, e the smallest integer with
+// max |x| <= 448 * 2^e (not below -149; 0 for an all-zero row), rounding to
+// nearest with ties to even.
+
+// Nearest-even E4M3 value of v, |v| <= 448: keep 4 significant bits, the
+// subnormal step 2^-9 being the finest.
+static double e4m3_round(double v) {
+  if (v == 0.0) return v;
+  int E = 0;
+  std::frexp(std::fabs(v), &E);  // |v| = m 2^E, m in [0.5, 1)
+  int qe = E - 4;                // weight of the last kept bit
+  if (qe < -9) qe = -9;
+  const double r = std::ldexp(std::nearbyint(std::ldexp(std::fabs(v), -qe)), qe);
+  return std::signbit(v) ? -r : r;
+}
+
+// Bit pattern of an E4M3 value r (one that e4m3_round returns).
+uint8_t orc_e4m3_bits(double v) {
+  const double r = e4m3_round(v);
+  const uint8_t sign = std::signbit(r) ? 0x80 : 0x00;
+  const double a = std::fabs(r);
+  if (a == 0.0) return sign;
+  if (a < std::ldexp(1.0, -6))  // subnormal: a = mant * 2^-9
+    return sign | static_cast<uint8_t>(std::ldexp(a, 9));
+  int E = 0;
+  std::frexp(a, &E);  // a = 1.f * 2^(E-1)
+  const int mant = static_cast<int>(std::ldexp(a, 4 - E)) - 8;  // 3 fraction bits
+  return sign | static_cast<uint8_t>(((E - 1 + 7) << 3) | mant);
+}
+
+// Value of an E4M3 bit pattern (finite patterns only).
+double orc_e4m3_value(uint8_t bits) {
+  const int ex = (bits >> 3) & 15, mant = bits & 7;
+  const double a = ex == 0 ? std::ldexp(mant, -9) : std::ldexp(8 + mant, ex - 7 - 3);
+  return (bits & 0x80) ? -a : a;
+}
+
+// Returns e and writes the n E4M3 codes of x / 2^e.
+int orc_quant_e4m3(const double* x, int n, uint8_t* codes) {
+  double amax = 0.0;
+  for (int i = 0; i < n; ++i) amax = std::max(amax, std::fabs(x[i]));
+  int e = 0;
+  if (amax > 0.0) {
+    e = std::ilogb(amax) + 1;  // amax < 2^e <= 448 * 2^e
+    while (e > -149 && amax <= 448.0 * std::ldexp(1.0, e - 1)) --e;
+  }
+  for (int i = 0; i < n; ++i) codes[i] = orc_e4m3_bits(std::ldexp(x[i], -e));
+  return e;
 }
 
 // Top-k block selection [W4 "수렴점 2": keep the 512 highest-scoring 4-token

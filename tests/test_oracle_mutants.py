@@ -73,6 +73,21 @@ MUTANTS = {
     "int8 ReLU after the weight": (
         "s += w_head[h] * qs[h] * (dot > 0.0 ? dot : 0.0);",
         "s += std::max(0.0, w_head[h] * qs[h] * dot);"),
+    # FP8 latent cache
+    "e4m3 ties away from zero": (
+        "const double r = std::ldexp(std::nearbyint(std::ldexp(std::fabs(v), -qe)), qe);",
+        "const double r = std::ldexp(std::round(std::ldexp(std::fabs(v), -qe)), qe);"),
+    "e4m3 one mantissa bit too many": ("int qe = E - 4;", "int qe = E - 5;"),
+    "e4m3 subnormal step 2^-10": ("if (qe < -9) qe = -9;", "if (qe < -10) qe = -10;"),
+    "e4m3 bound 512 instead of 448": (
+        "while (e > -149 && amax <= 448.0 * std::ldexp(1.0, e - 1)) --e;",
+        "while (e > -149 && amax <= 512.0 * std::ldexp(1.0, e - 1)) --e;"),
+    "e4m3 exponent one too high": (
+        "while (e > -149 && amax <= 448.0 * std::ldexp(1.0, e - 1)) --e;",
+        "while (e > -149 && amax <= 448.0 * std::ldexp(1.0, e - 1)) --e;\n    ++e;"),
+    "e4m3 exponent field bias 8": (
+        "return sign | static_cast<uint8_t>(((E - 1 + 7) << 3) | mant);",
+        "return sign | static_cast<uint8_t>(((E - 1 + 8) << 3) | mant);"),
     "int8 key operand transposed": (
         "static_cast<double>(codes[b * dim + d]);",
         "static_cast<double>(codes[d * nblk + b]);"),

@@ -530,3 +530,84 @@ def test_generator_i8_scores_are_exact_in_fp32():
             units = np.abs(f) / np.abs(f).min()
             assert np.array_equal(units, np.round(units))
             assert (np.maximum(dots, 0) * units).sum(axis=1).max() < 2 ** 24
+
+
+# ----------------------------------------------------------------------------
+# FP8 (E4M3) latent cache
+# ----------------------------------------------------------------------------
+def test_e4m3_rounding_matches_library():
+    rng = np.random.default_rng(41)
+    x = np.concatenate([
+        rng.uniform(-448, 448, 20000),
+        rng.standard_normal(20000) * 2.0 ** rng.integers(-12, 8, 20000),
+        # exact half-way points between neighbouring E4M3 values
+        (np.arange(1, 480) + 0.5) * 2.0 ** -9,
+        ((np.arange(8, 16) + 0.5)[None, :] * 2.0 ** np.arange(-6, 6)[:, None]).ravel(),
+    ]).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    ref = torch.tensor(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_bits(float(v)) for v in x], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+    # and the decoder inverts the library's encoding on every finite pattern
+    finite = np.array([b for b in range(256) if (b & 0x7F) != 0x7F], dtype=np.uint8)
+    lib = torch.tensor(finite).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    assert np.array_equal(oracle.e4m3_value(finite), lib)
+
+
+def test_e4m3_closed_forms():
+    # 16..32 has spacing 2: 17 and 19 are ties, going to the even mantissa
+    assert [oracle.e4m3_value(oracle.e4m3_bits(v)) for v in (17, 19, 448, 0.3)] == \
+        [16.0, 20.0, 448.0, 0.3125]
+    # subnormal step 2^-9: 2^-10 ties to 0, 3 * 2^-10 ties up to 2^-8
+    assert oracle.e4m3_bits(2.0 ** -10) == 0 and oracle.e4m3_bits(3 * 2.0 ** -10) == 2
+    assert oracle.e4m3_bits(2.0 ** -9) == 1 and oracle.e4m3_bits(2.0 ** -6) == 8
+    assert oracle.e4m3_bits(-5.5) == 0x80 | (9 << 3) | 3
+
+
+def test_quant_e4m3_invariants():
+    rng = np.random.default_rng(42)
+    for t in range(200):
+        x = (rng.standard_normal(512) * 2.0 ** rng.integers(-40, 40)).astype(np.float32)
+        x = x.astype(np.float64)
+        if t % 5 == 0:
+            x[rng.integers(0, 512, 100)] = 0.0
+        c, e = oracle.quant_e4m3(x)
+        v = oracle.e4m3_value(c)
+        amax = np.abs(x).max()
+        # the smallest exponent that keeps every value within 448
+        assert amax <= 448 * 2.0 ** e and amax > 448 * 2.0 ** (e - 1)
+        assert 224 <= np.abs(v).max() <= 448
+        # one nearest rounding: within half the local spacing (4 significant
+        # bits, subnormal step 2^-9 in code units)
+        y = np.abs(x) * 2.0 ** -e
+        spacing = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(y, 2.0 ** -9))) - 3), 2.0 ** -9)
+        assert (np.abs(x * 2.0 ** -e - v) <= spacing / 2).all()
+        c2, e2 = oracle.quant_e4m3(x * 2.0 ** 7)
+        assert e2 == e + 7 and np.array_equal(c2, c)
+    c, e = oracle.quant_e4m3(np.zeros(512))
+    assert e == 0 and not c.any()
+
+
+def test_fp8_latent_attention():
+    rng = np.random.default_rng(43)
+    H, S, D = 8, 40, 512
+    q = _normal_bits(rng, (H, D), 1 / np.sqrt(D))
+    rows = _normal_bits(rng, (S, D))
+    codes, e = oracle.latent_fp8(rows)
+    deq = oracle.dequant_fp8_bits(codes, e)
+    # attention over the FP8 cache is attention over the dequantised rows
+    out8, lse8 = oracle.attention_fp8(q, rows, 1.0)
+    out, lse = oracle.attention(q, deq, 1.0)
+    assert np.array_equal(out8, out) and np.array_equal(lse8, lse)
+    # rows already on the grid (4 significant bits, max in (224, 448]) are stored exactly
+    grid = oracle.e4m3_value(rng.integers(0, 126, (S, D)).astype(np.uint8))
+    grid[:, 0] = 448.0
+    gbits = bits_of(grid * 2.0 ** -6)
+    c2, e2 = oracle.latent_fp8(gbits)
+    assert (e2 == -6).all()
+    assert np.array_equal(oracle.dequant_fp8_bits(c2, e2), gbits)
+    out_g, _ = oracle.attention_fp8(q, gbits, 1.0)
+    assert np.array_equal(out_g, oracle.attention(q, gbits, 1.0)[0])
+    # the error of a 512-wide N(0,1) row: below 2^-4 of its scale per element
+    x = oracle.bf16_to_f64(rows)
+    assert (np.abs(oracle.bf16_to_f64(deq) - x) <= 2.0 ** (e[:, None] + 8 - 4)).all()
