@@ -627,11 +627,12 @@ cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
+  const bool cached = dev >= 0 && dev < 64;  // devices beyond the cache: set every call
+  if (!cached || !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(k_index_score<NQ, SELECT, I8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    if (cached) attr_set[dev] = true;
   }
   KParams p{};
   p.w_head = a.w_head;

@@ -538,11 +538,12 @@ cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream)
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
+  const bool cached = dev >= 0 && dev < 64;  // devices beyond the cache: set every call
+  if (!cached || !attr_set[dev]) {
     cudaError_t e =
         cudaFuncSetAttribute(k_select_blocks, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    if (cached) attr_set[dev] = true;
   }
   cudaError_t e = launch_ex(k_select_blocks, dim3(a.nchunk, a.rows), dim3(kThreads), kSmem,
                             stream, a.pdl, 1, a.scores, a.score_stride, a.n_vis, a.max_len,
