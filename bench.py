@@ -741,10 +741,6 @@ def run_prefill(args, world, rank, local):
     st = PrefillState(w, device)
     stream = torch.cuda.current_stream(device)
 
-    def reset():
-        st.pooled.copy_(st.pooled0)
-        st.tail.copy_(st.tail0)
-
     for _ in range(args.warmup):
         st.step()
     torch.cuda.synchronize(device)
