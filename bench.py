@@ -205,9 +205,6 @@ class PrefillState:
             spx.spx_pool_append(self.d, 1, raw.reshape(1, t1 - t, synth.IDX_DIM), t1 - t,
                                 self.pool_w, self.tail, self.pooled, self.cap_blk, ln, t1)
             t = t1
-        # snapshot of the cache before the chunk, so a step can be repeated
-        self.pooled0 = self.pooled.clone()
-        self.tail0 = self.tail.clone()
         self.latent = torch.empty(total, synth.LATENT, dtype=bf16, device=device)
         for t in range(0, total, GEN_CHUNK_TOKENS):
             t1 = min(total, t + GEN_CHUNK_TOKENS)
