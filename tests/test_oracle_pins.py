@@ -516,11 +516,13 @@ def test_generator_i8_scores_are_exact_in_fp32():
     """On the workloads, sum_h (w_h 2^e_h) relu(dot) is a sum of multiples of
     its smallest head factor whose total stays below 2^24 of them, and every
     dot is below 2^24: the device's fp32 head sum is exact in any order."""
-    for name in ("tiny", "mid", "1m"):
+    for name in ("tiny", "mid", "1m", "prefill"):
         w_ = synth.workload(name)
         raw = w_.raw_keys_np(0, 0, 32768)
         codes, scale = oracle.pool_i8(raw, w_.pool_weights())
-        for row in (0, w_.B - 1):
+        # decode rows are sequences; prefill rows are the chunk's query positions
+        rows = (w_.L, w_.L + w_.T - 1) if name == "prefill" else (0, w_.B - 1)
+        for row in rows:
             q = oracle.bf16_to_f64(w_.q_idx_np([row])[0])
             wh = w_.w_head_np([row])[0].astype(np.float64)
             qc, qe = zip(*(oracle.quant_i8(q[h]) for h in range(32)))
