@@ -41,3 +41,29 @@ def test_recorded_traffic_matches_only_the_current_kernel_source():
     alg = bench.score_algorithmic_bytes([262144] * 4, 4)
     assert t is None or alg <= t < 1.05 * alg  # recorded for this source, no re-reads
     assert bench.recorded_traffic("no such workload") is None
+
+
+def test_reference_arm_line_on_cpu():
+    """`bench.py --impl reference` (the oracle, timed on host cores) prints one
+    JSON line with the contract's keys; ranks other than 0 print nothing."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny", "--steps", "2",
+           "--warmup", "1"]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=300,
+                       env=dict(os.environ, RANK="0"))
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "queries/s" and d["value"] > 0
+    assert d["higher_is_better"] is True and d["steps"] == 2 and d["warmup"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    r1 = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=300,
+                        env=dict(os.environ, RANK="1"))
+    assert r1.returncode == 0 and not r1.stdout.strip()
