@@ -47,7 +47,6 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "index_score_traffic.json")
 SCORE_SRC = os.path.join(ROOT, "long_context_decode_indexpool_b200", "csrc", "index_score.cu")
 
 GEN_CHUNK_TOKENS = 1 << 18  # tokens per device generation chunk
-SCORE_SAMPLE = 16  # decode steps per timed scoring launch
 
 
 def spx_module():
@@ -264,24 +263,54 @@ def recorded_traffic(kernel_key: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock and throttle-reason samples while the timed region runs.
+
+    NVML is polled from a host thread every ~0.2 ms, so that even a timed
+    region of a millisecond or two holds several samples; nvidia-smi (one
+    sample per 50 ms) is the fallback when NVML is not importable."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, device_index: int):
-        self.samples = []
+    def __init__(self, device_index: int, period_s: float = 2e-4):
+        self.samples = []  # (sm_mhz, sm_max_mhz, set of reason names)
+        self.period = period_s
         self.proc = None
         self.thread = None
+        self.stop_flag = threading.Event()
+        self.source = None
         self.gpu_id = None
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             self.gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:
             self.gpu_id = None
+        self.nvml = None
+        self.handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.handle = (pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id) if self.gpu_id
+                           else pynvml.nvmlDeviceGetHandleByIndex(device_index))
+            self.nvml = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self.reason_bits = (
+                ("hw_slowdown", pynvml.nvmlClocksEventReasonHwSlowdown),
+                ("hw_thermal_slowdown", pynvml.nvmlClocksEventReasonHwThermalSlowdown),
+                ("sw_thermal_slowdown", pynvml.nvmlClocksEventReasonSwThermalSlowdown),
+                ("sw_power_cap", pynvml.nvmlClocksEventReasonSwPowerCap))
+        except Exception:
+            self.nvml = None
 
-    def _cmd(self, loop: bool):
+    def _nvml_sample(self):
+        n = self.nvml
+        mhz = float(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM))
+        bits = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        return (mhz, self.max_mhz, {name for name, b in self.reason_bits if bits & b})
+
+    def _smi_cmd(self, loop: bool):
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits"]
         if self.gpu_id:
             cmd += ["-i", self.gpu_id]
@@ -289,58 +318,87 @@ class ClockSampler:
             cmd += ["-lms", "50"]
         return cmd
 
-    def start(self):
+    @classmethod
+    def _parse_smi(cls, line):
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 9:
+            return None
         try:
-            self.proc = subprocess.Popen(self._cmd(True), stdout=subprocess.PIPE,
+            sm, smax = float(parts[1]), float(parts[2])
+        except ValueError:
+            return None
+        return (sm, smax, {n for n, v in zip(cls.NAMES, parts[5:9]) if v.lower() in ("active", "1")})
+
+    def start(self):
+        self.samples = []
+        self.stop_flag.clear()
+        if self.nvml is not None:
+            self.source = "nvml"
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        self.samples.append(self._nvml_sample())
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 2.0:
+                time.sleep(1e-4)
+            self.samples.clear()  # keep only samples taken once the region has started
+            return
+        self.source = "nvidia-smi"
+        try:
+            self.proc = subprocess.Popen(self._smi_cmd(True), stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
+
         def reader():
             for line in self.proc.stdout:
-                self.samples.append(line.strip())
+                r = self._parse_smi(line)
+                if r:
+                    self.samples.append(r)
         self.thread = threading.Thread(target=reader, daemon=True)
         self.thread.start()
-        # nvidia-smi takes a while to start: wait for its first line so that the
-        # sampling covers the timed region, then keep only later samples
         t0 = time.time()
         while not self.samples and time.time() - t0 < 5.0 and self.proc.poll() is None:
             time.sleep(0.01)
         self.samples.clear()
 
     def stop(self):
+        self.stop_flag.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-            if self.thread:
-                self.thread.join(timeout=2)
+        if self.thread:
+            self.thread.join(timeout=2)
         if not self.samples:  # region shorter than one sampling period
             try:
-                out = subprocess.run(self._cmd(False), capture_output=True, text=True, timeout=20)
-                self.samples = [l.strip() for l in out.stdout.splitlines() if l.strip()]
+                if self.nvml is not None:
+                    self.samples = [self._nvml_sample()]
+                else:
+                    out = subprocess.run(self._smi_cmd(False), capture_output=True, text=True,
+                                         timeout=20)
+                    self.samples = [r for r in map(self._parse_smi, out.stdout.splitlines()) if r]
             except Exception:
                 pass
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for s in self.samples:
-            parts = [x.strip() for x in s.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for name, v in zip(names, parts[5:9]):
-                if v.lower() in ("active", "1"):
-                    reasons.add(name)
+        sm = [x[0] for x in self.samples]
+        smax = self.samples[-1][1] if self.samples else None
+        reasons = set()
+        for x in self.samples:
+            reasons |= x[2]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "sm_mhz_min": min(sm) if sm else None, "source": self.source}
 
 
 def dist_setup():
@@ -377,15 +435,42 @@ def shard_offset(rank: int, per_rank: int) -> int:
 
 
 def score_algorithmic_bytes(nblk_per_row, rows: int, keys: str = "bf16") -> int:
-    """Bytes the scoring kernel must move: every pooled key read once (256 B;
-    INT8 cache: 128 B of codes + a 4 B scale), every score written once
-    (4 B), plus each query row (8 KiB; INT8: 4 KiB of codes) and its head
-    weights (128 B)."""
+    """Bytes the scoring kernel must read (the step's own accounting, which
+    leaves out the scores it materialises): every pooled key once (256 B;
+    INT8 cache: 128 B of codes + a 4 B scale), plus each query row (8 KiB;
+    INT8: 4 KiB of codes) and its head weights (128 B)."""
     if keys == "int8":
-        per_blk, per_row = synth.IDX_DIM + 4 + 4, synth.IDX_HEADS * synth.IDX_DIM + synth.IDX_HEADS * 4
+        per_blk, per_row = synth.IDX_DIM + 4, synth.IDX_HEADS * synth.IDX_DIM + synth.IDX_HEADS * 4
     else:
-        per_blk, per_row = synth.IDX_DIM * 2 + 4, synth.IDX_HEADS * synth.IDX_DIM * 2 + synth.IDX_HEADS * 4
+        per_blk, per_row = synth.IDX_DIM * 2, synth.IDX_HEADS * synth.IDX_DIM * 2 + synth.IDX_HEADS * 4
     return int(sum(nblk_per_row)) * per_blk + rows * per_row
+
+
+def score_write_bytes(nblk_per_row) -> int:
+    """Bytes of fp32 scores the scoring kernel writes (overhead outside the
+    algorithmic accounting)."""
+    return int(sum(nblk_per_row)) * 4
+
+
+def step_algorithmic_bytes(B: int, L: int, heads: int, keys: str = "bf16") -> int:
+    """Bytes one decode step must move for B queries that see L tokens each:
+    pooled keys, the selected latent rows (512 blocks of 4 tokens plus the
+    partial tail, 1 KiB each), the indexer query and head weights, the MLA
+    query and the output."""
+    nblk = L // synth.POOL
+    S = min(nblk, synth.TOPK_BLOCKS) * synth.POOL + L % synth.POOL
+    per_q = (score_algorithmic_bytes([nblk], 1, keys) + S * synth.LATENT * 2
+             + 2 * heads * synth.LATENT * 2)
+    return B * per_q
+
+
+def attention_flops_prefill(pos0: int, T: int, heads: int) -> int:
+    """QK^T and PV flops of a prefill chunk: 4 H D per attended token."""
+    tot = 0
+    for t in range(T):
+        n = pos0 + t + 1
+        tot += min(n // synth.POOL, synth.TOPK_BLOCKS) * synth.POOL + n % synth.POOL
+    return 4 * heads * synth.LATENT * tot
 
 
 def score_algorithmic_flops_prefill(pos0: int, T: int) -> int:
@@ -522,23 +607,15 @@ def run_decode(args, world, rank, local):
         raise RuntimeError("device error during warm-up")
 
     K = args.steps
-    # The scoring kernel is timed on every SCORE_SAMPLE-th step: an event
-    # between two launches keeps the next kernel from starting early, so the
-    # other steps run without them.
-    ev_score = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for k in range(0, K, SCORE_SAMPLE)}
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for a, b in ev_score.values():  # torch creates its events on first record
-        a.record(stream)
-        b.record(stream)
     barrier(world)
     torch.cuda.synchronize(device)
     clocks = ClockSampler(device.index)
     clocks.start()
     n0 = spx.spx_launch_count()
     ev0.record(stream)
-    for k in range(K):
-        st.step(timing=ev_score.get(k))
+    for _ in range(K):
+        st.step()
     ev1.record(stream)
     torch.cuda.synchronize(device)
     launches = spx.spx_launch_count() - n0
@@ -546,46 +623,10 @@ def run_decode(args, world, rank, local):
     barrier(world)
     ms = ev0.elapsed_time(ev1)
     ms_max = max_over_ranks(ms, world, device)
-    score_ms = [a.elapsed_time(b) for a, b in ev_score.values()]
-    score_avg = sum(score_ms) / len(score_ms)
+    score_avg = time_scoring_launches(st, stream, max(8, min(K, 64)))
 
     # ---- end to end: host buffers in, host result out, every step ----------
-    # The step's inputs (new raw key, indexer query and weights, MLA query)
-    # travel in one pinned host buffer and one copy; the output comes back
-    # with one copy.
-    ins = (st.raw_new, st.q_idx, st.w_head, st.q)
-    sizes = [t.numel() * t.element_size() for t in ins]
-    offs = [0]
-    for n in sizes[:-1]:
-        offs.append(offs[-1] + (n + 255) // 256 * 256)
-    total = offs[-1] + sizes[-1]
-    h_in = torch.empty(total, dtype=torch.uint8, pin_memory=True)
-    for t, o, n in zip(ins, offs, sizes):
-        h_in[o:o + n].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
-    d_in = torch.empty(total, dtype=torch.uint8, device=device)
-    d_raw, d_qidx, d_w, d_q = (d_in[o:o + n].view(t.dtype).view(t.shape)
-                               for t, o, n in zip(ins, offs, sizes))
-    h_out = torch.empty(st.out.shape, dtype=st.out.dtype, pin_memory=True)
-    h2d = total
-    d2h = h_out.numel() * h_out.element_size()
-
-    def e2e_step():
-        d_in.copy_(h_in, non_blocking=True)
-        st.step(raw_new=d_raw, q_idx=d_qidx, w_head=d_w, q=d_q)
-        h_out.copy_(st.out, non_blocking=True)
-        stream.synchronize()
-
-    for _ in range(args.warmup):
-        e2e_step()
-    barrier(world)
-    torch.cuda.synchronize(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    e2e_ms, h2d, d2h = run_e2e(st, stream, K, args.warmup, world, device)
     if spx.spx_device_error() != 0:
         raise RuntimeError("device error during the timed region")
 
@@ -595,6 +636,8 @@ def run_decode(args, world, rank, local):
     nblk = [L // synth.POOL] * B
     alg = score_algorithmic_bytes(nblk, B, args.keys)
     achieved = alg / (score_avg * 1e-3) / 1e9
+    step_bytes = step_algorithmic_bytes(B, L, st.H, args.keys)
+    step_gbs = step_bytes / (ms_max / K * 1e-3) / 1e9
     queries = B * world * K
     i8 = args.keys == "int8"
     line = {
@@ -617,18 +660,100 @@ def run_decode(args, world, rank, local):
                    "parallelism": f"dp{world} (independent sequences)",
                    "l2": "inputs larger than L2 (pooled keys + 4 GiB latent per GPU)"},
         "roofline": {"bound": "hbm",
-                     "kernel": "k_index_score<1> (decode scoring" + (", INT8 cache)" if i8 else ")"),
+                     "kernel": "k_index_score (decode scoring" + (", INT8 cache)" if i8 else ")"),
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": f"{src} hbm_gbs",
                      "traffic": None if i8 else recorded_traffic("decode_1m"),
-                     "algorithmic_bytes_per_launch": alg, "avg_launch_us": score_avg * 1e3,
+                     "algorithmic_bytes_per_launch": alg,
+                     "score_write_bytes_per_launch": score_write_bytes(nblk),
+                     "avg_launch_us": score_avg * 1e3,
+                     "timed": "separate pass after the timed region, events around the launch",
                      "vs_8tbs": achieved / 8000.0},
+        "roofline_step": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes,
+                          "achieved": step_gbs, "unit": "GB/s", "peak": hbm,
+                          "frac": step_gbs / hbm, "peak_source": f"{src} hbm_gbs",
+                          "frac_of_8tbs": step_gbs / 8000.0},
         "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
     }
     return line
+
+
+def run_e2e(st, stream, K: int, warmup: int, world: int, device):
+    """K decode steps through the public call with host buffers: every step
+    copies its inputs (new raw key, indexer query and weights, MLA query:
+    one packed pinned buffer, one copy) to the device and its output back
+    to pinned host memory, and the host waits for every step's output.
+    Copies run on a second stream into two alternating device buffers, so
+    step k+1's inputs and step k-1's output move while step k computes; the
+    host waits for step k-1's output after enqueuing step k.  Timed by the
+    host clock from the first copy to the last output in host memory
+    (max over ranks).  Returns (ms, h2d bytes per step, d2h bytes per step)."""
+    ins = (st.raw_new, st.q_idx, st.w_head, st.q)
+    sizes = [t.numel() * t.element_size() for t in ins]
+    offs = [0]
+    for n in sizes[:-1]:
+        offs.append(offs[-1] + (n + 255) // 256 * 256)
+    total = offs[-1] + sizes[-1]
+    h_in = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    for t, o, n in zip(ins, offs, sizes):
+        h_in[o:o + n].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
+    d_in = [torch.empty(total, dtype=torch.uint8, device=device) for _ in range(2)]
+    views = [tuple(d[o:o + n].view(t.dtype).view(t.shape) for t, o, n in zip(ins, offs, sizes))
+             for d in d_in]
+    d_out = [torch.empty_like(st.out) for _ in range(2)]
+    h_out = [torch.empty(st.out.shape, dtype=st.out.dtype, pin_memory=True) for _ in range(2)]
+    copy = torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()
+    in_ready, used, out_ready, out_home = ([ev(), ev()] for _ in range(4))
+
+    def run(n):
+        for k in range(n):
+            i = k & 1
+            with torch.cuda.stream(copy):
+                if k >= 2:
+                    copy.wait_event(used[i])  # step k-2 has finished reading d_in[i]
+                d_in[i].copy_(h_in, non_blocking=True)
+                in_ready[i].record(copy)
+            stream.wait_event(in_ready[i])
+            raw, qi, wh, q = views[i]
+            st.step(raw_new=raw, q_idx=qi, w_head=wh, q=q, out=d_out[i])
+            used[i].record(stream)
+            with torch.cuda.stream(copy):
+                copy.wait_event(used[i])
+                h_out[i].copy_(d_out[i], non_blocking=True)
+                out_home[i].record(copy)
+            if k >= 1:
+                out_home[i ^ 1].synchronize()  # the host has step k-1's output
+        out_home[(n - 1) & 1].synchronize()
+
+    run(max(warmup, 2))
+    barrier(world)
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
+    run(K)
+    ms = (time.perf_counter() - t0) * 1e3
+    torch.cuda.synchronize(device)
+    return max_over_ranks(ms, world, device), total, h_out[0].numel() * h_out[0].element_size()
+
+
+def time_scoring_launches(st, stream, n: int) -> float:
+    """Average duration (ms) of the decode scoring kernel, from CUDA events
+    the fused call records on its stream around that launch, over n extra
+    steps run after the timed region (an event between two launches stops
+    the next one from starting early, so the timed steps carry none)."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for a, b in evs:  # torch creates its events on first record
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    for ev in evs:
+        st.step(timing=ev)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / n
 
 
 def run_indexshare(args, world, rank, local):
@@ -730,57 +855,157 @@ def run_host_latent(args, world, rank, local):
                        "batch_per_gpu": st.B, "context": st.L}}
 
 
-def run_prefill(args, world, rank, local):
+def measure_prefill(device, steps: int, warmup: int, world: int = 1):
+    """Times the chunked-prefill workload (4096 new tokens on a 131,072-token
+    cache, one fused call per step) and its scoring kernel; returns the
+    per-rank numbers and the state (for the oracle sample)."""
     spx = spx_module()
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
     w = synth.workload("prefill")
     st = PrefillState(w, device)
     stream = torch.cuda.current_stream(device)
-
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         st.step()
     torch.cuda.synchronize(device)
-    K = args.steps
-    ev_score = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(K)]
-    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(K)]
-    for a, b in ev_score:
-        a.record(stream)
-        b.record(stream)
-    torch.cuda.synchronize(device)
+    if spx.spx_device_error() != 0:
+        raise RuntimeError("device error during the prefill warm-up")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
+    torch.cuda.synchronize(device)
     clocks = ClockSampler(device.index)
     clocks.start()
     n0 = spx.spx_launch_count()
-    for k in range(K):
-        ev_step[k][0].record(stream)
-        st.step(timing=ev_score[k])
-        ev_step[k][1].record(stream)
+    ev0.record(stream)
+    for _ in range(steps):
+        st.step()
+    ev1.record(stream)
     torch.cuda.synchronize(device)
     launches = spx.spx_launch_count() - n0
     clocks.stop()
-    ms = sum(a.elapsed_time(b) for a, b in ev_step)
-    ms_max = max_over_ranks(ms, world, device)
-    score_avg = sum(a.elapsed_time(b) for a, b in ev_score) / K
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
+    # the scoring kernel, in a separate pass (events around its launch)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(max(3, min(steps, 10)))]
+    for a, b in evs:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    for ev in evs:
+        st.step(timing=ev)
+    torch.cuda.synchronize(device)
+    if spx.spx_device_error() != 0:
+        raise RuntimeError("device error during the prefill timing")
+    score_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    return st, dict(ms=ms, steps=steps, score_ms=score_ms, launches=int(launches),
+                    clocks=clocks.summary())
+
+
+def prefill_summary(st, m, world: int = 1):
+    """The prefill numbers against the tensor roofline (measured bf16 peaks)."""
+    hbm, bf16, bf16s, src = measured_peaks()
+    ms_step = m["ms"] / m["steps"]
+    f_idx = score_algorithmic_flops_prefill(st.pos0, st.T)
+    f_att = attention_flops_prefill(st.pos0, st.T, st.H)
+    step_tf = (f_idx + f_att) / (ms_step * 1e-3) / 1e12
+    score_tf = f_idx / (m["score_ms"] * 1e-3) / 1e12
+    return {
+        "workload": st.w.name, "ms_per_step": ms_step,
+        "queries_per_s": st.T * world / (ms_step * 1e-3),
+        "flops_per_step": {"indexer": f_idx, "attention": f_att},
+        "step_tflops": step_tf, "step_frac_of_burst": step_tf / bf16,
+        "step_frac_of_sustained": step_tf / bf16s,
+        "scoring_kernel": {"avg_launch_us": m["score_ms"] * 1e3, "tflops": score_tf,
+                           "frac_of_burst": score_tf / bf16, "frac_of_sustained": score_tf / bf16s},
+        "peak": {"bf16_burst_tflops": bf16, "bf16_sustained_tflops": bf16s, "source": src},
+        "gpu_launches_per_step": m["launches"] / m["steps"],
+        "clocks": m["clocks"],
+    }
+
+
+def prefill_cpu_baseline(st, nq: int = 256):
+    """The oracle (as it stands) on a stratified sample of the prefill
+    chunk's queries: each query scores every visible pooled block, keeps
+    the top 512 and attends over the gathered rows.  Queries run in
+    parallel, one host thread each; inputs are prepared untimed."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    pw = st.w.pool_weights()
+    pooled = oracle.pool(st.raw_keys_host(), pw)
+    sub = stratified_prefill_queries(st.T, nq)
+    rows = st.pos0 + np.asarray(sub)
+    q_idx, w_head, q = st.w.q_idx_np(rows), st.w.w_head_np(rows).astype(np.float64), st.w.q_np(rows)
+    sels = [None] * len(sub)
+    nthreads = oracle.threads(0)
+
+    def select(i):
+        sels[i] = oracle.select_query(q_idx[i], w_head[i], pooled, st.pos0 + sub[i] + 1, nthreads=1)[1]
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=nthreads) as ex:
+        list(ex.map(select, range(len(sub))))
+    t_sel = time.perf_counter() - t0
+    lat = [st.w.latent_np(0, oracle.token_set(sels[i], st.pos0 + sub[i] + 1)) for i in range(len(sub))]
+
+    def attend(i):
+        oracle.attention(q[i], lat[i], st.w.sm_scale)
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=nthreads) as ex:
+        list(ex.map(attend, range(len(sub))))
+    t_att = time.perf_counter() - t0
+    tot = t_sel + t_att
+    return {"value": len(sub) / tot, "unit": "queries/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"{len(sub)} stratified queries of the {st.T}-token prefill chunk on a "
+                      f"{st.pos0}-token cache (scoring, top-512, attention), fp64, {tot:.2f} s"}
+
+
+def stratified_prefill_queries(T: int, n: int = 256, seed: int = 5) -> list:
+    """A stratified subset of a prefill chunk's queries: the first and last
+    ones, every phase of the partial tail block (t % 4), both sides of the
+    edges of the scoring kernel's 8-query groups and of 128-block key tiles,
+    then seeded random queries up to n."""
+    qs = set(range(min(12, T))) | set(range(max(0, T - 8), T))
+    for g in (1, 2, 3, 64, 127, 128, 255, 256, 383, 511):
+        for t in (8 * g - 1, 8 * g):
+            if 0 <= t < T:
+                qs.add(t)
+    for k in range(1, 9):
+        for t in (512 * k - 4, 512 * k - 1, 512 * k):
+            if 0 <= t < T:
+                qs.add(t)
+    rng = np.random.default_rng(seed)
+    while len(qs) < min(n, T):
+        qs.add(int(rng.integers(0, T)))
+    return sorted(qs)[:n]
+
+
+def run_prefill(args, world, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    st, m = measure_prefill(device, args.steps, args.warmup, world)
     if rank != 0:
         return None
-    hbm, bf16, bf16s, src = measured_peaks()
-    flops = score_algorithmic_flops_prefill(st.pos0, st.T)
-    achieved = flops / (score_avg * 1e-3) / 1e12
-    return {
-        "metric": "sparse-attn chunked prefill queries/s; indexer tensor-core TFLOP/s",
-        "value": st.T * world * K / (ms_max * 1e-3), "unit": "queries/s", "n_gpus": world,
-        "steps": K, "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "pos0": st.pos0, "T": st.T, "heads": st.H},
+    summ = prefill_summary(st, m, world)
+    line = {
+        "metric": "sparse-attn chunked prefill queries/s; % of bf16 tensor peak",
+        "value": summ["queries_per_s"], "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": summ["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": st.w.name, "pos0": st.pos0, "T": st.T,
+                                        "heads": st.H},
         "roofline": {"bound": "tensor", "kernel": "k_index_score<8> (prefill scoring)",
-                     "achieved": achieved, "peak": bf16s, "unit": "TFLOP/s",
-                     "frac": achieved / bf16s, "peak_source": f"{src} bf16_tflops_sustained",
-                     "traffic": recorded_traffic("prefill"), "avg_launch_us": score_avg * 1e3},
-        "gpu_launches": int(launches), "clocks": clocks.summary(),
+                     "achieved": summ["scoring_kernel"]["tflops"],
+                     "peak": summ["peak"]["bf16_burst_tflops"], "unit": "TFLOP/s",
+                     "frac": summ["scoring_kernel"]["frac_of_burst"],
+                     "peak_source": f"{summ['peak']['source']} bf16_tflops (burst)",
+                     "traffic": None, "avg_launch_us": summ["scoring_kernel"]["avg_launch_us"]},
+        "roofline_step": {"bound": "tensor", "achieved": summ["step_tflops"], "unit": "TFLOP/s",
+                          "frac_of_burst": summ["step_frac_of_burst"],
+                          "frac_of_sustained": summ["step_frac_of_sustained"]},
+        "gpu_launches": m["launches"], "clocks": m["clocks"],
     }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = prefill_cpu_baseline(st)
+    return line
 
 
 def run_score_only(args, world, rank, local):
@@ -830,6 +1055,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("spx", "reference"), default="spx")
     ap.add_argument("--workload", default="1m", choices=synth.WORKLOADS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="leave the nested prefill measurement out of the decode line")
     ap.add_argument("--host-latent", action="store_true",
                     help="decode with the latent cache in pinned host memory")
     ap.add_argument("--indexshare", type=int, default=0, metavar="N",
@@ -857,11 +1084,22 @@ def main(argv=None):
         else:
             line = run_decode(args, world, rank, local)
         if rank == 0 and line is not None:
-            if (world == 1 and not args.no_cpu_baseline and args.workload != "prefill"
-                    and not args.score_only and args.indexshare <= 1
-                    and not args.host_latent and args.keys == "bf16"):
+            plain_decode = (args.workload != "prefill" and not args.score_only
+                            and args.indexshare <= 1 and not args.host_latent)
+            if (world == 1 and not args.no_cpu_baseline and plain_decode
+                    and args.keys == "bf16"):
                 line["cpu_baseline"] = cpu_baseline(synth.workload(args.workload),
                                                     torch.device("cuda", local))
+            if plain_decode and args.workload == "1m" and not args.no_prefill:
+                # the second target of the layer: chunked prefill on the tensor cores
+                dev = torch.device("cuda", local)
+                torch.cuda.empty_cache()
+                st, m = measure_prefill(dev, 10, 3)
+                pre = prefill_summary(st, m)
+                if world == 1 and not args.no_cpu_baseline:
+                    pre["cpu_baseline"] = prefill_cpu_baseline(st)
+                line["prefill"] = pre
+                del st
             print(json.dumps(line))
     finally:
         if world > 1:

@@ -119,6 +119,28 @@ SPX_API uint64_t spx_launch_count(void);
  * kernel reported an error since the last call. */
 SPX_API spx_status spx_device_error(int32_t* code, spx_stream stream);
 
+/* Self-test of the failure path of the kernels' bounded waits.  The pages
+ * describe no such call: it is library plumbing, so that a test can make a
+ * device-side wait run out on purpose and check that the host learns of it
+ * while the context stays usable.  It launches one CTA in which one thread
+ * starts a 1 KiB bulk copy into shared memory and then waits, with a limit of
+ * limit_ns nanoseconds, on an mbarrier that nothing will ever complete; a
+ * second thread waits on another such barrier with a limit 1000 times longer.
+ * The first wait gives up, sets the device error word (read it with
+ * spx_device_error: code 1) and the CTA's abort flag, which makes the second
+ * thread give up at once; the first thread then waits for its copy to land,
+ * as every kernel of the library does before it exits after a timeout.
+ *
+ *   limit_ns  1,000 .. 1,000,000,000
+ *   result    DEVICE int64 [6]: [0] first wait succeeded (0: it gave up),
+ *             [1] second wait succeeded (0: it gave up), [2] the copy landed
+ *             (1), [3] and [4] nanoseconds each thread waited, [5] the copied
+ *             bytes are right (1)
+ * Errors: SPX_ERR_INVALID_ARG for a null or misaligned result or a limit
+ * outside the range.  Asynchronous on the stream, like every other call. */
+SPX_API spx_status spx_selftest_wait_timeout(int64_t limit_ns, int64_t* result,
+                                             spx_stream stream);
+
 /* ---------------------------------------------------------------------------
  * Step 1 -- IndexPool cache write.  [W1] "IndexPool": k_pool = sum_i w_i k_i,
  * i = 1..4, sum_i w_i = 1, learned w.
@@ -127,8 +149,9 @@ SPX_API spx_status spx_device_error(int32_t* code, spx_stream stream);
  * position in the sequence) belongs to block p / 4 at slot p % 4.  For every
  * block that the append completes, the pooled key
  *     pooled_k[b][blk][d] = bf16_rne( sum_{i=0..3} pool_w[i] * key(4 blk + i)[d] )
- * is written (the sum is formed in fp32 and rounded once to bf16), taking
- * the older keys of the block from `tail`.  Keys of the still-incomplete last
+ * is written (the sum is formed in fp64, where each product of a bf16 key
+ * and an fp32 weight is exact, adding the four in time order from +0, and
+ * rounded once to bf16), taking the older keys of the block from `tail`.  Keys of the still-incomplete last
  * block are stored in tail[b][p % 4].  The caller advances its lengths by
  * n_new afterwards.
  *
@@ -203,7 +226,9 @@ SPX_API spx_status spx_topk_blocks(const spx_dims* d, int32_t rows,
  * scratch need (spx_topk_workspace_size) exceeds that size return
  * SPX_ERR_WORKSPACE before launching anything.  The first call on each device
  * looks up the array's device address (cudaGetSymbolAddress), so make that
- * first call before any stream capture.  All calls share the array: calls
+ * first call before any stream capture; the address is kept for the life of
+ * the process, which assumes the device is not reset (cudaDeviceReset) in
+ * between.  All calls share the array: calls
  * whose kernels overlap on the GPU race and must be serialised by the caller.
  * Arguments and results are those of spx_topk_blocks.
  * ------------------------------------------------------------------------- */
@@ -292,8 +317,8 @@ SPX_API spx_status spx_decode_fused(const spx_dims* d, int32_t B, const void* ra
  *         -149; 0 for an all-zero block),
  *     code_d = round-half-even(x_d / 2^e)  in [-127, 127],
  *     k_scale = 2^e  (fp32),
- * where x is the block's pooled value summed in fp32 (as spx_pool_append,
- * before any bf16 rounding).  The scoring calls quantise every query head
+ * where x is the block's pooled value summed in fp64 (as spx_pool_append,
+ * before any rounding).  The scoring calls quantise every query head
  * the same way (codes and 2^e_h) and compute
  *     scores[b][blk] = k_scale[b][blk] * sum_h (w_head[b][h] * 2^e_h) *
  *                      max(0, sum_d qcode[b][h][d] * code[b][blk][d])

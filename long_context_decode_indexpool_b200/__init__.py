@@ -64,6 +64,7 @@ _SIGS = {
     "spx_launch_count": ([], ctypes.c_uint64),
     "spx_dims_init": ([_DIMS, _I32, ctypes.c_float], ctypes.c_int),
     "spx_device_error": ([ctypes.POINTER(_I32), _P], ctypes.c_int),
+    "spx_selftest_wait_timeout": ([_I64, _P, _P], ctypes.c_int),
     "spx_pool_append": ([_DIMS, _I32, _P, _I32, _P, _P, _P, _I64, _P, _I64, _P], ctypes.c_int),
     "spx_index_score": ([_DIMS, _I32, _P, _P, _P, _I64, _P, _I64, _P, _I64, _P], ctypes.c_int),
     "spx_topk_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
@@ -174,6 +175,12 @@ def spx_device_error(stream=None) -> int:
     code = _I32(0)
     _check(_lib.spx_device_error(ctypes.byref(code), _stream(stream)), "spx_device_error")
     return code.value
+
+
+def spx_selftest_wait_timeout(limit_ns, result, stream=None):
+    """Launches the bounded-wait self-test kernel; result: int64 [6] on the device."""
+    _check(_lib.spx_selftest_wait_timeout(int(limit_ns), _ptr(result), _stream(stream)),
+           "spx_selftest_wait_timeout")
 
 
 def spx_pool_append(d, B, raw_k, n_new, pool_w, tail, pooled_k, cap_blk, len_dev, max_len,

@@ -26,14 +26,32 @@
 // 16+i hands the logits of tokens 0-31 to its partner (one shuffle each), so
 // both threads work on 32 logits.
 //
-// Per tile: 16-byte cp.async gather of the latent rows into the
-// 128-byte-swizzle K-major layout (double-buffered); S = Q C^T as 32
+// Per tile: gather of the latent rows into the 128-byte-swizzle K-major
+// layout (double-buffered).  From device memory every selected 4-token block
+// (4 KiB, contiguous) arrives as 8 TMA tile loads of [4 tokens x 64 dims],
+// one per 128-byte swizzle region, each completing on the tile's mbarrier;
+// the <= 3 tokens of the partial tail block and any cache in host memory
+// (mapped pinned rows) come with 16-byte cp.async.  S = Q C^T as 32
 // tcgen05.mma (M = 64, N = 64, K = 16); softmax in registers (running max in
 // base 2, raised lazily: O is rescaled only when a tile's max exceeds it by
 // more than 8); P (bf16) to shared memory; O += P C as 8 tcgen05.mma
 // (M = 64, N = 256, K = 16, C read MN-major from the same tile).  While the
 // first tile's softmax runs, the tensor core already computes the second
 // tile's logits.
+//
+// Fused selection (decode, kSel): instead of reading block ids chosen by a
+// selection kernel, the CTAs of a row's cluster choose them from the row's
+// fp32 scores and the complete 2048-bin histogram of their keys that the
+// scoring kernel left.  The histogram gives the bin of the 512th-largest key
+// (every CTA finds the same one); CTA k brings its contiguous slice of the
+// row's scores into shared memory with one bulk copy, keeps the keys at or
+// above that bin's lower edge (an exact top-512 of them when more qualify,
+// ties to the lower block), and publishes the list in its shared memory.
+// After a cluster barrier every CTA reads all lists through distributed
+// shared memory (slice order = block order) and makes the final choice
+// itself; the union of the slices' exact top-512 lists holds the row's top
+// 512, so the result equals a full sort.  CTA 0 of the cluster also writes
+// the ids and the count to global memory (outputs of the fused call).
 //
 // A row with a single split writes its normalised output directly.  The n
 // splits of one (row, head group) otherwise form a thread-block cluster: each
@@ -44,7 +62,9 @@
 // (weights 2^(m_s - M) l_s / L) into the bf16 output and the log-sum-exp.
 // No second kernel runs.
 #include <atomic>
+#include <cstring>
 
+#include "select.cuh"
 #include "spx_device.cuh"
 #include "spx_internal.h"
 #include "spx_launch.cuh"
@@ -99,7 +119,35 @@ struct KParams {
   float* lse;
   __nv_bfloat16* part_o;  // [rows, groups, nsplit, 64, 512] O / l of each split (nsplit > 1)
   float* part_ml;         // [rows, groups, nsplit, 64, 2]   (m, l)
+  int lat_batched;        // TMA path: row r reads latent batch r (else batch 0 for every row)
+  int lat_evict_first;    // TMA path: rows are read once (decode), evict them from L2 first
+  // fused selection (kSel): scores [rows, score_stride] (stride a multiple of
+  // 4), their key histograms [rows, 2048]; the chosen ids and counts go to
+  // idx_out / cnt_out (may be null)
+  const float* scores;
+  int64_t score_stride;
+  const uint32_t* ghist;
+  int32_t* idx_out;
+  int32_t* cnt_out;
 };
+
+constexpr int kSelPass = 16384;  // scores staged in shared memory at once (64 KiB)
+
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t ld_dsmem_u64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
   const int n = valid ? 16 : 0;
@@ -201,12 +249,13 @@ struct RowInfo {
   int S;         // tokens in the list
 };
 
-__device__ __forceinline__ RowInfo row_info(const KParams& p, int r) {
+// cnt: the row's selected-block count (from p.count, or chosen in the kernel)
+__device__ __forceinline__ RowInfo row_info(const KParams& p, int r, int cnt) {
   RowInfo ri;
   int64_t n = p.n_vis[r];
   n = n < 0 ? 0 : (n > p.len_cap ? p.len_cap : n);
   ri.nblk = n / kPool;
-  int c = p.count[r];
+  int c = cnt;
   c = c < 0 ? 0 : (c > kTopK ? kTopK : c);
   if (c > ri.nblk) c = static_cast<int>(ri.nblk);
   ri.cnt = c;
@@ -224,7 +273,157 @@ __device__ __forceinline__ int64_t token_pos_of(const RowInfo& ri, int j, int b)
   return ri.nblk * kPool + (j - ri.cnt * kPool);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
+// kTma: full selected blocks come by TMA through map_lat (a 3-D map over
+// [batches, cap_tok, 512] bf16 with a [1, 4, 64] box and the 128-byte
+// swizzle); otherwise every row is gathered with cp.async and map_lat is
+// unused.
+// Selection phase of kSel, run by the worker threads of every CTA of the
+// row's cluster (rank = split), see above.  Leaves this CTA's list of at most
+// 512 (key << 32 | block) entries, in block order, in `mylist` and its
+// length in *list_n; stage is 128 KiB of free shared memory.
+__device__ __forceinline__ void select_slice(const KParams& p, int r, int n_cl, int rank,
+                                             int64_t nblk, uint32_t theta, uint8_t* stage,
+                                             uint64_t* mylist, int* list_n, uint64_t* bar,
+                                             SelectSmem& ssm, bool& ok) {
+  const int tid = threadIdx.x;
+  const int64_t per = ((nblk + n_cl - 1) / n_cl + 3) & ~int64_t(3);  // a multiple of 4
+  const int64_t s0 = min(nblk, static_cast<int64_t>(rank) * per);
+  const int64_t s1 = min(nblk, s0 + per);
+  const float* srow = p.scores + static_cast<int64_t>(r) * p.score_stride;
+  const float* sf = reinterpret_cast<const float*>(stage);
+  // [4 x 512]: the warps' lists of a pass (fast path), or a pass's list (crowded path)
+  uint64_t* tmp = reinterpret_cast<uint64_t*>(stage + kSelPass * 4);
+  if (tid == 0) *list_n = 0;
+  int pass = 0;
+#pragma unroll 1
+  for (int64_t base = s0; base < s1; base += kSelPass, ++pass) {
+    const int nb = static_cast<int>(min(static_cast<int64_t>(kSelPass), s1 - base));
+    // rows are padded to a multiple of 4 scores: the copy may read <= 3 past s1
+    const uint32_t bytes = static_cast<uint32_t>((nb + 3) & ~3) * 4u;
+    group_sync<kWork, kBarWork>();  // the stage is free; *list_n is set
+    if (tid == 0) {
+      fence_proxy_async();  // earlier passes' reads of the stage come first
+      mbar_arrive_expect_tx(bar, bytes);
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              smem_u32(stage)),
+          "l"(srow + base), "r"(bytes), "r"(smem_u32(bar))
+          : "memory");
+    }
+    {
+      volatile int no_abort = 0;
+      ok &= mbar_wait(bar, pass & 1, &no_abort);
+    }
+    // Fast path (a handful of candidates): warp w compacts the keys at or
+    // above theta of its quarter of the pass, in block order, with coalesced
+    // 16-byte reads (lane l takes 4 consecutive scores) and a ballot scan,
+    // into its own buffer of up to 512 entries.
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      const int nvec = (nb + 3) >> 2;
+      const int seg = ((nvec + 3) / 4 + 31) & ~31;  // float4 per warp, a multiple of 32
+      const int v_end = min(nvec, (warp + 1) * seg);
+      uint64_t* wbuf = tmp + warp * kTopK;
+      const uint4* st4 = reinterpret_cast<const uint4*>(stage);
+      int wn = 0;
+#pragma unroll 1
+      for (int v0 = warp * seg; v0 < v_end; v0 += 32) {
+        const int v = v0 + lane;
+        const uint4 x = v < v_end ? st4[v] : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+        uint32_t kk[4];
+        int c = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          kk[e] = order_key(__uint_as_float(xs[e]));
+          const bool in = v < v_end && v * 4 + e < nb && kk[e] >= theta;
+          kk[e] = in ? kk[e] : 0u;
+          c += in;
+        }
+        const int incl = warp_incl_scan(c);
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        int pos = wn + incl - c;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (kk[e] != 0u && pos < kTopK)
+            wbuf[pos++] = (static_cast<uint64_t>(kk[e]) << 32) |
+                          static_cast<uint32_t>(base + v * 4 + e);
+        }
+        wn += total;
+      }
+      if (lane == 0) ssm.hist[warp] = wn;
+      group_sync<kWork, kBarWork>();
+      int wcnt[kWork / 32], wsum = 0;
+#pragma unroll
+      for (int w = 0; w < kWork / 32; ++w) {
+        wcnt[w] = ssm.hist[w];
+        wsum += wcnt[w];
+      }
+      bool fits = *list_n + wsum <= kTopK;
+#pragma unroll
+      for (int w = 0; w < kWork / 32; ++w) fits &= wcnt[w] <= kTopK;
+      if (fits) {  // uniform: append the warps' buffers in warp (= block) order
+        int off = *list_n;
+#pragma unroll
+        for (int w = 0; w < kWork / 32; ++w) {
+          for (int j = tid; j < wcnt[w]; j += kWork) mylist[off + j] = tmp[w * kTopK + j];
+          off += wcnt[w];
+        }
+        group_sync<kWork, kBarWork>();
+        if (tid == 0) *list_n = off;
+        continue;  // next pass (the loop's barrier orders the count)
+      }
+      group_sync<kWork, kBarWork>();
+    }
+    // Crowded cut bin: exact top-512 of every 4096 scores, merged.
+#pragma unroll 1
+    for (int sub = 0; sub < nb; sub += kWork * 32) {
+      uint32_t key[32];
+      uint32_t valid = 0;
+      const int i0 = sub + tid * 32;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        key[i] = i0 + i < nb ? order_key(sf[i0 + i]) : 0u;
+        if (i0 + i < nb && key[i] >= theta) valid |= 1u << i;
+      }
+      uint32_t thr;
+      const int64_t b0 = base + i0;
+      const int n = group_select<32, kWork, kBarWork>(key, valid, kTopK, tid, ssm, &thr,
+                                                      [&](int i, int pos) {
+        tmp[pos] = (static_cast<uint64_t>(key[i]) << 32) | static_cast<uint32_t>(b0 + i);
+      });
+      group_sync<kWork, kBarWork>();
+      const int ln = *list_n;
+      if (ln + n <= kTopK) {  // uniform: append (block order is kept)
+        for (int j = tid; j < n; j += kWork) mylist[ln + j] = tmp[j];
+        group_sync<kWork, kBarWork>();
+        if (tid == 0) *list_n = ln + n;
+      } else {
+        // the exact top 512 of the list and this pass's survivors (<= 1024,
+        // list first: block order)
+        uint32_t k8[8];
+        uint64_t e8[8];
+        uint32_t v8 = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int q = tid * 8 + i;
+          e8[i] = q < ln ? mylist[q] : (q - ln < n ? tmp[q - ln] : 0ull);
+          k8[i] = static_cast<uint32_t>(e8[i] >> 32);
+          if (q < ln + n) v8 |= 1u << i;
+        }
+        const int m = group_select<8, kWork, kBarWork>(k8, v8, kTopK, tid, ssm, &thr,
+                                                       [&](int i, int pos) { mylist[pos] = e8[i]; });
+        group_sync<kWork, kBarWork>();
+        if (tid == 0) *list_n = m;
+      }
+    }
+  }
+  group_sync<kWork, kBarWork>();
+}
+
+template <bool kTma, bool kSel>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_sparse_attn(const __grid_constant__ CUtensorMap map_lat, const KParams p) {
   extern __shared__ uint8_t dyn[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -236,7 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   uint64_t* bar_qk = reinterpret_cast<uint64_t*>(vm_s + kPosCap / 32);  // [2]: S buffer b done
   uint64_t* bar_pv = bar_qk + 2;
   uint64_t* bar_red = bar_qk + 3;  // combine: rows of the other splits
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 4);
+  uint64_t* bar_kv = bar_qk + 4;   // [2]: TMA bytes of latent tile buffer b landed
+  uint64_t* bar_sc = bar_qk + 6;   // kSel: staged scores landed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 7);
 
   const int split = blockIdx.x, r = blockIdx.y, hg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -255,7 +456,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     mbar_init(&bar_qk[1], 1);
     mbar_init(bar_pv, 1);
     mbar_init(bar_red, 1);
+    mbar_init(&bar_kv[0], kWork / 32);  // one arrive.expect_tx per worker warp and tile
+    mbar_init(&bar_kv[1], kWork / 32);
+    mbar_init(bar_sc, 1);
     fence_mbar_init();
+  }
+  if constexpr (kTma && !kSel) {  // (kSel: after the selection, which uses the buffers)
+    if (tid == 0) prefetch_tensormap(&map_lat);
+    // Rows a tile does not load (skipped blocks, padding, the rest of the
+    // tail block) keep what the buffer held: zero at first, then latent rows
+    // of earlier tiles, so masked tokens (P = 0) never multiply a non-finite
+    // value.  The zeros are written before any TMA write to the buffers.
+    if (worker) {
+      for (int i = tid; i < 2 * kKVBytes / 16; i += kWork)
+        *reinterpret_cast<uint4*>(kv_s + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async();
+    }
   }
   if (warp == 0) {
     tmem_alloc(tmem_holder, 512);
@@ -273,36 +489,146 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     }
   }
   pdl_trigger();
-  pdl_wait();  // the selected blocks come from the previous kernel
+  pdl_wait();  // the selected blocks (or the scores) come from the previous kernel
+  bool ok_all = true;
+
+  const int32_t* idx_row = p.idx + static_cast<int64_t>(r) * kTopK;
+  int row_cnt;
+  if constexpr (kSel) {
+    __shared__ SelectSmem ssm;
+    __shared__ MergeSmem msm;
+    __shared__ int s_list_n, s_sel_n;
+    // the list of this CTA: in the tail of the position array, which this
+    // split's positions never reach while the cluster may read it
+    uint64_t* mylist = reinterpret_cast<uint64_t*>(pos_s + kPosCap - kTopK);
+    int32_t* sel_s = reinterpret_cast<int32_t*>(p_s);  // chosen ids, until P is written
+    int64_t nv = p.n_vis[r];
+    nv = nv < 0 ? 0 : (nv > p.len_cap ? p.len_cap : nv);
+    const int64_t nblk = nv / kPool;
+    const int rank = n_cl > 1 ? static_cast<int>(cluster_rank()) : 0;
+    int cut_bin = -1, above = 0;
+    if (worker) {
+      cut_bin_of<kWork, kBarWork>(p.ghist + static_cast<int64_t>(r) * kSelHistBins, kTopK, tid,
+                                  ssm, &cut_bin, &above);
+      const uint32_t theta = cut_bin < 0 ? 0u : static_cast<uint32_t>(cut_bin) << kSelKeyShift;
+      select_slice(p, r, n_cl, rank, nblk, theta, kv_s, mylist, &s_list_n, bar_sc, ssm, ok_all);
+    }
+    if (n_cl > 1) cluster_sync_all();  // every list is published
+    else __syncthreads();
+    if (worker) {
+      // the union of the lists, in rank (= block) order, into the stage
+      uint32_t* ukey = reinterpret_cast<uint32_t*>(kv_s);
+      int32_t* uid = reinterpret_cast<int32_t*>(kv_s + pad32(kMaxCluster * kTopK) * 4);
+      const uint32_t ln_local = smem_u32(&s_list_n), l_local = smem_u32(mylist);
+      int cnt_k = 0;
+      if (tid < n_cl) cnt_k = n_cl > 1 ? static_cast<int>(ld_dsmem_u32(dsmem_addr(ln_local, tid)))
+                                       : s_list_n;
+      int tot;
+      const int off_k = group_excl_scan<kWork, kBarWork>(cnt_k, tid, ssm.scan, &tot);
+      if (tid < n_cl) ssm.hist[tid] = off_k;  // (hist is free scratch here)
+      if (tid == 0) {
+        msm.kmin = 0xFFFFFFFFu;
+        msm.kmax = 0;
+      }
+      for (int b = tid; b < 3 * 128; b += kWork) (&msm.rh[0][0])[b] = 0;
+      if (tid < 3) {
+        msm.dig[tid] = 0;
+        msm.abv[tid] = 0;
+      }
+      group_sync<kWork, kBarWork>();
+#pragma unroll 1
+      for (int f = tid; f < tot; f += kWork) {
+        int k = 0;
+        while (k + 1 < n_cl && ssm.hist[k + 1] <= f) ++k;
+        const int j = f - ssm.hist[k];
+        const uint64_t e = n_cl > 1 ? ld_dsmem_u64(dsmem_addr(l_local + j * 8, k)) : mylist[j];
+        ukey[pad32(f)] = static_cast<uint32_t>(e >> 32);
+        uid[pad32(f)] = static_cast<int32_t>(static_cast<uint32_t>(e));
+      }
+      group_sync<kWork, kBarWork>();
+      const uint32_t theta = cut_bin < 0 ? 0u : static_cast<uint32_t>(cut_bin) << kSelKeyShift;
+      merge_final<kWork, kBarWork>(ukey, uid, tot, theta, cut_bin, above, ssm, msm, sel_s, &s_sel_n,
+                                   tid);
+      group_sync<kWork, kBarWork>();
+      if (rank == 0 && hg == 0) {
+        if (p.idx_out)
+          for (int j = tid; j < kTopK; j += kWork) p.idx_out[static_cast<int64_t>(r) * kTopK + j] = sel_s[j];
+        if (p.cnt_out && tid == 0) p.cnt_out[r] = s_sel_n;
+      }
+      if constexpr (kTma) {  // see the zero fill above: now the buffers are free
+        for (int i = tid; i < 2 * kKVBytes / 16; i += kWork)
+          *reinterpret_cast<uint4*>(kv_s + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async();
+      }
+    }
+    __syncthreads();
+    idx_row = sel_s;
+    row_cnt = s_sel_n;
+  } else {
+    row_cnt = p.count[r];
+  }
 
   // the block id of this thread's first list entry goes out with the row's
   // length and count (one round trip instead of two)
   const int j_first = split * p.split_tokens + tid;
-  const int32_t* idx_row = p.idx + static_cast<int64_t>(r) * kTopK;
   const int b_first = (worker && j_first < kTopK * kPool) ? idx_row[j_first >> 2] : -1;
-  const RowInfo ri = row_info(p, r);
+  const RowInfo ri = row_info(p, r, row_cnt);
   const int j_begin = split * p.split_tokens;
   const int j_end = split == n_cl - 1 ? ri.S : min(ri.S, j_begin + p.split_tokens);
   const int nlist = j_end > j_begin ? j_end - j_begin : 0;
   const int ntiles = (nlist + kTT - 1) / kTT;
   float m_run = -INFINITY, l_run = 0.f;  // of head hloc (both threads)
-  bool ok_all = true;
   uint32_t tmem = 0;
 
   if (ntiles > 0) {  // uniform
     const __nv_bfloat16* lat = p.latent + static_cast<int64_t>(r) * p.seq_stride;
+    const uint64_t lat_pol = p.lat_evict_first ? l2_evict_first_policy() : l2_evict_normal_policy();
     auto gather = [&](int tile) {
       const int row0 = (tile & 1) * kTT;
       const int64_t* ps = pos_s + tile * kTT;
+      if constexpr (kTma) {
+        // thread t: 4-token group g = t / 8 of the tile, swizzle region c = t % 8
+        const int g = tid >> 3, c = tid & 7;
+        const int64_t pos0 = ps[4 * g];
+        const bool full = j_begin + tile * kTT + 4 * g < ri.cnt * kPool && pos0 >= 0;
+        const uint32_t ball = __ballot_sync(0xffffffffu, full && c == 0);
+        uint64_t* bar = &bar_kv[tile & 1];
+        if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(__popc(ball)) * 4096u);
+        __syncwarp();
+        if (full)
+          tma_load_3d_hint(kv_s + c * kKVRegion + (row0 + 4 * g) * 128, &map_lat, bar, c * 64,
+                           static_cast<int>(pos0), p.lat_batched ? r : 0, lat_pol);
+        else {
+          // tokens of the partial tail block: this thread's 128-byte region of each
+#pragma unroll 1
+          for (int i = 0; i < 4; ++i) {
+            const int64_t pos = ps[4 * g + i];
+            if (pos < 0) continue;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              cp_async16(kv_u + kv_off(row0 + 4 * g + i, c * 8 + q),
+                         lat + pos * kLatent + (c * 8 + q) * 8, true);
+          }
+        }
+      } else {
 #pragma unroll 4
-      for (int i = 0; i < (kTT * 64) / kWork; ++i) {
-        const int c = i * kWork + tid;
-        const int t = c >> 6, piece = c & 63;
-        const int64_t pos = ps[t];
-        cp_async16(kv_u + kv_off(row0 + t, piece), lat + (pos >= 0 ? pos : 0) * kLatent + piece * 8,
-                   pos >= 0);
+        for (int i = 0; i < (kTT * 64) / kWork; ++i) {
+          const int c = i * kWork + tid;
+          const int t = c >> 6, piece = c & 63;
+          const int64_t pos = ps[t];
+          cp_async16(kv_u + kv_off(row0 + t, piece), lat + (pos >= 0 ? pos : 0) * kLatent + piece * 8,
+                     pos >= 0);
+        }
       }
       cp_async_commit();
+    };
+    // the TMA bytes of tile t have landed (cp.async parts are waited for by
+    // the caller with cp_async_wait)
+    auto tma_landed = [&](int t) {
+      if constexpr (kTma) {
+        volatile int no_abort = 0;
+        ok_all &= mbar_wait(&bar_kv[t & 1], (t >> 1) & 1, &no_abort);
+      }
     };
     if (worker) {
       // every token position of the split, once, with a validity bit per token
@@ -387,15 +713,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         if (j == 0) {
           if (ntiles > 1) cp_async_wait<1>();
           else cp_async_wait<0>();
+          tma_landed(0);
           fence_proxy_async();
           named_arrive(kBarData0, kThreads);
           if (ntiles > 1) {
             cp_async_wait<0>();
+            tma_landed(1);
             fence_proxy_async();
             named_arrive(kBarData1, kThreads);
           }
         } else if (j >= 2) {
           cp_async_wait<0>();
+          tma_landed(j);
           fence_proxy_async();
           named_arrive(kBarData0 + buf, kThreads);
         }
@@ -658,6 +987,7 @@ int active_clusters(int n) {
   int lg = 0;
   while ((1 << lg) < n) ++lg;
   if (dev < 64 && cache[dev][lg].load() > 0) return cache[dev][lg].load() - 1;
+  // both instantiations have the same launch shape and shared memory
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -670,7 +1000,7 @@ int active_clusters(int n) {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int num = 0;
-  if (cudaOccupancyMaxActiveClusters(&num, k_sparse_attn, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&num, k_sparse_attn<true, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     num = 0;
   }
@@ -692,19 +1022,37 @@ int pick_cluster(int want, int64_t units) {
   return fits_at_all;
 }
 
+template <bool kTma, bool kSel>
+bool set_attrs_for() {
+  return cudaFuncSetAttribute(k_sparse_attn<kTma, kSel>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) ==
+             cudaSuccess &&
+         cudaFuncSetAttribute(k_sparse_attn<kTma, kSel>,
+                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+}
+
 bool set_attrs() {
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && attr_set[dev]) return true;
-  if (cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmemBytes) != cudaSuccess)
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < 64 && attr_set[dev]) return true;
+  if (!set_attrs_for<true, false>() || !set_attrs_for<false, false>() ||
+      !set_attrs_for<true, true>() || !set_attrs_for<false, true>())
     return false;
-  if (cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-      cudaSuccess)
-    return false;
-  if (dev < 64) attr_set[dev] = true;
+  if (dev >= 0 && dev < 64) attr_set[dev] = true;
   return true;
+}
+
+// Whether the latent rows can come by TMA: device memory (not mapped host
+// rows), a row stride the tensor map can express.
+bool latent_tma_ok(const void* latent, int64_t seq_stride, int64_t cap_tok) {
+  if ((seq_stride * 2) % 16 != 0 || cap_tok > (int64_t(1) << 31) - 1) return false;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, latent) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeDevice;
 }
 
 }  // namespace
@@ -763,14 +1111,37 @@ cudaError_t launch_attn(const AttnPlan& pl0, const AttnArgs& a, cudaStream_t str
   p.lse = a.lse;
   p.part_o = nullptr;
   p.part_ml = nullptr;
+  const bool sel = a.sel_scores != nullptr;
+  p.scores = a.sel_scores;
+  p.score_stride = a.sel_stride;
+  p.ghist = a.sel_hist;
+  p.idx_out = sel ? const_cast<int32_t*>(a.idx) : nullptr;
+  p.cnt_out = sel ? const_cast<int32_t*>(a.count) : nullptr;
+  p.lat_batched = a.seq_stride != 0 ? 1 : 0;
+  p.lat_evict_first = a.seq_stride != 0 ? 1 : 0;  // decode rows are read once; a shared cache is reused
   if (pl.nsplit > 1) {
     const size_t units_n = static_cast<size_t>(pl.rows) * pl.groups * pl.nsplit * kHG;
     p.part_o = static_cast<__nv_bfloat16*>(a.ws);
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
                                          ((units_n * kLatent * 2 + 255) & ~static_cast<size_t>(255)));
   }
-  cudaError_t e = launch_ex(k_sparse_attn, dim3(pl.nsplit, pl.rows, pl.groups), dim3(kThreads),
-                            kSmemBytes, stream, a.pdl, pl.nsplit, p);
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof(map));
+  bool tma = latent_tma_ok(a.latent, a.seq_stride, a.cap_tok);
+  if (tma) {
+    const uint64_t nb = a.seq_stride != 0 ? static_cast<uint64_t>(pl.rows) : 1u;
+    const uint64_t dims[3] = {static_cast<uint64_t>(kLatent), static_cast<uint64_t>(a.cap_tok), nb};
+    const uint64_t strides[2] = {kLatent * 2ull,
+                                 a.seq_stride != 0 ? static_cast<uint64_t>(a.seq_stride) * 2ull
+                                                   : static_cast<uint64_t>(a.cap_tok) * kLatent * 2ull};
+    const uint32_t box[3] = {64, kPool, 1};
+    tma = encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.latent, dims, strides, box,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  auto kernel = tma ? (sel ? k_sparse_attn<true, true> : k_sparse_attn<true, false>)
+                    : (sel ? k_sparse_attn<false, true> : k_sparse_attn<false, false>);
+  cudaError_t e = launch_ex(kernel, dim3(pl.nsplit, pl.rows, pl.groups), dim3(kThreads),
+                            kSmemBytes, stream, a.pdl, pl.nsplit, map, p);
   count_launches(1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

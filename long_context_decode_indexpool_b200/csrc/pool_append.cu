@@ -7,12 +7,15 @@
 //
 // Block b holds tokens 4b..4b+3 in time order; w_i weighs the i-th of them.
 // A block is pooled when its last token is appended; until then its raw keys
-// wait in a 3-slot tail per sequence.  The pooled value is the fp32 sum
-// rounded once to bf16 (round-to-nearest-even), or, in the INT8 cache
-// ([W1] section "양자화: W8A8와 혼합 캐시": far, compressed indexer entries in
-// INT8), that sum as int8 codes with one power-of-two scale per block
-// (i8_exponent / i8_code); the 16 threads of a block find its max |x| by
-// shuffles.
+// wait in a 3-slot tail per sequence.  The pooled value is formed in fp64
+// (each product of a bf16 key and an fp32 weight is exact there; the four
+// are added in time order, starting from +0) and rounded once: to bf16
+// (round-to-nearest-even), or, in the INT8 cache ([W1] section "양자화:
+// W8A8와 혼합 캐시": far, compressed indexer entries in INT8), to int8 codes
+// with one power-of-two scale per block; the 16 threads of a block find its
+// max |x| by shuffles.  With learned (non-dyadic) weights an fp32 sum would
+// round twice and could land one bf16 step away from the single rounding of
+// the exact value; the fp64 sum does not.
 //
 // Work split: grid (x, B).  CTA x of sequence b pools blocks
 // blk_lo + x*kBlocksPerCta ..; 16 threads per block, 8 dims (16 bytes) per
@@ -21,6 +24,7 @@
 // tail slot is overwritten before it has been read.
 #include "spx_device.cuh"
 #include "spx_internal.h"
+#include "spx_launch.cuh"
 
 namespace spx {
 
@@ -30,6 +34,41 @@ constexpr int kPoolThreads = 128;
 constexpr int kChunksPerRow = kIdxDim / 8;                          // 16
 constexpr int kBlocksPerPass = kPoolThreads / kChunksPerRow;        // 8
 constexpr int kBlocksPerCta = 8 * kBlocksPerPass;                   // 64
+
+// bf16 bits of the nearest-even rounding of a double: 8 significant bits
+// from 2^-126 up, a fixed spacing of 2^-133 below (the bf16 subnormals).
+__device__ __forceinline__ uint16_t bf16_rne_f64(double v) {
+  const double a = fabs(v);
+  double r;
+  if (a >= 0x1p-126) {
+    // keep 7 of the 52 stored fraction bits: add just under half of the
+    // dropped weight (plus one on a tie with an odd kept part), then clear
+    uint64_t u = static_cast<uint64_t>(__double_as_longlong(a));
+    u += ((1ull << 44) - 1ull) + ((u >> 45) & 1ull);
+    u &= ~((1ull << 45) - 1ull);
+    r = __longlong_as_double(static_cast<long long>(u));
+  } else {
+    r = rint(a * 0x1p133) * 0x1p-133;  // exact scalings around one rounding
+  }
+  // r has at most 8 significant bits: its fp32 conversion is exact (or inf
+  // above the fp32 range), and bf16 is the fp32 pattern's top half
+  const uint32_t f = __float_as_uint(__double2float_rn(r));
+  return static_cast<uint16_t>((f >> 16) | (signbit(v) ? 0x8000u : 0u));
+}
+
+// INT8 code exponent of an fp64 vector maximum (as i8_exponent): the
+// smallest e with amax <= 127 * 2^e, not below -149, 0 for amax = 0.
+__device__ __forceinline__ int i8_exponent_f64(double amax) {
+  if (!(amax > 0.0)) return 0;
+  int E = 0;
+  const double m = frexp(amax, &E);
+  const int e = m <= 127.0 / 128.0 ? E - 7 : E - 6;
+  return e < -149 ? -149 : e;
+}
+
+__device__ __forceinline__ uint32_t i8_code_f64(double x, int e) {
+  return static_cast<uint32_t>(__double2int_rn(ldexp(x, -e))) & 0xffu;
+}
 
 __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
   uint4 u = *reinterpret_cast<const uint4*>(p);
@@ -90,6 +129,10 @@ struct PoolKParams {
 template <bool I8>
 __global__ void __launch_bounds__(kPoolThreads) k_pool_append(const PoolKParams p) {
   pdl_trigger();
+  // Launched early (after the previous step's last kernel started), it waits
+  // for that kernel to finish before touching anything: the previous step's
+  // selection state and lengths are rewritten here.
+  pdl_wait();
   const int b = blockIdx.y;
   int64_t len = p.len_dev ? p.len_dev[b] : p.len_host;
   // Clamp so that every access stays inside the caches whatever the device
@@ -124,7 +167,8 @@ __global__ void __launch_bounds__(kPoolThreads) k_pool_append(const PoolKParams 
     if (blk0 >= blk_done) break;  // uniform
     const int64_t blk = blk0 + sub;
     const bool active = blk < blk_done;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    // fp64 sum from +0 in time order (each product is exact)
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
     if (active) {
 #pragma unroll
       for (int i = 0; i < kPool; ++i) {
@@ -133,25 +177,24 @@ __global__ void __launch_bounds__(kPoolThreads) k_pool_append(const PoolKParams 
                                              : raw_b + (t - len) * kIdxDim;
         float f[8];
         load8(src + chunk * 8, f);
+        const double wi = static_cast<double>(p.w[i]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = (i == 0) ? f[e] * p.w[0] : __fmaf_rn(f[e], p.w[i], acc[e]);
+        for (int e = 0; e < 8; ++e) acc[e] = __fma_rn(static_cast<double>(f[e]), wi, acc[e]);
       }
     }
     if constexpr (I8) {
       // the block's 16 threads are lanes 0-15 or 16-31 of one warp
-      float amax = 0.f;
+      double amax = 0.0;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(acc[e]));
+      for (int e = 0; e < 8; ++e) amax = fmax(amax, fabs(acc[e]));
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const int ex = i8_exponent(amax);
+      for (int o = 8; o > 0; o >>= 1) amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const int ex = i8_exponent_f64(amax);
       uint32_t w2[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        w2[h] = (static_cast<uint32_t>(i8_code(acc[4 * h], ex)) & 0xffu) |
-                ((static_cast<uint32_t>(i8_code(acc[4 * h + 1], ex)) & 0xffu) << 8) |
-                ((static_cast<uint32_t>(i8_code(acc[4 * h + 2], ex)) & 0xffu) << 16) |
-                (static_cast<uint32_t>(i8_code(acc[4 * h + 3], ex)) << 24);
+        w2[h] = i8_code_f64(acc[4 * h], ex) | (i8_code_f64(acc[4 * h + 1], ex) << 8) |
+                (i8_code_f64(acc[4 * h + 2], ex) << 16) | (i8_code_f64(acc[4 * h + 3], ex) << 24);
       if (active) {
         int8_t* row = static_cast<int8_t*>(p.pooled) +
                       (static_cast<int64_t>(b) * p.cap_blk + blk) * kIdxDim;
@@ -160,10 +203,12 @@ __global__ void __launch_bounds__(kPoolThreads) k_pool_append(const PoolKParams 
       }
     } else {
       if (active) {
-        uint4 o;
-        __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&o);
+        uint32_t h2[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) oh[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+        for (int e = 0; e < 4; ++e)
+          h2[e] = static_cast<uint32_t>(bf16_rne_f64(acc[2 * e])) |
+                  (static_cast<uint32_t>(bf16_rne_f64(acc[2 * e + 1])) << 16);
+        const uint4 o = make_uint4(h2[0], h2[1], h2[2], h2[3]);
         __nv_bfloat16* row = static_cast<__nv_bfloat16*>(p.pooled) +
                              (static_cast<int64_t>(b) * p.cap_blk + blk) * kIdxDim;
         *reinterpret_cast<uint4*>(row + chunk * 8) = o;
@@ -223,11 +268,12 @@ cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream) {
   p.w_head = a.w_head;
   p.q8 = a.q8;
   p.wq = a.wq;
-  if (a.i8)
-    k_pool_append<true><<<grid, kPoolThreads, 0, stream>>>(p);
-  else
-    k_pool_append<false><<<grid, kPoolThreads, 0, stream>>>(p);
+  cudaError_t e = a.i8 ? launch_ex(k_pool_append<true>, grid, dim3(kPoolThreads), 0, stream,
+                                   a.pdl, 1, p)
+                       : launch_ex(k_pool_append<false>, grid, dim3(kPoolThreads), 0, stream,
+                                   a.pdl, 1, p);
   count_launches(1);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

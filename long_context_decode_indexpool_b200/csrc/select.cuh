@@ -9,6 +9,7 @@
 #pragma once
 
 #include "spx_device.cuh"
+#include "spx_internal.h"
 
 namespace spx {
 
@@ -192,6 +193,179 @@ __device__ __forceinline__ int group_select(const uint32_t (&key)[E], uint32_t v
   }
   *thr = prefix;
   return total;
+}
+
+// Scores are counted by their top 11 key bits (sign, exponent, 2 mantissa
+// bits) in 2048-bin histograms; the bin of a key is key >> kSelKeyShift.
+constexpr int kSelKeyShift = 32 - 11;
+
+// Shared state of the final choice.
+struct MergeSmem {
+  int rh[3][128];  // radix histograms of the three 7-bit digits below the cut bin
+  int dig[3], abv[3];
+  uint32_t kmin, kmax;
+};
+
+// The row's result from the n buffered (key, block) pairs, in block order;
+// entries below lo_key are not candidates.  Every candidate above the cut
+// bin is selected; the (K - above) best of the cut bin (ties: lower block)
+// complete the set.  Writes the ascending block ids, -1 padded, and the
+// count.  This code runs once per row: its loops stay rolled, so that it is
+// short (instruction fetch, not arithmetic, bounds a one-pass kernel).
+template <int NT, int BAR>
+__device__ __noinline__ void merge_final(const uint32_t* bk, const int32_t* bi, int n_in,
+                                         uint32_t lo_key, int cut_bin, int above, SelectSmem& sm,
+                                         MergeSmem& ms, int32_t* dst, int32_t* cnt_out,
+                                         int gtid) {
+  const int tid = gtid;
+  const int per = (n_in + NT - 1) / NT;
+  const int q0 = min(tid * per, n_in), q1 = min(q0 + per, n_in);
+  const bool cut = cut_bin >= 0;  // uniform
+  const uint32_t cut_lo = cut ? static_cast<uint32_t>(cut_bin) << kSelKeyShift : 0u;
+  const uint32_t cut_hi = cut ? cut_lo | ((1u << kSelKeyShift) - 1u) : 0xFFFFFFFFu;
+  const uint32_t in_lo = lo_key > cut_lo ? lo_key : cut_lo;
+  // candidate classes: sure (above the cut bin, or every candidate when no
+  // cut is needed) and in-cut
+  uint32_t T = 0xFFFFFFFFu;
+  int need_eq = 0;
+  if (cut) {
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0;
+#pragma unroll 1
+    for (int q = q0; q < q1; ++q) {
+      const uint32_t k = bk[pad32(q)];
+      if (k >= in_lo && k <= cut_hi) {
+        kmin = k < kmin ? k : kmin;
+        kmax = k > kmax ? k : kmax;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint32_t x = __shfl_xor_sync(0xffffffffu, kmin, o);
+      const uint32_t y = __shfl_xor_sync(0xffffffffu, kmax, o);
+      kmin = x < kmin ? x : kmin;
+      kmax = y > kmax ? y : kmax;
+    }
+    if ((tid & 31) == 0 && kmin <= kmax) {
+      atomicMin(&ms.kmin, kmin);
+      atomicMax(&ms.kmax, kmax);
+    }
+    group_sync<NT, BAR>();
+    // the candidates of the cut bin share every bit above the highest one
+    // where their min and max differ; the rest comes from radix passes
+    kmin = ms.kmin;
+    const uint32_t diff = kmin ^ ms.kmax;
+    uint32_t prefix = 0, pmask = 0;
+    int rem = kTopK - above;
+#pragma unroll 1
+    for (int d = 0; d < 3; ++d) {
+      const int shift = 14 - 7 * d;
+      if ((diff >> shift) == 0) {  // uniform
+        prefix |= kmin & (127u << shift);
+        pmask |= 127u << shift;
+        continue;
+      }
+#pragma unroll 1
+      for (int q = q0; q < q1; ++q) {
+        const uint32_t k = bk[pad32(q)];
+        if (k >= in_lo && k <= cut_hi && (k & pmask) == prefix)
+          atomicAdd(&ms.rh[d][(k >> shift) & 127u], 1);
+      }
+      group_sync<NT, BAR>();
+      if (tid < 32) {
+        int c[4], lsum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          c[j] = ms.rh[d][127 - (tid * 4 + j)];
+          lsum += c[j];
+        }
+        int cum = warp_incl_scan(lsum) - lsum;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (cum < rem && rem <= cum + c[j]) {
+            ms.dig[d] = 127 - (tid * 4 + j);
+            ms.abv[d] = cum;
+          }
+          cum += c[j];
+        }
+      }
+      group_sync<NT, BAR>();
+      prefix |= static_cast<uint32_t>(ms.dig[d]) << shift;
+      pmask |= 127u << shift;
+      rem -= ms.abv[d];
+    }
+    T = cut_lo | (prefix & ((1u << kSelKeyShift) - 1u));
+    need_eq = rem;
+  }
+  // chosen: every sure candidate, the in-cut ones above T and the first
+  // need_eq equal to T.  One scan of (above, equal) counts packed in 16-bit
+  // halves (at most 8192 each) places them.
+  auto sure = [&](uint32_t k) { return cut ? k > cut_hi : k >= lo_key; };
+  int ca = 0, ce = 0;
+#pragma unroll 1
+  for (int q = q0; q < q1; ++q) {
+    const uint32_t k = bk[pad32(q)];
+    if (sure(k)) ++ca;
+    else if (cut && k >= in_lo && k <= cut_hi) {
+      ca += k > T;
+      ce += k == T;
+    }
+  }
+  int tot;
+  const int ex = group_excl_scan<NT, BAR>((ca << 16) | ce, tid, sm.scan, &tot);
+  int eq_seen = ex & 0xFFFF;
+  int pos = (ex >> 16) + min(need_eq, eq_seen);
+#pragma unroll 1
+  for (int q = q0; q < q1; ++q) {
+    const uint32_t k = bk[pad32(q)];
+    bool take = sure(k);
+    if (!take && cut && k >= in_lo && k <= cut_hi) {
+      if (k > T) take = true;
+      else if (k == T) take = eq_seen++ < need_eq;
+    }
+    if (take && pos < kTopK) dst[pos++] = bi[pad32(q)];
+  }
+  int n = (tot >> 16) + min(need_eq, tot & 0xFFFF);
+  if (n > kTopK) n = kTopK;  // cannot happen for consistent inputs
+  for (int j = n + tid; j < kTopK; j += NT) dst[j] = -1;
+  if (tid == 0) *cnt_out = n;
+}
+
+
+// The bin of the K-th largest key of a row from the row's complete
+// 2048-bin key histogram h (global memory), and the number of keys in higher
+// bins; *bin = -1 when the row has at most K keys.  Thread gtid of the NT
+// owns the 2048/NT bins counted down from 2047 - gtid*(2048/NT).
+template <int NT, int BAR>
+__device__ __forceinline__ void cut_bin_of(const uint32_t* h, int K, int gtid, SelectSmem& sm,
+                                           int* bin, int* above) {
+  constexpr int kPer = 2048 / NT;
+  static_assert(2048 % NT == 0, "bins per thread");
+  int hc[kPer], sum = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    hc[j] = static_cast<int>(__ldcg(h + 2047 - (gtid * kPer + j)));
+    sum += hc[j];
+  }
+  if (gtid == 0) {
+    sm.digit = -1;
+    sm.above = 0;
+  }
+  int tot;
+  int cum = group_excl_scan<NT, BAR>(sum, gtid, sm.scan, &tot);
+  if (tot > K) {
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (cum < K && K <= cum + hc[j]) {
+        sm.digit = 2047 - (gtid * kPer + j);
+        sm.above = cum;
+      }
+      cum += hc[j];
+    }
+  }
+  group_sync<NT, BAR>();
+  *bin = sm.digit;
+  *above = sm.above;
+  group_sync<NT, BAR>();
 }
 
 }  // namespace spx

@@ -35,11 +35,58 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps of recent calls.  A decode loop passes the same
+// caches and query buffers on every step, so the maps are encoded once and
+// copied afterwards.  The key is everything the encoding depends on; a map
+// is a pure function of it (the device is part of the key only because the
+// same address may name memory of another device).
+struct MapKey {
+  int dev, dtype, rank, swizzle;
+  const void* base;
+  uint64_t dims[5], strides[4];
+  uint32_t box[5];
+};
+constexpr int kMapCacheSize = 32;
+struct MapCache {
+  std::mutex mu;
+  MapKey key[kMapCacheSize];
+  CUtensorMap map[kMapCacheSize];
+  bool used[kMapCacheSize] = {};
+  int next = 0;
+};
+MapCache& map_cache() {
+  static MapCache c;
+  return c;
+}
+
 }  // namespace
 
 bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
                        const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
                        CUtensorMapSwizzle swizzle) {
+  if (rank < 1 || rank > 5) return false;
+  MapKey k;
+  std::memset(&k, 0, sizeof(k));
+  if (cudaGetDevice(&k.dev) != cudaSuccess) return false;
+  k.dtype = static_cast<int>(dtype);
+  k.rank = rank;
+  k.swizzle = static_cast<int>(swizzle);
+  k.base = base;
+  for (int i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides_bytes[i];
+  MapCache& c = map_cache();
+  {
+    std::lock_guard<std::mutex> g(c.mu);
+    for (int i = 0; i < kMapCacheSize; ++i) {
+      if (c.used[i] && std::memcmp(&c.key[i], &k, sizeof(k)) == 0) {
+        *map = c.map[i];
+        return true;
+      }
+    }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -50,9 +97,19 @@ bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, co
     es[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
-  return fn(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gd, gs, bx, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const bool ok = fn(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gd, gs,
+                     bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (ok) {
+    std::lock_guard<std::mutex> g(c.mu);
+    const int i = c.next;
+    c.next = (c.next + 1) % kMapCacheSize;
+    c.key[i] = k;
+    c.map[i] = *map;
+    c.used[i] = true;
+  }
+  return ok;
 }
 
 namespace {
@@ -60,6 +117,17 @@ std::atomic<uint64_t> g_launches{0};
 }
 
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+spx_status check_dims(const spx_dims* d) {
+  if (!d) return SPX_ERR_INVALID_ARG;
+  if (d->idx_heads != kIdxHeads || d->idx_dim != kIdxDim || d->pool != kPool ||
+      d->topk_blocks != kTopK || d->latent != kLatent)
+    return SPX_ERR_UNSUPPORTED;
+  if (d->heads < kHeadGroup || d->heads > kMaxHeads || d->heads % kHeadGroup != 0)
+    return SPX_ERR_UNSUPPORTED;
+  if (!std::isfinite(d->sm_scale) || !(d->sm_scale > 0.f)) return SPX_ERR_INVALID_ARG;
+  return SPX_OK;
+}
 
 int device_sm_count() {
   static std::atomic<int> cache[64];  // zero-initialised: not queried yet
@@ -83,17 +151,6 @@ constexpr size_t kAlign = 256;
 inline size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool al4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
-
-spx_status check_dims(const spx_dims* d) {
-  if (!d) return SPX_ERR_INVALID_ARG;
-  if (d->idx_heads != kIdxHeads || d->idx_dim != kIdxDim || d->pool != kPool ||
-      d->topk_blocks != kTopK || d->latent != kLatent)
-    return SPX_ERR_UNSUPPORTED;
-  if (d->heads < kHeadGroup || d->heads > kMaxHeads || d->heads % kHeadGroup != 0)
-    return SPX_ERR_UNSUPPORTED;
-  if (!std::isfinite(d->sm_scale) || !(d->sm_scale > 0.f)) return SPX_ERR_INVALID_ARG;
-  return SPX_OK;
-}
 
 spx_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SPX_OK : SPX_ERR_CUDA; }
 
@@ -265,6 +322,13 @@ spx_status spx_device_error(int32_t* code, spx_stream stream) {
   }
   *code = v;
   return SPX_OK;
+}
+
+spx_status spx_selftest_wait_timeout(int64_t limit_ns, int64_t* result, spx_stream stream) {
+  if (!result || !al4(result)) return SPX_ERR_INVALID_ARG;
+  if (limit_ns < 1000 || limit_ns > 1000000000) return SPX_ERR_INVALID_ARG;
+  return cuda_status(launch_wait_selftest(static_cast<uint64_t>(limit_ns), result,
+                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
 // ---------------------------------------------------------------------------
@@ -541,6 +605,7 @@ spx_status decode_impl(const spx_dims* d, int32_t B, const void* raw_k, const fl
   pa.nvis_out = n_vis;
   pa.init_hist = hist;
   pa.init_done = done;
+  pa.pdl = true;
   int8_t* q8 = reinterpret_cast<int8_t*>(base + L.q8);
   float* wq = reinterpret_cast<float*>(base + L.wq);
   if (i8) {
@@ -583,26 +648,12 @@ spx_status decode_impl(const spx_dims* d, int32_t B, const void* raw_k, const fl
   if (timing && timing->score_end &&
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
     return SPX_ERR_CUDA;
-  // 3. top-512 blocks per row
-  SelectBlocksArgs ma{};
-  ma.rows = B;
-  ma.scores = scores;
-  ma.score_stride = L.stride;
-  ma.n_vis = n_vis;
-  ma.max_len = max_len;
-  ma.ghist = hist;
-  ma.nchunk = L.nchunk;
-  ma.list_key = reinterpret_cast<uint32_t*>(base + L.lkey);
-  ma.list_idx = reinterpret_cast<int32_t*>(base + L.lidx);
-  ma.list_cnt = reinterpret_cast<int32_t*>(base + L.lcnt);
-  ma.done = done;
-  ma.out_idx = idx;
-  ma.out_cnt = count;
-  ma.pdl = !(timing && timing->score_end);
-  if ((e = launch_select_blocks(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
-
-  // 4. attention
+  // 3 + 4. top-512 blocks per row (chosen by the attention clusters from the
+  // scores and their key histograms) and attention
   AttnArgs aa{};
+  aa.sel_scores = scores;
+  aa.sel_stride = L.stride;
+  aa.sel_hist = hist;
   aa.q = q;
   aa.latent = latent;
   aa.seq_stride = cap_tok * kLatent;
@@ -615,7 +666,7 @@ spx_status decode_impl(const spx_dims* d, int32_t B, const void* raw_k, const fl
   aa.out = out;
   aa.lse = lse;
   aa.ws = base + L.attn;
-  aa.pdl = true;
+  aa.pdl = !(timing && timing->score_end);
   return cuda_status(launch_attn(L.ap, aa, s));
 }
 

@@ -7,7 +7,14 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "spx.h"
+
 namespace spx {
+
+// Host check of the layer dimensions shared by every entry point:
+// SPX_ERR_INVALID_ARG for a null pointer or a non-finite / non-positive
+// softmax scale, SPX_ERR_UNSUPPORTED for dimensions v1 does not implement.
+spx_status check_dims(const spx_dims* d);
 
 // Dimensions v1 implements (the layer the pages describe).
 constexpr int kIdxHeads = 32;
@@ -44,6 +51,7 @@ struct PoolAppendArgs {
   const float* w_head;
   int8_t* q8;
   float* wq;
+  bool pdl;  // may start while the previous kernel of the stream finishes
 };
 cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream);
 // Query quantisation alone (one CTA per row), as in launch_pool_append.
@@ -140,8 +148,13 @@ struct AttnArgs {
   const void* latent;
   int64_t seq_stride;
   int64_t cap_tok;
+  // the selected blocks; with sel_scores set they are chosen by the kernel
+  // itself (decode: from the scores and their key histograms) and written here
   const int32_t* idx;
   const int32_t* count;
+  const float* sel_scores;  // [rows, sel_stride] (stride a multiple of 4) or NULL
+  int64_t sel_stride;
+  const uint32_t* sel_hist;  // [rows, kSelHistBins], complete
   const int64_t* n_vis;
   int64_t max_len;
   float sm_scale;
@@ -151,6 +164,10 @@ struct AttnArgs {
   bool pdl;
 };
 cudaError_t launch_attn(const AttnPlan& p, const AttnArgs& a, cudaStream_t stream);
+
+// Self-test of the bounded waits (one CTA; see selftest.cu).  res: device
+// int64 [6].
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int64_t* res, cudaStream_t stream);
 
 // Tensor-map encoding through the driver entry point (no libcuda link).
 bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank,

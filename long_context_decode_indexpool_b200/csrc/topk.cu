@@ -141,135 +141,6 @@ constexpr int kSelShift = 32 - 11;
 constexpr int kMergeCap = kThreads * 16;  // candidates held at once (16 per thread)
 constexpr int kMergePer = 4;              // list entries per thread per round (long rows)
 
-// Shared state of the final choice.
-struct MergeSmem {
-  int rh[3][128];  // radix histograms of the three 7-bit digits below the cut bin
-  int dig[3], abv[3];
-  uint32_t kmin, kmax;
-};
-
-// The row's result from the n buffered (key, block) pairs, in block order;
-// entries below lo_key are not candidates.  Every candidate above the cut
-// bin is selected; the (K - above) best of the cut bin (ties: lower block)
-// complete the set.  Writes the ascending block ids, -1 padded, and the
-// count.  This code runs once per row: its loops stay rolled, so that it is
-// short (instruction fetch, not arithmetic, bounds a one-pass kernel).
-__device__ __noinline__ void merge_final(const uint32_t* bk, const int32_t* bi, int n_in,
-                                         uint32_t lo_key, int cut_bin, int above, SelectSmem& sm,
-                                         MergeSmem& ms, int32_t* dst, int32_t* cnt_out) {
-  const int tid = threadIdx.x;
-  const int per = (n_in + kThreads - 1) / kThreads;
-  const int q0 = min(tid * per, n_in), q1 = min(q0 + per, n_in);
-  const bool cut = cut_bin >= 0;  // uniform
-  const uint32_t cut_lo = cut ? static_cast<uint32_t>(cut_bin) << kSelShift : 0u;
-  const uint32_t cut_hi = cut ? cut_lo | ((1u << kSelShift) - 1u) : 0xFFFFFFFFu;
-  const uint32_t in_lo = lo_key > cut_lo ? lo_key : cut_lo;
-  // candidate classes: sure (above the cut bin, or every candidate when no
-  // cut is needed) and in-cut
-  uint32_t T = 0xFFFFFFFFu;
-  int need_eq = 0;
-  if (cut) {
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0;
-#pragma unroll 1
-    for (int q = q0; q < q1; ++q) {
-      const uint32_t k = bk[pad32(q)];
-      if (k >= in_lo && k <= cut_hi) {
-        kmin = k < kmin ? k : kmin;
-        kmax = k > kmax ? k : kmax;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const uint32_t x = __shfl_xor_sync(0xffffffffu, kmin, o);
-      const uint32_t y = __shfl_xor_sync(0xffffffffu, kmax, o);
-      kmin = x < kmin ? x : kmin;
-      kmax = y > kmax ? y : kmax;
-    }
-    if ((tid & 31) == 0 && kmin <= kmax) {
-      atomicMin(&ms.kmin, kmin);
-      atomicMax(&ms.kmax, kmax);
-    }
-    __syncthreads();
-    // the candidates of the cut bin share every bit above the highest one
-    // where their min and max differ; the rest comes from radix passes
-    kmin = ms.kmin;
-    const uint32_t diff = kmin ^ ms.kmax;
-    uint32_t prefix = 0, pmask = 0;
-    int rem = kTopK - above;
-#pragma unroll 1
-    for (int d = 0; d < 3; ++d) {
-      const int shift = 14 - 7 * d;
-      if ((diff >> shift) == 0) {  // uniform
-        prefix |= kmin & (127u << shift);
-        pmask |= 127u << shift;
-        continue;
-      }
-#pragma unroll 1
-      for (int q = q0; q < q1; ++q) {
-        const uint32_t k = bk[pad32(q)];
-        if (k >= in_lo && k <= cut_hi && (k & pmask) == prefix)
-          atomicAdd(&ms.rh[d][(k >> shift) & 127u], 1);
-      }
-      __syncthreads();
-      if (tid < 32) {
-        int c[4], lsum = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          c[j] = ms.rh[d][127 - (tid * 4 + j)];
-          lsum += c[j];
-        }
-        int cum = warp_incl_scan(lsum) - lsum;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (cum < rem && rem <= cum + c[j]) {
-            ms.dig[d] = 127 - (tid * 4 + j);
-            ms.abv[d] = cum;
-          }
-          cum += c[j];
-        }
-      }
-      __syncthreads();
-      prefix |= static_cast<uint32_t>(ms.dig[d]) << shift;
-      pmask |= 127u << shift;
-      rem -= ms.abv[d];
-    }
-    T = cut_lo | (prefix & ((1u << kSelShift) - 1u));
-    need_eq = rem;
-  }
-  // chosen: every sure candidate, the in-cut ones above T and the first
-  // need_eq equal to T.  One scan of (above, equal) counts packed in 16-bit
-  // halves (at most 8192 each) places them.
-  auto sure = [&](uint32_t k) { return cut ? k > cut_hi : k >= lo_key; };
-  int ca = 0, ce = 0;
-#pragma unroll 1
-  for (int q = q0; q < q1; ++q) {
-    const uint32_t k = bk[pad32(q)];
-    if (sure(k)) ++ca;
-    else if (cut && k >= in_lo && k <= cut_hi) {
-      ca += k > T;
-      ce += k == T;
-    }
-  }
-  int tot;
-  const int ex = group_excl_scan<kThreads, 0>((ca << 16) | ce, tid, sm.scan, &tot);
-  int eq_seen = ex & 0xFFFF;
-  int pos = (ex >> 16) + min(need_eq, eq_seen);
-#pragma unroll 1
-  for (int q = q0; q < q1; ++q) {
-    const uint32_t k = bk[pad32(q)];
-    bool take = sure(k);
-    if (!take && cut && k >= in_lo && k <= cut_hi) {
-      if (k > T) take = true;
-      else if (k == T) take = eq_seen++ < need_eq;
-    }
-    if (take && pos < kTopK) dst[pos++] = bi[pad32(q)];
-  }
-  int n = (tot >> 16) + min(need_eq, tot & 0xFFFF);
-  if (n > kTopK) n = kTopK;  // cannot happen for consistent inputs
-  for (int j = n + tid; j < kTopK; j += kThreads) dst[j] = -1;
-  if (tid == 0) *cnt_out = n;
-}
-
 // Key histogram of scores written by another kernel (prefill): grid
 // (chunks of kSelChunk, rows); each CTA counts its chunk's keys in shared
 // memory and adds the non-zero bins into the row's histogram (zero on entry).
@@ -429,7 +300,8 @@ __global__ void __launch_bounds__(kThreads)
       buf_idx[pad32(f)] = __ldcg(list_idx + e);
     }
     __syncthreads();
-    merge_final(buf_key, buf_idx, mtot, theta, cut_bin, above, sm, ms, dst, out_cnt + r);
+    merge_final<kThreads, 0>(buf_key, buf_idx, mtot, theta, cut_bin, above, sm, ms, dst,
+                             out_cnt + r, tid);
     return;
   }
 
@@ -504,7 +376,8 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
   }
-  merge_final(buf_key, buf_idx, nbuf, thr_keep, cut_bin, above, sm, ms, dst, out_cnt + r);
+  merge_final<kThreads, 0>(buf_key, buf_idx, nbuf, thr_keep, cut_bin, above, sm, ms, dst,
+                           out_cnt + r, tid);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }

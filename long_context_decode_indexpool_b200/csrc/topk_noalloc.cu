@@ -12,9 +12,11 @@
 //
 // The array's name seen from host code is only a host-side handle, not a
 // device address: the device address is looked up once per device with
-// cudaGetSymbolAddress (with that device current) and cached.  That lookup
-// happens inside the first call on each device, so the first call on a device
-// should be made before any stream capture begins.
+// cudaGetSymbolAddress (with that device current) and cached for the life of
+// the process, which assumes the device is not reset (cudaDeviceReset) in
+// between.  That lookup happens inside the first call on each device, so the
+// first call on a device should be made before any stream capture begins.
+// Devices with an index beyond the cache look the address up on every call.
 //
 // Every call shares the one array and leaves its contents behind; nothing in
 // it has to start at zero (each list count is written before it is read).
@@ -38,7 +40,11 @@ void* g_scratch_addr[kMaxDevices] = {};
 // Device address of g_topk_scratch on the current device, or nullptr.
 void* scratch_address() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+  if (dev >= kMaxDevices) {  // not cached
+    void* p = nullptr;
+    return cudaGetSymbolAddress(&p, g_topk_scratch) == cudaSuccess ? p : nullptr;
+  }
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
@@ -54,12 +60,8 @@ extern "C" spx_status spx_topk_blocks_noalloc(const spx_dims* d, int32_t rows, c
                                               int64_t score_stride, const int64_t* n_vis,
                                               int64_t max_len, int32_t* idx, int32_t* count,
                                               spx_stream stream) {
-  if (!d) return SPX_ERR_INVALID_ARG;
-  if (d->idx_heads != spx::kIdxHeads || d->idx_dim != spx::kIdxDim || d->pool != spx::kPool ||
-      d->topk_blocks != spx::kTopK || d->latent != spx::kLatent || d->heads < spx::kHeadGroup ||
-      d->heads > spx::kMaxHeads || d->heads % spx::kHeadGroup != 0)
-    return SPX_ERR_UNSUPPORTED;
-  if (!std::isfinite(d->sm_scale) || !(d->sm_scale > 0.f)) return SPX_ERR_INVALID_ARG;
+  const spx_status st = spx::check_dims(d);
+  if (st != SPX_OK) return st;
   if (rows < 1 || rows > 65535 || max_len < 0) return SPX_ERR_SHAPE;
   if (max_len / spx::kPool > (int64_t(1) << 31) - 1) return SPX_ERR_SHAPE;
   if (score_stride < max_len / spx::kPool) return SPX_ERR_SHAPE;

@@ -180,3 +180,17 @@ def test_int8_cache_host_validation(spx):
                                 FAKE, FAKE, 8192, 8192, FAKE, ws=FAKE, ws_bytes=need - 256,
                                 stream=s)
     assert e.value.status == 4
+
+
+def test_selftest_host_validation(spx):
+    s = 0
+    for bad in (0, 999, 1_000_000_001):  # limit outside 1 us .. 1 s
+        with pytest.raises(spx.SpxError) as e:
+            spx.spx_selftest_wait_timeout(bad, FAKE, stream=s)
+        assert e.value.status == 1
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_selftest_wait_timeout(1_000_000, None, stream=s)
+    assert e.value.status == 1
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_selftest_wait_timeout(1_000_000, FAKE + 2, stream=s)
+    assert e.value.status == 1

@@ -51,6 +51,106 @@ def test_pool_append_ragged(lens, n_new):
             assert np.array_equal(got_tail[b, p % 4], raw[b][p])
 
 
+def _learned_pool_case(seed):
+    """Pool weights as a learned layer would hold them: the softmax of N(0,1)
+    logits in fp32 (not dyadic), and bf16 keys over a wide range of
+    magnitudes with exact zeros and -0 mixed in."""
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal(4).astype(np.float32)
+    pw = np.exp(z - z.max()).astype(np.float32)
+    pw = (pw / pw.sum()).astype(np.float32)
+    assert abs(float(pw.astype(np.float64).sum()) - 1.0) <= 1e-6
+    assert any(float(x) * 64 != int(float(x) * 64) for x in pw)  # not 1/64-dyadic
+    return rng, pw
+
+
+def _fp32_route_bits(raw_bits, pw):
+    """bf16 bits of the pooled key summed in fp32 (one rounding per step)
+    and then rounded to bf16: the double rounding the single-rounding
+    reading avoids.  Used only to show that the test data tells the two
+    apart."""
+    k = synth.bf16_bits_to_f64_np(raw_bits).astype(np.float32).reshape(-1, 4, raw_bits.shape[-1])
+    acc = np.zeros(k[:, 0].shape, np.float32)
+    for i in range(4):
+        acc = (acc + (k[:, i] * np.float32(pw[i])).astype(np.float32)).astype(np.float32)
+    return synth.f32_to_bf16_bits_np(acc)
+
+
+@pytest.mark.parametrize("lens,n_new", [([0, 6, 13], 4001), ([1, 2, 3], 2)])
+def test_pool_append_learned_weights_single_rounding(lens, n_new):
+    """[W1] "IndexPool": the pooling weights are learned.  With fp32 weights
+    that are not dyadic, the pooled key must still be the single
+    round-to-nearest-even of the exact weighted sum (the oracle's reading),
+    bit for bit; the data are chosen so that an fp32 sum would differ."""
+    spx = need_gpu()
+    rng, pw = _learned_pool_case(17 + n_new)
+    B = len(lens)
+    total = max(lens) + n_new
+    cap_blk = (total + 3) // 4 + 1
+    raws = []
+    for b in range(B):
+        v = rng.standard_normal((total, 128)) * np.exp2(rng.integers(-30, 30, (total, 1)))
+        v[rng.random((total, 128)) < 0.02] = 0.0
+        v[rng.random((total, 128)) < 0.01] = -0.0
+        raws.append(synth.f32_to_bf16_bits_np(v.astype(np.float32)))
+    tail0 = np.zeros((B, 3, 128), np.uint16)
+    for b, L0 in enumerate(lens):
+        for p in range((L0 // 4) * 4, L0):
+            tail0[b, p % 4] = raws[b][p]
+    new = np.stack([raws[b][lens[b]:lens[b] + n_new] for b in range(B)])
+    pooled = torch.zeros(B, cap_blk, 128, dtype=torch.bfloat16, device="cuda")
+    tail = to_dev_bf16(tail0)
+    len_dev = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    d = spx.dims(64)
+    spx.spx_pool_append(d, B, to_dev_bf16(new), n_new, pw, tail, pooled, cap_blk, len_dev, total)
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    got = bits_of(pooled)
+    differs = 0
+    for b, L0 in enumerate(lens):
+        end = L0 + n_new
+        ref = oracle.pool(raws[b][:end], pw.astype(np.float64))
+        lo, hi = L0 // 4, end // 4
+        assert np.array_equal(got[b, lo:hi], ref[lo:hi]), f"seq {b}"
+        differs += int((_fp32_route_bits(raws[b][4 * lo:4 * hi], pw) != ref[lo:hi]).sum())
+    if n_new > 100:
+        assert differs > 0, "the data do not separate single from double rounding"
+
+
+@pytest.mark.parametrize("lens,n_new", [([0, 6, 13], 4001)])
+def test_pool_append_i8_learned_weights(lens, n_new):
+    """The INT8 cache under learned fp32 weights: codes and block scales of
+    the exact weighted sum (one round-half-even after an exact power-of-two
+    scaling), bit for bit as in the oracle."""
+    spx = need_gpu()
+    rng, pw = _learned_pool_case(5)
+    B = len(lens)
+    total = max(lens) + n_new
+    cap_blk = (total + 3) // 4 + 1
+    raws = [synth.f32_to_bf16_bits_np((rng.standard_normal((total, 128)) *
+                                       np.exp2(rng.integers(-40, 24, (total, 1)))).astype(np.float32))
+            for _ in range(B)]
+    tail0 = np.zeros((B, 3, 128), np.uint16)
+    for b, L0 in enumerate(lens):
+        for p in range((L0 // 4) * 4, L0):
+            tail0[b, p % 4] = raws[b][p]
+    new = np.stack([raws[b][lens[b]:lens[b] + n_new] for b in range(B)])
+    codes = torch.zeros(B, cap_blk, 128, dtype=torch.int8, device="cuda")
+    scale = torch.zeros(B, cap_blk, dtype=torch.float32, device="cuda")
+    len_dev = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    spx.spx_pool_append_i8(spx.dims(64), B, to_dev_bf16(new), n_new, pw, to_dev_bf16(tail0),
+                           codes, scale, cap_blk, len_dev, total)
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    got, gscale = codes.cpu().numpy(), scale.cpu().numpy().astype(np.float64)
+    for b, L0 in enumerate(lens):
+        end = L0 + n_new
+        ref, rscale = oracle.pool_i8(raws[b][:end], pw.astype(np.float64))
+        lo, hi = L0 // 4, end // 4
+        assert np.array_equal(got[b, lo:hi], ref[lo:hi]), f"seq {b}"
+        assert np.array_equal(gscale[b, lo:hi], rscale[lo:hi]), f"seq {b}"
+
+
 # ----------------------------------------------------------------------------
 # Indexer scoring (tcgen05)
 # ----------------------------------------------------------------------------
