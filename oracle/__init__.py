@@ -51,6 +51,8 @@ def _load():
             lib.orc_bf16_rne.restype = ctypes.c_uint16
             lib.orc_pool.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P, P]
             lib.orc_pool.restype = None
+            lib.orc_pool_tok.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P, P]
+            lib.orc_pool_tok.restype = None
             lib.orc_score.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P, i64, P, ctypes.c_int]
             lib.orc_score.restype = None
             lib.orc_quant_i8.argtypes = [P, ctypes.c_int, P]
@@ -101,6 +103,19 @@ def pool(raw_bits: np.ndarray, w, pool_size: int = POOL) -> np.ndarray:
     assert w.shape == (pool_size,)
     out = np.zeros((n_tok // pool_size, dim), dtype=np.uint16)
     _load().orc_pool(_p(raw), n_tok, dim, pool_size, _p(w), _p(out))
+    return out
+
+
+def pool_tok(raw_bits: np.ndarray, wt, pool_size: int = POOL) -> np.ndarray:
+    """IndexPool with a weight per token: [n_tok, dim] raw bf16 keys and
+    [n_tok] weights (each block's four summing to 1) -> [n_tok // pool, dim]
+    bf16 bits."""
+    raw = np.ascontiguousarray(raw_bits, dtype=np.uint16)
+    n_tok, dim = raw.shape
+    wt = np.ascontiguousarray(wt, dtype=np.float64)
+    assert wt.shape == (n_tok,)
+    out = np.zeros((n_tok // pool_size, dim), dtype=np.uint16)
+    _load().orc_pool_tok(_p(raw), n_tok, dim, pool_size, _p(wt), _p(out))
     return out
 
 

@@ -97,6 +97,24 @@ void orc_pool(const uint16_t* raw, int64_t n_tok, int dim, int pool,
   }
 }
 
+// IndexPool with data-dependent weights (the per-token reading of [W1
+// "IndexPool"]: the learned weights come with the tokens): token p carries
+// its own pooling weight wt[p], the four weights of a block sum to 1, and
+// k_pool[b] = sum_{i=0..3} wt[4b+i] k[4b+i].  One fp64 sum in time order,
+// one rounding to bf16, as orc_pool.
+void orc_pool_tok(const uint16_t* raw, int64_t n_tok, int dim, int pool,
+                  const double* wt, uint16_t* pooled) {
+  const int64_t nblk = n_tok / pool;
+  for (int64_t b = 0; b < nblk; ++b) {
+    for (int d = 0; d < dim; ++d) {
+      double acc = 0.0;
+      for (int i = 0; i < pool; ++i)
+        acc += wt[b * pool + i] * bf16_to_f64(raw[(b * pool + i) * dim + d]);
+      pooled[b * dim + d] = f64_to_bf16_rne(acc);
+    }
+  }
+}
+
 // Lightning-indexer score of every pooled block against one query
 // [W3 "실제로 바꾸는 것"; formula as fixed by the workload specification]:
 //   s[b] = sum_h w_h * max(0, sum_d q[h][d] * k_pool[b][d]).

@@ -28,6 +28,15 @@ MUTANTS = {
     "bf16 truncation instead of nearest-even": (
         "double r = std::nearbyint(std::ldexp(std::fabs(v), -qe));",
         "double r = std::trunc(std::ldexp(std::fabs(v), -qe));"),
+    "per-token weight of the next token": (
+        "acc += wt[b * pool + i] * bf16_to_f64(raw[(b * pool + i) * dim + d]);",
+        "acc += wt[b * pool + (i + 1) % pool] * bf16_to_f64(raw[(b * pool + i) * dim + d]);"),
+    "per-token weights of the block's first token only": (
+        "acc += wt[b * pool + i] * bf16_to_f64(raw[(b * pool + i) * dim + d]);",
+        "acc += wt[b * pool] * bf16_to_f64(raw[(b * pool + i) * dim + d]);"),
+    "per-token sum in fp32": (
+        "      pooled[b * dim + d] = f64_to_bf16_rne(acc);\n    }\n  }\n}\n\n// Lightning",
+        "      pooled[b * dim + d] = f64_to_bf16_rne(static_cast<float>(acc));\n    }\n  }\n}\n\n// Lightning"),
     # indexer score
     "score without ReLU": (
         "s += w_head[h] * (dot > 0.0 ? dot : 0.0);", "s += w_head[h] * dot;"),

@@ -6,6 +6,7 @@ invariant, a library routine (torch's fp32->bf16 rounding, numpy matmul,
 scipy softmax) or brute force on tiny inputs.  CPU only.
 """
 import itertools
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -119,6 +120,86 @@ def test_pool_is_weighted_mean_bound():
     exact = np.einsum("i,bid->bd", w, blocks)
     # one bf16 rounding: relative error <= 2^-8 (unit roundoff of 8 significant bits)
     assert (np.abs(p - exact) <= np.abs(exact) * 2.0 ** -8).all()
+
+
+# ----------------------------------------------------------------------------
+# IndexPool with a weight per token
+# ----------------------------------------------------------------------------
+def _bf16_rne_exact(x: Fraction) -> float:
+    """Nearest-even bf16 value of an exact rational (8 significant bits, no
+    double rounding): an independent rounding for the brute-force pins."""
+    if x == 0:
+        return 0.0
+    sign = -1.0 if x < 0 else 1.0
+    a = abs(x)
+    e = 0
+    while a >= 2:
+        a /= 2
+        e += 1
+    while a < 1:
+        a *= 2
+        e -= 1
+    # a in [1, 2): keep 7 fraction bits
+    scaled = a * 128
+    lo = scaled.numerator // scaled.denominator
+    rem = scaled - lo
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2 == 1):
+        lo += 1
+    return sign * float(Fraction(lo, 128) * Fraction(2) ** e)
+
+
+def test_pool_tok_exact_rational_brute_force():
+    """Each pooled value equals the exact rational weighted sum of the bf16
+    keys with the fp32 per-token weights, rounded once to bf16."""
+    rng = np.random.default_rng(41)
+    n_tok, dim = 4 * 25 + 2, 6
+    vals = (rng.standard_normal((n_tok, dim)) * np.exp2(rng.integers(-12, 12, (n_tok, 1))))
+    raw = synth.f32_to_bf16_bits_np(vals.astype(np.float32))  # nearest bf16 values
+    g = rng.standard_normal(n_tok)
+    wt = np.empty(n_tok, np.float32)
+    for b in range(n_tok // 4):
+        e = np.exp(g[4 * b:4 * b + 4])
+        wt[4 * b:4 * b + 4] = e / e.sum()
+    wt[4 * 25:] = 0.5  # trailing tokens: no block
+    got = oracle.bf16_to_f64(oracle.pool_tok(raw, wt.astype(np.float64)))
+    kf = oracle.bf16_to_f64(raw)
+    assert got.shape == (25, dim)
+    for b in range(25):
+        for d in range(dim):
+            exact = sum(Fraction(float(wt[4 * b + i])) * Fraction(float(kf[4 * b + i, d]))
+                        for i in range(4))
+            assert got[b, d] == _bf16_rne_exact(exact), (b, d)
+    # a block whose sum, 1 + 2^-8 + 2^-30, sits just above a bf16 tie by less
+    # than an fp32 step: one rounding gives 1 + 2^-7, a sum rounded to fp32
+    # first would land on the tie and give 1.0
+    keys = bits_of(np.array([[4.0], [2.0 ** -6], [2.0 ** -28], [0.0]], np.float32))
+    got = oracle.bf16_to_f64(oracle.pool_tok(keys, np.full(4, 0.25)))
+    assert got[0, 0] == 1.0 + 2.0 ** -7
+
+
+def test_pool_tok_per_block_one_hot_picks_one_token():
+    rng = np.random.default_rng(42)
+    n_blk = 40
+    raw = synth.f32_to_bf16_bits_np(rng.standard_normal((4 * n_blk, 128)).astype(np.float32))
+    pick = rng.integers(0, 4, n_blk)
+    wt = np.zeros(4 * n_blk)
+    wt[4 * np.arange(n_blk) + pick] = 1.0
+    got = oracle.pool_tok(raw, wt)
+    assert np.array_equal(got, raw[4 * np.arange(n_blk) + pick])
+
+
+def test_pool_tok_identical_keys_and_static_weights():
+    rng = np.random.default_rng(43)
+    key = rng.integers(-8, 9, 128).astype(np.float32)
+    # identical keys in a block, dyadic weights summing to exactly 1 per block
+    wt = np.tile([0.5, 0.25, 0.125, 0.125], 3)
+    wt[4:8] = [1 / 64, 3 / 64, 12 / 64, 48 / 64]
+    got = oracle.pool_tok(bits_of(np.tile(key, (12, 1))), wt)
+    assert all(np.array_equal(oracle.bf16_to_f64(got[b]), key.astype(np.float64)) for b in range(3))
+    # the same weights on every block give the static-weight pooling
+    vals = rng.integers(-8, 9, (4 * 30, 128)).astype(np.float32)
+    w = synth.workload("mid").pool_weights()
+    assert np.array_equal(oracle.pool_tok(bits_of(vals), np.tile(w, 30)), oracle.pool(bits_of(vals), w))
 
 
 # ----------------------------------------------------------------------------
