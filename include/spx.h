@@ -171,6 +171,28 @@ SPX_API spx_status spx_pool_append(const spx_dims* d, int32_t B, const void* raw
                            spx_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * spx_pool_append_tok -- step 1 with a weight per token.  [W1] "IndexPool"
+ * says the pooling weights are learned; this is the data-dependent reading of
+ * that sentence: token p arrives with its own weight (for example a learned
+ * gate's output normalised over its block), and the pooled key of block blk is
+ *     pooled_k[b][blk][d] = bf16_rne( sum_{i=0..3} wt(4 blk + i) * key(4 blk + i)[d] )
+ * formed in fp64 and rounded once, as in spx_pool_append.  The four weights
+ * of a block are expected to sum to 1; they live on the device, so the call
+ * does not check that.  Weights of the still-incomplete block wait in tail_w
+ * beside the keys in tail.
+ *
+ *   raw_w     DEVICE float [B, n_new]    weights of the appended tokens
+ *   tail_w    DEVICE float [B, pool-1]   weights of the tail tokens (in/out)
+ * Other arguments, limits and errors as for spx_pool_append; compose with
+ * spx_decode_fused (raw_k = NULL) or the separate calls for the other steps.
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_pool_append_tok(const spx_dims* d, int32_t B, const void* raw_k,
+                                       const float* raw_w, int32_t n_new, void* tail,
+                                       float* tail_w, void* pooled_k, int64_t cap_blk,
+                                       const int64_t* len_dev, int64_t max_len,
+                                       spx_stream stream);
+
+/* ---------------------------------------------------------------------------
  * Step 2 -- lightning-indexer scores of every complete block (decode: one
  * query per sequence).  [W4] "수렴점 2" (32-head lightning indexer);
  * formula as fixed by the workload specification:

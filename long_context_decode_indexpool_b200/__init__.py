@@ -66,6 +66,7 @@ _SIGS = {
     "spx_device_error": ([ctypes.POINTER(_I32), _P], ctypes.c_int),
     "spx_selftest_wait_timeout": ([_I64, _P, _P], ctypes.c_int),
     "spx_pool_append": ([_DIMS, _I32, _P, _I32, _P, _P, _P, _I64, _P, _I64, _P], ctypes.c_int),
+    "spx_pool_append_tok": ([_DIMS, _I32, _P, _P, _I32, _P, _P, _P, _I64, _P, _I64, _P], ctypes.c_int),
     "spx_index_score": ([_DIMS, _I32, _P, _P, _P, _I64, _P, _I64, _P, _I64, _P], ctypes.c_int),
     "spx_topk_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_topk_blocks": ([_DIMS, _I32, _P, _I64, _P, _I64, _P, _P, _P, _SZ, _P], ctypes.c_int),
@@ -188,6 +189,13 @@ def spx_pool_append(d, B, raw_k, n_new, pool_w, tail, pooled_k, cap_blk, len_dev
     _check(_lib.spx_pool_append(ctypes.byref(d), B, _ptr(raw_k), n_new, _host_f32(pool_w),
                                 _ptr(tail), _ptr(pooled_k), cap_blk, _ptr(len_dev), max_len,
                                 _stream(stream)), "spx_pool_append")
+
+
+def spx_pool_append_tok(d, B, raw_k, raw_w, n_new, tail, tail_w, pooled_k, cap_blk, len_dev,
+                        max_len, stream=None):
+    _check(_lib.spx_pool_append_tok(ctypes.byref(d), B, _ptr(raw_k), _ptr(raw_w), n_new, _ptr(tail),
+                                    _ptr(tail_w), _ptr(pooled_k), cap_blk, _ptr(len_dev), max_len,
+                                    _stream(stream)), "spx_pool_append_tok")
 
 
 def spx_index_score(d, B, q_idx, w_head, pooled_k, cap_blk, n_vis, max_len, scores, score_stride,

@@ -18,8 +18,8 @@
 // sum over heads is a per-thread loop in the epilogue: no cross-thread
 // reduction at all.
 //
-// Roles (192 threads, one CTA per SM, persistent over a contiguous range of
-// (query group, key tile) work items):
+// Roles (192 threads, or 320 for eight queries per group; one CTA per SM,
+// persistent over a contiguous range of (query group, key tile) work items):
 //   warp 0      TMA producer: key tiles into a kStages ring (two 16 KiB
 //               boxes of 64 dims, 128-byte swizzle), query groups into
 //               kQSlots slots.
@@ -29,6 +29,10 @@
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator row, ReLU, weighted
 //               head sum in fp32, length mask; then either a store of the
 //               fp32 scores (and, with SELECT, a histogram of their keys).
+//               With eight queries per group (256 accumulator columns a
+//               tile) warps 2-9: the two warps of a TMEM lane quarter take
+//               four queries each and load their columns two 32-column
+//               blocks per wait, so the epilogue keeps up with the MMAs.
 //
 // SELECT (decode): besides the scores, the epilogue counts the row's keys
 // (scores mapped to order-preserving 32-bit keys) in a 2048-bin shared-memory
@@ -62,8 +66,6 @@ namespace {
 
 constexpr int kTileM = 128;
 constexpr int kHalfBytes = kTileM * 64 * 2;  // 128 rows x 128 bytes: one TMA box
-constexpr int kThreads = 192;
-constexpr int kEpi = 128;                    // epilogue threads
 constexpr int kHistBins = 2048;              // top 11 key bits
 constexpr int kHistShift = 21;
 // Decode work split: each CTA first takes an equal static range of 7/8 of the
@@ -79,6 +81,10 @@ template <int NQ, bool SELECT, bool I8>
 struct Cfg {
   static_assert(!I8 || NQ == 1, "the INT8 cache is scored one query per group");
   static constexpr int kN = 32 * NQ;
+  static constexpr int kEpiWarps = NQ == 8 ? 8 : 4;
+  static constexpr int kEpi = 32 * kEpiWarps;        // epilogue threads
+  static constexpr int kThreads = 64 + kEpi;
+  static constexpr int kQPerWarp = NQ * 4 / kEpiWarps;  // queries of one epilogue thread
   static constexpr int kTileBytes = I8 ? kHalfBytes : 2 * kHalfBytes;  // 128 keys
   static constexpr int kStages = I8 ? 10 : (NQ == 1 ? 6 : 4);
   static constexpr int kQSlots = NQ == 1 ? 2 : 1;
@@ -239,15 +245,16 @@ struct WorkSrc {
   }
 };
 
-__device__ __forceinline__ void epi_sync() { group_sync<kEpi, 1>(); }
-
 }  // namespace
 
 template <int NQ, bool SELECT, bool I8>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
     k_index_score(const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_q, const KParams p) {
   using C = Cfg<NQ, SELECT, I8>;
+  constexpr int kThreads = C::kThreads;
+  constexpr int kEpi = C::kEpi;
+  auto epi_sync = [] { group_sync<C::kEpi, 1>(); };
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -346,12 +353,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < C::kAcc; ++s) {
       mbar_init(&accfull[s], 1);
-      mbar_init(&accempty[s], 4);
+      mbar_init(&accempty[s], C::kEpiWarps);
     }
     mbar_init(drain, 1);
     for (int s = 0; s < kRing; ++s) {
-      mbar_init(&ring_bars[s], 1);              // full: the TMA warp posted a chunk
-      mbar_init(&ring_bars[kRing + s], 1 + 4);  // empty: MMA thread + 4 epilogue warps read it
+      mbar_init(&ring_bars[s], 1);  // full: the TMA warp posted a chunk
+      mbar_init(&ring_bars[kRing + s], 1 + C::kEpiWarps);  // empty: MMA thread + epilogue warps
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -397,6 +404,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d_hint(dst, &map_k, &full[stage], 0, w.t * kTileM, kb, stream_pol);
         if constexpr (!I8)
           tma_load_3d_hint(dst + kHalfBytes, &map_k, &full[stage], 64, w.t * kTileM, kb, stream_pol);
+        if constexpr (I8) {
+          // the tile's 128 block scales (512 B) into L2 now, so that the
+          // epilogue's load of them does not wait for DRAM
+          const float* sc = p.k_scale + static_cast<int64_t>(kb) * p.cap_blk +
+                            static_cast<int64_t>(w.t) * kTileM;
+          const int64_t left = p.cap_blk - static_cast<int64_t>(w.t) * kTileM;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (q * 32 < left)
+              asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(sc + q * 32) : "memory");
+        }
         ++issued;
         if (++stage == C::kStages) {
           stage = 0;
@@ -475,8 +493,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ======================= epilogue =====================================
     const int quarter = warp & 3;  // TMEM lanes quarter*32 .. +31
-    const int et = tid - 64;       // 0..127
+    const int et = tid - 64;       // 0 .. kEpi-1
     const int row_in_tile = quarter * 32 + lane;
+    const int q0 = ((warp - 2) >> 2) * C::kQPerWarp;  // first query of this thread
     WorkSrc<NQ> src;
     const Walker<NQ>& w = src.w;
     int acc = 0, cur_g = -1;
@@ -531,31 +550,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float scv[NQ];
-#pragma unroll 1
-      for (int j = 0; j < NQ; ++j) {
-        const int r = w.g * NQ + j;
-        if (r >= p.rows) break;  // uniform
-        float v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                               static_cast<uint32_t>(acc * C::kN + j * 32),
-                           v);
+      constexpr int kQ = C::kQPerWarp;
+      float scv[kQ];
+      // ReLU-weighted head sum of one query's 32 accumulator columns; four
+      // interleaved partial sums over the heads (short dependency chains)
+      auto head_sum = [&](const uint32_t* v, int j) {
         const float* wj = w_smem + j * kIdxHeads;
-        // four interleaved partial sums over the heads (short dependency chains)
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int h = 0; h < kIdxHeads; ++h) {
           float x;
           if constexpr (I8) {
-            const int dot = __float_as_int(v[h]);  // exact s32 dot product
+            const int dot = static_cast<int>(v[h]);  // exact s32 dot product
             x = static_cast<float>(dot > 0 ? dot : 0);
           } else {
-            x = v[h] > 0.f ? v[h] : 0.f;
+            const float f = __uint_as_float(v[h]);
+            x = f > 0.f ? f : 0.f;
           }
           s4[h & 3] = __fmaf_rn(wj[h], x, s4[h & 3]);
         }
-        scv[j] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        if constexpr (I8) scv[j] *= ksc;
+        float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        if constexpr (I8) sc *= ksc;
+        return sc;
+      };
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                            static_cast<uint32_t>(acc * C::kN);
+      if constexpr (kQ == 1) {
+        uint32_t v[32];
+        tmem_ld_x32_async(trow + q0 * 32, v);
+        tmem_ld_wait_regs<32>(v);
+        scv[0] = head_sum(v, q0);
+      } else {
+#pragma unroll 1
+        for (int j = 0; j < kQ; j += 2) {  // two 32-column loads per wait
+          uint32_t v0[32], v1[32];
+          tmem_ld_x32_async(trow + (q0 + j) * 32, v0);
+          tmem_ld_x32_async(trow + (q0 + j + 1) * 32, v1);
+          tmem_ld_wait_regs<32>(v0);
+          tmem_ld_wait_regs<32>(v1);
+          scv[j] = head_sum(v0, q0 + j);
+          scv[j + 1] = head_sum(v1, q0 + j + 1);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -565,11 +600,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_ph ^= 1;
       }
 
-#pragma unroll 1
-      for (int j = 0; j < NQ; ++j) {
-        const int r = w.g * NQ + j;
-        if (r >= p.rows) break;
-        if (blk < nb_smem[j]) {
+#pragma unroll
+      for (int j = 0; j < kQ; ++j) {
+        const int r = w.g * NQ + q0 + j;
+        if (r < p.rows && blk < nb_smem[q0 + j]) {
           p.scores[static_cast<int64_t>(r) * p.score_stride + blk] = scv[j];
           if constexpr (SELECT) atomicAdd(&lhist[order_key(scv[j]) >> kHistShift], 1u);
         }
@@ -649,7 +683,7 @@ cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
   p.work_counter = a.work_counter;
   const int grid = score_grid(a.nq, a.rows, a.max_len, a.num_sms);
   if (grid == 0) return cudaSuccess;
-  cudaError_t e = launch_ex(k_index_score<NQ, SELECT, I8>, dim3(grid), dim3(kThreads), C::kSmem,
+  cudaError_t e = launch_ex(k_index_score<NQ, SELECT, I8>, dim3(grid), dim3(C::kThreads), C::kSmem,
                             stream, a.pdl, 1, map_k, map_q, p);
   count_launches(1);
   if (e != cudaSuccess) return e;

@@ -461,17 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_sc, 1);
     fence_mbar_init();
   }
-  if constexpr (kTma && !kSel) {  // (kSel: after the selection, which uses the buffers)
+  if constexpr (kTma) {
     if (tid == 0) prefetch_tensormap(&map_lat);
-    // Rows a tile does not load (skipped blocks, padding, the rest of the
-    // tail block) keep what the buffer held: zero at first, then latent rows
-    // of earlier tiles, so masked tokens (P = 0) never multiply a non-finite
-    // value.  The zeros are written before any TMA write to the buffers.
-    if (worker) {
-      for (int i = tid; i < 2 * kKVBytes / 16; i += kWork)
-        *reinterpret_cast<uint4*>(kv_s + i * 16) = make_uint4(0u, 0u, 0u, 0u);
-      fence_proxy_async();
-    }
   }
   if (warp == 0) {
     tmem_alloc(tmem_holder, 512);
@@ -536,14 +527,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         msm.abv[tid] = 0;
       }
       group_sync<kWork, kBarWork>();
+      // up to 8 entries per thread per round, their loads issued back to back
 #pragma unroll 1
-      for (int f = tid; f < tot; f += kWork) {
-        int k = 0;
-        while (k + 1 < n_cl && ssm.hist[k + 1] <= f) ++k;
-        const int j = f - ssm.hist[k];
-        const uint64_t e = n_cl > 1 ? ld_dsmem_u64(dsmem_addr(l_local + j * 8, k)) : mylist[j];
-        ukey[pad32(f)] = static_cast<uint32_t>(e >> 32);
-        uid[pad32(f)] = static_cast<int32_t>(static_cast<uint32_t>(e));
+      for (int f0 = 0; f0 < tot; f0 += kWork * 8) {
+        uint64_t e[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int f = f0 + u * kWork + tid;
+          e[u] = 0;
+          if (f < tot) {
+            int k = 0;
+            while (k + 1 < n_cl && ssm.hist[k + 1] <= f) ++k;
+            const int j = f - ssm.hist[k];
+            e[u] = n_cl > 1 ? ld_dsmem_u64(dsmem_addr(l_local + j * 8, k)) : mylist[j];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int f = f0 + u * kWork + tid;
+          if (f < tot) {
+            ukey[pad32(f)] = static_cast<uint32_t>(e[u] >> 32);
+            uid[pad32(f)] = static_cast<int32_t>(static_cast<uint32_t>(e[u]));
+          }
+        }
       }
       group_sync<kWork, kBarWork>();
       const uint32_t theta = cut_bin < 0 ? 0u : static_cast<uint32_t>(cut_bin) << kSelKeyShift;
@@ -555,11 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = tid; j < kTopK; j += kWork) p.idx_out[static_cast<int64_t>(r) * kTopK + j] = sel_s[j];
         if (p.cnt_out && tid == 0) p.cnt_out[r] = s_sel_n;
       }
-      if constexpr (kTma) {  // see the zero fill above: now the buffers are free
-        for (int i = tid; i < 2 * kKVBytes / 16; i += kWork)
-          *reinterpret_cast<uint4*>(kv_s + i * 16) = make_uint4(0u, 0u, 0u, 0u);
-        fence_proxy_async();
-      }
+      // the stage held generic writes; TMA writes to it come next
+      fence_proxy_async();
     }
     __syncthreads();
     idx_row = sel_s;
@@ -599,15 +602,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d_hint(kv_s + c * kKVRegion + (row0 + 4 * g) * 128, &map_lat, bar, c * 64,
                            static_cast<int>(pos0), p.lat_batched ? r : 0, lat_pol);
         else {
-          // tokens of the partial tail block: this thread's 128-byte region of each
+          // Tokens of the partial tail block come with cp.async (this
+          // thread's 128-byte region of each); token slots with nothing to
+          // load (skipped blocks, padding) are zeroed, so that a masked
+          // token (P = 0) never multiplies what the buffer held before
+          // (earlier tiles' rows, or other data of this kernel).
 #pragma unroll 1
           for (int i = 0; i < 4; ++i) {
             const int64_t pos = ps[4 * g + i];
-            if (pos < 0) continue;
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              cp_async16(kv_u + kv_off(row0 + 4 * g + i, c * 8 + q),
-                         lat + pos * kLatent + (c * 8 + q) * 8, true);
+            for (int q = 0; q < 8; ++q) {
+              const uint32_t dst = kv_u + kv_off(row0 + 4 * g + i, c * 8 + q);
+              if (pos >= 0)
+                cp_async16(dst, lat + pos * kLatent + (c * 8 + q) * 8, true);
+              else
+                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u)
+                             : "memory");
+            }
           }
         }
       } else {

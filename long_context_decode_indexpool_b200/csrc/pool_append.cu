@@ -17,6 +17,11 @@
 // round twice and could land one bf16 step away from the single rounding of
 // the exact value; the fp64 sum does not.
 //
+// Per-token weights (spx_pool_append_tok): instead of four weights per
+// layer, token p brings its own weight (a learned gate's output; the four
+// weights of a block sum to 1), and the weights of a still-incomplete block
+// wait in a 3-slot weight tail beside the key tail.
+//
 // Work split: grid (x, B).  CTA x of sequence b pools blocks
 // blk_lo + x*kBlocksPerCta ..; 16 threads per block, 8 dims (16 bytes) per
 // thread.  Only the first block of an append can read the tail, and only CTA
@@ -110,6 +115,8 @@ struct PoolKParams {
   const __nv_bfloat16* raw_k;
   int n_new;
   float w[4];
+  const float* raw_w;  // per-token weights [B, n_new] (or NULL: w)
+  float* tail_w;       // per-token weights of the tail [B, pool-1]
   __nv_bfloat16* tail;
   void* pooled;        // bf16 rows, or int8 code rows
   float* k_scale;      // int8 cache: per-block scale
@@ -177,7 +184,10 @@ __global__ void __launch_bounds__(kPoolThreads) k_pool_append(const PoolKParams 
                                              : raw_b + (t - len) * kIdxDim;
         float f[8];
         load8(src + chunk * 8, f);
-        const double wi = static_cast<double>(p.w[i]);
+        const double wi = static_cast<double>(
+            !p.raw_w ? p.w[i]
+                     : (t < len ? p.tail_w[static_cast<int64_t>(b) * (kPool - 1) + t % kPool]
+                                : p.raw_w[static_cast<int64_t>(b) * p.n_new + (t - len)]));
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = __fma_rn(static_cast<double>(f[e]), wi, acc[e]);
       }
@@ -224,6 +234,9 @@ __global__ void __launch_bounds__(kPoolThreads) k_pool_append(const PoolKParams 
     for (int64_t t = (p0 > len ? p0 : len) + sub; t < end; t += kBlocksPerPass) {
       const uint4 v = *reinterpret_cast<const uint4*>(raw_b + (t - len) * kIdxDim + chunk * 8);
       *reinterpret_cast<uint4*>(tail_b + (t % kPool) * kIdxDim + chunk * 8) = v;
+      if (p.raw_w && chunk == 0)
+        p.tail_w[static_cast<int64_t>(b) * (kPool - 1) + t % kPool] =
+            p.raw_w[static_cast<int64_t>(b) * p.n_new + (t - len)];
     }
   }
 }
@@ -254,6 +267,8 @@ cudaError_t launch_pool_append(const PoolAppendArgs& a, cudaStream_t stream) {
   p.raw_k = static_cast<const __nv_bfloat16*>(a.raw_k);
   p.n_new = a.n_new;
   for (int i = 0; i < 4; ++i) p.w[i] = a.w[i];
+  p.raw_w = a.raw_w;
+  p.tail_w = a.tail_w;
   p.tail = static_cast<__nv_bfloat16*>(a.tail);
   p.pooled = a.pooled_k;
   p.k_scale = a.k_scale;

@@ -394,6 +394,34 @@ spx_status spx_pool_append(const spx_dims* d, int32_t B, const void* raw_k, int3
                           len_dev, max_len, stream);
 }
 
+spx_status spx_pool_append_tok(const spx_dims* d, int32_t B, const void* raw_k, const float* raw_w,
+                               int32_t n_new, void* tail, float* tail_w, void* pooled_k,
+                               int64_t cap_blk, const int64_t* len_dev, int64_t max_len,
+                               spx_stream stream) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (B < 1 || B > 65535 || n_new < 0 || cap_blk < 1) return SPX_ERR_SHAPE;
+  if (max_len < n_new || max_len > kPool * cap_blk) return SPX_ERR_SHAPE;
+  if (!tail || !tail_w || !pooled_k || !len_dev || (n_new > 0 && (!raw_k || !raw_w)))
+    return SPX_ERR_INVALID_ARG;
+  if (!al16(tail) || !al16(pooled_k) || (raw_k && !al16(raw_k)) || !al4(len_dev) ||
+      !al4(tail_w) || (raw_w && !al4(raw_w)))
+    return SPX_ERR_INVALID_ARG;
+  if (n_new == 0) return SPX_OK;
+  PoolAppendArgs a{};
+  a.B = B;
+  a.raw_k = raw_k;
+  a.n_new = n_new;
+  a.raw_w = raw_w;
+  a.tail_w = tail_w;
+  a.tail = tail;
+  a.pooled_k = pooled_k;
+  a.cap_blk = cap_blk;
+  a.len_dev = len_dev;
+  a.max_len = max_len;
+  return cuda_status(launch_pool_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 spx_status spx_pool_append_i8(const spx_dims* d, int32_t B, const void* raw_k, int32_t n_new,
                               const float* pool_w, void* tail, void* pooled_k8, float* k_scale,
                               int64_t cap_blk, const int64_t* len_dev, int64_t max_len,

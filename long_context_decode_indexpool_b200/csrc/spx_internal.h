@@ -30,6 +30,8 @@ struct PoolAppendArgs {
   const void* raw_k;
   int n_new;
   float w[4];
+  const float* raw_w;  // optional per-token weights [B, n_new]; tail_w [B, 3] then
+  float* tail_w;
   void* tail;
   void* pooled_k;
   int64_t cap_blk;

@@ -151,6 +151,60 @@ def test_pool_append_i8_learned_weights(lens, n_new):
         assert np.array_equal(gscale[b, lo:hi], rscale[lo:hi]), f"seq {b}"
 
 
+def _token_weights(rng, n_tok):
+    """Per-token pooling weights: each block's four are the softmax of N(0,1)
+    logits (fp32), as a learned gate normalised over its block would give."""
+    g = rng.standard_normal(n_tok + 4)
+    wt = np.empty(n_tok, np.float32)
+    for b in range(0, n_tok, 4):
+        e = np.exp(g[b:b + 4])
+        wt[b:b + 4] = (e / e.sum())[:min(4, n_tok - b)]
+    return wt
+
+
+@pytest.mark.parametrize("lens,n_new", [([0, 5, 10, 3], 7), ([3, 0, 1, 2], 1), ([2, 9, 0, 4], 1003)])
+def test_pool_append_tok_ragged(lens, n_new):
+    """[W1] "IndexPool" with a weight per token: pooled rows, the key tail and
+    the weight tail bit for bit against the oracle, over ragged appends that
+    complete blocks half from the tail and half from the new tokens."""
+    spx = need_gpu()
+    rng = np.random.default_rng(100 + n_new)
+    w = synth.workload("mid")
+    d = spx.dims(64)
+    B = len(lens)
+    total = max(lens) + n_new
+    cap_blk = (total + 3) // 4 + 2
+    raw = [synth.f32_to_bf16_bits_np(rng.standard_normal((total, 128)).astype(np.float32))
+           for _ in range(B)]
+    wts = [_token_weights(rng, total) for _ in range(B)]
+    tail0 = np.zeros((B, 3, 128), np.uint16)
+    tailw0 = np.zeros((B, 3), np.float32)
+    for b, L0 in enumerate(lens):
+        for p_ in range((L0 // 4) * 4, L0):
+            tail0[b, p_ % 4] = raw[b][p_]
+            tailw0[b, p_ % 4] = wts[b][p_]
+    new = np.stack([raw[b][lens[b]:lens[b] + n_new] for b in range(B)])
+    neww = np.stack([wts[b][lens[b]:lens[b] + n_new] for b in range(B)])
+    pooled = torch.zeros(B, cap_blk, 128, dtype=torch.bfloat16, device="cuda")
+    tail = to_dev_bf16(tail0)
+    tail_w = torch.from_numpy(tailw0).cuda()
+    len_dev = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    spx.spx_pool_append_tok(d, B, to_dev_bf16(new), torch.from_numpy(neww).cuda(), n_new, tail,
+                            tail_w, pooled, cap_blk, len_dev, total)
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    got, got_tail, got_tw = bits_of(pooled), bits_of(tail), tail_w.cpu().numpy()
+    for b, L0 in enumerate(lens):
+        end = L0 + n_new
+        ref = oracle.pool_tok(raw[b][:end], wts[b][:end].astype(np.float64))
+        lo, hi = L0 // 4, end // 4
+        assert np.array_equal(got[b, lo:hi], ref[lo:hi]), f"seq {b}"
+        assert (got[b, :lo] == 0).all() and (got[b, hi:] == 0).all()
+        for p_ in range((end // 4) * 4, end):
+            assert np.array_equal(got_tail[b, p_ % 4], raw[b][p_])
+            assert got_tw[b, p_ % 4] == wts[b][p_]
+
+
 # ----------------------------------------------------------------------------
 # Indexer scoring (tcgen05)
 # ----------------------------------------------------------------------------

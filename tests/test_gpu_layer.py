@@ -387,3 +387,63 @@ def test_host_resident_latent_cache_matches_oracle(name):
     assert torch.equal(st.idx, idx_dev)
     assert torch.equal(out.view(torch.int16), out_dev.view(torch.int16))
     assert torch.equal(lse, lse_dev)
+
+
+def test_decode_with_per_token_pool_weights():
+    """A decode step whose IndexPool weights come with the tokens: the cache
+    is built and the new token appended with spx_pool_append_tok, then the
+    fused call runs steps 2-4 (raw_k = NULL).  Block ids bit-exact and
+    attention within tolerance against the oracle's per-token pooling."""
+    spx = need_gpu()
+    w = synth.workload("mid")
+    rng = np.random.default_rng(77)
+    B, L, H = 3, 32768 + 4, 64
+    cap_blk, cap_tok = L // 4, L
+    d = spx.dims(H, w.sm_scale)
+    dev = torch.device("cuda", 0)
+    raw = [w.raw_keys_np(b, 0, L) for b in range(B)]
+    g = rng.standard_normal((B, L))
+    wt = np.exp(g.reshape(B, L // 4, 4))
+    wt = (wt / wt.sum(axis=2, keepdims=True)).astype(np.float32).reshape(B, L)
+    pooled = torch.zeros(B, cap_blk, 128, dtype=torch.bfloat16, device=dev)
+    tail = torch.zeros(B, 3, 128, dtype=torch.bfloat16, device=dev)
+    tail_w = torch.zeros(B, 3, device=dev)
+    zero = torch.zeros(B, dtype=torch.int64, device=dev)
+    # the cache as earlier steps left it: L - 1 tokens, then the new token
+    spx.spx_pool_append_tok(d, B, to_dev_bf16(np.stack([r[:L - 1] for r in raw])),
+                            torch.from_numpy(wt[:, :L - 1].copy()).to(dev), L - 1, tail, tail_w,
+                            pooled, cap_blk, zero, L - 1)
+    len_dev = torch.full((B,), L - 1, dtype=torch.int64, device=dev)
+    spx.spx_pool_append_tok(d, B, to_dev_bf16(np.stack([r[L - 1:] for r in raw])),
+                            torch.from_numpy(wt[:, L - 1:].copy()).to(dev), 1, tail, tail_w,
+                            pooled, cap_blk, len_dev, L)
+    n_vis = torch.full((B,), L, dtype=torch.int64, device=dev)
+    rows = np.arange(B)
+    q_idx = w.q_idx_np(rows)
+    w_head = w.w_head_np(rows)
+    q = w.q_np(rows)
+    g2 = torch.Generator(device=dev).manual_seed(5)
+    lat = (torch.randint(-8, 9, (B, cap_tok, 512), generator=g2, device=dev,
+                         dtype=torch.int16).to(torch.bfloat16) / 16)
+    out = torch.empty(B, H, 512, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, H, device=dev)
+    idx = torch.empty(B, 512, dtype=torch.int32, device=dev)
+    cnt = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = spx.workspace(spx.spx_decode_workspace_size(d, B, L), dev)
+    spx.spx_decode_fused(d, B, None, None, None, pooled, cap_blk, n_vis, to_dev_bf16(q_idx),
+                         torch.from_numpy(w_head).to(dev), to_dev_bf16(q), lat, cap_tok, L, out,
+                         lse, idx, cnt, ws)
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    idx, cnt, lse = idx.cpu().numpy(), cnt.cpu().numpy(), lse.cpu().numpy()
+    refs = []
+    for b in range(B):
+        pk = oracle.pool_tok(raw[b], wt[b].astype(np.float64))
+        assert np.array_equal(bits_of(pooled[b]), pk), f"pooled cache of seq {b}"
+        r = oracle.decode_query(q_idx[b], w_head[b].astype(np.float64), pk, L, q[b],
+                                lambda pos, b=b: bits_of(lat[b, torch.from_numpy(pos).to(dev)]),
+                                w.sm_scale)
+        assert cnt[b] == r["idx"].size and np.array_equal(idx[b, :cnt[b]], r["idx"]), f"seq {b}"
+        assert np.allclose(lse[b], r["lse"], atol=LSE_ATOL, rtol=0)
+        refs.append(r["out"])
+    assert_attention_close(f64_of(out), np.stack(refs), "per-token pooling")
