@@ -134,7 +134,8 @@ class DecodeState:
         self._call = None
         torch.cuda.synchronize(device)
 
-    def step(self, timing=None, raw_new=None, q_idx=None, w_head=None, q=None, out=None):
+    def step(self, timing=None, raw_new=None, q_idx=None, w_head=None, q=None, out=None,
+             stream=None):
         spx = spx_module()
         if self._call is None:  # device pointers and host arguments, resolved once
             self._call = dict(
@@ -155,13 +156,13 @@ class DecodeState:
                 self.d, self.B, raw_new, c["pool_w"], c["tail"], c["pooled"], self.k_scale,
                 self.cap_blk, c["len_dev"], q_idx, w_head, q, c["latent"], self.cap_tok,
                 self.max_len, out, c["lse"], c["idx"], c["count"], c["ws"], ws_bytes=c["ws_bytes"],
-                timing=timing, stream=c["stream"])
+                timing=timing, stream=c["stream"] if stream is None else stream)
         else:
             spx.spx_decode_fused(
                 self.d, self.B, raw_new, c["pool_w"], c["tail"], c["pooled"], self.cap_blk,
                 c["len_dev"], q_idx, w_head, q, c["latent"], self.cap_tok, self.max_len, out,
                 c["lse"], c["idx"], c["count"], c["ws"], ws_bytes=c["ws_bytes"], timing=timing,
-                stream=c["stream"])
+                stream=c["stream"] if stream is None else stream)
 
     # ---- host copies of what the oracle needs (generator output) ----
     def raw_keys_host(self, b: int) -> np.ndarray:
@@ -626,7 +627,7 @@ def run_decode(args, world, rank, local):
     score_avg = time_scoring_launches(st, stream, max(8, min(K, 64)))
 
     # ---- end to end: host buffers in, host result out, every step ----------
-    e2e_ms, h2d, d2h = run_e2e(st, stream, K, args.warmup, world, device)
+    e2e_ms, h2d, d2h, e2e_mode = run_e2e(st, stream, K, args.warmup, world, device)
     if spx.spx_device_error() != 0:
         raise RuntimeError("device error during the timed region")
 
@@ -674,7 +675,7 @@ def run_decode(args, world, rank, local):
                           "frac": step_gbs / hbm, "peak_source": f"{src} hbm_gbs",
                           "frac_of_8tbs": step_gbs / 8000.0},
         "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": "queries/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "launch": e2e_mode},
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
     }
@@ -684,13 +685,14 @@ def run_decode(args, world, rank, local):
 def run_e2e(st, stream, K: int, warmup: int, world: int, device):
     """K decode steps through the public call with host buffers: every step
     copies its inputs (new raw key, indexer query and weights, MLA query:
-    one packed pinned buffer, one copy) to the device and its output back
-    to pinned host memory, and the host waits for every step's output.
-    Copies run on a second stream into two alternating device buffers, so
-    step k+1's inputs and step k-1's output move while step k computes; the
-    host waits for step k-1's output after enqueuing step k.  Timed by the
-    host clock from the first copy to the last output in host memory
-    (max over ranks).  Returns (ms, h2d bytes per step, d2h bytes per step)."""
+    one packed pinned buffer, one copy) to the device, runs the fused call
+    and copies the output back to pinned host memory; the host waits for
+    every step's output, one step behind (it enqueues step k, then waits for
+    step k-1).  Each step is one replay of a CUDA graph captured from those
+    three operations (two graphs, alternating device and host buffers), so
+    the host's per-step cost is one graph launch.  Timed by the host clock
+    from the first copy to the last output in host memory (max over ranks).
+    Returns (ms, h2d bytes per step, d2h bytes per step, mode)."""
     ins = (st.raw_new, st.q_idx, st.w_head, st.q)
     sizes = [t.numel() * t.element_size() for t in ins]
     offs = [0]
@@ -705,29 +707,43 @@ def run_e2e(st, stream, K: int, warmup: int, world: int, device):
              for d in d_in]
     d_out = [torch.empty_like(st.out) for _ in range(2)]
     h_out = [torch.empty(st.out.shape, dtype=st.out.dtype, pin_memory=True) for _ in range(2)]
-    copy = torch.cuda.Stream(device)
-    ev = lambda: torch.cuda.Event()
-    in_ready, used, out_ready, out_home = ([ev(), ev()] for _ in range(4))
+    d2h = h_out[0].numel() * h_out[0].element_size()
+
+    def body(i, s):
+        d_in[i].copy_(h_in, non_blocking=True)
+        raw, qi, wh, q = views[i]
+        st.step(raw_new=raw, q_idx=qi, w_head=wh, q=q, out=d_out[i], stream=s.cuda_stream)
+        h_out[i].copy_(d_out[i], non_blocking=True)
+
+    graphs = None
+    try:
+        cap = torch.cuda.Stream(device)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            body(0, cap)  # (warm the library's per-device caches on this stream)
+        cap.synchronize()
+        graphs = []
+        for i in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                body(i, cap)
+            graphs.append(g)
+        stream.wait_stream(cap)
+    except Exception:
+        graphs = None  # capture not available: the same three operations, eagerly
+    done = [torch.cuda.Event(), torch.cuda.Event()]
 
     def run(n):
         for k in range(n):
             i = k & 1
-            with torch.cuda.stream(copy):
-                if k >= 2:
-                    copy.wait_event(used[i])  # step k-2 has finished reading d_in[i]
-                d_in[i].copy_(h_in, non_blocking=True)
-                in_ready[i].record(copy)
-            stream.wait_event(in_ready[i])
-            raw, qi, wh, q = views[i]
-            st.step(raw_new=raw, q_idx=qi, w_head=wh, q=q, out=d_out[i])
-            used[i].record(stream)
-            with torch.cuda.stream(copy):
-                copy.wait_event(used[i])
-                h_out[i].copy_(d_out[i], non_blocking=True)
-                out_home[i].record(copy)
+            if graphs is not None:
+                graphs[i].replay()
+            else:
+                body(i, stream)
+            done[i].record(stream)
             if k >= 1:
-                out_home[i ^ 1].synchronize()  # the host has step k-1's output
-        out_home[(n - 1) & 1].synchronize()
+                done[i ^ 1].synchronize()  # the host has step k-1's output
+        done[(n - 1) & 1].synchronize()
 
     run(max(warmup, 2))
     barrier(world)
@@ -736,7 +752,8 @@ def run_e2e(st, stream, K: int, warmup: int, world: int, device):
     run(K)
     ms = (time.perf_counter() - t0) * 1e3
     torch.cuda.synchronize(device)
-    return max_over_ranks(ms, world, device), total, h_out[0].numel() * h_out[0].element_size()
+    return (max_over_ranks(ms, world, device), total, d2h,
+            "graph replay" if graphs is not None else "eager")
 
 
 def time_scoring_launches(st, stream, n: int) -> float:

@@ -298,6 +298,40 @@ SPX_API spx_status spx_sparse_mla_attn(const spx_dims* d, int32_t rows, const vo
                                size_t ws_bytes, spx_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * FP8 (E4M3) latent cache.  [W1] section "양자화: W8A8와 혼합 캐시": recent,
+ * important cache entries are kept in FP8.  The page gives no format or
+ * scale; libspx stores a 512-wide latent row x as E4M3 codes (4 exponent
+ * bits with bias 7, 3 mantissa bits, largest 448, subnormal step 2^-9) of
+ * x / 2^e, rounded to nearest (ties to even), with one power-of-two scale
+ * per row: e the smallest integer with max |x| <= 448 * 2^e (not below -149;
+ * 0 for an all-zero row).  Half the bytes of the bf16 cache; a dequantised
+ * row (code value * 2^e) is exact in bf16.
+ *
+ * spx_latent_quant_fp8 writes n rows: codes uint8 [n, 512] (16-byte aligned)
+ * and exps int32 [n] from latent bf16 [n, 512] (all DEVICE memory); the
+ * caller points it at the rows of its cache that are new.
+ *
+ * spx_sparse_mla_attn_fp8 is step 4 over such a cache: the same attended set
+ * and result definition as spx_sparse_mla_attn, with the latent rows read as
+ * their dequantised values.  codes uint8: row r reads tokens
+ * codes + r*seq_stride + t*512 (seq_stride 0: a shared cache; a multiple of
+ * 512), exps int32 at r*(seq_stride/512) + t.  It first gathers the attended
+ * rows, dequantised, into the workspace (about 2.1 MB per row), then runs the
+ * attention kernel on them; ws is spx_attn_fp8_workspace_size bytes.
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_latent_quant_fp8(const void* latent, int64_t n, void* codes,
+                                        int32_t* exps, spx_stream stream);
+SPX_API spx_status spx_attn_fp8_workspace_size(const spx_dims* d, int32_t rows,
+                                               int64_t max_len, size_t* bytes);
+SPX_API spx_status spx_sparse_mla_attn_fp8(const spx_dims* d, int32_t rows, const void* q,
+                                           const void* codes, const int32_t* exps,
+                                           int64_t seq_stride, int64_t cap_tok,
+                                           const int32_t* idx, const int32_t* count,
+                                           const int64_t* n_vis, int64_t max_len, void* out,
+                                           float* lse, void* ws, size_t ws_bytes,
+                                           spx_stream stream);
+
+/* ---------------------------------------------------------------------------
  * Fused decode step: steps 1-4 for one new token per sequence, in one call.
  * If raw_k is non-NULL the step first appends raw_k[b] (bf16 [B, 1, idx_dim])
  * at position len_dev[b], and the query sees n = len_dev[b] + 1 tokens;

@@ -74,6 +74,10 @@ _SIGS = {
     "spx_attn_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_sparse_mla_attn": ([_DIMS, _I32, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P],
                             ctypes.c_int),
+    "spx_latent_quant_fp8": ([_P, _I64, _P, _P, _P], ctypes.c_int),
+    "spx_attn_fp8_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "spx_sparse_mla_attn_fp8": ([_DIMS, _I32, _P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P,
+                                 _SZ, _P], ctypes.c_int),
     "spx_decode_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_decode_fused": ([_DIMS, _I32, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _I64, _I64, _P,
                           _P, _P, _P, _P, _SZ, ctypes.POINTER(spx_timing), _P], ctypes.c_int),
@@ -248,6 +252,28 @@ def spx_sparse_mla_attn(d, rows, q, latent, seq_stride, cap_tok, idx, count, n_v
                                     cap_tok, _ptr(idx), _ptr(count), _ptr(n_vis), max_len,
                                     _ptr(out), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
            "spx_sparse_mla_attn")
+
+
+def spx_latent_quant_fp8(latent, n, codes, exps, stream=None):
+    _check(_lib.spx_latent_quant_fp8(_ptr(latent), n, _ptr(codes), _ptr(exps), _stream(stream)),
+           "spx_latent_quant_fp8")
+
+
+def spx_attn_fp8_workspace_size(d, rows, max_len) -> int:
+    n = _SZ(0)
+    _check(_lib.spx_attn_fp8_workspace_size(ctypes.byref(d), rows, max_len, ctypes.byref(n)),
+           "spx_attn_fp8_workspace_size")
+    return n.value
+
+
+def spx_sparse_mla_attn_fp8(d, rows, q, codes, exps, seq_stride, cap_tok, idx, count, n_vis,
+                            max_len, out, lse=None, ws=None, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.spx_sparse_mla_attn_fp8(ctypes.byref(d), rows, _ptr(q), _ptr(codes), _ptr(exps),
+                                        seq_stride, cap_tok, _ptr(idx), _ptr(count), _ptr(n_vis),
+                                        max_len, _ptr(out), _ptr(lse), _ptr(ws), ws_bytes,
+                                        _stream(stream)), "spx_sparse_mla_attn_fp8")
 
 
 def spx_decode_workspace_size(d, B, max_len) -> int:

@@ -73,13 +73,12 @@ namespace spx {
 
 namespace {
 
-constexpr int kThreads = 160;                   // 4 worker warps + 1 MMA warp
+constexpr int kThreads = 192;                   // 4 worker warps, MMA warp, gather warp
 constexpr int kWork = 128;                      // worker threads
-// named barriers (0 is __syncthreads)
+constexpr int kMmaWarp = 4;
+constexpr int kProdWarp = 5;
+// named barrier (0 is __syncthreads)
 constexpr int kBarWork = 1;                     // workers only
-constexpr int kBarData0 = 2;                    // tile data ready (S buffer 0 / 1)
-constexpr int kBarData1 = 3;
-constexpr int kBarP = 4;                        // P of a tile written
 constexpr int kTT = 64;                         // tokens per tile
 constexpr int kHG = 64;                         // heads per CTA (MMA M)
 constexpr int kRegion = 64 * 128;               // [64 rows x 128 B] = 8 KiB
@@ -88,13 +87,13 @@ constexpr int kKVBytes = 8 * kRegion;           // 64 KiB per tile
 // The two latent tiles share 8 regions of [128 rows x 128 B] (tile b in rows
 // 64b..64b+63), so that both together also form one N = 128 operand.
 constexpr int kKVRegion = 2 * kRegion;          // 16 KiB
-constexpr int kPBytes = kRegion;                // [64 heads x 64 tokens] bf16
+constexpr int kPBytes = kRegion;                // [64 heads x 64 tokens] bf16 (two buffers)
 constexpr int kMaxList = kTopK * kPool + kPool - 1;             // tokens in a list, at most
 constexpr int kPosCap = (kMaxList + kTT - 1) / kTT * kTT;       // position slots
 constexpr int kMaxCluster = 16;                 // splits per (row, head group)
-constexpr int kSmemBytes = 1024 + kQBytes + 2 * kKVBytes + kPBytes + kPosCap * 8 +
-                           (kPosCap / 32) * 4 + 64;
-static_assert(((kPosCap * 8 + (kPosCap / 32) * 4) & 7) == 0, "barriers 8-byte aligned");
+constexpr int kSmemBytes = 1024 + kQBytes + 2 * kKVBytes + 2 * kPBytes + kPosCap * 4 +
+                           (kPosCap / 32) * 4 + 128;
+static_assert(((kPosCap * 4 + (kPosCap / 32) * 4) & 7) == 0, "barriers 8-byte aligned");
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLazy = 8.f;                    // rescale threshold (log2 units)
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, kTT);
@@ -429,19 +428,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* q_s = sm;
   uint8_t* kv_s = q_s + kQBytes;  // two latent tiles; afterwards the combine rows
-  uint8_t* p_s = kv_s + 2 * kKVBytes;
-  int64_t* pos_s = reinterpret_cast<int64_t*>(p_s + kPBytes);     // [kPosCap]
-  uint32_t* vm_s = reinterpret_cast<uint32_t*>(pos_s + kPosCap);  // [kPosCap / 32] valid bits
-  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(vm_s + kPosCap / 32);  // [2]: S buffer b done
-  uint64_t* bar_pv = bar_qk + 2;
-  uint64_t* bar_red = bar_qk + 3;  // combine: rows of the other splits
-  uint64_t* bar_kv = bar_qk + 4;   // [2]: TMA bytes of latent tile buffer b landed
-  uint64_t* bar_sc = bar_qk + 6;   // kSel: staged scores landed
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 7);
+  uint8_t* p_s = kv_s + 2 * kKVBytes;                               // [2] P buffers
+  int32_t* pos_s = reinterpret_cast<int32_t*>(p_s + 2 * kPBytes);   // [kPosCap]
+  uint32_t* vm_s = reinterpret_cast<uint32_t*>(pos_s + kPosCap);    // [kPosCap / 32] valid bits
+  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(vm_s + kPosCap / 32);  // [2]: S(t) in buffer t&1
+  uint64_t* bar_pv = bar_qk + 2;   // [2]: PV(t) done, t & 1
+  uint64_t* bar_kv = bar_qk + 4;   // [2]: tile t in latent buffer t & 1
+  uint64_t* bar_p = bar_qk + 6;    // [2]: P(t) written, t & 1
+  uint64_t* bar_q = bar_qk + 8;    // Q landed
+  uint64_t* bar_red = bar_qk + 9;  // combine: rows of the other splits
+  uint64_t* bar_sc = bar_qk + 10;  // kSel: staged scores landed
+  uint64_t* bar_drain = bar_qk + 11;  // every MMA of the CTA done
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 12);
 
   const int split = blockIdx.x, r = blockIdx.y, hg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool worker = tid < kWork;  // warps 0-3; warp 4 issues the MMAs
+  const bool worker = tid < kWork;  // warps 0-3; warp 4 issues the MMAs, warp 5 gathers
   const int h0 = hg * kHG;
   const int n_cl = p.nsplit;
   // head of this thread; lanes i and 16+i of a worker warp share it
@@ -452,13 +454,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- set-up that needs nothing from the previous kernel -------------------
   if (tid == 0) {
-    mbar_init(&bar_qk[0], 1);
-    mbar_init(&bar_qk[1], 1);
-    mbar_init(bar_pv, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_qk[i], 1);
+      mbar_init(&bar_pv[i], 1);
+      mbar_init(&bar_kv[i], 1);          // the gather warp, plus the tile's TMA bytes
+      mbar_init(&bar_p[i], kWork / 32);  // one arrive per worker warp
+    }
+    mbar_init(bar_q, kWork / 32);
     mbar_init(bar_red, 1);
-    mbar_init(&bar_kv[0], kWork / 32);  // one arrive.expect_tx per worker warp and tile
-    mbar_init(&bar_kv[1], kWork / 32);
     mbar_init(bar_sc, 1);
+    mbar_init(bar_drain, 1);
     fence_mbar_init();
   }
   if constexpr (kTma) {
@@ -491,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ int s_list_n, s_sel_n;
     // the list of this CTA: in the tail of the position array, which this
     // split's positions never reach while the cluster may read it
-    uint64_t* mylist = reinterpret_cast<uint64_t*>(pos_s + kPosCap - kTopK);
+    uint64_t* mylist = reinterpret_cast<uint64_t*>(pos_s + kPosCap - 2 * kTopK);
     int32_t* sel_s = reinterpret_cast<int32_t*>(p_s);  // chosen ids, until P is written
     int64_t nv = p.n_vis[r];
     nv = nv < 0 ? 0 : (nv > p.len_cap ? p.len_cap : nv);
@@ -585,62 +590,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (ntiles > 0) {  // uniform
     const __nv_bfloat16* lat = p.latent + static_cast<int64_t>(r) * p.seq_stride;
-    const uint64_t lat_pol = p.lat_evict_first ? l2_evict_first_policy() : l2_evict_normal_policy();
-    auto gather = [&](int tile) {
-      const int row0 = (tile & 1) * kTT;
-      const int64_t* ps = pos_s + tile * kTT;
-      if constexpr (kTma) {
-        // thread t: 4-token group g = t / 8 of the tile, swizzle region c = t % 8
-        const int g = tid >> 3, c = tid & 7;
-        const int64_t pos0 = ps[4 * g];
-        const bool full = j_begin + tile * kTT + 4 * g < ri.cnt * kPool && pos0 >= 0;
-        const uint32_t ball = __ballot_sync(0xffffffffu, full && c == 0);
-        uint64_t* bar = &bar_kv[tile & 1];
-        if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(__popc(ball)) * 4096u);
-        __syncwarp();
-        if (full)
-          tma_load_3d_hint(kv_s + c * kKVRegion + (row0 + 4 * g) * 128, &map_lat, bar, c * 64,
-                           static_cast<int>(pos0), p.lat_batched ? r : 0, lat_pol);
-        else {
-          // Tokens of the partial tail block come with cp.async (this
-          // thread's 128-byte region of each); token slots with nothing to
-          // load (skipped blocks, padding) are zeroed, so that a masked
-          // token (P = 0) never multiplies what the buffer held before
-          // (earlier tiles' rows, or other data of this kernel).
-#pragma unroll 1
-          for (int i = 0; i < 4; ++i) {
-            const int64_t pos = ps[4 * g + i];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const uint32_t dst = kv_u + kv_off(row0 + 4 * g + i, c * 8 + q);
-              if (pos >= 0)
-                cp_async16(dst, lat + pos * kLatent + (c * 8 + q) * 8, true);
-              else
-                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u)
-                             : "memory");
-            }
-          }
-        }
-      } else {
-#pragma unroll 4
-        for (int i = 0; i < (kTT * 64) / kWork; ++i) {
-          const int c = i * kWork + tid;
-          const int t = c >> 6, piece = c & 63;
-          const int64_t pos = ps[t];
-          cp_async16(kv_u + kv_off(row0 + t, piece), lat + (pos >= 0 ? pos : 0) * kLatent + piece * 8,
-                     pos >= 0);
-        }
-      }
-      cp_async_commit();
-    };
-    // the TMA bytes of tile t have landed (cp.async parts are waited for by
-    // the caller with cp_async_wait)
-    auto tma_landed = [&](int t) {
-      if constexpr (kTma) {
-        volatile int no_abort = 0;
-        ok_all &= mbar_wait(&bar_kv[t & 1], (t >> 1) & 1, &no_abort);
-      }
-    };
     if (worker) {
       // every token position of the split, once, with a validity bit per token
 #pragma unroll 1
@@ -652,106 +601,163 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int b = i0 == 0 ? b_first : (j < ri.cnt * kPool ? idx_row[j >> 2] : -1);
           pos = token_pos_of(ri, j, b);
         }
-        if (i < ntiles * kTT) pos_s[i] = pos;
+        if (i < ntiles * kTT) pos_s[i] = static_cast<int32_t>(pos);
         const uint32_t bits = __ballot_sync(0xffffffffu, pos >= 0);
         if (lane == 0 && i < ntiles * kTT) vm_s[i >> 5] = bits;
       }
-      named_sync(kBarWork, kWork);
-      gather(0);                   // group: Q + tile 0
-      if (ntiles > 1) gather(1);   // group: tile 1
+      // Q has landed (the workers' only cp.async group)
+      cp_async_wait<0>();
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_q);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     tmem = *tmem_holder;
 
-    if (!worker) {
-      // ======================= MMA issuer (warp 4) ===========================
-      // S = Q C^T of tile t into S buffer t&1 (TMEM lanes 16-31 of each
-      // quarter, columns 256+64b ..), once the workers report its data.
-      // pair: tiles 0 and 1 as one N = 128 product (S buffers 0 and 1 are
-      // adjacent columns), committed to both buffers' barriers
-      auto qk = [&](int t, bool pair) {
-        named_sync(kBarData0 + (t & 1), kThreads);
-        if (pair) named_sync(kBarData1, kThreads);
-        if (lane == 0) {
-          tc_fence_after();
-          const uint32_t kvb = kv_u + (t & 1) * kTT * 128;
-          const uint32_t d = tmem + (16u << 16) + 256 + 64 * (t & 1);
-#pragma unroll 4
-          for (int k = 0; k < kLatent / 16; ++k) {
-            const uint32_t qoff = (k >> 2) * kRegion + (k & 3) * 32;
-            const uint32_t koff = (k >> 2) * kKVRegion + (k & 3) * 32;
-            umma_bf16(d, sdesc_kmajor_sw128(q_u + qoff), sdesc_kmajor_sw128(kvb + koff),
-                      pair ? kIdescQK2 : kIdescQK, k > 0 ? 1u : 0u);
-          }
-          umma_commit(&bar_qk[t & 1]);
-          if (pair) umma_commit(&bar_qk[1]);
-        }
-        __syncwarp();
-      };
-      qk(0, ntiles > 1);
+    if (warp == kProdWarp) {
+      // ======================= gather producer (warp 5) ======================
+      // Tile t goes into buffer t & 1 as soon as PV(t-2) has released it.
+      const uint64_t lat_pol =
+          p.lat_evict_first ? l2_evict_first_policy() : l2_evict_normal_policy();
 #pragma unroll 1
-      for (int j = 0; j < ntiles; ++j) {
-        // O += P C once the workers have written P of tile j
-        named_sync(kBarP, kThreads);
-        if (lane == 0) {
-          tc_fence_after();
-          const uint32_t kvb = kv_u + (j & 1) * kTT * 128;
+      for (int t = 0; t < ntiles; ++t) {
+        if (t >= 2) {
+          volatile int no_abort = 0;
+          ok_all &= mbar_wait(&bar_pv[t & 1], ((t - 2) >> 1) & 1, &no_abort);
+        }
+        const int row0 = (t & 1) * kTT;
+        const int32_t* ps = pos_s + t * kTT;
+        uint64_t* bar = &bar_kv[t & 1];
+        if constexpr (kTma) {
+          // 16 four-token groups x 8 swizzle regions; lane l takes (g, c) for
+          // l, l+32, l+64, l+96; a group is a selected block in range, by
+          // TMA, or anything else (tail tokens by cp.async, empty slots zeroed)
+          const int glane = lane & 15;
+          const bool gfull =
+              j_begin + t * kTT + 4 * glane < ri.cnt * kPool && ps[4 * glane] >= 0;
+          const uint32_t fullmask = __ballot_sync(0xffffffffu, lane < 16 && gfull);
+          if (lane == 0) mbar_expect_tx(bar, static_cast<uint32_t>(__popc(fullmask)) * 4096u);
+          __syncwarp();
+#pragma unroll 1
+          for (int u = 0; u < 4; ++u) {
+            const int id = u * 32 + lane;
+            const int g = id >> 3, c = id & 7;
+            if ((fullmask >> g) & 1u) {
+              tma_load_3d_hint(kv_s + c * kKVRegion + (row0 + 4 * g) * 128, &map_lat, bar, c * 64,
+                               ps[4 * g], p.lat_batched ? r : 0, lat_pol);
+            } else {
+#pragma unroll 1
+              for (int i = 0; i < 4; ++i) {
+                const int pos = ps[4 * g + i];
 #pragma unroll
-          for (int k = 0; k < kTT / 16; ++k) {
-            const uint64_t ad = sdesc_kmajor_sw128(p_u + k * 32);
-#pragma unroll
-            for (int nh = 0; nh < 2; ++nh) {
-              const uint64_t bd =
-                  sdesc_mn_sw128(kvb + nh * 4 * kKVRegion + k * 16 * 128, kKVRegion, 1024);
-              umma_bf16(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
-                        (j > 0 || k > 0) ? 1u : 0u);
+                for (int q = 0; q < 8; ++q) {
+                  const uint32_t dst = kv_u + kv_off(row0 + 4 * g + i, c * 8 + q);
+                  if (pos >= 0)
+                    cp_async16(dst, lat + static_cast<int64_t>(pos) * kLatent + (c * 8 + q) * 8,
+                               true);
+                  else
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u)
+                                 : "memory");
+                }
+              }
             }
           }
-          umma_commit(bar_pv);
+        } else {
+#pragma unroll 4
+          for (int i = 0; i < (kTT * 64) / 32; ++i) {
+            const int c = i * 32 + lane;
+            const int tk = c >> 6, piece = c & 63;
+            const int pos = ps[tk];
+            cp_async16(kv_u + kv_off(row0 + tk, piece),
+                       lat + static_cast<int64_t>(pos >= 0 ? pos : 0) * kLatent + piece * 8,
+                       pos >= 0);
+          }
         }
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async();
         __syncwarp();
-        if (j + 2 < ntiles) qk(j + 2, false);
+        if (lane == 0) mbar_arrive(bar);  // with the TMA bytes: tile t is in place
       }
-    } else {
+    } else if (warp == kMmaWarp) {
+      // ======================= MMA issuer (warp 4) ===========================
+      // Issues whichever is ready first: S = Q C^T of the next tile (its data
+      // landed, and the softmax of the tile that last used its S buffer is
+      // done), or O += P C of the oldest tile whose P is written.  Tiles 0
+      // and 1 go as one N = 128 product (their S buffers are adjacent).
+      if (lane == 0) {
+        volatile int no_abort = 0;
+        ok_all &= mbar_wait(bar_q, 0, &no_abort);
+        const uint32_t aq = smem_u32(&bar_kv[0]), aq1 = smem_u32(&bar_kv[1]);
+        const uint32_t ap0 = smem_u32(&bar_p[0]), ap1 = smem_u32(&bar_p[1]);
+        int nq = 0, np = 0;
+        uint64_t t_last = globaltimer_ns();
+        while (np < ntiles && ok_all) {
+          const bool pair = nq == 0 && ntiles > 1;
+          bool qk_ready = false;
+          if (nq < ntiles && nq <= np + 1) {
+            qk_ready = mbar_try_wait((nq & 1) ? aq1 : aq, (nq >> 1) & 1);
+            if (qk_ready && pair) qk_ready = mbar_try_wait(aq1, 0);
+          }
+          if (qk_ready) {
+            tc_fence_after();
+            const uint32_t kvb = kv_u + (nq & 1) * kTT * 128;
+            const uint32_t d = tmem + (16u << 16) + 256 + 64 * (nq & 1);
+#pragma unroll 4
+            for (int k = 0; k < kLatent / 16; ++k) {
+              const uint32_t qoff = (k >> 2) * kRegion + (k & 3) * 32;
+              const uint32_t koff = (k >> 2) * kKVRegion + (k & 3) * 32;
+              umma_bf16(d, sdesc_kmajor_sw128(q_u + qoff), sdesc_kmajor_sw128(kvb + koff),
+                        pair ? kIdescQK2 : kIdescQK, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&bar_qk[nq & 1]);
+            if (pair) umma_commit(&bar_qk[1]);
+            nq += pair ? 2 : 1;
+            t_last = globaltimer_ns();
+            continue;
+          }
+          if (np < nq && mbar_try_wait((np & 1) ? ap1 : ap0, (np >> 1) & 1)) {
+            tc_fence_after();
+            const uint32_t kvb = kv_u + (np & 1) * kTT * 128;
+            const uint32_t pb = p_u + (np & 1) * kPBytes;
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+#pragma unroll
+              for (int k = 0; k < kTT / 16; ++k) {
+                const uint64_t ad = sdesc_kmajor_sw128(pb + k * 32);
+                const uint64_t bd =
+                    sdesc_mn_sw128(kvb + nh * 4 * kKVRegion + k * 16 * 128, kKVRegion, 1024);
+                umma_bf16(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
+                          (np > 0 || k > 0) ? 1u : 0u);
+              }
+            }
+            umma_commit(&bar_pv[np & 1]);
+            ++np;
+            t_last = globaltimer_ns();
+            continue;
+          }
+          if (globaltimer_ns() - t_last > kWaitLimitNs) {
+            ok_all = false;
+            atomicExch(&g_device_error, kErrWaitTimeout);
+          }
+        }
+        // every MMA issued here completes before TMEM is read or released
+        umma_commit(bar_drain);
+        mbar_wait(bar_drain, 0, &no_abort);
+      }
+      __syncwarp();
+    } else if (worker) {
       // ======================= workers (warps 0-3) ==========================
 #pragma unroll 1
       for (int j = 0; j < ntiles; ++j) {
         const int buf = j & 1;
-        // report tile data to the MMA warp (tiles 0 and 1 were requested
-        // together; tile j >= 2 one iteration ago)
-        if (j == 0) {
-          if (ntiles > 1) cp_async_wait<1>();
-          else cp_async_wait<0>();
-          tma_landed(0);
-          fence_proxy_async();
-          named_arrive(kBarData0, kThreads);
-          if (ntiles > 1) {
-            cp_async_wait<0>();
-            tma_landed(1);
-            fence_proxy_async();
-            named_arrive(kBarData1, kThreads);
-          }
-        } else if (j >= 2) {
-          cp_async_wait<0>();
-          tma_landed(j);
-          fence_proxy_async();
-          named_arrive(kBarData0 + buf, kThreads);
-        }
         {
           volatile int no_abort = 0;
           ok_all &= mbar_wait(&bar_qk[buf], (j >> 1) & 1, &no_abort);
         }
         tc_fence_after();
-        // the previous PV must be done before its buffer is refilled and before
-        // P or O are touched again
-        if (j > 0) {
-          volatile int no_abort = 0;
-          ok_all &= mbar_wait(bar_pv, (j - 1) & 1, &no_abort);
-          tc_fence_after();
-          if (j + 1 < ntiles) gather(j + 1);
-        }
 
         // ---- softmax: 32 logits of head hloc per thread --------------------
         float s[32];
@@ -787,7 +793,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_run = mt;
         }
         if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
-          // each thread scales its half of the O row of its head
+          // O holds tiles up to j-1: let PV(j-1) finish, then each thread
+          // scales its half of the O row of its head
+          {
+            volatile int no_abort = 0;
+            ok_all &= mbar_wait(&bar_pv[(j - 1) & 1], ((j - 1) >> 1) & 1, &no_abort);
+          }
+          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             float v[32];
@@ -814,22 +826,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         float lsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
         l_run = l_run * alpha + lsum;
+        // P buffer j & 1 is free once PV(j-2) is done
+        if (j >= 2) {
+          volatile int no_abort = 0;
+          ok_all &= mbar_wait(&bar_pv[buf], ((j - 2) >> 1) & 1, &no_abort);
+        }
         // row hloc of P, pieces 4*half .. 4*half+3 (16 B each)
+        const uint32_t pb = p_u + buf * kPBytes;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int piece = 4 * half + c;
-          const uint32_t a = p_u + hloc * 128 + ((piece ^ (hloc & 7)) << 4);
+          const uint32_t a = pb + hloc * 128 + ((piece ^ (hloc & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(packed[4 * c]),
                        "r"(packed[4 * c + 1]), "r"(packed[4 * c + 2]), "r"(packed[4 * c + 3])
                        : "memory");
         }
         fence_proxy_async();
         tc_fence_before();
-        named_arrive(kBarP, kThreads);  // the MMA warp issues O += P C
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_p[buf]);  // the MMA warp issues O += P C
       }
       {
         volatile int no_abort = 0;
-        ok_all &= mbar_wait(bar_pv, (ntiles - 1) & 1, &no_abort);
+        ok_all &= mbar_wait(&bar_pv[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, &no_abort);
       }
       tc_fence_after();
     }

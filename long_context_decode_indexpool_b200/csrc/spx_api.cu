@@ -567,6 +567,104 @@ spx_status spx_sparse_mla_attn(const spx_dims* d, int32_t rows, const void* q, c
 }
 
 // ---------------------------------------------------------------------------
+spx_status spx_latent_quant_fp8(const void* latent, int64_t n, void* codes, int32_t* exps,
+                                spx_stream stream) {
+  if (n < 0) return SPX_ERR_SHAPE;
+  if (n == 0) return SPX_OK;
+  if (!latent || !codes || !exps) return SPX_ERR_INVALID_ARG;
+  if (!al16(latent) || !al16(codes) || !al4(exps)) return SPX_ERR_INVALID_ARG;
+  return cuda_status(launch_latent_quant_fp8(latent, n, static_cast<uint8_t*>(codes), exps,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace of spx_sparse_mla_attn_fp8: compact bf16 rows [rows, 2052, 512]
+// | ids [rows, 512] | counts [rows] | lengths [rows] | attention scratch
+struct Fp8Layout {
+  size_t dense, cidx, ccnt, cnvis, attn, total;
+  AttnPlan ap;
+};
+
+Fp8Layout fp8_layout(int rows, int heads) {
+  Fp8Layout L{};
+  L.ap = plan_attn(rows, heads, kFp8Dense, device_sm_count());
+  size_t o = 0;
+  L.dense = o;
+  o += up(static_cast<size_t>(rows) * kFp8Dense * kLatent * 2);
+  L.cidx = o;
+  o += up(static_cast<size_t>(rows) * kTopK * 4);
+  L.ccnt = o;
+  o += up(static_cast<size_t>(rows) * 4);
+  L.cnvis = o;
+  o += up(static_cast<size_t>(rows) * 8);
+  L.attn = o;
+  o += up(L.ap.ws_bytes);
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+spx_status spx_attn_fp8_workspace_size(const spx_dims* d, int32_t rows, int64_t max_len,
+                                       size_t* bytes) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (!bytes) return SPX_ERR_INVALID_ARG;
+  if (rows < 1 || rows > 65535 || max_len < 0) return SPX_ERR_SHAPE;
+  *bytes = fp8_layout(rows, d->heads).total;
+  return SPX_OK;
+}
+
+spx_status spx_sparse_mla_attn_fp8(const spx_dims* d, int32_t rows, const void* q,
+                                   const void* codes, const int32_t* exps, int64_t seq_stride,
+                                   int64_t cap_tok, const int32_t* idx, const int32_t* count,
+                                   const int64_t* n_vis, int64_t max_len, void* out, float* lse,
+                                   void* ws, size_t ws_bytes, spx_stream stream) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (rows < 1 || rows > 65535 || max_len < 0 || cap_tok < 1 || seq_stride < 0)
+    return SPX_ERR_SHAPE;
+  if (seq_stride != 0 && seq_stride < cap_tok * kLatent) return SPX_ERR_SHAPE;
+  if (seq_stride % kLatent != 0) return SPX_ERR_SHAPE;
+  if (!q || !codes || !exps || !idx || !count || !n_vis || !out) return SPX_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(codes) || !al4(exps) || !al16(out) || !al4(idx) || !al4(count) ||
+      (lse && !al4(lse)))
+    return SPX_ERR_INVALID_ARG;
+  const Fp8Layout L = fp8_layout(rows, d->heads);
+  if (!ws || ws_bytes < L.total || !al16(ws)) return SPX_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* cidx = reinterpret_cast<int32_t*>(base + L.cidx);
+  int32_t* ccnt = reinterpret_cast<int32_t*>(base + L.ccnt);
+  int64_t* cnvis = reinterpret_cast<int64_t*>(base + L.cnvis);
+  const int64_t len_cap = max_len < cap_tok ? max_len : cap_tok;
+  cudaError_t e = launch_gather_fp8(rows, static_cast<const uint8_t*>(codes), exps, seq_stride,
+                                    len_cap, idx, count, n_vis, base + L.dense,
+                                    static_cast<int64_t>(kFp8Dense) * kLatent, cidx, ccnt, cnvis,
+                                    s);
+  if (e != cudaSuccess) return SPX_ERR_CUDA;
+  AttnArgs a{};
+  a.q = q;
+  a.latent = base + L.dense;
+  a.seq_stride = static_cast<int64_t>(kFp8Dense) * kLatent;
+  a.cap_tok = kFp8Dense;
+  a.idx = cidx;
+  a.count = ccnt;
+  a.n_vis = cnvis;
+  a.max_len = kFp8Dense;
+  a.sm_scale = d->sm_scale;
+  a.out = out;
+  a.lse = lse;
+  a.ws = base + L.attn;
+  return cuda_status(launch_attn(L.ap, a, s));
+}
+
+// ---------------------------------------------------------------------------
 spx_status spx_decode_workspace_size(const spx_dims* d, int32_t B, int64_t max_len,
                                      size_t* bytes) {
   spx_status st = check_dims(d);

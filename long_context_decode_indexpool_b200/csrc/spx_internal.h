@@ -167,6 +167,19 @@ struct AttnArgs {
 };
 cudaError_t launch_attn(const AttnPlan& p, const AttnArgs& a, cudaStream_t stream);
 
+// FP8 (E4M3) latent cache (latent_fp8.cu): quantisation of n bf16 rows into
+// codes [n, 512] and row exponents [n]; gather of a rows' attended tokens,
+// dequantised, into a compact bf16 buffer [rows, kFp8Dense, 512] with the
+// ids, counts and lengths that describe it to launch_attn.
+constexpr int kFp8Dense = kTopK * kPool + kPool;  // 2052 rows per query
+cudaError_t launch_latent_quant_fp8(const void* lat, int64_t n, uint8_t* codes, int32_t* exps,
+                                    cudaStream_t stream);
+cudaError_t launch_gather_fp8(int rows, const uint8_t* codes, const int32_t* exps,
+                              int64_t seq_stride, int64_t len_cap, const int32_t* idx,
+                              const int32_t* count, const int64_t* n_vis, void* dense,
+                              int64_t dense_stride, int32_t* c_idx, int32_t* c_cnt,
+                              int64_t* c_nvis, cudaStream_t stream);
+
 // Self-test of the bounded waits (one CTA; see selftest.cu).  res: device
 // int64 [6].
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int64_t* res, cudaStream_t stream);
