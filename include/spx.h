@@ -332,6 +332,45 @@ SPX_API spx_status spx_sparse_mla_attn_fp8(const spx_dims* d, int32_t rows, cons
                                            spx_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * Step 4 with the latent cache in host memory and a device working set.
+ * [W3] "HiSparse는 전체 이력을 GPU 밖으로 옮긴다": the full history stays in
+ * host memory, recently used entries stay on the GPU, and a step fetches only
+ * the selected entries that are not resident.  The result is the same, bit
+ * for bit, as spx_sparse_mla_attn over the same rows in device memory.
+ *
+ * The working set of a row is a pool of nslots slots of one 4-token block
+ * (4 KiB) each, plus one slot for the partial tail block of the step.  A
+ * block selected by the step stays resident; each missing block takes the
+ * next slot, in ring order from the row's hand, that the step does not use,
+ * and is fetched from host memory (the tail tokens are fetched every call).
+ *
+ *   host_latent  bf16, pinned host memory mapped into the device's address
+ *                space (row r reads tokens host_latent + r*seq_stride + t*512)
+ *   pool         DEVICE bf16 [rows, nslots + 1, 4, 512]
+ *   nslots       >= 512 slots per row
+ *   slot_blk     DEVICE int32 [rows, nslots]       block in each slot; -1 at first
+ *   blk_slot     DEVICE int32 [rows, cap_tok / 4]  slot of each block; -1 at first
+ *   slot_stamp   DEVICE int32 [rows, nslots]       last step a slot was used; -1 at first
+ *   hand         DEVICE int32 [rows]               next slot in ring order; 0 at first
+ *   step         a value that differs from the previous call's
+ *   stats        DEVICE int64 [rows, 2]            hits and fetched blocks, accumulated
+ *   ws           spx_ws_workspace_size(d, rows, nslots) bytes
+ * Other arguments as for spx_sparse_mla_attn.  The state buffers belong to
+ * one cache: calls on it must not overlap on the GPU.
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_ws_workspace_size(const spx_dims* d, int32_t rows, int32_t nslots,
+                                         size_t* bytes);
+SPX_API spx_status spx_sparse_mla_attn_ws(const spx_dims* d, int32_t rows, const void* q,
+                                          const void* host_latent, int64_t seq_stride,
+                                          int64_t cap_tok, const int32_t* idx,
+                                          const int32_t* count, const int64_t* n_vis,
+                                          int64_t max_len, void* pool, int32_t nslots,
+                                          int32_t* slot_blk, int32_t* blk_slot,
+                                          int32_t* slot_stamp, int32_t* hand, int32_t step,
+                                          int64_t* stats, void* out, float* lse, void* ws,
+                                          size_t ws_bytes, spx_stream stream);
+
+/* ---------------------------------------------------------------------------
  * Fused decode step: steps 1-4 for one new token per sequence, in one call.
  * If raw_k is non-NULL the step first appends raw_k[b] (bf16 [B, 1, idx_dim])
  * at position len_dev[b], and the query sees n = len_dev[b] + 1 tokens;

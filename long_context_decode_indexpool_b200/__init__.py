@@ -78,6 +78,9 @@ _SIGS = {
     "spx_attn_fp8_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_sparse_mla_attn_fp8": ([_DIMS, _I32, _P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P,
                                  _SZ, _P], ctypes.c_int),
+    "spx_ws_workspace_size": ([_DIMS, _I32, _I32, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "spx_sparse_mla_attn_ws": ([_DIMS, _I32, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _I32, _P, _P,
+                                _P, _P, _I32, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "spx_decode_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_decode_fused": ([_DIMS, _I32, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _I64, _I64, _P,
                           _P, _P, _P, _P, _SZ, ctypes.POINTER(spx_timing), _P], ctypes.c_int),
@@ -274,6 +277,26 @@ def spx_sparse_mla_attn_fp8(d, rows, q, codes, exps, seq_stride, cap_tok, idx, c
                                         seq_stride, cap_tok, _ptr(idx), _ptr(count), _ptr(n_vis),
                                         max_len, _ptr(out), _ptr(lse), _ptr(ws), ws_bytes,
                                         _stream(stream)), "spx_sparse_mla_attn_fp8")
+
+
+def spx_ws_workspace_size(d, rows, nslots) -> int:
+    n = _SZ(0)
+    _check(_lib.spx_ws_workspace_size(ctypes.byref(d), rows, nslots, ctypes.byref(n)),
+           "spx_ws_workspace_size")
+    return n.value
+
+
+def spx_sparse_mla_attn_ws(d, rows, q, host_latent, seq_stride, cap_tok, idx, count, n_vis,
+                           max_len, pool, nslots, slot_blk, blk_slot, slot_stamp, hand, step,
+                           stats, out, lse=None, ws=None, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.spx_sparse_mla_attn_ws(ctypes.byref(d), rows, _ptr(q), _ptr(host_latent),
+                                       seq_stride, cap_tok, _ptr(idx), _ptr(count), _ptr(n_vis),
+                                       max_len, _ptr(pool), nslots, _ptr(slot_blk),
+                                       _ptr(blk_slot), _ptr(slot_stamp), _ptr(hand), step,
+                                       _ptr(stats), _ptr(out), _ptr(lse), _ptr(ws), ws_bytes,
+                                       _stream(stream)), "spx_sparse_mla_attn_ws")
 
 
 def spx_decode_workspace_size(d, B, max_len) -> int:

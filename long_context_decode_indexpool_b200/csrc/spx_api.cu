@@ -664,6 +664,118 @@ spx_status spx_sparse_mla_attn_fp8(const spx_dims* d, int32_t rows, const void* 
   return cuda_status(launch_attn(L.ap, a, s));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Workspace of spx_sparse_mla_attn_ws: remapped ids [rows, 512] | counts |
+// lengths | fill blocks, fill slots [rows, 512] | fill counts | attention
+struct WsLayout {
+  size_t ridx, rcnt, rnvis, fblk, fslot, fn, attn, total;
+  AttnPlan ap;
+};
+
+WsLayout ws_layout(int rows, int heads, int nslots) {
+  WsLayout L{};
+  L.ap = plan_attn(rows, heads, static_cast<int64_t>(nslots + 1) * kPool, device_sm_count());
+  size_t o = 0;
+  L.ridx = o;
+  o += up(static_cast<size_t>(rows) * kTopK * 4);
+  L.rcnt = o;
+  o += up(static_cast<size_t>(rows) * 4);
+  L.rnvis = o;
+  o += up(static_cast<size_t>(rows) * 8);
+  L.fblk = o;
+  o += up(static_cast<size_t>(rows) * kTopK * 4);
+  L.fslot = o;
+  o += up(static_cast<size_t>(rows) * kTopK * 4);
+  L.fn = o;
+  o += up(static_cast<size_t>(rows) * 4);
+  L.attn = o;
+  o += up(L.ap.ws_bytes);
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+spx_status spx_ws_workspace_size(const spx_dims* d, int32_t rows, int32_t nslots, size_t* bytes) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (!bytes) return SPX_ERR_INVALID_ARG;
+  if (rows < 1 || rows > 65535 || nslots < kTopK || nslots > (1 << 26)) return SPX_ERR_SHAPE;
+  *bytes = ws_layout(rows, d->heads, nslots).total;
+  return SPX_OK;
+}
+
+spx_status spx_sparse_mla_attn_ws(const spx_dims* d, int32_t rows, const void* q,
+                                  const void* host_latent, int64_t seq_stride, int64_t cap_tok,
+                                  const int32_t* idx, const int32_t* count, const int64_t* n_vis,
+                                  int64_t max_len, void* pool, int32_t nslots, int32_t* slot_blk,
+                                  int32_t* blk_slot, int32_t* slot_stamp, int32_t* hand,
+                                  int32_t step, int64_t* stats, void* out, float* lse, void* ws,
+                                  size_t ws_bytes, spx_stream stream) {
+  spx_status st = check_dims(d);
+  if (st != SPX_OK) return st;
+  if (rows < 1 || rows > 65535 || max_len < 0 || cap_tok < 1 || seq_stride < 0)
+    return SPX_ERR_SHAPE;
+  if (seq_stride != 0 && seq_stride < cap_tok * kLatent) return SPX_ERR_SHAPE;
+  if (nslots < kTopK || nslots > (1 << 26)) return SPX_ERR_SHAPE;
+  if (!q || !host_latent || !idx || !count || !n_vis || !pool || !slot_blk || !blk_slot ||
+      !slot_stamp || !hand || !stats || !out)
+    return SPX_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(host_latent) || !al16(pool) || !al16(out) || !al4(idx) || !al4(count) ||
+      !al4(slot_blk) || !al4(blk_slot) || !al4(slot_stamp) || !al4(hand) || (lse && !al4(lse)) ||
+      (reinterpret_cast<uintptr_t>(stats) & 7u) || (reinterpret_cast<uintptr_t>(n_vis) & 7u))
+    return SPX_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(rows, d->heads, nslots);
+  if (!ws || ws_bytes < L.total || !al16(ws)) return SPX_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  WsArgs w{};
+  w.rows = rows;
+  w.idx = idx;
+  w.count = count;
+  w.n_vis = n_vis;
+  w.len_cap = max_len < cap_tok ? max_len : cap_tok;
+  w.cap_blk = cap_tok / kPool;
+  w.nslots = nslots;
+  w.slot_blk = slot_blk;
+  w.blk_slot = blk_slot;
+  w.slot_stamp = slot_stamp;
+  w.hand = hand;
+  w.step = step;
+  w.stats = stats;
+  w.host_latent = host_latent;
+  w.seq_stride = seq_stride;
+  w.pool = pool;
+  w.r_idx = reinterpret_cast<int32_t*>(base + L.ridx);
+  w.r_cnt = reinterpret_cast<int32_t*>(base + L.rcnt);
+  w.r_nvis = reinterpret_cast<int64_t*>(base + L.rnvis);
+  w.fill_blk = reinterpret_cast<int32_t*>(base + L.fblk);
+  w.fill_slot = reinterpret_cast<int32_t*>(base + L.fslot);
+  w.fill_n = reinterpret_cast<int32_t*>(base + L.fn);
+  cudaError_t e = launch_ws_update(w, s);
+  if (e != cudaSuccess) return SPX_ERR_CUDA;
+  const int64_t pool_tok = static_cast<int64_t>(nslots + 1) * kPool;
+  AttnArgs a{};
+  a.q = q;
+  a.latent = pool;
+  a.seq_stride = pool_tok * kLatent;
+  a.cap_tok = pool_tok;
+  a.idx = w.r_idx;
+  a.count = w.r_cnt;
+  a.n_vis = w.r_nvis;
+  a.max_len = pool_tok;
+  a.sm_scale = d->sm_scale;
+  a.out = out;
+  a.lse = lse;
+  a.ws = base + L.attn;
+  return cuda_status(launch_attn(L.ap, a, s));
+}
+
 // ---------------------------------------------------------------------------
 spx_status spx_decode_workspace_size(const spx_dims* d, int32_t B, int64_t max_len,
                                      size_t* bytes) {

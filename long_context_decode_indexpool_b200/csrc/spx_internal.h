@@ -180,6 +180,35 @@ cudaError_t launch_gather_fp8(int rows, const uint8_t* codes, const int32_t* exp
                               int64_t dense_stride, int32_t* c_idx, int32_t* c_cnt,
                               int64_t* c_nvis, cudaStream_t stream);
 
+// Device working set of a host-resident latent cache (working_set.cu): the
+// per-step hit/miss pass and the fetch of the missed blocks and tail tokens
+// into the slot pool [rows, nslots + 1, 4, 512].
+struct WsArgs {
+  int rows;
+  const int32_t* idx;
+  const int32_t* count;
+  const int64_t* n_vis;
+  int64_t len_cap;  // min(max_len, cap_tok)
+  int64_t cap_blk;  // blk_slot entries per sequence
+  int nslots;
+  int32_t* slot_blk;
+  int32_t* blk_slot;
+  int32_t* slot_stamp;
+  int32_t* hand;
+  int32_t step;
+  int64_t* stats;
+  const void* host_latent;
+  int64_t seq_stride;
+  void* pool;
+  int32_t* r_idx;   // [rows, 512] ids remapped to slots
+  int32_t* r_cnt;   // [rows]
+  int64_t* r_nvis;  // [rows] nslots*4 + tail
+  int32_t* fill_blk;   // [rows, 512]
+  int32_t* fill_slot;  // [rows, 512]
+  int32_t* fill_n;     // [rows]
+};
+cudaError_t launch_ws_update(const WsArgs& a, cudaStream_t stream);
+
 // Self-test of the bounded waits (one CTA; see selftest.cu).  res: device
 // int64 [6].
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int64_t* res, cudaStream_t stream);
