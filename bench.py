@@ -685,14 +685,15 @@ def run_decode(args, world, rank, local):
 def run_e2e(st, stream, K: int, warmup: int, world: int, device):
     """K decode steps through the public call with host buffers: every step
     copies its inputs (new raw key, indexer query and weights, MLA query:
-    one packed pinned buffer, one copy) to the device, runs the fused call
+    one packed pinned buffer, one copy) to the device, runs the fused call,
     and copies the output back to pinned host memory; the host waits for
     every step's output, one step behind (it enqueues step k, then waits for
-    step k-1).  Each step is one replay of a CUDA graph captured from those
-    three operations (two graphs, alternating device and host buffers), so
-    the host's per-step cost is one graph launch.  Timed by the host clock
-    from the first copy to the last output in host memory (max over ranks).
-    Returns (ms, h2d bytes per step, d2h bytes per step, mode)."""
+    step k-1).  The copies run on a second stream into two alternating device
+    buffers, so step k+1's inputs and step k-1's output move while step k
+    computes; the fused call of each buffer pair is replayed from a captured
+    CUDA graph (eager calls if capture is unavailable).  Timed by the host
+    clock from the first copy to the last output in host memory (max over
+    ranks).  Returns (ms, h2d bytes per step, d2h bytes per step, mode)."""
     ins = (st.raw_new, st.q_idx, st.w_head, st.q)
     sizes = [t.numel() * t.element_size() for t in ins]
     offs = [0]
@@ -709,41 +710,51 @@ def run_e2e(st, stream, K: int, warmup: int, world: int, device):
     h_out = [torch.empty(st.out.shape, dtype=st.out.dtype, pin_memory=True) for _ in range(2)]
     d2h = h_out[0].numel() * h_out[0].element_size()
 
-    def body(i, s):
-        d_in[i].copy_(h_in, non_blocking=True)
+    def compute(i, s):
         raw, qi, wh, q = views[i]
         st.step(raw_new=raw, q_idx=qi, w_head=wh, q=q, out=d_out[i], stream=s.cuda_stream)
-        h_out[i].copy_(d_out[i], non_blocking=True)
 
     graphs = None
     try:
         cap = torch.cuda.Stream(device)
         cap.wait_stream(stream)
         with torch.cuda.stream(cap):
-            body(0, cap)  # (warm the library's per-device caches on this stream)
+            compute(0, cap)  # (warms the library's per-device caches on this stream)
         cap.synchronize()
         graphs = []
         for i in range(2):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap):
-                body(i, cap)
+                compute(i, cap)
             graphs.append(g)
         stream.wait_stream(cap)
     except Exception:
-        graphs = None  # capture not available: the same three operations, eagerly
-    done = [torch.cuda.Event(), torch.cuda.Event()]
+        graphs = None
+    copy = torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()
+    in_ready, used, out_home = ([ev(), ev()] for _ in range(3))
 
     def run(n):
         for k in range(n):
             i = k & 1
+            with torch.cuda.stream(copy):
+                if k >= 2:
+                    copy.wait_event(used[i])  # step k-2 has finished with d_in[i], d_out[i]
+                d_in[i].copy_(h_in, non_blocking=True)
+                in_ready[i].record(copy)
+            stream.wait_event(in_ready[i])
             if graphs is not None:
                 graphs[i].replay()
             else:
-                body(i, stream)
-            done[i].record(stream)
+                compute(i, stream)
+            used[i].record(stream)
+            with torch.cuda.stream(copy):
+                copy.wait_event(used[i])
+                h_out[i].copy_(d_out[i], non_blocking=True)
+                out_home[i].record(copy)
             if k >= 1:
-                done[i ^ 1].synchronize()  # the host has step k-1's output
-        done[(n - 1) & 1].synchronize()
+                out_home[i ^ 1].synchronize()  # the host has step k-1's output
+        out_home[(n - 1) & 1].synchronize()
 
     run(max(warmup, 2))
     barrier(world)
@@ -832,42 +843,89 @@ def run_indexshare(args, world, rank, local):
 def run_host_latent(args, world, rank, local):
     """Decode with the latent cache in pinned host memory ([W3] "HiSparse는 전체
     이력을 GPU 밖으로 옮긴다": the full history lives off the GPU and only the
-    selected rows are fetched): the attention reads the 2048 selected rows per
-    query through the host link; pooled keys stay in HBM."""
+    selected rows are fetched); pooled keys stay in HBM.  Two ways are timed:
+    (1) the fused call reading the 2048 selected rows per query straight from
+    host memory every step; (2) a device working set of --ws-slots 4-token
+    blocks per sequence (spx_sparse_mla_attn_ws), where a step fetches only
+    the selected blocks not already resident.  The indexer query cycles over
+    four different queries, so that consecutive steps select partly
+    different blocks; the hit rate is reported."""
     spx = spx_module()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = synth.workload(args.workload)
     st = DecodeState(w, device, b_offset=shard_offset(rank, w.B))
+    B, L = st.B, st.L
     host_lat = st.latent.cpu().pin_memory()
-    st.latent = None  # the device copy is released; the call reads the host rows
+    st.latent = None  # the device copy is released; the calls read the host rows
     torch.cuda.empty_cache()
     st.latent = host_lat  # step() passes its data_ptr (mapped under unified addressing)
     st._call = None
     stream = torch.cuda.current_stream(device)
-    for _ in range(args.warmup):
-        st.step()
-    torch.cuda.synchronize(device)
+    g = torch.Generator(device=device).manual_seed(99 + rank)
+    qs = [st.q_idx] + [torch.randint(-4, 5, st.q_idx.shape, generator=g, device=device)
+                       .to(torch.bfloat16) for _ in range(3)]
     K = args.steps
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize(device)
-    ev0.record(stream)
-    for _ in range(K):
-        st.step()
-    ev1.record(stream)
-    torch.cuda.synchronize(device)
-    ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
-    if spx.spx_device_error() != 0:
-        raise RuntimeError("device error during the timed region")
+
+    def timed(fn):
+        for i in range(args.warmup):
+            fn(i)
+        torch.cuda.synchronize(device)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(device)
+        ev0.record(stream)
+        for i in range(K):
+            fn(args.warmup + i)
+        ev1.record(stream)
+        torch.cuda.synchronize(device)
+        if spx.spx_device_error() != 0:
+            raise RuntimeError("device error during the timed region")
+        return max_over_ranks(ev0.elapsed_time(ev1), world, device)
+
+    # (1) zero-copy: the fused call reads the selected rows from host memory
+    ms_zc = timed(lambda i: st.step(q_idx=qs[i % 4]))
+
+    # (2) working set: pooled-key append, scores and top-k on the device, then
+    # attention through the slot pool
+    nslots = args.ws_slots
+    cap_blk = L // synth.POOL
+    pool = torch.zeros(B, nslots + 1, 4, synth.LATENT, dtype=torch.bfloat16, device=device)
+    slot_blk = torch.full((B, nslots), -1, dtype=torch.int32, device=device)
+    blk_slot = torch.full((B, cap_blk), -1, dtype=torch.int32, device=device)
+    stamp = torch.full((B, nslots), -1, dtype=torch.int32, device=device)
+    hand = torch.zeros(B, dtype=torch.int32, device=device)
+    stats = torch.zeros(B, 2, dtype=torch.int64, device=device)
+    ws = spx.workspace(spx.spx_ws_workspace_size(st.d, B, nslots), device)
+    ws_t = spx.workspace(spx.spx_topk_workspace_size(st.d, B, L), device)
+    n_vis = torch.full((B,), L, dtype=torch.int64, device=device)
+    stride = (L // synth.POOL + 3) // 4 * 4
+    scores = torch.empty(B, stride, device=device)
+
+    def ws_step(i):
+        spx.spx_pool_append(st.d, B, st.raw_new, 1, st.pool_w, st.tail, st.pooled, st.cap_blk,
+                            st.len_dev, L)
+        spx.spx_index_score(st.d, B, qs[i % 4], st.w_head, st.pooled, st.cap_blk, n_vis, L,
+                            scores, stride)
+        spx.spx_topk_blocks(st.d, B, scores, stride, n_vis, L, st.idx, st.count, ws_t)
+        spx.spx_sparse_mla_attn_ws(st.d, B, st.q, host_lat.data_ptr(), L * synth.LATENT, L, st.idx,
+                                   st.count, n_vis, L, pool, nslots, slot_blk, blk_slot, stamp,
+                                   hand, i, stats, st.out, st.lse, ws)
+
+    ms_ws = timed(ws_step)
+    hits, fetched = (int(x) for x in stats.sum(dim=0).tolist())
     if rank != 0:
         return None
     rows_bytes = st.B * (synth.TOPK_BLOCKS * synth.POOL) * synth.LATENT * 2
     return {"metric": "decode queries/s with the latent cache in pinned host memory",
-            "value": st.B * world * K / (ms * 1e-3), "unit": "queries/s", "n_gpus": world,
-            "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
-            "scaling": "weak", "dtype": "bf16", "data": "synthetic",
-            "host_rows_gbs": rows_bytes / (ms / K * 1e-3) / 1e9,
+            "value": st.B * world * K / (ms_ws * 1e-3), "unit": "queries/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms_ws / K, "higher_is_better": True,
+            "scaling": "weak", "dtype": "bf16", "data": "synthetic (indexer query cycling over 4)",
+            "working_set": {"slots_per_sequence": nslots, "tokens_per_sequence": nslots * 4,
+                            "hit_rate": hits / max(1, hits + fetched),
+                            "fetched_blocks_per_step": fetched / max(1, args.warmup + K) / st.B},
+            "zero_copy": {"ms_per_step": ms_zc / K, "queries_per_s": st.B * world * K / (ms_zc * 1e-3),
+                          "host_rows_gbs": rows_bytes / (ms_zc / K * 1e-3) / 1e9},
             "config": {"workload": w.name, "latent": "pinned host memory",
                        "batch_per_gpu": st.B, "context": st.L}}
 
@@ -1076,6 +1134,8 @@ def main(argv=None):
                     help="leave the nested prefill measurement out of the decode line")
     ap.add_argument("--host-latent", action="store_true",
                     help="decode with the latent cache in pinned host memory")
+    ap.add_argument("--ws-slots", type=int, default=8192,
+                    help="device working-set slots (4-token blocks) per sequence, --host-latent")
     ap.add_argument("--indexshare", type=int, default=0, metavar="N",
                     help="IndexShare decode: one indexer per N layers (reports per-layer rate)")
     ap.add_argument("--keys", choices=("bf16", "int8"), default="bf16",

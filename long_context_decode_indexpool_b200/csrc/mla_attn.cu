@@ -26,12 +26,10 @@
 // 16+i hands the logits of tokens 0-31 to its partner (one shuffle each), so
 // both threads work on 32 logits.
 //
-// Per tile: gather of the latent rows into the 128-byte-swizzle K-major
-// layout (double-buffered).  From device memory every selected 4-token block
-// (4 KiB, contiguous) arrives as 8 TMA tile loads of [4 tokens x 64 dims],
-// one per 128-byte swizzle region, each completing on the tile's mbarrier;
-// the <= 3 tokens of the partial tail block and any cache in host memory
-// (mapped pinned rows) come with 16-byte cp.async.  S = Q C^T as 32
+// Per tile: 16-byte cp.async gather of the latent rows into the
+// 128-byte-swizzle K-major layout by four gather warps (double-buffered; a
+// buffer is refilled as soon as the PV of its previous tile is done; the
+// cache may be device memory or mapped pinned host memory).  S = Q C^T as 32
 // tcgen05.mma (M = 64, N = 64, K = 16); softmax in registers (running max in
 // base 2, raised lazily: O is rescaled only when a tile's max exceeds it by
 // more than 8); P (bf16) to shared memory; O += P C as 8 tcgen05.mma
@@ -62,7 +60,6 @@
 // (weights 2^(m_s - M) l_s / L) into the bf16 output and the log-sum-exp.
 // No second kernel runs.
 #include <atomic>
-#include <cstring>
 
 #include "select.cuh"
 #include "spx_device.cuh"
@@ -73,10 +70,11 @@ namespace spx {
 
 namespace {
 
-constexpr int kThreads = 192;                   // 4 worker warps, MMA warp, gather warp
+constexpr int kThreads = 320;                   // 4 worker warps, MMA warp, idle warp, 4 gather warps
 constexpr int kWork = 128;                      // worker threads
 constexpr int kMmaWarp = 4;
-constexpr int kProdWarp = 5;
+constexpr int kProdWarp0 = 6;                   // gather warps 6-9
+constexpr int kProd = 128;                      // gather threads
 // named barrier (0 is __syncthreads)
 constexpr int kBarWork = 1;                     // workers only
 constexpr int kTT = 64;                         // tokens per tile
@@ -118,8 +116,6 @@ struct KParams {
   float* lse;
   __nv_bfloat16* part_o;  // [rows, groups, nsplit, 64, 512] O / l of each split (nsplit > 1)
   float* part_ml;         // [rows, groups, nsplit, 64, 2]   (m, l)
-  int lat_batched;        // TMA path: row r reads latent batch r (else batch 0 for every row)
-  int lat_evict_first;    // TMA path: rows are read once (decode), evict them from L2 first
   // fused selection (kSel): scores [rows, score_stride] (stride a multiple of
   // 4), their key histograms [rows, 2048]; the chosen ids and counts go to
   // idx_out / cnt_out (may be null)
@@ -272,10 +268,6 @@ __device__ __forceinline__ int64_t token_pos_of(const RowInfo& ri, int j, int b)
   return ri.nblk * kPool + (j - ri.cnt * kPool);
 }
 
-// kTma: full selected blocks come by TMA through map_lat (a 3-D map over
-// [batches, cap_tok, 512] bf16 with a [1, 4, 64] box and the 128-byte
-// swizzle); otherwise every row is gathered with cp.async and map_lat is
-// unused.
 // Selection phase of kSel, run by the worker threads of every CTA of the
 // row's cluster (rank = split), see above.  Leaves this CTA's list of at most
 // 512 (key << 32 | block) entries, in block order, in `mylist` and its
@@ -325,28 +317,40 @@ __device__ __forceinline__ void select_slice(const KParams& p, int r, int n_cl, 
       uint64_t* wbuf = tmp + warp * kTopK;
       const uint4* st4 = reinterpret_cast<const uint4*>(stage);
       int wn = 0;
-#pragma unroll 1
+      const uint32_t lanes_below = (1u << lane) - 1u;
+#pragma unroll 4
       for (int v0 = warp * seg; v0 < v_end; v0 += 32) {
         const int v = v0 + lane;
         const uint4 x = v < v_end ? st4[v] : make_uint4(0u, 0u, 0u, 0u);
         const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
         uint32_t kk[4];
-        int c = 0;
+        bool in[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           kk[e] = order_key(__uint_as_float(xs[e]));
-          const bool in = v < v_end && v * 4 + e < nb && kk[e] >= theta;
-          kk[e] = in ? kk[e] : 0u;
-          c += in;
+          in[e] = v < v_end && v * 4 + e < nb && kk[e] >= theta;
         }
-        const int incl = warp_incl_scan(c);
-        const int total = __shfl_sync(0xffffffffu, incl, 31);
-        int pos = wn + incl - c;
+        // most groups of 128 scores hold no candidate
+        if (!__any_sync(0xffffffffu, in[0] || in[1] || in[2] || in[3])) continue;
+        // block order is lane-major, then e: count the candidates of the
+        // lanes below with one ballot per e
+        uint32_t ball[4];
+        int below = 0, total = 0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          if (kk[e] != 0u && pos < kTopK)
-            wbuf[pos++] = (static_cast<uint64_t>(kk[e]) << 32) |
+          ball[e] = __ballot_sync(0xffffffffu, in[e]);
+          below += __popc(ball[e] & lanes_below);
+          total += __popc(ball[e]);
+        }
+        int pos = wn + below;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (in[e]) {
+            if (pos < kTopK)
+              wbuf[pos] = (static_cast<uint64_t>(kk[e]) << 32) |
                           static_cast<uint32_t>(base + v * 4 + e);
+            ++pos;
+          }
         }
         wn += total;
       }
@@ -420,9 +424,10 @@ __device__ __forceinline__ void select_slice(const KParams& p, int r, int n_cl, 
   group_sync<kWork, kBarWork>();
 }
 
-template <bool kTma, bool kSel>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_sparse_attn(const __grid_constant__ CUtensorMap map_lat, const KParams p) {
+// kSel: the block ids are chosen in the kernel from the scores (decode and
+// prefill); otherwise they come from idx / count.
+template <bool kSel>
+__global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   extern __shared__ uint8_t dyn[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -443,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int split = blockIdx.x, r = blockIdx.y, hg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool worker = tid < kWork;  // warps 0-3; warp 4 issues the MMAs, warp 5 gathers
+  const bool worker = tid < kWork;  // warps 0-3; warp 4 issues the MMAs, warps 6-9 gather
   const int h0 = hg * kHG;
   const int n_cl = p.nsplit;
   // head of this thread; lanes i and 16+i of a worker warp share it
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_qk[i], 1);
       mbar_init(&bar_pv[i], 1);
-      mbar_init(&bar_kv[i], 1);          // the gather warp, plus the tile's TMA bytes
+      mbar_init(&bar_kv[i], kProd / 32);  // one arrive per gather warp, plus any TMA bytes
       mbar_init(&bar_p[i], kWork / 32);  // one arrive per worker warp
     }
     mbar_init(bar_q, kWork / 32);
@@ -465,9 +470,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_sc, 1);
     mbar_init(bar_drain, 1);
     fence_mbar_init();
-  }
-  if constexpr (kTma) {
-    if (tid == 0) prefetch_tensormap(&map_lat);
   }
   if (warp == 0) {
     tmem_alloc(tmem_holder, 512);
@@ -616,11 +618,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem = *tmem_holder;
 
-    if (warp == kProdWarp) {
-      // ======================= gather producer (warp 5) ======================
-      // Tile t goes into buffer t & 1 as soon as PV(t-2) has released it.
-      const uint64_t lat_pol =
-          p.lat_evict_first ? l2_evict_first_policy() : l2_evict_normal_policy();
+    if (warp >= kProdWarp0) {
+      // ======================= gather warps (6-9) ============================
+      // Tile t goes into buffer t & 1 as soon as PV(t-2) has released it:
+      // 64 tokens x 64 pieces of 16 bytes, 32 cp.async per thread; token
+      // slots with nothing to load are zero-filled by the same copies.
+      const int gt = tid - kProdWarp0 * 32;  // 0 .. 127
 #pragma unroll 1
       for (int t = 0; t < ntiles; ++t) {
         if (t >= 2) {
@@ -629,57 +632,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int row0 = (t & 1) * kTT;
         const int32_t* ps = pos_s + t * kTT;
-        uint64_t* bar = &bar_kv[t & 1];
-        if constexpr (kTma) {
-          // 16 four-token groups x 8 swizzle regions; lane l takes (g, c) for
-          // l, l+32, l+64, l+96; a group is a selected block in range, by
-          // TMA, or anything else (tail tokens by cp.async, empty slots zeroed)
-          const int glane = lane & 15;
-          const bool gfull =
-              j_begin + t * kTT + 4 * glane < ri.cnt * kPool && ps[4 * glane] >= 0;
-          const uint32_t fullmask = __ballot_sync(0xffffffffu, lane < 16 && gfull);
-          if (lane == 0) mbar_expect_tx(bar, static_cast<uint32_t>(__popc(fullmask)) * 4096u);
-          __syncwarp();
-#pragma unroll 1
-          for (int u = 0; u < 4; ++u) {
-            const int id = u * 32 + lane;
-            const int g = id >> 3, c = id & 7;
-            if ((fullmask >> g) & 1u) {
-              tma_load_3d_hint(kv_s + c * kKVRegion + (row0 + 4 * g) * 128, &map_lat, bar, c * 64,
-                               ps[4 * g], p.lat_batched ? r : 0, lat_pol);
-            } else {
-#pragma unroll 1
-              for (int i = 0; i < 4; ++i) {
-                const int pos = ps[4 * g + i];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  const uint32_t dst = kv_u + kv_off(row0 + 4 * g + i, c * 8 + q);
-                  if (pos >= 0)
-                    cp_async16(dst, lat + static_cast<int64_t>(pos) * kLatent + (c * 8 + q) * 8,
-                               true);
-                  else
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u)
-                                 : "memory");
-                }
-              }
-            }
-          }
-        } else {
-#pragma unroll 4
-          for (int i = 0; i < (kTT * 64) / 32; ++i) {
-            const int c = i * 32 + lane;
-            const int tk = c >> 6, piece = c & 63;
-            const int pos = ps[tk];
-            cp_async16(kv_u + kv_off(row0 + tk, piece),
-                       lat + static_cast<int64_t>(pos >= 0 ? pos : 0) * kLatent + piece * 8,
-                       pos >= 0);
-          }
+#pragma unroll 8
+        for (int i = 0; i < (kTT * 64) / kProd; ++i) {
+          const int c = i * kProd + gt;
+          const int tk = c >> 6, piece = c & 63;
+          const int pos = ps[tk];
+          cp_async16(kv_u + kv_off(row0 + tk, piece),
+                     lat + static_cast<int64_t>(pos >= 0 ? pos : 0) * kLatent + piece * 8,
+                     pos >= 0);
         }
         cp_async_commit();
         cp_async_wait<0>();
         fence_proxy_async();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar);  // with the TMA bytes: tile t is in place
+        if (lane == 0) mbar_arrive(&bar_kv[t & 1]);  // this warp's part of tile t is in place
       }
     } else if (warp == kMmaWarp) {
       // ======================= MMA issuer (warp 4) ===========================
@@ -1030,7 +996,7 @@ int active_clusters(int n) {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int num = 0;
-  if (cudaOccupancyMaxActiveClusters(&num, k_sparse_attn<true, false>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&num, k_sparse_attn<false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     num = 0;
   }
@@ -1052,12 +1018,11 @@ int pick_cluster(int want, int64_t units) {
   return fits_at_all;
 }
 
-template <bool kTma, bool kSel>
+template <bool kSel>
 bool set_attrs_for() {
-  return cudaFuncSetAttribute(k_sparse_attn<kTma, kSel>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) ==
-             cudaSuccess &&
-         cudaFuncSetAttribute(k_sparse_attn<kTma, kSel>,
+  return cudaFuncSetAttribute(k_sparse_attn<kSel>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(k_sparse_attn<kSel>,
                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
 }
 
@@ -1066,24 +1031,11 @@ bool set_attrs() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (dev >= 0 && dev < 64 && attr_set[dev]) return true;
-  if (!set_attrs_for<true, false>() || !set_attrs_for<false, false>() ||
-      !set_attrs_for<true, true>() || !set_attrs_for<false, true>())
-    return false;
+  if (!set_attrs_for<false>() || !set_attrs_for<true>()) return false;
   if (dev >= 0 && dev < 64) attr_set[dev] = true;
   return true;
 }
 
-// Whether the latent rows can come by TMA: device memory (not mapped host
-// rows), a row stride the tensor map can express.
-bool latent_tma_ok(const void* latent, int64_t seq_stride, int64_t cap_tok) {
-  if ((seq_stride * 2) % 16 != 0 || cap_tok > (int64_t(1) << 31) - 1) return false;
-  cudaPointerAttributes at;
-  if (cudaPointerGetAttributes(&at, latent) != cudaSuccess) {
-    cudaGetLastError();
-    return false;
-  }
-  return at.type == cudaMemoryTypeDevice;
-}
 
 }  // namespace
 
@@ -1147,31 +1099,15 @@ cudaError_t launch_attn(const AttnPlan& pl0, const AttnArgs& a, cudaStream_t str
   p.ghist = a.sel_hist;
   p.idx_out = sel ? const_cast<int32_t*>(a.idx) : nullptr;
   p.cnt_out = sel ? const_cast<int32_t*>(a.count) : nullptr;
-  p.lat_batched = a.seq_stride != 0 ? 1 : 0;
-  p.lat_evict_first = a.seq_stride != 0 ? 1 : 0;  // decode rows are read once; a shared cache is reused
   if (pl.nsplit > 1) {
     const size_t units_n = static_cast<size_t>(pl.rows) * pl.groups * pl.nsplit * kHG;
     p.part_o = static_cast<__nv_bfloat16*>(a.ws);
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
                                          ((units_n * kLatent * 2 + 255) & ~static_cast<size_t>(255)));
   }
-  CUtensorMap map;
-  std::memset(&map, 0, sizeof(map));
-  bool tma = latent_tma_ok(a.latent, a.seq_stride, a.cap_tok);
-  if (tma) {
-    const uint64_t nb = a.seq_stride != 0 ? static_cast<uint64_t>(pl.rows) : 1u;
-    const uint64_t dims[3] = {static_cast<uint64_t>(kLatent), static_cast<uint64_t>(a.cap_tok), nb};
-    const uint64_t strides[2] = {kLatent * 2ull,
-                                 a.seq_stride != 0 ? static_cast<uint64_t>(a.seq_stride) * 2ull
-                                                   : static_cast<uint64_t>(a.cap_tok) * kLatent * 2ull};
-    const uint32_t box[3] = {64, kPool, 1};
-    tma = encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.latent, dims, strides, box,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
-  }
-  auto kernel = tma ? (sel ? k_sparse_attn<true, true> : k_sparse_attn<true, false>)
-                    : (sel ? k_sparse_attn<false, true> : k_sparse_attn<false, false>);
+  auto kernel = sel ? k_sparse_attn<true> : k_sparse_attn<false>;
   cudaError_t e = launch_ex(kernel, dim3(pl.nsplit, pl.rows, pl.groups), dim3(kThreads),
-                            kSmemBytes, stream, a.pdl, pl.nsplit, map, p);
+                            kSmemBytes, stream, a.pdl, pl.nsplit, p);
   count_launches(1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

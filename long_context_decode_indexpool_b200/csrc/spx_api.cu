@@ -1016,8 +1016,9 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
     return SPX_ERR_CUDA;
 
-  // top-512 per query: key histograms of the scores, then the chunked
-  // selection with the exact cut bin (as in decode)
+  // top-512 per query: key histograms of the scores, then the selection
+  // inside the attention kernel (each query's CTA scans its row of scores
+  // against the exact cut bin, as the decode clusters do)
   SelectBlocksArgs ma{};
   ma.rows = T;
   ma.scores = scores;
@@ -1034,9 +1035,11 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
   ma.out_cnt = count;
   ma.pdl = false;
   if ((e = launch_key_hist(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
-  if ((e = launch_select_blocks(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
 
   AttnArgs aa{};
+  aa.sel_scores = scores;
+  aa.sel_stride = L.stride;
+  aa.sel_hist = reinterpret_cast<const uint32_t*>(base + L.hist);
   aa.q = q;
   aa.latent = latent;
   aa.seq_stride = 0;
