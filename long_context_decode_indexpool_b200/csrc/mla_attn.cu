@@ -28,28 +28,15 @@
 //
 // Per tile: 16-byte cp.async gather of the latent rows into the
 // 128-byte-swizzle K-major layout by four gather warps (double-buffered; a
-// buffer is refilled as soon as the PV of its previous tile is done; the
-// cache may be device memory or mapped pinned host memory).  S = Q C^T as 32
+// buffer is refilled as soon as the PV of its previous tile is done, the
+// first two tiles load at once; the cache may be device memory or mapped
+// pinned host memory).  S = Q C^T as 32
 // tcgen05.mma (M = 64, N = 64, K = 16); softmax in registers (running max in
 // base 2, raised lazily: O is rescaled only when a tile's max exceeds it by
 // more than 8); P (bf16) to shared memory; O += P C as 8 tcgen05.mma
 // (M = 64, N = 256, K = 16, C read MN-major from the same tile).  While the
 // first tile's softmax runs, the tensor core already computes the second
 // tile's logits.
-//
-// Fused selection (decode, kSel): instead of reading block ids chosen by a
-// selection kernel, the CTAs of a row's cluster choose them from the row's
-// fp32 scores and the complete 2048-bin histogram of their keys that the
-// scoring kernel left.  The histogram gives the bin of the 512th-largest key
-// (every CTA finds the same one); CTA k brings its contiguous slice of the
-// row's scores into shared memory with one bulk copy, keeps the keys at or
-// above that bin's lower edge (an exact top-512 of them when more qualify,
-// ties to the lower block), and publishes the list in its shared memory.
-// After a cluster barrier every CTA reads all lists through distributed
-// shared memory (slice order = block order) and makes the final choice
-// itself; the union of the slices' exact top-512 lists holds the row's top
-// 512, so the result equals a full sort.  CTA 0 of the cluster also writes
-// the ids and the count to global memory (outputs of the fused call).
 //
 // A row with a single split writes its normalised output directly.  The n
 // splits of one (row, head group) otherwise form a thread-block cluster: each
@@ -61,7 +48,6 @@
 // No second kernel runs.
 #include <atomic>
 
-#include "select.cuh"
 #include "spx_device.cuh"
 #include "spx_internal.h"
 #include "spx_launch.cuh"
@@ -70,13 +56,12 @@ namespace spx {
 
 namespace {
 
-constexpr int kThreads = 320;                   // 4 worker warps, MMA warp, idle warp, 4 gather warps
 constexpr int kWork = 128;                      // worker threads
 constexpr int kMmaWarp = 4;
-constexpr int kProdWarp0 = 6;                   // gather warps 6-9
+constexpr int kProdWarp0 = 6;                   // gather warps 6 ..
 constexpr int kProd = 128;                      // gather threads
-// named barrier (0 is __syncthreads)
-constexpr int kBarWork = 1;                     // workers only
+// 4 worker warps, the MMA warp, an idle warp, the gather warps
+constexpr int kThreads = kProdWarp0 * 32 + kProd;
 constexpr int kTT = 64;                         // tokens per tile
 constexpr int kHG = 64;                         // heads per CTA (MMA M)
 constexpr int kRegion = 64 * 128;               // [64 rows x 128 B] = 8 KiB
@@ -116,33 +101,7 @@ struct KParams {
   float* lse;
   __nv_bfloat16* part_o;  // [rows, groups, nsplit, 64, 512] O / l of each split (nsplit > 1)
   float* part_ml;         // [rows, groups, nsplit, 64, 2]   (m, l)
-  // fused selection (kSel): scores [rows, score_stride] (stride a multiple of
-  // 4), their key histograms [rows, 2048]; the chosen ids and counts go to
-  // idx_out / cnt_out (may be null)
-  const float* scores;
-  int64_t score_stride;
-  const uint32_t* ghist;
-  int32_t* idx_out;
-  int32_t* cnt_out;
 };
-
-constexpr int kSelPass = 16384;  // scores staged in shared memory at once (64 KiB)
-
-__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local), "r"(rank));
-  return a;
-}
-__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ uint64_t ld_dsmem_u64(uint32_t addr) {
-  uint64_t v;
-  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
-  return v;
-}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
   const int n = valid ? 16 : 0;
@@ -158,13 +117,6 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ void named_arrive(int id, int n) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 // Thread-block cluster helpers.
@@ -268,165 +220,6 @@ __device__ __forceinline__ int64_t token_pos_of(const RowInfo& ri, int j, int b)
   return ri.nblk * kPool + (j - ri.cnt * kPool);
 }
 
-// Selection phase of kSel, run by the worker threads of every CTA of the
-// row's cluster (rank = split), see above.  Leaves this CTA's list of at most
-// 512 (key << 32 | block) entries, in block order, in `mylist` and its
-// length in *list_n; stage is 128 KiB of free shared memory.
-__device__ __forceinline__ void select_slice(const KParams& p, int r, int n_cl, int rank,
-                                             int64_t nblk, uint32_t theta, uint8_t* stage,
-                                             uint64_t* mylist, int* list_n, uint64_t* bar,
-                                             SelectSmem& ssm, bool& ok) {
-  const int tid = threadIdx.x;
-  const int64_t per = ((nblk + n_cl - 1) / n_cl + 3) & ~int64_t(3);  // a multiple of 4
-  const int64_t s0 = min(nblk, static_cast<int64_t>(rank) * per);
-  const int64_t s1 = min(nblk, s0 + per);
-  const float* srow = p.scores + static_cast<int64_t>(r) * p.score_stride;
-  const float* sf = reinterpret_cast<const float*>(stage);
-  // [4 x 512]: the warps' lists of a pass (fast path), or a pass's list (crowded path)
-  uint64_t* tmp = reinterpret_cast<uint64_t*>(stage + kSelPass * 4);
-  if (tid == 0) *list_n = 0;
-  int pass = 0;
-#pragma unroll 1
-  for (int64_t base = s0; base < s1; base += kSelPass, ++pass) {
-    const int nb = static_cast<int>(min(static_cast<int64_t>(kSelPass), s1 - base));
-    // rows are padded to a multiple of 4 scores: the copy may read <= 3 past s1
-    const uint32_t bytes = static_cast<uint32_t>((nb + 3) & ~3) * 4u;
-    group_sync<kWork, kBarWork>();  // the stage is free; *list_n is set
-    if (tid == 0) {
-      fence_proxy_async();  // earlier passes' reads of the stage come first
-      mbar_arrive_expect_tx(bar, bytes);
-      asm volatile(
-          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-              smem_u32(stage)),
-          "l"(srow + base), "r"(bytes), "r"(smem_u32(bar))
-          : "memory");
-    }
-    {
-      volatile int no_abort = 0;
-      ok &= mbar_wait(bar, pass & 1, &no_abort);
-    }
-    // Fast path (a handful of candidates): warp w compacts the keys at or
-    // above theta of its quarter of the pass, in block order, with coalesced
-    // 16-byte reads (lane l takes 4 consecutive scores) and a ballot scan,
-    // into its own buffer of up to 512 entries.
-    {
-      const int warp = tid >> 5, lane = tid & 31;
-      const int nvec = (nb + 3) >> 2;
-      const int seg = ((nvec + 3) / 4 + 31) & ~31;  // float4 per warp, a multiple of 32
-      const int v_end = min(nvec, (warp + 1) * seg);
-      uint64_t* wbuf = tmp + warp * kTopK;
-      const uint4* st4 = reinterpret_cast<const uint4*>(stage);
-      int wn = 0;
-      const uint32_t lanes_below = (1u << lane) - 1u;
-#pragma unroll 4
-      for (int v0 = warp * seg; v0 < v_end; v0 += 32) {
-        const int v = v0 + lane;
-        const uint4 x = v < v_end ? st4[v] : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-        uint32_t kk[4];
-        bool in[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          kk[e] = order_key(__uint_as_float(xs[e]));
-          in[e] = v < v_end && v * 4 + e < nb && kk[e] >= theta;
-        }
-        // most groups of 128 scores hold no candidate
-        if (!__any_sync(0xffffffffu, in[0] || in[1] || in[2] || in[3])) continue;
-        // block order is lane-major, then e: count the candidates of the
-        // lanes below with one ballot per e
-        uint32_t ball[4];
-        int below = 0, total = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          ball[e] = __ballot_sync(0xffffffffu, in[e]);
-          below += __popc(ball[e] & lanes_below);
-          total += __popc(ball[e]);
-        }
-        int pos = wn + below;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (in[e]) {
-            if (pos < kTopK)
-              wbuf[pos] = (static_cast<uint64_t>(kk[e]) << 32) |
-                          static_cast<uint32_t>(base + v * 4 + e);
-            ++pos;
-          }
-        }
-        wn += total;
-      }
-      if (lane == 0) ssm.hist[warp] = wn;
-      group_sync<kWork, kBarWork>();
-      int wcnt[kWork / 32], wsum = 0;
-#pragma unroll
-      for (int w = 0; w < kWork / 32; ++w) {
-        wcnt[w] = ssm.hist[w];
-        wsum += wcnt[w];
-      }
-      bool fits = *list_n + wsum <= kTopK;
-#pragma unroll
-      for (int w = 0; w < kWork / 32; ++w) fits &= wcnt[w] <= kTopK;
-      if (fits) {  // uniform: append the warps' buffers in warp (= block) order
-        int off = *list_n;
-#pragma unroll
-        for (int w = 0; w < kWork / 32; ++w) {
-          for (int j = tid; j < wcnt[w]; j += kWork) mylist[off + j] = tmp[w * kTopK + j];
-          off += wcnt[w];
-        }
-        group_sync<kWork, kBarWork>();
-        if (tid == 0) *list_n = off;
-        continue;  // next pass (the loop's barrier orders the count)
-      }
-      group_sync<kWork, kBarWork>();
-    }
-    // Crowded cut bin: exact top-512 of every 4096 scores, merged.
-#pragma unroll 1
-    for (int sub = 0; sub < nb; sub += kWork * 32) {
-      uint32_t key[32];
-      uint32_t valid = 0;
-      const int i0 = sub + tid * 32;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        key[i] = i0 + i < nb ? order_key(sf[i0 + i]) : 0u;
-        if (i0 + i < nb && key[i] >= theta) valid |= 1u << i;
-      }
-      uint32_t thr;
-      const int64_t b0 = base + i0;
-      const int n = group_select<32, kWork, kBarWork>(key, valid, kTopK, tid, ssm, &thr,
-                                                      [&](int i, int pos) {
-        tmp[pos] = (static_cast<uint64_t>(key[i]) << 32) | static_cast<uint32_t>(b0 + i);
-      });
-      group_sync<kWork, kBarWork>();
-      const int ln = *list_n;
-      if (ln + n <= kTopK) {  // uniform: append (block order is kept)
-        for (int j = tid; j < n; j += kWork) mylist[ln + j] = tmp[j];
-        group_sync<kWork, kBarWork>();
-        if (tid == 0) *list_n = ln + n;
-      } else {
-        // the exact top 512 of the list and this pass's survivors (<= 1024,
-        // list first: block order)
-        uint32_t k8[8];
-        uint64_t e8[8];
-        uint32_t v8 = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int q = tid * 8 + i;
-          e8[i] = q < ln ? mylist[q] : (q - ln < n ? tmp[q - ln] : 0ull);
-          k8[i] = static_cast<uint32_t>(e8[i] >> 32);
-          if (q < ln + n) v8 |= 1u << i;
-        }
-        const int m = group_select<8, kWork, kBarWork>(k8, v8, kTopK, tid, ssm, &thr,
-                                                       [&](int i, int pos) { mylist[pos] = e8[i]; });
-        group_sync<kWork, kBarWork>();
-        if (tid == 0) *list_n = m;
-      }
-    }
-  }
-  group_sync<kWork, kBarWork>();
-}
-
-// kSel: the block ids are chosen in the kernel from the scores (decode and
-// prefill); otherwise they come from idx / count.
-template <bool kSel>
 __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   extern __shared__ uint8_t dyn[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) &
@@ -442,9 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   uint64_t* bar_p = bar_qk + 6;    // [2]: P(t) written, t & 1
   uint64_t* bar_q = bar_qk + 8;    // Q landed
   uint64_t* bar_red = bar_qk + 9;  // combine: rows of the other splits
-  uint64_t* bar_sc = bar_qk + 10;  // kSel: staged scores landed
-  uint64_t* bar_drain = bar_qk + 11;  // every MMA of the CTA done
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 12);
+  uint64_t* bar_drain = bar_qk + 10;  // every MMA of the CTA done
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 11);
 
   const int split = blockIdx.x, r = blockIdx.y, hg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -462,12 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_qk[i], 1);
       mbar_init(&bar_pv[i], 1);
-      mbar_init(&bar_kv[i], kProd / 32);  // one arrive per gather warp, plus any TMA bytes
+      mbar_init(&bar_kv[i], kProd / 32);  // one arrive per gather warp
       mbar_init(&bar_p[i], kWork / 32);  // one arrive per worker warp
     }
     mbar_init(bar_q, kWork / 32);
     mbar_init(bar_red, 1);
-    mbar_init(bar_sc, 1);
     mbar_init(bar_drain, 1);
     fence_mbar_init();
   }
@@ -487,96 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     }
   }
   pdl_trigger();
-  pdl_wait();  // the selected blocks (or the scores) come from the previous kernel
+  pdl_wait();  // the selected blocks come from the previous kernel
   bool ok_all = true;
 
   const int32_t* idx_row = p.idx + static_cast<int64_t>(r) * kTopK;
-  int row_cnt;
-  if constexpr (kSel) {
-    __shared__ SelectSmem ssm;
-    __shared__ MergeSmem msm;
-    __shared__ int s_list_n, s_sel_n;
-    // the list of this CTA: in the tail of the position array, which this
-    // split's positions never reach while the cluster may read it
-    uint64_t* mylist = reinterpret_cast<uint64_t*>(pos_s + kPosCap - 2 * kTopK);
-    int32_t* sel_s = reinterpret_cast<int32_t*>(p_s);  // chosen ids, until P is written
-    int64_t nv = p.n_vis[r];
-    nv = nv < 0 ? 0 : (nv > p.len_cap ? p.len_cap : nv);
-    const int64_t nblk = nv / kPool;
-    const int rank = n_cl > 1 ? static_cast<int>(cluster_rank()) : 0;
-    int cut_bin = -1, above = 0;
-    if (worker) {
-      cut_bin_of<kWork, kBarWork>(p.ghist + static_cast<int64_t>(r) * kSelHistBins, kTopK, tid,
-                                  ssm, &cut_bin, &above);
-      const uint32_t theta = cut_bin < 0 ? 0u : static_cast<uint32_t>(cut_bin) << kSelKeyShift;
-      select_slice(p, r, n_cl, rank, nblk, theta, kv_s, mylist, &s_list_n, bar_sc, ssm, ok_all);
-    }
-    if (n_cl > 1) cluster_sync_all();  // every list is published
-    else __syncthreads();
-    if (worker) {
-      // the union of the lists, in rank (= block) order, into the stage
-      uint32_t* ukey = reinterpret_cast<uint32_t*>(kv_s);
-      int32_t* uid = reinterpret_cast<int32_t*>(kv_s + pad32(kMaxCluster * kTopK) * 4);
-      const uint32_t ln_local = smem_u32(&s_list_n), l_local = smem_u32(mylist);
-      int cnt_k = 0;
-      if (tid < n_cl) cnt_k = n_cl > 1 ? static_cast<int>(ld_dsmem_u32(dsmem_addr(ln_local, tid)))
-                                       : s_list_n;
-      int tot;
-      const int off_k = group_excl_scan<kWork, kBarWork>(cnt_k, tid, ssm.scan, &tot);
-      if (tid < n_cl) ssm.hist[tid] = off_k;  // (hist is free scratch here)
-      if (tid == 0) {
-        msm.kmin = 0xFFFFFFFFu;
-        msm.kmax = 0;
-      }
-      for (int b = tid; b < 3 * 128; b += kWork) (&msm.rh[0][0])[b] = 0;
-      if (tid < 3) {
-        msm.dig[tid] = 0;
-        msm.abv[tid] = 0;
-      }
-      group_sync<kWork, kBarWork>();
-      // up to 8 entries per thread per round, their loads issued back to back
-#pragma unroll 1
-      for (int f0 = 0; f0 < tot; f0 += kWork * 8) {
-        uint64_t e[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int f = f0 + u * kWork + tid;
-          e[u] = 0;
-          if (f < tot) {
-            int k = 0;
-            while (k + 1 < n_cl && ssm.hist[k + 1] <= f) ++k;
-            const int j = f - ssm.hist[k];
-            e[u] = n_cl > 1 ? ld_dsmem_u64(dsmem_addr(l_local + j * 8, k)) : mylist[j];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int f = f0 + u * kWork + tid;
-          if (f < tot) {
-            ukey[pad32(f)] = static_cast<uint32_t>(e[u] >> 32);
-            uid[pad32(f)] = static_cast<int32_t>(static_cast<uint32_t>(e[u]));
-          }
-        }
-      }
-      group_sync<kWork, kBarWork>();
-      const uint32_t theta = cut_bin < 0 ? 0u : static_cast<uint32_t>(cut_bin) << kSelKeyShift;
-      merge_final<kWork, kBarWork>(ukey, uid, tot, theta, cut_bin, above, ssm, msm, sel_s, &s_sel_n,
-                                   tid);
-      group_sync<kWork, kBarWork>();
-      if (rank == 0 && hg == 0) {
-        if (p.idx_out)
-          for (int j = tid; j < kTopK; j += kWork) p.idx_out[static_cast<int64_t>(r) * kTopK + j] = sel_s[j];
-        if (p.cnt_out && tid == 0) p.cnt_out[r] = s_sel_n;
-      }
-      // the stage held generic writes; TMA writes to it come next
-      fence_proxy_async();
-    }
-    __syncthreads();
-    idx_row = sel_s;
-    row_cnt = s_sel_n;
-  } else {
-    row_cnt = p.count[r];
-  }
+  const int row_cnt = p.count[r];
 
   // the block id of this thread's first list entry goes out with the row's
   // length and count (one round trip instead of two)
@@ -619,17 +325,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     tmem = *tmem_holder;
 
     if (warp >= kProdWarp0) {
-      // ======================= gather warps (6-9) ============================
-      // Tile t goes into buffer t & 1 as soon as PV(t-2) has released it:
-      // 64 tokens x 64 pieces of 16 bytes, 32 cp.async per thread; token
-      // slots with nothing to load are zero-filled by the same copies.
-      const int gt = tid - kProdWarp0 * 32;  // 0 .. 127
-#pragma unroll 1
-      for (int t = 0; t < ntiles; ++t) {
-        if (t >= 2) {
-          volatile int no_abort = 0;
-          ok_all &= mbar_wait(&bar_pv[t & 1], ((t - 2) >> 1) & 1, &no_abort);
-        }
+      // ======================= gather warps =================================
+      // Tile t goes into latent buffer t & 1 as soon as PV(t-2) has released
+      // it: 64 tokens x 64 pieces of 16 bytes, spread over all gather
+      // threads; token slots with nothing to load are zero-filled by the
+      // same copies.  Tiles 0 and 1 go out at once as two cp.async groups.
+      const int gt = tid - kProdWarp0 * 32;
+      auto issue_tile = [&](int t) {
         const int row0 = (t & 1) * kTT;
         const int32_t* ps = pos_s + t * kTT;
 #pragma unroll 8
@@ -642,77 +344,108 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
                      pos >= 0);
         }
         cp_async_commit();
-        cp_async_wait<0>();
+      };
+      auto publish = [&](int t) {  // this warp's part of tile t is in place
         fence_proxy_async();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_kv[t & 1]);  // this warp's part of tile t is in place
+        if (lane == 0) mbar_arrive(&bar_kv[t & 1]);
+      };
+      issue_tile(0);
+      if (ntiles > 1) {
+        issue_tile(1);
+        cp_async_wait<1>();
+        publish(0);
+        cp_async_wait<0>();
+        publish(1);
+      } else {
+        cp_async_wait<0>();
+        publish(0);
+      }
+#pragma unroll 1
+      for (int t = 2; t < ntiles; ++t) {
+        {
+          volatile int no_abort = 0;
+          ok_all &= mbar_wait(&bar_pv[t & 1], ((t - 2) >> 1) & 1, &no_abort);
+        }
+        issue_tile(t);
+        cp_async_wait<0>();
+        publish(t);
       }
     } else if (warp == kMmaWarp) {
       // ======================= MMA issuer (warp 4) ===========================
       // Issues whichever is ready first: S = Q C^T of the next tile (its data
       // landed, and the softmax of the tile that last used its S buffer is
       // done), or O += P C of the oldest tile whose P is written.  Tiles 0
-      // and 1 go as one N = 128 product (their S buffers are adjacent).
-      if (lane == 0) {
-        volatile int no_abort = 0;
-        ok_all &= mbar_wait(bar_q, 0, &no_abort);
-        const uint32_t aq = smem_u32(&bar_kv[0]), aq1 = smem_u32(&bar_kv[1]);
-        const uint32_t ap0 = smem_u32(&bar_p[0]), ap1 = smem_u32(&bar_p[1]);
-        int nq = 0, np = 0;
-        uint64_t t_last = globaltimer_ns();
-        while (np < ntiles && ok_all) {
-          const bool pair = nq == 0 && ntiles > 1;
-          bool qk_ready = false;
-          if (nq < ntiles && nq <= np + 1) {
-            qk_ready = mbar_try_wait((nq & 1) ? aq1 : aq, (nq >> 1) & 1);
-            if (qk_ready && pair) qk_ready = mbar_try_wait(aq1, 0);
-          }
-          if (qk_ready) {
-            tc_fence_after();
-            const uint32_t kvb = kv_u + (nq & 1) * kTT * 128;
-            const uint32_t d = tmem + (16u << 16) + 256 + 64 * (nq & 1);
-#pragma unroll 4
-            for (int k = 0; k < kLatent / 16; ++k) {
-              const uint32_t qoff = (k >> 2) * kRegion + (k & 3) * 32;
-              const uint32_t koff = (k >> 2) * kKVRegion + (k & 3) * 32;
-              umma_bf16(d, sdesc_kmajor_sw128(q_u + qoff), sdesc_kmajor_sw128(kvb + koff),
-                        pair ? kIdescQK2 : kIdescQK, k > 0 ? 1u : 0u);
-            }
-            umma_commit(&bar_qk[nq & 1]);
-            if (pair) umma_commit(&bar_qk[1]);
-            nq += pair ? 2 : 1;
-            t_last = globaltimer_ns();
-            continue;
-          }
-          if (np < nq && mbar_try_wait((np & 1) ? ap1 : ap0, (np >> 1) & 1)) {
-            tc_fence_after();
-            const uint32_t kvb = kv_u + (np & 1) * kTT * 128;
-            const uint32_t pb = p_u + (np & 1) * kPBytes;
-#pragma unroll
-            for (int nh = 0; nh < 2; ++nh) {
-#pragma unroll
-              for (int k = 0; k < kTT / 16; ++k) {
-                const uint64_t ad = sdesc_kmajor_sw128(pb + k * 32);
-                const uint64_t bd =
-                    sdesc_mn_sw128(kvb + nh * 4 * kKVRegion + k * 16 * 128, kKVRegion, 1024);
-                umma_bf16(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
-                          (np > 0 || k > 0) ? 1u : 0u);
-              }
-            }
-            umma_commit(&bar_pv[np & 1]);
-            ++np;
-            t_last = globaltimer_ns();
-            continue;
-          }
-          if (globaltimer_ns() - t_last > kWaitLimitNs) {
-            ok_all = false;
-            atomicExch(&g_device_error, kErrWaitTimeout);
-          }
-        }
-        // every MMA issued here completes before TMEM is read or released
-        umma_commit(bar_drain);
-        mbar_wait(bar_drain, 0, &no_abort);
+      // and 1 go as one N = 128 product (their S buffers are adjacent).  The
+      // whole warp runs the loop (lane 0 polls the barriers and broadcasts
+      // the decision), so the descriptors are warp-uniform and one elected
+      // lane issues each MMA.
+      volatile int no_abort = 0;
+      {
+        int okq = 1;
+        if (lane == 0) okq = mbar_wait(bar_q, 0, &no_abort) ? 1 : 0;
+        ok_all &= __shfl_sync(0xffffffffu, okq, 0) != 0;
       }
+      const uint32_t aq = smem_u32(&bar_kv[0]), aq1 = smem_u32(&bar_kv[1]);
+      const uint32_t ap0 = smem_u32(&bar_p[0]), ap1 = smem_u32(&bar_p[1]);
+      int nq = 0, np = 0;
+      uint64_t t_last = globaltimer_ns();
+      while (np < ntiles && ok_all) {
+        const bool pair = nq == 0 && ntiles > 1;
+        int ready = 0;  // 1: QK(nq), 2: PV(np), 3: waited too long
+        if (lane == 0) {
+          if (nq < ntiles && nq <= np + 1) {
+            bool r = mbar_try_wait((nq & 1) ? aq1 : aq, (nq >> 1) & 1);
+            if (r && pair) r = mbar_try_wait(aq1, 0);
+            if (r) ready = 1;
+          }
+          if (ready == 0 && np < nq && mbar_try_wait((np & 1) ? ap1 : ap0, (np >> 1) & 1))
+            ready = 2;
+          if (ready == 0 && globaltimer_ns() - t_last > kWaitLimitNs) ready = 3;
+        }
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        if (ready == 1) {
+          tc_fence_after();
+          const uint32_t kvb = kv_u + (nq & 1) * kTT * 128;
+          const uint32_t d = tmem + (16u << 16) + 256 + 64 * (nq & 1);
+          const uint32_t idesc = pair ? kIdescQK2 : kIdescQK;
+#pragma unroll
+          for (int k = 0; k < kLatent / 16; ++k) {
+            const uint32_t qoff = (k >> 2) * kRegion + (k & 3) * 32;
+            const uint32_t koff = (k >> 2) * kKVRegion + (k & 3) * 32;
+            umma_bf16_elect(d, sdesc_kmajor_sw128(q_u + qoff), sdesc_kmajor_sw128(kvb + koff),
+                            idesc, k > 0 ? 1u : 0u);
+          }
+          umma_commit_elect(&bar_qk[nq & 1]);
+          if (pair) umma_commit_elect(&bar_qk[1]);
+          nq += pair ? 2 : 1;
+          t_last = globaltimer_ns();
+        } else if (ready == 2) {
+          tc_fence_after();
+          const uint32_t kvb = kv_u + (np & 1) * kTT * 128;
+          const uint32_t pb = p_u + (np & 1) * kPBytes;
+#pragma unroll
+          for (int nh = 0; nh < 2; ++nh) {
+#pragma unroll
+            for (int k = 0; k < kTT / 16; ++k) {
+              const uint64_t ad = sdesc_kmajor_sw128(pb + k * 32);
+              const uint64_t bd =
+                  sdesc_mn_sw128(kvb + nh * 4 * kKVRegion + k * 16 * 128, kKVRegion, 1024);
+              umma_bf16_elect(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
+                              (np > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit_elect(&bar_pv[np & 1]);
+          ++np;
+          t_last = globaltimer_ns();
+        } else if (ready == 3) {
+          ok_all = false;
+          if (lane == 0) atomicExch(&g_device_error, kErrWaitTimeout);
+        }
+      }
+      // every MMA issued here completes before TMEM is read or released
+      umma_commit_elect(bar_drain);
+      if (lane == 0) mbar_wait(bar_drain, 0, &no_abort);
       __syncwarp();
     } else if (worker) {
       // ======================= workers (warps 0-3) ==========================
@@ -996,7 +729,7 @@ int active_clusters(int n) {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int num = 0;
-  if (cudaOccupancyMaxActiveClusters(&num, k_sparse_attn<false>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&num, k_sparse_attn, &cfg) != cudaSuccess) {
     cudaGetLastError();
     num = 0;
   }
@@ -1018,20 +751,16 @@ int pick_cluster(int want, int64_t units) {
   return fits_at_all;
 }
 
-template <bool kSel>
-bool set_attrs_for() {
-  return cudaFuncSetAttribute(k_sparse_attn<kSel>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              kSmemBytes) == cudaSuccess &&
-         cudaFuncSetAttribute(k_sparse_attn<kSel>,
-                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
-}
-
 bool set_attrs() {
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (dev >= 0 && dev < 64 && attr_set[dev]) return true;
-  if (!set_attrs_for<false>() || !set_attrs_for<true>()) return false;
+  if (cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess)
+    return false;
   if (dev >= 0 && dev < 64) attr_set[dev] = true;
   return true;
 }
@@ -1093,20 +822,13 @@ cudaError_t launch_attn(const AttnPlan& pl0, const AttnArgs& a, cudaStream_t str
   p.lse = a.lse;
   p.part_o = nullptr;
   p.part_ml = nullptr;
-  const bool sel = a.sel_scores != nullptr;
-  p.scores = a.sel_scores;
-  p.score_stride = a.sel_stride;
-  p.ghist = a.sel_hist;
-  p.idx_out = sel ? const_cast<int32_t*>(a.idx) : nullptr;
-  p.cnt_out = sel ? const_cast<int32_t*>(a.count) : nullptr;
   if (pl.nsplit > 1) {
     const size_t units_n = static_cast<size_t>(pl.rows) * pl.groups * pl.nsplit * kHG;
     p.part_o = static_cast<__nv_bfloat16*>(a.ws);
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
                                          ((units_n * kLatent * 2 + 255) & ~static_cast<size_t>(255)));
   }
-  auto kernel = sel ? k_sparse_attn<true> : k_sparse_attn<false>;
-  cudaError_t e = launch_ex(kernel, dim3(pl.nsplit, pl.rows, pl.groups), dim3(kThreads),
+  cudaError_t e = launch_ex(k_sparse_attn, dim3(pl.nsplit, pl.rows, pl.groups), dim3(kThreads),
                             kSmemBytes, stream, a.pdl, pl.nsplit, p);
   count_launches(1);
   if (e != cudaSuccess) return e;

@@ -331,41 +331,4 @@ __device__ __noinline__ void merge_final(const uint32_t* bk, const int32_t* bi, 
 }
 
 
-// The bin of the K-th largest key of a row from the row's complete
-// 2048-bin key histogram h (global memory), and the number of keys in higher
-// bins; *bin = -1 when the row has at most K keys.  Thread gtid of the NT
-// owns the 2048/NT bins counted down from 2047 - gtid*(2048/NT).
-template <int NT, int BAR>
-__device__ __forceinline__ void cut_bin_of(const uint32_t* h, int K, int gtid, SelectSmem& sm,
-                                           int* bin, int* above) {
-  constexpr int kPer = 2048 / NT;
-  static_assert(2048 % NT == 0, "bins per thread");
-  int hc[kPer], sum = 0;
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    hc[j] = static_cast<int>(__ldcg(h + 2047 - (gtid * kPer + j)));
-    sum += hc[j];
-  }
-  if (gtid == 0) {
-    sm.digit = -1;
-    sm.above = 0;
-  }
-  int tot;
-  int cum = group_excl_scan<NT, BAR>(sum, gtid, sm.scan, &tot);
-  if (tot > K) {
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      if (cum < K && K <= cum + hc[j]) {
-        sm.digit = 2047 - (gtid * kPer + j);
-        sm.above = cum;
-      }
-      cum += hc[j];
-    }
-  }
-  group_sync<NT, BAR>();
-  *bin = sm.digit;
-  *above = sm.above;
-  group_sync<NT, BAR>();
-}
-
 }  // namespace spx

@@ -886,12 +886,28 @@ spx_status decode_impl(const spx_dims* d, int32_t B, const void* raw_k, const fl
   if (timing && timing->score_end &&
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
     return SPX_ERR_CUDA;
-  // 3 + 4. top-512 blocks per row (chosen by the attention clusters from the
-  // scores and their key histograms) and attention
+  // 3. top-512 blocks per row: chunks of the scores filtered at the exact
+  // cut bin of the scoring kernel's key histogram, the last chunk's CTA
+  // making the final choice
+  SelectBlocksArgs ma{};
+  ma.rows = B;
+  ma.scores = scores;
+  ma.score_stride = L.stride;
+  ma.n_vis = n_vis;
+  ma.max_len = max_len;
+  ma.ghist = hist;
+  ma.nchunk = L.nchunk;
+  ma.list_key = reinterpret_cast<uint32_t*>(base + L.lkey);
+  ma.list_idx = reinterpret_cast<int32_t*>(base + L.lidx);
+  ma.list_cnt = reinterpret_cast<int32_t*>(base + L.lcnt);
+  ma.done = done;
+  ma.out_idx = idx;
+  ma.out_cnt = count;
+  ma.pdl = !(timing && timing->score_end);
+  if ((e = launch_select_blocks(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
+
+  // 4. attention over the selected blocks' tokens and the partial tail
   AttnArgs aa{};
-  aa.sel_scores = scores;
-  aa.sel_stride = L.stride;
-  aa.sel_hist = hist;
   aa.q = q;
   aa.latent = latent;
   aa.seq_stride = cap_tok * kLatent;
@@ -1016,9 +1032,8 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
     return SPX_ERR_CUDA;
 
-  // top-512 per query: key histograms of the scores, then the selection
-  // inside the attention kernel (each query's CTA scans its row of scores
-  // against the exact cut bin, as the decode clusters do)
+  // top-512 per query: key histograms of the scores, then the chunked
+  // selection at the exact cut bin
   SelectBlocksArgs ma{};
   ma.rows = T;
   ma.scores = scores;
@@ -1035,11 +1050,9 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
   ma.out_cnt = count;
   ma.pdl = false;
   if ((e = launch_key_hist(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
+  if ((e = launch_select_blocks(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
 
   AttnArgs aa{};
-  aa.sel_scores = scores;
-  aa.sel_stride = L.stride;
-  aa.sel_hist = reinterpret_cast<const uint32_t*>(base + L.hist);
   aa.q = q;
   aa.latent = latent;
   aa.seq_stride = 0;

@@ -150,13 +150,8 @@ struct AttnArgs {
   const void* latent;
   int64_t seq_stride;
   int64_t cap_tok;
-  // the selected blocks; with sel_scores set they are chosen by the kernel
-  // itself (decode: from the scores and their key histograms) and written here
-  const int32_t* idx;
-  const int32_t* count;
-  const float* sel_scores;  // [rows, sel_stride] (stride a multiple of 4) or NULL
-  int64_t sel_stride;
-  const uint32_t* sel_hist;  // [rows, kSelHistBins], complete
+  const int32_t* idx;    // the selected blocks [rows, 512]
+  const int32_t* count;  // [rows]
   const int64_t* n_vis;
   int64_t max_len;
   float sm_scale;

@@ -41,9 +41,8 @@ __global__ void __launch_bounds__(kWsThreads)
                 int64_t* __restrict__ r_nvis, int32_t* __restrict__ fill_blk,
                 int32_t* __restrict__ fill_slot, int32_t* __restrict__ fill_n) {
   __shared__ int scan[33];
-  __shared__ int s_miss_pos[kTopK];  // list positions of the misses, in order
   __shared__ int s_victim[kTopK];    // victim slot of each miss, in order
-  __shared__ int s_nmiss, s_found, s_hand;
+  __shared__ int s_found, s_hand;
   const int r = blockIdx.x, tid = threadIdx.x;
   int64_t n = n_vis[r];
   n = n < 0 ? 0 : (n > len_cap ? len_cap : n);
@@ -64,9 +63,7 @@ __global__ void __launch_bounds__(kWsThreads)
   const bool miss = valid && !hit;
   int nmiss;
   const int mpos = group_excl_scan<kWsThreads, 0>(miss ? 1 : 0, tid, scan, &nmiss);
-  if (miss) s_miss_pos[mpos] = j;
   if (tid == 0) {
-    s_nmiss = nmiss;
     s_found = 0;
     s_hand = hand[r];
   }
