@@ -18,21 +18,22 @@
 // sum over heads is a per-thread loop in the epilogue: no cross-thread
 // reduction at all.
 //
-// Roles (192 threads, or 320 for eight queries per group; one CTA per SM,
+// Roles (192 threads, or 576 for eight queries per group; one CTA per SM,
 // persistent over a contiguous range of (query group, key tile) work items):
 //   warp 0      TMA producer: key tiles into a kStages ring (two 16 KiB
 //               boxes of 64 dims, 128-byte swizzle), query groups into
 //               kQSlots slots.
-//   warp 1      allocates TMEM; one lane issues 8 tcgen05.mma (K = 16 each)
-//               per tile into a ring of TMEM accumulators (4 slots for one
-//               query per group, 2 for eight).
+//   warp 1      allocates TMEM; issues 8 tcgen05.mma (K = 16 each) per tile
+//               into a ring of TMEM accumulators (4 slots for one query per
+//               group, 2 for eight), the whole warp running the loop and one
+//               elected lane issuing (warp-uniform descriptors).
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator row, ReLU, weighted
 //               head sum in fp32, length mask; then either a store of the
 //               fp32 scores (and, with SELECT, a histogram of their keys).
 //               With eight queries per group (256 accumulator columns a
-//               tile) warps 2-9: the two warps of a TMEM lane quarter take
-//               four queries each and load their columns two 32-column
-//               blocks per wait, so the epilogue keeps up with the MMAs.
+//               tile) warps 2-17: the four warps of a TMEM lane quarter take
+//               two queries each, so that enough warps hide the latency of
+//               the loads and of the head sums to keep up with the MMAs.
 //
 // SELECT (decode): besides the scores, the epilogue counts the row's keys
 // (scores mapped to order-preserving 32-bit keys) in a 2048-bin shared-memory
@@ -81,7 +82,7 @@ template <int NQ, bool SELECT, bool I8>
 struct Cfg {
   static_assert(!I8 || NQ == 1, "the INT8 cache is scored one query per group");
   static constexpr int kN = 32 * NQ;
-  static constexpr int kEpiWarps = NQ == 8 ? 8 : 4;
+  static constexpr int kEpiWarps = NQ == 8 ? 16 : 4;
   static constexpr int kEpi = 32 * kEpiWarps;        // epilogue threads
   static constexpr int kThreads = 64 + kEpi;
   static constexpr int kQPerWarp = NQ * 4 / kEpiWarps;  // queries of one epilogue thread
@@ -216,15 +217,22 @@ struct WorkSrc {
       if (k >= sc.nchunk) k = -1;
       sc.ring[slot] = k;
       mbar_arrive(&sc.ring_full[slot]);
+    } else if (role == kMmaRole) {
+      // a whole warp: lane 0 waits and reads the slot, the warp follows
+      int ok = 1, kk = -1;
+      if (lane == 0) {
+        ok = mbar_wait(&sc.ring_full[slot], ph, abort) ? 1 : 0;
+        if (ok) kk = sc.ring[slot];
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      k = __shfl_sync(0xffffffffu, kk, 0);
+      if (!ok) return false;
+      if (lane == 0) mbar_arrive(&sc.ring_empty[slot]);
     } else {
       if (!mbar_wait(&sc.ring_full[slot], ph, abort)) return false;
       k = sc.ring[slot];
-      if (role == kMmaRole) {
-        mbar_arrive(&sc.ring_empty[slot]);
-      } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sc.ring_empty[slot]);
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sc.ring_empty[slot]);
     }
     if (++slot == kRing) {
       slot = 0;
@@ -436,60 +444,69 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ======================= MMA issuer ====================================
-    if (lane == 0) {
-      WorkSrc<NQ> src;
-      const Walker<NQ>& w = src.w;
-      int stage = 0, acc = 0, cur_g = -1, qs = C::kQSlots - 1;
-      uint32_t ph = 0, acc_ph = 0, qf_ph[2] = {0, 0};
-      const uint32_t a_base = smem_u32(a_smem);
-      const uint32_t q_base = smem_u32(q_smem);
-      while (src.next(p, sc, kMmaRole, lane, abort_flag)) {
-        if (w.g != cur_g) {
-          if (cur_g >= 0) umma_commit(&qempty[qs]);
-          qs = (qs + 1) % C::kQSlots;
-          if (!mbar_wait(&qfull[qs], qf_ph[qs], abort_flag)) break;
-          qf_ph[qs] ^= 1;
-          cur_g = w.g;
-        }
-        if (!mbar_wait(&accempty[acc], acc_ph ^ 1, abort_flag)) break;
-        if (!mbar_wait(&full[stage], ph, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::kN);
-        const uint32_t a0 = a_base + stage * C::kTileBytes;
-        const uint32_t b0 = q_base + qs * C::kQBytes;
-        if constexpr (I8) {
-          // K = 32 int8 per MMA: four 32-byte steps along the 128-byte rows
+    // The whole warp runs the loop (lane 0 waits on the barriers and the warp
+    // follows its result), so the descriptors are warp-uniform and one
+    // elected lane issues each MMA.
+    auto wait0 = [&](uint64_t* bar, uint32_t parity) {
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+      return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
+    WorkSrc<NQ> src;
+    const Walker<NQ>& w = src.w;
+    int stage = 0, acc = 0, cur_g = -1, qs = C::kQSlots - 1;
+    uint32_t ph = 0, acc_ph = 0, qf_ph[2] = {0, 0};
+    const uint32_t a_base = smem_u32(a_smem);
+    const uint32_t q_base = smem_u32(q_smem);
+    while (src.next(p, sc, kMmaRole, lane, abort_flag)) {
+      if (w.g != cur_g) {
+        if (cur_g >= 0) umma_commit_elect(&qempty[qs]);
+        qs = (qs + 1) % C::kQSlots;
+        if (!wait0(&qfull[qs], qf_ph[qs])) break;
+        qf_ph[qs] ^= 1;
+        cur_g = w.g;
+      }
+      if (!wait0(&accempty[acc], acc_ph ^ 1)) break;
+      if (!wait0(&full[stage], ph)) break;
+      tc_fence_after();
+      const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::kN);
+      const uint32_t a0 = a_base + stage * C::kTileBytes;
+      const uint32_t b0 = q_base + qs * C::kQBytes;
+      if constexpr (I8) {
+        // K = 32 int8 per MMA: four 32-byte steps along the 128-byte rows
 #pragma unroll
-          for (int k = 0; k < kIdxDim / 32; ++k) {
-            const uint64_t ad = sdesc_kmajor_sw128(a0 + k * 32);
-            const uint64_t bd = sdesc_kmajor_sw128(b0 + k * 32);
-            umma_s8(d, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
-          }
-        } else {
+        for (int k = 0; k < kIdxDim / 32; ++k) {
+          const uint64_t ad = sdesc_kmajor_sw128(a0 + k * 32);
+          const uint64_t bd = sdesc_kmajor_sw128(b0 + k * 32);
+          umma_s8_elect(d, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
+        }
+      } else {
 #pragma unroll
-          for (int k = 0; k < kIdxDim / 16; ++k) {
-            const uint32_t koff = (k & 3) * 32;
-            const uint64_t ad = sdesc_kmajor_sw128(a0 + (k >> 2) * kHalfBytes + koff);
-            const uint64_t bd = sdesc_kmajor_sw128(b0 + (k >> 2) * C::kQHalf + koff);
-            umma_bf16(d, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
-          }
-        }
-        umma_commit(&empty[stage]);
-        umma_commit(&accfull[acc]);
-        if (++stage == C::kStages) {
-          stage = 0;
-          ph ^= 1;
-        }
-        if (++acc == C::kAcc) {
-          acc = 0;
-          acc_ph ^= 1;
+        for (int k = 0; k < kIdxDim / 16; ++k) {
+          const uint32_t koff = (k & 3) * 32;
+          const uint64_t ad = sdesc_kmajor_sw128(a0 + (k >> 2) * kHalfBytes + koff);
+          const uint64_t bd = sdesc_kmajor_sw128(b0 + (k >> 2) * C::kQHalf + koff);
+          umma_bf16_elect(d, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
         }
       }
-      // Wait for every MMA issued by this thread before TMEM is released.
-      umma_commit(drain);
+      umma_commit_elect(&empty[stage]);
+      umma_commit_elect(&accfull[acc]);
+      if (++stage == C::kStages) {
+        stage = 0;
+        ph ^= 1;
+      }
+      if (++acc == C::kAcc) {
+        acc = 0;
+        acc_ph ^= 1;
+      }
+    }
+    // Wait for every MMA issued by this warp before TMEM is released.
+    umma_commit_elect(drain);
+    if (lane == 0) {
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
+    __syncwarp();
   } else {
     // ======================= epilogue =====================================
     const int quarter = warp & 3;  // TMEM lanes quarter*32 .. +31
@@ -575,22 +592,12 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
       };
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                             static_cast<uint32_t>(acc * C::kN);
-      if constexpr (kQ == 1) {
+#pragma unroll
+      for (int j = 0; j < kQ; ++j) {
         uint32_t v[32];
-        tmem_ld_x32_async(trow + q0 * 32, v);
+        tmem_ld_x32_async(trow + (q0 + j) * 32, v);
         tmem_ld_wait_regs<32>(v);
-        scv[0] = head_sum(v, q0);
-      } else {
-#pragma unroll 1
-        for (int j = 0; j < kQ; j += 2) {  // two 32-column loads per wait
-          uint32_t v0[32], v1[32];
-          tmem_ld_x32_async(trow + (q0 + j) * 32, v0);
-          tmem_ld_x32_async(trow + (q0 + j + 1) * 32, v1);
-          tmem_ld_wait_regs<32>(v0);
-          tmem_ld_wait_regs<32>(v1);
-          scv[j] = head_sum(v0, q0 + j);
-          scv[j + 1] = head_sum(v1, q0 + j + 1);
-        }
+        scv[j] = head_sum(v, q0 + j);
       }
       tc_fence_before();
       __syncwarp();

@@ -27,7 +27,7 @@
 // both threads work on 32 logits.
 //
 // Per tile: 16-byte cp.async gather of the latent rows into the
-// 128-byte-swizzle K-major layout by four gather warps (double-buffered; a
+// 128-byte-swizzle K-major layout by eight gather warps (double-buffered; a
 // buffer is refilled as soon as the PV of its previous tile is done, the
 // first two tiles load at once; the cache may be device memory or mapped
 // pinned host memory).  S = Q C^T as 32
@@ -59,7 +59,7 @@ namespace {
 constexpr int kWork = 128;                      // worker threads
 constexpr int kMmaWarp = 4;
 constexpr int kProdWarp0 = 6;                   // gather warps 6 ..
-constexpr int kProd = 128;                      // gather threads
+constexpr int kProd = 256;                      // gather threads (8 warps)
 // 4 worker warps, the MMA warp, an idle warp, the gather warps
 constexpr int kThreads = kProdWarp0 * 32 + kProd;
 constexpr int kTT = 64;                         // tokens per tile
@@ -394,16 +394,38 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         const bool pair = nq == 0 && ntiles > 1;
         int ready = 0;  // 1: QK(nq), 2: PV(np), 3: waited too long
         if (lane == 0) {
+          // test_wait, not try_wait: a try_wait suspended on one barrier
+          // would miss the other completing (measured: QK started up to
+          // 0.5 us after its tile landed)
           if (nq < ntiles && nq <= np + 1) {
-            bool r = mbar_try_wait((nq & 1) ? aq1 : aq, (nq >> 1) & 1);
-            if (r && pair) r = mbar_try_wait(aq1, 0);
+            bool r = mbar_test_wait((nq & 1) ? aq1 : aq, (nq >> 1) & 1);
+            if (r && pair) r = mbar_test_wait(aq1, 0);
             if (r) ready = 1;
           }
-          if (ready == 0 && np < nq && mbar_try_wait((np & 1) ? ap1 : ap0, (np >> 1) & 1))
+          if (ready == 0 && np < nq && mbar_test_wait((np & 1) ? ap1 : ap0, (np >> 1) & 1))
             ready = 2;
           if (ready == 0 && globaltimer_ns() - t_last > kWaitLimitNs) ready = 3;
         }
         ready = __shfl_sync(0xffffffffu, ready, 0);
+        // O += P C of tile np (its P written)
+        auto issue_pv = [&]() {
+          tc_fence_after();
+          const uint32_t kvb = kv_u + (np & 1) * kTT * 128;
+          const uint32_t pb = p_u + (np & 1) * kPBytes;
+#pragma unroll
+          for (int nh = 0; nh < 2; ++nh) {
+#pragma unroll
+            for (int k = 0; k < kTT / 16; ++k) {
+              const uint64_t ad = sdesc_kmajor_sw128(pb + k * 32);
+              const uint64_t bd =
+                  sdesc_mn_sw128(kvb + nh * 4 * kKVRegion + k * 16 * 128, kKVRegion, 1024);
+              umma_bf16_elect(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
+                              (np > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit_elect(&bar_pv[np & 1]);
+          ++np;
+        };
         if (ready == 1) {
           tc_fence_after();
           const uint32_t kvb = kv_u + (nq & 1) * kTT * 128;
@@ -421,22 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
           nq += pair ? 2 : 1;
           t_last = globaltimer_ns();
         } else if (ready == 2) {
-          tc_fence_after();
-          const uint32_t kvb = kv_u + (np & 1) * kTT * 128;
-          const uint32_t pb = p_u + (np & 1) * kPBytes;
-#pragma unroll
-          for (int nh = 0; nh < 2; ++nh) {
-#pragma unroll
-            for (int k = 0; k < kTT / 16; ++k) {
-              const uint64_t ad = sdesc_kmajor_sw128(pb + k * 32);
-              const uint64_t bd =
-                  sdesc_mn_sw128(kvb + nh * 4 * kKVRegion + k * 16 * 128, kKVRegion, 1024);
-              umma_bf16_elect(tmem + (static_cast<uint32_t>(16 * nh) << 16), ad, bd, kIdescPV,
-                              (np > 0 || k > 0) ? 1u : 0u);
-            }
-          }
-          umma_commit_elect(&bar_pv[np & 1]);
-          ++np;
+          issue_pv();
           t_last = globaltimer_ns();
         } else if (ready == 3) {
           ok_all = false;

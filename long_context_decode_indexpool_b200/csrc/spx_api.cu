@@ -988,8 +988,12 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  // the selection's key histograms and chunk counters start at zero
-  if (cudaMemsetAsync(base + L.hist, 0, L.lkey - L.hist, s) != cudaSuccess) return SPX_ERR_CUDA;
+  // rows short enough are selected by one CTA each (scores staged in shared
+  // memory); longer ones by key histograms and chunk lists, whose
+  // histograms and chunk counters start at zero
+  const bool rows_sel = select_rows_fits(max_len);
+  if (!rows_sel && cudaMemsetAsync(base + L.hist, 0, L.lkey - L.hist, s) != cudaSuccess)
+    return SPX_ERR_CUDA;
   int64_t* n_vis = reinterpret_cast<int64_t*>(base + L.nvis);
   float* scores = reinterpret_cast<float*>(base + L.scores);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + L.idx);
@@ -1032,8 +1036,7 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_end), s) != cudaSuccess)
     return SPX_ERR_CUDA;
 
-  // top-512 per query: key histograms of the scores, then the chunked
-  // selection at the exact cut bin
+  // top-512 per query
   SelectBlocksArgs ma{};
   ma.rows = T;
   ma.scores = scores;
@@ -1048,9 +1051,16 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
   ma.done = reinterpret_cast<int32_t*>(base + L.done);
   ma.out_idx = idx;
   ma.out_cnt = count;
-  ma.pdl = false;
-  if ((e = launch_key_hist(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
-  if ((e = launch_select_blocks(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
+  // the selection may start while scoring finishes (except across a timing
+  // event); it waits before reading the scores
+  ma.pdl = rows_sel && !(timing && timing->score_end);
+  if (rows_sel) {
+    if ((e = launch_select_rows(ma, device_sm_count(), s)) != cudaSuccess)
+      return SPX_ERR_CUDA;
+  } else {
+    if ((e = launch_key_hist(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
+    if ((e = launch_select_blocks(ma, s)) != cudaSuccess) return SPX_ERR_CUDA;
+  }
 
   AttnArgs aa{};
   aa.q = q;
@@ -1065,6 +1075,7 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
   aa.out = out;
   aa.lse = lse;
   aa.ws = base + L.attn;
+  aa.pdl = true;  // set-up overlaps the selection; the ids are read after the wait
   return cuda_status(launch_attn(L.ap, aa, s));
 }
 

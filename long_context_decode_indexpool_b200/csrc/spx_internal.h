@@ -121,6 +121,15 @@ cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream)
 // without one (prefill); uses rows, scores, score_stride, n_vis, max_len,
 // ghist, nchunk and pdl of the same arguments.
 cudaError_t launch_key_hist(const SelectBlocksArgs& a, cudaStream_t stream);
+// Prefill top-k, one CTA per row (rows of at most select_rows_fits(max_len)
+// blocks): a sampled threshold and one pass over the row's scores, then the
+// exact choice on the survivors; rows the sample misjudges are redone by a
+// second kernel with the row staged in shared memory.  Uses rows, scores,
+// score_stride, n_vis, max_len, out_idx, out_cnt, pdl, and done ([rows]
+// flags between the two kernels; no initial value needed).  Same result as
+// the two kernels above.
+bool select_rows_fits(int64_t max_len);
+cudaError_t launch_select_rows(const SelectBlocksArgs& a, int num_sms, cudaStream_t stream);
 
 // Top-k blocks.
 struct TopkPlan {

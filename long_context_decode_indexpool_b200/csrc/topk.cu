@@ -140,6 +140,9 @@ constexpr int kSelBins = kSelHistBins;
 constexpr int kSelShift = 32 - 11;
 constexpr int kMergeCap = kThreads * 16;  // candidates held at once (16 per thread)
 constexpr int kMergePer = 4;              // list entries per thread per round (long rows)
+constexpr int kSpecChunks = kThreads / 16;  // rows of at most this many chunks: one-round list load
+constexpr int kSpecPer = 4;                  // entries per thread loaded before the counts are known
+constexpr int kRowCap = 49152;               // k_select_rows: scores of a row staged at once (192 KiB)
 
 // Key histogram of scores written by another kernel (prefill): grid
 // (chunks of kSelChunk, rows); each CTA counts its chunk's keys in shared
@@ -280,13 +283,71 @@ __global__ void __launch_bounds__(kThreads)
   __threadfence();
   int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
   const int64_t slot0 = static_cast<int64_t>(r) * nchunk;
-  const int m = tid < nchunk ? __ldcg(list_cnt + slot0 + tid) : 0;
-  int mtot;
-  const int off = group_excl_scan<kThreads, 0>(m, tid, sm.scan, &mtot);
-  if (tid < nchunk) seg_off[tid] = off;
-  if (tid == 0) seg_off[nchunk] = mtot;
-  __syncthreads();
   if (tid == 0) done[r] = 0;  // ready for the next launch
+  if (nchunk <= kSpecChunks) {  // uniform
+    // One round trip for the common case: thread t reads the count of chunk
+    // t / 16 and, speculatively, entries t % 16 + 16 u (u < 4) of its list
+    // (a list slot always holds 512 entries, so the reads stay in bounds;
+    // entries past the count are ignored).
+    const int cc = tid >> 4, jj = tid & 15;
+    int cnt_c = 0;
+    uint32_t k4[kSpecPer];
+    int32_t i4[kSpecPer];
+    if (cc < nchunk) {
+      cnt_c = __ldcg(list_cnt + slot0 + cc);
+#pragma unroll
+      for (int u = 0; u < kSpecPer; ++u) {
+        const int64_t e = (slot0 + cc) * kTopK + jj + 16 * u;
+        k4[u] = __ldcg(list_key + e);
+        i4[u] = __ldcg(list_idx + e);
+      }
+    }
+    if (jj == 0 && cc < nchunk) seg_off[cc] = cnt_c;
+    __syncthreads();
+    if (tid < 32) {
+      const int x = tid < nchunk ? seg_off[tid] : 0;
+      const int xi = warp_incl_scan(x);
+      __syncwarp();
+      if (tid < nchunk) seg_off[tid] = xi - x;
+      if (tid == 31) seg_off[kThreads] = xi;  // the total
+    }
+    __syncthreads();
+    const int mtot = seg_off[kThreads];
+    if (tid == 0) seg_off[nchunk] = mtot;
+    if (mtot <= kMergeCap) {  // uniform
+      if (cc < nchunk) {
+        const int base = seg_off[cc];
+#pragma unroll
+        for (int u = 0; u < kSpecPer; ++u) {
+          const int j = jj + 16 * u;
+          if (j < cnt_c) {
+            buf_key[pad32(base + j)] = k4[u];
+            buf_idx[pad32(base + j)] = i4[u];
+          }
+        }
+        // longer lists (crowded cut bins): the rest in a second round
+#pragma unroll 1
+        for (int j = jj + 16 * kSpecPer; j < cnt_c; j += 16) {
+          const int64_t e = (slot0 + cc) * kTopK + j;
+          buf_key[pad32(base + j)] = __ldcg(list_key + e);
+          buf_idx[pad32(base + j)] = __ldcg(list_idx + e);
+        }
+      }
+      __syncthreads();
+      merge_final<kThreads, 0>(buf_key, buf_idx, mtot, theta, cut_bin, above, sm, ms, dst,
+                               out_cnt + r, tid);
+      return;
+    }
+    __syncthreads();  // (seg_off[nchunk] is read below)
+  } else {
+    const int m = tid < nchunk ? __ldcg(list_cnt + slot0 + tid) : 0;
+    int tot;
+    const int off = group_excl_scan<kThreads, 0>(m, tid, sm.scan, &tot);
+    if (tid < nchunk) seg_off[tid] = off;
+    if (tid == 0) seg_off[nchunk] = tot;
+    __syncthreads();
+  }
+  const int mtot = seg_off[nchunk];
   if (mtot <= kMergeCap) {  // uniform: every list entry into the buffer
 #pragma unroll 1
     for (int f = tid; f < mtot; f += kThreads) {
@@ -380,6 +441,418 @@ __global__ void __launch_bounds__(kThreads)
                            out_cnt + r, tid);
 }
 
+// Prefill top-k, fast path, one CTA per row.  The row comes into shared
+// memory with bulk copies (per-thread loads of a 135 KiB row were bound by
+// the misses an SM keeps in flight: 11 us a row).  2048 evenly spaced scores
+// give a threshold theta, a 22-bit key prefix above which about
+// 2.5 x 512 x 2048 / nblk of the samples lie, found by two 11-bit radix
+// passes over the samples.  Each warp then keeps the keys at or above theta
+// of a contiguous range and appends them, in block order, to a list of its
+// own (ballots place them).  If
+// at least 512 keys survive, the row's top 512 are all among them (theta is
+// at most the 512th key), and the exact choice of the selection kernels
+// (merge_final, ties to the lower block) finishes on the survivors in block
+// order.  A row whose sample misjudges it (fewer than 512 survivors, or more
+// than a warp list holds, as with thousands of tied scores) is flagged in
+// need_full[r] for k_select_rows_full; every row's flag is written.
+constexpr int kWarpCap = 256;                 // survivors per warp list
+constexpr int kCandCap = (kThreads / 32) * kWarpCap;  // 4096
+constexpr int kTargetSurvivors = 1280;        // 2.5 x 512 expected
+constexpr int kSampPer = 4;                   // samples per thread (2048 per row)
+constexpr int kFastRowCap = 36864;            // scores of a row staged by the fast path (144 KiB)
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_select_rows_fast(const float* __restrict__ scores, int64_t score_stride,
+                       const int64_t* __restrict__ n_vis, int64_t max_len,
+                       int32_t* __restrict__ out_idx, int32_t* __restrict__ out_cnt,
+                       int32_t* __restrict__ need_full) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  constexpr int kWarps = kThreads / 32;
+  uint32_t* wl_key = reinterpret_cast<uint32_t*>(dyn);           // [kWarps][kWarpCap]
+  int32_t* wl_id = reinterpret_cast<int32_t*>(wl_key + kWarps * kWarpCap);
+  uint32_t* buf_key = reinterpret_cast<uint32_t*>(wl_id + kWarps * kWarpCap);  // pad32(kCandCap)
+  int32_t* buf_idx = reinterpret_cast<int32_t*>(buf_key + pad32(kCandCap));
+  __shared__ int hist[kSelBins];
+  __shared__ SelectSmem sm;
+  __shared__ MergeSmem ms;
+  __shared__ int wcnt[kWarps + 1], woff[kWarps + 1];
+  __shared__ int s_b1, s_a1, s_b2, s_fail, s_abort;
+  __shared__ __align__(8) uint64_t s_bar;
+  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int b = tid; b < kSelBins; b += kThreads) hist[b] = 0;
+  if (tid == 0) {
+    s_fail = 0;
+    s_abort = 0;
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();  // the scores come from the scoring kernel
+  const int nblk = static_cast<int>(clamp_blocks(n_vis, r, max_len));
+  int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
+  const float* row = scores + static_cast<int64_t>(r) * score_stride;
+  if (nblk <= kTopK) {  // uniform: every visible block
+    for (int j = tid; j < kTopK; j += kThreads) dst[j] = j < nblk ? j : -1;
+    if (tid == 0) {
+      out_cnt[r] = nblk;
+      need_full[r] = 0;
+    }
+    return;
+  }
+  // The row into shared memory with bulk copies (rows are padded to a
+  // multiple of 4 scores: the copy may read <= 3 past nblk); longer rows than
+  // the stage holds go to the full kernel.
+  if (nblk > kFastRowCap) {  // uniform
+    if (tid == 0) need_full[r] = 1;
+    return;
+  }
+  const float* rs = reinterpret_cast<const float*>(buf_idx + pad32(kCandCap));
+  {
+    const uint32_t bytes = static_cast<uint32_t>((nblk + 3) & ~3) * 4u;
+    if (tid == 0) {
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(row);
+      mbar_arrive_expect_tx(&s_bar, bytes);
+      for (uint32_t off = 0; off < bytes; off += 65536u) {
+        const uint32_t n = bytes - off < 65536u ? bytes - off : 65536u;
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+            "[%3];" ::"r"(smem_u32(rs) + off),
+            "l"(src + off), "r"(n), "r"(smem_u32(&s_bar))
+            : "memory");
+      }
+    }
+    const bool landed = mbar_wait(&s_bar, 0, &s_abort);
+    if (__syncthreads_or(!landed)) {  // timed out: the error word is set
+      if (tid == 0) need_full[r] = 0;
+      return;
+    }
+  }
+  // 1. theta from 2048 evenly spaced samples (every key when the row fits the
+  //    buffer)
+  uint32_t theta = 0;
+  if (nblk > kCandCap) {  // uniform
+    uint32_t sk[kSampPer];
+#pragma unroll
+    for (int u = 0; u < kSampPer; ++u) {
+      const int i = tid + u * kThreads;
+      sk[u] = order_key(rs[static_cast<int64_t>(i) * nblk / (kSampPer * kThreads)]);
+      atomicAdd(&hist[sk[u] >> kSelShift], 1);
+    }
+    __syncthreads();
+    constexpr int kS = kSampPer * kThreads;
+    int m_t = static_cast<int>((static_cast<int64_t>(kS) * kTargetSurvivors + nblk - 1) / nblk);
+    m_t = m_t < 1 ? 1 : (m_t > kS ? kS : m_t);
+    {
+      int hc[4], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        hc[j] = hist[kSelBins - 1 - (tid * 4 + j)];
+        sum += hc[j];
+      }
+      int tot;
+      int cum = group_excl_scan<kThreads, 0>(sum, tid, sm.scan, &tot);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (cum < m_t && m_t <= cum + hc[j]) {
+          s_b1 = kSelBins - 1 - (tid * 4 + j);
+          s_a1 = cum;
+        }
+        cum += hc[j];
+      }
+    }
+    __syncthreads();
+    const uint32_t b1 = static_cast<uint32_t>(s_b1);
+    const int m2 = m_t - s_a1;
+    for (int b = tid; b < kSelBins; b += kThreads) hist[b] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kSampPer; ++u)
+      if ((sk[u] >> kSelShift) == b1) atomicAdd(&hist[(sk[u] >> 10) & (kSelBins - 1)], 1);
+    __syncthreads();
+    {
+      int hc[4], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        hc[j] = hist[kSelBins - 1 - (tid * 4 + j)];
+        sum += hc[j];
+      }
+      int tot;
+      int cum = group_excl_scan<kThreads, 0>(sum, tid, sm.scan, &tot);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (cum < m2 && m2 <= cum + hc[j]) s_b2 = kSelBins - 1 - (tid * 4 + j);
+        cum += hc[j];
+      }
+    }
+    __syncthreads();
+    theta = (b1 << kSelShift) | (static_cast<uint32_t>(s_b2) << 10);
+  }
+  // 2. each warp keeps the keys >= theta of a contiguous range, in block
+  //    order (a lane reads four consecutive scores of each 128; ballots of
+  //    the four place them)
+  {
+    const int per = ((nblk + kWarps - 1) / kWarps + 127) & ~127;  // multiple of 128
+    const int w0 = min(warp * per, nblk), w1 = min(w0 + per, nblk);
+    uint32_t* lk = wl_key + warp * kWarpCap;
+    int32_t* li = wl_id + warp * kWarpCap;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int wc = 0;
+    bool over = false;
+#pragma unroll 2
+    for (int base = w0; base < w1; base += 128) {
+      const int i = base + lane * 4;
+      const float4 v4 = i < w1 ? *reinterpret_cast<const float4*>(rs + i)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float f[4] = {v4.x, v4.y, v4.z, v4.w};
+      uint32_t k[4], bal[4];
+      bool keep[4];
+      int tot = 0, before = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        k[j] = order_key(f[j]);
+        keep[j] = i + j < w1 && k[j] >= theta;
+        bal[j] = __ballot_sync(0xffffffffu, keep[j]);
+        tot += __popc(bal[j]);
+        before += __popc(bal[j] & lt_mask);  // kept by lower lanes (they come first)
+      }
+      if (tot > 0) {  // uniform
+        if (wc + tot > kWarpCap) {
+          over = true;
+        } else {
+          int pos = wc + before;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (keep[j]) {
+              lk[pos] = k[j];
+              li[pos] = i + j;
+              ++pos;
+            }
+          }
+        }
+        wc += over ? 0 : tot;
+      }
+    }
+    if (lane == 0) {
+      wcnt[warp] = wc;
+      if (over) s_fail = 1;
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const int x = tid < kWarps ? wcnt[tid] : 0;
+    const int xi = warp_incl_scan(x);
+    if (tid < kWarps) woff[tid] = xi - x;
+    if (tid == 31) woff[kWarps] = xi;
+  }
+  __syncthreads();
+  const int c = woff[kWarps];
+  if (s_fail || c < kTopK) {  // uniform: the full kernel selects this row
+    if (tid == 0) need_full[r] = 1;
+    return;
+  }
+  if (tid == 0) need_full[r] = 0;
+  // 3. the survivors in block order, and the histogram of their keys
+  for (int b = tid; b < kSelBins; b += kThreads) hist[b] = 0;
+  for (int b = tid; b < 3 * 128; b += kThreads) (&ms.rh[0][0])[b] = 0;
+  if (tid < 3) {
+    ms.dig[tid] = 0;
+    ms.abv[tid] = 0;
+  }
+  if (tid == 0) {
+    ms.kmin = 0xFFFFFFFFu;
+    ms.kmax = 0;
+  }
+  __syncthreads();
+  {
+    const uint32_t* lk = wl_key + warp * kWarpCap;
+    const int32_t* li = wl_id + warp * kWarpCap;
+    const int n = wcnt[warp], o = woff[warp];
+    for (int e = lane; e < n; e += 32) {
+      buf_key[pad32(o + e)] = lk[e];
+      buf_idx[pad32(o + e)] = li[e];
+      atomicAdd(&hist[lk[e] >> kSelShift], 1);
+    }
+  }
+  __syncthreads();
+  int cut_bin = -1, above = 0;
+  {
+    int hc[4], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      hc[j] = hist[kSelBins - 1 - (tid * 4 + j)];
+      sum += hc[j];
+    }
+    int tot;
+    int cum = group_excl_scan<kThreads, 0>(sum, tid, sm.scan, &tot);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (cum < kTopK && kTopK <= cum + hc[j]) {
+        s_b1 = kSelBins - 1 - (tid * 4 + j);
+        s_a1 = cum;
+      }
+      cum += hc[j];
+    }
+    __syncthreads();
+    cut_bin = s_b1;
+    above = s_a1;
+  }
+  merge_final<kThreads, 0>(buf_key, buf_idx, c, theta, cut_bin, above, sm, ms, dst, out_cnt + r,
+                           tid);
+}
+
+// Prefill top-k for the rows k_select_rows_fast flagged (need_full[r] != 0;
+// cleared here), persistent over the rows.  The row's scores (at most
+// kRowCap) come into shared memory with bulk copies and turn into order keys
+// in place; an exact radix select (an 11-bit digit, then three 7-bit digits,
+// each counting the keys that share the prefix chosen so far) finds the key
+// T of the 512th-best block and how many of the blocks equal to T are taken
+// (the lowest).  An ordered compaction over contiguous per-thread ranges
+// then writes the blocks above T and those taken at T in ascending order.
+// Any distribution of scores, ties included, is handled.
+__global__ void __launch_bounds__(kThreads, 1)
+    k_select_rows_full(const float* __restrict__ scores, int64_t score_stride,
+                       const int64_t* __restrict__ n_vis, int64_t max_len, int rows,
+                       int32_t* __restrict__ out_idx, int32_t* __restrict__ out_cnt,
+                       int32_t* __restrict__ need_full) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dyn);
+  __shared__ int hist[kSelBins];
+  __shared__ int scan_s[33];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_dig, s_abv;
+  __shared__ int s_abort;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();  // the flags come from k_select_rows_fast
+  uint32_t phase = 0;
+#pragma unroll 1
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    if (need_full[r] == 0) continue;  // uniform
+    const int nblk = static_cast<int>(clamp_blocks(n_vis, r, max_len));  // > 512, <= kRowCap
+    int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
+    for (int b = tid; b < kSelBins; b += kThreads) hist[b] = 0;
+    __syncthreads();  // (also: the previous row is done with the keys)
+    // rows are padded to a multiple of 4 scores: the copy may read <= 3 past nblk
+    const uint32_t bytes = static_cast<uint32_t>((nblk + 3) & ~3) * 4u;
+    if (tid == 0) {
+      const uint8_t* src =
+          reinterpret_cast<const uint8_t*>(scores + static_cast<int64_t>(r) * score_stride);
+      mbar_arrive_expect_tx(&bar, bytes);
+      for (uint32_t off = 0; off < bytes; off += 65536u) {
+        const uint32_t n = bytes - off < 65536u ? bytes - off : 65536u;
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+            "[%3];" ::"r"(smem_u32(dyn) + off),
+            "l"(src + off), "r"(n), "r"(smem_u32(&bar))
+            : "memory");
+      }
+    }
+    const bool landed = mbar_wait(&bar, phase, &s_abort);
+    phase ^= 1;
+    if (__syncthreads_or(!landed)) return;  // timed out: the error word is set
+
+    // 1. keys in place, counted by their top 11 bits
+#pragma unroll 4
+    for (int b = tid; b < nblk; b += kThreads) {
+      const uint32_t k = order_key(__uint_as_float(keys[b]));
+      keys[b] = k;
+      atomicAdd(&hist[k >> kSelShift], 1);
+    }
+    __syncthreads();
+    int above = 0, cut = 0;
+    {
+      int hc[4], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        hc[j] = hist[kSelBins - 1 - (tid * 4 + j)];
+        sum += hc[j];
+      }
+      int tot;
+      int cum = group_excl_scan<kThreads, 0>(sum, tid, scan_s, &tot);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (cum < kTopK && kTopK <= cum + hc[j]) {
+          s_dig = kSelBins - 1 - (tid * 4 + j);
+          s_abv = cum;
+        }
+        cum += hc[j];
+      }
+      __syncthreads();
+      cut = s_dig;
+      above = s_abv;
+    }
+    // 2. three 7-bit digits of the keys in the cut bin
+    uint32_t prefix = static_cast<uint32_t>(cut) << kSelShift;
+    uint32_t pmask = ~((1u << kSelShift) - 1u);
+    int rem = kTopK - above;
+#pragma unroll 1
+    for (int d = 0; d < 3; ++d) {
+      const int shift = kSelShift - 7 * (d + 1);
+      __syncthreads();  // s_dig of the previous digit has been read
+      if (tid < 128) hist[tid] = 0;
+      __syncthreads();
+#pragma unroll 4
+      for (int b = tid; b < nblk; b += kThreads) {
+        const uint32_t k = keys[b];
+        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 127u], 1);
+      }
+      __syncthreads();
+      if (tid < 32) {
+        int c[4], lsum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          c[j] = hist[127 - (tid * 4 + j)];
+          lsum += c[j];
+        }
+        int cum = warp_incl_scan(lsum) - lsum;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (cum < rem && rem <= cum + c[j]) {
+            s_dig = 127 - (tid * 4 + j);
+            s_abv = cum;
+          }
+          cum += c[j];
+        }
+      }
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(s_dig) << shift;
+      pmask |= 127u << shift;
+      rem -= s_abv;
+    }
+    // 3. blocks above T = prefix, then the first rem equal to it, in order
+    const uint32_t T = prefix;
+    const int per = (nblk + kThreads - 1) / kThreads;
+    const int q0 = min(tid * per, nblk), q1 = min(q0 + per, nblk);
+    int cg = 0, ce = 0;
+#pragma unroll 1
+    for (int q = q0; q < q1; ++q) {
+      const uint32_t k = keys[q];
+      cg += k > T;
+      ce += k == T;
+    }
+    int tot;
+    const int ex = group_excl_scan<kThreads, 0>((cg << 16) | ce, tid, scan_s, &tot);
+    int eq_seen = ex & 0xFFFF;
+    int pos = (ex >> 16) + min(rem, eq_seen);
+#pragma unroll 1
+    for (int q = q0; q < q1; ++q) {
+      const uint32_t k = keys[q];
+      if (k > T || (k == T && eq_seen++ < rem)) dst[pos++] = q;
+    }
+    if (tid == 0) {
+      out_cnt[r] = kTopK;
+      need_full[r] = 0;
+    }
+  }
+}
+
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 template <int E>
@@ -422,6 +895,44 @@ cudaError_t launch_select_blocks(const SelectBlocksArgs& a, cudaStream_t stream)
                             stream, a.pdl, 1, a.scores, a.score_stride, a.n_vis, a.max_len,
                             a.ghist, a.nchunk, a.list_key, a.list_idx, a.list_cnt, a.done,
                             a.out_idx, a.out_cnt);
+  count_launches(1);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+bool select_rows_fits(int64_t max_len) { return max_len / kPool <= kRowCap; }
+
+cudaError_t launch_select_rows(const SelectBlocksArgs& a, int num_sms, cudaStream_t stream) {
+  if (a.rows == 0) return cudaSuccess;
+  if (!select_rows_fits(a.max_len) || (a.score_stride & 3) != 0 || !a.done)
+    return cudaErrorInvalidValue;
+  constexpr int kFastSmem =
+      2 * (kThreads / 32) * kWarpCap * 4 + 2 * pad32(kCandCap) * 4 + kFastRowCap * 4;
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool cached = dev >= 0 && dev < 64;  // devices beyond the cache: set every call
+  if (!cached || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_select_rows_fast,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kFastSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_select_rows_full, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kRowCap * 4);
+    if (e != cudaSuccess) return e;
+    if (cached) attr_set[dev] = true;
+  }
+  cudaError_t e = launch_ex(k_select_rows_fast, dim3(a.rows), dim3(kThreads), kFastSmem, stream,
+                            a.pdl, 1, a.scores, a.score_stride, a.n_vis, a.max_len, a.out_idx,
+                            a.out_cnt, a.done);
+  count_launches(1);
+  if (e != cudaSuccess) return e;
+  // the rows the fast path could not settle; shared memory for the longest
+  const int64_t nb = a.max_len / kPool;
+  const int smem = static_cast<int>(((nb + 3) & ~int64_t(3)) * 4);
+  const int grid = a.rows < num_sms ? a.rows : num_sms;
+  e = launch_ex(k_select_rows_full, dim3(grid), dim3(kThreads), smem > 0 ? smem : 16, stream,
+                true, 1, a.scores, a.score_stride, a.n_vis, a.max_len, a.rows, a.out_idx,
+                a.out_cnt, a.done);
   count_launches(1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -215,6 +215,53 @@ def test_prefill_short_context_dense():
     _check_prefill(st, list(range(64)))
 
 
+@pytest.mark.parametrize("nblk0,levels", [(40000, 4), (40000, 256), (40000, 1), (50001, 4)])
+def test_prefill_selection_heavy_ties(nblk0, levels):
+    """Prefill rows whose scores take few distinct values, so that the
+    512th-best score is shared by thousands of blocks.  40,000 cached blocks
+    go through the one-CTA-per-row selection, 50,001 (past its row limit)
+    through the key histograms and chunk lists; both must return the oracle's
+    ids (ties to the lower block) for every query of the chunk."""
+    spx = need_gpu()
+    rng = np.random.default_rng(nblk0 + levels)
+    T = 8
+    pos0 = 4 * nblk0
+    total = pos0 + T
+    cap_blk = total // 4 + 1
+    # cached pooled key b = c_b e_0; query heads all e_0 with weight 1:
+    # s_b = 32 c_b; the chunk's own tokens are zero keys (score 0)
+    c = rng.integers(0, levels, nblk0).astype(np.float32)
+    keys = np.zeros((1, cap_blk, 128), np.float32)
+    keys[0, :nblk0, 0] = c
+    pooled = torch.from_numpy(keys).to(torch.bfloat16).cuda()
+    tail = torch.zeros(1, 3, 128, dtype=torch.bfloat16, device="cuda")
+    raw = torch.zeros(T, 128, dtype=torch.bfloat16, device="cuda")
+    pool_w = np.full(4, 0.25, np.float32)
+    q_idx = torch.zeros(T, 32, 128, dtype=torch.bfloat16, device="cuda")
+    q_idx[:, :, 0] = 1.0
+    w_head = torch.ones(T, 32, device="cuda")
+    d = spx.dims(16, 1.0)
+    q = torch.zeros(T, 16, 512, dtype=torch.bfloat16, device="cuda")
+    latent = torch.zeros(total, 512, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(T, 16, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(T, 16, dtype=torch.float32, device="cuda")
+    idx = torch.empty(T, 512, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(T, dtype=torch.int32, device="cuda")
+    ws = spx.workspace(spx.spx_prefill_workspace_size(d, T, pos0), "cuda")
+    spx.spx_prefill_chunk(d, T, raw, pool_w, tail, pooled, cap_blk, pos0, q_idx, w_head, q,
+                          latent, total, out, lse, idx, cnt, ws)
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    scores = np.zeros(cap_blk, np.float64)
+    scores[:nblk0] = 32.0 * c
+    for t in range(T):
+        nb = (pos0 + t + 1) // 4
+        ref = oracle.topk(scores[:nb], 512)
+        assert cnt[t] == ref.size and np.array_equal(idx[t, :cnt[t]], ref), f"query {t}"
+        assert (idx[t, cnt[t]:] == -1).all()
+
+
 @pytest.mark.slow
 def test_prefill_full_chunk_all_ids_stratified_attention():
     """The benchmark's prefill workload (4096 new tokens on a 131,072-token
