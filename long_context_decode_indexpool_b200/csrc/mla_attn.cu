@@ -21,13 +21,16 @@
 //   O dims   0-255: lanes 32w+i,    columns 0-255
 //   O dims 256-511: lanes 32w+16+i, columns 0-255
 //   S (64 tokens):  lanes 32w+16+i, columns 256+64b .. (b = S buffer 0/1)
-// The two threads of warp w that own TMEM lanes i and 16+i share head 16w+i:
-// each holds half of its output row, and for the softmax the thread of lane
-// 16+i hands the logits of tokens 0-31 to its partner (one shuffle each), so
-// both threads work on 32 logits.
+// Worker warps w and w+4 (w < 4) both reach lanes 32w .. 32w+31.  Warp w
+// takes tokens 0-31 of each tile and columns 0-127 of O, warp w+4 tokens
+// 32-63 and columns 128-255.  In each, the two threads of TMEM lanes i and
+// 16+i share head 16w+i: the thread of lane 16+i hands the logits of the
+// first 16 tokens to its partner (one shuffle each), so a thread works on 16
+// logits; the two warps exchange their tile maxima per head through shared
+// memory (a barrier of the pair) and keep partial row sums.
 //
 // Per tile: 16-byte cp.async gather of the latent rows into the
-// 128-byte-swizzle K-major layout by eight gather warps (double-buffered; a
+// 128-byte-swizzle K-major layout by seven gather warps (double-buffered; a
 // buffer is refilled as soon as the PV of its previous tile is done, the
 // first two tiles load at once; the cache may be device memory or mapped
 // pinned host memory).  S = Q C^T as 32
@@ -56,11 +59,13 @@ namespace spx {
 
 namespace {
 
-constexpr int kWork = 128;                      // worker threads
-constexpr int kMmaWarp = 4;
-constexpr int kProdWarp0 = 6;                   // gather warps 6 ..
-constexpr int kProd = 256;                      // gather threads (8 warps)
-// 4 worker warps, the MMA warp, an idle warp, the gather warps
+constexpr int kWork = 256;                      // worker threads (warps 0-7)
+constexpr int kMmaWarp = 8;
+constexpr int kProdWarp0 = 9;                   // gather warps 9 ..
+// gather threads (7 warps): 16 warps in all leave 128 registers a thread
+// (registers are granted in groups of 4 warps: 17 warps would get 96)
+constexpr int kProd = 224;
+// 8 worker warps, the MMA warp, the gather warps
 constexpr int kThreads = kProdWarp0 * 32 + kProd;
 constexpr int kTT = 64;                         // tokens per tile
 constexpr int kHG = 64;                         // heads per CTA (MMA M)
@@ -117,6 +122,11 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Barrier of the two worker warps that share TMEM lane quarter qd (ids 1-4).
+__device__ __forceinline__ void pair_sync(int qd) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + qd) : "memory");
 }
 
 // Thread-block cluster helpers.
@@ -237,15 +247,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   uint64_t* bar_red = bar_qk + 9;  // combine: rows of the other splits
   uint64_t* bar_drain = bar_qk + 10;  // every MMA of the CTA done
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_qk + 11);
+  __shared__ float red_m[2][2][kHG];  // [tile parity][token half][head]: tile maxima
+  __shared__ float red_l[2][kHG];     // [token half][head]: row sums
 
   const int split = blockIdx.x, r = blockIdx.y, hg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool worker = tid < kWork;  // warps 0-3; warp 4 issues the MMAs, warps 6-9 gather
+  const bool worker = tid < kWork;  // warps 0-7; warp 8 issues the MMAs, warps 9-15 gather
   const int h0 = hg * kHG;
   const int n_cl = p.nsplit;
   // head of this thread; lanes i and 16+i of a worker warp share it
   const int hloc = (warp & 3) * 16 + (lane & 15);
-  const int half = lane >> 4;  // 0: tokens 0-31 / dims 0-255, 1: tokens 32-63 / dims 256-511
+  const int half = lane >> 4;  // 0: dims 0-255, 1: dims 256-511 (and a token sub-half)
+  const int qd = warp & 3;      // workers: TMEM lane quarter
+  const int th = (warp >> 2) & 1;  // workers: half of a tile's tokens, of O's columns
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const uint32_t q_u = smem_u32(q_s), kv_u = smem_u32(kv_s), p_u = smem_u32(p_s);
 
@@ -335,13 +349,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         const int row0 = (t & 1) * kTT;
         const int32_t* ps = pos_s + t * kTT;
 #pragma unroll 8
-        for (int i = 0; i < (kTT * 64) / kProd; ++i) {
+        for (int i = 0; i < (kTT * 64 + kProd - 1) / kProd; ++i) {
           const int c = i * kProd + gt;
-          const int tk = c >> 6, piece = c & 63;
-          const int pos = ps[tk];
-          cp_async16(kv_u + kv_off(row0 + tk, piece),
-                     lat + static_cast<int64_t>(pos >= 0 ? pos : 0) * kLatent + piece * 8,
-                     pos >= 0);
+          if (c < kTT * 64) {
+            const int tk = c >> 6, piece = c & 63;
+            const int pos = ps[tk];
+            cp_async16(kv_u + kv_off(row0 + tk, piece),
+                       lat + static_cast<int64_t>(pos >= 0 ? pos : 0) * kLatent + piece * 8,
+                       pos >= 0);
+          }
         }
         cp_async_commit();
       };
@@ -372,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         publish(t);
       }
     } else if (warp == kMmaWarp) {
-      // ======================= MMA issuer (warp 4) ===========================
+      // ======================= MMA issuer (warp 8) ===========================
       // Issues whichever is ready first: S = Q C^T of the next tile (its data
       // landed, and the softmax of the tile that last used its S buffer is
       // done), or O += P C of the oldest tile whose P is written.  Tiles 0
@@ -455,7 +471,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       if (lane == 0) mbar_wait(bar_drain, 0, &no_abort);
       __syncwarp();
     } else if (worker) {
-      // ======================= workers (warps 0-3) ==========================
+      // ======================= workers (warps 0-7) ==========================
+      // Warps w and w + 4 share TMEM lane quarter w & 3 (heads 16(w&3) ..
+      // +15): warp w takes tokens 0-31 of each tile, warp w + 4 tokens 32-63,
+      // so a thread works on 16 logits.  The tile's maximum per head is
+      // exchanged between the two through shared memory, so both raise the
+      // running maximum alike; each keeps a partial row sum.
 #pragma unroll 1
       for (int j = 0; j < ntiles; ++j) {
         const int buf = j & 1;
@@ -465,32 +486,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         }
         tc_fence_after();
 
-        // ---- softmax: 32 logits of head hloc per thread --------------------
-        float s[32];
+        // ---- softmax: 16 logits of head hloc per thread --------------------
+        float s[16];
         {
-          // lanes 16-31 receive the 64 logits of their head; tokens 0-31 go
-          // to the partner lane (lanes 0-15 receive unused columns)
-          uint32_t a[32], b[32];
-          tmem_ld_x32_async(tmem + lane_base + 256 + 64 * buf, a);
-          tmem_ld_x32_async(tmem + lane_base + 256 + 64 * buf + 32, b);
+          // lanes 16-31 receive the 32 logits of their head in this warp's
+          // half of the tile; tokens 0-15 of it go to the partner lane
+          uint32_t a[32];
+          tmem_ld_x32_async(tmem + lane_base + 256 + 64 * buf + 32 * th, a);
           tmem_ld_wait_regs<32>(a);
-          tmem_ld_wait_regs<32>(b);
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
+          for (int t = 0; t < 16; ++t) {
             const uint32_t x = __shfl_xor_sync(0xffffffffu, a[t], 16);
-            s[t] = __uint_as_float(half ? b[t] : x);
+            s[t] = __uint_as_float(half ? a[16 + t] : x);
           }
         }
-        const uint32_t vm = vm_s[j * 2 + half];
-        float mx[8];
+        const uint32_t vm = (vm_s[j * 2 + th] >> (16 * half)) & 0xFFFFu;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) s[t] = ((vm >> t) & 1u) ? s[t] * p.scale_log2 : -INFINITY;
+        for (int t = 0; t < 16; ++t) s[t] = ((vm >> t) & 1u) ? s[t] * p.scale_log2 : -INFINITY;
+        float mx[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < 4; ++u)
           mx[u] = fmaxf(fmaxf(s[4 * u], s[4 * u + 1]), fmaxf(s[4 * u + 2], s[4 * u + 3]));
-        float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+        // the other half of the tile (double-buffered by tile parity: a slot
+        // is rewritten only after the partner passed the next exchange)
+        if (half == 0) red_m[buf][th][hloc] = mt;
+        pair_sync(qd);
+        mt = fmaxf(mt, red_m[buf][th ^ 1][hloc]);
         float alpha = 1.f;
         if (m_run == -INFINITY) {
           m_run = mt;
@@ -500,14 +523,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         }
         if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
           // O holds tiles up to j-1: let PV(j-1) finish, then each thread
-          // scales its half of the O row of its head
+          // scales its half of the O row of its head, this warp's columns
           {
             volatile int no_abort = 0;
             ok_all &= mbar_wait(&bar_pv[(j - 1) & 1], ((j - 1) >> 1) & 1, &no_abort);
           }
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < 256; c += 32) {
+          for (int c = 128 * th; c < 128 * th + 128; c += 32) {
             float v[32];
             tmem_ld_32x32b_x32(tmem + lane_base + c, v);
 #pragma unroll
@@ -515,10 +538,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
             tmem_st_32x32b_x32(tmem + lane_base + c, v);
           }
         }
-        uint32_t packed[16];
-        float ps[8];
+        uint32_t packed[8];
+        float ps[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 4; ++u) {
           float e[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -529,19 +552,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
           packed[2 * u + 1] = *reinterpret_cast<const uint32_t*>(&b);
           ps[u] = (__low2float(a) + __high2float(a)) + (__low2float(b) + __high2float(b));
         }
-        float lsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        float lsum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
-        l_run = l_run * alpha + lsum;
+        l_run = l_run * alpha + lsum;  // this warp's half of the tokens
         // P buffer j & 1 is free once PV(j-2) is done
         if (j >= 2) {
           volatile int no_abort = 0;
           ok_all &= mbar_wait(&bar_pv[buf], ((j - 2) >> 1) & 1, &no_abort);
         }
-        // row hloc of P, pieces 4*half .. 4*half+3 (16 B each)
+        // row hloc of P, pieces 4 th + 2 half .. +1 (16 B each)
         const uint32_t pb = p_u + buf * kPBytes;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int piece = 4 * half + c;
+        for (int c = 0; c < 2; ++c) {
+          const int piece = 4 * th + 2 * half + c;
           const uint32_t a = pb + hloc * 128 + ((piece ^ (hloc & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(packed[4 * c]),
                        "r"(packed[4 * c + 1]), "r"(packed[4 * c + 2]), "r"(packed[4 * c + 3])
@@ -557,6 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         ok_all &= mbar_wait(&bar_pv[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, &no_abort);
       }
       tc_fence_after();
+      // the row sum over both halves of the tokens
+      if (half == 0) red_l[th][hloc] = l_run;
+      pair_sync(qd);
+      l_run += red_l[th ^ 1][hloc];
     }
     __syncwarp();
   }
@@ -573,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
   if (ntiles > 0 && worker) {
     const float inv = have ? 1.f / l_run : 0.f;
 #pragma unroll 1
-    for (int c0 = 0; c0 < 256; c0 += 32) {
+    for (int c0 = 128 * th; c0 < 128 * th + 128; c0 += 32) {
       float v[32];
       tmem_ld_32x32b_x32(tmem + lane_base + c0, v);
 #pragma unroll
@@ -591,20 +618,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       }
     }
     if (n_cl > 1) {
-      // this warp's 16 rows (16 KiB, contiguous) go to L2 at once, while the
-      // other warps are still staging theirs
+      // this quarter's 16 rows (16 KiB, contiguous) go to L2 at once, while
+      // the other quarters are still staging theirs
       const int64_t first_row = (unit * n_cl + split) * kHG;
       fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) {
-        bulk_store(p.part_o + (first_row + warp * 16) * kLatent, stage_u + warp * 16 * 1024,
+      pair_sync(qd);  // both warps' columns are staged
+      if (th == 0 && lane == 0) {
+        bulk_store(p.part_o + (first_row + qd * 16) * kLatent, stage_u + qd * 16 * 1024,
                    16 * kLatent * 2);
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       }
     }
   }
   if (n_cl == 1) {
-    if (worker && half == 0 && h0 + hloc < p.heads && p.lse)
+    if (worker && half == 0 && th == 0 && h0 + hloc < p.heads && p.lse)
       p.lse[static_cast<int64_t>(r) * p.heads + h0 + hloc] =
           have ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
     __syncthreads();
@@ -627,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
       asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // this warp's rows are in L2
       asm volatile("fence.proxy.async.global;" ::: "memory");
     }
-    if (worker && half == 0) {
+    if (worker && half == 0 && th == 0) {
       float* pm = p.part_ml + (first_row + hloc) * 2;
       pm[0] = have ? m_run : -INFINITY;
       pm[1] = have ? l_run : 0.f;

@@ -215,13 +215,17 @@ def test_prefill_short_context_dense():
     _check_prefill(st, list(range(64)))
 
 
-@pytest.mark.parametrize("nblk0,levels", [(40000, 4), (40000, 256), (40000, 1), (50001, 4)])
+@pytest.mark.parametrize("nblk0,levels", [(30000, 4), (30000, 256), (30000, 1), (40000, 256),
+                                          (50001, 4)])
 def test_prefill_selection_heavy_ties(nblk0, levels):
     """Prefill rows whose scores take few distinct values, so that the
-    512th-best score is shared by thousands of blocks.  40,000 cached blocks
-    go through the one-CTA-per-row selection, 50,001 (past its row limit)
-    through the key histograms and chunk lists; both must return the oracle's
-    ids (ties to the lower block) for every query of the chunk."""
+    512th-best score is shared by thousands of blocks.  30,000 cached blocks
+    go through the sampled one-CTA-per-row selection (4 and 1 levels overflow
+    its survivor lists and fall back to the staged radix kernel, 256 levels
+    do not), 40,000 (past the sampled path's stage) straight to the staged
+    kernel, 50,001 (past that) through the key histograms and chunk lists;
+    every path must return the oracle's ids (ties to the lower block) for
+    every query of the chunk."""
     spx = need_gpu()
     rng = np.random.default_rng(nblk0 + levels)
     T = 8
