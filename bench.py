@@ -688,10 +688,11 @@ def run_e2e(st, stream, K: int, warmup: int, world: int, device):
     one packed pinned buffer, one copy) to the device, runs the fused call,
     and copies the output back to pinned host memory; the host waits for
     every step's output, one step behind (it enqueues step k, then waits for
-    step k-1).  The copies run on a second stream into two alternating device
-    buffers, so step k+1's inputs and step k-1's output move while step k
-    computes; the fused call of each buffer pair is replayed from a captured
-    CUDA graph (eager calls if capture is unavailable).  Timed by the host
+    step k-1).  The copies run on two more streams, one per direction, into
+    two alternating device buffers, so step k+1's inputs and step k-1's output
+    move while step k computes; the fused call of each buffer pair is replayed
+    from a captured CUDA graph (eager calls if capture is unavailable).
+    Timed by the host
     clock from the first copy to the last output in host memory (max over
     ranks).  Returns (ms, h2d bytes per step, d2h bytes per step, mode)."""
     ins = (st.raw_new, st.q_idx, st.w_head, st.q)
@@ -730,28 +731,32 @@ def run_e2e(st, stream, K: int, warmup: int, world: int, device):
         stream.wait_stream(cap)
     except Exception:
         graphs = None
-    copy = torch.cuda.Stream(device)
+    # one stream per direction: an input copy must not queue behind the
+    # previous step's output copy, which waits for that step's compute
+    h2d, d2h_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
     ev = lambda: torch.cuda.Event()
     in_ready, used, out_home = ([ev(), ev()] for _ in range(3))
 
     def run(n):
         for k in range(n):
             i = k & 1
-            with torch.cuda.stream(copy):
+            with torch.cuda.stream(h2d):
                 if k >= 2:
-                    copy.wait_event(used[i])  # step k-2 has finished with d_in[i], d_out[i]
+                    h2d.wait_event(used[i])  # step k-2 has finished with d_in[i]
                 d_in[i].copy_(h_in, non_blocking=True)
-                in_ready[i].record(copy)
+                in_ready[i].record(h2d)
             stream.wait_event(in_ready[i])
+            if k >= 2:
+                stream.wait_event(out_home[i])  # step k-2's output has left d_out[i]
             if graphs is not None:
                 graphs[i].replay()
             else:
                 compute(i, stream)
             used[i].record(stream)
-            with torch.cuda.stream(copy):
-                copy.wait_event(used[i])
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(used[i])
                 h_out[i].copy_(d_out[i], non_blocking=True)
-                out_home[i].record(copy)
+                out_home[i].record(d2h_s)
             if k >= 1:
                 out_home[i ^ 1].synchronize()  # the host has step k-1's output
         out_home[(n - 1) & 1].synchronize()
