@@ -18,7 +18,7 @@
 // sum over heads is a per-thread loop in the epilogue: no cross-thread
 // reduction at all.
 //
-// Roles (192 threads, or 576 for eight queries per group; one CTA per SM,
+// Roles (320 threads, or 576 for eight queries per group; one CTA per SM,
 // persistent over a contiguous range of (query group, key tile) work items):
 //   warp 0      TMA producer: key tiles into a kStages ring (two 16 KiB
 //               boxes of 64 dims, 128-byte swizzle), query groups into
@@ -27,9 +27,11 @@
 //               into a ring of TMEM accumulators (4 slots for one query per
 //               group, 2 for eight), the whole warp running the loop and one
 //               elected lane issuing (warp-uniform descriptors).
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator row, ReLU, weighted
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator row, ReLU, weighted
 //               head sum in fp32, length mask; then either a store of the
 //               fp32 scores (and, with SELECT, a histogram of their keys).
+//               Warps 2-5 take the even tiles, 6-9 the odd ones (4 warps,
+//               one per scheduler, left the epilogue latency-bound).
 //               With eight queries per group (256 accumulator columns a
 //               tile) warps 2-17: the four warps of a TMEM lane quarter take
 //               two queries each, so that enough warps hide the latency of
@@ -82,11 +84,16 @@ template <int NQ, bool SELECT, bool I8>
 struct Cfg {
   static_assert(!I8 || NQ == 1, "the INT8 cache is scored one query per group");
   static constexpr int kN = 32 * NQ;
-  static constexpr int kEpiWarps = NQ == 8 ? 16 : 4;
+  static constexpr int kEpiWarps = NQ == 8 ? 16 : 8;
+  // one query: two groups of 4 warps take alternate tiles (accumulator
+  // slots 0, 2 and 1, 3); eight queries: every warp takes every tile
+  static constexpr int kEpiGroups = NQ == 8 ? 1 : 2;
   static constexpr int kEpi = 32 * kEpiWarps;        // epilogue threads
   static constexpr int kThreads = 64 + kEpi;
-  static constexpr int kQPerWarp = NQ * 4 / kEpiWarps;  // queries of one epilogue thread
+  static constexpr int kQPerWarp = NQ * 4 * kEpiGroups / kEpiWarps;  // queries of one thread
   static constexpr int kTileBytes = I8 ? kHalfBytes : 2 * kHalfBytes;  // 128 keys
+  // I8: the tile's 128 block scales (512 B) follow it in the stage
+  static constexpr int kStageBytes = I8 ? kTileBytes + 1024 : kTileBytes;
   static constexpr int kStages = I8 ? 10 : (NQ == 1 ? 6 : 4);
   static constexpr int kQSlots = NQ == 1 ? 2 : 1;
   static constexpr int kQHalf = kN * 128;  // one 128-byte-wide box of Q
@@ -95,7 +102,7 @@ struct Cfg {
   // tile t+4 waits for the epilogue of tile t), 2 of 256 for eight
   static constexpr int kAcc = NQ == 1 ? 4 : 2;
   static constexpr int kTmemCols = kAcc * kN;
-  static constexpr int kQOff = kStages * kTileBytes;
+  static constexpr int kQOff = kStages * kStageBytes;
   static constexpr int kWOff = kQOff + kQSlots * kQBytes;
   static constexpr int kNbOff = kWOff + kN * 4;
   static constexpr int kSelOff = (kNbOff + NQ * 8 + 15) & ~15;
@@ -212,11 +219,20 @@ struct WorkSrc {
     if (!sc.dyn) return false;
     int k;
     if (role == kProducer) {
-      if (!mbar_wait(&sc.ring_empty[slot], ph ^ 1, abort)) return false;
-      k = atomicAdd(sc.counter, 1);
-      if (k >= sc.nchunk) k = -1;
-      sc.ring[slot] = k;
-      mbar_arrive(&sc.ring_full[slot]);
+      // a whole warp: lane 0 takes the chunk and posts it, the warp follows
+      int ok = 1, kk = -1;
+      if (lane == 0) {
+        ok = mbar_wait(&sc.ring_empty[slot], ph ^ 1, abort) ? 1 : 0;
+        if (ok) {
+          kk = atomicAdd(sc.counter, 1);
+          if (kk >= sc.nchunk) kk = -1;
+          sc.ring[slot] = kk;
+          mbar_arrive(&sc.ring_full[slot]);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      k = __shfl_sync(0xffffffffu, kk, 0);
+      if (!ok) return false;
     } else if (role == kMmaRole) {
       // a whole warp: lane 0 waits and reads the slot, the warp follows
       int ok = 1, kk = -1;
@@ -352,8 +368,10 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
   // ---- barriers and TMEM ---------------------------------------------------
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      // I8: full also counts the producer lanes' scale copies, empty the
+      // epilogue group that reads the scales
+      mbar_init(&full[s], I8 ? 1 + 32 : 1);
+      mbar_init(&empty[s], I8 ? 1 + C::kEpiWarps / C::kEpiGroups : 1);
     }
     for (int s = 0; s < C::kQSlots; ++s) {
       mbar_init(&qfull[s], 1);
@@ -361,7 +379,7 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
     }
     for (int s = 0; s < C::kAcc; ++s) {
       mbar_init(&accfull[s], 1);
-      mbar_init(&accempty[s], C::kEpiWarps);
+      mbar_init(&accempty[s], C::kEpiWarps / C::kEpiGroups);
     }
     mbar_init(drain, 1);
     for (int s = 0; s < kRing; ++s) {
@@ -382,55 +400,75 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
 
   if (warp == 0) {
     // ======================= TMA producer =================================
-    if (lane == 0) {
-      // per-row keys are read once (decode); keys shared by every query
-      // group (prefill) are re-read from L2
-      const uint64_t stream_pol = p.shared_keys ? l2_evict_normal_policy() : l2_evict_first_policy();
-      WorkSrc<NQ> src;
-      const Walker<NQ>& w = src.w;
-      int stage = 0, cur_g = -1, qs = C::kQSlots - 1;
-      uint32_t ph = 0, qe_ph[2] = {0, 0};
-      int issued = 0, q_issued_slot = -1;
-      uint32_t q_issued_ph = 0;
-      while (src.next(p, sc, kProducer, lane, abort_flag)) {
-        if (w.g != cur_g) {
-          qs = (qs + 1) % C::kQSlots;
-          if (!mbar_wait(&qempty[qs], qe_ph[qs] ^ 1, abort_flag)) break;
-          qe_ph[qs] ^= 1;
+    // The whole warp runs the loop (lane 0 waits and issues the TMA copies;
+    // with the INT8 cache every lane also copies four block scales).
+    auto wait0 = [&](uint64_t* bar, uint32_t parity) {
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+      return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
+    // per-row keys are read once (decode); keys shared by every query
+    // group (prefill) are re-read from L2
+    const uint64_t stream_pol = p.shared_keys ? l2_evict_normal_policy() : l2_evict_first_policy();
+    WorkSrc<NQ> src;
+    const Walker<NQ>& w = src.w;
+    int stage = 0, cur_g = -1, qs = C::kQSlots - 1;
+    uint32_t ph = 0, qe_ph[2] = {0, 0};
+    int issued = 0, q_issued_slot = -1;
+    uint32_t q_issued_ph = 0;
+    while (src.next(p, sc, kProducer, lane, abort_flag)) {
+      if (w.g != cur_g) {
+        qs = (qs + 1) % C::kQSlots;
+        if (!wait0(&qempty[qs], qe_ph[qs] ^ 1)) break;
+        qe_ph[qs] ^= 1;
+        if (lane == 0) {
           uint8_t* dst = q_smem + qs * C::kQBytes;
           mbar_arrive_expect_tx(&qfull[qs], C::kQBytes);
           tma_load_2d(dst, &map_q, &qfull[qs], 0, w.g * C::kN);
           if constexpr (!I8) tma_load_2d(dst + C::kQHalf, &map_q, &qfull[qs], 64, w.g * C::kN);
-          q_issued_slot = qs;
-          q_issued_ph = qe_ph[qs] ^ 1;
-          cur_g = w.g;
         }
-        if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) break;
-        uint8_t* dst = a_smem + stage * C::kTileBytes;
-        const int kb = p.shared_keys ? 0 : w.g;
+        q_issued_slot = qs;
+        q_issued_ph = qe_ph[qs] ^ 1;
+        cur_g = w.g;
+      }
+      if (!wait0(&empty[stage], ph ^ 1)) break;
+      uint8_t* dst = a_smem + stage * C::kStageBytes;
+      const int kb = p.shared_keys ? 0 : w.g;
+      if (lane == 0) {
         mbar_arrive_expect_tx(&full[stage], C::kTileBytes);
         tma_load_3d_hint(dst, &map_k, &full[stage], 0, w.t * kTileM, kb, stream_pol);
         if constexpr (!I8)
           tma_load_3d_hint(dst + kHalfBytes, &map_k, &full[stage], 64, w.t * kTileM, kb, stream_pol);
-        if constexpr (I8) {
-          // the tile's 128 block scales (512 B) into L2 now, so that the
-          // epilogue's load of them does not wait for DRAM
-          const float* sc = p.k_scale + static_cast<int64_t>(kb) * p.cap_blk +
-                            static_cast<int64_t>(w.t) * kTileM;
-          const int64_t left = p.cap_blk - static_cast<int64_t>(w.t) * kTileM;
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (q * 32 < left)
-              asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(sc + q * 32) : "memory");
-        }
-        ++issued;
-        if (++stage == C::kStages) {
-          stage = 0;
-          ph ^= 1;
-        }
       }
-      if (*abort_flag) {
-        // Let the copies already issued land before the CTA exits.
+      if constexpr (I8) {
+        // the tile's 128 block scales into the stage behind the codes (zeros
+        // past the cache); each lane's copies arrive on the stage's barrier
+        // when they land, so the epilogue reads them from shared memory
+        const int64_t base = static_cast<int64_t>(kb) * p.cap_blk + static_cast<int64_t>(w.t) * kTileM;
+        const int64_t left = p.cap_blk - static_cast<int64_t>(w.t) * kTileM;
+        const uint32_t sdst = smem_u32(dst + C::kTileBytes);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = lane * 4 + u;
+          const bool v = j < left;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(sdst + j * 4),
+                       "l"(v ? p.k_scale + base + j : p.k_scale), "r"(v ? 4 : 0)
+                       : "memory");
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                         smem_u32(&full[stage]))
+                     : "memory");
+      }
+      ++issued;
+      if (++stage == C::kStages) {
+        stage = 0;
+        ph ^= 1;
+      }
+    }
+    if (*abort_flag) {
+      // Let the copies already issued land before the CTA exits.
+      if constexpr (I8) asm volatile("cp.async.wait_all;" ::: "memory");
+      if (lane == 0) {
         const int first = issued > C::kStages ? issued - C::kStages : 0;
         for (int i = first; i < issued; ++i) {
           volatile int no_abort = 0;
@@ -442,6 +480,7 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
         }
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ======================= MMA issuer ====================================
     // The whole warp runs the loop (lane 0 waits on the barriers and the warp
@@ -470,7 +509,7 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
       if (!wait0(&full[stage], ph)) break;
       tc_fence_after();
       const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::kN);
-      const uint32_t a0 = a_base + stage * C::kTileBytes;
+      const uint32_t a0 = a_base + stage * C::kStageBytes;
       const uint32_t b0 = q_base + qs * C::kQBytes;
       if constexpr (I8) {
         // K = 32 int8 per MMA: four 32-byte steps along the 128-byte rows
@@ -512,7 +551,12 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
     const int quarter = warp & 3;  // TMEM lanes quarter*32 .. +31
     const int et = tid - 64;       // 0 .. kEpi-1
     const int row_in_tile = quarter * 32 + lane;
-    const int q0 = ((warp - 2) >> 2) * C::kQPerWarp;  // first query of this thread
+    const int wq = (warp - 2) >> 2;                  // this warp's set of 4
+    const int grp = wq % C::kEpiGroups;              // tiles with seq % groups == grp
+    const int q0 = (wq / C::kEpiGroups) * C::kQPerWarp;  // first query of this thread
+    static_assert(C::kAcc % C::kEpiGroups == 0, "a group owns whole accumulator slots");
+    int seq = 0, est = 0;  // tile sequence number; its key stage (I8 scales)
+    uint32_t est_ph = 0;
     WorkSrc<NQ> src;
     const Walker<NQ>& w = src.w;
     int acc = 0, cur_g = -1;
@@ -556,17 +600,38 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
         epi_sync();
         cur_g = w.g;
       }
-      const int64_t blk = static_cast<int64_t>(w.t) * kTileM + row_in_tile;
-      float ksc = 1.f;  // I8: the block's scale, fetched before the wait
-      if constexpr (I8) {
-        if (blk < nb_smem[0])
-          ksc = __ldg(p.k_scale + (p.shared_keys ? 0 : static_cast<int64_t>(w.g)) * p.cap_blk + blk);
+      const int my_st = est;
+      const uint32_t my_st_ph = est_ph;
+      if (++est == C::kStages) {
+        est = 0;
+        est_ph ^= 1;
       }
+      if ((seq++ % C::kEpiGroups) != grp) {  // the other group's tile
+        if (++acc == C::kAcc) {
+          acc = 0;
+          acc_ph ^= 1;
+        }
+        continue;
+      }
+      const int64_t blk = static_cast<int64_t>(w.t) * kTileM + row_in_tile;
       if (!mbar_wait(&accfull[acc], acc_ph, abort_flag)) {
         aborted = true;
         break;
       }
       tc_fence_after();
+      float ksc = 1.f;  // I8: the block's scale, from the key stage
+      if constexpr (I8) {
+        // (the stage's barrier completed before the MMA ran; waiting on it
+        // again orders the scale copies before these reads)
+        if (!mbar_wait(&full[my_st], my_st_ph, abort_flag)) {
+          aborted = true;
+          break;
+        }
+        ksc = reinterpret_cast<const float*>(a_smem + my_st * C::kStageBytes +
+                                             C::kTileBytes)[row_in_tile];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[my_st]);  // this warp is done with the stage
+      }
       constexpr int kQ = C::kQPerWarp;
       float scv[kQ];
       // ReLU-weighted head sum of one query's 32 accumulator columns; four

@@ -661,8 +661,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     }
     cluster_sync_all();
     // CTA k combines heads [k*rows_per, (k+1)*rows_per) of the group: the
-    // n_cl rows of each come back with bulk copies into the latent buffers
-    // (slot hh*n_cl + c); weights 2^(m_c - M) l_c / L from the (m, l).
+    // rows of split c come back with one bulk copy (they are contiguous in
+    // L2) into the latent buffers (slot c*nh + hh); weights 2^(m_c - M) l_c /
+    // L from the (m, l).
     const int k = static_cast<int>(cluster_rank());
     const int rows_per = kHG / n_cl;
     const int hk = k * rows_per;
@@ -674,10 +675,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
     if (nh > 0) {  // uniform
       const int nrows = nh * n_cl;
       if (tid == 0) mbar_arrive_expect_tx(bar_red, static_cast<uint32_t>(nrows) * 1024u);
-      if (tid < nrows) {
-        const int hh = tid / n_cl, c = tid % n_cl;
-        bulk_load(stage_u + tid * 1024, po_all + (static_cast<int64_t>(c) * kHG + hk + hh) * kLatent,
-                  1024u, bar_red);
+      if (tid < n_cl) {  // split c's rows of heads hk .. hk+nh-1: contiguous, one copy
+        const int c = tid;
+        bulk_load(stage_u + c * nh * 1024, po_all + (static_cast<int64_t>(c) * kHG + hk) * kLatent,
+                  static_cast<uint32_t>(nh) * 1024u, bar_red);
       }
       if (tid < kHG) {  // warps 0-1: groups of n_cl lanes, one group per head
         const int hh = tid / n_cl, c = tid % n_cl;
@@ -709,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_sparse_attn(const KParams p) {
         for (int c = 0; c < kMaxCluster; ++c) {
           wc[c] = c < n_cl ? w_s[hh * n_cl + c] : 0.f;
           v[c] = wc[c] != 0.f ? *reinterpret_cast<const uint4*>(
-                                    stage + (hh * n_cl + c) * 1024 + ((piece + h) & 63) * 16)
+                                    stage + (c * nh + hh) * 1024 + ((piece + h) & 63) * 16)
                               : make_uint4(0u, 0u, 0u, 0u);
         }
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};

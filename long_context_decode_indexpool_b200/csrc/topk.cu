@@ -597,6 +597,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* lk = wl_key + warp * kWarpCap;
     int32_t* li = wl_id + warp * kWarpCap;
     const uint32_t lt_mask = (1u << lane) - 1u;
+    // keys >= theta are the scores >= the float whose key is theta (order_key
+    // is monotone; theta at or below the lowest finite key keeps every
+    // score); a NaN passes here and the final choice's key bound settles it
+    const float ft = theta <= 0x00800000u ? -INFINITY
+                     : __uint_as_float(theta >= 0x80000000u ? (theta & 0x7FFFFFFFu) : ~theta);
     int wc = 0;
     bool over = false;
 #pragma unroll 2
@@ -605,13 +610,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float4 v4 = i < w1 ? *reinterpret_cast<const float4*>(rs + i)
                                : make_float4(0.f, 0.f, 0.f, 0.f);
       const float f[4] = {v4.x, v4.y, v4.z, v4.w};
-      uint32_t k[4], bal[4];
+      uint32_t bal[4];
       bool keep[4];
       int tot = 0, before = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        k[j] = order_key(f[j]);
-        keep[j] = i + j < w1 && k[j] >= theta;
+        keep[j] = i + j < w1 && !(f[j] < ft);  // (a NaN is kept: its key decides below)
         bal[j] = __ballot_sync(0xffffffffu, keep[j]);
         tot += __popc(bal[j]);
         before += __popc(bal[j] & lt_mask);  // kept by lower lanes (they come first)
@@ -624,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (keep[j]) {
-              lk[pos] = k[j];
+              lk[pos] = order_key(f[j]);
               li[pos] = i + j;
               ++pos;
             }
