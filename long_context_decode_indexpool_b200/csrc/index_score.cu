@@ -130,6 +130,20 @@ struct KParams {
   int* work_counter;   // zero on entry; NULL: static split only
 };
 
+// (a0, a1) += (w0 x0, w1 x1): one fma.rn.f32x2, each lane rounded once like
+// a scalar fma.rn.f32.
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, float x0,
+                                      float x1) {
+  asm("{\n\t.reg .b64 a, w, x;\n\t"
+      "mov.b64 a, {%0, %1};\n\t"
+      "mov.b64 w, {%2, %3};\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "fma.rn.f32x2 a, w, x, a;\n\t"
+      "mov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
+}
+
 template <int NQ>
 __device__ __forceinline__ int64_t row_blocks(const KParams& p, int row) {
   int64_t n = p.n_vis[row];
@@ -639,18 +653,20 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
       auto head_sum = [&](const uint32_t* v, int j) {
         const float* wj = w_smem + j * kIdxHeads;
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int h = 0; h < kIdxHeads; ++h) {
-          float x;
+        auto relu = [&](int h) {
           if constexpr (I8) {
             const int dot = static_cast<int>(v[h]);  // exact s32 dot product
-            x = static_cast<float>(dot > 0 ? dot : 0);
+            return static_cast<float>(dot > 0 ? dot : 0);
           } else {
             const float f = __uint_as_float(v[h]);
-            x = f > 0.f ? f : 0.f;
+            return f > 0.f ? f : 0.f;
           }
-          s4[h & 3] = __fmaf_rn(wj[h], x, s4[h & 3]);
-        }
+        };
+        // heads h and h+1 go to partial sums h & 3 and (h & 3) + 1 with one
+        // paired fp32 FMA (each lane rounds as a scalar FMA would)
+#pragma unroll
+        for (int h = 0; h < kIdxHeads; h += 2)
+          ffma2(s4[h & 3], s4[(h & 3) + 1], wj[h], wj[h + 1], relu(h), relu(h + 1));
         float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
         if constexpr (I8) sc *= ksc;
         return sc;
