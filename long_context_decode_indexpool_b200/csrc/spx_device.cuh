@@ -186,35 +186,14 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[smem] * B[smem]^T, signed 8-bit inputs, exact s32 accumulate.
-__device__ __forceinline__ void umma_s8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The same product issued by one elected lane of a warp that runs this call
-// with all 32 lanes: the descriptors are then warp-uniform values, so the
-// issue needs no per-MMA move into uniform registers.  A single thread
-// issuing from a lane-0 branch took about 114 cycles per MMA on sm_100a,
-// the whole warp with an unrolled loop about 40 (an M = 64, N = 64, K = 16
-// product computes in 32).  elect.sync always elects the same lane, so
-// umma_commit_elect commits the MMAs of that lane.
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate (D is
+// overwritten when accumulate is 0), issued by one elected lane of a warp
+// that runs this call with all 32 lanes: the descriptors are then
+// warp-uniform values, so the issue needs no per-MMA move into uniform
+// registers.  A single thread issuing from a lane-0 branch took about 114
+// cycles per MMA on sm_100a, the whole warp with an unrolled loop about 40
+// (an M = 64, N = 64, K = 16 product computes in 32).  elect.sync always
+// elects the same lane, so umma_commit_elect commits the MMAs of that lane.
 __device__ __forceinline__ void umma_bf16_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                                 uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -226,16 +205,7 @@ __device__ __forceinline__ void umma_bf16_elect(uint32_t d_tmem, uint64_t adesc,
       : "memory");
 }
 
-// Arrives once on `bar` when every tcgen05.mma issued so far by this thread
-// has completed.
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-
-// umma_s8 issued by one elected lane of a whole warp (see umma_bf16_elect).
+// The same with signed 8-bit A and B and an exact s32 accumulator.
 __device__ __forceinline__ void umma_s8_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                               uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -247,7 +217,8 @@ __device__ __forceinline__ void umma_s8_elect(uint32_t d_tmem, uint64_t adesc, u
       : "memory");
 }
 
-// umma_commit by the lane that elect.sync elects (see umma_bf16_elect).
+// Arrives once on `bar` when every tcgen05.mma issued so far by the lane
+// that elect.sync elects has completed (see umma_bf16_elect).
 __device__ __forceinline__ void umma_commit_elect(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
