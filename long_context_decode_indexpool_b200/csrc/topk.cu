@@ -445,7 +445,7 @@ __global__ void __launch_bounds__(kThreads)
 // memory with bulk copies (per-thread loads of a 135 KiB row were bound by
 // the misses an SM keeps in flight: 11 us a row).  2048 evenly spaced scores
 // give a threshold theta, a 22-bit key prefix above which about
-// 2.5 x 512 x 2048 / nblk of the samples lie, found by two 11-bit radix
+// 2 x 512 x 2048 / nblk of the samples lie, found by two 11-bit radix
 // passes over the samples.  Each warp then keeps the keys at or above theta
 // of a contiguous range and appends them, in block order, to a list of its
 // own (ballots place them).  If
@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(kThreads)
 // need_full[r] for k_select_rows_full; every row's flag is written.
 constexpr int kWarpCap = 256;                 // survivors per warp list
 constexpr int kCandCap = (kThreads / 32) * kWarpCap;  // 4096
-constexpr int kTargetSurvivors = 1280;        // 2.5 x 512 expected
+constexpr int kTargetSurvivors = 1024;        // 2 x 512 expected
 constexpr int kSampPer = 4;                   // samples per thread (2048 per row)
 constexpr int kFastRowCap = 36864;            // scores of a row staged by the fast path (144 KiB)
 
