@@ -120,6 +120,8 @@ struct KParams {
   const float* k_scale;  // I8: [key batches, cap_blk] block scales
   int64_t cap_blk;
   const int64_t* n_vis;
+  const int64_t* len_spec;  // optional: lengths before the append (planning only)
+  int n_add;
   float* scores;
   int64_t score_stride;
   int64_t max_len;
@@ -144,21 +146,31 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, 
       : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
 }
 
+// Pooled blocks of a row: from n_vis or, with `spec`, from the lengths
+// before the append the way the pool kernel turns them into n_vis.
 template <int NQ>
-__device__ __forceinline__ int64_t row_blocks(const KParams& p, int row) {
-  int64_t n = p.n_vis[row];
+__device__ __forceinline__ int64_t row_blocks(const KParams& p, int row, bool spec = false) {
+  int64_t n;
+  if (spec) {
+    int64_t len = p.len_spec[row];
+    if (len < 0) len = 0;
+    if (len > p.max_len - p.n_add) len = p.max_len - p.n_add;
+    n = len + p.n_add;
+  } else {
+    n = p.n_vis[row];
+  }
   n = n < 0 ? 0 : (n > p.max_len ? p.max_len : n);
   return n / kPool;
 }
 
 template <int NQ>
-__device__ __forceinline__ int group_tiles(const KParams& p, int g) {
+__device__ __forceinline__ int group_tiles(const KParams& p, int g, bool spec = false) {
   int64_t nb = 0;
 #pragma unroll
   for (int j = 0; j < NQ; ++j) {
     const int r = g * NQ + j;
     if (r < p.rows) {
-      const int64_t v = row_blocks<NQ>(p, r);
+      const int64_t v = row_blocks<NQ>(p, r, spec);
       nb = v > nb ? v : nb;
     }
   }
@@ -166,15 +178,21 @@ __device__ __forceinline__ int group_tiles(const KParams& p, int g) {
 }
 
 // Walks (group, tile) work items in order; `gstart` is the global index of
-// tile 0 of the current group.
+// tile 0 of the current group.  `tab` (shared memory, or NULL) holds the
+// first flat tile of every group and the total, [groups + 1].
 template <int NQ>
 struct Walker {
   int g, t, nt;
   int64_t gstart;
-  __device__ void init(const KParams& p, int g0, int t0, int64_t lo) {
+  const int* tab;
+  __device__ int tiles(const KParams& p, int gg) const {
+    return tab ? tab[gg + 1] - tab[gg] : group_tiles<NQ>(p, gg);
+  }
+  __device__ void init(const KParams& p, int g0, int t0, int64_t lo, const int* tab_) {
+    tab = tab_;
     g = g0;
     t = t0;
-    nt = group_tiles<NQ>(p, g0);
+    nt = tiles(p, g0);
     gstart = lo - t0;
   }
   __device__ void advance(const KParams& p) {
@@ -183,7 +201,7 @@ struct Walker {
       t = 0;
       do {
         ++g;
-        nt = (g < p.groups) ? group_tiles<NQ>(p, g) : 1;
+        nt = (g < p.groups) ? tiles(p, g) : 1;
       } while (nt == 0);
     }
   }
@@ -199,6 +217,7 @@ struct Sched {
   int64_t dyn_begin, total;
   int nchunk;
   const int* pre;  // smem [groups + 1]: first flat tile of each group
+  const int* gt;   // the same table when the Walker may use it, or NULL
   int* ring;       // smem [kRing]
   uint64_t* ring_full;
   uint64_t* ring_empty;
@@ -221,7 +240,7 @@ struct WorkSrc {
     if (!started) {
       started = true;
       if (sc.n_static > 0) {
-        w.init(p, sc.g0, sc.t0, sc.lo);
+        w.init(p, sc.g0, sc.t0, sc.lo, sc.gt);
         left = sc.n_static - 1;
         return true;
       }
@@ -277,7 +296,7 @@ struct WorkSrc {
       if (sc.pre[mid] <= f) lo_g = mid; else hi_g = mid - 1;
     }
     while (sc.pre[lo_g + 1] <= f) ++lo_g;  // skip groups without tiles
-    w.init(p, lo_g, static_cast<int>(f - sc.pre[lo_g]), f);
+    w.init(p, lo_g, static_cast<int>(f - sc.pre[lo_g]), f, sc.gt);
     left = static_cast<int>(n) - 1;
     return true;
   }
@@ -323,63 +342,8 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
     prefetch_tensormap(&map_q);
   }
   pdl_trigger();  // the next kernel's CTAs may be scheduled as SMs free up
-  pdl_wait();     // lengths, keys and the histogram come from the previous kernel
 
-  // ---- this CTA's work: a contiguous static range, then dynamic chunks ----
-  const bool dyn = p.work_counter != nullptr && p.groups <= kMaxDynGroups;  // uniform
-  int64_t total = 0;
-  for (int base = 0; base < p.groups; base += kThreads) {
-    const int g = base + tid;
-    int sum;
-    const int ex = block_excl_scan(g < p.groups ? group_tiles<NQ>(p, g) : 0, s_scan, &sum);
-    if (dyn && g < p.groups) s_pre[g] = static_cast<int>(total + ex);
-    total += sum;
-  }
-  if (dyn && tid == 0) s_pre[p.groups] = static_cast<int>(total);
-  const int64_t G = gridDim.x;
-  Sched sc;
-  sc.dyn = dyn;
-  sc.total = total;
-  if (dyn) {
-    const int64_t per = total * 7 / (8 * G);
-    sc.lo = per * blockIdx.x;
-    sc.n_static = static_cast<int>(per);
-    sc.dyn_begin = per * G;
-    sc.nchunk = static_cast<int>((total - sc.dyn_begin + kDynChunk - 1) / kDynChunk);
-  } else {
-    sc.lo = total * blockIdx.x / G;
-    sc.n_static = static_cast<int>(total * (blockIdx.x + 1) / G - sc.lo);
-    sc.dyn_begin = total;
-    sc.nchunk = 0;
-    if (sc.n_static <= 0) return;  // uniform
-  }
-  sc.pre = s_pre;
-  sc.ring = s_ring;
-  sc.ring_full = ring_bars;
-  sc.ring_empty = ring_bars + kRing;
-  sc.counter = p.work_counter;
-  sc.g0 = 0;
-  sc.t0 = 0;
-  if (sc.n_static > 0) {
-    int64_t run = 0;
-    for (int base = 0; base < p.groups; base += kThreads) {
-      const int g = base + tid;
-      const int c = g < p.groups ? group_tiles<NQ>(p, g) : 0;
-      int sum;
-      const int ex = block_excl_scan(c, s_scan, &sum);
-      if (c > 0 && run + ex <= sc.lo && sc.lo < run + ex + c) {
-        s_g0 = g;
-        s_t0 = static_cast<int>(sc.lo - run - ex);
-      }
-      run += sum;
-      if (run > sc.lo) break;  // uniform
-    }
-    __syncthreads();
-    sc.g0 = s_g0;
-    sc.t0 = s_t0;
-  }
-
-  // ---- barriers and TMEM ---------------------------------------------------
+  // ---- barriers and TMEM (nothing here depends on the previous kernel) ---
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       // I8: full also counts the producer lanes' scale copies, empty the
@@ -411,6 +375,84 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+
+  // ---- this CTA's work: a contiguous static range, then dynamic chunks ----
+  const bool tab = p.groups <= kMaxDynGroups;         // uniform: tile counts in shared memory
+  const bool dyn = p.work_counter != nullptr && tab;  // uniform
+  const int64_t G = gridDim.x;
+  Sched sc;
+  sc.dyn = dyn;
+  sc.pre = s_pre;
+  sc.gt = tab ? s_pre : nullptr;
+  sc.ring = s_ring;
+  sc.ring_full = ring_bars;
+  sc.ring_empty = ring_bars + kRing;
+  sc.counter = p.work_counter;
+  // the split of the tiles over the CTAs, from n_vis or (spec) from the
+  // lengths before the append
+  auto plan = [&](bool spec) {
+    int64_t total = 0;
+    for (int base = 0; base < p.groups; base += kThreads) {
+      const int g = base + tid;
+      const int c = g < p.groups ? group_tiles<NQ>(p, g, spec) : 0;
+      int sum;
+      const int ex = block_excl_scan(c, s_scan, &sum);
+      if (tab && g < p.groups) s_pre[g] = static_cast<int>(total + ex);
+      total += sum;
+    }
+    if (tab && tid == 0) s_pre[p.groups] = static_cast<int>(total);
+    __syncthreads();
+    sc.total = total;
+    if (dyn) {
+      const int64_t per = total * 7 / (8 * G);
+      sc.lo = per * blockIdx.x;
+      sc.n_static = static_cast<int>(per);
+      sc.dyn_begin = per * G;
+      sc.nchunk = static_cast<int>((total - sc.dyn_begin + kDynChunk - 1) / kDynChunk);
+    } else {
+      sc.lo = total * blockIdx.x / G;
+      sc.n_static = static_cast<int>(total * (blockIdx.x + 1) / G - sc.lo);
+      sc.dyn_begin = total;
+      sc.nchunk = 0;
+    }
+    sc.g0 = 0;
+    sc.t0 = 0;
+    if (sc.n_static > 0) {  // uniform
+      int64_t run = 0;
+      for (int base = 0; base < p.groups; base += kThreads) {
+        const int g = base + tid;
+        const int c = g < p.groups ? (tab ? s_pre[g + 1] - s_pre[g] : group_tiles<NQ>(p, g, spec)) : 0;
+        int sum;
+        const int ex = block_excl_scan(c, s_scan, &sum);
+        if (c > 0 && run + ex <= sc.lo && sc.lo < run + ex + c) {
+          s_g0 = g;
+          s_t0 = static_cast<int>(sc.lo - run - ex);
+        }
+        run += sum;
+        if (run > sc.lo) break;  // uniform
+      }
+      __syncthreads();
+      sc.g0 = s_g0;
+      sc.t0 = s_t0;
+    }
+  };
+  // Decode plans from the caller's lengths while the previous kernel (the
+  // append) still runs, and keeps the plan if n_vis agrees after the wait.
+  const bool spec = tab && p.len_spec != nullptr;  // uniform
+  if (spec) plan(true);
+  pdl_wait();  // lengths, keys and the histogram come from the previous kernel
+  if (spec) {
+    int bad = 0;
+    for (int g = tid; g < p.groups; g += kThreads)
+      bad |= s_pre[g + 1] - s_pre[g] != group_tiles<NQ>(p, g);
+    if (__syncthreads_or(bad)) plan(false);  // uniform
+  } else {
+    plan(false);
+  }
+  if (!dyn && sc.n_static <= 0) {  // uniform: no tiles for this CTA
+    if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+    return;
+  }
 
   if (warp == 0) {
     // ======================= TMA producer =================================
@@ -761,6 +803,8 @@ cudaError_t launch_cfg(const ScoreArgs& a, cudaStream_t stream) {
   p.k_scale = a.k_scale;
   p.cap_blk = a.cap_blk;
   p.n_vis = a.n_vis;
+  p.len_spec = a.len_spec;
+  p.n_add = a.n_add;
   p.scores = a.scores;
   p.score_stride = a.score_stride;
   p.max_len = a.max_len;

@@ -872,6 +872,8 @@ spx_status decode_impl(const spx_dims* d, int32_t B, const void* raw_k, const fl
   sa.pooled_k = pooled_k;
   sa.cap_blk = cap_blk;
   sa.n_vis = n_vis;
+  sa.len_spec = len_dev;  // plans the work before the append finishes
+  sa.n_add = pa.n_new;
   sa.max_len = max_len;
   sa.scores = scores;
   sa.score_stride = L.stride;

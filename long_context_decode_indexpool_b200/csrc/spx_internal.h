@@ -77,6 +77,11 @@ struct ScoreArgs {
   const void* pooled_k;  // [key_batches, cap_blk, 128] bf16
   int64_t cap_blk;
   const int64_t* n_vis;  // [rows]
+  // optional (decode): the lengths before the append that writes n_vis,
+  // n_vis = clamp(len_spec, 0, max_len - n_add) + n_add; read before the
+  // wait on the previous kernel to plan the work, then checked against n_vis
+  const int64_t* len_spec;
+  int n_add;
   int64_t max_len;
   float* scores;        // [rows, score_stride]
   int64_t score_stride;
