@@ -77,6 +77,7 @@ constexpr int kHistShift = 21;
 constexpr int kDynChunk = 4;
 constexpr int kMaxDynGroups = 512;
 constexpr int kRing = 4;  // chunk indices handed from the TMA warp to the others
+constexpr int kPrefetchTiles = 6;  // decode: first tiles of a CTA sent to L2 before the wait
 
 // I8: the INT8 cache (decode only): 128-byte key rows (one box per tile),
 // int8 query codes, kind::i8 MMAs into s32 accumulators.
@@ -440,6 +441,20 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
   // append) still runs, and keeps the plan if n_vis agrees after the wait.
   const bool spec = tab && p.len_spec != nullptr;  // uniform
   if (spec) plan(true);
+  if (spec && tid == 0 && sc.n_static > 0) {
+    // the first tiles of the static range head for L2 while the append runs
+    // (a prefetch reads no data into the CTA, so a plan that turns out
+    // wrong costs only the traffic)
+    Walker<NQ> pw;
+    pw.init(p, sc.g0, sc.t0, sc.lo, sc.gt);
+    const int n = sc.n_static < kPrefetchTiles ? sc.n_static : kPrefetchTiles;
+    for (int i = 0; i < n; ++i) {
+      if (i) pw.advance(p);
+      const int kb = p.shared_keys ? 0 : pw.g;
+      tma_prefetch_3d(&map_k, 0, pw.t * kTileM, kb);
+      if constexpr (!I8) tma_prefetch_3d(&map_k, 64, pw.t * kTileM, kb);
+    }
+  }
   pdl_wait();  // lengths, keys and the histogram come from the previous kernel
   if (spec) {
     int bad = 0;
