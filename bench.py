@@ -180,11 +180,14 @@ class DecodeState:
 
 class PrefillState:
     """Caches and inputs of a chunked-prefill workload (batch 1): a cache of
-    pos0 tokens built with spx_pool_append, then T new tokens."""
+    pos0 tokens built with spx_pool_append (spx_pool_append_i8 with
+    keys="int8": int8 codes plus one scale per block), then T new tokens."""
 
-    def __init__(self, w: synth.Workload, device, pos0: int | None = None, T: int | None = None):
+    def __init__(self, w: synth.Workload, device, pos0: int | None = None, T: int | None = None,
+                 keys: str = "bf16"):
         spx = spx_module()
         self.w = w
+        self.i8 = keys == "int8"
         self.device = device
         self.pos0 = pos0 = w.L if pos0 is None else pos0
         self.T = T = w.T if T is None else T
@@ -195,15 +198,23 @@ class PrefillState:
         self.cap_blk = (total + 3) // 4
         self.cap_tok = total
         bf16 = torch.bfloat16
-        self.pooled = torch.zeros(1, self.cap_blk, synth.IDX_DIM, dtype=bf16, device=device)
+        self.pooled = torch.zeros(1, self.cap_blk, synth.IDX_DIM,
+                                  dtype=torch.int8 if self.i8 else bf16, device=device)
+        self.k_scale = (torch.zeros(1, self.cap_blk, dtype=torch.float32, device=device)
+                        if self.i8 else None)
         self.tail = torch.zeros(1, 3, synth.IDX_DIM, dtype=bf16, device=device)
         t = 0
         while t < pos0:
             t1 = min(pos0, t + GEN_CHUNK_TOKENS)
             raw = w.raw_keys_t(0, t, t1, device).view(bf16)
             ln = torch.tensor([t], dtype=torch.int64, device=device)
-            spx.spx_pool_append(self.d, 1, raw.reshape(1, t1 - t, synth.IDX_DIM), t1 - t,
-                                self.pool_w, self.tail, self.pooled, self.cap_blk, ln, t1)
+            if self.i8:
+                spx.spx_pool_append_i8(self.d, 1, raw.reshape(1, t1 - t, synth.IDX_DIM), t1 - t,
+                                       self.pool_w, self.tail, self.pooled, self.k_scale,
+                                       self.cap_blk, ln, t1)
+            else:
+                spx.spx_pool_append(self.d, 1, raw.reshape(1, t1 - t, synth.IDX_DIM), t1 - t,
+                                    self.pool_w, self.tail, self.pooled, self.cap_blk, ln, t1)
             t = t1
         self.latent = torch.empty(total, synth.LATENT, dtype=bf16, device=device)
         for t in range(0, total, GEN_CHUNK_TOKENS):
@@ -223,6 +234,13 @@ class PrefillState:
 
     def step(self, timing=None):
         spx = spx_module()
+        if self.i8:
+            spx.spx_prefill_chunk_i8(self.d, self.T, self.raw_k, self.pool_w, self.tail,
+                                     self.pooled, self.k_scale, self.cap_blk, self.pos0,
+                                     self.q_idx, self.w_head, self.q, self.latent, self.cap_tok,
+                                     self.out, self.lse, self.idx, self.count, self.ws,
+                                     timing=timing)
+            return
         spx.spx_prefill_chunk(self.d, self.T, self.raw_k, self.pool_w, self.tail, self.pooled,
                               self.cap_blk, self.pos0, self.q_idx, self.w_head, self.q,
                               self.latent, self.cap_tok, self.out, self.lse, self.idx, self.count,
@@ -935,13 +953,13 @@ def run_host_latent(args, world, rank, local):
                        "batch_per_gpu": st.B, "context": st.L}}
 
 
-def measure_prefill(device, steps: int, warmup: int, world: int = 1):
+def measure_prefill(device, steps: int, warmup: int, world: int = 1, keys: str = "bf16"):
     """Times the chunked-prefill workload (4096 new tokens on a 131,072-token
     cache, one fused call per step) and its scoring kernel; returns the
     per-rank numbers and the state (for the oracle sample)."""
     spx = spx_module()
     w = synth.workload("prefill")
-    st = PrefillState(w, device)
+    st = PrefillState(w, device, keys=keys)
     stream = torch.cuda.current_stream(device)
     for _ in range(warmup):
         st.step()
@@ -982,6 +1000,8 @@ def measure_prefill(device, steps: int, warmup: int, world: int = 1):
 def prefill_summary(st, m, world: int = 1):
     """The prefill numbers against the tensor roofline (measured bf16 peaks)."""
     hbm, bf16, bf16s, src = measured_peaks()
+    # the INT8 cache scores on kind::i8 (twice the bf16 rate, nominally)
+    sc_peak, sc_peak_s = (2 * bf16, 2 * bf16s) if st.i8 else (bf16, bf16s)
     ms_step = m["ms"] / m["steps"]
     f_idx = score_algorithmic_flops_prefill(st.pos0, st.T)
     f_att = attention_flops_prefill(st.pos0, st.T, st.H)
@@ -994,7 +1014,9 @@ def prefill_summary(st, m, world: int = 1):
         "step_tflops": step_tf, "step_frac_of_burst": step_tf / bf16,
         "step_frac_of_sustained": step_tf / bf16s,
         "scoring_kernel": {"avg_launch_us": m["score_ms"] * 1e3, "tflops": score_tf,
-                           "frac_of_burst": score_tf / bf16, "frac_of_sustained": score_tf / bf16s},
+                           "frac_of_burst": score_tf / sc_peak,
+                           "frac_of_sustained": score_tf / sc_peak_s,
+                           "peak_dtype": "int8 (2 x bf16)" if st.i8 else "bf16"},
         "peak": {"bf16_burst_tflops": bf16, "bf16_sustained_tflops": bf16s, "source": src},
         "gpu_launches_per_step": m["launches"] / m["steps"],
         "clocks": m["clocks"],
@@ -1061,7 +1083,7 @@ def stratified_prefill_queries(T: int, n: int = 256, seed: int = 5) -> list:
 def run_prefill(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    st, m = measure_prefill(device, args.steps, args.warmup, world)
+    st, m = measure_prefill(device, args.steps, args.warmup, world, keys=args.keys)
     if rank != 0:
         return None
     summ = prefill_summary(st, m, world)
@@ -1071,19 +1093,21 @@ def run_prefill(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": summ["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": {"workload": st.w.name, "pos0": st.pos0, "T": st.T,
-                                        "heads": st.H},
+                                        "heads": st.H, "pooled_keys": args.keys},
         "roofline": {"bound": "tensor", "kernel": "k_index_score<8> (prefill scoring)",
                      "achieved": summ["scoring_kernel"]["tflops"],
-                     "peak": summ["peak"]["bf16_burst_tflops"], "unit": "TFLOP/s",
+                     "peak": summ["scoring_kernel"]["tflops"] / summ["scoring_kernel"]["frac_of_burst"],
+                     "unit": "TFLOP/s",
                      "frac": summ["scoring_kernel"]["frac_of_burst"],
-                     "peak_source": f"{summ['peak']['source']} bf16_tflops (burst)",
+                     "peak_source": f"{summ['peak']['source']} bf16_tflops (burst)"
+                                    + (" x 2 for int8" if st.i8 else ""),
                      "traffic": None, "avg_launch_us": summ["scoring_kernel"]["avg_launch_us"]},
         "roofline_step": {"bound": "tensor", "achieved": summ["step_tflops"], "unit": "TFLOP/s",
                           "frac_of_burst": summ["step_frac_of_burst"],
                           "frac_of_sustained": summ["step_frac_of_sustained"]},
         "gpu_launches": m["launches"], "clocks": m["clocks"],
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not st.i8:
         line["cpu_baseline"] = prefill_cpu_baseline(st)
     return line
 
@@ -1144,7 +1168,7 @@ def main(argv=None):
     ap.add_argument("--indexshare", type=int, default=0, metavar="N",
                     help="IndexShare decode: one indexer per N layers (reports per-layer rate)")
     ap.add_argument("--keys", choices=("bf16", "int8"), default="bf16",
-                    help="pooled-key cache format of the decode workloads")
+                    help="pooled-key cache format (decode and prefill workloads)")
     ap.add_argument("--score-only", action="store_true",
                     help="time the decode scoring kernel alone (profiling aid)")
     args = ap.parse_args(argv)

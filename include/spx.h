@@ -485,6 +485,29 @@ SPX_API spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* r
                              void* ws, size_t ws_bytes,
                              const spx_timing* timing, spx_stream stream);
 
+/* ---------------------------------------------------------------------------
+ * Chunked prefill on the INT8 pooled-key cache ([W1] section "양자화: W8A8와
+ * 혼합 캐시"; codes, scales and scores as for the INT8 calls above).  The
+ * chunk's complete blocks are appended as codes and scales (as
+ * spx_pool_append_i8 does), the T indexer queries are quantised per head,
+ * and each query scores the codes of its floor(n_t/4) blocks on the int8
+ * tensor cores; top-k and attention as in spx_prefill_chunk.
+ *
+ *   pooled_k8  int8 [1, cap_blk, idx_dim]  codes (16-byte aligned base)
+ *   k_scale    float [1, cap_blk]          block scales (4-byte aligned)
+ *   ws         workspace of spx_prefill_workspace_size(d, T, pos0) bytes
+ * Other arguments, limits and errors as for spx_prefill_chunk.
+ * ------------------------------------------------------------------------- */
+SPX_API spx_status spx_prefill_chunk_i8(const spx_dims* d, int32_t T, const void* raw_k,
+                                const float* pool_w, void* tail, void* pooled_k8,
+                                float* k_scale, int64_t cap_blk, int64_t pos0,
+                                const void* q_idx, const float* w_head,
+                                const void* q, const void* latent,
+                                int64_t cap_tok, void* out, float* lse,
+                                int32_t* idx_out, int32_t* count_out, void* ws,
+                                size_t ws_bytes, const spx_timing* timing,
+                                spx_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -95,6 +95,9 @@ _SIGS = {
     "spx_prefill_workspace_size": ([_DIMS, _I32, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "spx_prefill_chunk": ([_DIMS, _I32, _P, _P, _P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P,
                            _P, _P, _P, _SZ, ctypes.POINTER(spx_timing), _P], ctypes.c_int),
+    "spx_prefill_chunk_i8": ([_DIMS, _I32, _P, _P, _P, _P, _P, _I64, _I64, _P, _P, _P, _P, _I64,
+                              _P, _P, _P, _P, _P, _SZ, ctypes.POINTER(spx_timing), _P],
+                             ctypes.c_int),
 }
 
 for _name, (_args, _res) in _SIGS.items():
@@ -374,6 +377,19 @@ def spx_prefill_chunk(d, T, raw_k, pool_w, tail, pooled_k, cap_blk, pos0, q_idx,
                                   _ptr(q), _ptr(latent), cap_tok, _ptr(out), _ptr(lse),
                                   _ptr(idx_out), _ptr(count_out), _ptr(ws), ws_bytes,
                                   _timing(timing), _stream(stream)), "spx_prefill_chunk")
+
+
+def spx_prefill_chunk_i8(d, T, raw_k, pool_w, tail, pooled_k8, k_scale, cap_blk, pos0, q_idx,
+                         w_head, q, latent, cap_tok, out, lse=None, idx_out=None, count_out=None,
+                         ws=None, ws_bytes=None, timing=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.spx_prefill_chunk_i8(ctypes.byref(d), T, _ptr(raw_k), _host_f32(pool_w),
+                                     _ptr(tail), _ptr(pooled_k8), _ptr(k_scale), cap_blk, pos0,
+                                     _ptr(q_idx), _ptr(w_head), _ptr(q), _ptr(latent), cap_tok,
+                                     _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(count_out),
+                                     _ptr(ws), ws_bytes, _timing(timing), _stream(stream)),
+           "spx_prefill_chunk_i8")
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:

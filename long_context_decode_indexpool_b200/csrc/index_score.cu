@@ -79,11 +79,12 @@ constexpr int kMaxDynGroups = 512;
 constexpr int kRing = 4;  // chunk indices handed from the TMA warp to the others
 constexpr int kPrefetchTiles = 6;  // decode: first tiles of a CTA sent to L2 before the wait
 
-// I8: the INT8 cache (decode only): 128-byte key rows (one box per tile),
-// int8 query codes, kind::i8 MMAs into s32 accumulators.
+// I8: the INT8 cache: 128-byte key rows (one box per tile), int8 query
+// codes, kind::i8 MMAs into s32 accumulators (N = 32 heads for one query,
+// 256 for eight).
 template <int NQ, bool SELECT, bool I8>
 struct Cfg {
-  static_assert(!I8 || NQ == 1, "the INT8 cache is scored one query per group");
+  static_assert(!I8 || !SELECT || NQ == 1, "the key histogram is kept for one query per group");
   static constexpr int kN = 32 * NQ;
   static constexpr int kEpiWarps = NQ == 8 ? 16 : 8;
   // one query: two groups of 4 warps take alternate tiles (accumulator
@@ -855,7 +856,10 @@ cudaError_t launch_index_score(const ScoreArgs& a, cudaStream_t stream) {
     if (a.sel_ghist) return launch_cfg<1, true, false>(a, stream);
     return launch_cfg<1, false, false>(a, stream);
   }
-  if (a.nq == 8 && !a.i8) return launch_cfg<8, false, false>(a, stream);
+  if (a.nq == 8) {
+    if (a.i8) return launch_cfg<8, false, true>(a, stream);
+    return launch_cfg<8, false, false>(a, stream);
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -164,8 +164,9 @@ inline int64_t score_stride_for(int64_t max_len) {
 //   n_vis [rows] int64 | scores [rows, stride] f32 | idx [rows, 512] | count [rows]
 //   | key histograms [rows, 2048] | chunk counters [rows] | list keys, list
 //   ids [rows*nchunk, 512] | list counts [rows*nchunk] | attention scratch
+//   | INT8 cache: query codes [rows, 32, 128] int8, head weights [rows, 32]
 struct FusedLayout {
-  size_t nvis, scores, idx, count, hist, done, lkey, lidx, lcnt, attn, total;
+  size_t nvis, scores, idx, count, hist, done, lkey, lidx, lcnt, attn, q8, wq, total;
   int64_t stride;
   int nchunk;
   AttnPlan ap;
@@ -200,6 +201,10 @@ FusedLayout fused_layout(int rows, int heads, int64_t max_len) {
   o += up(lists * 4);
   L.attn = o;
   o += up(L.ap.ws_bytes);
+  L.q8 = o;  // INT8 cache: query codes [rows, 32, 128] and scaled head weights [rows, 32]
+  o += up(static_cast<size_t>(rows) * kIdxHeads * kIdxDim);
+  L.wq = o;
+  o += up(static_cast<size_t>(rows) * kIdxHeads * 4);
   L.total = o;
   return L;
 }
@@ -964,12 +969,13 @@ spx_status spx_prefill_workspace_size(const spx_dims* d, int32_t T, int64_t pos0
   return SPX_OK;
 }
 
-spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, const float* pool_w,
-                             void* tail, void* pooled_k, int64_t cap_blk, int64_t pos0,
-                             const void* q_idx, const float* w_head, const void* q,
-                             const void* latent, int64_t cap_tok, void* out, float* lse,
-                             int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
-                             const spx_timing* timing, spx_stream stream) {
+// Chunked prefill, bf16 or INT8 (k_scale set) pooled-key cache.
+static spx_status prefill_impl(const spx_dims* d, int32_t T, const void* raw_k, const float* pool_w,
+                        void* tail, void* pooled_k, float* k_scale, int64_t cap_blk,
+                        int64_t pos0, const void* q_idx, const float* w_head, const void* q,
+                        const void* latent, int64_t cap_tok, void* out, float* lse,
+                        int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
+                        const spx_timing* timing, spx_stream stream, bool i8) {
   spx_status st = check_dims(d);
   if (st != SPX_OK) return st;
   float w[4];
@@ -980,6 +986,7 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
   if (cap_blk > (int64_t(1) << 31) - 1) return SPX_ERR_SHAPE;
   if (!raw_k || !tail || !pooled_k || !q_idx || !w_head || !q || !latent || !out)
     return SPX_ERR_INVALID_ARG;
+  if (i8 && (!k_scale || !al4(k_scale))) return SPX_ERR_INVALID_ARG;
   if (!al16(raw_k) || !al16(tail) || !al16(pooled_k) || !al16(q_idx) || !al16(q) ||
       !al16(latent) || !al16(out) || !al4(w_head) || (lse && !al4(lse)) ||
       (idx_out && !al4(idx_out)) || (count_out && !al4(count_out)))
@@ -1013,19 +1020,26 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
   pa.len_host = pos0;
   pa.max_len = max_len;
   pa.nvis_out = nullptr;
+  pa.i8 = i8;
+  pa.k_scale = k_scale;
   cudaError_t e = launch_pool_append(pa, s);
   if (e != cudaSuccess) return SPX_ERR_CUDA;
   if ((e = launch_prefill_nvis(n_vis, T, pos0, s)) != cudaSuccess) return SPX_ERR_CUDA;
+  int8_t* q8 = reinterpret_cast<int8_t*>(base + L.q8);
+  float* wq = reinterpret_cast<float*>(base + L.wq);
+  if (i8 && (e = launch_quant_q(T, q_idx, w_head, q8, wq, s)) != cudaSuccess) return SPX_ERR_CUDA;
 
   if (timing && timing->score_begin &&
       cudaEventRecord(static_cast<cudaEvent_t>(timing->score_begin), s) != cudaSuccess)
     return SPX_ERR_CUDA;
   ScoreArgs sa{};
   sa.nq = 8;
+  sa.i8 = i8;
+  sa.k_scale = k_scale;
   sa.rows = T;
   sa.key_batches = 1;
-  sa.q_idx = q_idx;
-  sa.w_head = w_head;
+  sa.q_idx = i8 ? static_cast<const void*>(q8) : q_idx;
+  sa.w_head = i8 ? wq : w_head;
   sa.pooled_k = pooled_k;
   sa.cap_blk = cap_blk;
   sa.n_vis = n_vis;
@@ -1079,6 +1093,29 @@ spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, co
   aa.ws = base + L.attn;
   aa.pdl = true;  // set-up overlaps the selection; the ids are read after the wait
   return cuda_status(launch_attn(L.ap, aa, s));
+}
+
+spx_status spx_prefill_chunk(const spx_dims* d, int32_t T, const void* raw_k, const float* pool_w,
+                             void* tail, void* pooled_k, int64_t cap_blk, int64_t pos0,
+                             const void* q_idx, const float* w_head, const void* q,
+                             const void* latent, int64_t cap_tok, void* out, float* lse,
+                             int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
+                             const spx_timing* timing, spx_stream stream) {
+  return prefill_impl(d, T, raw_k, pool_w, tail, pooled_k, nullptr, cap_blk, pos0, q_idx, w_head,
+                      q, latent, cap_tok, out, lse, idx_out, count_out, ws, ws_bytes, timing,
+                      stream, false);
+}
+
+spx_status spx_prefill_chunk_i8(const spx_dims* d, int32_t T, const void* raw_k,
+                                const float* pool_w, void* tail, void* pooled_k8, float* k_scale,
+                                int64_t cap_blk, int64_t pos0, const void* q_idx,
+                                const float* w_head, const void* q, const void* latent,
+                                int64_t cap_tok, void* out, float* lse, int32_t* idx_out,
+                                int32_t* count_out, void* ws, size_t ws_bytes,
+                                const spx_timing* timing, spx_stream stream) {
+  return prefill_impl(d, T, raw_k, pool_w, tail, pooled_k8, k_scale, cap_blk, pos0, q_idx, w_head,
+                      q, latent, cap_tok, out, lse, idx_out, count_out, ws, ws_bytes, timing,
+                      stream, true);
 }
 
 }  // extern "C"

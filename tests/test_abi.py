@@ -169,6 +169,17 @@ def test_int8_cache_host_validation(spx):
         spx.spx_index_score_i8(d, 4, FAKE, FAKE, FAKE, FAKE, 1024, FAKE, 4096, FAKE, 1000, FAKE,
                                ws_bytes=need, stream=s)
     assert e.value.status == 2
+    # INT8 prefill: scales required and 4-byte aligned, the bf16 prefill workspace
+    need = spx.spx_prefill_workspace_size(d, 64, 10)
+    for ks, status in ((None, 1), (FAKE + 2, 1)):
+        with pytest.raises(spx.SpxError) as e:
+            spx.spx_prefill_chunk_i8(d, 64, FAKE, [0.25] * 4, FAKE, FAKE, ks, 32, 10, FAKE, FAKE,
+                                     FAKE, FAKE, 128, FAKE, ws=FAKE, ws_bytes=need, stream=s)
+        assert e.value.status == status
+    with pytest.raises(spx.SpxError) as e:
+        spx.spx_prefill_chunk_i8(d, 64, FAKE, [0.25] * 4, FAKE, FAKE, FAKE, 32, 10, FAKE, FAKE,
+                                 FAKE, FAKE, 128, FAKE, ws=FAKE, ws_bytes=need - 1, stream=s)
+    assert e.value.status == 4
     # fused decode: same workspace as the bf16 call; scales required
     need = spx.spx_decode_workspace_size(d, 4, 8192)
     with pytest.raises(spx.SpxError) as e:

@@ -258,3 +258,78 @@ def test_fused_i8_equals_composed():
     for b in range(B):
         a = set(st16.idx[b].cpu().tolist())
         assert len(a & set(idx_f[b].cpu().tolist())) >= 400
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill on the INT8 cache (spx_prefill_chunk_i8)
+
+def _prefill_state_i8(pos0, T):
+    need_gpu()
+    import bench
+    return bench.PrefillState(synth.workload("prefill"), torch.device("cuda", 0), pos0=pos0, T=T,
+                              keys="int8")
+
+
+def _check_prefill_i8(st, queries, attn_queries=None):
+    """Codes and scales of the chunk's blocks, the ids of `queries` bit-exact
+    against the oracle's INT8 steps (pool_i8, score_i8 over the query's
+    visible blocks, full-sort top-k), and attention of `attn_queries` (all of
+    `queries` by default) within the bf16 tolerance."""
+    from concurrent.futures import ThreadPoolExecutor
+    spx = need_gpu()
+    st.step()
+    torch.cuda.synchronize()
+    assert spx.spx_device_error() == 0
+    codes, scale = oracle.pool_i8(st.raw_keys_host(), st.w.pool_weights())
+    lo, hi = st.pos0 // 4, (st.pos0 + st.T) // 4
+    assert np.array_equal(st.pooled[0, lo:hi].cpu().numpy(), codes[lo:hi]), "codes of the chunk"
+    assert np.array_equal(st.k_scale[0, lo:hi].cpu().numpy().astype(np.float64), scale[lo:hi])
+    idx, cnt = st.idx.cpu().numpy(), st.count.cpu().numpy()
+    rows = st.pos0 + np.asarray(queries)
+    q_idx = st.w.q_idx_np(rows)
+    w_head = st.w.w_head_np(rows).astype(np.float64)
+
+    def select(i):
+        n = st.pos0 + queries[i] + 1
+        s = oracle.score_i8(q_idx[i], w_head[i], codes[:n // 4], scale[:n // 4], nthreads=1)
+        sel = oracle.topk(s)
+        return sel, oracle.token_set(sel, n)
+
+    with ThreadPoolExecutor(max_workers=oracle.threads(0)) as ex:
+        ref = list(ex.map(select, range(len(queries))))
+    bad = [t for t, (sel, _) in zip(queries, ref)
+           if cnt[t] != sel.size or not np.array_equal(idx[t, :cnt[t]], sel)
+           or not (idx[t, cnt[t]:] == -1).all()]
+    assert not bad, f"{len(bad)} of {len(queries)} queries select other blocks, first {bad[:8]}"
+    attn = list(queries) if attn_queries is None else list(attn_queries)
+    pos_of = {t: pos for t, (_, pos) in zip(queries, ref)}
+    q = st.w.q_np(st.pos0 + np.asarray(attn))
+    out, lse = f64_of(st.out), st.lse.cpu().numpy()
+    outs = []
+    for i, t in enumerate(attn):
+        o, l = oracle.attention(q[i], st.w.latent_np(0, pos_of[t]), st.w.sm_scale)
+        assert np.allclose(lse[t], l, atol=LSE_ATOL, rtol=0), f"query {t}"
+        outs.append(o)
+    assert_attention_close(out[attn], np.stack(outs), "prefill int8")
+
+
+def test_prefill_i8_small_all_queries():
+    # 8190 cached tokens (a 2-token tail), 100 new ones: the 2048-token budget
+    # boundary, several 128-block tiles and a partial group of 8 queries
+    st = _prefill_state_i8(8190, 100)
+    _check_prefill_i8(st, list(range(100)))
+
+
+def test_prefill_i8_short_context_dense():
+    st = _prefill_state_i8(1000, 64)
+    _check_prefill_i8(st, list(range(64)))
+
+
+def test_prefill_i8_full_chunk_stratified():
+    """The prefill benchmark's shape (4096 new tokens on 131,072 cached ones)
+    on the INT8 cache: ids of the 256-query stratified subset bit-exact, and
+    the attention of 32 of them."""
+    import bench
+    st = _prefill_state_i8(None, None)
+    sub = bench.stratified_prefill_queries(st.T)
+    _check_prefill_i8(st, sub, attn_queries=sub[::8])
