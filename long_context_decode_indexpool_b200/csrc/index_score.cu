@@ -94,8 +94,12 @@ struct Cfg {
   static constexpr int kThreads = 64 + kEpi;
   static constexpr int kQPerWarp = NQ * 4 * kEpiGroups / kEpiWarps;  // queries of one thread
   static constexpr int kTileBytes = I8 ? kHalfBytes : 2 * kHalfBytes;  // 128 keys
-  // I8: the tile's 128 block scales (512 B) follow it in the stage
-  static constexpr int kStageBytes = I8 ? kTileBytes + 1024 : kTileBytes;
+  // I8 with one query: the tile's 128 block scales (512 B) follow it in the
+  // stage; with eight (keys shared by the queries, L2-resident) each
+  // epilogue thread loads its key's scale while the MMA runs, so the MMA's
+  // commit alone releases the stage
+  static constexpr bool kScaleInStage = I8 && NQ == 1;
+  static constexpr int kStageBytes = kScaleInStage ? kTileBytes + 1024 : kTileBytes;
   static constexpr int kStages = I8 ? 10 : (NQ == 1 ? 6 : 4);
   static constexpr int kQSlots = NQ == 1 ? 2 : 1;
   static constexpr int kQHalf = kN * 128;  // one 128-byte-wide box of Q
@@ -350,8 +354,8 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
     for (int s = 0; s < C::kStages; ++s) {
       // I8: full also counts the producer lanes' scale copies, empty the
       // epilogue group that reads the scales
-      mbar_init(&full[s], I8 ? 1 + 32 : 1);
-      mbar_init(&empty[s], I8 ? 1 + C::kEpiWarps / C::kEpiGroups : 1);
+      mbar_init(&full[s], C::kScaleInStage ? 1 + 32 : 1);
+      mbar_init(&empty[s], C::kScaleInStage ? 1 + C::kEpiWarps / C::kEpiGroups : 1);
     }
     for (int s = 0; s < C::kQSlots; ++s) {
       mbar_init(&qfull[s], 1);
@@ -512,7 +516,7 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
         if constexpr (!I8)
           tma_load_3d_hint(dst + kHalfBytes, &map_k, &full[stage], 64, w.t * kTileM, kb, stream_pol);
       }
-      if constexpr (I8) {
+      if constexpr (C::kScaleInStage) {
         // the tile's 128 block scales into the stage behind the codes (zeros
         // past the cache); each lane's copies arrive on the stage's barrier
         // when they land, so the epilogue reads them from shared memory
@@ -539,7 +543,7 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
     }
     if (*abort_flag) {
       // Let the copies already issued land before the CTA exits.
-      if constexpr (I8) asm volatile("cp.async.wait_all;" ::: "memory");
+      if constexpr (C::kScaleInStage) asm volatile("cp.async.wait_all;" ::: "memory");
       if (lane == 0) {
         const int first = issued > C::kStages ? issued - C::kStages : 0;
         for (int i = first; i < issued; ++i) {
@@ -686,13 +690,17 @@ __global__ void __launch_bounds__(Cfg<NQ, SELECT, I8>::kThreads, 1)
         continue;
       }
       const int64_t blk = static_cast<int64_t>(w.t) * kTileM + row_in_tile;
+      float ksc = 1.f;  // I8: the block's scale
+      if constexpr (I8 && !C::kScaleInStage) {
+        const int kb = p.shared_keys ? 0 : w.g;
+        if (blk < p.cap_blk) ksc = __ldg(p.k_scale + static_cast<int64_t>(kb) * p.cap_blk + blk);
+      }
       if (!mbar_wait(&accfull[acc], acc_ph, abort_flag)) {
         aborted = true;
         break;
       }
       tc_fence_after();
-      float ksc = 1.f;  // I8: the block's scale, from the key stage
-      if constexpr (I8) {
+      if constexpr (C::kScaleInStage) {
         // (the stage's barrier completed before the MMA ran; waiting on it
         // again orders the scale copies before these reads)
         if (!mbar_wait(&full[my_st], my_st_ph, abort_flag)) {
