@@ -1,5 +1,6 @@
-// Lightning-indexer scoring on the 5th-generation tensor cores, with the
-// top-k block selection fused into the epilogue on the decode path.
+// Lightning-indexer scoring on the 5th-generation tensor cores; on the
+// decode path the epilogue also keeps the key histogram that the top-k
+// block selection starts from.
 //
 // [W4] "GLM-5.3-Flash vs Qwen3.8-Flash-Next: 두 중국 AI 연구소가 독립적으로 같은
 // 모델 설계로 수렴한 이유", section "수렴점 2 — 4배 압축 후 2,048 토큰만 유지":
@@ -44,13 +45,18 @@
 // the bin of the row's 512th-largest key exactly; the selection kernel
 // (topk.cu) then only keeps blocks at or above that bin.
 //
-// INT8 cache (decode, [W1] section "양자화: W8A8와 혼합 캐시"): the keys are
-// int8 codes with one power-of-two scale per block and the query heads come
-// quantised the same way, their scales folded into w.  A tile is then one
-// 16 KiB box of 128-byte rows (half the bytes), the MMA is 4 tcgen05.mma
-// kind::i8 (K = 32 each) into exact s32 accumulators, and the epilogue takes
-// ReLU on the integer dot, sums w_h * dot over the heads in fp32 and
-// multiplies by the block's scale.
+// INT8 cache (decode and prefill, [W1] section "양자화: W8A8와 혼합 캐시"):
+// the keys are int8 codes with one power-of-two scale per block and the
+// query heads come quantised the same way, their scales folded into w.  A
+// tile is then one 16 KiB box of 128-byte rows (half the bytes), the MMA is
+// 4 tcgen05.mma kind::i8 (K = 32 each) into exact s32 accumulators, and the
+// epilogue takes ReLU on the integer dot, sums w_h * dot over the heads in
+// fp32 and multiplies by the block's scale.
+//
+// Before its wait on the previous kernel a CTA sets up its barriers and
+// TMEM and, on the decode path, plans its work from the lengths before the
+// append and sends its first key tiles to L2; after the wait the plan is
+// checked against the lengths the append wrote.
 //
 // Every wait is bounded; on a timeout the CTA drains and exits with the
 // device error word set.
