@@ -43,12 +43,14 @@
 //
 // A row with a single split writes its normalised output directly.  The n
 // splits of one (row, head group) otherwise form a thread-block cluster: each
-// CTA writes its output rows normalised by its own l (bf16, like P) and its
-// per-head (m, l) (fp32) to L2 with one bulk copy, the cluster barrier
-// publishes them, and CTA k reads back heads [k*64/n, (k+1)*64/n) of all
-// splits with bulk copies and combines them with the log-sum-exp rule
-// (weights 2^(m_s - M) l_s / L) into the bf16 output and the log-sum-exp.
-// No second kernel runs.
+// CTA writes its output rows normalised by its own l (bf16, like P) to L2
+// (one bulk copy per TMEM lane quarter of 16 rows) and its per-head (m, l)
+// (fp32) with plain stores, the cluster barrier publishes them, and CTA k
+// reads back heads [k*64/n, (k+1)*64/n) of all splits with bulk copies and
+// combines them with the log-sum-exp rule (weights 2^(m_s - M) l_s / L) into
+// the bf16 output and the log-sum-exp.  No second kernel runs.  (Moving the
+// partials through distributed shared memory instead, by loads or by bulk
+// copies between the CTAs, measured slower.)
 #include <atomic>
 
 #include "spx_device.cuh"
