@@ -274,13 +274,21 @@ __global__ void __launch_bounds__(kThreads)
     if (tid == 0) list_cnt[slot] = n;
   }
 
-  // 3. the last CTA of the row continues
-  __threadfence();
+  // 3. the last CTA of the row continues.  After the CTA barrier one
+  // acquire-release count per CTA orders every thread's list writes before
+  // it and the last CTA's reads after it (a fence in every thread instead
+  // cost 0.6 us per 1M decode step).
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(done + r, 1) == nchunk - 1;
+  if (tid == 0) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
+                 : "=r"(old)
+                 : "l"(done + r)
+                 : "memory");
+    s_last = old == nchunk - 1;
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   int32_t* dst = out_idx + static_cast<int64_t>(r) * kTopK;
   const int64_t slot0 = static_cast<int64_t>(r) * nchunk;
   if (tid == 0) done[r] = 0;  // ready for the next launch
