@@ -88,16 +88,29 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
 
 // INT8 codes of the query heads of row b (the scoring kernel's B operand):
 // warp w quantises heads w, w+4, ..; lane l holds dims 4l..4l+3.  The
-// head's scale is folded into its weight: wq = w_head * 2^e.
+// head's scale is folded into its weight: wq = w_head * 2^e.  Every load
+// is issued before the first head is worked on (one round trip, not one a
+// head: this runs on the decode step's critical path).
 __device__ void quant_q_row(const __nv_bfloat16* __restrict__ q_idx,
                             const float* __restrict__ w_head, int8_t* __restrict__ q8,
                             float* __restrict__ wq, int b) {
+  constexpr int kWarps = kPoolThreads / 32;
+  constexpr int kPer = kIdxHeads / kWarps;  // heads of one warp
+  static_assert(kIdxHeads % kWarps == 0, "whole heads per warp");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int h = warp; h < kIdxHeads; h += kPoolThreads / 32) {
-    const int64_t row = static_cast<int64_t>(b) * kIdxHeads + h;
-    const uint2 u = *reinterpret_cast<const uint2*>(q_idx + row * kIdxDim + 4 * lane);
-    const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-    const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  uint2 u[kPer];
+  float wh[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t row = static_cast<int64_t>(b) * kIdxHeads + warp + kWarps * i;
+    u[i] = *reinterpret_cast<const uint2*>(q_idx + row * kIdxDim + 4 * lane);
+    wh[i] = lane == 0 ? w_head[row] : 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t row = static_cast<int64_t>(b) * kIdxHeads + warp + kWarps * i;
+    const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[i].x));
+    const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[i].y));
     float amax = fmaxf(fmaxf(fabsf(x01.x), fabsf(x01.y)), fmaxf(fabsf(x23.x), fabsf(x23.y)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -107,7 +120,7 @@ __device__ void quant_q_row(const __nv_bfloat16* __restrict__ q_idx,
                             ((static_cast<uint32_t>(i8_code(x23.x, e)) & 0xffu) << 16) |
                             (static_cast<uint32_t>(i8_code(x23.y, e)) << 24);
     *reinterpret_cast<uint32_t*>(q8 + row * kIdxDim + 4 * lane) = packed;
-    if (lane == 0) wq[row] = w_head[row] * ldexpf(1.f, e);
+    if (lane == 0) wq[row] = wh[i] * ldexpf(1.f, e);
   }
 }
 
