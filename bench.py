@@ -594,10 +594,10 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
-        "config": {"workload": w.name, "queries_per_step": 1, "context": w.L,
-                   "indexer": "32x128, pool 4, top-512 blocks", "mla_heads": w.heads},
+        "config": decode_config(w, w.B, w.L, w.heads, max(1, args.gpus), args.keys == "int8"),
         "cpu_baseline": {"value": value, "unit": "queries/s", "cores": nthreads, "kind": "oracle",
-                         "sample": f"one query of {w.name} per step"},
+                         "sample": f"one query of {w.name} per step (a bounded sample of its "
+                                   f"{w.B} queries; value = queries / oracle time)"},
         "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -605,6 +605,16 @@ def run_reference(args):
 
 
 METRIC = "sparse-attn decode queries/s at 1M ctx; achieved HBM GB/s vs 8 TB/s peak"
+
+
+def decode_config(w, B: int, L: int, heads: int, world: int, i8: bool = False) -> dict:
+    """The `config` of a decode line; both arms (this library and the oracle)
+    report the same dict for the same workload."""
+    return {"workload": w.name, "batch_per_gpu": B, "context": L, "heads": heads,
+            "indexer": "32 heads x 128, pool 4, top-512 blocks", "latent": 512,
+            "pooled_keys": "int8 codes + fp32 scale per block" if i8 else "bf16",
+            "parallelism": f"dp{world} (independent sequences)",
+            "l2": "inputs larger than L2 (pooled keys + 4 GiB latent per GPU)"}
 
 
 # ---------------------------------------------------------------------------
@@ -673,11 +683,7 @@ def run_decode(args, world, rank, local):
         "dtype": "s8 indexer keys and queries (s32 dots), bf16 attention" if i8 else "bf16",
         "data": "synthetic (seeded generator; int-valued indexer keys, dyadic pool weights, "
                 "600 needles/seq, N(0,1) latent)",
-        "config": {"workload": w.name, "batch_per_gpu": B, "context": L, "heads": st.H,
-                   "indexer": "32 heads x 128, pool 4, top-512 blocks", "latent": 512,
-                   "pooled_keys": "int8 codes + fp32 scale per block" if i8 else "bf16",
-                   "parallelism": f"dp{world} (independent sequences)",
-                   "l2": "inputs larger than L2 (pooled keys + 4 GiB latent per GPU)"},
+        "config": decode_config(w, B, L, st.H, world, i8),
         "roofline": {"bound": "hbm",
                      "kernel": "k_index_score (decode scoring" + (", INT8 cache)" if i8 else ")"),
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,

@@ -89,6 +89,12 @@ def test_reference_arm_line_on_cpu():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+    # the same config dict as this library's decode line on that workload
+    import bench
+    import synth
+    w = synth.workload("tiny")
+    assert d["config"] == bench.decode_config(w, w.B, w.L, w.heads, 1)
+    assert d["metric"] == bench.METRIC
     r1 = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=300,
                         env=dict(os.environ, RANK="1"))
     assert r1.returncode == 0 and not r1.stdout.strip()
